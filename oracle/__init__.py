@@ -1,0 +1,202 @@
+"""CPU oracle for N:M structured sparsity (test infrastructure only).
+
+This package is the plain, slow, fp64 definition that the CUDA library is
+checked against.  Only the tests, ``__graft_entry__.smoke()`` and the CPU
+baseline leg of ``bench.py`` may import it; the product package never does.
+
+The arithmetic lives in ``nm_oracle.c`` (plain C, double accumulation).  This
+module compiles it with gcc on first use (or via :func:`build`) and wraps each
+function for numpy arrays.  bf16 values travel as their uint16 bit patterns.
+
+Sources, by page title and passage:
+  * "M:N sparsity on NVIDIA tensor cores" -- opening passage (2:4 definition
+    and the worked row), "Fine-grained in what it removes, structured in how
+    many" (2-bit positions, groups along the reduction axis), "Where this
+    sits among the three case studies" (push-left format, 36-bit groups,
+    sparse x dense = dense), "The recipe" (magnitude pruning).
+  * "Technische Samenvatting: SHUFFLESPARSE", "2. Methodologie": y = (W Pi) x
+    with Pi applied as an index map on the input read.
+  * "Structured Sparsity" topic cards, PATCH abstract: per-tile dense / 2:4.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "nm_oracle.c")
+_LIB = os.path.join(_HERE, "libnm_oracle.so")
+_lock = threading.Lock()
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile nm_oracle.c into libnm_oracle.so next to it (gcc -O2)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + f".tmp{os.getpid()}"
+        subprocess.check_call(["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-o", tmp, _SRC, "-lm"])
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+def _load():
+    global _lib
+    with _lock:
+        if _lib is None:
+            lib = ctypes.CDLL(build())
+            P, I64, I = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int
+            sig = {
+                "oracle_index_bits": ([I], I),
+                "oracle_positions_per_word": ([I], I),
+                "oracle_value_cols": ([I64, I, I], I64),
+                "oracle_meta_cols": ([I64, I, I], I64),
+                "oracle_prune_mask": ([P, I64, I64, I64, I, I, P], I),
+                "oracle_compress": ([P, I64, I64, I64, I, I, P, P], I),
+                "oracle_decompress": ([P, P, I64, I64, I, I, P, I64], I),
+                "oracle_spmm": ([P, P, I, I, I64, I64, P, I64, I64, P, P, I64], I),
+                "oracle_spmm_sampled": ([P, P, I, I, I64, I64, P, I64, I64, P, P, P, I64, P, P], I),
+                "oracle_dense_gemm": ([P, I64, I64, I64, P, I64, I64, P, P, P, I64], I),
+                "oracle_hybrid_weights": ([P, I64, I64, I64, P, I64, P], I),
+                "oracle_hybrid_spmm": ([P, I64, I64, I64, P, I64, P, I64, I64, P, P, I64], I),
+            }
+            for name, (args, res) in sig.items():
+                fn = getattr(lib, name)
+                fn.argtypes = args
+                fn.restype = res
+            _lib = lib
+    return _lib
+
+
+def _ptr(a):
+    return None if a is None else a.ctypes.data
+
+
+def _u16(a):
+    a = np.ascontiguousarray(a)
+    assert a.dtype == np.uint16, "bf16 data travels as uint16 bit patterns"
+    return a
+
+
+def _check(rc, what):
+    if rc != 0:
+        raise ValueError(f"oracle {what} rejected its arguments (code {rc})")
+
+
+def index_bits(m: int) -> int:
+    return _load().oracle_index_bits(m)
+
+
+def positions_per_word(m: int) -> int:
+    return _load().oracle_positions_per_word(m)
+
+
+def value_cols(K: int, n: int, m: int) -> int:
+    return _load().oracle_value_cols(K, n, m)
+
+
+def meta_cols(K: int, n: int, m: int) -> int:
+    return _load().oracle_meta_cols(K, n, m)
+
+
+def prune_mask(W: np.ndarray, n: int, m: int) -> np.ndarray:
+    """uint8 R x K mask of the N:M survivors of bf16 W (R x K)."""
+    W = _u16(W)
+    R, K = W.shape
+    mask = np.zeros((R, K), np.uint8)
+    _check(_load().oracle_prune_mask(_ptr(W), R, K, K, n, m, _ptr(mask)), "prune_mask")
+    return mask
+
+
+def compress(W: np.ndarray, n: int, m: int):
+    """(values R x K*n/m uint16, meta R x meta_cols uint32) of bf16 W."""
+    W = _u16(W)
+    R, K = W.shape
+    vals = np.zeros((R, value_cols(K, n, m)), np.uint16)
+    meta = np.zeros((R, meta_cols(K, n, m)), np.uint32)
+    _check(_load().oracle_compress(_ptr(W), R, K, K, n, m, _ptr(vals), _ptr(meta)), "compress")
+    return vals, meta
+
+
+def decompress(values: np.ndarray, meta: np.ndarray, K: int, n: int, m: int) -> np.ndarray:
+    values = _u16(values)
+    meta = np.ascontiguousarray(meta, dtype=np.uint32)
+    R = values.shape[0]
+    out = np.zeros((R, K), np.uint16)
+    _check(_load().oracle_decompress(_ptr(values), _ptr(meta), R, K, n, m, _ptr(out), K), "decompress")
+    return out
+
+
+def spmm(values, meta, n, m, K, X, idx=None) -> np.ndarray:
+    """fp64 y = (W' Pi) X from the compressed operand (idx = None: Pi = I)."""
+    values = _u16(values)
+    meta = np.ascontiguousarray(meta, dtype=np.uint32)
+    X = _u16(X)
+    R = values.shape[0]
+    T = X.shape[1]
+    if idx is not None:
+        idx = np.ascontiguousarray(idx, dtype=np.int32)
+    Y = np.zeros((R, T), np.float64)
+    _check(_load().oracle_spmm(_ptr(values), _ptr(meta), n, m, R, K, _ptr(X), T, T,
+                               _ptr(idx), _ptr(Y), T), "spmm")
+    return Y
+
+
+def spmm_sampled(values, meta, n, m, K, X, rows, cols, idx=None):
+    """fp64 y[rows[i], cols[i]] and sum |w||x| for each sampled coordinate."""
+    values = _u16(values)
+    meta = np.ascontiguousarray(meta, dtype=np.uint32)
+    X = _u16(X)
+    R = values.shape[0]
+    T = X.shape[1]
+    rows = np.ascontiguousarray(rows, dtype=np.int64)
+    cols = np.ascontiguousarray(cols, dtype=np.int64)
+    if idx is not None:
+        idx = np.ascontiguousarray(idx, dtype=np.int32)
+    out = np.zeros(rows.shape[0], np.float64)
+    mag = np.zeros(rows.shape[0], np.float64)
+    _check(_load().oracle_spmm_sampled(_ptr(values), _ptr(meta), n, m, R, K, _ptr(X), T, T,
+                                       _ptr(idx), _ptr(rows), _ptr(cols), rows.shape[0],
+                                       _ptr(out), _ptr(mag)), "spmm_sampled")
+    return out, mag
+
+
+def dense_gemm(W, X, idx=None, with_abs=False):
+    """fp64 y = W X[idx] for bf16 W (R x K) and X (K x T); optionally sum |w||x|."""
+    W = _u16(W)
+    X = _u16(X)
+    R, K = W.shape
+    T = X.shape[1]
+    if idx is not None:
+        idx = np.ascontiguousarray(idx, dtype=np.int32)
+    Y = np.zeros((R, T), np.float64)
+    A = np.zeros((R, T), np.float64) if with_abs else None
+    _check(_load().oracle_dense_gemm(_ptr(W), R, K, K, _ptr(X), T, T, _ptr(idx), _ptr(Y),
+                                     _ptr(A), T), "dense_gemm")
+    return (Y, A) if with_abs else Y
+
+
+def hybrid_weights(W, tile_map, tile=128):
+    W = _u16(W)
+    R, K = W.shape
+    tile_map = np.ascontiguousarray(tile_map, dtype=np.uint8)
+    out = np.zeros((R, K), np.uint16)
+    _check(_load().oracle_hybrid_weights(_ptr(W), R, K, K, _ptr(tile_map), tile, _ptr(out)),
+           "hybrid_weights")
+    return out
+
+
+def hybrid_spmm(W, tile_map, X, tile=128, with_abs=False):
+    W = _u16(W)
+    X = _u16(X)
+    R, K = W.shape
+    T = X.shape[1]
+    tile_map = np.ascontiguousarray(tile_map, dtype=np.uint8)
+    Y = np.zeros((R, T), np.float64)
+    A = np.zeros((R, T), np.float64) if with_abs else None
+    _check(_load().oracle_hybrid_spmm(_ptr(W), R, K, K, _ptr(tile_map), tile, _ptr(X), T, T,
+                                      _ptr(Y), _ptr(A), T), "hybrid_spmm")
+    return (Y, A) if with_abs else Y

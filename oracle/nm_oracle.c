@@ -1,0 +1,328 @@
+/*
+ * nm_oracle.c -- plain, slow, obviously-correct CPU definition of N:M
+ * structured weight sparsity: magnitude prune, push-left compression,
+ * decompression, and the sparse x dense GEMM (plain, column-permuted and
+ * PATCH-style hybrid).  Every sum is accumulated in double precision.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing on the product path may call, link or
+ * load this file: only the tests, the package's smoke check and the
+ * benchmark's CPU-baseline leg use it.  It shares no code, header or table
+ * with the CUDA library.
+ *
+ * Sources (page title, then the passage):
+ *  [MN-def]   "M:N sparsity on NVIDIA tensor cores", opening passage: a 2:4
+ *             row is read four cells at a time; every group of four
+ *             consecutive weights along a row keeps exactly two survivors,
+ *             anywhere inside the group; the metadata of the worked row
+ *             [v,0,0,v | 0,v,v,0] is [[0,3],[1,2]]; the general a:b form.
+ *  [MN-fine]  same page, "Fine-grained in what it removes, structured in how
+ *             many": two bits per survivor say which slot it came from; the
+ *             groups run along the row of W, which is the reduction axis K.
+ *  [MN-fmt]   same page, "Where this sits among the three case studies",
+ *             storage paragraphs: an R x C matrix is stored as an R x C/2
+ *             block of values with all survivors pushed left, plus an
+ *             R x C/2 block of 2-bit indices; 36 bits per group of four
+ *             FP16 weights.
+ *  [MN-gemm]  same page and section, GEMM paragraphs: only the first operand
+ *             is compressed; the indices pick the elements of the dense
+ *             second operand that the kept weights multiply (the K = 8
+ *             example); the result is a dense matrix.
+ *  [MN-prune] same page, "The recipe: one prune, one retrain, no search",
+ *             step 2: in every group of four along the row, zero the two
+ *             with the smallest absolute value.
+ *  [SS-perm]  "Technische Samenvatting: SHUFFLESPARSE ...", section
+ *             "2. Methodologie": y = (W Pi) x; at inference the hard Pi is
+ *             a precomputed index map and the structured sparse GEMM reads
+ *             its input at the permuted addresses (same FLOP count).
+ *  [PATCH]    "Structured Sparsity" topic cards, the PATCH abstract: weight
+ *             matrices are split into tiles, each tile either dense or 2:4.
+ *
+ * Readings where the pages are silent (each listed in the design notes):
+ *  - ties in magnitude go to the lower index inside the group;
+ *  - exactly N survivors are always stored, zeros included, so the format
+ *    stays fixed-rate;
+ *  - survivors of a group are stored in ascending position order, as in the
+ *    worked row;
+ *  - magnitudes are compared on the bf16 value; +0 and -0 tie; a NaN ranks
+ *    above every number (Inf included) and NaNs tie among themselves;
+ *  - positions use b = ceil(log2 M) bits; survivor j of a row goes to
+ *    32-bit word floor(j/S) at bit b*(j mod S), S = floor(32/b); unused
+ *    bits are zero;
+ *  - the permutation is applied as X_perm[k][t] = X[idx[k]][t];
+ *  - W (dense, R x K) and the compressed values hold bf16 bit patterns
+ *    (uint16); X is K x T row-major; Y is R x T (double here).
+ */
+#include <math.h>
+#include <stddef.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+/* ------------------------------------------------------------------ */
+/* bf16 <-> double.  bf16 is the upper half of an IEEE binary32, so the */
+/* conversion to double is exact.                                       */
+/* ------------------------------------------------------------------ */
+static double bf16_value(uint16_t bits)
+{
+    uint32_t u = (uint32_t)bits << 16;
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return (double)f;
+}
+
+/* Bits per stored position for a group of M: ceil(log2 M). */
+int oracle_index_bits(int m)
+{
+    int b = 0;
+    while ((1 << b) < m) b++;
+    return b;
+}
+
+/* Positions packed into one 32-bit word. */
+int oracle_positions_per_word(int m)
+{
+    return 32 / oracle_index_bits(m);
+}
+
+/* Columns of the value block: K * N / M. */
+int64_t oracle_value_cols(int64_t K, int n, int m)
+{
+    return K / m * n;
+}
+
+/* 32-bit metadata words per row: ceil(value_cols / S). */
+int64_t oracle_meta_cols(int64_t K, int n, int m)
+{
+    int64_t s = oracle_positions_per_word(m);
+    return (oracle_value_cols(K, n, m) + s - 1) / s;
+}
+
+static int pattern_ok(int n, int m)
+{
+    return (m == 2 || m == 4 || m == 8 || m == 16) && n >= 1 && n < m;
+}
+
+/* ------------------------------------------------------------------ */
+/* Selection [MN-def], [MN-prune].                                      */
+/* ------------------------------------------------------------------ */
+
+/* Does element a of a group beat element b (a != b)?  Larger magnitude
+ * wins; a NaN beats every number; equal magnitudes (and NaN vs NaN) go to
+ * the lower index. */
+static int beats(double wa, int a, double wb, int b)
+{
+    int na = isnan(wa), nb = isnan(wb);
+    if (na || nb) {
+        if (na && !nb) return 1;
+        if (nb && !na) return 0;
+        return a < b;
+    }
+    double ma = fabs(wa), mb = fabs(wb);
+    if (ma != mb) return ma > mb;
+    return a < b;
+}
+
+/* mask[r*K + k] = 1 if W[r][k] survives N:M pruning, else 0.  An element
+ * survives when fewer than N elements of its group beat it. */
+int oracle_prune_mask(const uint16_t *W, int64_t R, int64_t K, int64_t ldw,
+                      int n, int m, uint8_t *mask)
+{
+    if (!pattern_ok(n, m) || K % m != 0 || ldw < K) return 1;
+    for (int64_t r = 0; r < R; r++) {
+        for (int64_t g = 0; g < K / m; g++) {
+            const uint16_t *grp = W + r * ldw + g * m;
+            for (int i = 0; i < m; i++) {
+                int rank = 0;
+                for (int j = 0; j < m; j++)
+                    if (j != i && beats(bf16_value(grp[j]), j, bf16_value(grp[i]), i))
+                        rank++;
+                mask[r * K + g * m + i] = (uint8_t)(rank < n);
+            }
+        }
+    }
+    return 0;
+}
+
+/* ------------------------------------------------------------------ */
+/* Push-left compression [MN-fmt].                                      */
+/* values: R x (K*N/M) bf16 bits, survivors in ascending position.      */
+/* meta:   R x meta_cols words, b-bit in-group positions, LSB first.    */
+/* ------------------------------------------------------------------ */
+int oracle_compress(const uint16_t *W, int64_t R, int64_t K, int64_t ldw,
+                    int n, int m, uint16_t *values, uint32_t *meta)
+{
+    if (!pattern_ok(n, m) || K % m != 0 || ldw < K) return 1;
+    int64_t vcols = oracle_value_cols(K, n, m);
+    int64_t mcols = oracle_meta_cols(K, n, m);
+    int b = oracle_index_bits(m);
+    int s = oracle_positions_per_word(m);
+    uint8_t *mask = (uint8_t *)malloc((size_t)(R * K > 0 ? R * K : 1));
+    if (!mask) return 2;
+    oracle_prune_mask(W, R, K, ldw, n, m, mask);
+    memset(meta, 0, (size_t)(R * mcols) * sizeof(uint32_t));
+    for (int64_t r = 0; r < R; r++) {
+        int64_t j = 0; /* survivor index inside the row */
+        for (int64_t g = 0; g < K / m; g++) {
+            for (int p = 0; p < m; p++) {
+                if (!mask[r * K + g * m + p]) continue;
+                values[r * vcols + j] = W[r * ldw + g * m + p];
+                meta[r * mcols + j / s] |= (uint32_t)p << (b * (j % s));
+                j++;
+            }
+        }
+    }
+    free(mask);
+    return 0;
+}
+
+/* In-group position of survivor j of row r. */
+static int position_of(const uint32_t *meta, int64_t mcols, int64_t r, int64_t j, int m)
+{
+    int b = oracle_index_bits(m);
+    int s = oracle_positions_per_word(m);
+    uint32_t word = meta[r * mcols + j / s];
+    return (int)((word >> (b * (j % s))) & ((1u << b) - 1u));
+}
+
+/* ------------------------------------------------------------------ */
+/* Decompression: put every survivor back at its position, +0 (bits     */
+/* 0x0000) everywhere else.                                             */
+/* ------------------------------------------------------------------ */
+int oracle_decompress(const uint16_t *values, const uint32_t *meta, int64_t R, int64_t K,
+                      int n, int m, uint16_t *W_out, int64_t ldw)
+{
+    if (!pattern_ok(n, m) || K % m != 0 || ldw < K) return 1;
+    int64_t vcols = oracle_value_cols(K, n, m);
+    int64_t mcols = oracle_meta_cols(K, n, m);
+    for (int64_t r = 0; r < R; r++) {
+        for (int64_t k = 0; k < K; k++) W_out[r * ldw + k] = 0;
+        for (int64_t j = 0; j < vcols; j++) {
+            int64_t g = j / n;
+            int p = position_of(meta, mcols, r, j, m);
+            W_out[r * ldw + g * m + p] = values[r * vcols + j];
+        }
+    }
+    return 0;
+}
+
+/* ------------------------------------------------------------------ */
+/* Sparse x dense GEMM on the compressed operand [MN-gemm], [SS-perm]:  */
+/*   y[r][t] = sum_j V[r][j] * X[pi(g*M + pos_j)][t],  g = j / N,       */
+/* pi(k) = idx[k] when idx is given, else k.  Products and the sum are  */
+/* in double, in survivor order.                                         */
+/* ------------------------------------------------------------------ */
+int oracle_spmm(const uint16_t *values, const uint32_t *meta, int n, int m,
+                int64_t R, int64_t K, const uint16_t *X, int64_t ldx, int64_t T,
+                const int32_t *idx, double *Y, int64_t ldy)
+{
+    if (!pattern_ok(n, m) || K % m != 0 || ldx < T || ldy < T) return 1;
+    int64_t vcols = oracle_value_cols(K, n, m);
+    int64_t mcols = oracle_meta_cols(K, n, m);
+    for (int64_t r = 0; r < R; r++) {
+        for (int64_t t = 0; t < T; t++) {
+            double acc = 0.0;
+            for (int64_t j = 0; j < vcols; j++) {
+                int64_t k = (j / n) * m + position_of(meta, mcols, r, j, m);
+                int64_t src = idx ? (int64_t)idx[k] : k;
+                acc += bf16_value(values[r * vcols + j]) * bf16_value(X[src * ldx + t]);
+            }
+            Y[r * ldy + t] = acc;
+        }
+    }
+    return 0;
+}
+
+/* The same sum for a list of (row, column) output coordinates only: the
+ * per-element form used to check full-size results by sampling. */
+int oracle_spmm_sampled(const uint16_t *values, const uint32_t *meta, int n, int m,
+                        int64_t R, int64_t K, const uint16_t *X, int64_t ldx, int64_t T,
+                        const int32_t *idx, const int64_t *rows, const int64_t *cols,
+                        int64_t count, double *out, double *out_abs)
+{
+    if (!pattern_ok(n, m) || K % m != 0 || ldx < T) return 1;
+    int64_t vcols = oracle_value_cols(K, n, m);
+    int64_t mcols = oracle_meta_cols(K, n, m);
+    for (int64_t i = 0; i < count; i++) {
+        int64_t r = rows[i], t = cols[i];
+        if (r < 0 || r >= R || t < 0 || t >= T) return 3;
+        double acc = 0.0, mag = 0.0;
+        for (int64_t j = 0; j < vcols; j++) {
+            int64_t k = (j / n) * m + position_of(meta, mcols, r, j, m);
+            int64_t src = idx ? (int64_t)idx[k] : k;
+            double w = bf16_value(values[r * vcols + j]);
+            double x = bf16_value(X[src * ldx + t]);
+            acc += w * x;
+            mag += fabs(w) * fabs(x);
+        }
+        out[i] = acc;
+        if (out_abs) out_abs[i] = mag;
+    }
+    return 0;
+}
+
+/* ------------------------------------------------------------------ */
+/* Plain dense GEMM of a bf16 matrix, the closed form a sparse GEMM     */
+/* must equal once the pruned weights are written out densely:          */
+/*   y[r][t] = sum_k W[r][k] * X[pi(k)][t].                              */
+/* y_abs (optional) receives sum_k |W[r][k]| * |X[pi(k)][t]|, the scale */
+/* of the floating-point tolerance.                                     */
+/* ------------------------------------------------------------------ */
+int oracle_dense_gemm(const uint16_t *W, int64_t R, int64_t K, int64_t ldw,
+                      const uint16_t *X, int64_t ldx, int64_t T, const int32_t *idx,
+                      double *Y, double *Y_abs, int64_t ldy)
+{
+    if (ldw < K || ldx < T || ldy < T) return 1;
+    for (int64_t r = 0; r < R; r++) {
+        for (int64_t t = 0; t < T; t++) {
+            double acc = 0.0, mag = 0.0;
+            for (int64_t k = 0; k < K; k++) {
+                int64_t src = idx ? (int64_t)idx[k] : k;
+                double w = bf16_value(W[r * ldw + k]);
+                double x = bf16_value(X[src * ldx + t]);
+                acc += w * x;
+                mag += fabs(w) * fabs(x);
+            }
+            Y[r * ldy + t] = acc;
+            if (Y_abs) Y_abs[r * ldy + t] = mag;
+        }
+    }
+    return 0;
+}
+
+/* ------------------------------------------------------------------ */
+/* PATCH-style hybrid [PATCH]: tile (i, j) of size tile x tile uses the */
+/* dense weights when tile_map[i][j] == 0, and the 2:4-pruned weights   */
+/* (survivors kept, +0 elsewhere) when it is 1.  W_eff is written out   */
+/* and multiplied densely.  tile_map is ceil(R/tile) x ceil(K/tile).    */
+/* ------------------------------------------------------------------ */
+int oracle_hybrid_weights(const uint16_t *W, int64_t R, int64_t K, int64_t ldw,
+                          const uint8_t *tile_map, int64_t tile, uint16_t *W_eff)
+{
+    if (K % 4 != 0 || tile <= 0 || tile % 4 != 0 || ldw < K) return 1;
+    uint8_t *mask = (uint8_t *)malloc((size_t)(R * K > 0 ? R * K : 1));
+    if (!mask) return 2;
+    oracle_prune_mask(W, R, K, ldw, 2, 4, mask);
+    int64_t tiles_k = (K + tile - 1) / tile;
+    for (int64_t r = 0; r < R; r++) {
+        for (int64_t k = 0; k < K; k++) {
+            int sparse = tile_map[(r / tile) * tiles_k + k / tile] != 0;
+            uint16_t w = W[r * ldw + k];
+            W_eff[r * K + k] = (sparse && !mask[r * K + k]) ? (uint16_t)0 : w;
+        }
+    }
+    free(mask);
+    return 0;
+}
+
+int oracle_hybrid_spmm(const uint16_t *W, int64_t R, int64_t K, int64_t ldw,
+                       const uint8_t *tile_map, int64_t tile,
+                       const uint16_t *X, int64_t ldx, int64_t T, double *Y, double *Y_abs,
+                       int64_t ldy)
+{
+    uint16_t *W_eff = (uint16_t *)malloc((size_t)(R * K > 0 ? R * K : 1) * sizeof(uint16_t));
+    if (!W_eff) return 2;
+    int rc = oracle_hybrid_weights(W, R, K, ldw, tile_map, tile, W_eff);
+    if (rc == 0) rc = oracle_dense_gemm(W_eff, R, K, K, X, ldx, T, NULL, Y, Y_abs, ldy);
+    free(W_eff);
+    return rc;
+}

@@ -1,0 +1,315 @@
+"""Pins of the CPU oracle against what the pages and the mathematics fix.
+
+Each check here comes from somewhere other than the oracle itself: the
+worked row and the storage arithmetic printed on the pages (fixtures under
+tests/golden/), brute-force enumeration of the selection rule, a stable
+library sort, numpy's float64 matmul as the closed form of the GEMM, an
+explicit permutation matrix, and special cases (identity permutation, all
+dense / all 2:4 tile maps) that reduce one function to another.
+"""
+import itertools
+import json
+import os
+
+import numpy as np
+import pytest
+
+import oracle
+import workloads as wl
+
+PATTERNS = [(2, 4), (1, 4), (1, 8), (3, 4), (1, 2), (4, 8), (3, 8), (2, 8), (5, 16), (1, 16)]
+
+
+def f64(bits):
+    return wl.bf16_to_f32(bits).astype(np.float64)
+
+
+def bits_of(values):
+    return wl.bf16_bits(np.asarray(values, dtype=np.float32))
+
+
+def positions(meta_row, count, m):
+    b = oracle.index_bits(m)
+    s = oracle.positions_per_word(m)
+    return [int((int(meta_row[j // s]) >> (b * (j % s))) & ((1 << b) - 1)) for j in range(count)]
+
+
+# ---------------------------------------------------------------------------
+# The worked row of the pages
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("v", [1.0, -3.5, 0.0078125, 65280.0])
+def test_worked_row(golden_dir, v):
+    g = json.load(open(os.path.join(golden_dir, "worked_row_2of4.json")))
+    row = [v if c == "v" else 0.0 for c in g["row_template"]]
+    W = bits_of([row])
+    vals, meta = oracle.compress(W, 2, 4)
+    pos = positions(meta[0], 4, 4)
+    assert [pos[0:2], pos[2:4]] == g["metadata"]
+    assert int(meta[0, 0]) & 0xFF == g["packed_low_byte"]
+    assert int(meta[0, 0]) >> 8 == 0
+    assert np.array_equal(vals[0], bits_of([v, v, v, v]))
+
+
+# ---------------------------------------------------------------------------
+# Selection rule
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("n,m", PATTERNS)
+def test_exactly_n_survivors(n, m):
+    W = wl.normal_bf16((37, 16 * m), 1.0, seed=n * 100 + m)
+    mask = oracle.prune_mask(W, n, m)
+    assert np.all(mask.reshape(37, -1, m).sum(axis=2) == n)
+
+
+def _preferred(w, i, j):
+    """i is kept ahead of j: larger |w|, equal magnitudes to the lower index."""
+    return (abs(w[i]), -i) > (abs(w[j]), -j)
+
+
+@pytest.mark.parametrize("n,m", [(2, 4), (1, 4), (3, 4), (1, 8), (2, 8), (5, 8), (1, 2)])
+def test_selection_bruteforce(n, m):
+    """Exactly one N-subset dominates its complement, and it is the oracle's."""
+    rng = np.random.default_rng(7 + n + m)
+    groups = rng.integers(-3, 4, size=(300, m)).astype(np.float32)  # many ties
+    W = bits_of(groups.reshape(1, -1))
+    mask = oracle.prune_mask(W, n, m).reshape(-1, m)
+    for gi, grp in enumerate(groups):
+        w = [float(x) for x in grp]
+        winners = [S for S in itertools.combinations(range(m), n)
+                   if all(_preferred(w, i, j) for i in S for j in range(m) if j not in S)]
+        assert len(winners) == 1
+        assert [p for p in range(m) if mask[gi, p]] == list(winners[0])
+
+
+def _stable_sort_select(w, n):
+    order = sorted(range(len(w)), key=lambda i: -abs(w[i]))  # stable: ties keep lower index first
+    return sorted(order[:n])
+
+
+@pytest.mark.parametrize("n,m,alphabet", [
+    (2, 4, [-2.0, -1.0, -0.0, 0.0, 1.0, 2.0]),
+    (1, 4, [-2.0, -1.0, -0.0, 0.0, 1.0, 2.0]),
+    (3, 4, [-2.0, -1.0, -0.0, 0.0, 1.0, 2.0]),
+    (1, 8, [0.0, 1.0, 2.0]),
+    (2, 8, [0.0, -1.0, 2.0]),
+])
+def test_exhaustive_alphabet(n, m, alphabet):
+    groups = np.array(list(itertools.product(alphabet, repeat=m)), dtype=np.float32)
+    W = bits_of(groups.reshape(1, -1))
+    vals, meta = oracle.compress(W, n, m)
+    pos = positions(meta[0], groups.shape[0] * n, m)
+    for gi, grp in enumerate(groups):
+        want = _stable_sort_select([float(x) for x in grp], n)
+        assert pos[gi * n:(gi + 1) * n] == want
+        # values are the exact bit patterns at those positions (-0.0 kept as -0.0)
+        assert np.array_equal(vals[0, gi * n:(gi + 1) * n], bits_of(grp[want]))
+
+
+def test_nan_inf_order():
+    """Reading for non-finite inputs: NaN above Inf, Inf above finite, ties to the lower index."""
+    nan, inf = float("nan"), float("inf")
+    rows = [[nan, inf, 1.0, -inf], [1.0, nan, nan, 5.0], [-inf, 3.0, inf, 2.0], [0.0, -0.0, 0.0, -0.0]]
+    want = [[0, 1], [1, 2], [0, 2], [0, 1]]
+    W = bits_of(rows)
+    mask = oracle.prune_mask(W, 2, 4)
+    for r, w in enumerate(want):
+        assert [p for p in range(4) if mask[r, p]] == w
+
+
+# ---------------------------------------------------------------------------
+# Storage format
+# ---------------------------------------------------------------------------
+def test_storage_36_bits(golden_dir):
+    g = json.load(open(os.path.join(golden_dir, "storage_bits.json")))
+    R, K = 64, 4096
+    W = wl.normal_bf16((R, K), 1.0, seed=3)
+    vals, meta = oracle.compress(W, 2, 4)
+    groups = R * K // 4
+    bits_per_group = (vals.nbytes + meta.nbytes) * 8 / groups
+    assert bits_per_group == g["fp16_2of4_bits"]
+    assert W.nbytes * 8 / groups == g["fp16_dense_bits"]
+    assert round(100 * (1 - bits_per_group / g["fp16_dense_bits"])) == g["fp16_saving_percent_about"]
+    # value block R x C/2, index block R x C/2 positions of 2 bits
+    assert vals.shape == (R, K // 2)
+    assert meta.size * 32 == R * (K // 2) * 2
+    # the 2-bit index against a 16-bit and an 8-bit value; the INT8 saving
+    assert 100 * 2 / 16 == g["index_overhead_fp16_percent"]
+    assert 100 * 2 / 8 == g["index_overhead_int8_percent"]
+    assert 100 * (1 - (2 * 8 + 2 * 2) / (4 * 8)) == g["int8_saving_percent"]
+
+
+@pytest.mark.parametrize("K,n,m,words", [(128, 2, 4, 4), (24, 2, 4, 1), (24, 1, 8, 1), (768, 1, 8, 10),
+                                         (256, 1, 4, 4), (4096, 2, 4, 128), (11008, 2, 4, 344)])
+def test_meta_sizes(K, n, m, words):
+    assert oracle.meta_cols(K, n, m) == words
+    assert oracle.value_cols(K, n, m) == K * n // m
+
+
+# ---------------------------------------------------------------------------
+# Decompression
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("n,m", PATTERNS)
+def test_roundtrip(n, m):
+    W = wl.integer_bf16((19, 8 * m), -2, 2, seed=11)  # many zeros and ties
+    W[0, :m] = bits_of([-0.0] * m)                    # a group of negative zeros
+    vals, meta = oracle.compress(W, n, m)
+    mask = oracle.prune_mask(W, n, m)
+    D = oracle.decompress(vals, meta, W.shape[1], n, m)
+    assert np.array_equal(D, np.where(mask == 1, W, np.uint16(0)))
+    vals2, meta2 = oracle.compress(D, n, m)
+    assert np.array_equal(vals2, vals) and np.array_equal(meta2, meta)
+
+
+# ---------------------------------------------------------------------------
+# Sparse GEMM
+# ---------------------------------------------------------------------------
+def test_k8_example(golden_dir):
+    g = json.load(open(os.path.join(golden_dir, "k8_example.json")))
+    W = bits_of([g["a_row"]])
+    vals, meta = oracle.compress(W, 2, 4)
+    assert vals.shape[1] == g["sparse_products"] and W.shape[1] == g["dense_products"]
+    assert np.array_equal(f64(vals[0]), np.array(g["expected_values"]))
+    pos = positions(meta[0], 4, 4)
+    assert [pos[0:2], pos[2:4]] == g["expected_positions"]
+    X = bits_of(np.array(g["b_col"], dtype=np.float32).reshape(8, 1))
+    y = oracle.spmm(vals, meta, 2, 4, 8, X)
+    assert y[0, 0] == g["expected_dot"]
+
+
+@pytest.mark.parametrize("n,m", [(2, 4), (1, 4), (1, 8), (3, 8)])
+def test_spmm_equals_dense_of_masked(n, m):
+    R, K, T = 23, 64 * m // 4 + 8 * m, 19
+    W = wl.normal_bf16((R, K), 1.0, seed=21)
+    X = wl.normal_bf16((K, T), 1.0, seed=22)
+    vals, meta = oracle.compress(W, n, m)
+    Wm = np.where(oracle.prune_mask(W, n, m) == 1, f64(W), 0.0)
+    ref = Wm @ f64(X)
+    y = oracle.spmm(vals, meta, n, m, K, X)
+    np.testing.assert_allclose(y, ref, rtol=1e-12, atol=1e-12)
+    yd = oracle.dense_gemm(oracle.decompress(vals, meta, K, n, m), X)
+    np.testing.assert_allclose(yd, ref, rtol=1e-12, atol=1e-12)
+
+
+def test_spmm_integer_exact():
+    """Integer inputs: every partial sum is an exact integer, so the result is exact."""
+    R, K, T = 17, 96, 13
+    W = wl.integer_bf16((R, K), -8, 8, seed=31)
+    X = wl.integer_bf16((K, T), -8, 8, seed=32)
+    vals, meta = oracle.compress(W, 2, 4)
+    Wm = np.where(oracle.prune_mask(W, 2, 4) == 1, f64(W), 0.0).astype(np.int64)
+    ref = Wm @ f64(X).astype(np.int64)
+    assert np.array_equal(oracle.spmm(vals, meta, 2, 4, K, X), ref.astype(np.float64))
+
+
+def test_spmm_bruteforce_tiny():
+    """Tiny case worked by hand-rolled loops: subset selection, then pure-Python dot products."""
+    rng = np.random.default_rng(5)
+    for n, m in [(2, 4), (1, 4), (1, 8)]:
+        Wf = rng.integers(-3, 4, size=(3, 2 * m)).astype(np.float32)
+        Xf = rng.integers(-3, 4, size=(2 * m, 2)).astype(np.float32)
+        W, X = bits_of(Wf), bits_of(Xf)
+        vals, meta = oracle.compress(W, n, m)
+        y = oracle.spmm(vals, meta, n, m, 2 * m, X)
+        for r in range(3):
+            kept = []
+            for g0 in range(0, 2 * m, m):
+                w = [float(v) for v in Wf[r, g0:g0 + m]]
+                win = [S for S in itertools.combinations(range(m), n)
+                       if all(_preferred(w, i, j) for i in S for j in range(m) if j not in S)]
+                kept += [g0 + p for p in win[0]]
+            for t in range(2):
+                assert y[r, t] == sum(float(Wf[r, k]) * float(Xf[k, t]) for k in kept)
+
+
+def test_sampled_matches_full():
+    R, K, T = 31, 256, 40
+    W = wl.normal_bf16((R, K), 0.02, seed=41)
+    X = wl.normal_bf16((K, T), 1.0, seed=42)
+    idx = wl.permutation(K, 43)
+    vals, meta = oracle.compress(W, 2, 4)
+    full = oracle.spmm(vals, meta, 2, 4, K, X, idx)
+    rows = np.array([0, 30, 7, 15, 30]); cols = np.array([0, 39, 20, 1, 0])
+    out, mag = oracle.spmm_sampled(vals, meta, 2, 4, K, X, rows, cols, idx)
+    assert np.array_equal(out, full[rows, cols])
+    Wm = np.abs(f64(oracle.decompress(vals, meta, K, 2, 4)))
+    np.testing.assert_allclose(mag, (Wm @ np.abs(f64(X)[idx]))[rows, cols], rtol=1e-12)
+
+
+def test_dense_gemm_matches_numpy():
+    W = wl.normal_bf16((9, 40), 1.0, seed=51)
+    X = wl.normal_bf16((40, 11), 1.0, seed=52)
+    Y, A = oracle.dense_gemm(W, X, with_abs=True)
+    np.testing.assert_allclose(Y, f64(W) @ f64(X), rtol=1e-12, atol=1e-13)
+    np.testing.assert_allclose(A, np.abs(f64(W)) @ np.abs(f64(X)), rtol=1e-12)
+
+
+# ---------------------------------------------------------------------------
+# Permuted input read, y = (W Pi) x
+# ---------------------------------------------------------------------------
+def test_identity_permutation_reduces_to_plain():
+    R, K, T = 20, 128, 24
+    W = wl.normal_bf16((R, K), 0.02, seed=61)
+    X = wl.normal_bf16((K, T), 1.0, seed=62)
+    vals, meta = oracle.compress(W, 2, 4)
+    a = oracle.spmm(vals, meta, 2, 4, K, X)
+    b = oracle.spmm(vals, meta, 2, 4, K, X, np.arange(K, dtype=np.int32))
+    assert np.array_equal(a, b)
+
+
+def test_permutation_matrix_form():
+    """y = (W' Pi) X with an explicit K x K permutation matrix, Pi[k, idx[k]] = 1."""
+    R, K, T = 6, 16, 5
+    W = wl.integer_bf16((R, K), -4, 4, seed=71)
+    X = wl.integer_bf16((K, T), -4, 4, seed=72)
+    idx = wl.permutation(K, 73)
+    vals, meta = oracle.compress(W, 2, 4)
+    Wm = f64(oracle.decompress(vals, meta, K, 2, 4))
+    Pi = np.zeros((K, K))
+    Pi[np.arange(K), idx] = 1.0
+    assert np.array_equal(oracle.spmm(vals, meta, 2, 4, K, X, idx), (Wm @ Pi) @ f64(X))
+
+
+def test_permutation_equals_permuted_input():
+    R, K, T = 12, 64, 9
+    W = wl.normal_bf16((R, K), 1.0, seed=81)
+    X = wl.normal_bf16((K, T), 1.0, seed=82)
+    idx = wl.permutation(K, 83)
+    vals, meta = oracle.compress(W, 1, 8)
+    assert np.array_equal(oracle.spmm(vals, meta, 1, 8, K, X, idx),
+                          oracle.spmm(vals, meta, 1, 8, K, np.ascontiguousarray(X[idx])))
+
+
+# ---------------------------------------------------------------------------
+# PATCH hybrid
+# ---------------------------------------------------------------------------
+def test_hybrid_special_cases():
+    R, K, T, tile = 40, 96, 7, 32
+    W = wl.integer_bf16((R, K), -5, 5, seed=91)
+    X = wl.integer_bf16((K, T), -5, 5, seed=92)
+    tiles = (-(-R // tile), -(-K // tile))
+    dense = oracle.hybrid_spmm(W, np.zeros(tiles, np.uint8), X, tile)
+    assert np.array_equal(dense, f64(W) @ f64(X))
+    vals, meta = oracle.compress(W, 2, 4)
+    sparse = oracle.hybrid_spmm(W, np.ones(tiles, np.uint8), X, tile)
+    assert np.array_equal(sparse, oracle.spmm(vals, meta, 2, 4, K, X))
+
+
+def test_hybrid_mixed_tiles():
+    R, K, T, tile = 64, 128, 10, 32
+    W = wl.normal_bf16((R, K), 0.02, seed=101)
+    X = wl.normal_bf16((K, T), 1.0, seed=102)
+    tm = wl.tile_map(2, 4, 0.5, seed=103)
+    mask = oracle.prune_mask(W, 2, 4)
+    sparse_el = np.kron(tm, np.ones((tile, tile), np.uint8)).astype(bool)
+    Weff = np.where(sparse_el & (mask == 0), 0.0, f64(W))
+    np.testing.assert_allclose(oracle.hybrid_spmm(W, tm, X, tile), Weff @ f64(X), rtol=1e-12, atol=1e-14)
+    assert np.array_equal(f64(oracle.hybrid_weights(W, tm, tile)), Weff)
+
+
+def test_rejects_bad_arguments():
+    W = wl.normal_bf16((4, 10), 1.0, seed=1)
+    with pytest.raises(ValueError):
+        oracle.compress(W, 2, 4)      # K % M != 0
+    with pytest.raises(ValueError):
+        oracle.compress(wl.normal_bf16((4, 12), 1.0, 1), 4, 4)  # N must be below M
+    with pytest.raises(ValueError):
+        oracle.compress(wl.normal_bf16((4, 12), 1.0, 1), 1, 3)  # M not a power of two
