@@ -1,0 +1,405 @@
+#!/usr/bin/env python
+"""Benchmark of the N:M sparse path on B200: useful TFLOP/s and roofline fraction.
+
+One step is one pass of the whole hot path over the LLaMA-7B-shaped 2:4
+workload with the learned-permutation stand-in: for each of the three linear
+shapes (4096x4096, 11008x4096, 4096x11008; T = 2048 tokens) the weights are
+magnitude-pruned and compressed to 2:4 (nm_prune_compress), then
+Y = (W' Pi) X runs with Pi applied as an index map on the input read
+(nm_spmm_permuted).  `value` is useful (non-zero) GEMM FLOPs per second of the
+whole step, inputs resident in HBM.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Under torchrun (N > 1) every rank runs its own replica of the workload (the
+path has no exchange step); timing is the max over ranks.  `--impl reference`
+times the fp64 CPU oracle on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads as wl  # noqa: E402
+
+METRIC = "N:M sparse GEMM useful TFLOP/s & % of sparse-TC/HBM roofline (1×B200)"
+WORKLOAD = "llama7b"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def parse_args(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--e2e-steps", type=int, default=5)
+    ap.add_argument("--cpu-seconds", type=float, default=10.0, help="target length of the oracle baseline sample")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    return ap.parse_args(argv)
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ----------------------------------------------------------------------------
+# Clock sampling during the timed region
+# ----------------------------------------------------------------------------
+class ClockSampler:
+    FIELDS = ("uuid,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, uuid: str, period_ms: int = 100):
+        self.uuid = uuid
+        self.period_ms = period_ms
+        self.rows = []
+        self.proc = None
+        self.thread = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 f"-lms", str(self.period_ms)], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (OSError, ValueError):
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+        time.sleep(0.3)
+
+    def _read(self):
+        for line in self.proc.stdout:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) >= 9:
+                self.rows.append(parts)
+
+    def stop(self):
+        if self.proc is None:
+            return
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        if self.thread:
+            self.thread.join(timeout=5)
+
+    def summary(self):
+        mine = [r for r in self.rows if self.uuid and self.uuid in r[0]] or self.rows
+        if not mine:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
+
+        def num(x):
+            try:
+                return float(x)
+            except ValueError:
+                return None
+        sm = [num(r[1]) for r in mine if num(r[1]) is not None]
+        mx = [num(r[2]) for r in mine if num(r[2]) is not None]
+        load = [s for s in sm if s > 0] or sm
+        reasons = set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in mine:
+            for name, v in zip(names, r[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(load) if load else None,
+                "sm_max_mhz": max(mx) if mx else None,
+                "reasons": sorted(reasons), "samples": len(mine)}
+
+
+# ----------------------------------------------------------------------------
+# Oracle baseline (CPU)
+# ----------------------------------------------------------------------------
+def oracle_sample(d, rows: int, cols: int):
+    """Oracle compress of `rows` weight rows and its permuted GEMM over `cols` tokens."""
+    import oracle
+    L = d.layer
+    Xs = np.ascontiguousarray(d.X[:, :cols])
+    t0 = time.perf_counter()
+    vals, meta = oracle.compress(np.ascontiguousarray(d.W[:rows]), 2, 4)
+    oracle.spmm(vals, meta, 2, 4, L.K, Xs, d.idx)
+    dt = time.perf_counter() - t0
+    flops = 2.0 * rows * cols * (L.K // 2)
+    return flops, dt
+
+
+def cpu_baseline(data, target_s: float):
+    d = data[0]
+    f0, t0 = oracle_sample(d, 16, 16)
+    rate = f0 / max(t0, 1e-9)
+    # scale the sample to about target_s seconds of single-thread oracle work
+    side = int(np.sqrt(max(target_s * rate / (2.0 * (d.layer.K // 2)), 256.0)))
+    rows = int(min(max(side, 16), d.layer.R))
+    cols = int(min(max(side, 16), d.layer.T))
+    flops, dt = oracle_sample(d, rows, cols)
+    return {"value": flops / dt / 1e12, "unit": "TFLOP/s", "cores": 1, "kind": "oracle",
+            "sample": f"{d.layer.name}: oracle compress of {rows} weight rows + permuted spmm of those rows "
+                      f"over {cols} of {d.layer.T} tokens ({flops / 1e9:.2f} useful GFLOP, {dt:.1f} s, "
+                      f"single thread)"}
+
+
+def run_reference(args, rank: int, world: int):
+    if rank != 0:
+        return
+    data = [wl.make_layer(L) for L in wl.workload(WORKLOAD)]
+    d = data[0]
+    rows, cols = 48, 64  # bounded sample per step
+    for _ in range(args.warmup):
+        oracle_sample(d, rows, cols)
+    t = 0.0
+    flops = 0.0
+    for _ in range(args.steps):
+        f, dt = oracle_sample(d, rows, cols)
+        t += dt
+        flops += f
+    value = flops / t / 1e12
+    cfg = {"workload": f"{WORKLOAD}_2of4_permuted", "shapes": [[L.layer.R, L.layer.K] for L in data],
+           "T": d.layer.T, "pattern": "2:4", "sample_per_step": f"{rows} rows x {cols} tokens of {d.layer.name}"}
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * t / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": cfg,
+            "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": 1, "kind": "oracle",
+                             "sample": cfg["sample_per_step"]},
+            "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ----------------------------------------------------------------------------
+# Our CUDA path
+# ----------------------------------------------------------------------------
+def run_ours(args, rank: int, world: int, dist):
+    import torch
+    import sparse_gemm_nm_b200 as nm
+
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    stream = torch.cuda.current_stream(dev)
+    sp = stream.cuda_stream
+    L_ = nm.lib()
+
+    layers = wl.workload(WORKLOAD)
+    data = [wl.make_layer(L) for L in layers]
+
+    def up(bits):
+        return torch.from_numpy(bits.view(np.int16)).to(dev).view(torch.bfloat16)
+
+    bufs = []
+    for d in data:
+        L = d.layer
+        W = up(d.W)
+        X = up(d.X)
+        idx = torch.from_numpy(d.idx).to(dev)
+        vals = torch.empty((L.R, L.K // 2), dtype=torch.bfloat16, device=dev)
+        meta = torch.empty((L.R, L.K // 32), dtype=torch.int32, device=dev)
+        Y = torch.empty((L.R, L.T), dtype=torch.bfloat16, device=dev)
+        bufs.append((L, W, X, idx, vals, meta, Y))
+    torch.cuda.synchronize()
+
+    def check(st, what):
+        if st != 0:
+            raise RuntimeError(f"{what}: {L_.nm_last_error().decode()}")
+
+    def launch_compress(b):
+        L, W, X, idx, vals, meta, Y = b
+        check(L_.nm_prune_compress(W.data_ptr(), L.R, L.K, L.K, 2, 4, vals.data_ptr(), meta.data_ptr(), sp),
+              "nm_prune_compress")
+
+    def launch_spmm(b):
+        L, W, X, idx, vals, meta, Y = b
+        check(L_.nm_spmm_permuted(vals.data_ptr(), meta.data_ptr(), 2, 4, L.R, L.K, idx.data_ptr(),
+                                  X.data_ptr(), L.T, L.T, Y.data_ptr(), L.T, 0, sp), "nm_spmm_permuted")
+
+    def step(evs=None):
+        for i, b in enumerate(bufs):
+            if evs is not None:
+                evs[2 * i].record(stream)
+            launch_compress(b)
+            if evs is not None:
+                evs[2 * i + 1].record(stream)
+            launch_spmm(b)
+        if evs is not None:
+            evs[2 * len(bufs)].record(stream)
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+
+    useful = sum(2.0 * L.T * L.R * (L.K // 2) for (L, *_rest) in bufs)
+    comp_bytes = [2.0 * L.R * L.K + L.R * L.K + L.R * L.K / 8.0 for (L, *_r) in bufs]
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    nm.nm_device_status(sp)
+
+    props = torch.cuda.get_device_properties(dev)
+    sampler = ClockSampler(f"GPU-{props.uuid}" if getattr(props, "uuid", None) else "")
+    sampler.start()
+
+    nev = 2 * len(bufs) + 1
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(nev)] for _ in range(args.steps)]
+    launches0 = nm.nm_launch_count()
+    barrier()
+    torch.cuda.synchronize()
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    t_start.record(stream)
+    for k in range(args.steps):
+        step(evs[k])
+    t_end.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    launches = nm.nm_launch_count() - launches0
+    sampler.stop()
+    nm.nm_device_status(sp)
+
+    elapsed_ms = t_start.elapsed_time(t_end)
+    if dist is not None:
+        t = torch.tensor([elapsed_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        elapsed_ms = float(t.item())
+    ms_per_step = elapsed_ms / args.steps
+
+    # per-kernel durations over the timed region (same stream as the launches)
+    comp_ms = np.zeros(len(bufs))
+    spmm_ms = np.zeros(len(bufs))
+    for k in range(args.steps):
+        e = evs[k]
+        for i in range(len(bufs)):
+            comp_ms[i] += e[2 * i].elapsed_time(e[2 * i + 1])
+            spmm_ms[i] += e[2 * i + 1].elapsed_time(e[2 * i + 2])
+    comp_ms /= args.steps
+    spmm_ms /= args.steps
+
+    peaks, peak_src = load_peaks()
+    timed_s = elapsed_ms / 1e3
+    sustained = timed_s > 1.0
+    tc_peak = peaks["bf16_tflops_sustained" if sustained else "bf16_tflops"]
+    hbm_peak = peaks["hbm_gbs"]
+    spmm_flops = [2.0 * L.T * L.R * (L.K // 2) for (L, *_r) in bufs]
+    achieved = sum(spmm_flops) / (spmm_ms.sum() * 1e-3) / 1e12
+    kernels = {}
+    for i, (L, *_r) in enumerate(bufs):
+        kernels[L.name] = {
+            "spmm_us": 1e3 * spmm_ms[i], "spmm_tflops": spmm_flops[i] / (spmm_ms[i] * 1e-3) / 1e12,
+            "spmm_frac": spmm_flops[i] / (spmm_ms[i] * 1e-3) / 1e12 / tc_peak,
+            "compress_us": 1e3 * comp_ms[i], "compress_gbs": comp_bytes[i] / (comp_ms[i] * 1e-3) / 1e9,
+            "compress_frac": comp_bytes[i] / (comp_ms[i] * 1e-3) / 1e9 / hbm_peak}
+    traffic = None
+    tfile = os.path.join(ROOT, "profiles", "spmm_traffic.json")
+    if os.path.exists(tfile):
+        with open(tfile) as f:
+            traffic = json.load(f).get("bytes_per_launch")
+    roofline = {"bound": "tensor", "achieved": achieved, "peak": tc_peak, "unit": "TFLOP/s",
+                "frac": achieved / tc_peak, "traffic": traffic,
+                "kernel": "nm_spmm_permuted (tcgen05.mma.sp, 2:4 + index-map gather)",
+                "peak_source": f"{peak_src} bf16 {'sustained' if sustained else 'burst'} dense peak; useful "
+                               "2:4 FLOPs run at half the sparse MMA rate, i.e. at the dense rate",
+                "algorithmic_flops_per_launch": spmm_flops}
+
+    line = {"metric": METRIC, "value": world * useful / (ms_per_step * 1e-3) / 1e12, "unit": "TFLOP/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded numpy PCG64, N(0,0.02) weights, N(0,1) inputs, random permutation)",
+            "config": {"workload": f"{WORKLOAD}_2of4_permuted", "shapes": [[L.R, L.K] for (L, *_r) in bufs],
+                       "T": bufs[0][0].T, "pattern": "2:4", "step": "prune+compress then permuted spmm, 3 layers",
+                       "l2": "inputs larger than L2 (about 290 MB touched per step > 126 MB)",
+                       "parallelism": f"replicas x{world}"},
+            "roofline": roofline, "kernels": kernels, "gpu_launches": launches,
+            "clocks": sampler.summary()}
+
+    # end-to-end through the public API with host buffers
+    if not args.no_e2e:
+        hW = [torch.from_numpy(d.W.view(np.int16)).pin_memory() for d in data]
+        hX = [torch.from_numpy(d.X.view(np.int16)).pin_memory() for d in data]
+        hI = [torch.from_numpy(d.idx).pin_memory() for d in data]
+        hY = [torch.empty((b[0].R, b[0].T), dtype=torch.int16).pin_memory() for b in bufs]
+        h2d = sum(a.numel() * a.element_size() for a in hW + hX + hI)
+        d2h = sum(a.numel() * a.element_size() for a in hY)
+
+        def e2e_step():
+            for i, b in enumerate(bufs):
+                L, W, X, idx, vals, meta, Y = b
+                W.view(torch.int16).copy_(hW[i], non_blocking=True)
+                X.view(torch.int16).copy_(hX[i], non_blocking=True)
+                idx.copy_(hI[i], non_blocking=True)
+                launch_compress(b)
+                launch_spmm(b)
+                hY[i].copy_(Y.view(torch.int16), non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize()
+        barrier()
+        a = torch.cuda.Event(enable_timing=True)
+        z = torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(args.e2e_steps):
+            e2e_step()
+        z.record(stream)
+        torch.cuda.synchronize()
+        e_ms = a.elapsed_time(z)
+        if dist is not None:
+            t = torch.tensor([e_ms], dtype=torch.float64, device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            e_ms = float(t.item())
+        line["e2e"] = {"value": world * useful * args.e2e_steps / (e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+                       "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                       "ms_per_step": e_ms / args.e2e_steps}
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(data, args.cpu_seconds)
+    elif rank == 0:
+        line["cpu_baseline"] = None
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        return 0
+    dist = None
+    if world > 1:
+        import datetime
+
+        import torch
+        import torch.distributed as tdist
+        torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", "0")))
+        tdist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+        dist = tdist
+    try:
+        run_ours(args, rank, world, dist)
+    finally:
+        if dist is not None:
+            dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

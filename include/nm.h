@@ -1,0 +1,199 @@
+/*
+ * nm.h -- C ABI of libnm_b200, N:M structured weight sparsity on NVIDIA B200
+ * (sm_100a): magnitude prune + push-left compression, decompression, and the
+ * sparse x dense GEMM y = (W Pi) x in plain, column-permuted and PATCH-style
+ * hybrid forms.
+ *
+ * Conventions shared by every call
+ *  - bf16 data is passed as its 16-bit pattern (uint16_t).  All matrices are
+ *    row-major.  W is R x K (R output features, K the reduction axis), X is
+ *    K x T (T tokens, contiguous), Y is R x T.
+ *  - An N:M pattern groups M consecutive weights along K.  Supported M is 2,
+ *    4, 8 or 16 with 1 <= N < M, and K must be a multiple of M.
+ *  - Compressed form ("values" + "meta"):
+ *      values  R x (K*N/M) bf16, the N survivors of each group pushed left in
+ *              ascending position order; row stride K*N/M.
+ *      meta    R x nm_meta_cols(K,N,M) uint32 words; survivor j of a row
+ *              stores its in-group position (b = ceil(log2 M) bits) in word
+ *              floor(j/S) at bit b*(j mod S), S = floor(32/b); unused bits 0.
+ *              For 2:4 this is one nibble per group, first survivor in the
+ *              low two bits, group 0 in the lowest nibble.
+ *  - Every pointer is DEVICE memory owned by the caller (none is freed or
+ *    retained).  The library allocates no device memory on these paths.
+ *  - Calls are asynchronous on `stream` (a cudaStream_t; NULL = the legacy
+ *    default stream).  Argument errors are detected on the host and returned
+ *    before anything is launched.  Each successful call launches exactly one
+ *    kernel (none when the output is empty).
+ *  - Device pointers given to the GEMMs must be 16-byte aligned, and leading
+ *    dimensions of X and Y must keep every row 16-byte aligned
+ *    (NM_ERR_MISALIGNED otherwise).
+ *  - Waits inside the GEMM kernels are bounded (about 2 s); a kernel that gives
+ *    up records it in a device status word read by nm_device_status().
+ *  - Inputs are expected to be finite.  With an Inf or NaN in X the result may
+ *    differ from the sum over stored survivors (zeros padded in by the kernel
+ *    can meet it).
+ */
+#ifndef NM_B200_H
+#define NM_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define NM_API __attribute__((visibility("default")))
+#else
+#define NM_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum nm_status {
+  NM_OK = 0,
+  NM_ERR_INVALID_ARG = 1, /* null pointer, bad shape or pattern, ld too small */
+  NM_ERR_UNSUPPORTED = 2, /* valid request outside what this build implements */
+  NM_ERR_MISALIGNED = 3,  /* pointer / leading dimension breaks 16-byte rows   */
+  NM_ERR_CUDA = 4,        /* a CUDA runtime or driver call failed              */
+  NM_ERR_TIMEOUT = 5,     /* a kernel's bounded wait gave up (device status)   */
+  NM_ERR_NO_DEVICE = 6    /* no sm_100 device is current                       */
+} nm_status;
+
+typedef enum nm_out_dtype { NM_OUT_BF16 = 0, NM_OUT_F32 = 1 } nm_out_dtype;
+
+/* Kernel design for nm_spmm_algo.  AUTO: 2:4 and patterns that fit inside
+ * 2:4 (1:2, 1:4, 1:8, 2:8) use the sparse tensor-core MMA, other patterns the
+ * dense expansion. */
+typedef enum nm_algo {
+  NM_ALGO_AUTO = 0,
+  NM_ALGO_SPARSE_TC = 1, /* tcgen05.mma.sp; 1:4 / 1:8 re-encoded as 2:4 while loading */
+  NM_ALGO_DENSE_TC = 2   /* survivors expanded into a dense tile, dense tcgen05.mma   */
+} nm_algo;
+
+/* ------------------------------------------------------------------ sizes */
+/* Bits per stored position, ceil(log2 m); 0 for an unsupported m. */
+NM_API int nm_index_bits(int m);
+/* Columns of the value block, K*n/m (-1 on a bad pattern or K % m != 0). */
+NM_API int64_t nm_value_cols(int64_t K, int n, int m);
+/* 32-bit metadata words per row (-1 on a bad pattern or K % m != 0). */
+NM_API int64_t nm_meta_cols(int64_t K, int n, int m);
+
+/* ------------------------------------------------------------- compress */
+/*
+ * nm_prune_compress -- keep the n largest-magnitude weights of every group of
+ * m consecutive weights along each row of W, ties going to the lower index,
+ * and write them in compressed form.
+ * Source: "M:N sparsity on NVIDIA tensor cores" -- opening passage (groups of
+ * four along a row, two survivors anywhere inside, metadata [[0,3],[1,2]] of
+ * the worked row), "The recipe" step 2 (zero the smallest magnitudes), and the
+ * storage paragraphs of "Where this sits among the three case studies"
+ * (survivors pushed left into an R x C/2 block plus 2-bit positions).
+ *   W       [in]  R x K bf16, row stride ldw >= K (elements)
+ *   values  [out] R x nm_value_cols(K,n,m) bf16
+ *   meta    [out] R x nm_meta_cols(K,n,m) uint32 (fully written, unused bits 0)
+ * Magnitudes are compared on the bf16 value: +0 and -0 tie, a NaN ranks above
+ * every number.  Exactly n survivors are stored per group, zeros included.
+ * Errors: NM_ERR_INVALID_ARG (bad pattern, K % m, ldw < K, null pointer).
+ */
+NM_API nm_status nm_prune_compress(const uint16_t* W, int64_t R, int64_t K, int64_t ldw, int n, int m,
+                            uint16_t* values, uint32_t* meta, void* stream);
+
+/*
+ * nm_decompress -- scatter the survivors back to their positions; every other
+ * element becomes +0 (bits 0x0000).  decompress(compress(W)) is W with the
+ * pruned weights replaced by +0.
+ * Source: same storage paragraphs (a survivor's place follows from its group
+ * and its stored position; no pointers are needed).
+ *   values, meta [in]  compressed form of an R x K matrix (layout above)
+ *   W_out        [out] R x K bf16, row stride ldw >= K
+ * Errors: NM_ERR_INVALID_ARG.
+ */
+NM_API nm_status nm_decompress(const uint16_t* values, const uint32_t* meta, int64_t R, int64_t K, int n, int m,
+                        uint16_t* W_out, int64_t ldw, void* stream);
+
+/* ----------------------------------------------------------------- GEMM */
+/*
+ * nm_spmm -- Y = W' X with W' the decompressed weights, computed from the
+ * compressed operand (only the weights are compressed; X and Y are dense).
+ * Products are exact and accumulate in fp32 on the tensor cores; Y is rounded
+ * once (bf16 round-to-nearest-even, or stored as fp32).
+ * Source: "M:N sparsity on NVIDIA tensor cores", GEMM paragraphs of "Where
+ * this sits among the three case studies" (the indices pick the elements of
+ * the dense operand; sparse x dense = dense) and the K-axis rule.
+ *   values, meta [in] compressed R x K weights, pattern n:m
+ *   X            [in] K x T bf16, row stride ldx >= T, ldx % 8 == 0
+ *   Y            [out] R x T, bf16 or fp32 (y_dtype), row stride ldy >= T
+ * Errors: NM_ERR_INVALID_ARG, NM_ERR_MISALIGNED, NM_ERR_CUDA.
+ */
+NM_API nm_status nm_spmm(const uint16_t* values, const uint32_t* meta, int n, int m, int64_t R, int64_t K,
+                  const uint16_t* X, int64_t ldx, int64_t T, void* Y, int64_t ldy, nm_out_dtype y_dtype,
+                  void* stream);
+
+/*
+ * nm_spmm_permuted -- Y = (W' Pi) X with the hard column permutation Pi given
+ * as an index map: row k of the permuted input is X[idx[k]], so
+ * y[r][t] = sum_k W'[r][k] * X[idx[k]][t].  The kernel reads X at the mapped
+ * rows while staging its tiles; there is no separate permute pass and the
+ * FLOP count is that of nm_spmm.  An identity map gives nm_spmm's result.
+ * Source: "Technische Samenvatting: SHUFFLESPARSE", section "2. Methodologie"
+ * (y = (W Pi) x; at inference Pi is a precomputed index map and the structured
+ * sparse GEMM reads its input at the permuted addresses).
+ *   idx [in] K int32 device array; entries outside [0, K) read as zero rows.
+ * Other arguments as nm_spmm.
+ */
+NM_API nm_status nm_spmm_permuted(const uint16_t* values, const uint32_t* meta, int n, int m, int64_t R, int64_t K,
+                           const int32_t* idx, const uint16_t* X, int64_t ldx, int64_t T, void* Y, int64_t ldy,
+                           nm_out_dtype y_dtype, void* stream);
+
+/*
+ * nm_hybrid_spmm -- PATCH-style hybrid GEMM: W is split into tile x tile
+ * blocks; block (i, j) uses the dense weights when tile_map[i][j] == 0 and the
+ * 2:4-pruned weights when it is 1.  Dense blocks are read from W, 2:4 blocks
+ * from the 2:4 compressed form of the whole W (nm_prune_compress(W, 2, 4));
+ * both accumulate into one output tile.
+ * Source: "Structured Sparsity" topic cards, PATCH abstract (weight matrices
+ * partitioned into tiles, each tile either dense or 2:4 sparse).
+ *   W        [in] R x K bf16, row stride ldw >= K, ldw % 8 == 0 (dense tiles)
+ *   values, meta [in] nm_prune_compress(W, 2, 4) (2:4 tiles)
+ *   tile_map [in] ceil(R/tile) x ceil(K/tile) uint8, 0 = dense, 1 = 2:4
+ *   tile     [in] must be 128
+ * Other arguments as nm_spmm.  Errors: as nm_spmm, NM_ERR_UNSUPPORTED for
+ * tile != 128 or K % 16 != 0.
+ */
+NM_API nm_status nm_hybrid_spmm(const uint16_t* W, int64_t ldw, const uint16_t* values, const uint32_t* meta,
+                         const uint8_t* tile_map, int tile, int64_t R, int64_t K, const uint16_t* X,
+                         int64_t ldx, int64_t T, void* Y, int64_t ldy, nm_out_dtype y_dtype, void* stream);
+
+/*
+ * nm_spmm_algo -- nm_spmm / nm_spmm_permuted (idx may be NULL) with the kernel
+ * design chosen explicitly, to compare the sparse tensor-core path with the
+ * dense expansion on the same pattern.  NM_ERR_UNSUPPORTED when the pattern
+ * does not fit the requested design (NM_ALGO_SPARSE_TC with 3:4, say).
+ */
+NM_API nm_status nm_spmm_algo(const uint16_t* values, const uint32_t* meta, int n, int m, int64_t R, int64_t K,
+                       const int32_t* idx, const uint16_t* X, int64_t ldx, int64_t T, void* Y, int64_t ldy,
+                       nm_out_dtype y_dtype, nm_algo algo, void* stream);
+
+/* ------------------------------------------------------------ utilities */
+/* Synchronises `stream`, then returns NM_ERR_TIMEOUT if any kernel of this
+ * library recorded a bounded wait that gave up since the previous call (and
+ * clears the record), NM_ERR_CUDA on a pending CUDA error, else NM_OK. */
+NM_API nm_status nm_device_status(void* stream);
+
+/* Static description of a status code. */
+NM_API const char* nm_status_string(nm_status s);
+
+/* Text of the most recent error of the calling host thread ("" if none). */
+NM_API const char* nm_last_error(void);
+
+/* Number of kernels this library has launched in this process. */
+NM_API uint64_t nm_launch_count(void);
+
+/* ABI version: major * 10000 + minor * 100 + patch. */
+NM_API int nm_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* NM_B200_H */

@@ -1,0 +1,229 @@
+"""sparse_gemm_nm_b200 -- N:M structured weight sparsity on NVIDIA B200 (sm_100a).
+
+Python binding of the C ABI in ``include/nm.h`` (library ``libnm_b200.so``).
+The functions named like the C entry points (``nm_prune_compress``,
+``nm_decompress``, ``nm_spmm``, ``nm_spmm_permuted``, ``nm_hybrid_spmm``,
+``nm_spmm_algo``) only marshal arguments: tensors become device pointers, the
+stream defaults to torch's current stream, and a non-zero status raises
+:class:`NmError`.  Every step of the computation runs in the library's CUDA
+kernels; there is no fallback of any kind.  The convenience wrappers
+(``prune_compress``, ``decompress``, ``spmm``, ``hybrid_spmm``) also allocate
+the outputs with torch.
+
+bf16 data is accepted as ``torch.bfloat16`` tensors (or int16/uint16 views of
+the same bits).  Matrices are row-major: W is R x K, X is K x T, Y is R x T.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Tuple
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libnm_b200.so")
+
+NM_OK = 0
+NM_ERR_INVALID_ARG = 1
+NM_ERR_UNSUPPORTED = 2
+NM_ERR_MISALIGNED = 3
+NM_ERR_CUDA = 4
+NM_ERR_TIMEOUT = 5
+NM_ERR_NO_DEVICE = 6
+
+NM_OUT_BF16 = 0
+NM_OUT_F32 = 1
+
+NM_ALGO_AUTO = 0
+NM_ALGO_SPARSE_TC = 1
+NM_ALGO_DENSE_TC = 2
+
+# Every symbol include/nm.h declares, with its ctypes signature.
+_P, _I64, _I, _U64 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_uint64
+SIGNATURES = {
+    "nm_index_bits": ([_I], _I),
+    "nm_value_cols": ([_I64, _I, _I], _I64),
+    "nm_meta_cols": ([_I64, _I, _I], _I64),
+    "nm_prune_compress": ([_P, _I64, _I64, _I64, _I, _I, _P, _P, _P], _I),
+    "nm_decompress": ([_P, _P, _I64, _I64, _I, _I, _P, _I64, _P], _I),
+    "nm_spmm": ([_P, _P, _I, _I, _I64, _I64, _P, _I64, _I64, _P, _I64, _I, _P], _I),
+    "nm_spmm_permuted": ([_P, _P, _I, _I, _I64, _I64, _P, _P, _I64, _I64, _P, _I64, _I, _P], _I),
+    "nm_hybrid_spmm": ([_P, _I64, _P, _P, _P, _I, _I64, _I64, _P, _I64, _I64, _P, _I64, _I, _P], _I),
+    "nm_spmm_algo": ([_P, _P, _I, _I, _I64, _I64, _P, _P, _I64, _I64, _P, _I64, _I, _I, _P], _I),
+    "nm_device_status": ([_P], _I),
+    "nm_status_string": ([_I], ctypes.c_char_p),
+    "nm_last_error": ([], ctypes.c_char_p),
+    "nm_launch_count": ([], _U64),
+    "nm_version": ([], _I),
+}
+
+
+class NmError(RuntimeError):
+    def __init__(self, status: int, where: str, detail: str):
+        super().__init__(f"{where}: status {status} ({_status_text(status)}): {detail}")
+        self.status = status
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded libnm_b200.so.  Raises ImportError when it has not been built."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"{LIB_PATH} is missing: build it with `python -m sparse_gemm_nm_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        for name, (args, res) in SIGNATURES.items():
+            fn = getattr(L, name)
+            fn.argtypes = args
+            fn.restype = res
+        _lib = L
+    return _lib
+
+
+def _status_text(s: int) -> str:
+    try:
+        return lib().nm_status_string(s).decode()
+    except Exception:  # pragma: no cover - only while reporting another failure
+        return "?"
+
+
+def _check(status: int, where: str) -> None:
+    if status != NM_OK:
+        raise NmError(status, where, lib().nm_last_error().decode())
+
+
+def _ptr(x) -> Optional[int]:
+    if x is None:
+        return None
+    if isinstance(x, int):
+        return x
+    return x.data_ptr()
+
+
+def _stream(stream) -> Optional[int]:
+    if stream is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+# ----------------------------------------------------------------------------
+# C-ABI names (argument marshalling only)
+# ----------------------------------------------------------------------------
+def nm_index_bits(m: int) -> int:
+    return lib().nm_index_bits(m)
+
+
+def nm_value_cols(K: int, n: int, m: int) -> int:
+    return lib().nm_value_cols(K, n, m)
+
+
+def nm_meta_cols(K: int, n: int, m: int) -> int:
+    return lib().nm_meta_cols(K, n, m)
+
+
+def nm_prune_compress(W, R, K, ldw, n, m, values, meta, stream=None) -> None:
+    _check(lib().nm_prune_compress(_ptr(W), R, K, ldw, n, m, _ptr(values), _ptr(meta), _stream(stream)),
+           "nm_prune_compress")
+
+
+def nm_decompress(values, meta, R, K, n, m, W_out, ldw, stream=None) -> None:
+    _check(lib().nm_decompress(_ptr(values), _ptr(meta), R, K, n, m, _ptr(W_out), ldw, _stream(stream)),
+           "nm_decompress")
+
+
+def nm_spmm(values, meta, n, m, R, K, X, ldx, T, Y, ldy, y_dtype=NM_OUT_BF16, stream=None) -> None:
+    _check(lib().nm_spmm(_ptr(values), _ptr(meta), n, m, R, K, _ptr(X), ldx, T, _ptr(Y), ldy, y_dtype,
+                         _stream(stream)), "nm_spmm")
+
+
+def nm_spmm_permuted(values, meta, n, m, R, K, idx, X, ldx, T, Y, ldy, y_dtype=NM_OUT_BF16,
+                     stream=None) -> None:
+    _check(lib().nm_spmm_permuted(_ptr(values), _ptr(meta), n, m, R, K, _ptr(idx), _ptr(X), ldx, T, _ptr(Y),
+                                  ldy, y_dtype, _stream(stream)), "nm_spmm_permuted")
+
+
+def nm_hybrid_spmm(W, ldw, values, meta, tile_map, tile, R, K, X, ldx, T, Y, ldy, y_dtype=NM_OUT_BF16,
+                   stream=None) -> None:
+    _check(lib().nm_hybrid_spmm(_ptr(W), ldw, _ptr(values), _ptr(meta), _ptr(tile_map), tile, R, K, _ptr(X),
+                                ldx, T, _ptr(Y), ldy, y_dtype, _stream(stream)), "nm_hybrid_spmm")
+
+
+def nm_spmm_algo(values, meta, n, m, R, K, idx, X, ldx, T, Y, ldy, y_dtype=NM_OUT_BF16, algo=NM_ALGO_AUTO,
+                 stream=None) -> None:
+    _check(lib().nm_spmm_algo(_ptr(values), _ptr(meta), n, m, R, K, _ptr(idx), _ptr(X), ldx, T, _ptr(Y), ldy,
+                              y_dtype, algo, _stream(stream)), "nm_spmm_algo")
+
+
+def nm_device_status(stream=None) -> None:
+    _check(lib().nm_device_status(_stream(stream)), "nm_device_status")
+
+
+def nm_launch_count() -> int:
+    return int(lib().nm_launch_count())
+
+
+def nm_version() -> int:
+    return int(lib().nm_version())
+
+
+# ----------------------------------------------------------------------------
+# Convenience wrappers that allocate outputs with torch
+# ----------------------------------------------------------------------------
+def _require_cuda(*ts):
+    for t in ts:
+        if t is not None and not t.is_cuda:
+            raise ValueError("tensors must live on a CUDA device")
+
+
+def prune_compress(W, n: int, m: int, stream=None):
+    """(values R x K*n/m bf16, meta R x nm_meta_cols uint32-as-int32) of bf16 W (R x K)."""
+    import torch
+    _require_cuda(W)
+    R, K = W.shape
+    vals = torch.empty((R, nm_value_cols(K, n, m)), dtype=torch.bfloat16, device=W.device)
+    meta = torch.empty((R, max(nm_meta_cols(K, n, m), 0)), dtype=torch.int32, device=W.device)
+    nm_prune_compress(W, R, K, W.stride(0), n, m, vals, meta, stream)
+    return vals, meta
+
+
+def decompress(values, meta, K: int, n: int, m: int, stream=None):
+    import torch
+    _require_cuda(values, meta)
+    R = values.shape[0]
+    out = torch.empty((R, K), dtype=torch.bfloat16, device=values.device)
+    nm_decompress(values, meta, R, K, n, m, out, K, stream)
+    return out
+
+
+def spmm(values, meta, n: int, m: int, K: int, X, idx=None, out_dtype=None, algo: int = NM_ALGO_AUTO,
+         stream=None):
+    """Y = (W' Pi) X from the compressed operand; idx=None means Pi = I."""
+    import torch
+    _require_cuda(values, meta, X, idx)
+    out_dtype = out_dtype or torch.bfloat16
+    R, T = values.shape[0], X.shape[1]
+    Y = torch.empty((R, T), dtype=out_dtype, device=X.device)
+    yt = NM_OUT_F32 if out_dtype == torch.float32 else NM_OUT_BF16
+    if algo == NM_ALGO_AUTO and idx is None:
+        nm_spmm(values, meta, n, m, R, K, X, X.stride(0), T, Y, T, yt, stream)
+    elif algo == NM_ALGO_AUTO:
+        nm_spmm_permuted(values, meta, n, m, R, K, idx, X, X.stride(0), T, Y, T, yt, stream)
+    else:
+        nm_spmm_algo(values, meta, n, m, R, K, idx, X, X.stride(0), T, Y, T, yt, algo, stream)
+    return Y
+
+
+def hybrid_spmm(W, values, meta, tile_map, X, tile: int = 128, out_dtype=None, stream=None):
+    import torch
+    _require_cuda(W, values, meta, tile_map, X)
+    out_dtype = out_dtype or torch.bfloat16
+    R, K = W.shape
+    T = X.shape[1]
+    Y = torch.empty((R, T), dtype=out_dtype, device=X.device)
+    yt = NM_OUT_F32 if out_dtype == torch.float32 else NM_OUT_BF16
+    nm_hybrid_spmm(W, W.stride(0), values, meta, tile_map, tile, R, K, X, X.stride(0), T, Y, T, yt, stream)
+    return Y

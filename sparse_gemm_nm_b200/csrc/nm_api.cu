@@ -1,0 +1,377 @@
+// nm_api.cu -- the C ABI of libnm_b200 (declared in include/nm.h): argument
+// checks on the host, tensor-map encoding, choice of kernel variant, launch.
+#include <atomic>
+#include <cstdarg>
+#include <cstdint>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <string>
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include "../../include/nm.h"
+#include "nm_internal.h"
+#include "nm_spmm.h"
+
+namespace nmk {
+
+static std::atomic<uint64_t> g_launches{0};
+void count_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
+
+static thread_local std::string t_last_error;
+
+static nm_status fail(nm_status s, const char* fmt, ...) __attribute__((format(printf, 2, 3)));
+static nm_status fail(nm_status s, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof buf, fmt, ap);
+  va_end(ap);
+  t_last_error = buf;
+  return s;
+}
+
+static nm_status cuda_fail(cudaError_t e, const char* what) {
+  return fail(NM_ERR_CUDA, "%s: %s (%s)", what, cudaGetErrorName(e), cudaGetErrorString(e));
+}
+
+struct DeviceInfo {
+  int sms = 0;
+  int major = 0;
+  bool known = false;
+};
+static DeviceInfo g_dev[64];
+static std::mutex g_dev_mu;
+
+static const DeviceInfo* device_info() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  std::lock_guard<std::mutex> lk(g_dev_mu);
+  DeviceInfo& d = g_dev[dev];
+  if (!d.known) {
+    if (cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return nullptr;
+    if (cudaDeviceGetAttribute(&d.major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess) return nullptr;
+    d.known = true;
+  }
+  return &d;
+}
+
+int sm_count_current() {
+  const DeviceInfo* d = device_info();
+  return d ? d->sms : 148;
+}
+
+static nm_status require_device() {
+  const DeviceInfo* d = device_info();
+  if (!d) return fail(NM_ERR_NO_DEVICE, "no CUDA device is current");
+  if (d->major != 10) return fail(NM_ERR_NO_DEVICE, "device is sm_%d0, this library is built for sm_100a", d->major);
+  return NM_OK;
+}
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point.
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+static nm_status make_tmap(CUtensorMap* tm, const void* base, uint64_t inner, uint64_t outer,
+                           uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer, int swizzle_bytes,
+                           const char* what) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return fail(NM_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {row_bytes};
+  cuuint32_t box[2] = {box_inner, box_outer};
+  cuuint32_t estr[2] = {1, 1};
+  CUtensorMapSwizzle swz = swizzle_bytes == 128  ? CU_TENSOR_MAP_SWIZZLE_128B
+                           : swizzle_bytes == 64 ? CU_TENSOR_MAP_SWIZZLE_64B
+                                                 : CU_TENSOR_MAP_SWIZZLE_32B;
+  CUresult r = fn(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(NM_ERR_CUDA, "cuTensorMapEncodeTiled(%s) failed with %d", what, (int)r);
+  return NM_OK;
+}
+
+static bool al16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+static int pattern_id(int n, int m) {
+  if (n == 2 && m == 4) return PAT_2_4;
+  if (n == 1 && m == 2) return PAT_1_2;
+  if (n == 1 && m == 4) return PAT_1_4;
+  if (n == 1 && m == 8) return PAT_1_8;
+  if (n == 2 && m == 8) return PAT_2_8;
+  return PAT_OTHER;
+}
+
+static int pick_bn(int64_t T) {
+  int bn = 16;
+  while (bn < T && bn < 256) bn *= 2;
+  return bn;
+}
+
+struct GemmRequest {
+  const uint16_t* values;
+  const uint32_t* meta;
+  int n, m;
+  int64_t R, K, T;
+  const int32_t* idx;
+  const uint16_t* X;
+  int64_t ldx;
+  void* Y;
+  int64_t ldy;
+  int y_dtype;
+  nm_algo algo;
+  // hybrid
+  bool hybrid;
+  const uint16_t* W;
+  int64_t ldw;
+  const uint8_t* tile_map;
+  int tile;
+};
+
+static nm_status run_gemm(const GemmRequest& q, cudaStream_t stream) {
+  t_last_error.clear();
+  if (q.R < 0 || q.K < 0 || q.T < 0) return fail(NM_ERR_INVALID_ARG, "negative dimension");
+  if (!pattern_ok(q.n, q.m)) return fail(NM_ERR_INVALID_ARG, "pattern %d:%d not supported (M in 2,4,8,16; 1<=N<M)", q.n, q.m);
+  if (q.K % q.m != 0) return fail(NM_ERR_INVALID_ARG, "K=%lld is not a multiple of M=%d", (long long)q.K, q.m);
+  if (q.y_dtype != NM_OUT_BF16 && q.y_dtype != NM_OUT_F32) return fail(NM_ERR_INVALID_ARG, "bad output dtype");
+  if (q.algo != NM_ALGO_AUTO && q.algo != NM_ALGO_SPARSE_TC && q.algo != NM_ALGO_DENSE_TC)
+    return fail(NM_ERR_INVALID_ARG, "bad algorithm");
+  if (q.R == 0 || q.T == 0) return NM_OK;
+  if (!q.Y) return fail(NM_ERR_INVALID_ARG, "Y is null");
+  if (q.ldy < q.T) return fail(NM_ERR_INVALID_ARG, "ldy < T");
+  const int esize = q.y_dtype == NM_OUT_F32 ? 4 : 2;
+  if (!al16(q.Y) || (q.ldy * esize) % 16 != 0) return fail(NM_ERR_MISALIGNED, "Y rows must be 16-byte aligned");
+  nm_status st = require_device();
+  if (st != NM_OK) return st;
+  if (q.K == 0) {
+    cudaError_t e = launch_fill_zero(q.Y, q.R, q.T, q.ldy, esize, stream);
+    return e == cudaSuccess ? NM_OK : cuda_fail(e, "zero fill");
+  }
+  if (!q.values || !q.meta || !q.X) return fail(NM_ERR_INVALID_ARG, "null operand");
+  if (q.ldx < q.T) return fail(NM_ERR_INVALID_ARG, "ldx < T");
+  if (!al16(q.X) || q.ldx % 8 != 0) return fail(NM_ERR_MISALIGNED, "X rows must be 16-byte aligned");
+  if (q.R >= (1ll << 31) || q.K >= (1ll << 31) || q.T >= (1ll << 31))
+    return fail(NM_ERR_UNSUPPORTED, "dimensions must stay below 2^31");
+
+  SpmmParams p;
+  std::memset(&p, 0, sizeof p);
+  p.vals = q.values;
+  p.meta = q.meta;
+  p.idx = q.idx;
+  p.Y = q.Y;
+  p.ldy = q.ldy;
+  p.R = q.R;
+  p.K = q.K;
+  p.T = q.T;
+  p.n = q.n;
+  p.m = q.m;
+  p.vcols = value_cols(q.K, q.n, q.m);
+  p.mcols = meta_cols(q.K, q.n, q.m);
+  p.pattern = pattern_id(q.n, q.m);
+  p.permuted = q.idx != nullptr;
+  p.out_f32 = q.y_dtype == NM_OUT_F32;
+
+  const bool tma_values_ok = q.n == 2 && q.m == 4 && q.K % 16 == 0 && al16(q.values);
+  if (q.hybrid) {
+    if (q.tile != 128) return fail(NM_ERR_UNSUPPORTED, "hybrid tile must be 128");
+    if (!q.W || !q.tile_map) return fail(NM_ERR_INVALID_ARG, "null hybrid operand");
+    if (q.ldw < q.K) return fail(NM_ERR_INVALID_ARG, "ldw < K");
+    if (!tma_values_ok) return fail(NM_ERR_UNSUPPORTED, "hybrid needs K %% 16 == 0 and 16-byte aligned values");
+    if (!al16(q.W) || q.ldw % 8 != 0) return fail(NM_ERR_MISALIGNED, "W rows must be 16-byte aligned");
+    p.a_mode = A_HYBRID;
+    p.tile_map = q.tile_map;
+    p.hyb_tiles_k = (int)((q.K + 127) / 128);
+  } else if (q.algo == NM_ALGO_DENSE_TC) {
+    p.a_mode = A_BUILD_DENSE;
+  } else if (tma_values_ok) {
+    p.a_mode = A_TMA_SPARSE;
+  } else if (fits_2of4(q.n, q.m)) {
+    p.a_mode = A_BUILD_SPARSE;
+  } else if (q.algo == NM_ALGO_AUTO) {
+    p.a_mode = A_BUILD_DENSE;
+  } else {
+    return fail(NM_ERR_UNSUPPORTED, "pattern %d:%d does not fit the 2:4 sparse MMA", q.n, q.m);
+  }
+
+  const int bn = pick_bn(q.T);
+  const int bsw = bn >= 64 ? 128 : bn * 2;
+  p.a_slot_bytes = (p.a_mode == A_BUILD_DENSE || p.a_mode == A_HYBRID) ? 16384u : 8192u;
+  p.stages = spmm_max_stages(bn, p.a_slot_bytes);
+  p.tiles_m = (int)((q.R + 127) / 128);
+  p.tiles_n = (int)((q.T + bn - 1) / bn);
+  if ((int64_t)p.tiles_m * p.tiles_n >= (1ll << 31)) return fail(NM_ERR_UNSUPPORTED, "too many tiles");
+  p.num_tiles = p.tiles_m * p.tiles_n;
+  p.k_tiles = (q.K + 63) / 64;
+
+  st = make_tmap(&p.tm_x, q.X, (uint64_t)q.T, (uint64_t)q.K, (uint64_t)q.ldx * 2, bsw / 2, p.permuted ? 1 : 64,
+                 bsw, "X");
+  if (st != NM_OK) return st;
+  if (p.a_mode == A_TMA_SPARSE || p.a_mode == A_HYBRID) {
+    st = make_tmap(&p.tm_vals, q.values, (uint64_t)p.vcols, (uint64_t)q.R, (uint64_t)p.vcols * 2, 32, 128, 64,
+                   "values");
+    if (st != NM_OK) return st;
+  }
+  if (p.a_mode == A_HYBRID) {
+    st = make_tmap(&p.tm_w, q.W, (uint64_t)q.K, (uint64_t)q.R, (uint64_t)q.ldw * 2, 64, 128, 128, "W");
+    if (st != NM_OK) return st;
+  }
+  cudaError_t e = launch_spmm(p, bn, stream);
+  return e == cudaSuccess ? NM_OK : cuda_fail(e, "spmm launch");
+}
+
+}  // namespace nmk
+
+using namespace nmk;
+
+extern "C" {
+
+int nm_index_bits(int m) { return index_bits(m); }
+
+int64_t nm_value_cols(int64_t K, int n, int m) {
+  if (!pattern_ok(n, m) || K < 0 || K % m != 0) return -1;
+  return value_cols(K, n, m);
+}
+
+int64_t nm_meta_cols(int64_t K, int n, int m) {
+  if (!pattern_ok(n, m) || K < 0 || K % m != 0) return -1;
+  return meta_cols(K, n, m);
+}
+
+nm_status nm_prune_compress(const uint16_t* W, int64_t R, int64_t K, int64_t ldw, int n, int m, uint16_t* values,
+                            uint32_t* meta, void* stream) {
+  t_last_error.clear();
+  if (R < 0 || K < 0) return fail(NM_ERR_INVALID_ARG, "negative dimension");
+  if (!pattern_ok(n, m)) return fail(NM_ERR_INVALID_ARG, "pattern %d:%d not supported", n, m);
+  if (K % m != 0) return fail(NM_ERR_INVALID_ARG, "K=%lld is not a multiple of M=%d", (long long)K, m);
+  if (ldw < K) return fail(NM_ERR_INVALID_ARG, "ldw < K");
+  if (R == 0 || K == 0) return NM_OK;
+  if (!W || !values || !meta) return fail(NM_ERR_INVALID_ARG, "null pointer");
+  nm_status st = require_device();
+  if (st != NM_OK) return st;
+  cudaError_t e = launch_compress(W, R, K, ldw, n, m, values, meta, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? NM_OK : cuda_fail(e, "compress launch");
+}
+
+nm_status nm_decompress(const uint16_t* values, const uint32_t* meta, int64_t R, int64_t K, int n, int m,
+                        uint16_t* W_out, int64_t ldw, void* stream) {
+  t_last_error.clear();
+  if (R < 0 || K < 0) return fail(NM_ERR_INVALID_ARG, "negative dimension");
+  if (!pattern_ok(n, m)) return fail(NM_ERR_INVALID_ARG, "pattern %d:%d not supported", n, m);
+  if (K % m != 0) return fail(NM_ERR_INVALID_ARG, "K=%lld is not a multiple of M=%d", (long long)K, m);
+  if (ldw < K) return fail(NM_ERR_INVALID_ARG, "ldw < K");
+  if (R == 0 || K == 0) return NM_OK;
+  if (!W_out || !values || !meta) return fail(NM_ERR_INVALID_ARG, "null pointer");
+  nm_status st = require_device();
+  if (st != NM_OK) return st;
+  cudaError_t e = launch_decompress(values, meta, R, K, n, m, W_out, ldw, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? NM_OK : cuda_fail(e, "decompress launch");
+}
+
+nm_status nm_spmm_algo(const uint16_t* values, const uint32_t* meta, int n, int m, int64_t R, int64_t K,
+                       const int32_t* idx, const uint16_t* X, int64_t ldx, int64_t T, void* Y, int64_t ldy,
+                       nm_out_dtype y_dtype, nm_algo algo, void* stream) {
+  GemmRequest q{};
+  q.values = values;
+  q.meta = meta;
+  q.n = n;
+  q.m = m;
+  q.R = R;
+  q.K = K;
+  q.T = T;
+  q.idx = idx;
+  q.X = X;
+  q.ldx = ldx;
+  q.Y = Y;
+  q.ldy = ldy;
+  q.y_dtype = (int)y_dtype;
+  q.algo = algo;
+  q.hybrid = false;
+  return run_gemm(q, static_cast<cudaStream_t>(stream));
+}
+
+nm_status nm_spmm(const uint16_t* values, const uint32_t* meta, int n, int m, int64_t R, int64_t K,
+                  const uint16_t* X, int64_t ldx, int64_t T, void* Y, int64_t ldy, nm_out_dtype y_dtype,
+                  void* stream) {
+  return nm_spmm_algo(values, meta, n, m, R, K, nullptr, X, ldx, T, Y, ldy, y_dtype, NM_ALGO_AUTO, stream);
+}
+
+nm_status nm_spmm_permuted(const uint16_t* values, const uint32_t* meta, int n, int m, int64_t R, int64_t K,
+                           const int32_t* idx, const uint16_t* X, int64_t ldx, int64_t T, void* Y, int64_t ldy,
+                           nm_out_dtype y_dtype, void* stream) {
+  if (!idx && R > 0 && K > 0 && T > 0) return fail(NM_ERR_INVALID_ARG, "idx is null");
+  return nm_spmm_algo(values, meta, n, m, R, K, idx, X, ldx, T, Y, ldy, y_dtype, NM_ALGO_AUTO, stream);
+}
+
+nm_status nm_hybrid_spmm(const uint16_t* W, int64_t ldw, const uint16_t* values, const uint32_t* meta,
+                         const uint8_t* tile_map, int tile, int64_t R, int64_t K, const uint16_t* X, int64_t ldx,
+                         int64_t T, void* Y, int64_t ldy, nm_out_dtype y_dtype, void* stream) {
+  GemmRequest q{};
+  q.values = values;
+  q.meta = meta;
+  q.n = 2;
+  q.m = 4;
+  q.R = R;
+  q.K = K;
+  q.T = T;
+  q.idx = nullptr;
+  q.X = X;
+  q.ldx = ldx;
+  q.Y = Y;
+  q.ldy = ldy;
+  q.y_dtype = (int)y_dtype;
+  q.algo = NM_ALGO_AUTO;
+  q.hybrid = true;
+  q.W = W;
+  q.ldw = ldw;
+  q.tile_map = tile_map;
+  q.tile = tile;
+  return run_gemm(q, static_cast<cudaStream_t>(stream));
+}
+
+nm_status nm_device_status(void* stream) {
+  cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "stream synchronize");
+  uint32_t word = 0;
+  e = read_and_clear_status(&word);
+  if (e != cudaSuccess) return cuda_fail(e, "status read");
+  if (word & 1u) return fail(NM_ERR_TIMEOUT, "a kernel's bounded wait gave up");
+  return NM_OK;
+}
+
+const char* nm_status_string(nm_status s) {
+  switch (s) {
+    case NM_OK: return "ok";
+    case NM_ERR_INVALID_ARG: return "invalid argument";
+    case NM_ERR_UNSUPPORTED: return "unsupported";
+    case NM_ERR_MISALIGNED: return "misaligned pointer or leading dimension";
+    case NM_ERR_CUDA: return "CUDA error";
+    case NM_ERR_TIMEOUT: return "bounded wait gave up";
+    case NM_ERR_NO_DEVICE: return "no sm_100 device";
+  }
+  return "unknown status";
+}
+
+const char* nm_last_error(void) { return t_last_error.c_str(); }
+
+uint64_t nm_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+int nm_version(void) { return 100; }
+
+}  // extern "C"

@@ -1,0 +1,32 @@
+// nm_internal.h -- declarations shared by the host entry points and the
+// kernel launchers of libnm_b200 (not part of the public ABI).
+#pragma once
+#include <cstdint>
+#include <cuda_runtime.h>
+
+namespace nmk {
+
+// Bits per stored position and positions per 32-bit word for a group of m.
+inline int index_bits(int m) { return m == 2 ? 1 : m == 4 ? 2 : m == 8 ? 3 : m == 16 ? 4 : 0; }
+inline int positions_per_word(int m) { return 32 / index_bits(m); }
+inline bool pattern_ok(int n, int m) { return index_bits(m) > 0 && n >= 1 && n < m; }
+inline int64_t value_cols(int64_t K, int n, int m) { return K / m * n; }
+inline int64_t meta_cols(int64_t K, int n, int m) {
+  const int64_t s = positions_per_word(m);
+  return (value_cols(K, n, m) + s - 1) / s;
+}
+
+// Patterns whose survivors never exceed two per aligned group of four, so a
+// tile of them can be re-encoded as 2:4 for the sparse MMA.
+inline bool fits_2of4(int n, int m) { return (m == 2 && n == 1) || ((m == 4 || m == 8) && n <= 2); }
+
+int sm_count_current();
+void count_launch();
+
+cudaError_t launch_compress(const uint16_t* W, int64_t R, int64_t K, int64_t ldw, int n, int m, uint16_t* values,
+                            uint32_t* meta, cudaStream_t s);
+cudaError_t launch_decompress(const uint16_t* values, const uint32_t* meta, int64_t R, int64_t K, int n, int m,
+                              uint16_t* W_out, int64_t ldw, cudaStream_t s);
+cudaError_t launch_fill_zero(void* Y, int64_t R, int64_t T, int64_t ldy, int esize, cudaStream_t s);
+
+}  // namespace nmk

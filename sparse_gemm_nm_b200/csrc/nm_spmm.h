@@ -1,0 +1,47 @@
+// nm_spmm.h -- parameter block of the tcgen05 GEMM kernel (internal).
+#pragma once
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+namespace nmk {
+
+enum AMode : int {
+  A_TMA_SPARSE = 0,    // 2:4 values by TMA, metadata re-laid by the builders
+  A_BUILD_SPARSE = 1,  // builders re-encode an N:M row segment as 2:4 (values + metadata)
+  A_BUILD_DENSE = 2,   // builders expand an N:M row segment into a dense tile
+  A_HYBRID = 3         // per 128x128 tile: dense W by TMA, or 2:4 values by TMA
+};
+
+enum Pattern : int { PAT_2_4 = 0, PAT_1_2 = 1, PAT_1_4 = 2, PAT_1_8 = 3, PAT_2_8 = 4, PAT_OTHER = 5 };
+
+struct SpmmParams {
+  CUtensorMap tm_vals;  // compressed values R x K*n/m, box {32, 128}, 64B swizzle
+  CUtensorMap tm_w;     // dense W R x K, box {64, 128}, 128B swizzle (hybrid)
+  CUtensorMap tm_x;     // X K x T, box {strip, 64} or {strip, 1} (gather4)
+  const uint16_t* vals;
+  const uint32_t* meta;
+  const int32_t* idx;
+  const uint8_t* tile_map;
+  void* Y;
+  uint32_t* status;
+  int64_t ldy;
+  int64_t R, K, T;
+  int64_t vcols, mcols;
+  int64_t k_tiles;
+  int n, m;
+  int pattern;
+  int a_mode;
+  int permuted;
+  int out_f32;
+  int tiles_m, tiles_n, num_tiles;
+  int hyb_tiles_k;
+  int stages;
+  uint32_t a_slot_bytes;
+};
+
+int spmm_max_stages(int bn, uint32_t a_slot);
+cudaError_t launch_spmm(SpmmParams& p, int bn, cudaStream_t stream);
+cudaError_t read_and_clear_status(uint32_t* out);
+
+}  // namespace nmk

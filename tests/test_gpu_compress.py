@@ -1,0 +1,113 @@
+"""GPU prune + compress and decompress against the oracle, bit for bit."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import sparse_gemm_nm_b200 as nm
+import workloads as wl
+from gpu_helpers import DEV, bits, to_dev, words
+
+pytestmark = pytest.mark.gpu
+
+PATTERNS = [(2, 4), (1, 4), (1, 8), (3, 4), (1, 2), (2, 8), (5, 8), (3, 16)]
+
+
+def gpu_compress(W_bits, n, m, ldw=None):
+    R, K = W_bits.shape
+    if ldw is not None and ldw != K:  # strided rows
+        buf = np.zeros((R, ldw), np.uint16)
+        buf[:, :K] = W_bits
+        Wd = to_dev(buf)
+        vals = torch.empty((R, nm.nm_value_cols(K, n, m)), dtype=torch.bfloat16, device=DEV)
+        meta = torch.empty((R, nm.nm_meta_cols(K, n, m)), dtype=torch.int32, device=DEV)
+        nm.nm_prune_compress(Wd, R, K, ldw, n, m, vals, meta)
+    else:
+        vals, meta = nm.prune_compress(to_dev(W_bits), n, m)
+    torch.cuda.synchronize()
+    return bits(vals), words(meta)
+
+
+@pytest.mark.parametrize("n,m", PATTERNS)
+@pytest.mark.parametrize("R,K", [(64, 128), (37, 96), (5, 48), (130, 1040), (3, 16)])
+def test_compress_matches_oracle(n, m, R, K):
+    if K % m:
+        pytest.skip("K must be a multiple of M")
+    W = wl.normal_bf16((R, K), 1.0, seed=R * 7 + K + n + m)
+    v, mt = gpu_compress(W, n, m)
+    ov, om = oracle.compress(W, n, m)
+    assert np.array_equal(v, ov)
+    assert np.array_equal(mt, om)
+
+
+@pytest.mark.parametrize("n,m", [(2, 4), (1, 8), (3, 4)])
+def test_compress_strided_rows(n, m):
+    W = wl.normal_bf16((33, 256), 1.0, seed=5)
+    v, mt = gpu_compress(W, n, m, ldw=264)
+    ov, om = oracle.compress(W, n, m)
+    assert np.array_equal(v, ov) and np.array_equal(mt, om)
+
+
+@pytest.mark.parametrize("n,m", [(2, 4), (1, 4), (1, 8)])
+def test_compress_ties_and_signed_zeros(n, m):
+    """Small-integer weights (many ties), negative zeros and whole zero groups."""
+    W = wl.integer_bf16((50, 64 * m), -2, 2, seed=17)
+    W[3, :] = wl.bf16_bits(np.full(64 * m, -0.0, np.float32))
+    W[4, :] = 0
+    v, mt = gpu_compress(W, n, m)
+    ov, om = oracle.compress(W, n, m)
+    assert np.array_equal(v, ov) and np.array_equal(mt, om)
+
+
+def test_compress_nonfinite():
+    nan, inf = float("nan"), float("inf")
+    rows = np.array([[nan, inf, 1.0, -inf] * 8, [1.0, nan, nan, 5.0] * 8, [-inf, 3.0, inf, 2.0] * 8,
+                     [0.0, -0.0, 0.0, -0.0] * 8], np.float32)
+    W = wl.bf16_bits(rows)
+    W[1, 1] = 0x7FC1  # a second NaN payload ties with the first
+    v, mt = gpu_compress(W, 2, 4)
+    ov, om = oracle.compress(W, 2, 4)
+    assert np.array_equal(v, ov) and np.array_equal(mt, om)
+
+
+def test_worked_row_on_gpu():
+    W = wl.bf16_bits(np.array([[1.5, 0, 0, -2.0, 0, 0.25, 3.0, 0] * 4], np.float32))
+    _, mt = gpu_compress(W, 2, 4)
+    assert int(mt[0, 0]) == 0x9C9C9C9C
+
+
+@pytest.mark.parametrize("n,m", PATTERNS)
+def test_decompress_roundtrip(n, m):
+    R, K = 45, 64 * m
+    W = wl.normal_bf16((R, K), 1.0, seed=99 + m)
+    vals, meta = nm.prune_compress(to_dev(W), n, m)
+    D = nm.decompress(vals, meta, K, n, m)
+    torch.cuda.synchronize()
+    ov, om = oracle.compress(W, n, m)
+    assert np.array_equal(bits(D), oracle.decompress(ov, om, K, n, m))
+    assert np.array_equal(bits(D), np.where(oracle.prune_mask(W, n, m) == 1, W, np.uint16(0)))
+
+
+@pytest.mark.parametrize("R,K", [(4096, 4096), (11008, 4096), (4096, 11008), (13824, 5120)])
+def test_compress_full_size_2of4(R, K):
+    """Full LLaMA-7B and decode weight shapes, whole arrays compared."""
+    W = wl.normal_bf16((R, K), 0.02, seed=0)
+    v, mt = gpu_compress(W, 2, 4)
+    ov, om = oracle.compress(W, 2, 4)
+    assert np.array_equal(v, ov) and np.array_equal(mt, om)
+
+
+@pytest.mark.parametrize("R,K", [(3072, 768), (768, 3072)])
+def test_compress_full_size_1of8(R, K):
+    W = wl.normal_bf16((R, K), 0.02, seed=0)
+    v, mt = gpu_compress(W, 1, 8)
+    ov, om = oracle.compress(W, 1, 8)
+    assert np.array_equal(v, ov) and np.array_equal(mt, om)
+
+
+def test_empty_shapes():
+    W = torch.empty((0, 64), dtype=torch.bfloat16, device=DEV)
+    v, mt = nm.prune_compress(W, 2, 4)
+    assert v.shape == (0, 32) and mt.shape == (0, 2)
+    with pytest.raises(nm.NmError):
+        nm.prune_compress(torch.zeros((4, 10), dtype=torch.bfloat16, device=DEV), 2, 4)

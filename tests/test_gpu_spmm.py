@@ -1,0 +1,277 @@
+"""GPU sparse GEMMs (plain, permuted, hybrid, 1:4 / 1:8) against the oracle.
+
+Sizes the oracle finishes in seconds span several 128-row tiles, several
+column tiles and ragged tails in R, K and T; the full workload sizes are
+checked on sampled outputs computed one by one by the oracle.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import sparse_gemm_nm_b200 as nm
+import workloads as wl
+from gpu_helpers import (DEV, assert_gemm_close, bf16_rne_of, bits, to_dev, to_dev_i32, to_dev_u8,
+                         values_f64)
+
+pytestmark = pytest.mark.gpu
+
+
+def run_spmm(W, X, n, m, idx=None, out_dtype=torch.bfloat16, algo=nm.NM_ALGO_AUTO):
+    K = W.shape[1]
+    vals, meta = nm.prune_compress(to_dev(W), n, m)
+    Y = nm.spmm(vals, meta, n, m, K, to_dev(X), idx=None if idx is None else to_dev_i32(idx),
+                out_dtype=out_dtype, algo=algo)
+    torch.cuda.synchronize()
+    nm.nm_device_status()
+    return Y
+
+
+def reference(W, X, n, m, idx=None):
+    ov, om = oracle.compress(W, n, m)
+    Wd = oracle.decompress(ov, om, W.shape[1], n, m)
+    return oracle.dense_gemm(Wd, X, idx, with_abs=True)
+
+
+def check(W, X, n, m, idx=None, algo=nm.NM_ALGO_AUTO, out_dtype=torch.bfloat16, what=""):
+    Y = run_spmm(W, X, n, m, idx, out_dtype, algo)
+    ref, mag = reference(W, X, n, m, idx)
+    assert_gemm_close(values_f64(Y), ref, mag, what)
+    return Y
+
+
+# ----------------------------------------------------------------------------
+def test_tiny_2of4():
+    L = wl.workload("tiny")[0]
+    d = wl.make_layer(L)
+    Y = check(d.W, d.X, 2, 4, what="tiny")
+    Yi = run_spmm(d.W, d.X, 2, 4, idx=np.arange(L.K, dtype=np.int32))
+    assert torch.equal(Y, Yi)  # identity permutation reduces to the plain kernel
+
+
+@pytest.mark.parametrize("name", ["rl_mlp_2of4", "rl_mlp_1of4", "rl_mlp_1of8"])
+@pytest.mark.parametrize("algo", [nm.NM_ALGO_AUTO, nm.NM_ALGO_DENSE_TC])
+def test_rl_mlp(name, algo):
+    for L in wl.workload(name):
+        d = wl.make_layer(L)
+        check(d.W, d.X, L.n, L.m, algo=algo, what=L.name)
+
+
+@pytest.mark.parametrize("n,m", [(2, 4), (1, 4), (1, 8), (1, 2), (2, 8), (3, 4), (3, 8)])
+@pytest.mark.parametrize("R,K,T", [(300, 1040, 264), (129, 512, 40), (7, 64, 8)])
+def test_ragged_multi_tile(n, m, R, K, T):
+    if K % m:
+        pytest.skip("K must be a multiple of M")
+    W = wl.normal_bf16((R, K), 0.02, seed=R + K)
+    X = wl.normal_bf16((K, T), 1.0, seed=T)
+    check(W, X, n, m, what=f"{n}:{m} {R}x{K}x{T}")
+
+
+@pytest.mark.parametrize("n,m", [(1, 4), (1, 8), (2, 4)])
+def test_sparse_and_dense_designs_agree(n, m):
+    R, K, T = 256, 1024, 128
+    W = wl.normal_bf16((R, K), 0.02, seed=3)
+    X = wl.normal_bf16((K, T), 1.0, seed=4)
+    a = check(W, X, n, m, algo=nm.NM_ALGO_SPARSE_TC, what="sparse")
+    b = check(W, X, n, m, algo=nm.NM_ALGO_DENSE_TC, what="dense")
+    assert values_f64(a).shape == values_f64(b).shape
+
+
+@pytest.mark.parametrize("n,m", [(2, 4), (1, 8)])
+@pytest.mark.parametrize("algo", [nm.NM_ALGO_AUTO, nm.NM_ALGO_DENSE_TC])
+def test_integer_inputs_exact(n, m, algo):
+    """Integer weights and inputs: the fp32 accumulation is exact, so the results match bit for bit."""
+    R, K, T = 200, 512, 96
+    W = wl.integer_bf16((R, K), -8, 8, seed=11)
+    X = wl.integer_bf16((K, T), -8, 8, seed=12)
+    ref, _ = reference(W, X, n, m)
+    Y32 = run_spmm(W, X, n, m, out_dtype=torch.float32, algo=algo)
+    assert np.array_equal(Y32.cpu().numpy().astype(np.float64), ref)
+    Y16 = run_spmm(W, X, n, m, algo=algo)
+    assert np.array_equal(bits(Y16), bf16_rne_of(ref))
+
+
+def test_fp32_output():
+    W = wl.normal_bf16((160, 384), 0.02, seed=21)
+    X = wl.normal_bf16((384, 200), 1.0, seed=22)
+    check(W, X, 2, 4, out_dtype=torch.float32, what="fp32 out")
+
+
+def test_unaligned_k_2of4_uses_built_tiles():
+    """K = 24 (a 17-wide layer padded to a multiple of 8): values rows are not 16-byte aligned."""
+    W = wl.normal_bf16((256, 24), 0.2, seed=31)
+    X = wl.normal_bf16((24, 256), 1.0, seed=32)
+    check(W, X, 2, 4, what="K=24")
+
+
+def test_ragged_columns_with_padded_ld():
+    R, K, T, ldx = 140, 256, 20, 24
+    W = wl.normal_bf16((R, K), 0.02, seed=41)
+    X = wl.normal_bf16((K, T), 1.0, seed=42)
+    Xp = np.zeros((K, ldx), np.uint16)
+    Xp[:, :T] = X
+    vals, meta = nm.prune_compress(to_dev(W), 2, 4)
+    Y = torch.full((R, 24), 7.0, dtype=torch.bfloat16, device=DEV)
+    nm.nm_spmm(vals, meta, 2, 4, R, K, to_dev(Xp), ldx, T, Y, 24)
+    torch.cuda.synchronize()
+    ref, mag = reference(W, X, 2, 4)
+    assert_gemm_close(values_f64(Y[:, :T]), ref, mag, "ragged T")
+    assert torch.all(Y[:, T:] == 7.0)  # columns past T untouched
+
+
+def test_k_zero_gives_zeros():
+    Y = torch.full((8, 16), 3.0, dtype=torch.bfloat16, device=DEV)
+    vals = torch.empty((8, 0), dtype=torch.bfloat16, device=DEV)
+    meta = torch.empty((8, 0), dtype=torch.int32, device=DEV)
+    X = torch.empty((0, 16), dtype=torch.bfloat16, device=DEV)
+    nm.nm_spmm(vals, meta, 2, 4, 8, 0, X, 16, 16, Y, 16)
+    torch.cuda.synchronize()
+    assert torch.all(Y == 0)
+
+
+def test_misaligned_arguments_are_refused():
+    vals, meta = nm.prune_compress(torch.zeros((8, 64), dtype=torch.bfloat16, device=DEV), 2, 4)
+    X = torch.zeros((64, 24), dtype=torch.bfloat16, device=DEV)
+    Y = torch.zeros((8, 24), dtype=torch.bfloat16, device=DEV)
+    with pytest.raises(nm.NmError) as e:
+        nm.nm_spmm(vals, meta, 2, 4, 8, 64, X, 20, 20, Y, 24)   # ldx % 8 != 0
+    assert e.value.status == nm.NM_ERR_MISALIGNED
+
+
+# ----------------------------------------------------------------------------
+# Permuted input read
+# ----------------------------------------------------------------------------
+@pytest.mark.parametrize("n,m", [(2, 4), (1, 8)])
+def test_permuted_matches_oracle(n, m):
+    R, K, T = 270, 1024, 300
+    W = wl.normal_bf16((R, K), 0.02, seed=51)
+    X = wl.normal_bf16((K, T), 1.0, seed=52)
+    idx = wl.permutation(K, 53)
+    check(W, X, n, m, idx=idx, what="permuted")
+
+
+def test_permuted_identity_equals_plain_and_host_permuted():
+    R, K, T = 256, 768, 256
+    W = wl.normal_bf16((R, K), 0.02, seed=61)
+    X = wl.normal_bf16((K, T), 1.0, seed=62)
+    plain = run_spmm(W, X, 2, 4)
+    ident = run_spmm(W, X, 2, 4, idx=np.arange(K, dtype=np.int32))
+    assert torch.equal(plain, ident)
+    idx = wl.permutation(K, 63)
+    perm = run_spmm(W, X, 2, 4, idx=idx)
+    host = run_spmm(W, np.ascontiguousarray(X[idx]), 2, 4)
+    assert torch.equal(perm, host)  # same tiles, same MMA order: bitwise equal
+
+
+def test_permuted_ragged_k():
+    R, K, T = 130, 1040, 64
+    W = wl.normal_bf16((R, K), 0.02, seed=71)
+    X = wl.normal_bf16((K, T), 1.0, seed=72)
+    check(W, X, 2, 4, idx=wl.permutation(K, 73), what="permuted ragged K")
+
+
+# ----------------------------------------------------------------------------
+# PATCH hybrid
+# ----------------------------------------------------------------------------
+def run_hybrid(W, X, tmap):
+    Wd = to_dev(W)
+    vals, meta = nm.prune_compress(Wd, 2, 4)
+    Y = nm.hybrid_spmm(Wd, vals, meta, to_dev_u8(tmap), to_dev(X))
+    torch.cuda.synchronize()
+    nm.nm_device_status()
+    return Y
+
+
+@pytest.mark.parametrize("p", [0.0, 0.25, 0.5, 1.0])
+def test_hybrid_matches_oracle(p):
+    R, K, T = 384, 640, 256
+    W = wl.normal_bf16((R, K), 0.02, seed=81)
+    X = wl.normal_bf16((K, T), 1.0, seed=82)
+    tm = wl.tile_map(3, 5, p, seed=83)
+    Y = run_hybrid(W, X, tm)
+    ref, mag = oracle.hybrid_spmm(W, tm, X, 128, with_abs=True)
+    assert_gemm_close(values_f64(Y), ref, mag, f"hybrid p={p}")
+
+
+def test_hybrid_all_sparse_equals_spmm():
+    R, K, T = 256, 512, 256
+    W = wl.normal_bf16((R, K), 0.02, seed=91)
+    X = wl.normal_bf16((K, T), 1.0, seed=92)
+    Y = run_hybrid(W, X, np.ones((2, 4), np.uint8))
+    assert torch.equal(Y, run_spmm(W, X, 2, 4))
+
+
+def test_hybrid_integer_exact():
+    R, K, T = 256, 512, 128
+    W = wl.integer_bf16((R, K), -8, 8, seed=93)
+    X = wl.integer_bf16((K, T), -8, 8, seed=94)
+    tm = wl.tile_map(2, 4, 0.5, seed=95)
+    Y = run_hybrid(W, X, tm)
+    ref = oracle.hybrid_spmm(W, tm, X, 128)
+    assert np.array_equal(bits(Y), bf16_rne_of(ref))
+
+
+# ----------------------------------------------------------------------------
+# Full workload sizes, sampled outputs
+# ----------------------------------------------------------------------------
+def sampled_check(vals, meta, n, m, W_unused, X, Y, idx=None, count=3000, seed=0):
+    R, T = Y.shape
+    K = X.shape[0]
+    rng = np.random.default_rng(seed)
+    rows = np.concatenate([rng.integers(0, R, count), [0, R - 1, 0, R - 1]])
+    cols = np.concatenate([rng.integers(0, T, count), [0, T - 1, T - 1, 0]])
+    ref, mag = oracle.spmm_sampled(bits(vals), meta.cpu().numpy().view(np.uint32), n, m, K, X, rows, cols, idx)
+    got = values_f64(Y)[rows, cols]
+    assert_gemm_close(got, ref, mag, "sampled")
+
+
+@pytest.mark.parametrize("li", [0, 1, 2])
+def test_llama_full_size_sampled(li):
+    L = wl.workload("llama7b")[li]
+    d = wl.make_layer(L)
+    Wd, Xd, idxd = to_dev(d.W), to_dev(d.X), to_dev_i32(d.idx)
+    vals, meta = nm.prune_compress(Wd, 2, 4)
+    Y = nm.spmm(vals, meta, 2, 4, L.K, Xd, idx=idxd)
+    torch.cuda.synchronize()
+    nm.nm_device_status()
+    sampled_check(vals, meta, 2, 4, d.W, d.X, Y, idx=d.idx)
+    # identity map at full size reduces to the plain kernel, bit for bit
+    Yp = nm.spmm(vals, meta, 2, 4, L.K, Xd[idxd.long()].contiguous())
+    assert torch.equal(Y, Yp)
+
+
+def test_decode_full_size_sampled():
+    L = wl.workload("decode")[0]
+    d = wl.make_layer(L)
+    vals, meta = nm.prune_compress(to_dev(d.W), 2, 4)
+    Y = nm.spmm(vals, meta, 2, 4, L.K, to_dev(d.X))
+    torch.cuda.synchronize()
+    sampled_check(vals, meta, 2, 4, d.W, d.X, Y, count=20000)
+
+
+@pytest.mark.parametrize("li", [0, 1])
+def test_vit_full_size_sampled(li):
+    L = wl.workload("vit")[li]
+    d = wl.make_layer(L)
+    vals, meta = nm.prune_compress(to_dev(d.W), 1, 8)
+    Y = nm.spmm(vals, meta, 1, 8, L.K, to_dev(d.X))
+    torch.cuda.synchronize()
+    nm.nm_device_status()
+    sampled_check(vals, meta, 1, 8, d.W, d.X, Y)
+
+
+def test_patch_full_size_sampled():
+    L = wl.workload("patch_p50")[0]
+    d = wl.make_layer(L)
+    Wd = to_dev(d.W)
+    vals, meta = nm.prune_compress(Wd, 2, 4)
+    Y = nm.hybrid_spmm(Wd, vals, meta, to_dev_u8(d.tmap), to_dev(d.X))
+    torch.cuda.synchronize()
+    nm.nm_device_status()
+    rng = np.random.default_rng(1)
+    rows, cols = rng.integers(0, L.R, 64), rng.integers(0, L.T, 64)
+    Weff = oracle.hybrid_weights(d.W, d.tmap, 128)
+    ref, mag = oracle.dense_gemm(np.ascontiguousarray(Weff[rows]), np.ascontiguousarray(d.X[:, cols]),
+                                 with_abs=True)
+    i = np.arange(rows.shape[0])
+    assert_gemm_close(values_f64(Y)[rows, cols], ref[i, i], mag[i, i], "patch sampled")
