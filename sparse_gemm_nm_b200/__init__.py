@@ -184,6 +184,8 @@ def prune_compress(W, n: int, m: int, stream=None):
     import torch
     _require_cuda(W)
     R, K = W.shape
+    if nm_value_cols(K, n, m) < 0:  # let the library name the bad argument
+        _check(lib().nm_prune_compress(None, R, K, K, n, m, None, None, None), "nm_prune_compress")
     vals = torch.empty((R, nm_value_cols(K, n, m)), dtype=torch.bfloat16, device=W.device)
     meta = torch.empty((R, max(nm_meta_cols(K, n, m), 0)), dtype=torch.int32, device=W.device)
     nm_prune_compress(W, R, K, W.stride(0), n, m, vals, meta, stream)

@@ -356,7 +356,9 @@ __global__ void __launch_bounds__(kThreads, 1) spmm_kernel(const __grid_constant
             for (int kk = 0; kk < 2; ++kk) {
               const uint64_t ad = smem_desc(a_addr + kk * 32, 16, 512, SWZ_64B);
               const uint64_t bd = smem_desc(b_addr + kk * 32 * BSW, STRIP_BYTES, 8 * BSW, B_SWZ);
-              tc_mma_sp(d_tmem, ad, bd, e_tmem + kk, IDESC_SP, (kt > 0 || kk > 0) ? 1u : 0u);
+              // The metadata operand address stays column-pair aligned; the
+              // descriptor's sparsity selector picks the column within the pair.
+              tc_mma_sp(d_tmem, ad, bd, e_tmem, IDESC_SP | (uint32_t)kk, (kt > 0 || kk > 0) ? 1u : 0u);
             }
           } else {
 #pragma unroll
