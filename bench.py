@@ -48,6 +48,13 @@ def parse_args(argv=None):
     ap.add_argument("--cpu-seconds", type=float, default=10.0, help="target length of the oracle baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--workload", default=WORKLOAD, choices=wl.ALL_WORKLOADS,
+                    help="llama7b (default, the headline), decode, vit, patch_p25/p50/p75, tiny, rl_mlp_*")
+    ap.add_argument("--layers", default=None, help="comma-separated subset of the workload's layers")
+    ap.add_argument("--algo", choices=["auto", "sparse", "dense"], default="auto",
+                    help="kernel design for 1:4 / 1:8 (nm_spmm_algo)")
+    ap.add_argument("--quick", action="store_true",
+                    help="timed region only: no clock sampling, end-to-end pass, oracle baseline or extras")
     return ap.parse_args(argv)
 
 
@@ -190,6 +197,18 @@ def run_reference(args, rank: int, world: int):
 # ----------------------------------------------------------------------------
 # Our CUDA path
 # ----------------------------------------------------------------------------
+def gemm_bytes(L, d) -> float:
+    """Algorithmic HBM bytes of one GEMM launch: values + metadata + X + Y (+ index map, + dense tiles)."""
+    b = 2.0 * L.R * (L.K // L.m * L.n) + 4.0 * L.R * -(-(L.K // L.m * L.n) // (32 // {2: 1, 4: 2, 8: 3, 16: 4}[L.m]))
+    b += 2.0 * L.K * L.T + 2.0 * L.R * L.T
+    if d.idx is not None:
+        b += 4.0 * L.K
+    if d.tmap is not None:  # dense tiles are read from W instead of the compressed form
+        dense = float((d.tmap == 0).sum()) * L.tile * L.tile
+        b += 2.0 * dense - 1.125 * dense + d.tmap.size
+    return b
+
+
 def run_ours(args, rank: int, world: int, dist):
     import torch
     import sparse_gemm_nm_b200 as nm
@@ -200,8 +219,11 @@ def run_ours(args, rank: int, world: int, dist):
     stream = torch.cuda.current_stream(dev)
     sp = stream.cuda_stream
     L_ = nm.lib()
+    algo = {"auto": nm.NM_ALGO_AUTO, "sparse": nm.NM_ALGO_SPARSE_TC, "dense": nm.NM_ALGO_DENSE_TC}[args.algo]
 
-    layers = wl.workload(WORKLOAD)
+    layers = wl.workload(args.workload)
+    if args.layers:
+        layers = [layers[int(i)] for i in args.layers.split(",")]
     data = [wl.make_layer(L) for L in layers]
 
     def up(bits):
@@ -210,13 +232,16 @@ def run_ours(args, rank: int, world: int, dist):
     bufs = []
     for d in data:
         L = d.layer
-        W = up(d.W)
-        X = up(d.X)
-        idx = torch.from_numpy(d.idx).to(dev)
-        vals = torch.empty((L.R, L.K // 2), dtype=torch.bfloat16, device=dev)
-        meta = torch.empty((L.R, L.K // 32), dtype=torch.int32, device=dev)
-        Y = torch.empty((L.R, L.T), dtype=torch.bfloat16, device=dev)
-        bufs.append((L, W, X, idx, vals, meta, Y))
+        b = {"L": L, "d": d, "W": up(d.W), "X": up(d.X),
+             "idx": torch.from_numpy(d.idx).to(dev) if d.idx is not None else None,
+             "tmap": torch.from_numpy(d.tmap).to(dev) if d.tmap is not None else None,
+             "vals": torch.empty((L.R, max(nm.nm_value_cols(L.K, L.n, L.m), 0)), dtype=torch.bfloat16, device=dev),
+             "meta": torch.empty((L.R, max(nm.nm_meta_cols(L.K, L.n, L.m), 0)), dtype=torch.int32, device=dev),
+             "Y": torch.empty((L.R, L.T), dtype=torch.bfloat16, device=dev)}
+        b["flops"] = float(wl.hybrid_useful_flops(d) if d.tmap is not None else L.useful_flops)
+        b["gemm_bytes"] = gemm_bytes(L, d)
+        b["comp_bytes"] = 2.0 * L.R * L.K + 2.0 * b["vals"].numel() + 4.0 * b["meta"].numel()
+        bufs.append(b)
     torch.cuda.synchronize()
 
     def check(st, what):
@@ -224,14 +249,26 @@ def run_ours(args, rank: int, world: int, dist):
             raise RuntimeError(f"{what}: {L_.nm_last_error().decode()}")
 
     def launch_compress(b):
-        L, W, X, idx, vals, meta, Y = b
-        check(L_.nm_prune_compress(W.data_ptr(), L.R, L.K, L.K, 2, 4, vals.data_ptr(), meta.data_ptr(), sp),
-              "nm_prune_compress")
+        L = b["L"]
+        check(L_.nm_prune_compress(b["W"].data_ptr(), L.R, L.K, L.K, L.n, L.m, b["vals"].data_ptr(),
+                                   b["meta"].data_ptr(), sp), "nm_prune_compress")
 
-    def launch_spmm(b):
-        L, W, X, idx, vals, meta, Y = b
-        check(L_.nm_spmm_permuted(vals.data_ptr(), meta.data_ptr(), 2, 4, L.R, L.K, idx.data_ptr(),
-                                  X.data_ptr(), L.T, L.T, Y.data_ptr(), L.T, 0, sp), "nm_spmm_permuted")
+    def launch_gemm(b, permuted=True):
+        L = b["L"]
+        if b["tmap"] is not None:
+            check(L_.nm_hybrid_spmm(b["W"].data_ptr(), L.K, b["vals"].data_ptr(), b["meta"].data_ptr(),
+                                    b["tmap"].data_ptr(), L.tile, L.R, L.K, b["X"].data_ptr(), L.T, L.T,
+                                    b["Y"].data_ptr(), L.T, 0, sp), "nm_hybrid_spmm")
+        elif b["idx"] is not None and permuted:
+            check(L_.nm_spmm_permuted(b["vals"].data_ptr(), b["meta"].data_ptr(), L.n, L.m, L.R, L.K,
+                                      b["idx"].data_ptr(), b["X"].data_ptr(), L.T, L.T, b["Y"].data_ptr(), L.T, 0,
+                                      sp), "nm_spmm_permuted")
+        elif algo != nm.NM_ALGO_AUTO:
+            check(L_.nm_spmm_algo(b["vals"].data_ptr(), b["meta"].data_ptr(), L.n, L.m, L.R, L.K, None,
+                                  b["X"].data_ptr(), L.T, L.T, b["Y"].data_ptr(), L.T, 0, algo, sp), "nm_spmm_algo")
+        else:
+            check(L_.nm_spmm(b["vals"].data_ptr(), b["meta"].data_ptr(), L.n, L.m, L.R, L.K, b["X"].data_ptr(),
+                             L.T, L.T, b["Y"].data_ptr(), L.T, 0, sp), "nm_spmm")
 
     def step(evs=None):
         for i, b in enumerate(bufs):
@@ -240,7 +277,7 @@ def run_ours(args, rank: int, world: int, dist):
             launch_compress(b)
             if evs is not None:
                 evs[2 * i + 1].record(stream)
-            launch_spmm(b)
+            launch_gemm(b)
         if evs is not None:
             evs[2 * len(bufs)].record(stream)
 
@@ -248,8 +285,14 @@ def run_ours(args, rank: int, world: int, dist):
         if dist is not None:
             dist.barrier()
 
-    useful = sum(2.0 * L.T * L.R * (L.K // 2) for (L, *_rest) in bufs)
-    comp_bytes = [2.0 * L.R * L.K + L.R * L.K + L.R * L.K / 8.0 for (L, *_r) in bufs]
+    def max_over_ranks(ms):
+        if dist is None:
+            return ms
+        t = torch.tensor([ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    useful = sum(b["flops"] for b in bufs)
 
     for _ in range(args.warmup):
         step()
@@ -257,8 +300,10 @@ def run_ours(args, rank: int, world: int, dist):
     nm.nm_device_status(sp)
 
     props = torch.cuda.get_device_properties(dev)
-    sampler = ClockSampler(f"GPU-{props.uuid}" if getattr(props, "uuid", None) else "")
-    sampler.start()
+    sampler = None
+    if not args.quick:
+        sampler = ClockSampler(f"GPU-{props.uuid}" if getattr(props, "uuid", None) else "")
+        sampler.start()
 
     nev = 2 * len(bufs) + 1
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(nev)] for _ in range(args.steps)]
@@ -274,82 +319,117 @@ def run_ours(args, rank: int, world: int, dist):
     torch.cuda.synchronize()
     barrier()
     launches = nm.nm_launch_count() - launches0
-    sampler.stop()
+    if sampler:
+        sampler.stop()
     nm.nm_device_status(sp)
 
-    elapsed_ms = t_start.elapsed_time(t_end)
-    if dist is not None:
-        t = torch.tensor([elapsed_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        elapsed_ms = float(t.item())
+    elapsed_ms = max_over_ranks(t_start.elapsed_time(t_end))
     ms_per_step = elapsed_ms / args.steps
 
     # per-kernel durations over the timed region (same stream as the launches)
     comp_ms = np.zeros(len(bufs))
-    spmm_ms = np.zeros(len(bufs))
+    gemm_ms = np.zeros(len(bufs))
     for k in range(args.steps):
         e = evs[k]
         for i in range(len(bufs)):
             comp_ms[i] += e[2 * i].elapsed_time(e[2 * i + 1])
-            spmm_ms[i] += e[2 * i + 1].elapsed_time(e[2 * i + 2])
+            gemm_ms[i] += e[2 * i + 1].elapsed_time(e[2 * i + 2])
     comp_ms /= args.steps
-    spmm_ms /= args.steps
+    gemm_ms /= args.steps
 
     peaks, peak_src = load_peaks()
-    timed_s = elapsed_ms / 1e3
-    sustained = timed_s > 1.0
+    sustained = elapsed_ms > 1000.0
     tc_peak = peaks["bf16_tflops_sustained" if sustained else "bf16_tflops"]
     hbm_peak = peaks["hbm_gbs"]
-    spmm_flops = [2.0 * L.T * L.R * (L.K // 2) for (L, *_r) in bufs]
-    achieved = sum(spmm_flops) / (spmm_ms.sum() * 1e-3) / 1e12
     kernels = {}
-    for i, (L, *_r) in enumerate(bufs):
+    for i, b in enumerate(bufs):
+        L = b["L"]
+        t_tc = b["flops"] / (tc_peak * 1e12)
+        t_hbm = b["gemm_bytes"] / (hbm_peak * 1e9)
         kernels[L.name] = {
-            "spmm_us": 1e3 * spmm_ms[i], "spmm_tflops": spmm_flops[i] / (spmm_ms[i] * 1e-3) / 1e12,
-            "spmm_frac": spmm_flops[i] / (spmm_ms[i] * 1e-3) / 1e12 / tc_peak,
-            "compress_us": 1e3 * comp_ms[i], "compress_gbs": comp_bytes[i] / (comp_ms[i] * 1e-3) / 1e9,
-            "compress_frac": comp_bytes[i] / (comp_ms[i] * 1e-3) / 1e9 / hbm_peak}
+            "gemm_us": 1e3 * gemm_ms[i],
+            "gemm_tflops": b["flops"] / (gemm_ms[i] * 1e-3) / 1e12,
+            "gemm_gbs": b["gemm_bytes"] / (gemm_ms[i] * 1e-3) / 1e9,
+            "gemm_bound": "tensor" if t_tc >= t_hbm else "hbm",
+            "gemm_frac": max(t_tc, t_hbm) / (gemm_ms[i] * 1e-3),
+            "compress_us": 1e3 * comp_ms[i],
+            "compress_gbs": b["comp_bytes"] / (comp_ms[i] * 1e-3) / 1e9,
+            "compress_frac": b["comp_bytes"] / (comp_ms[i] * 1e-3) / 1e9 / hbm_peak}
+
+    # dominant kernel: the GEMM (all launches of the step together)
+    flops_all = sum(b["flops"] for b in bufs)
+    bytes_all = sum(b["gemm_bytes"] for b in bufs)
+    gsec = gemm_ms.sum() * 1e-3
+    tensor_bound = flops_all / (tc_peak * 1e12) >= bytes_all / (hbm_peak * 1e9)
     traffic = None
-    tfile = os.path.join(ROOT, "profiles", "spmm_traffic.json")
+    tfile = os.path.join(ROOT, "profiles", f"{args.workload}_gemm_traffic.json")
     if os.path.exists(tfile):
         with open(tfile) as f:
             traffic = json.load(f).get("bytes_per_launch")
-    roofline = {"bound": "tensor", "achieved": achieved, "peak": tc_peak, "unit": "TFLOP/s",
-                "frac": achieved / tc_peak, "traffic": traffic,
-                "kernel": "nm_spmm_permuted (tcgen05.mma.sp, 2:4 + index-map gather)",
-                "peak_source": f"{peak_src} bf16 {'sustained' if sustained else 'burst'} dense peak; useful "
-                               "2:4 FLOPs run at half the sparse MMA rate, i.e. at the dense rate",
-                "algorithmic_flops_per_launch": spmm_flops}
+    if tensor_bound:
+        achieved, peak, unit = flops_all / gsec / 1e12, tc_peak, "TFLOP/s"
+        src = (f"{peak_src} bf16 {'sustained' if sustained else 'burst'} dense peak; useful 2:4 FLOPs run at "
+               "half the sparse-MMA rate, i.e. at the dense rate")
+    else:
+        achieved, peak, unit = bytes_all / gsec / 1e9, hbm_peak, "GB/s"
+        src = f"{peak_src} HBM copy bandwidth"
+    roofline = {"bound": "tensor" if tensor_bound else "hbm", "achieved": achieved, "peak": peak, "unit": unit,
+                "frac": achieved / peak, "traffic": traffic, "kernel": "spmm_kernel (tcgen05 GEMM)",
+                "peak_source": src,
+                "algorithmic_per_launch": [b["flops"] if tensor_bound else b["gemm_bytes"] for b in bufs]}
 
+    cfg = {"workload": args.workload, "shapes": [[b["L"].R, b["L"].K] for b in bufs],
+           "T": [b["L"].T for b in bufs], "pattern": [f"{b['L'].n}:{b['L'].m}" for b in bufs],
+           "permuted": any(b["idx"] is not None for b in bufs), "algo": args.algo,
+           "step": "prune+compress, then the sparse GEMM, for every layer",
+           "l2": "inputs larger than L2 (126 MB) per step" if sum(
+               b["W"].numel() * 2 + b["X"].numel() * 2 + b["Y"].numel() * 2 for b in bufs) > 126e6
+           else "working set below L2 size (small config)",
+           "parallelism": f"replicas x{world}"}
     line = {"metric": METRIC, "value": world * useful / (ms_per_step * 1e-3) / 1e12, "unit": "TFLOP/s",
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
-            "data": "synthetic (seeded numpy PCG64, N(0,0.02) weights, N(0,1) inputs, random permutation)",
-            "config": {"workload": f"{WORKLOAD}_2of4_permuted", "shapes": [[L.R, L.K] for (L, *_r) in bufs],
-                       "T": bufs[0][0].T, "pattern": "2:4", "step": "prune+compress then permuted spmm, 3 layers",
-                       "l2": "inputs larger than L2 (about 290 MB touched per step > 126 MB)",
-                       "parallelism": f"replicas x{world}"},
-            "roofline": roofline, "kernels": kernels, "gpu_launches": launches,
-            "clocks": sampler.summary()}
+            "data": "synthetic (seeded numpy PCG64 draws rounded to bf16; shapes and distributions of the workload)",
+            "config": cfg, "roofline": roofline, "kernels": kernels, "gpu_launches": launches,
+            "clocks": sampler.summary() if sampler else None}
+
+    if not args.quick and any(b["idx"] is not None for b in bufs):
+        # cost of the index-map read: the same GEMMs without the permutation
+        for b in bufs:
+            launch_gemm(b, permuted=False)
+        torch.cuda.synchronize()
+        plain_ms = []
+        for b in bufs:
+            a, z = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            reps = max(10, min(200, args.steps))
+            a.record(stream)
+            for _ in range(reps):
+                launch_gemm(b, permuted=False)
+            z.record(stream)
+            torch.cuda.synchronize()
+            plain_ms.append(a.elapsed_time(z) / reps)
+        line["permutation_overhead"] = {
+            b["L"].name: {"plain_us": 1e3 * plain_ms[i], "permuted_us": 1e3 * gemm_ms[i],
+                          "overhead": gemm_ms[i] / plain_ms[i] - 1.0} for i, b in enumerate(bufs)}
 
     # end-to-end through the public API with host buffers
-    if not args.no_e2e:
-        hW = [torch.from_numpy(d.W.view(np.int16)).pin_memory() for d in data]
-        hX = [torch.from_numpy(d.X.view(np.int16)).pin_memory() for d in data]
-        hI = [torch.from_numpy(d.idx).pin_memory() for d in data]
-        hY = [torch.empty((b[0].R, b[0].T), dtype=torch.int16).pin_memory() for b in bufs]
-        h2d = sum(a.numel() * a.element_size() for a in hW + hX + hI)
+    if not args.quick and not args.no_e2e:
+        hW = [torch.from_numpy(b["d"].W.view(np.int16)).pin_memory() for b in bufs]
+        hX = [torch.from_numpy(b["d"].X.view(np.int16)).pin_memory() for b in bufs]
+        hI = [torch.from_numpy(b["d"].idx).pin_memory() if b["idx"] is not None else None for b in bufs]
+        hY = [torch.empty((b["L"].R, b["L"].T), dtype=torch.int16).pin_memory() for b in bufs]
+        h2d = sum(a.numel() * a.element_size() for a in hW + hX + [h for h in hI if h is not None])
         d2h = sum(a.numel() * a.element_size() for a in hY)
 
         def e2e_step():
             for i, b in enumerate(bufs):
-                L, W, X, idx, vals, meta, Y = b
-                W.view(torch.int16).copy_(hW[i], non_blocking=True)
-                X.view(torch.int16).copy_(hX[i], non_blocking=True)
-                idx.copy_(hI[i], non_blocking=True)
+                b["W"].view(torch.int16).copy_(hW[i], non_blocking=True)
+                b["X"].view(torch.int16).copy_(hX[i], non_blocking=True)
+                if hI[i] is not None:
+                    b["idx"].copy_(hI[i], non_blocking=True)
                 launch_compress(b)
-                launch_spmm(b)
-                hY[i].copy_(Y.view(torch.int16), non_blocking=True)
+                launch_gemm(b)
+                hY[i].copy_(b["Y"].view(torch.int16), non_blocking=True)
 
         e2e_step()
         torch.cuda.synchronize()
@@ -361,15 +441,11 @@ def run_ours(args, rank: int, world: int, dist):
             e2e_step()
         z.record(stream)
         torch.cuda.synchronize()
-        e_ms = a.elapsed_time(z)
-        if dist is not None:
-            t = torch.tensor([e_ms], dtype=torch.float64, device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            e_ms = float(t.item())
+        e_ms = max_over_ranks(a.elapsed_time(z))
         line["e2e"] = {"value": world * useful * args.e2e_steps / (e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
                        "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                        "ms_per_step": e_ms / args.e2e_steps}
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+    if rank == 0 and world == 1 and not args.quick and not args.no_cpu_baseline and args.workload == "llama7b":
         line["cpu_baseline"] = cpu_baseline(data, args.cpu_seconds)
     elif rank == 0:
         line["cpu_baseline"] = None

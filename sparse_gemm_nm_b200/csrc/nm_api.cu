@@ -175,6 +175,8 @@ static nm_status run_gemm(const GemmRequest& q, cudaStream_t stream) {
   p.vals = q.values;
   p.meta = q.meta;
   p.idx = q.idx;
+  p.X = q.X;
+  p.ldx = q.ldx;
   p.Y = q.Y;
   p.ldy = q.ldy;
   p.R = q.R;
@@ -220,7 +222,7 @@ static nm_status run_gemm(const GemmRequest& q, cudaStream_t stream) {
   p.num_tiles = p.tiles_m * p.tiles_n;
   p.k_tiles = (q.K + 63) / 64;
 
-  st = make_tmap(&p.tm_x, q.X, (uint64_t)q.T, (uint64_t)q.K, (uint64_t)q.ldx * 2, bsw / 2, p.permuted ? 1 : 64,
+  st = make_tmap(&p.tm_x, q.X, (uint64_t)q.T, (uint64_t)q.K, (uint64_t)q.ldx * 2, bsw / 2, 64,
                  bsw, "X");
   if (st != NM_OK) return st;
   if (p.a_mode == A_TMA_SPARSE || p.a_mode == A_HYBRID) {

@@ -42,36 +42,48 @@ __device__ __forceinline__ void select_2of4(uint32_t e0, uint32_t e1, uint32_t e
   packed = v0 | (v1 << 16);
 }
 
-// 2:4 fast path: one thread per metadata word = 32 weights = 8 groups.
-// 64 B of W in (4 x 16 B), 32 B of values + 4 B of metadata out.
-__global__ void __launch_bounds__(256) compress_2of4_kernel(const uint16_t* __restrict__ W, int64_t R,
-                                                            int64_t K, int64_t ldw, uint16_t* __restrict__ V,
+// 2:4 fast path.  A warp walks the matrix in 512-byte pieces (32 lanes x 8
+// weights = 8 metadata words); each lane loads 16 contiguous bytes, selects
+// its two groups, stores 8 bytes of values, and four neighbouring lanes merge
+// their metadata bytes into one word with shuffles.  Loads and stores of a
+// warp instruction are contiguous.  U pieces per lane are kept in flight.
+constexpr int kCompressUnroll = 4;
+
+__global__ void __launch_bounds__(256) compress_2of4_kernel(const uint16_t* __restrict__ W, uint32_t R,
+                                                            uint32_t K, int64_t ldw, uint16_t* __restrict__ V,
                                                             uint32_t* __restrict__ meta) {
-  const int64_t wpr = K >> 5;  // words per row
-  const int64_t total = R * wpr;
-  for (int64_t w = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; w < total;
-       w += (int64_t)gridDim.x * blockDim.x) {
-    const int64_t r = w / wpr;
-    const int64_t c = w - r * wpr;
-    const uint4* src = reinterpret_cast<const uint4*>(W + r * ldw + (c << 5));
-    uint4 in[4];
+  // R * K / 8 < 2^32 is checked by the launcher: 32-bit index arithmetic.
+  const uint32_t lane = threadIdx.x & 31u;
+  const uint32_t cpr = K >> 3;           // 8-weight chunks per row
+  const uint32_t total = R * cpr;        // chunks in the matrix
+  const uint32_t warp_id = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const uint32_t nwarps = (gridDim.x * blockDim.x) >> 5;
+  for (uint32_t base = warp_id * 32u * kCompressUnroll; base < total; base += nwarps * 32u * kCompressUnroll) {
+    uint4 in[kCompressUnroll];
+    uint32_t rr[kCompressUnroll], cc[kCompressUnroll];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) in[i] = __ldg(src + i);
-    uint32_t word = 0, out[8];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      uint32_t nib, pk;
-      select_2of4(in[i].x & 0xFFFFu, in[i].x >> 16, in[i].y & 0xFFFFu, in[i].y >> 16, nib, pk);
-      word |= nib << (8 * i);
-      out[2 * i] = pk;
-      select_2of4(in[i].z & 0xFFFFu, in[i].z >> 16, in[i].w & 0xFFFFu, in[i].w >> 16, nib, pk);
-      word |= nib << (8 * i + 4);
-      out[2 * i + 1] = pk;
+    for (int u = 0; u < kCompressUnroll; ++u) {
+      const uint32_t c = base + u * 32u + lane;
+      rr[u] = c / cpr;
+      cc[u] = c - rr[u] * cpr;
+      in[u] = c < total ? __ldg(reinterpret_cast<const uint4*>(W + (int64_t)rr[u] * ldw + (cc[u] << 3)))
+                        : make_uint4(0, 0, 0, 0);
     }
-    uint4* dst = reinterpret_cast<uint4*>(V + r * (K >> 1) + (c << 4));
-    dst[0] = make_uint4(out[0], out[1], out[2], out[3]);
-    dst[1] = make_uint4(out[4], out[5], out[6], out[7]);
-    meta[w] = word;
+#pragma unroll
+    for (int u = 0; u < kCompressUnroll; ++u) {
+      uint32_t nib0, nib1, pk0, pk1;
+      select_2of4(in[u].x & 0xFFFFu, in[u].x >> 16, in[u].y & 0xFFFFu, in[u].y >> 16, nib0, pk0);
+      select_2of4(in[u].z & 0xFFFFu, in[u].z >> 16, in[u].w & 0xFFFFu, in[u].w >> 16, nib1, pk1);
+      // byte of this lane inside its metadata word: lanes 4q..4q+3 -> bytes 0..3
+      uint32_t word = (nib0 | (nib1 << 4)) << (8 * (lane & 3));
+      word |= __shfl_xor_sync(0xffffffffu, word, 1);
+      word |= __shfl_xor_sync(0xffffffffu, word, 2);
+      if (base + u * 32u + lane < total) {
+        const int64_t r = rr[u];
+        *reinterpret_cast<uint2*>(V + r * (K >> 1) + (cc[u] << 2)) = make_uint2(pk0, pk1);
+        if ((lane & 3) == 0) meta[r * (K >> 5) + (cc[u] >> 2)] = word;
+      }
+    }
   }
 }
 
@@ -211,9 +223,11 @@ static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 
 cudaError_t launch_compress(const uint16_t* W, int64_t R, int64_t K, int64_t ldw, int n, int m, uint16_t* values,
                             uint32_t* meta, cudaStream_t s) {
   const int threads = 256;
-  if (n == 2 && m == 4 && K % 32 == 0 && ldw % 8 == 0 && aligned16(W) && aligned16(values)) {
-    const int64_t work = R * (K / 32);
-    compress_2of4_kernel<<<grid_for(work, threads), threads, 0, s>>>(W, R, K, ldw, values, meta);
+  if (n == 2 && m == 4 && K % 32 == 0 && ldw % 8 == 0 && aligned16(W) && aligned16(values) &&
+      R * (K / 8) < (int64_t(1) << 32) - 4096 * kCompressUnroll) {
+    const int64_t work = R * (K / 8) / kCompressUnroll;
+    compress_2of4_kernel<<<grid_for(work, threads), threads, 0, s>>>(W, (uint32_t)R, (uint32_t)K, ldw, values,
+                                                                     meta);
   } else {
     const int64_t work = R * meta_cols(K, n, m);
     const int grid = grid_for(work, threads);

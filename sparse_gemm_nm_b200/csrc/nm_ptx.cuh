@@ -1,5 +1,5 @@
 // nm_ptx.cuh -- thin inline-PTX wrappers for sm_100a: mbarriers with bounded
-// waits, TMA tile and gather4 loads, tcgen05 (TMEM alloc, MMA, sparse MMA,
+// waits, TMA tile loads, cp.async, tcgen05 (TMEM alloc, MMA, sparse MMA,
 // smem->TMEM copy, TMEM loads) and the shared-memory matrix descriptor.
 #pragma once
 #include <cstdint>
@@ -86,16 +86,19 @@ __device__ __forceinline__ void tma_load_2d(void* smem_dst, const void* tmap, ui
       : "memory");
 }
 
-// Four rows y0..y3 (each one box high) of columns [x, x+box) land as four
-// consecutive box rows in shared memory.
-__device__ __forceinline__ void tma_gather4(void* smem_dst, const void* tmap, uint64_t* bar, int32_t x,
-                                            int32_t y0, int32_t y1, int32_t y2, int32_t y3) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%3, %4, %5, %6, %7}], [%2];" ::"r"(smem_u32(smem_dst)),
-      "l"(reinterpret_cast<uint64_t>(tmap)), "r"(smem_u32(bar)), "r"(x), "r"(y0), "r"(y1), "r"(y2),
-      "r"(y3)
-      : "memory");
+// ---------------------------------------------------------------- cp.async
+// 16-byte global -> shared copy through L2 only; bytes beyond src_bytes (0..16)
+// are written as zeros and not read.
+__device__ __forceinline__ void cp_async_16(void* smem_dst, const void* gsrc, uint32_t src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(smem_dst)), "l"(gsrc),
+               "r"(src_bytes)
+               : "memory");
+}
+
+// Arrive on the mbarrier once all cp.async of this thread issued so far have
+// landed; the arrival counts towards the phase's expected count.
+__device__ __forceinline__ void cp_async_arrive_noinc(uint64_t* bar) {
+  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
 
 // ---------------------------------------------------------------- tcgen05

@@ -10,9 +10,8 @@
 // Sparsity" topic cards, PATCH abstract (tiles either dense or 2:4).
 //
 // One persistent CTA per SM walks output tiles of 128 x BN.  Warp roles:
-//   warp 0      TMA producer: compressed A tile (or dense W tile) and the X
-//               tile; with an index map, X rows are gathered four at a time
-//               (tile::gather4) straight into the swizzled shared tile.
+//   warp 0      TMA producer: compressed A tile (or dense W tile) and, without
+//               an index map, the X tile.
 //   warp 1      TMEM owner and MMA issuer (one thread): per stage it copies
 //               the metadata tile into TMEM (tcgen05.cp) and issues
 //               tcgen05.mma.sp (2:4) or tcgen05.mma (dense) into the fp32
@@ -20,7 +19,9 @@
 //   warps 2-5   builders, one thread per tile row: re-lay the row-wise
 //               metadata into the tensor-core metadata order, or build the A
 //               tile in shared memory from the compressed operand (1:4 / 1:8
-//               re-encoded as 2:4, or any N:M expanded to a dense tile).
+//               re-encoded as 2:4, or any N:M expanded to a dense tile).  With
+//               an index map they also gather the X rows X[idx[k]] with
+//               coalesced 16-byte cp.async straight into the swizzled B tile.
 //   warps 6-9   epilogue: TMEM -> registers -> bf16/fp32 -> global.
 // Stages of the shared-memory ring are handed over with mbarriers; every wait
 // is bounded in time and reports through a device status word.
@@ -257,7 +258,7 @@ __global__ void __launch_bounds__(kThreads, 1) spmm_kernel(const __grid_constant
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < stages; ++s) {
-      mbar_init(&full[s], 1 + 4);
+      mbar_init(&full[s], 1 + 4 + (p.permuted ? 128 : 0));
       mbar_init(&empty[s], 1);
     }
     for (int b = 0; b < 2; ++b) {
@@ -303,28 +304,13 @@ __global__ void __launch_bounds__(kThreads, 1) spmm_kernel(const __grid_constant
         uint8_t* a_dst = a_base + s * p.a_slot_bytes;
         uint8_t* b_dst = b_base + s * B_BYTES;
         if (lane == 0) {
-          mbar_arrive_expect_tx(&full[s], a_bytes + B_BYTES);
+          mbar_arrive_expect_tx(&full[s], a_bytes + (p.permuted ? 0u : B_BYTES));
           if (a_kind == 1) tma_load_2d(a_dst, &p.tm_vals, &full[s], (int32_t)(kt * 32), m0);
           else if (a_kind == 2) tma_load_2d(a_dst, &p.tm_w, &full[s], (int32_t)(kt * 64), m0);
         }
         __syncwarp();
-        const int64_t k0 = kt * 64;
-        if (!p.permuted) {
-          if (lane < N_STRIPS)
-            tma_load_2d(b_dst + lane * STRIP_BYTES, &p.tm_x, &full[s], n0 + lane * STRIP_COLS, (int32_t)k0);
-        } else {
-          for (int i = lane; i < 16 * N_STRIPS; i += 32) {
-            const int strip = i >> 4, g = i & 15;
-            int32_t y[4];
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-              const int64_t k = k0 + 4 * g + j;
-              y[j] = k < p.K ? __ldg(p.idx + k) : (int32_t)p.K;
-            }
-            tma_gather4(b_dst + strip * STRIP_BYTES + 4 * g * BSW, &p.tm_x, &full[s], n0 + strip * STRIP_COLS,
-                        y[0], y[1], y[2], y[3]);
-          }
-        }
+        if (!p.permuted && lane < N_STRIPS)
+          tma_load_2d(b_dst + lane * STRIP_BYTES, &p.tm_x, &full[s], n0 + lane * STRIP_COLS, (int32_t)(kt * 64));
         if (++s == stages) { s = 0; ph ^= 1u; }
       }
     }
@@ -384,40 +370,114 @@ __global__ void __launch_bounds__(kThreads, 1) spmm_kernel(const __grid_constant
   } else if (warp < kEpilogueWarp0) {
     // ------------------------------------------------------------ builders
     const int r = threadIdx.x - 32 * kBuilderWarp0;  // tile row 0..127
+    const int bw = r >> 5;                           // builder warp 0..3
+    const bool e_from_meta = p.a_mode == A_TMA_SPARSE || p.a_mode == A_HYBRID;
+    // The stages of this CTA in order: tile blockIdx.x + j*gridDim.x, kt.
+    const int64_t my_tiles = (p.num_tiles - 1 - blockIdx.x) / gridDim.x + 1;
+    const int64_t total = my_tiles * k_tiles;
+    // Prefetch ring, PF stages ahead: this row's two 2:4 metadata words, and
+    // (permuted) the source row of X for K-row 16*bw + lane of the stage.
+    constexpr int PF = 6;
+    uint2 mq[PF];
+    int32_t iq[PF];
+    // prefetch cursor (stage it + PF) advanced incrementally, no divisions
+    int f_tile = blockIdx.x;
+    int64_t f_kt = 0, f_it = 0;
+    auto fetch = [&](uint2& mw, int32_t& ix) {
+      mw = make_uint2(0x44444444u, 0x44444444u);
+      ix = -1;
+      if (f_it < total) {
+        if (e_from_meta) {
+          const int64_t row = (int64_t)(f_tile % p.tiles_m) * 128 + r;
+          if (row < p.R) {
+            const int64_t c = f_kt * 2;
+            const uint32_t* mrow = p.meta + row * p.mcols;
+            if (c < p.mcols) mw.x = clamp_meta_word(__ldg(mrow + c), c * 32, p.K);
+            if (c + 1 < p.mcols) mw.y = clamp_meta_word(__ldg(mrow + c + 1), (c + 1) * 32, p.K);
+          }
+        }
+        if (p.permuted && lane < 16) {
+          const int64_t k = f_kt * 64 + bw * 16 + lane;
+          if (k < p.K) ix = __ldg(p.idx + k);
+        }
+      }
+      ++f_it;
+      if (++f_kt == k_tiles) { f_kt = 0; f_tile += gridDim.x; }
+    };
+#pragma unroll
+    for (int j = 0; j < PF; ++j) fetch(mq[j], iq[j]);
     int s = 0;
     uint32_t ph = 0;
-    for (int tile = blockIdx.x; tile < p.num_tiles && ok; tile += gridDim.x) {
-      const int tm = tile % p.tiles_m;
-      const int64_t row = (int64_t)tm * 128 + r;
-      for (int64_t kt = 0; kt < k_tiles; ++kt) {
-        ok = mbar_wait(&empty[s], ph ^ 1u, abort_flag, p.status, kWaitLimitNs);
-        if (!ok) break;
-        uint8_t* a_dst = a_base + s * p.a_slot_bytes;
-        uint8_t* e_dst = e_base + s * 2048;
-        if (p.a_mode == A_TMA_SPARSE) {
-          build_e_2of4(p, e_dst, r, row, kt);
-        } else if (p.a_mode == A_HYBRID) {
-          if (__ldg(p.tile_map + (int64_t)tm * p.hyb_tiles_k + kt / 2)) build_e_2of4(p, e_dst, r, row, kt);
-        } else if (p.a_mode == A_BUILD_SPARSE) {
-          uint32_t vals[16], w0, w1;
-          switch (p.pattern) {
-            case PAT_2_4: reencode_row<2, 4>(p, row, kt, vals, w0, w1); break;
-            case PAT_1_2: reencode_row<1, 2>(p, row, kt, vals, w0, w1); break;
-            case PAT_1_4: reencode_row<1, 4>(p, row, kt, vals, w0, w1); break;
-            case PAT_1_8: reencode_row<1, 8>(p, row, kt, vals, w0, w1); break;
-            default: reencode_row<2, 8>(p, row, kt, vals, w0, w1); break;
-          }
-          store_row_sw64(a_dst, r, vals);
-          put_e_word(e_dst, r, 0, w0);
-          put_e_word(e_dst, r, 1, w1);
-        } else {  // A_BUILD_DENSE
-          expand_row_sw128(p, a_dst, r, row, kt);
-        }
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&full[s]);
-        if (++s == stages) { s = 0; ph ^= 1u; }
+    int tile = blockIdx.x;
+    int64_t kt = 0;
+    for (int64_t it = 0; it < total; ++it) {
+      const uint2 mw = mq[0];
+      const int32_t ix = iq[0];
+#pragma unroll
+      for (int j = 0; j < PF - 1; ++j) {
+        mq[j] = mq[j + 1];
+        iq[j] = iq[j + 1];
       }
+      fetch(mq[PF - 1], iq[PF - 1]);
+      const int tm = tile % p.tiles_m, tn = tile / p.tiles_m;
+      const int64_t row = (int64_t)tm * 128 + r;
+      ok = mbar_wait(&empty[s], ph ^ 1u, abort_flag, p.status, kWaitLimitNs);
+      if (!ok) break;
+      uint8_t* a_dst = a_base + s * p.a_slot_bytes;
+      uint8_t* e_dst = e_base + s * 2048;
+      if (p.a_mode == A_TMA_SPARSE) {
+        put_e_word(e_dst, r, 0, mw.x);
+        put_e_word(e_dst, r, 1, mw.y);
+      } else if (p.a_mode == A_HYBRID) {
+        if (__ldg(p.tile_map + (int64_t)tm * p.hyb_tiles_k + kt / 2)) {
+          put_e_word(e_dst, r, 0, mw.x);
+          put_e_word(e_dst, r, 1, mw.y);
+        }
+      } else if (p.a_mode == A_BUILD_SPARSE) {
+        uint32_t vals[16], w0, w1;
+        switch (p.pattern) {
+          case PAT_2_4: reencode_row<2, 4>(p, row, kt, vals, w0, w1); break;
+          case PAT_1_2: reencode_row<1, 2>(p, row, kt, vals, w0, w1); break;
+          case PAT_1_4: reencode_row<1, 4>(p, row, kt, vals, w0, w1); break;
+          case PAT_1_8: reencode_row<1, 8>(p, row, kt, vals, w0, w1); break;
+          default: reencode_row<2, 8>(p, row, kt, vals, w0, w1); break;
+        }
+        store_row_sw64(a_dst, r, vals);
+        put_e_word(e_dst, r, 0, w0);
+        put_e_word(e_dst, r, 1, w1);
+      } else {  // A_BUILD_DENSE
+        expand_row_sw128(p, a_dst, r, row, kt);
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&full[s]);
+      if (p.permuted) {
+        // Gather K-rows 16*bw .. 16*bw+15 of the stage: row k of the tile is
+        // X[idx[k]][n0 .. n0+BN), 16 bytes per lane, written at its swizzled
+        // place in the MN-major B tile.
+        constexpr int LPR = BN / 8;       // lanes per row segment
+        constexpr int RPI = 32 / LPR;     // rows per warp instruction
+        uint8_t* b_dst = b_base + s * B_BYTES;
+        const int chunk = lane % LPR;
+        const int64_t col = (int64_t)tn * BN + chunk * 8;
+        const uint32_t cbytes = col >= p.T ? 0u : (col + 8 <= p.T ? 16u : (uint32_t)(p.T - col) * 2u);
+        const int strip = (chunk * 8) / STRIP_COLS;
+        const int cis = ((chunk * 8) % STRIP_COLS) / 8;  // 16-byte chunk inside the strip row
+#pragma unroll
+        for (int q = 0; q < 16 / RPI; ++q) {
+          const int i = q * RPI + lane / LPR;   // 0..15
+          const int32_t src = __shfl_sync(0xffffffffu, ix, i);
+          const int kr = bw * 16 + i;           // K-row inside the stage
+          const bool valid = src >= 0 && (int64_t)src < p.K;
+          const uint32_t nbytes = valid ? cbytes : 0u;
+          const uint16_t* g = nbytes ? p.X + (int64_t)src * p.ldx + col : p.X;
+          const int sw = cis ^ ((kr * BSW >> 7) & (BSW / 16 - 1));
+          cp_async_16(b_dst + strip * STRIP_BYTES + kr * BSW + (sw << 4), g, nbytes);
+        }
+        cp_async_arrive_noinc(&full[s]);
+      }
+      if (++s == stages) { s = 0; ph ^= 1u; }
+      if (++kt == k_tiles) { kt = 0; tile += gridDim.x; }
     }
   } else {
     // ------------------------------------------------------------ epilogue

@@ -18,10 +18,12 @@ enum Pattern : int { PAT_2_4 = 0, PAT_1_2 = 1, PAT_1_4 = 2, PAT_1_8 = 3, PAT_2_8
 struct SpmmParams {
   CUtensorMap tm_vals;  // compressed values R x K*n/m, box {32, 128}, 64B swizzle
   CUtensorMap tm_w;     // dense W R x K, box {64, 128}, 128B swizzle (hybrid)
-  CUtensorMap tm_x;     // X K x T, box {strip, 64} or {strip, 1} (gather4)
+  CUtensorMap tm_x;     // X K x T, box {strip, 64}
   const uint16_t* vals;
   const uint32_t* meta;
   const int32_t* idx;
+  const uint16_t* X;  // K x T, row stride ldx (read directly when permuted)
+  int64_t ldx;
   const uint8_t* tile_map;
   void* Y;
   uint32_t* status;
