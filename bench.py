@@ -53,6 +53,7 @@ def parse_args(argv=None):
     ap.add_argument("--layers", default=None, help="comma-separated subset of the workload's layers")
     ap.add_argument("--algo", choices=["auto", "sparse", "dense"], default="auto",
                     help="kernel design for 1:4 / 1:8 (nm_spmm_algo)")
+    ap.add_argument("--plain", action="store_true", help="ignore the workload's index map (y = W x)")
     ap.add_argument("--quick", action="store_true",
                     help="timed region only: no clock sampling, end-to-end pass, oracle baseline or extras")
     return ap.parse_args(argv)
@@ -233,10 +234,10 @@ def run_ours(args, rank: int, world: int, dist):
     for d in data:
         L = d.layer
         b = {"L": L, "d": d, "W": up(d.W), "X": up(d.X),
-             "idx": torch.from_numpy(d.idx).to(dev) if d.idx is not None else None,
+             "idx": torch.from_numpy(d.idx).to(dev) if d.idx is not None and not args.plain else None,
              "tmap": torch.from_numpy(d.tmap).to(dev) if d.tmap is not None else None,
              "vals": torch.empty((L.R, max(nm.nm_value_cols(L.K, L.n, L.m), 0)), dtype=torch.bfloat16, device=dev),
-             "meta": torch.empty((L.R, max(nm.nm_meta_cols(L.K, L.n, L.m), 0)), dtype=torch.int32, device=dev),
+             "meta": torch.empty((max(nm.nm_meta_words(L.R, L.K, L.n, L.m), 0),), dtype=torch.int32, device=dev),
              "Y": torch.empty((L.R, L.T), dtype=torch.bfloat16, device=dev)}
         b["flops"] = float(wl.hybrid_useful_flops(d) if d.tmap is not None else L.useful_flops)
         b["gemm_bytes"] = gemm_bytes(L, d)

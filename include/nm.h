@@ -13,11 +13,19 @@
  *  - Compressed form ("values" + "meta"):
  *      values  R x (K*N/M) bf16, the N survivors of each group pushed left in
  *              ascending position order; row stride K*N/M.
- *      meta    R x nm_meta_cols(K,N,M) uint32 words; survivor j of a row
- *              stores its in-group position (b = ceil(log2 M) bits) in word
- *              floor(j/S) at bit b*(j mod S), S = floor(32/b); unused bits 0.
- *              For 2:4 this is one nibble per group, first survivor in the
- *              low two bits, group 0 in the lowest nibble.
+ *      meta    nm_meta_words(R,K,N,M) uint32 words of in-group positions.
+ *        2:4   "tiled": one nibble p0 | p1 << 2 per group (first survivor in
+ *              the low bits), tiled in the order a sparse tensor-core MMA
+ *              reads them.  Rows go 16 at a time and columns 128 at a time;
+ *              block (rb, cb) is 64 words at word (rb*ceil(K/128) + cb)*64.
+ *              Word 4*l + q of a block (lane l = 0..15, quarter q = 0..3)
+ *              covers block columns 32q + 16h .. 32q + 16h + 15, h = l/8: row
+ *              16rb + (l%8) in bits 0..15 and row 16rb + 8 + (l%8) in bits
+ *              16..31, four nibbles in column order.  Groups past R or K in
+ *              the padded blocks hold 0x4, the positions (0,1) of a zero group.
+ *        other "row-wise": survivor j of row r stores its position
+ *              (b = ceil(log2 M) bits) in word r*ceil(K*N/M/S) + floor(j/S) at
+ *              bit b*(j mod S), S = floor(32/b); unused bits 0.
  *  - Every pointer is DEVICE memory owned by the caller (none is freed or
  *    retained).  The library allocates no device memory on these paths.
  *  - Calls are asynchronous on `stream` (a cudaStream_t; NULL = the legacy
@@ -75,8 +83,8 @@ typedef enum nm_algo {
 NM_API int nm_index_bits(int m);
 /* Columns of the value block, K*n/m (-1 on a bad pattern or K % m != 0). */
 NM_API int64_t nm_value_cols(int64_t K, int n, int m);
-/* 32-bit metadata words per row (-1 on a bad pattern or K % m != 0). */
-NM_API int64_t nm_meta_cols(int64_t K, int n, int m);
+/* 32-bit metadata words of an R x K matrix (-1 on a bad pattern or K % m != 0). */
+NM_API int64_t nm_meta_words(int64_t R, int64_t K, int n, int m);
 
 /* ------------------------------------------------------------- compress */
 /*
@@ -90,7 +98,7 @@ NM_API int64_t nm_meta_cols(int64_t K, int n, int m);
  * (survivors pushed left into an R x C/2 block plus 2-bit positions).
  *   W       [in]  R x K bf16, row stride ldw >= K (elements)
  *   values  [out] R x nm_value_cols(K,n,m) bf16
- *   meta    [out] R x nm_meta_cols(K,n,m) uint32 (fully written, unused bits 0)
+ *   meta    [out] nm_meta_words(R,K,n,m) uint32, every word written
  * Magnitudes are compared on the bf16 value: +0 and -0 tie, a NaN ranks above
  * every number.  Exactly n survivors are stored per group, zeros included.
  * Errors: NM_ERR_INVALID_ARG (bad pattern, K % m, ldw < K, null pointer).

@@ -54,6 +54,8 @@ def _load():
                 "oracle_positions_per_word": ([I], I),
                 "oracle_value_cols": ([I64, I, I], I64),
                 "oracle_meta_cols": ([I64, I, I], I64),
+                "oracle_meta_words": ([I64, I64, I, I], I64),
+                "oracle_positions": ([P, I64, I64, I, I, P], I),
                 "oracle_prune_mask": ([P, I64, I64, I64, I, I, P], I),
                 "oracle_compress": ([P, I64, I64, I64, I, I, P, P], I),
                 "oracle_decompress": ([P, P, I64, I64, I, I, P, I64], I),
@@ -102,6 +104,19 @@ def meta_cols(K: int, n: int, m: int) -> int:
     return _load().oracle_meta_cols(K, n, m)
 
 
+def meta_words(R: int, K: int, n: int, m: int) -> int:
+    """Total uint32 metadata words of an R x K matrix (tiled for 2:4, row-wise otherwise)."""
+    return _load().oracle_meta_words(R, K, n, m)
+
+
+def positions(meta: np.ndarray, R: int, K: int, n: int, m: int) -> np.ndarray:
+    """R x K*n/m in-group positions of the survivors, read back from the metadata."""
+    meta = np.ascontiguousarray(meta, dtype=np.uint32)
+    out = np.zeros((R, value_cols(K, n, m)), np.uint8)
+    _check(_load().oracle_positions(_ptr(meta), R, K, n, m, _ptr(out)), "positions")
+    return out
+
+
 def prune_mask(W: np.ndarray, n: int, m: int) -> np.ndarray:
     """uint8 R x K mask of the N:M survivors of bf16 W (R x K)."""
     W = _u16(W)
@@ -112,11 +127,13 @@ def prune_mask(W: np.ndarray, n: int, m: int) -> np.ndarray:
 
 
 def compress(W: np.ndarray, n: int, m: int):
-    """(values R x K*n/m uint16, meta R x meta_cols uint32) of bf16 W."""
+    """(values R x K*n/m uint16, meta: meta_words uint32, flat) of bf16 W."""
     W = _u16(W)
     R, K = W.shape
+    if K % m or not (1 <= n < m) or m not in (2, 4, 8, 16):
+        raise ValueError(f"oracle compress rejected its arguments (K={K}, {n}:{m})")
     vals = np.zeros((R, value_cols(K, n, m)), np.uint16)
-    meta = np.zeros((R, meta_cols(K, n, m)), np.uint32)
+    meta = np.zeros(meta_words(R, K, n, m), np.uint32)
     _check(_load().oracle_compress(_ptr(W), R, K, K, n, m, _ptr(vals), _ptr(meta)), "compress")
     return vals, meta
 

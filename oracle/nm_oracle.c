@@ -45,9 +45,14 @@
  *    worked row;
  *  - magnitudes are compared on the bf16 value; +0 and -0 tie; a NaN ranks
  *    above every number (Inf included) and NaNs tie among themselves;
- *  - positions use b = ceil(log2 M) bits; survivor j of a row goes to
- *    32-bit word floor(j/S) at bit b*(j mod S), S = floor(32/b); unused
- *    bits are zero;
+ *  - positions use b = ceil(log2 M) bits.  For every pattern except 2:4,
+ *    survivor j of a row goes to 32-bit word floor(j/S) at bit b*(j mod S),
+ *    S = floor(32/b), rows one after the other, unused bits zero
+ *    ("row-wise" packing).  For 2:4 a group's two positions form one nibble
+ *    p0 | p1 << 2 (first survivor low), and the nibbles are tiled in the order
+ *    a B200 sparse tensor-core instruction reads them ("tiled" packing, see
+ *    meta_slot_2of4 below); groups past R or K in the padded tiles hold the
+ *    nibble of an all-zero group, positions (0,1);
  *  - the permutation is applied as X_perm[k][t] = X[idx[k]][t];
  *  - W (dense, R x K) and the compressed values hold bf16 bit patterns
  *    (uint16); X is K x T row-major; Y is R x T (double here).
@@ -78,7 +83,7 @@ int oracle_index_bits(int m)
     return b;
 }
 
-/* Positions packed into one 32-bit word. */
+/* Positions packed into one 32-bit word (row-wise packing). */
 int oracle_positions_per_word(int m)
 {
     return 32 / oracle_index_bits(m);
@@ -90,11 +95,36 @@ int64_t oracle_value_cols(int64_t K, int n, int m)
     return K / m * n;
 }
 
-/* 32-bit metadata words per row: ceil(value_cols / S). */
+/* 32-bit metadata words per row (row-wise packing): ceil(value_cols / S). */
 int64_t oracle_meta_cols(int64_t K, int n, int m)
 {
     int64_t s = oracle_positions_per_word(m);
     return (oracle_value_cols(K, n, m) + s - 1) / s;
+}
+
+/* Total 32-bit metadata words of an R x K matrix.  Tiled 2:4: one block of
+ * 64 words per 16 rows x 128 columns, rows and columns padded up. */
+int64_t oracle_meta_words(int64_t R, int64_t K, int n, int m)
+{
+    if (n == 2 && m == 4) return (R + 15) / 16 * ((K + 127) / 128) * 64;
+    return R * oracle_meta_cols(K, n, m);
+}
+
+/* Tiled 2:4 packing: word and bit offset of the nibble of group g (columns
+ * 4g..4g+3) of row r.  Rows are taken 16 at a time and columns 128 at a
+ * time; block (rb, cb) holds 64 words at word (rb * ceil(K/128) + cb) * 64.
+ * Inside a block, word 4*l + q (lane l = 0..15, quarter q = 0..3) covers
+ * columns 32q + 16h .. 32q + 16h + 15 of the block, h = l / 8, for row
+ * (l mod 8) of the 16 in bits 0..15 and row 8 + (l mod 8) in bits 16..31,
+ * four nibbles each in column order. */
+static int64_t meta_slot_2of4(int64_t r, int64_t g, int64_t K, int *bit)
+{
+    int64_t cblocks = (K + 127) / 128;
+    int64_t rb = r / 16, cb = g / 32;
+    int q = (int)((g % 32) / 8), h = (int)((g % 8) / 4), t = (int)(g % 4);
+    int l = (int)(r % 8) + 8 * h;
+    *bit = 16 * (int)((r / 8) % 2) + 4 * t;
+    return (rb * cblocks + cb) * 64 + 4 * l + q;
 }
 
 static int pattern_ok(int n, int m)
@@ -146,7 +176,7 @@ int oracle_prune_mask(const uint16_t *W, int64_t R, int64_t K, int64_t ldw,
 /* ------------------------------------------------------------------ */
 /* Push-left compression [MN-fmt].                                      */
 /* values: R x (K*N/M) bf16 bits, survivors in ascending position.      */
-/* meta:   R x meta_cols words, b-bit in-group positions, LSB first.    */
+/* meta:   oracle_meta_words words (tiled 2:4, else row-wise b-bit).    */
 /* ------------------------------------------------------------------ */
 int oracle_compress(const uint16_t *W, int64_t R, int64_t K, int64_t ldw,
                     int n, int m, uint16_t *values, uint32_t *meta)
@@ -159,15 +189,28 @@ int oracle_compress(const uint16_t *W, int64_t R, int64_t K, int64_t ldw,
     uint8_t *mask = (uint8_t *)malloc((size_t)(R * K > 0 ? R * K : 1));
     if (!mask) return 2;
     oracle_prune_mask(W, R, K, ldw, n, m, mask);
-    memset(meta, 0, (size_t)(R * mcols) * sizeof(uint32_t));
+    int tiled = (n == 2 && m == 4);
+    int64_t words = oracle_meta_words(R, K, n, m);
+    for (int64_t i = 0; i < words; i++) meta[i] = tiled ? 0x44444444u : 0u;
     for (int64_t r = 0; r < R; r++) {
         int64_t j = 0; /* survivor index inside the row */
         for (int64_t g = 0; g < K / m; g++) {
+            uint32_t nib = 0;
+            int seen = 0;
             for (int p = 0; p < m; p++) {
                 if (!mask[r * K + g * m + p]) continue;
                 values[r * vcols + j] = W[r * ldw + g * m + p];
-                meta[r * mcols + j / s] |= (uint32_t)p << (b * (j % s));
+                if (tiled)
+                    nib |= (uint32_t)p << (2 * seen);
+                else
+                    meta[r * mcols + j / s] |= (uint32_t)p << (b * (j % s));
+                seen++;
                 j++;
+            }
+            if (tiled) {
+                int bit;
+                int64_t w = meta_slot_2of4(r, g, K, &bit);
+                meta[w] = (meta[w] & ~(0xFu << bit)) | (nib << bit);
             }
         }
     }
@@ -175,13 +218,30 @@ int oracle_compress(const uint16_t *W, int64_t R, int64_t K, int64_t ldw,
     return 0;
 }
 
-/* In-group position of survivor j of row r. */
-static int position_of(const uint32_t *meta, int64_t mcols, int64_t r, int64_t j, int m)
+/* In-group position of survivor j of row r (an R x K matrix). */
+static int position_of(const uint32_t *meta, int64_t K, int64_t r, int64_t j, int n, int m)
 {
+    if (n == 2 && m == 4) {
+        int bit;
+        int64_t w = meta_slot_2of4(r, j / 2, K, &bit);
+        return (int)((meta[w] >> (bit + 2 * (int)(j % 2))) & 3u);
+    }
     int b = oracle_index_bits(m);
     int s = oracle_positions_per_word(m);
+    int64_t mcols = oracle_meta_cols(K, n, m);
     uint32_t word = meta[r * mcols + j / s];
     return (int)((word >> (b * (j % s))) & ((1u << b) - 1u));
+}
+
+/* positions[r * vcols + j] = in-group position of survivor j of row r. */
+int oracle_positions(const uint32_t *meta, int64_t R, int64_t K, int n, int m, uint8_t *positions)
+{
+    if (!pattern_ok(n, m) || K % m != 0) return 1;
+    int64_t vcols = oracle_value_cols(K, n, m);
+    for (int64_t r = 0; r < R; r++)
+        for (int64_t j = 0; j < vcols; j++)
+            positions[r * vcols + j] = (uint8_t)position_of(meta, K, r, j, n, m);
+    return 0;
 }
 
 /* ------------------------------------------------------------------ */
@@ -193,12 +253,11 @@ int oracle_decompress(const uint16_t *values, const uint32_t *meta, int64_t R, i
 {
     if (!pattern_ok(n, m) || K % m != 0 || ldw < K) return 1;
     int64_t vcols = oracle_value_cols(K, n, m);
-    int64_t mcols = oracle_meta_cols(K, n, m);
     for (int64_t r = 0; r < R; r++) {
         for (int64_t k = 0; k < K; k++) W_out[r * ldw + k] = 0;
         for (int64_t j = 0; j < vcols; j++) {
             int64_t g = j / n;
-            int p = position_of(meta, mcols, r, j, m);
+            int p = position_of(meta, K, r, j, n, m);
             W_out[r * ldw + g * m + p] = values[r * vcols + j];
         }
     }
@@ -217,12 +276,11 @@ int oracle_spmm(const uint16_t *values, const uint32_t *meta, int n, int m,
 {
     if (!pattern_ok(n, m) || K % m != 0 || ldx < T || ldy < T) return 1;
     int64_t vcols = oracle_value_cols(K, n, m);
-    int64_t mcols = oracle_meta_cols(K, n, m);
     for (int64_t r = 0; r < R; r++) {
         for (int64_t t = 0; t < T; t++) {
             double acc = 0.0;
             for (int64_t j = 0; j < vcols; j++) {
-                int64_t k = (j / n) * m + position_of(meta, mcols, r, j, m);
+                int64_t k = (j / n) * m + position_of(meta, K, r, j, n, m);
                 int64_t src = idx ? (int64_t)idx[k] : k;
                 acc += bf16_value(values[r * vcols + j]) * bf16_value(X[src * ldx + t]);
             }
@@ -241,13 +299,12 @@ int oracle_spmm_sampled(const uint16_t *values, const uint32_t *meta, int n, int
 {
     if (!pattern_ok(n, m) || K % m != 0 || ldx < T) return 1;
     int64_t vcols = oracle_value_cols(K, n, m);
-    int64_t mcols = oracle_meta_cols(K, n, m);
     for (int64_t i = 0; i < count; i++) {
         int64_t r = rows[i], t = cols[i];
         if (r < 0 || r >= R || t < 0 || t >= T) return 3;
         double acc = 0.0, mag = 0.0;
         for (int64_t j = 0; j < vcols; j++) {
-            int64_t k = (j / n) * m + position_of(meta, mcols, r, j, m);
+            int64_t k = (j / n) * m + position_of(meta, K, r, j, n, m);
             int64_t src = idx ? (int64_t)idx[k] : k;
             double w = bf16_value(values[r * vcols + j]);
             double x = bf16_value(X[src * ldx + t]);

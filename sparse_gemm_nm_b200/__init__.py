@@ -42,7 +42,7 @@ _P, _I64, _I, _U64 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_uin
 SIGNATURES = {
     "nm_index_bits": ([_I], _I),
     "nm_value_cols": ([_I64, _I, _I], _I64),
-    "nm_meta_cols": ([_I64, _I, _I], _I64),
+    "nm_meta_words": ([_I64, _I64, _I, _I], _I64),
     "nm_prune_compress": ([_P, _I64, _I64, _I64, _I, _I, _P, _P, _P], _I),
     "nm_decompress": ([_P, _P, _I64, _I64, _I, _I, _P, _I64, _P], _I),
     "nm_spmm": ([_P, _P, _I, _I, _I64, _I64, _P, _I64, _I64, _P, _I64, _I, _P], _I),
@@ -121,8 +121,8 @@ def nm_value_cols(K: int, n: int, m: int) -> int:
     return lib().nm_value_cols(K, n, m)
 
 
-def nm_meta_cols(K: int, n: int, m: int) -> int:
-    return lib().nm_meta_cols(K, n, m)
+def nm_meta_words(R: int, K: int, n: int, m: int) -> int:
+    return lib().nm_meta_words(R, K, n, m)
 
 
 def nm_prune_compress(W, R, K, ldw, n, m, values, meta, stream=None) -> None:
@@ -180,14 +180,14 @@ def _require_cuda(*ts):
 
 
 def prune_compress(W, n: int, m: int, stream=None):
-    """(values R x K*n/m bf16, meta R x nm_meta_cols uint32-as-int32) of bf16 W (R x K)."""
+    """(values R x K*n/m bf16, meta: nm_meta_words uint32 as int32, flat) of bf16 W (R x K)."""
     import torch
     _require_cuda(W)
     R, K = W.shape
     if nm_value_cols(K, n, m) < 0:  # let the library name the bad argument
         _check(lib().nm_prune_compress(None, R, K, K, n, m, None, None, None), "nm_prune_compress")
     vals = torch.empty((R, nm_value_cols(K, n, m)), dtype=torch.bfloat16, device=W.device)
-    meta = torch.empty((R, max(nm_meta_cols(K, n, m), 0)), dtype=torch.int32, device=W.device)
+    meta = torch.empty((max(nm_meta_words(R, K, n, m), 0),), dtype=torch.int32, device=W.device)
     nm_prune_compress(W, R, K, W.stride(0), n, m, vals, meta, stream)
     return vals, meta
 

@@ -91,7 +91,7 @@ static EncodeTiledFn encode_fn() {
 
 static nm_status make_tmap(CUtensorMap* tm, const void* base, uint64_t inner, uint64_t outer,
                            uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer, int swizzle_bytes,
-                           const char* what) {
+                           const char* what, CUtensorMapDataType dtype = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return fail(NM_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
   cuuint64_t dims[2] = {inner, outer};
@@ -100,11 +100,26 @@ static nm_status make_tmap(CUtensorMap* tm, const void* base, uint64_t inner, ui
   cuuint32_t estr[2] = {1, 1};
   CUtensorMapSwizzle swz = swizzle_bytes == 128  ? CU_TENSOR_MAP_SWIZZLE_128B
                            : swizzle_bytes == 64 ? CU_TENSOR_MAP_SWIZZLE_64B
-                                                 : CU_TENSOR_MAP_SWIZZLE_32B;
-  CUresult r = fn(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
-                  CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+                           : swizzle_bytes == 32 ? CU_TENSOR_MAP_SWIZZLE_32B
+                                                 : CU_TENSOR_MAP_SWIZZLE_NONE;
+  CUresult r = fn(tm, dtype, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return fail(NM_ERR_CUDA, "cuTensorMapEncodeTiled(%s) failed with %d", what, (int)r);
+  return NM_OK;
+}
+
+// 3-D map of the tiled 2:4 metadata: {64 words of a block, column blocks, row blocks}.
+static nm_status make_meta_tmap(CUtensorMap* tm, const void* meta, int64_t rblocks, int64_t cblocks) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return fail(NM_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
+  cuuint64_t dims[3] = {64, (cuuint64_t)cblocks, (cuuint64_t)rblocks};
+  cuuint64_t strides[2] = {256, (cuuint64_t)cblocks * 256};
+  cuuint32_t box[3] = {64, 1, 8};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(tm, CU_TENSOR_MAP_DATA_TYPE_UINT32, 3, const_cast<void*>(meta), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(NM_ERR_CUDA, "cuTensorMapEncodeTiled(meta) failed with %d", (int)r);
   return NM_OK;
 }
 
@@ -186,6 +201,8 @@ static nm_status run_gemm(const GemmRequest& q, cudaStream_t stream) {
   p.m = q.m;
   p.vcols = value_cols(q.K, q.n, q.m);
   p.mcols = meta_cols(q.K, q.n, q.m);
+  p.meta_rblocks = meta_row_blocks(q.R);
+  p.meta_cblocks = meta_col_blocks(q.K);
   p.pattern = pattern_id(q.n, q.m);
   p.permuted = q.idx != nullptr;
   p.out_f32 = q.y_dtype == NM_OUT_F32;
@@ -212,6 +229,27 @@ static nm_status run_gemm(const GemmRequest& q, cudaStream_t stream) {
     return fail(NM_ERR_UNSUPPORTED, "pattern %d:%d does not fit the 2:4 sparse MMA", q.n, q.m);
   }
 
+  p.status = status_word_ptr();
+  if (!p.status) return fail(NM_ERR_CUDA, "device status word is unavailable");
+
+  // Two SMs per 256 x 256 tile when the shape allows it (2:4 from TMA, K % 128 == 0).
+  if (q.algo != NM_ALGO_DENSE_TC && pair_kernel_fits(p) && al16(q.meta)) {
+    p.tiles_m = (int)((q.R + 255) / 256);
+    p.tiles_n = (int)((q.T + 255) / 256);
+    if ((int64_t)p.tiles_m * p.tiles_n >= (1ll << 31)) return fail(NM_ERR_UNSUPPORTED, "too many tiles");
+    p.num_tiles = p.tiles_m * p.tiles_n;
+    p.k_tiles = q.K / 128;
+    st = make_tmap(&p.tm_x, q.X, (uint64_t)q.T, (uint64_t)q.K, (uint64_t)q.ldx * 2, 64, 128, 128, "X");
+    if (st != NM_OK) return st;
+    st = make_tmap(&p.tm_vals, q.values, (uint64_t)p.vcols, (uint64_t)q.R, (uint64_t)p.vcols * 2, 64, 128, 128,
+                   "values");
+    if (st != NM_OK) return st;
+    st = make_meta_tmap(&p.tm_meta, q.meta, p.meta_rblocks, p.meta_cblocks);
+    if (st != NM_OK) return st;
+    cudaError_t e = launch_spmm_pair(p, stream);
+    return e == cudaSuccess ? NM_OK : cuda_fail(e, "spmm pair launch");
+  }
+
   const int bn = pick_bn(q.T);
   const int bsw = bn >= 64 ? 128 : bn * 2;
   p.a_slot_bytes = (p.a_mode == A_BUILD_DENSE || p.a_mode == A_HYBRID) ? 16384u : 8192u;
@@ -222,8 +260,7 @@ static nm_status run_gemm(const GemmRequest& q, cudaStream_t stream) {
   p.num_tiles = p.tiles_m * p.tiles_n;
   p.k_tiles = (q.K + 63) / 64;
 
-  st = make_tmap(&p.tm_x, q.X, (uint64_t)q.T, (uint64_t)q.K, (uint64_t)q.ldx * 2, bsw / 2, 64,
-                 bsw, "X");
+  st = make_tmap(&p.tm_x, q.X, (uint64_t)q.T, (uint64_t)q.K, (uint64_t)q.ldx * 2, bsw / 2, 64, bsw, "X");
   if (st != NM_OK) return st;
   if (p.a_mode == A_TMA_SPARSE || p.a_mode == A_HYBRID) {
     st = make_tmap(&p.tm_vals, q.values, (uint64_t)p.vcols, (uint64_t)q.R, (uint64_t)p.vcols * 2, 32, 128, 64,
@@ -251,9 +288,9 @@ int64_t nm_value_cols(int64_t K, int n, int m) {
   return value_cols(K, n, m);
 }
 
-int64_t nm_meta_cols(int64_t K, int n, int m) {
-  if (!pattern_ok(n, m) || K < 0 || K % m != 0) return -1;
-  return meta_cols(K, n, m);
+int64_t nm_meta_words(int64_t R, int64_t K, int n, int m) {
+  if (!pattern_ok(n, m) || R < 0 || K < 0 || K % m != 0) return -1;
+  return meta_words(R, K, n, m);
 }
 
 nm_status nm_prune_compress(const uint16_t* W, int64_t R, int64_t K, int64_t ldw, int n, int m, uint16_t* values,
@@ -265,6 +302,8 @@ nm_status nm_prune_compress(const uint16_t* W, int64_t R, int64_t K, int64_t ldw
   if (ldw < K) return fail(NM_ERR_INVALID_ARG, "ldw < K");
   if (R == 0 || K == 0) return NM_OK;
   if (!W || !values || !meta) return fail(NM_ERR_INVALID_ARG, "null pointer");
+  if (R >= (1ll << 31) || K >= (1ll << 31) || meta_words(R, K, n, m) >= (1ll << 31))
+    return fail(NM_ERR_UNSUPPORTED, "matrix too large for one call");
   nm_status st = require_device();
   if (st != NM_OK) return st;
   cudaError_t e = launch_compress(W, R, K, ldw, n, m, values, meta, static_cast<cudaStream_t>(stream));
@@ -280,6 +319,8 @@ nm_status nm_decompress(const uint16_t* values, const uint32_t* meta, int64_t R,
   if (ldw < K) return fail(NM_ERR_INVALID_ARG, "ldw < K");
   if (R == 0 || K == 0) return NM_OK;
   if (!W_out || !values || !meta) return fail(NM_ERR_INVALID_ARG, "null pointer");
+  if (R >= (1ll << 31) || K >= (1ll << 31) || meta_words(R, K, n, m) >= (1ll << 31))
+    return fail(NM_ERR_UNSUPPORTED, "matrix too large for one call");
   nm_status st = require_device();
   if (st != NM_OK) return st;
   cudaError_t e = launch_decompress(values, meta, R, K, n, m, W_out, ldw, static_cast<cudaStream_t>(stream));

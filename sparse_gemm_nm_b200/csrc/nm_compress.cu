@@ -8,7 +8,9 @@
 // which orders finite values and infinities exactly as |w| does; NaNs are
 // folded to one key just above +Inf so they tie among themselves.
 // Storage (same page, storage paragraphs of "Where this sits among the three
-// case studies"): survivors pushed left in ascending position; b-bit
+// case studies"): survivors pushed left in ascending position.  2:4 positions
+// are tiled in the sparse tensor core's order (one nibble per group, see
+// compress_2of4_tiled_kernel); other patterns are packed row-wise, b-bit
 // positions, survivor j of a row in word j/S at bit b*(j%S).
 #include <cstdint>
 #include <cuda_runtime.h>
@@ -42,48 +44,67 @@ __device__ __forceinline__ void select_2of4(uint32_t e0, uint32_t e1, uint32_t e
   packed = v0 | (v1 << 16);
 }
 
-// 2:4 fast path.  A warp walks the matrix in 512-byte pieces (32 lanes x 8
-// weights = 8 metadata words); each lane loads 16 contiguous bytes, selects
-// its two groups, stores 8 bytes of values, and four neighbouring lanes merge
-// their metadata bytes into one word with shuffles.  Loads and stores of a
-// warp instruction are contiguous.  U pieces per lane are kept in flight.
-constexpr int kCompressUnroll = 4;
+// 2:4 with tiled metadata.  One thread per metadata word: word 4*l + q of
+// block (rb, cb) holds, for K columns k0 = 128*cb + 32*q + 16*(l/8) .. k0+15,
+// the four nibbles of row 16*rb + (l%8) in bits 0..15 and of that row + 8 in
+// bits 16..31.  The thread reads those 2 x 16 weights, selects, writes the
+// 2 x 8 survivors and the word.  Rows or columns past R or K (block padding)
+// get the nibble of an all-zero group, positions (0,1), and write no values.
+__device__ __forceinline__ uint32_t compress_half16(const uint16_t* __restrict__ wrow, uint16_t* __restrict__ vrow,
+                                                    uint32_t k0, uint32_t K, bool vec) {
+  uint32_t e[16];
+  if (vec && k0 + 16 <= K) {
+    const uint4 a = __ldg(reinterpret_cast<const uint4*>(wrow + k0));
+    const uint4 b = __ldg(reinterpret_cast<const uint4*>(wrow + k0 + 8));
+    const uint32_t w8[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      e[2 * i] = w8[i] & 0xFFFFu;
+      e[2 * i + 1] = w8[i] >> 16;
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < 16; ++i) e[i] = (k0 + i < K) ? (uint32_t)wrow[k0 + i] : 0u;
+  }
+  uint32_t nibs = 0, pk[4];
+#pragma unroll
+  for (int t = 0; t < 4; ++t) {
+    uint32_t nib;
+    select_2of4(e[4 * t], e[4 * t + 1], e[4 * t + 2], e[4 * t + 3], nib, pk[t]);
+    nibs |= (k0 + 4 * t < K ? nib : 0x4u) << (4 * t);
+  }
+  if (vec && k0 + 16 <= K) {
+    *reinterpret_cast<uint4*>(vrow + k0 / 2) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+  } else {
+#pragma unroll
+    for (int t = 0; t < 4; ++t)
+      if (k0 + 4 * t < K) *reinterpret_cast<uint32_t*>(vrow + k0 / 2 + 2 * t) = pk[t];
+  }
+  return nibs;
+}
 
-__global__ void __launch_bounds__(256) compress_2of4_kernel(const uint16_t* __restrict__ W, uint32_t R,
-                                                            uint32_t K, int64_t ldw, uint16_t* __restrict__ V,
-                                                            uint32_t* __restrict__ meta) {
-  // R * K / 8 < 2^32 is checked by the launcher: 32-bit index arithmetic.
-  const uint32_t lane = threadIdx.x & 31u;
-  const uint32_t cpr = K >> 3;           // 8-weight chunks per row
-  const uint32_t total = R * cpr;        // chunks in the matrix
-  const uint32_t warp_id = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-  const uint32_t nwarps = (gridDim.x * blockDim.x) >> 5;
-  for (uint32_t base = warp_id * 32u * kCompressUnroll; base < total; base += nwarps * 32u * kCompressUnroll) {
-    uint4 in[kCompressUnroll];
-    uint32_t rr[kCompressUnroll], cc[kCompressUnroll];
-#pragma unroll
-    for (int u = 0; u < kCompressUnroll; ++u) {
-      const uint32_t c = base + u * 32u + lane;
-      rr[u] = c / cpr;
-      cc[u] = c - rr[u] * cpr;
-      in[u] = c < total ? __ldg(reinterpret_cast<const uint4*>(W + (int64_t)rr[u] * ldw + (cc[u] << 3)))
-                        : make_uint4(0, 0, 0, 0);
+__global__ void __launch_bounds__(256) compress_2of4_tiled_kernel(const uint16_t* __restrict__ W, uint32_t R,
+                                                                  uint32_t K, int64_t ldw,
+                                                                  uint16_t* __restrict__ V,
+                                                                  uint32_t* __restrict__ meta, uint32_t cblocks,
+                                                                  uint32_t total, bool vec) {
+  for (uint32_t w = blockIdx.x * blockDim.x + threadIdx.x; w < total; w += gridDim.x * blockDim.x) {
+    const uint32_t blk = w >> 6, wi = w & 63u;
+    const uint32_t l = wi >> 2, q = wi & 3u;
+    const uint32_t rb = blk / cblocks, cb = blk - rb * cblocks;
+    const uint32_t r_lo = rb * 16 + (l & 7u);
+    const uint32_t k0 = cb * 128 + q * 32 + (l >> 3) * 16;
+    uint32_t word = 0x44444444u;
+    if (k0 < K) {
+      if (r_lo < R)
+        word = (word & 0xFFFF0000u) |
+               compress_half16(W + (int64_t)r_lo * ldw, V + (int64_t)r_lo * (K >> 1), k0, K, vec);
+      if (r_lo + 8 < R)
+        word = (word & 0x0000FFFFu) |
+               (compress_half16(W + (int64_t)(r_lo + 8) * ldw, V + (int64_t)(r_lo + 8) * (K >> 1), k0, K, vec)
+                << 16);
     }
-#pragma unroll
-    for (int u = 0; u < kCompressUnroll; ++u) {
-      uint32_t nib0, nib1, pk0, pk1;
-      select_2of4(in[u].x & 0xFFFFu, in[u].x >> 16, in[u].y & 0xFFFFu, in[u].y >> 16, nib0, pk0);
-      select_2of4(in[u].z & 0xFFFFu, in[u].z >> 16, in[u].w & 0xFFFFu, in[u].w >> 16, nib1, pk1);
-      // byte of this lane inside its metadata word: lanes 4q..4q+3 -> bytes 0..3
-      uint32_t word = (nib0 | (nib1 << 4)) << (8 * (lane & 3));
-      word |= __shfl_xor_sync(0xffffffffu, word, 1);
-      word |= __shfl_xor_sync(0xffffffffu, word, 2);
-      if (base + u * 32u + lane < total) {
-        const int64_t r = rr[u];
-        *reinterpret_cast<uint2*>(V + r * (K >> 1) + (cc[u] << 2)) = make_uint2(pk0, pk1);
-        if ((lane & 3) == 0) meta[r * (K >> 5) + (cc[u] >> 2)] = word;
-      }
-    }
+    meta[w] = word;
   }
 }
 
@@ -137,35 +158,54 @@ __global__ void __launch_bounds__(256) compress_generic_kernel(const uint16_t* _
   }
 }
 
-// 2:4 fast decompress: one thread per metadata word -> 32 output weights.
-__global__ void __launch_bounds__(256) decompress_2of4_kernel(const uint16_t* __restrict__ V,
-                                                              const uint32_t* __restrict__ meta, int64_t R,
-                                                              int64_t K, uint16_t* __restrict__ W, int64_t ldw) {
-  const int64_t wpr = K >> 5;
-  const int64_t total = R * wpr;
-  for (int64_t w = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; w < total;
-       w += (int64_t)gridDim.x * blockDim.x) {
-    const int64_t r = w / wpr;
-    const int64_t c = w - r * wpr;
+// 2:4 decompress from tiled metadata: one thread per word -> 2 x 16 weights.
+__device__ __forceinline__ void decompress_half16(const uint16_t* __restrict__ vrow, uint16_t* __restrict__ wrow,
+                                                  uint32_t nibs, uint32_t k0, uint32_t K, bool vec) {
+  uint32_t out[8];
+#pragma unroll
+  for (int t = 0; t < 4; ++t) {
+    const uint32_t nib = (nibs >> (4 * t)) & 0xFu;
+    const uint32_t p0 = nib & 3u, p1 = nib >> 2;
+    uint32_t v = 0;
+    if (k0 + 4 * t < K) v = *reinterpret_cast<const uint32_t*>(vrow + k0 / 2 + 2 * t);
+    const uint32_t v0 = v & 0xFFFFu, v1 = v >> 16;
+    uint32_t e[4];
+#pragma unroll
+    for (uint32_t i = 0; i < 4; ++i) e[i] = (i == p0) ? v0 : (i == p1) ? v1 : 0u;
+    out[2 * t] = e[0] | (e[1] << 16);
+    out[2 * t + 1] = e[2] | (e[3] << 16);
+  }
+  if (vec && k0 + 16 <= K) {
+    uint4* dst = reinterpret_cast<uint4*>(wrow + k0);
+    dst[0] = make_uint4(out[0], out[1], out[2], out[3]);
+    dst[1] = make_uint4(out[4], out[5], out[6], out[7]);
+  } else {
+#pragma unroll
+    for (int t = 0; t < 4; ++t)
+      if (k0 + 4 * t < K) {
+        *reinterpret_cast<uint32_t*>(wrow + k0 + 4 * t) = out[2 * t];
+        *reinterpret_cast<uint32_t*>(wrow + k0 + 4 * t + 2) = out[2 * t + 1];
+      }
+  }
+}
+
+__global__ void __launch_bounds__(256) decompress_2of4_tiled_kernel(const uint16_t* __restrict__ V,
+                                                                    const uint32_t* __restrict__ meta, uint32_t R,
+                                                                    uint32_t K, uint16_t* __restrict__ W,
+                                                                    int64_t ldw, uint32_t cblocks, uint32_t total,
+                                                                    bool vec) {
+  for (uint32_t w = blockIdx.x * blockDim.x + threadIdx.x; w < total; w += gridDim.x * blockDim.x) {
+    const uint32_t blk = w >> 6, wi = w & 63u;
+    const uint32_t l = wi >> 2, q = wi & 3u;
+    const uint32_t rb = blk / cblocks, cb = blk - rb * cblocks;
+    const uint32_t r_lo = rb * 16 + (l & 7u);
+    const uint32_t k0 = cb * 128 + q * 32 + (l >> 3) * 16;
+    if (k0 >= K) continue;
     const uint32_t word = __ldg(meta + w);
-    const uint4* src = reinterpret_cast<const uint4*>(V + r * (K >> 1) + (c << 4));
-    const uint4 a = __ldg(src), b = __ldg(src + 1);
-    const uint32_t vals[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
-    uint32_t out[16];
-#pragma unroll
-    for (int g = 0; g < 8; ++g) {
-      const uint32_t nib = (word >> (4 * g)) & 0xFu;
-      const uint32_t p0 = nib & 3u, p1 = nib >> 2;
-      const uint32_t v0 = vals[g] & 0xFFFFu, v1 = vals[g] >> 16;
-      uint32_t e[4];
-#pragma unroll
-      for (uint32_t i = 0; i < 4; ++i) e[i] = (i == p0) ? v0 : (i == p1) ? v1 : 0u;
-      out[2 * g] = e[0] | (e[1] << 16);
-      out[2 * g + 1] = e[2] | (e[3] << 16);
-    }
-    uint4* dst = reinterpret_cast<uint4*>(W + r * ldw + (c << 5));
-#pragma unroll
-    for (int i = 0; i < 4; ++i) dst[i] = make_uint4(out[4 * i], out[4 * i + 1], out[4 * i + 2], out[4 * i + 3]);
+    if (r_lo < R)
+      decompress_half16(V + (int64_t)r_lo * (K >> 1), W + (int64_t)r_lo * ldw, word & 0xFFFFu, k0, K, vec);
+    if (r_lo + 8 < R)
+      decompress_half16(V + (int64_t)(r_lo + 8) * (K >> 1), W + (int64_t)(r_lo + 8) * ldw, word >> 16, k0, K, vec);
   }
 }
 
@@ -223,11 +263,11 @@ static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 
 cudaError_t launch_compress(const uint16_t* W, int64_t R, int64_t K, int64_t ldw, int n, int m, uint16_t* values,
                             uint32_t* meta, cudaStream_t s) {
   const int threads = 256;
-  if (n == 2 && m == 4 && K % 32 == 0 && ldw % 8 == 0 && aligned16(W) && aligned16(values) &&
-      R * (K / 8) < (int64_t(1) << 32) - 4096 * kCompressUnroll) {
-    const int64_t work = R * (K / 8) / kCompressUnroll;
-    compress_2of4_kernel<<<grid_for(work, threads), threads, 0, s>>>(W, (uint32_t)R, (uint32_t)K, ldw, values,
-                                                                     meta);
+  if (tiled_meta(n, m)) {
+    const int64_t total = meta_words(R, K, n, m);
+    const bool vec = K % 16 == 0 && ldw % 8 == 0 && aligned16(W) && aligned16(values);
+    compress_2of4_tiled_kernel<<<grid_for(total, threads), threads, 0, s>>>(
+        W, (uint32_t)R, (uint32_t)K, ldw, values, meta, (uint32_t)meta_col_blocks(K), (uint32_t)total, vec);
   } else {
     const int64_t work = R * meta_cols(K, n, m);
     const int grid = grid_for(work, threads);
@@ -245,9 +285,11 @@ cudaError_t launch_compress(const uint16_t* W, int64_t R, int64_t K, int64_t ldw
 cudaError_t launch_decompress(const uint16_t* values, const uint32_t* meta, int64_t R, int64_t K, int n, int m,
                               uint16_t* W_out, int64_t ldw, cudaStream_t s) {
   const int threads = 256;
-  if (n == 2 && m == 4 && K % 32 == 0 && ldw % 8 == 0 && aligned16(W_out) && aligned16(values)) {
-    const int64_t work = R * (K / 32);
-    decompress_2of4_kernel<<<grid_for(work, threads), threads, 0, s>>>(values, meta, R, K, W_out, ldw);
+  if (tiled_meta(n, m)) {
+    const int64_t total = meta_words(R, K, n, m);
+    const bool vec = K % 16 == 0 && ldw % 8 == 0 && aligned16(W_out) && aligned16(values);
+    decompress_2of4_tiled_kernel<<<grid_for(total, threads), threads, 0, s>>>(
+        values, meta, (uint32_t)R, (uint32_t)K, W_out, ldw, (uint32_t)meta_col_blocks(K), (uint32_t)total, vec);
   } else {
     const int64_t work = R * (K / m);
     const int grid = grid_for(work, threads);

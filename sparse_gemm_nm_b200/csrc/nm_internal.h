@@ -15,6 +15,14 @@ inline int64_t meta_cols(int64_t K, int n, int m) {
   const int64_t s = positions_per_word(m);
   return (value_cols(K, n, m) + s - 1) / s;
 }
+// 2:4 metadata is tiled for the sparse tensor core: 64 words per block of
+// 16 rows x 128 columns, rows and columns padded up to whole blocks.
+inline bool tiled_meta(int n, int m) { return n == 2 && m == 4; }
+inline int64_t meta_row_blocks(int64_t R) { return (R + 15) / 16; }
+inline int64_t meta_col_blocks(int64_t K) { return (K + 127) / 128; }
+inline int64_t meta_words(int64_t R, int64_t K, int n, int m) {
+  return tiled_meta(n, m) ? meta_row_blocks(R) * meta_col_blocks(K) * 64 : R * meta_cols(K, n, m);
+}
 
 // Patterns whose survivors never exceed two per aligned group of four, so a
 // tile of them can be re-encoded as 2:4 for the sparse MMA.

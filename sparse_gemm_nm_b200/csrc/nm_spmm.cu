@@ -75,31 +75,19 @@ __device__ __forceinline__ void put_e_word(uint8_t* e_slot, int r, int kk, uint3
   *hi = static_cast<uint16_t>(w >> 16);
 }
 
-// Nibbles of groups at or beyond K become (0,1), a valid pair over zero values.
-__device__ __forceinline__ uint32_t clamp_meta_word(uint32_t w, int64_t k_word0, int64_t K) {
-  const int64_t valid = (K - k_word0) / 4;  // groups of this word inside K
-  if (valid >= 8) return w;
-  if (valid <= 0) return 0x44444444u;
-  const uint32_t keep = (1u << (4 * valid)) - 1u;
-  return (w & keep) | (0x44444444u & ~keep);
-}
-
-// 2:4 metadata of one row for stage kt (two 32-K words) from the row-wise form.
-__device__ __forceinline__ void build_e_2of4(const SpmmParams& p, uint8_t* e_slot, int r, int64_t row,
-                                             int64_t kt) {
-#pragma unroll
-  for (int kk = 0; kk < 2; ++kk) {
-    const int64_t c = kt * 2 + kk;
-    uint32_t w = 0x44444444u;
-    if (row < p.R && c < p.mcols) w = clamp_meta_word(__ldg(p.meta + row * p.mcols + c), c * 32, p.K);
-    put_e_word(e_slot, r, kk, w);
-  }
-}
-
-// Position of survivor j of a row (b-bit fields, S per word).
+// Position of survivor j of a row (row-wise packing: b-bit fields, S per word).
 __device__ __forceinline__ uint32_t pos_of(const uint32_t* mrow, int64_t j, int b, int s) {
   const uint32_t w = __ldg(mrow + j / s);
   return (w >> (b * (int)(j % s))) & ((1u << b) - 1u);
+}
+
+// 2:4 nibble (p0 | p1 << 2) of group g of row `row` in the tiled packing.
+__device__ __forceinline__ uint32_t nibble_2of4(const SpmmParams& p, int64_t row, int64_t g) {
+  const int64_t blk = (row >> 4) * p.meta_cblocks + (g >> 5);
+  const int l = (int)(row & 7) + 8 * (int)((g >> 2) & 1);
+  const int q = (int)((g >> 3) & 3);
+  const int bit = 16 * (int)((row >> 3) & 1) + 4 * (int)(g & 3);
+  return (__ldg(p.meta + blk * 64 + 4 * l + q) >> bit) & 0xFu;
 }
 
 // One 2:4 group from a single survivor at in-group position q (0..3) value v.
@@ -119,7 +107,7 @@ __device__ __forceinline__ void reencode_row(const SpmmParams& p, int64_t row, i
   if (row >= p.R) return;
   const int64_t k0 = kt * 64;
   const uint16_t* vrow = p.vals + row * p.vcols;
-  const uint32_t* mrow = p.meta + row * p.mcols;
+  const uint32_t* mrow = p.meta + row * p.mcols;  // row-wise patterns only
   constexpr int B = M == 2 ? 1 : M == 4 ? 2 : 3;
   constexpr int S = 32 / B;
   uint32_t nibs[16];
@@ -131,7 +119,7 @@ __device__ __forceinline__ void reencode_row(const SpmmParams& p, int64_t row, i
       const int64_t g = k0 / 4 + q;
       if (g * 4 < p.K) {
         vals[q] = (uint32_t)vrow[2 * g] | ((uint32_t)vrow[2 * g + 1] << 16);
-        nibs[q] = pos_of(mrow, 2 * g, B, S) | (pos_of(mrow, 2 * g + 1, B, S) << 2);
+        nibs[q] = nibble_2of4(p, row, g);
       }
     }
   } else if (N == 1 && M == 2) {
@@ -215,9 +203,11 @@ __device__ __forceinline__ void expand_row_sw128(const SpmmParams& p, uint8_t* t
   if (g1 * m > p.K) g1 = p.K / m;
   const uint16_t* vrow = p.vals + row * p.vcols;
   const uint32_t* mrow = p.meta + row * p.mcols;
+  const bool tiled = n == 2 && m == 4;
   for (int64_t j = g0 * n; j < g1 * n; ++j) {
     const int64_t g = j / n;
-    const int kr = (int)(g * m + pos_of(mrow, j, b, s) - k0);  // 0..63
+    const uint32_t pos = tiled ? (nibble_2of4(p, row, g) >> (2 * (j & 1))) & 3u : pos_of(mrow, j, b, s);
+    const int kr = (int)(g * m + pos - k0);  // 0..63
     const int c = kr >> 3;
     *reinterpret_cast<uint16_t*>(base + (((c ^ x) << 4) | ((kr & 7) << 1))) = vrow[j];
   }
@@ -388,12 +378,12 @@ __global__ void __launch_bounds__(kThreads, 1) spmm_kernel(const __grid_constant
       ix = -1;
       if (f_it < total) {
         if (e_from_meta) {
-          const int64_t row = (int64_t)(f_tile % p.tiles_m) * 128 + r;
-          if (row < p.R) {
-            const int64_t c = f_kt * 2;
-            const uint32_t* mrow = p.meta + row * p.mcols;
-            if (c < p.mcols) mw.x = clamp_meta_word(__ldg(mrow + c), c * 32, p.K);
-            if (c + 1 < p.mcols) mw.y = clamp_meta_word(__ldg(mrow + c + 1), (c + 1) * 32, p.K);
+          // TMEM lane r of the tile is lane r%16 of row block (m0 + r)/16 in the
+          // tiled 2:4 metadata; this stage's 64 columns are words q = 2*(kt%2), +1.
+          const int64_t rb = (int64_t)(f_tile % p.tiles_m) * 8 + (r >> 4);
+          if (rb < p.meta_rblocks) {
+            const uint32_t* blk = p.meta + (rb * p.meta_cblocks + (f_kt >> 1)) * 64;
+            mw = __ldg(reinterpret_cast<const uint2*>(blk + 4 * (r & 15) + 2 * (f_kt & 1)));
           }
         }
         if (p.permuted && lane < 16) {
@@ -426,13 +416,9 @@ __global__ void __launch_bounds__(kThreads, 1) spmm_kernel(const __grid_constant
       uint8_t* a_dst = a_base + s * p.a_slot_bytes;
       uint8_t* e_dst = e_base + s * 2048;
       if (p.a_mode == A_TMA_SPARSE) {
-        put_e_word(e_dst, r, 0, mw.x);
-        put_e_word(e_dst, r, 1, mw.y);
+        *reinterpret_cast<uint2*>(e_dst + r * 16) = mw;
       } else if (p.a_mode == A_HYBRID) {
-        if (__ldg(p.tile_map + (int64_t)tm * p.hyb_tiles_k + kt / 2)) {
-          put_e_word(e_dst, r, 0, mw.x);
-          put_e_word(e_dst, r, 1, mw.y);
-        }
+        if (__ldg(p.tile_map + (int64_t)tm * p.hyb_tiles_k + kt / 2)) *reinterpret_cast<uint2*>(e_dst + r * 16) = mw;
       } else if (p.a_mode == A_BUILD_SPARSE) {
         uint32_t vals[16], w0, w1;
         switch (p.pattern) {
@@ -604,15 +590,18 @@ int spmm_max_stages(int bn, uint32_t a_slot) {
   return st;
 }
 
-cudaError_t launch_spmm(SpmmParams& p, int bn, cudaStream_t stream) {
+uint32_t* status_word_ptr() {
   static uint32_t* status_ptr[64] = {};
   int dev = 0;
   cudaGetDevice(&dev);
-  if (dev < 64 && !status_ptr[dev]) {
-    cudaError_t e = cudaGetSymbolAddress(reinterpret_cast<void**>(&status_ptr[dev]), g_status);
-    if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64) dev = 0;
+  if (!status_ptr[dev]) {
+    if (cudaGetSymbolAddress(reinterpret_cast<void**>(&status_ptr[dev]), g_status) != cudaSuccess) return nullptr;
   }
-  p.status = status_ptr[dev < 64 ? dev : 0];
+  return status_ptr[dev];
+}
+
+cudaError_t launch_spmm(SpmmParams& p, int bn, cudaStream_t stream) {
   const int sms = sm_count_current();
   const int grid = p.num_tiles < sms ? p.num_tiles : sms;
   cudaError_t e;

@@ -18,7 +18,8 @@ enum Pattern : int { PAT_2_4 = 0, PAT_1_2 = 1, PAT_1_4 = 2, PAT_1_8 = 3, PAT_2_8
 struct SpmmParams {
   CUtensorMap tm_vals;  // compressed values R x K*n/m, box {32, 128}, 64B swizzle
   CUtensorMap tm_w;     // dense W R x K, box {64, 128}, 128B swizzle (hybrid)
-  CUtensorMap tm_x;     // X K x T, box {strip, 64}
+  CUtensorMap tm_x;     // X K x T, box {strip, 64} (one SM) or {64, 128} (SM pair)
+  CUtensorMap tm_meta;  // tiled 2:4 metadata {64 words, col blocks, row blocks}, box {64, 1, 8} (SM pair)
   const uint16_t* vals;
   const uint32_t* meta;
   const int32_t* idx;
@@ -29,7 +30,8 @@ struct SpmmParams {
   uint32_t* status;
   int64_t ldy;
   int64_t R, K, T;
-  int64_t vcols, mcols;
+  int64_t vcols, mcols;             // mcols: row-wise patterns
+  int64_t meta_rblocks, meta_cblocks; // tiled 2:4 metadata blocks (16 rows x 128 columns)
   int64_t k_tiles;
   int n, m;
   int pattern;
@@ -45,5 +47,8 @@ struct SpmmParams {
 int spmm_max_stages(int bn, uint32_t a_slot);
 cudaError_t launch_spmm(SpmmParams& p, int bn, cudaStream_t stream);
 cudaError_t read_and_clear_status(uint32_t* out);
+uint32_t* status_word_ptr();
+bool pair_kernel_fits(const SpmmParams& p);
+cudaError_t launch_spmm_pair(SpmmParams& p, cudaStream_t stream);
 
 }  // namespace nmk

@@ -1,0 +1,272 @@
+// nm_spmm_pair.cu -- 2:4 sparse x dense GEMM on a pair of SMs (tcgen05 cta_group::2).
+//
+// Same operation as nm_spmm.cu (Y = W' X with W' stored as 2:4 values plus
+// row-wise 2-bit positions; "M:N sparsity on NVIDIA tensor cores", GEMM
+// paragraphs of "Where this sits among the three case studies"), laid out so
+// that the tensor cores of two SMs share one 256 x 256 output tile: each CTA
+// of the cluster stages its own 128 rows of the compressed weights and its own
+// 128 columns of X, and one MMA instruction of the leader CTA consumes both.
+// Per SM this halves the X bytes per useful FLOP compared with a 128 x 256
+// tile on one SM, which is what bounds a 2:4 GEMM: the sparse MMA reads a
+// dense X tile twice as fast as the dense MMA would.
+//
+// Pipeline (per CTA, 4 stages of 128 logical K):
+//   A  compressed values, 128 rows x 64 (16 KB), TMA, 128-byte swizzle
+//   B  X rows k0..k0+127, this CTA's 128 columns (2 x 16 KB), TMA
+//   E  2:4 metadata of the 128 rows (2 KB): eight tiled 16-row blocks, already
+//      in the order tcgen05.cp hands to the tensor core, one 3-D TMA box
+// The A, B and E copies are issued by four different warps (a single issuing
+// thread serialises its copies; several overlap), and none of them waits for
+// anything but a free stage.  All copies of both CTAs complete on the
+// leader's barrier, which expects the bytes of both.  The leader's MMA thread
+// copies E into TMEM (tcgen05.cp, both CTAs) and issues four tcgen05.mma.sp
+// (M = 256, N = 256, K = 32) per stage; its commits release the stage in both
+// CTAs.  Each CTA drains its own 128 x 256 fp32 accumulator.
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include "nm_internal.h"
+#include "nm_ptx.cuh"
+#include "nm_spmm.h"
+
+namespace nmk {
+
+namespace pair {
+constexpr int kThreads = 320;
+constexpr int kStages = 4;
+constexpr uint32_t kA = 16384, kB = 32768, kE = 2048;
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kECol = 256;
+constexpr uint64_t kWaitNs = 2000000000ull;
+constexpr uint32_t kTxPerStage = 2u * (kA + kB + kE);  // both CTAs' A, B and E bytes
+constexpr uint32_t kIdesc = idesc_bf16(256, true, 256);
+
+struct Layout {
+  uint32_t a, b, e, bar, total;
+};
+__host__ __device__ constexpr Layout layout() {
+  return Layout{0u, kStages * kA, kStages * (kA + kB), kStages * (kA + kB + kE),
+                kStages * (kA + kB + kE) + (2 * kStages + 4) * 8 + 64};
+}
+}  // namespace pair
+
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pair::kThreads, 1)
+    spmm_pair_kernel(const __grid_constant__ SpmmParams p) {
+  using namespace pair;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  constexpr Layout L = layout();
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + L.bar);
+  uint64_t* empty = full + kStages;
+  uint64_t* acc_full = empty + kStages;
+  uint64_t* acc_empty = acc_full + 1;
+  uint64_t* spare = acc_empty + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(spare + 2);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const uint32_t rank = cluster_ctarank();  // 0: leader (issues the MMAs), 1: follower
+  const int pair_id = blockIdx.x >> 1;
+  const int npairs = gridDim.x >> 1;
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&full[s], 1);  // the leader's expect_tx; bytes from both CTAs
+      mbar_init(&empty[s], 1);
+    }
+    mbar_init(acc_full, 1);
+    mbar_init(acc_empty, 8);
+    mbar_init(spare, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+    fence_proxy_async_smem();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&p.tm_vals);
+    tma_prefetch_desc(&p.tm_x);
+    tma_prefetch_desc(&p.tm_meta);
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(tmem_slot, kTmemCols);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  const int64_t k_tiles = p.K / 128;
+  const uint32_t lead_full0 = map_to_cta(smem_u32(&full[0]), 0);
+  const uint32_t lead_acc_empty = map_to_cta(smem_u32(acc_empty), 0);
+  bool ok = true;
+
+  if (warp < 6) {
+    if (warp == 1) {
+      // ---------------------------------------------------------- MMA (leader)
+      if (rank == 0 && lane == 0) {
+        int s = 0;
+        uint32_t ph = 0, aph = 0;
+        for (int tile = pair_id; tile < p.num_tiles && ok; tile += npairs) {
+          ok = mbar_wait(acc_empty, aph ^ 1u, abort_flag, p.status, kWaitNs);
+          if (!ok) break;
+          tc_fence_after();
+          for (int64_t kt = 0; kt < k_tiles; ++kt) {
+            ok = mbar_wait(&full[s], ph, abort_flag, p.status, kWaitNs);
+            if (!ok) break;
+            tc_fence_after();
+            const uint32_t a_addr = smem_u32(smem + L.a + s * kA);
+            const uint32_t b_addr = smem_u32(smem + L.b + s * kB);
+            const uint32_t e_tmem = tmem_base + kECol + 4u * s;
+            tc_cp_128x128b_pair(e_tmem, smem_desc(smem_u32(smem + L.e + s * kE), 2048, 128, SWZ_NONE));
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) {
+              const uint64_t ad = smem_desc(a_addr + kk * 32, 16, 1024, SWZ_128B);
+              const uint64_t bd = smem_desc(b_addr + kk * 4096, 16384, 1024, SWZ_128B);
+              tc_mma_sp_pair(tmem_base, ad, bd, e_tmem + (uint32_t)(kk & 2), kIdesc | (uint32_t)(kk & 1),
+                             (kt > 0 || kk > 0) ? 1u : 0u);
+            }
+            tc_commit_pair(&empty[s], 0x3);
+            if (++s == kStages) { s = 0; ph ^= 1u; }
+          }
+          if (!ok) break;
+          tc_commit_pair(acc_full, 0x3);
+          aph ^= 1u;
+        }
+        if (!ok) {
+          tc_commit_pair(spare, 0x1);
+          volatile int dummy = 0;
+          mbar_wait(spare, 0, &dummy, p.status, 100000000ull);
+        }
+      }
+    } else if (warp <= 4) {
+      // ------------------- copy issuers: warp 0 A, warps 2/3 B strips, warp 4 metadata (E)
+      if (lane == 0) {
+        int s = 0;
+        uint32_t ph = 0;
+        for (int tile = pair_id; tile < p.num_tiles && ok; tile += npairs) {
+          const int tm = tile % p.tiles_m, tn = tile / p.tiles_m;
+          const int32_t row0 = tm * 256 + 128 * (int)rank;
+          const int32_t col0 = tn * 256 + 128 * (int)rank;
+          for (int64_t kt = 0; kt < k_tiles; ++kt) {
+            ok = mbar_wait(&empty[s], ph ^ 1u, abort_flag, p.status, kWaitNs);
+            if (!ok) break;
+            const uint32_t lead_full = lead_full0 + 8u * s;
+            if (warp == 0) {
+              if (rank == 0) mbar_arrive_expect_tx(&full[s], kTxPerStage);
+              tma_load_2d_pair(smem + L.a + s * kA, &p.tm_vals, lead_full, (int32_t)(kt * 64), row0);
+            } else if (warp == 2 || warp == 3) {
+              const int j = warp - 2;
+              tma_load_2d_pair(smem + L.b + s * kB + j * 16384, &p.tm_x, lead_full, col0 + 64 * j,
+                               (int32_t)(kt * 128));
+            } else {  // eight 16-row metadata blocks of column block kt
+              tma_load_3d_pair(smem + L.e + s * kE, &p.tm_meta, lead_full, 0, (int32_t)kt, row0 / 16);
+            }
+            if (++s == kStages) { s = 0; ph ^= 1u; }
+          }
+        }
+      }
+    }
+  } else {
+    // -------------------------------------------------------------- epilogue
+    const int quarter = warp & 3;
+    uint32_t aph = 0;
+    for (int tile = pair_id; tile < p.num_tiles && ok; tile += npairs) {
+      const int tm = tile % p.tiles_m, tn = tile / p.tiles_m;
+      const int64_t row = (int64_t)tm * 256 + 128 * rank + quarter * 32 + lane;
+      const int64_t n0 = (int64_t)tn * 256;
+      ok = mbar_wait(acc_full, aph, abort_flag, p.status, kWaitNs);
+      if (!ok) break;
+      tc_fence_after();
+      const uint32_t t_addr = tmem_base + ((uint32_t)(quarter * 32) << 16);
+      const bool row_ok = row < p.R;
+      if (!p.out_f32 && n0 + 256 <= p.T) {
+        uint32_t pk[128];
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          uint32_t v[32];
+          tmem_ld_32x32b_x32(t_addr + c * 32, v);
+          tc_wait_ld();
+#pragma unroll
+          for (int i = 0; i < 16; ++i)
+            pk[c * 16 + i] = pack_bf16x2(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1]));
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_cluster(lead_acc_empty);
+        if (row_ok) {
+          uint4* yrow = reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.Y) + row * p.ldy + n0);
+#pragma unroll
+          for (int c8 = 0; c8 < 32; ++c8)
+            yrow[c8] = make_uint4(pk[4 * c8], pk[4 * c8 + 1], pk[4 * c8 + 2], pk[4 * c8 + 3]);
+        }
+      } else {
+#pragma unroll 1
+        for (int c = 0; c < 16; ++c) {
+          uint32_t v[16];
+          tmem_ld_32x32b_x16(t_addr + c * 16, v);
+          tc_wait_ld();
+          if (!row_ok) continue;
+          const int64_t col0 = n0 + c * 16;
+          if (p.out_f32) {
+            float* yrow = static_cast<float*>(p.Y) + row * p.ldy;
+#pragma unroll
+            for (int e = 0; e < 16; ++e)
+              if (col0 + e < p.T) yrow[col0 + e] = __uint_as_float(v[e]);
+          } else {
+            uint16_t* yrow = static_cast<uint16_t*>(p.Y) + row * p.ldy;
+#pragma unroll
+            for (int e = 0; e < 16; e += 2) {
+              const uint32_t pk = pack_bf16x2(__uint_as_float(v[e]), __uint_as_float(v[e + 1]));
+              if (col0 + e < p.T) yrow[col0 + e] = (uint16_t)(pk & 0xFFFFu);
+              if (col0 + e + 1 < p.T) yrow[col0 + e + 1] = (uint16_t)(pk >> 16);
+            }
+          }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_cluster(lead_acc_empty);
+      }
+      aph ^= 1u;
+    }
+  }
+
+  // -------------------------------------------------------------- teardown
+  __syncthreads();
+  if (*abort_flag && threadIdx.x == 0) {
+    const uint64_t t0 = global_timer_ns();
+    while (global_timer_ns() - t0 < 200000ull) __nanosleep(1000);
+  }
+  cluster_sync();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc_pair(tmem_base, kTmemCols);
+  }
+}
+
+bool pair_kernel_fits(const SpmmParams& p) {
+  return p.a_mode == A_TMA_SPARSE && !p.permuted && p.K % 128 == 0 && p.K > 0 && p.T >= 192 && p.R >= 1;
+}
+
+cudaError_t launch_spmm_pair(SpmmParams& p, cudaStream_t stream) {
+  constexpr pair::Layout L = pair::layout();
+  const size_t bytes = L.total + 1024;
+  static bool configured[64] = {};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 64 && !configured[dev]) {
+    cudaError_t e = cudaFuncSetAttribute(spmm_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+    if (e != cudaSuccess) return e;
+    configured[dev] = true;
+  }
+  const int pairs_avail = sm_count_current() / 2;
+  const int pairs = p.num_tiles < pairs_avail ? p.num_tiles : pairs_avail;
+  spmm_pair_kernel<<<2 * pairs, pair::kThreads, bytes, stream>>>(p);
+  count_launch();
+  return cudaGetLastError();
+}
+
+}  // namespace nmk

@@ -40,15 +40,24 @@ def test_every_declared_symbol_is_exported(lib):
         assert name in nm.SIGNATURES, f"binding lacks a signature for {name}"
 
 
+def test_size_helpers_match_oracle(lib):
+    import oracle
+    for R, K, n, m in [(4096, 11008, 2, 4), (13824, 5120, 2, 4), (6, 24, 2, 4), (3072, 768, 1, 8),
+                       (256, 24, 1, 4), (33, 96, 3, 4), (5, 48, 5, 8)]:
+        assert nm.nm_meta_words(R, K, n, m) == oracle.meta_words(R, K, n, m)
+        assert nm.nm_value_cols(K, n, m) == oracle.value_cols(K, n, m)
+
+
 def test_size_helpers(lib):
     assert nm.nm_index_bits(4) == 2 and nm.nm_index_bits(8) == 3 and nm.nm_index_bits(2) == 1
     assert nm.nm_index_bits(3) == 0
     assert nm.nm_value_cols(4096, 2, 4) == 2048
-    assert nm.nm_meta_cols(4096, 2, 4) == 128
-    assert nm.nm_meta_cols(768, 1, 8) == 10
-    assert nm.nm_meta_cols(24, 2, 4) == 1
-    assert nm.nm_meta_cols(10, 2, 4) == -1      # K % M != 0
-    assert nm.nm_value_cols(16, 4, 4) == -1     # N must be below M
+    assert nm.nm_meta_words(4096, 4096, 2, 4) == 4096 * 4096 // 32   # tiled 2:4
+    assert nm.nm_meta_words(16, 24, 2, 4) == 64                      # one padded block
+    assert nm.nm_meta_words(17, 128, 2, 4) == 128
+    assert nm.nm_meta_words(3, 768, 1, 8) == 30                      # row-wise, 10 words a row
+    assert nm.nm_meta_words(4, 10, 2, 4) == -1     # K % M != 0
+    assert nm.nm_value_cols(16, 4, 4) == -1        # N must be below M
 
 
 def test_host_argument_checks(lib):

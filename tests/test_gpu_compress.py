@@ -20,7 +20,7 @@ def gpu_compress(W_bits, n, m, ldw=None):
         buf[:, :K] = W_bits
         Wd = to_dev(buf)
         vals = torch.empty((R, nm.nm_value_cols(K, n, m)), dtype=torch.bfloat16, device=DEV)
-        meta = torch.empty((R, nm.nm_meta_cols(K, n, m)), dtype=torch.int32, device=DEV)
+        meta = torch.empty((nm.nm_meta_words(R, K, n, m),), dtype=torch.int32, device=DEV)
         nm.nm_prune_compress(Wd, R, K, ldw, n, m, vals, meta)
     else:
         vals, meta = nm.prune_compress(to_dev(W_bits), n, m)
@@ -73,7 +73,8 @@ def test_compress_nonfinite():
 def test_worked_row_on_gpu():
     W = wl.bf16_bits(np.array([[1.5, 0, 0, -2.0, 0, 0.25, 3.0, 0] * 4], np.float32))
     _, mt = gpu_compress(W, 2, 4)
-    assert int(mt[0, 0]) == 0x9C9C9C9C
+    # row 0, columns 0..15 -> word 0 low half; columns 16..31 -> word 0 of lane 8 (word 32)
+    assert int(mt[0]) == 0x44449C9C and int(mt[32]) == 0x44449C9C
 
 
 @pytest.mark.parametrize("n,m", PATTERNS)
@@ -108,6 +109,6 @@ def test_compress_full_size_1of8(R, K):
 def test_empty_shapes():
     W = torch.empty((0, 64), dtype=torch.bfloat16, device=DEV)
     v, mt = nm.prune_compress(W, 2, 4)
-    assert v.shape == (0, 32) and mt.shape == (0, 2)
+    assert v.shape == (0, 32) and mt.shape == (0,)
     with pytest.raises(nm.NmError):
         nm.prune_compress(torch.zeros((4, 10), dtype=torch.bfloat16, device=DEV), 2, 4)

@@ -275,3 +275,26 @@ def test_patch_full_size_sampled():
                                  with_abs=True)
     i = np.arange(rows.shape[0])
     assert_gemm_close(values_f64(Y)[rows, cols], ref[i, i], mag[i, i], "patch sampled")
+
+
+# ----------------------------------------------------------------------------
+# Shapes served by the two-SM (256 x 256 tile) kernel: 2:4, K % 128 == 0, T >= 192
+# ----------------------------------------------------------------------------
+@pytest.mark.parametrize("R,K,T", [(600, 1024, 520), (256, 4096, 256), (1000, 384, 200), (130, 256, 1000)])
+def test_pair_kernel_ragged(R, K, T):
+    W = wl.normal_bf16((R, K), 0.02, seed=R * 3 + K)
+    X = wl.normal_bf16((K, T), 1.0, seed=T * 5)
+    check(W, X, 2, 4, what=f"pair {R}x{K}x{T}")
+
+
+@pytest.mark.parametrize("out", [torch.bfloat16, torch.float32])
+def test_pair_kernel_integer_exact(out):
+    R, K, T = 512, 512, 384
+    W = wl.integer_bf16((R, K), -8, 8, seed=111)
+    X = wl.integer_bf16((K, T), -8, 8, seed=112)
+    ref, _ = reference(W, X, 2, 4)
+    Y = run_spmm(W, X, 2, 4, out_dtype=out)
+    if out == torch.float32:
+        assert np.array_equal(Y.cpu().numpy().astype(np.float64), ref)
+    else:
+        assert np.array_equal(bits(Y), bf16_rne_of(ref))

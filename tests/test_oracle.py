@@ -28,10 +28,9 @@ def bits_of(values):
     return wl.bf16_bits(np.asarray(values, dtype=np.float32))
 
 
-def positions(meta_row, count, m):
-    b = oracle.index_bits(m)
-    s = oracle.positions_per_word(m)
-    return [int((int(meta_row[j // s]) >> (b * (j % s))) & ((1 << b) - 1)) for j in range(count)]
+def positions(meta, R, K, n, m):
+    """Survivor positions read back from the packed metadata (list of rows)."""
+    return oracle.positions(meta, R, K, n, m).astype(int).tolist()
 
 
 # ---------------------------------------------------------------------------
@@ -43,10 +42,12 @@ def test_worked_row(golden_dir, v):
     row = [v if c == "v" else 0.0 for c in g["row_template"]]
     W = bits_of([row])
     vals, meta = oracle.compress(W, 2, 4)
-    pos = positions(meta[0], 4, 4)
+    pos = positions(meta, 1, 8, 2, 4)[0]
     assert [pos[0:2], pos[2:4]] == g["metadata"]
-    assert int(meta[0, 0]) & 0xFF == g["packed_low_byte"]
-    assert int(meta[0, 0]) >> 8 == 0
+    assert int(meta[0]) & 0xFF == g["packed_low_byte"]
+    # the rest of the tile is padding: all-zero groups, positions (0,1), nibble 0x4
+    assert int(meta[0]) >> 8 == 0x444444
+    assert np.all(meta[1:] == 0x44444444)
     assert np.array_equal(vals[0], bits_of([v, v, v, v]))
 
 
@@ -96,7 +97,7 @@ def test_exhaustive_alphabet(n, m, alphabet):
     groups = np.array(list(itertools.product(alphabet, repeat=m)), dtype=np.float32)
     W = bits_of(groups.reshape(1, -1))
     vals, meta = oracle.compress(W, n, m)
-    pos = positions(meta[0], groups.shape[0] * n, m)
+    pos = positions(meta, 1, W.shape[1], n, m)[0]
     for gi, grp in enumerate(groups):
         want = _stable_sort_select([float(x) for x in grp], n)
         assert pos[gi * n:(gi + 1) * n] == want
@@ -137,11 +138,32 @@ def test_storage_36_bits(golden_dir):
     assert 100 * (1 - (2 * 8 + 2 * 2) / (4 * 8)) == g["int8_saving_percent"]
 
 
-@pytest.mark.parametrize("K,n,m,words", [(128, 2, 4, 4), (24, 2, 4, 1), (24, 1, 8, 1), (768, 1, 8, 10),
-                                         (256, 1, 4, 4), (4096, 2, 4, 128), (11008, 2, 4, 344)])
-def test_meta_sizes(K, n, m, words):
-    assert oracle.meta_cols(K, n, m) == words
+@pytest.mark.parametrize("R,K,n,m,words", [(16, 128, 2, 4, 64), (16, 24, 2, 4, 64), (17, 128, 2, 4, 128),
+                                           (1, 24, 1, 8, 1), (1, 768, 1, 8, 10), (1, 256, 1, 4, 4),
+                                           (4096, 4096, 2, 4, 4096 * 4096 // 32),
+                                           (11008, 4096, 2, 4, 11008 * 4096 // 32), (3, 768, 1, 8, 30)])
+def test_meta_sizes(R, K, n, m, words):
+    assert oracle.meta_words(R, K, n, m) == words
     assert oracle.value_cols(K, n, m) == K * n // m
+
+
+def test_tiled_2of4_every_group_once():
+    """Each group's nibble sits in its own slot; everything else is the padding nibble."""
+    R, K = 21, 200                       # padded to 32 rows x 256 columns
+    W = wl.normal_bf16((R, K), 1.0, seed=12)
+    _, meta = oracle.compress(W, 2, 4)
+    assert meta.size == 2 * 2 * 64
+    nibbles = (meta[:, None] >> (4 * np.arange(8))) & 0xF
+    real = nibbles[nibbles != 0x4]
+    # valid 2:4 position pairs only, and no more non-padding nibbles than groups
+    assert set(np.unique(real).tolist()) <= {0x8, 0xC, 0x9, 0xD, 0xE}
+    assert real.size <= R * K // 4
+    # the padded rows 21..31 and columns 200..255 decode as positions (0,1)
+    wide = np.zeros((32, 256), np.uint16)
+    wide[:R, :K] = W
+    _, meta_wide = oracle.compress(wide, 2, 4)
+    pos_wide = oracle.positions(meta_wide, 32, 256, 2, 4)
+    assert np.all(pos_wide[R:] == np.tile([0, 1], 64))
 
 
 # ---------------------------------------------------------------------------
@@ -168,7 +190,7 @@ def test_k8_example(golden_dir):
     vals, meta = oracle.compress(W, 2, 4)
     assert vals.shape[1] == g["sparse_products"] and W.shape[1] == g["dense_products"]
     assert np.array_equal(f64(vals[0]), np.array(g["expected_values"]))
-    pos = positions(meta[0], 4, 4)
+    pos = positions(meta, 1, 8, 2, 4)[0]
     assert [pos[0:2], pos[2:4]] == g["expected_positions"]
     X = bits_of(np.array(g["b_col"], dtype=np.float32).reshape(8, 1))
     y = oracle.spmm(vals, meta, 2, 4, 8, X)
