@@ -234,19 +234,38 @@ static nm_status run_gemm(const GemmRequest& q, cudaStream_t stream) {
 
   // Two SMs per 256 x 256 tile when the shape allows it (2:4 from TMA, K % 128 == 0).
   if (q.algo != NM_ALGO_DENSE_TC && pair_kernel_fits(p) && al16(q.meta)) {
+    // With an index map, one gather pass stages Xp[k] = X[idx[k]] in a
+    // stream-ordered buffer and the pair kernel streams Xp with TMA boxes.
+    const uint16_t* xsrc = q.X;
+    int64_t ldsrc = q.ldx;
+    void* staged = nullptr;
+    if (p.permuted) {
+      const int64_t ldp = (q.T + 7) / 8 * 8;
+      cudaError_t e = cudaMallocAsync(&staged, (size_t)(q.K * ldp * 2), stream);
+      if (e != cudaSuccess) return cuda_fail(e, "staging buffer for the permuted input");
+      e = launch_gather_rows(q.X, q.ldx, q.idx, q.K, q.T, static_cast<uint16_t*>(staged), ldp, stream);
+      if (e != cudaSuccess) {
+        cudaFreeAsync(staged, stream);
+        return cuda_fail(e, "gather launch");
+      }
+      xsrc = static_cast<const uint16_t*>(staged);
+      ldsrc = ldp;
+      p.permuted = 0;
+    }
     p.tiles_m = (int)((q.R + 255) / 256);
     p.tiles_n = (int)((q.T + 255) / 256);
     if ((int64_t)p.tiles_m * p.tiles_n >= (1ll << 31)) return fail(NM_ERR_UNSUPPORTED, "too many tiles");
     p.num_tiles = p.tiles_m * p.tiles_n;
     p.k_tiles = q.K / 128;
-    st = make_tmap(&p.tm_x, q.X, (uint64_t)q.T, (uint64_t)q.K, (uint64_t)q.ldx * 2, 64, 128, 128, "X");
+    st = make_tmap(&p.tm_x, xsrc, (uint64_t)q.T, (uint64_t)q.K, (uint64_t)ldsrc * 2, 64, 128, 128, "X");
+    if (st == NM_OK)
+      st = make_tmap(&p.tm_vals, q.values, (uint64_t)p.vcols, (uint64_t)q.R, (uint64_t)p.vcols * 2, 64, 128, 128,
+                     "values");
+    if (st == NM_OK) st = make_meta_tmap(&p.tm_meta, q.meta, p.meta_rblocks, p.meta_cblocks);
+    cudaError_t e = cudaSuccess;
+    if (st == NM_OK) e = launch_spmm_pair(p, stream);
+    if (staged) cudaFreeAsync(staged, stream);
     if (st != NM_OK) return st;
-    st = make_tmap(&p.tm_vals, q.values, (uint64_t)p.vcols, (uint64_t)q.R, (uint64_t)p.vcols * 2, 64, 128, 128,
-                   "values");
-    if (st != NM_OK) return st;
-    st = make_meta_tmap(&p.tm_meta, q.meta, p.meta_rblocks, p.meta_cblocks);
-    if (st != NM_OK) return st;
-    cudaError_t e = launch_spmm_pair(p, stream);
     return e == cudaSuccess ? NM_OK : cuda_fail(e, "spmm pair launch");
   }
 

@@ -252,6 +252,38 @@ __global__ void fill_zero_kernel(uint8_t* Y, int64_t R, int64_t row_bytes, int64
   }
 }
 
+// Row gather Xp[k][0..T) = X[idx[k]][0..T): one warp per row, 16-byte pieces,
+// all of a lane's pieces loaded before any is stored.  Entries of idx outside
+// [0, K) give zero rows.  X and Xp rows are 16-byte aligned (T % 8 == 0 on
+// the vector path).
+__global__ void __launch_bounds__(256) gather_rows_kernel(const uint16_t* __restrict__ X, int64_t ldx,
+                                                          const int32_t* __restrict__ idx, int64_t K, int64_t T,
+                                                          uint16_t* __restrict__ Xp, int64_t ldp) {
+  const int lane = threadIdx.x & 31;
+  const int64_t warp = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) >> 5;
+  const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
+  const int64_t pieces = T >> 3;  // 16-byte pieces per row
+  for (int64_t k = warp; k < K; k += nwarps) {
+    const int32_t src = __ldg(idx + k);
+    const bool valid = src >= 0 && (int64_t)src < K;
+    const uint4* in = reinterpret_cast<const uint4*>(X + (valid ? (int64_t)src : 0) * ldx);
+    uint4* out = reinterpret_cast<uint4*>(Xp + k * ldp);
+    for (int64_t c0 = 0; c0 < pieces; c0 += 32 * 8) {
+      uint4 v[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int64_t c = c0 + u * 32 + lane;
+        v[u] = (valid && c < pieces) ? __ldg(in + c) : make_uint4(0, 0, 0, 0);
+      }
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int64_t c = c0 + u * 32 + lane;
+        if (c < pieces) out[c] = v[u];
+      }
+    }
+  }
+}
+
 static int grid_for(int64_t work, int threads) {
   const int64_t want = (work + threads - 1) / threads;
   const int64_t cap = (int64_t)sm_count_current() * 16;
@@ -300,6 +332,14 @@ cudaError_t launch_decompress(const uint16_t* values, const uint32_t* meta, int6
       default: decompress_generic_kernel<16><<<grid, threads, 0, s>>>(values, meta, R, K, n, W_out, ldw); break;
     }
   }
+  count_launch();
+  return cudaGetLastError();
+}
+
+cudaError_t launch_gather_rows(const uint16_t* X, int64_t ldx, const int32_t* idx, int64_t K, int64_t T,
+                               uint16_t* Xp, int64_t ldp, cudaStream_t s) {
+  const int threads = 256;
+  gather_rows_kernel<<<grid_for(K * 32, threads), threads, 0, s>>>(X, ldx, idx, K, T, Xp, ldp);
   count_launch();
   return cudaGetLastError();
 }

@@ -35,6 +35,8 @@ cudaError_t launch_compress(const uint16_t* W, int64_t R, int64_t K, int64_t ldw
                             uint32_t* meta, cudaStream_t s);
 cudaError_t launch_decompress(const uint16_t* values, const uint32_t* meta, int64_t R, int64_t K, int n, int m,
                               uint16_t* W_out, int64_t ldw, cudaStream_t s);
+cudaError_t launch_gather_rows(const uint16_t* X, int64_t ldx, const int32_t* idx, int64_t K, int64_t T,
+                               uint16_t* Xp, int64_t ldp, cudaStream_t s);
 cudaError_t launch_fill_zero(void* Y, int64_t R, int64_t T, int64_t ldy, int esize, cudaStream_t s);
 
 }  // namespace nmk

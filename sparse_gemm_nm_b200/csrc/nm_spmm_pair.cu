@@ -248,7 +248,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pair::kThreads, 1)
 }
 
 bool pair_kernel_fits(const SpmmParams& p) {
-  return p.a_mode == A_TMA_SPARSE && !p.permuted && p.K % 128 == 0 && p.K > 0 && p.T >= 192 && p.R >= 1;
+  return p.a_mode == A_TMA_SPARSE && p.K % 128 == 0 && p.K > 0 && p.T >= 192 && p.R >= 1 && p.T % 8 == 0;
 }
 
 cudaError_t launch_spmm_pair(SpmmParams& p, cudaStream_t stream) {
