@@ -182,6 +182,32 @@ NM_API nm_status nm_spmm_algo(const uint16_t* values, const uint32_t* meta, int 
                        const int32_t* idx, const uint16_t* X, int64_t ldx, int64_t T, void* Y, int64_t ldy,
                        nm_out_dtype y_dtype, nm_algo algo, void* stream);
 
+/*
+ * nm_spmm_permuted_noalloc -- nm_spmm_permuted without any device allocation.
+ * The pages have no counterpart to this call; it exists for callers that
+ * cannot let a library allocate device memory: runtimes that budget every
+ * byte up front, processes whose memory pool belongs to another allocator, or
+ * loops that cannot afford a pool that has to grow.  nm_spmm_permuted stages
+ * the gathered input X[idx[k]] in a buffer taken from the device's memory pool
+ * on `stream`; this call stages it instead in a fixed 32 MiB array inside the
+ * library, which every device that loads the library holds until the process
+ * exits, and works through the columns of X in chunks that fit it.  Results
+ * match nm_spmm_permuted.  Arguments and errors as nm_spmm_permuted, plus:
+ *  - NM_ERR_UNSUPPORTED when K > 65536 on the two-SM path (a 256-column chunk
+ *    of K rows must fit the array);
+ *  - the first call on each device looks up the array's device address
+ *    (cudaGetSymbolAddress); make that first call before any stream capture;
+ *  - all calls share the one array and each leaves its last chunk in it: calls
+ *    that may overlap on the GPU (different streams, or other host threads)
+ *    race and must be serialised by the caller.  Nothing in the array needs to
+ *    start at zero: each chunk writes every element it later reads.
+ * Shapes that the two-SM path does not take (not 2:4, K % 128 != 0, T < 192,
+ * T % 8 != 0) stage nothing and run exactly as nm_spmm_permuted.
+ */
+NM_API nm_status nm_spmm_permuted_noalloc(const uint16_t* values, const uint32_t* meta, int n, int m, int64_t R,
+                                          int64_t K, const int32_t* idx, const uint16_t* X, int64_t ldx, int64_t T,
+                                          void* Y, int64_t ldy, nm_out_dtype y_dtype, void* stream);
+
 /* ------------------------------------------------------------ utilities */
 /* Synchronises `stream`, then returns NM_ERR_TIMEOUT if any kernel of this
  * library recorded a bounded wait that gave up since the previous call (and

@@ -49,6 +49,7 @@ SIGNATURES = {
     "nm_spmm_permuted": ([_P, _P, _I, _I, _I64, _I64, _P, _P, _I64, _I64, _P, _I64, _I, _P], _I),
     "nm_hybrid_spmm": ([_P, _I64, _P, _P, _P, _I, _I64, _I64, _P, _I64, _I64, _P, _I64, _I, _P], _I),
     "nm_spmm_algo": ([_P, _P, _I, _I, _I64, _I64, _P, _P, _I64, _I64, _P, _I64, _I, _I, _P], _I),
+    "nm_spmm_permuted_noalloc": ([_P, _P, _I, _I, _I64, _I64, _P, _P, _I64, _I64, _P, _I64, _I, _P], _I),
     "nm_device_status": ([_P], _I),
     "nm_status_string": ([_I], ctypes.c_char_p),
     "nm_last_error": ([], ctypes.c_char_p),
@@ -156,6 +157,12 @@ def nm_spmm_algo(values, meta, n, m, R, K, idx, X, ldx, T, Y, ldy, y_dtype=NM_OU
                  stream=None) -> None:
     _check(lib().nm_spmm_algo(_ptr(values), _ptr(meta), n, m, R, K, _ptr(idx), _ptr(X), ldx, T, _ptr(Y), ldy,
                               y_dtype, algo, _stream(stream)), "nm_spmm_algo")
+
+
+def nm_spmm_permuted_noalloc(values, meta, n, m, R, K, idx, X, ldx, T, Y, ldy, y_dtype=NM_OUT_BF16,
+                             stream=None) -> None:
+    _check(lib().nm_spmm_permuted_noalloc(_ptr(values), _ptr(meta), n, m, R, K, _ptr(idx), _ptr(X), ldx, T,
+                                          _ptr(Y), ldy, y_dtype, _stream(stream)), "nm_spmm_permuted_noalloc")
 
 
 def nm_device_status(stream=None) -> None:

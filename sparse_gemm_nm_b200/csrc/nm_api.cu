@@ -294,6 +294,54 @@ static nm_status run_gemm(const GemmRequest& q, cudaStream_t stream) {
   return e == cudaSuccess ? NM_OK : cuda_fail(e, "spmm launch");
 }
 
+// ---- helpers for entry points defined in other files (additive) ----
+void set_last_error(const char* msg) { t_last_error = msg ? msg : ""; }
+
+bool pair_path_for(int n, int m, int64_t R, int64_t K, int64_t T, const void* values, const void* meta) {
+  SpmmParams p;
+  std::memset(&p, 0, sizeof p);
+  p.a_mode = (n == 2 && m == 4 && K % 16 == 0 && al16(values)) ? A_TMA_SPARSE : A_BUILD_SPARSE;
+  p.R = R;
+  p.K = K;
+  p.T = T;
+  return pair_kernel_fits(p) && al16(meta);
+}
+
+nm_status build_pair_params(SpmmParams& p, const uint16_t* values, const uint32_t* meta, int64_t R, int64_t K,
+                            const uint16_t* X, int64_t ldx, int64_t T, void* Y, int64_t ldy, bool out_f32) {
+  std::memset(&p, 0, sizeof p);
+  p.vals = values;
+  p.meta = meta;
+  p.X = X;
+  p.ldx = ldx;
+  p.Y = Y;
+  p.ldy = ldy;
+  p.R = R;
+  p.K = K;
+  p.T = T;
+  p.n = 2;
+  p.m = 4;
+  p.vcols = value_cols(K, 2, 4);
+  p.mcols = meta_cols(K, 2, 4);
+  p.meta_rblocks = meta_row_blocks(R);
+  p.meta_cblocks = meta_col_blocks(K);
+  p.pattern = PAT_2_4;
+  p.a_mode = A_TMA_SPARSE;
+  p.out_f32 = out_f32 ? 1 : 0;
+  p.status = status_word_ptr();
+  if (!p.status) return fail(NM_ERR_CUDA, "device status word is unavailable");
+  p.tiles_m = (int)((R + 255) / 256);
+  p.tiles_n = (int)((T + 255) / 256);
+  p.num_tiles = p.tiles_m * p.tiles_n;
+  p.k_tiles = K / 128;
+  nm_status st = make_tmap(&p.tm_x, X, (uint64_t)T, (uint64_t)K, (uint64_t)ldx * 2, 64, 128, 128, "X");
+  if (st == NM_OK)
+    st = make_tmap(&p.tm_vals, values, (uint64_t)p.vcols, (uint64_t)R, (uint64_t)p.vcols * 2, 64, 128, 128,
+                   "values");
+  if (st == NM_OK) st = make_meta_tmap(&p.tm_meta, meta, p.meta_rblocks, p.meta_cblocks);
+  return st;
+}
+
 }  // namespace nmk
 
 using namespace nmk;
