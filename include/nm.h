@@ -27,11 +27,13 @@
  *              (b = ceil(log2 M) bits) in word r*ceil(K*N/M/S) + floor(j/S) at
  *              bit b*(j mod S), S = floor(32/b); unused bits 0.
  *  - Every pointer is DEVICE memory owned by the caller (none is freed or
- *    retained).  The library allocates no device memory on these paths.
+ *    retained).  The library allocates no device memory, except the staging
+ *    buffer of nm_spmm_permuted (see there).
  *  - Calls are asynchronous on `stream` (a cudaStream_t; NULL = the legacy
  *    default stream).  Argument errors are detected on the host and returned
- *    before anything is launched.  Each successful call launches exactly one
- *    kernel (none when the output is empty).
+ *    before anything is launched.  Each successful call launches one kernel
+ *    (none when the output is empty), except nm_spmm_permuted on the two-SM
+ *    path, which launches two.
  *  - Device pointers given to the GEMMs must be 16-byte aligned, and leading
  *    dimensions of X and Y must keep every row 16-byte aligned
  *    (NM_ERR_MISALIGNED otherwise).
@@ -140,9 +142,19 @@ NM_API nm_status nm_spmm(const uint16_t* values, const uint32_t* meta, int n, in
 /*
  * nm_spmm_permuted -- Y = (W' Pi) X with the hard column permutation Pi given
  * as an index map: row k of the permuted input is X[idx[k]], so
- * y[r][t] = sum_k W'[r][k] * X[idx[k]][t].  The kernel reads X at the mapped
- * rows while staging its tiles; there is no separate permute pass and the
- * FLOP count is that of nm_spmm.  An identity map gives nm_spmm's result.
+ * y[r][t] = sum_k W'[r][k] * X[idx[k]][t].  The FLOP count is that of
+ * nm_spmm, and an identity map gives nm_spmm's result.  How X is read:
+ *  - 2:4 weights with K % 128 == 0, T >= 192 and T % 8 == 0 (the two-SM
+ *    path): a gather pass first writes Xp[k] = X[idx[k]] into a staging
+ *    buffer of K x ceil8(T) bf16, which the GEMM then streams like X.  The
+ *    buffer comes from a stream-ordered pool that the library owns (one per
+ *    device) and goes back to it, on `stream`, when the call's kernels are
+ *    done; the pool keeps its memory for later calls (high-water mark: the
+ *    largest K x ceil8(T) x 2 bytes, times the calls in flight on different
+ *    streams) until nm_release_staging().  A failed allocation returns
+ *    NM_ERR_CUDA.
+ *  - every other shape: the GEMM kernel reads the mapped rows of X while it
+ *    stages its tiles; there is no separate pass and no allocation.
  * Source: "Technische Samenvatting: SHUFFLESPARSE", section "2. Methodologie"
  * (y = (W Pi) x; at inference Pi is a precomputed index map and the structured
  * sparse GEMM reads its input at the permuted addresses).
@@ -183,13 +195,22 @@ NM_API nm_status nm_spmm_algo(const uint16_t* values, const uint32_t* meta, int 
                        nm_out_dtype y_dtype, nm_algo algo, void* stream);
 
 /*
+ * nm_release_staging -- return the memory that nm_spmm_permuted's staging pools
+ * keep reserved (all devices) to the driver.  Memory still in use by calls
+ * in flight stays reserved.  The pages have no counterpart to this
+ * call; it exists because the pool deliberately keeps its memory between calls.
+ * Errors: NM_ERR_CUDA.
+ */
+NM_API nm_status nm_release_staging(void);
+
+/*
  * nm_spmm_permuted_noalloc -- nm_spmm_permuted without any device allocation.
  * The pages have no counterpart to this call; it exists for callers that
  * cannot let a library allocate device memory: runtimes that budget every
  * byte up front, processes whose memory pool belongs to another allocator, or
  * loops that cannot afford a pool that has to grow.  nm_spmm_permuted stages
- * the gathered input X[idx[k]] in a buffer taken from the device's memory pool
- * on `stream`; this call stages it instead in a fixed 32 MiB array inside the
+ * the gathered input X[idx[k]] in a buffer taken from a library-owned memory
+ * pool on `stream`; this call stages it instead in a fixed 32 MiB array inside the
  * library, which every device that loads the library holds until the process
  * exits, and works through the columns of X in chunks that fit it.  Results
  * match nm_spmm_permuted.  Arguments and errors as nm_spmm_permuted, plus:

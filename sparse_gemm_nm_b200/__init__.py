@@ -50,6 +50,7 @@ SIGNATURES = {
     "nm_hybrid_spmm": ([_P, _I64, _P, _P, _P, _I, _I64, _I64, _P, _I64, _I64, _P, _I64, _I, _P], _I),
     "nm_spmm_algo": ([_P, _P, _I, _I, _I64, _I64, _P, _P, _I64, _I64, _P, _I64, _I, _I, _P], _I),
     "nm_spmm_permuted_noalloc": ([_P, _P, _I, _I, _I64, _I64, _P, _P, _I64, _I64, _P, _I64, _I, _P], _I),
+    "nm_release_staging": ([], _I),
     "nm_device_status": ([_P], _I),
     "nm_status_string": ([_I], ctypes.c_char_p),
     "nm_last_error": ([], ctypes.c_char_p),
@@ -163,6 +164,10 @@ def nm_spmm_permuted_noalloc(values, meta, n, m, R, K, idx, X, ldx, T, Y, ldy, y
                              stream=None) -> None:
     _check(lib().nm_spmm_permuted_noalloc(_ptr(values), _ptr(meta), n, m, R, K, _ptr(idx), _ptr(X), ldx, T,
                                           _ptr(Y), ldy, y_dtype, _stream(stream)), "nm_spmm_permuted_noalloc")
+
+
+def nm_release_staging() -> None:
+    _check(lib().nm_release_staging(), "nm_release_staging")
 
 
 def nm_device_status(stream=None) -> None:

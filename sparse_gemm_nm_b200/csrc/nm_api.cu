@@ -89,6 +89,40 @@ static EncodeTiledFn encode_fn() {
   return fn;
 }
 
+// Library-owned stream-ordered pool for the permuted GEMM's staging buffers,
+// one per device.  Its release threshold is "never", so memory returned by
+// cudaFreeAsync stays reserved for the next call instead of going back to the
+// driver at each synchronisation: re-mapping tens of MB on every call costs
+// far more than the GEMM.  nm_release_staging() hands the memory back.
+static std::mutex g_pool_mu;
+static cudaMemPool_t g_pool[64];
+
+static cudaError_t staging_pool(cudaMemPool_t* out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lk(g_pool_mu);
+  if (!g_pool[dev]) {
+    cudaMemPoolProps props = {};
+    props.allocType = cudaMemAllocationTypePinned;
+    props.location.type = cudaMemLocationTypeDevice;
+    props.location.id = dev;
+    cudaMemPool_t pool = nullptr;
+    e = cudaMemPoolCreate(&pool, &props);
+    if (e != cudaSuccess) return e;
+    uint64_t keep = ~0ull;
+    e = cudaMemPoolSetAttribute(pool, cudaMemPoolAttrReleaseThreshold, &keep);
+    if (e != cudaSuccess) {
+      cudaMemPoolDestroy(pool);
+      return e;
+    }
+    g_pool[dev] = pool;
+  }
+  *out = g_pool[dev];
+  return cudaSuccess;
+}
+
 static nm_status make_tmap(CUtensorMap* tm, const void* base, uint64_t inner, uint64_t outer,
                            uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer, int swizzle_bytes,
                            const char* what, CUtensorMapDataType dtype = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16) {
@@ -235,13 +269,17 @@ static nm_status run_gemm(const GemmRequest& q, cudaStream_t stream) {
   // Two SMs per 256 x 256 tile when the shape allows it (2:4 from TMA, K % 128 == 0).
   if (q.algo != NM_ALGO_DENSE_TC && pair_kernel_fits(p) && al16(q.meta)) {
     // With an index map, one gather pass stages Xp[k] = X[idx[k]] in a
-    // stream-ordered buffer and the pair kernel streams Xp with TMA boxes.
+    // stream-ordered buffer from the staging pool and the pair kernel streams
+    // Xp with TMA boxes.
     const uint16_t* xsrc = q.X;
     int64_t ldsrc = q.ldx;
     void* staged = nullptr;
     if (p.permuted) {
       const int64_t ldp = (q.T + 7) / 8 * 8;
-      cudaError_t e = cudaMallocAsync(&staged, (size_t)(q.K * ldp * 2), stream);
+      cudaMemPool_t pool = nullptr;
+      cudaError_t e = staging_pool(&pool);
+      if (e != cudaSuccess) return cuda_fail(e, "staging pool");
+      e = cudaMallocFromPoolAsync(&staged, (size_t)(q.K * ldp * 2), pool, stream);
       if (e != cudaSuccess) return cuda_fail(e, "staging buffer for the permuted input");
       e = launch_gather_rows(q.X, q.ldx, q.idx, q.K, q.T, static_cast<uint16_t*>(staged), ldp, stream);
       if (e != cudaSuccess) {
@@ -257,9 +295,9 @@ static nm_status run_gemm(const GemmRequest& q, cudaStream_t stream) {
     if ((int64_t)p.tiles_m * p.tiles_n >= (1ll << 31)) return fail(NM_ERR_UNSUPPORTED, "too many tiles");
     p.num_tiles = p.tiles_m * p.tiles_n;
     p.k_tiles = q.K / 128;
-    st = make_tmap(&p.tm_x, xsrc, (uint64_t)q.T, (uint64_t)q.K, (uint64_t)ldsrc * 2, 64, 128, 128, "X");
+    st = make_tmap(&p.tm_x, xsrc, (uint64_t)q.T, (uint64_t)q.K, (uint64_t)ldsrc * 2, 64, kPairBoxRows, 128, "X");
     if (st == NM_OK)
-      st = make_tmap(&p.tm_vals, q.values, (uint64_t)p.vcols, (uint64_t)q.R, (uint64_t)p.vcols * 2, 64, 128, 128,
+      st = make_tmap(&p.tm_vals, q.values, (uint64_t)p.vcols, (uint64_t)q.R, (uint64_t)p.vcols * 2, 64, kPairBoxRows, 128,
                      "values");
     if (st == NM_OK) st = make_meta_tmap(&p.tm_meta, q.meta, p.meta_rblocks, p.meta_cblocks);
     cudaError_t e = cudaSuccess;
@@ -334,9 +372,9 @@ nm_status build_pair_params(SpmmParams& p, const uint16_t* values, const uint32_
   p.tiles_n = (int)((T + 255) / 256);
   p.num_tiles = p.tiles_m * p.tiles_n;
   p.k_tiles = K / 128;
-  nm_status st = make_tmap(&p.tm_x, X, (uint64_t)T, (uint64_t)K, (uint64_t)ldx * 2, 64, 128, 128, "X");
+  nm_status st = make_tmap(&p.tm_x, X, (uint64_t)T, (uint64_t)K, (uint64_t)ldx * 2, 64, kPairBoxRows, 128, "X");
   if (st == NM_OK)
-    st = make_tmap(&p.tm_vals, values, (uint64_t)p.vcols, (uint64_t)R, (uint64_t)p.vcols * 2, 64, 128, 128,
+    st = make_tmap(&p.tm_vals, values, (uint64_t)p.vcols, (uint64_t)R, (uint64_t)p.vcols * 2, 64, kPairBoxRows, 128,
                    "values");
   if (st == NM_OK) st = make_meta_tmap(&p.tm_meta, meta, p.meta_rblocks, p.meta_cblocks);
   return st;
@@ -483,5 +521,16 @@ const char* nm_last_error(void) { return t_last_error.c_str(); }
 uint64_t nm_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
 
 int nm_version(void) { return 100; }
+
+nm_status nm_release_staging(void) {
+  set_last_error("");
+  std::lock_guard<std::mutex> lk(g_pool_mu);
+  for (int d = 0; d < 64; ++d) {
+    if (!g_pool[d]) continue;
+    cudaError_t e = cudaMemPoolTrimTo(g_pool[d], 0);
+    if (e != cudaSuccess) return cuda_fail(e, "trimming the staging pool");
+  }
+  return NM_OK;
+}
 
 }  // extern "C"

@@ -24,87 +24,109 @@ __device__ __forceinline__ uint32_t mag_key(uint32_t bits16) {
   return k > 0x7F80u ? 0x7F81u : k;
 }
 
-// One group of four (e[0..3] as 16-bit patterns) -> 2:4 nibble (p0 | p1 << 2)
-// and the two survivors packed lo | hi << 16.
-__device__ __forceinline__ void select_2of4(uint32_t e0, uint32_t e1, uint32_t e2, uint32_t e3, uint32_t& nib,
-                                            uint32_t& packed) {
-  // Composite keys are distinct: magnitude first, then the lower index.
-  const uint32_t c0 = (mag_key(e0) << 2) | 3u, c1 = (mag_key(e1) << 2) | 2u;
-  const uint32_t c2 = (mag_key(e2) << 2) | 1u, c3 = (mag_key(e3) << 2) | 0u;
-  const uint32_t r0 = (c1 > c0) + (c2 > c0) + (c3 > c0);
-  const uint32_t r1 = (c0 > c1) + (c2 > c1) + (c3 > c1);
-  const uint32_t r2 = (c0 > c2) + (c1 > c2) + (c3 > c2);
-  const uint32_t r3 = (c0 > c3) + (c1 > c3) + (c2 > c3);
-  const uint32_t keep = (r0 < 2u) | ((r1 < 2u) << 1) | ((r2 < 2u) << 2) | ((r3 < 2u) << 3);
-  const uint32_t p0 = __ffs(keep) - 1u;
-  const uint32_t p1 = 31u - __clz(keep);
-  nib = p0 | (p1 << 2);
-  const uint32_t v0 = p0 == 0 ? e0 : p0 == 1 ? e1 : e2;  // p0 <= 2
-  const uint32_t v1 = p1 == 3 ? e3 : p1 == 2 ? e2 : e1;  // p1 >= 1
-  packed = v0 | (v1 << 16);
+// 2:4 with tiled metadata.  One warp per metadata block (16 rows x 128
+// columns): lane i takes row 16*rb + i/2, columns 128*cb + 64*(i%2) .. +63
+// (sixteen groups), so every 16-byte load of the warp covers 16 rows x 32
+// bytes.  The lane selects its sixteen groups, stores its 32 survivors
+// (64 contiguous bytes) and keeps the sixteen nibbles; the block's 64 words
+// are then assembled with shuffles, 2 per lane.
+//
+// Selection of one group (keys k_i = bf16 magnitude field, NaNs folded just
+// above +Inf): with s_ij = (k_i >= k_j) for i < j, element i beats j iff
+// s_ij, and j beats i iff !s_ij (equal keys go to the lower index).  An
+// element survives iff it beats at least two of the other three, a 3-input
+// majority.
+__device__ __forceinline__ uint32_t maj3(uint32_t a, uint32_t b, uint32_t c) { return (a & b) | (a & c) | (b & c); }
+
+// Nibble p0 | p1 << 2 for each of the six 2-of-4 keep masks (others unused).
+__device__ __forceinline__ uint32_t nibble_of_keep(uint32_t kb) {
+  constexpr uint64_t lut = (0x4ull << (4 * 3)) | (0x8ull << (4 * 5)) | (0x9ull << (4 * 6)) | (0xCull << (4 * 9)) |
+                           (0xDull << (4 * 10)) | (0xEull << (4 * 12));
+  return (uint32_t)(lut >> (4 * kb)) & 0xFu;
 }
 
-// 2:4 with tiled metadata.  One thread per metadata word: word 4*l + q of
-// block (rb, cb) holds, for K columns k0 = 128*cb + 32*q + 16*(l/8) .. k0+15,
-// the four nibbles of row 16*rb + (l%8) in bits 0..15 and of that row + 8 in
-// bits 16..31.  The thread reads those 2 x 16 weights, selects, writes the
-// 2 x 8 survivors and the word.  Rows or columns past R or K (block padding)
-// get the nibble of an all-zero group, positions (0,1), and write no values.
-__device__ __forceinline__ uint32_t compress_half16(const uint16_t* __restrict__ wrow, uint16_t* __restrict__ vrow,
-                                                    uint32_t k0, uint32_t K, bool vec) {
-  uint32_t e[16];
-  if (vec && k0 + 16 <= K) {
-    const uint4 a = __ldg(reinterpret_cast<const uint4*>(wrow + k0));
-    const uint4 b = __ldg(reinterpret_cast<const uint4*>(wrow + k0 + 8));
-    const uint32_t w8[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      e[2 * i] = w8[i] & 0xFFFFu;
-      e[2 * i + 1] = w8[i] >> 16;
-    }
-  } else {
-#pragma unroll
-    for (int i = 0; i < 16; ++i) e[i] = (k0 + i < K) ? (uint32_t)wrow[k0 + i] : 0u;
-  }
-  uint32_t nibs = 0, pk[4];
-#pragma unroll
-  for (int t = 0; t < 4; ++t) {
-    uint32_t nib;
-    select_2of4(e[4 * t], e[4 * t + 1], e[4 * t + 2], e[4 * t + 3], nib, pk[t]);
-    nibs |= (k0 + 4 * t < K ? nib : 0x4u) << (4 * t);
-  }
-  if (vec && k0 + 16 <= K) {
-    *reinterpret_cast<uint4*>(vrow + k0 / 2) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-  } else {
-#pragma unroll
-    for (int t = 0; t < 4; ++t)
-      if (k0 + 4 * t < K) *reinterpret_cast<uint32_t*>(vrow + k0 / 2 + 2 * t) = pk[t];
-  }
-  return nibs;
+// Group of four in (lo, hi) = (e0 | e1 << 16, e2 | e3 << 16): returns the
+// nibble, and in `pk` the two survivors (first in the low half).
+__device__ __forceinline__ uint32_t select_pair(uint32_t lo, uint32_t hi, uint32_t& pk) {
+  const uint32_t k0 = min(lo & 0x7FFFu, 0x7F81u), k1 = min((lo >> 16) & 0x7FFFu, 0x7F81u);
+  const uint32_t k2 = min(hi & 0x7FFFu, 0x7F81u), k3 = min((hi >> 16) & 0x7FFFu, 0x7F81u);
+  const uint32_t s01 = k0 >= k1, s02 = k0 >= k2, s03 = k0 >= k3;
+  const uint32_t s12 = k1 >= k2, s13 = k1 >= k3, s23 = k2 >= k3;
+  const uint32_t keep = maj3(s01, s02, s03) | (maj3(s01 ^ 1u, s12, s13) << 1) | (maj3(s02 ^ 1u, s12 ^ 1u, s23) << 2) |
+                        (maj3(s03 ^ 1u, s13 ^ 1u, s23 ^ 1u) << 3);
+  const uint32_t nib = nibble_of_keep(keep);
+  const uint32_t p0 = nib & 3u, p1 = nib >> 2;
+  pk = __byte_perm(lo, hi, 0x1010u + p0 * 0x22u + p1 * 0x2200u);
+  return nib;
 }
 
 __global__ void __launch_bounds__(256) compress_2of4_tiled_kernel(const uint16_t* __restrict__ W, uint32_t R,
                                                                   uint32_t K, int64_t ldw,
                                                                   uint16_t* __restrict__ V,
                                                                   uint32_t* __restrict__ meta, uint32_t cblocks,
-                                                                  uint32_t total, bool vec) {
-  for (uint32_t w = blockIdx.x * blockDim.x + threadIdx.x; w < total; w += gridDim.x * blockDim.x) {
-    const uint32_t blk = w >> 6, wi = w & 63u;
-    const uint32_t l = wi >> 2, q = wi & 3u;
+                                                                  uint32_t nblocks, bool vec) {
+  const uint32_t lane = threadIdx.x & 31u;
+  const uint32_t warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const uint32_t nwarps = (gridDim.x * blockDim.x) >> 5;
+  for (uint32_t blk = warp; blk < nblocks; blk += nwarps) {
     const uint32_t rb = blk / cblocks, cb = blk - rb * cblocks;
-    const uint32_t r_lo = rb * 16 + (l & 7u);
-    const uint32_t k0 = cb * 128 + q * 32 + (l >> 3) * 16;
-    uint32_t word = 0x44444444u;
-    if (k0 < K) {
-      if (r_lo < R)
-        word = (word & 0xFFFF0000u) |
-               compress_half16(W + (int64_t)r_lo * ldw, V + (int64_t)r_lo * (K >> 1), k0, K, vec);
-      if (r_lo + 8 < R)
-        word = (word & 0x0000FFFFu) |
-               (compress_half16(W + (int64_t)(r_lo + 8) * ldw, V + (int64_t)(r_lo + 8) * (K >> 1), k0, K, vec)
-                << 16);
+    const uint32_t r = rb * 16 + (lane >> 1);
+    const uint32_t c0 = cb * 128 + (lane & 1u) * 64;  // first of this lane's 64 columns
+    uint32_t nib_lo = 0x44444444u, nib_hi = 0x44444444u;  // groups 0..7, 8..15
+    if (r < R && c0 < K) {
+      const uint16_t* wrow = W + (int64_t)r * ldw + c0;
+      uint32_t* vrow = reinterpret_cast<uint32_t*>(V + (int64_t)r * (K >> 1) + c0 / 2);
+      if (vec && c0 + 64 <= K) {
+        uint4 in[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) in[i] = __ldg(reinterpret_cast<const uint4*>(wrow) + i);
+        uint32_t pk[16];
+        uint32_t n0 = 0, n1 = 0;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const uint32_t a = select_pair(in[i].x, in[i].y, pk[2 * i]);
+          const uint32_t b = select_pair(in[i].z, in[i].w, pk[2 * i + 1]);
+          const uint32_t two = a | (b << 4);
+          if (i < 4) n0 |= two << (8 * i);
+          else n1 |= two << (8 * (i - 4));
+        }
+        nib_lo = n0;
+        nib_hi = n1;
+        uint4* vout = reinterpret_cast<uint4*>(vrow);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) vout[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+      } else {
+        uint32_t n0 = 0, n1 = 0;
+        for (int g = 0; g < 16; ++g) {
+          const uint32_t cg = c0 + 4 * g;
+          uint32_t nib = 0x4u;
+          if (cg < K) {
+            const uint32_t lo = (uint32_t)wrow[4 * g] | ((uint32_t)wrow[4 * g + 1] << 16);
+            const uint32_t hi = (uint32_t)wrow[4 * g + 2] | ((uint32_t)wrow[4 * g + 3] << 16);
+            uint32_t pk;
+            nib = select_pair(lo, hi, pk);
+            vrow[g] = pk;
+          }
+          if (g < 8) n0 |= nib << (4 * g);
+          else n1 |= nib << (4 * (g - 8));
+        }
+        nib_lo = n0;
+        nib_hi = n1;
+      }
     }
-    meta[w] = word;
+    // Words 2L, 2L+1 of the block: lane l = L/2 of the tile (row l%8 and row
+    // 8 + l%8), quarters q = 2*(L%2) and 2*(L%2)+1, K half h = l/8.  Their
+    // 16-bit halves live in lanes 2*(l%8) + L%2 (low row) and 2*(l%8 + 8) +
+    // L%2 (high row), in 16-bit chunk h of nib_lo (q even) and nib_hi (q odd).
+    const uint32_t l = lane >> 1, rr = l & 7u, h = l >> 3;
+    const uint32_t src_lo = 2 * rr + (lane & 1u), src_hi = 2 * (rr + 8) + (lane & 1u);
+    const uint32_t a_lo = __shfl_sync(0xffffffffu, nib_lo, src_lo);
+    const uint32_t a_hi = __shfl_sync(0xffffffffu, nib_hi, src_lo);
+    const uint32_t b_lo = __shfl_sync(0xffffffffu, nib_lo, src_hi);
+    const uint32_t b_hi = __shfl_sync(0xffffffffu, nib_hi, src_hi);
+    const uint32_t w0 = ((a_lo >> (16 * h)) & 0xFFFFu) | (((b_lo >> (16 * h)) & 0xFFFFu) << 16);
+    const uint32_t w1 = ((a_hi >> (16 * h)) & 0xFFFFu) | (((b_hi >> (16 * h)) & 0xFFFFu) << 16);
+    *reinterpret_cast<uint2*>(meta + (int64_t)blk * 64 + 2 * lane) = make_uint2(w0, w1);
   }
 }
 
@@ -296,10 +318,10 @@ cudaError_t launch_compress(const uint16_t* W, int64_t R, int64_t K, int64_t ldw
                             uint32_t* meta, cudaStream_t s) {
   const int threads = 256;
   if (tiled_meta(n, m)) {
-    const int64_t total = meta_words(R, K, n, m);
+    const int64_t nblocks = meta_row_blocks(R) * meta_col_blocks(K);
     const bool vec = K % 16 == 0 && ldw % 8 == 0 && aligned16(W) && aligned16(values);
-    compress_2of4_tiled_kernel<<<grid_for(total, threads), threads, 0, s>>>(
-        W, (uint32_t)R, (uint32_t)K, ldw, values, meta, (uint32_t)meta_col_blocks(K), (uint32_t)total, vec);
+    compress_2of4_tiled_kernel<<<grid_for(nblocks * 32, threads), threads, 0, s>>>(
+        W, (uint32_t)R, (uint32_t)K, ldw, values, meta, (uint32_t)meta_col_blocks(K), (uint32_t)nblocks, vec);
   } else {
     const int64_t work = R * meta_cols(K, n, m);
     const int grid = grid_for(work, threads);

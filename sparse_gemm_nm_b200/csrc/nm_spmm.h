@@ -13,12 +13,16 @@ enum AMode : int {
   A_HYBRID = 3         // per 128x128 tile: dense W by TMA, or 2:4 values by TMA
 };
 
+// Height of the A and B boxes of the SM-pair kernel: each stage's 128 rows
+// of values and 128 rows of X arrive as 64-row boxes from separate warps.
+constexpr uint32_t kPairBoxRows = 64;
+
 enum Pattern : int { PAT_2_4 = 0, PAT_1_2 = 1, PAT_1_4 = 2, PAT_1_8 = 3, PAT_2_8 = 4, PAT_OTHER = 5 };
 
 struct SpmmParams {
-  CUtensorMap tm_vals;  // compressed values R x K*n/m, box {32, 128}, 64B swizzle
+  CUtensorMap tm_vals;  // compressed values R x K*n/m, box {32, 128} 64B swizzle (one SM) or {64, kPairBoxRows} 128B (SM pair)
   CUtensorMap tm_w;     // dense W R x K, box {64, 128}, 128B swizzle (hybrid)
-  CUtensorMap tm_x;     // X K x T, box {strip, 64} (one SM) or {64, 128} (SM pair)
+  CUtensorMap tm_x;     // X K x T, box {strip, 64} (one SM) or {64, kPairBoxRows} (SM pair)
   CUtensorMap tm_meta;  // tiled 2:4 metadata {64 words, col blocks, row blocks}, box {64, 1, 8} (SM pair)
   const uint16_t* vals;
   const uint32_t* meta;

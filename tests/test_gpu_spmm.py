@@ -298,3 +298,19 @@ def test_pair_kernel_integer_exact(out):
         assert np.array_equal(Y.cpu().numpy().astype(np.float64), ref)
     else:
         assert np.array_equal(bits(Y), bf16_rne_of(ref))
+
+
+def test_permuted_pair_path_after_release_staging():
+    """The two-SM permuted path stages Xp in a library pool; handing the pool's
+    memory back between calls must not change the result."""
+    R, K, T = 512, 1024, 512
+    W = wl.normal_bf16((R, K), 0.02, seed=121)
+    X = wl.normal_bf16((K, T), 1.0, seed=122)
+    idx = wl.permutation(K, 123)
+    first = run_spmm(W, X, 2, 4, idx=idx)
+    nm.nm_release_staging()
+    second = run_spmm(W, X, 2, 4, idx=idx)
+    nm.nm_release_staging()
+    assert torch.equal(first, second)
+    ref, mag = reference(W, X, 2, 4, idx)
+    assert_gemm_close(values_f64(second), ref, mag, "permuted after release")
