@@ -25,39 +25,38 @@ __device__ __forceinline__ uint32_t mag_key(uint32_t bits16) {
 }
 
 // 2:4 with tiled metadata.  One warp per metadata block (16 rows x 128
-// columns): lane i takes row 16*rb + i/2, columns 128*cb + 64*(i%2) .. +63
-// (sixteen groups), so every 16-byte load of the warp covers 16 rows x 32
-// bytes.  The lane selects its sixteen groups, stores its 32 survivors
-// (64 contiguous bytes) and keeps the sixteen nibbles; the block's 64 words
-// are then assembled with shuffles, 2 per lane.
+// columns).  Load i (0..7) of the warp reads rows 2i and 2i+1 of the block,
+// 256 contiguous bytes each: lane l takes row 2i + l/16 and the eight
+// columns 8*(l%16) .. +7 (two groups).  So a lane holds the same two groups of
+// eight rows, every load and every value store of the warp covers whole
+// 128-byte lines, and each lane keeps one byte of nibbles per row (rows
+// 2k + l/16: k = 0..3 in `lo8`, k = 4..7 in `hi8`).  The block's 64 words are
+// assembled with shuffles, two per lane.
 //
-// Selection of one group (keys k_i = bf16 magnitude field, NaNs folded just
-// above +Inf): with s_ij = (k_i >= k_j) for i < j, element i beats j iff
-// s_ij, and j beats i iff !s_ij (equal keys go to the lower index).  An
-// element survives iff it beats at least two of the other three, a 3-input
-// majority.
-__device__ __forceinline__ uint32_t maj3(uint32_t a, uint32_t b, uint32_t c) { return (a & b) | (a & c) | (b & c); }
-
-// Nibble p0 | p1 << 2 for each of the six 2-of-4 keep masks (others unused).
-__device__ __forceinline__ uint32_t nibble_of_keep(uint32_t kb) {
-  constexpr uint64_t lut = (0x4ull << (4 * 3)) | (0x8ull << (4 * 5)) | (0x9ull << (4 * 6)) | (0xCull << (4 * 9)) |
-                           (0xDull << (4 * 10)) | (0xEull << (4 * 12));
-  return (uint32_t)(lut >> (4 * kb)) & 0xFu;
+// Selection of one group.  Composite keys c_i = (magnitude field of e_i) * 4
+// + (3 - i), NaNs folded to one key just above +Inf: all four are distinct,
+// and a larger key means a larger magnitude or, on equal magnitudes, a lower
+// index.  The two largest keys come from a four-input network (max/min of
+// each pair, then the larger maximum and the larger of the smaller maximum and
+// the larger minimum); their low bits give the positions.
+__device__ __forceinline__ uint32_t ckey(uint32_t shifted_by2, uint32_t tie) {
+  return min((shifted_by2 & 0x1FFFCu) | tie, 0x1FE04u | tie);  // 0x1FE04 = (0x7F81 << 2)
 }
 
 // Group of four in (lo, hi) = (e0 | e1 << 16, e2 | e3 << 16): returns the
-// nibble, and in `pk` the two survivors (first in the low half).
+// nibble p0 | p1 << 2 (p0 < p1), and in `pk` the two survivors (first in the
+// low half).
 __device__ __forceinline__ uint32_t select_pair(uint32_t lo, uint32_t hi, uint32_t& pk) {
-  const uint32_t k0 = min(lo & 0x7FFFu, 0x7F81u), k1 = min((lo >> 16) & 0x7FFFu, 0x7F81u);
-  const uint32_t k2 = min(hi & 0x7FFFu, 0x7F81u), k3 = min((hi >> 16) & 0x7FFFu, 0x7F81u);
-  const uint32_t s01 = k0 >= k1, s02 = k0 >= k2, s03 = k0 >= k3;
-  const uint32_t s12 = k1 >= k2, s13 = k1 >= k3, s23 = k2 >= k3;
-  const uint32_t keep = maj3(s01, s02, s03) | (maj3(s01 ^ 1u, s12, s13) << 1) | (maj3(s02 ^ 1u, s12 ^ 1u, s23) << 2) |
-                        (maj3(s03 ^ 1u, s13 ^ 1u, s23 ^ 1u) << 3);
-  const uint32_t nib = nibble_of_keep(keep);
-  const uint32_t p0 = nib & 3u, p1 = nib >> 2;
+  const uint32_t c0 = ckey(lo << 2, 3u), c1 = ckey(lo >> 14, 2u);
+  const uint32_t c2 = ckey(hi << 2, 1u), c3 = ckey(hi >> 14, 0u);
+  const uint32_t m01 = max(c0, c1), n01 = min(c0, c1);
+  const uint32_t m23 = max(c2, c3), n23 = min(c2, c3);
+  const uint32_t top = max(m01, m23);
+  const uint32_t second = max(min(m01, m23), max(n01, n23));
+  const uint32_t pa = (top & 3u) ^ 3u, pb = (second & 3u) ^ 3u;
+  const uint32_t p0 = min(pa, pb), p1 = max(pa, pb);
   pk = __byte_perm(lo, hi, 0x1010u + p0 * 0x22u + p1 * 0x2200u);
-  return nib;
+  return p0 | (p1 << 2);
 }
 
 __global__ void __launch_bounds__(256) compress_2of4_tiled_kernel(const uint16_t* __restrict__ W, uint32_t R,
@@ -68,64 +67,68 @@ __global__ void __launch_bounds__(256) compress_2of4_tiled_kernel(const uint16_t
   const uint32_t lane = threadIdx.x & 31u;
   const uint32_t warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const uint32_t nwarps = (gridDim.x * blockDim.x) >> 5;
+  const uint32_t half = lane >> 4, piece = lane & 15u;
   for (uint32_t blk = warp; blk < nblocks; blk += nwarps) {
     const uint32_t rb = blk / cblocks, cb = blk - rb * cblocks;
-    const uint32_t r = rb * 16 + (lane >> 1);
-    const uint32_t c0 = cb * 128 + (lane & 1u) * 64;  // first of this lane's 64 columns
-    uint32_t nib_lo = 0x44444444u, nib_hi = 0x44444444u;  // groups 0..7, 8..15
-    if (r < R && c0 < K) {
-      const uint16_t* wrow = W + (int64_t)r * ldw + c0;
-      uint32_t* vrow = reinterpret_cast<uint32_t*>(V + (int64_t)r * (K >> 1) + c0 / 2);
-      if (vec && c0 + 64 <= K) {
-        uint4 in[8];
+    const uint32_t col = cb * 128 + 8 * piece;  // this lane's first column
+    uint32_t lo8 = 0x44444444u, hi8 = 0x44444444u;
+    if (vec) {  // K % 8 == 0: a piece is wholly inside or wholly outside
+      uint4 in[8];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) in[i] = __ldg(reinterpret_cast<const uint4*>(wrow) + i);
-        uint32_t pk[16];
-        uint32_t n0 = 0, n1 = 0;
+      for (int i = 0; i < 8; ++i) {
+        const uint32_t row = rb * 16 + 2 * i + half;
+        if (row < R && col < K) in[i] = __ldg(reinterpret_cast<const uint4*>(W + (int64_t)row * ldw + col));
+      }
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          const uint32_t a = select_pair(in[i].x, in[i].y, pk[2 * i]);
-          const uint32_t b = select_pair(in[i].z, in[i].w, pk[2 * i + 1]);
-          const uint32_t two = a | (b << 4);
-          if (i < 4) n0 |= two << (8 * i);
-          else n1 |= two << (8 * (i - 4));
+      for (int i = 0; i < 8; ++i) {
+        const uint32_t row = rb * 16 + 2 * i + half;
+        uint32_t byte = 0x44u;
+        if (row < R && col < K) {
+          uint32_t v0, v1;
+          byte = select_pair(in[i].x, in[i].y, v0) | (select_pair(in[i].z, in[i].w, v1) << 4);
+          *reinterpret_cast<uint2*>(V + (int64_t)row * (K >> 1) + col / 2) = make_uint2(v0, v1);
         }
-        nib_lo = n0;
-        nib_hi = n1;
-        uint4* vout = reinterpret_cast<uint4*>(vrow);
+        if (i < 4) lo8 = (lo8 & ~(0xFFu << (8 * i))) | (byte << (8 * i));
+        else hi8 = (hi8 & ~(0xFFu << (8 * (i - 4)))) | (byte << (8 * (i - 4)));
+      }
+    } else {
+      for (int i = 0; i < 8; ++i) {
+        const uint32_t row = rb * 16 + 2 * i + half;
+        uint32_t byte = 0x44u;
+        if (row < R) {
+          const uint16_t* wrow = W + (int64_t)row * ldw;
+          uint32_t* vrow = reinterpret_cast<uint32_t*>(V + (int64_t)row * (K >> 1));
 #pragma unroll
-        for (int i = 0; i < 4; ++i) vout[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
-      } else {
-        uint32_t n0 = 0, n1 = 0;
-        for (int g = 0; g < 16; ++g) {
-          const uint32_t cg = c0 + 4 * g;
-          uint32_t nib = 0x4u;
-          if (cg < K) {
-            const uint32_t lo = (uint32_t)wrow[4 * g] | ((uint32_t)wrow[4 * g + 1] << 16);
-            const uint32_t hi = (uint32_t)wrow[4 * g + 2] | ((uint32_t)wrow[4 * g + 3] << 16);
-            uint32_t pk;
-            nib = select_pair(lo, hi, pk);
-            vrow[g] = pk;
+          for (int g = 0; g < 2; ++g) {
+            const uint32_t cg = col + 4 * g;
+            if (cg < K) {
+              const uint32_t lo = (uint32_t)wrow[cg] | ((uint32_t)wrow[cg + 1] << 16);
+              const uint32_t hi = (uint32_t)wrow[cg + 2] | ((uint32_t)wrow[cg + 3] << 16);
+              uint32_t pk;
+              const uint32_t nib = select_pair(lo, hi, pk);
+              vrow[cg / 4] = pk;  // value column cg / 2
+              byte = (byte & ~(0xFu << (4 * g))) | (nib << (4 * g));
+            }
           }
-          if (g < 8) n0 |= nib << (4 * g);
-          else n1 |= nib << (4 * (g - 8));
         }
-        nib_lo = n0;
-        nib_hi = n1;
+        if (i < 4) lo8 = (lo8 & ~(0xFFu << (8 * i))) | (byte << (8 * i));
+        else hi8 = (hi8 & ~(0xFFu << (8 * (i - 4)))) | (byte << (8 * (i - 4)));
       }
     }
-    // Words 2L, 2L+1 of the block: lane l = L/2 of the tile (row l%8 and row
-    // 8 + l%8), quarters q = 2*(L%2) and 2*(L%2)+1, K half h = l/8.  Their
-    // 16-bit halves live in lanes 2*(l%8) + L%2 (low row) and 2*(l%8 + 8) +
-    // L%2 (high row), in 16-bit chunk h of nib_lo (q even) and nib_hi (q odd).
-    const uint32_t l = lane >> 1, rr = l & 7u, h = l >> 3;
-    const uint32_t src_lo = 2 * rr + (lane & 1u), src_hi = 2 * (rr + 8) + (lane & 1u);
-    const uint32_t a_lo = __shfl_sync(0xffffffffu, nib_lo, src_lo);
-    const uint32_t a_hi = __shfl_sync(0xffffffffu, nib_hi, src_lo);
-    const uint32_t b_lo = __shfl_sync(0xffffffffu, nib_lo, src_hi);
-    const uint32_t b_hi = __shfl_sync(0xffffffffu, nib_hi, src_hi);
-    const uint32_t w0 = ((a_lo >> (16 * h)) & 0xFFFFu) | (((b_lo >> (16 * h)) & 0xFFFFu) << 16);
-    const uint32_t w1 = ((a_hi >> (16 * h)) & 0xFFFFu) | (((b_hi >> (16 * h)) & 0xFFFFu) << 16);
+    // Words 2L (quarter q = 2*(L%2)) and 2L+1 (q + 1) of tile lane l = L/2:
+    // row r = l%8 (low half) and 8 + r (high half), column half h = l/8.
+    // The nibble byte of (row r, piece p) sits in lane 16*(r%2) + p, byte
+    // r/2 of lo8 (low row) or hi8 (high row); quarter q takes pieces
+    // 4q + 2h and 4q + 2h + 1.
+    const uint32_t l = lane >> 1, r = l & 7u, h = l >> 3, k = r >> 1;
+    const uint32_t s0 = 16 * (r & 1u) + 8 * (lane & 1u) + 2 * h;  // source lane of quarter q's first piece
+    const uint32_t a0 = __shfl_sync(0xffffffffu, lo8, s0), a1 = __shfl_sync(0xffffffffu, lo8, s0 + 1);
+    const uint32_t b0 = __shfl_sync(0xffffffffu, hi8, s0), b1 = __shfl_sync(0xffffffffu, hi8, s0 + 1);
+    const uint32_t c0 = __shfl_sync(0xffffffffu, lo8, s0 + 4), c1 = __shfl_sync(0xffffffffu, lo8, s0 + 5);
+    const uint32_t d0 = __shfl_sync(0xffffffffu, hi8, s0 + 4), d1 = __shfl_sync(0xffffffffu, hi8, s0 + 5);
+    const uint32_t pick = k | ((k + 4) << 4);  // byte k of the first operand, then byte k of the second
+    const uint32_t w0 = __byte_perm(__byte_perm(a0, a1, pick), __byte_perm(b0, b1, pick), 0x5410u);
+    const uint32_t w1 = __byte_perm(__byte_perm(c0, c1, pick), __byte_perm(d0, d1, pick), 0x5410u);
     *reinterpret_cast<uint2*>(meta + (int64_t)blk * 64 + 2 * lane) = make_uint2(w0, w1);
   }
 }
@@ -319,7 +322,7 @@ cudaError_t launch_compress(const uint16_t* W, int64_t R, int64_t K, int64_t ldw
   const int threads = 256;
   if (tiled_meta(n, m)) {
     const int64_t nblocks = meta_row_blocks(R) * meta_col_blocks(K);
-    const bool vec = K % 16 == 0 && ldw % 8 == 0 && aligned16(W) && aligned16(values);
+    const bool vec = K % 8 == 0 && ldw % 8 == 0 && aligned16(W) && aligned16(values);
     compress_2of4_tiled_kernel<<<grid_for(nblocks * 32, threads), threads, 0, s>>>(
         W, (uint32_t)R, (uint32_t)K, ldw, values, meta, (uint32_t)meta_col_blocks(K), (uint32_t)nblocks, vec);
   } else {
