@@ -59,7 +59,7 @@ __device__ __forceinline__ uint32_t select_pair(uint32_t lo, uint32_t hi, uint32
   return p0 | (p1 << 2);
 }
 
-__global__ void __launch_bounds__(256) compress_2of4_tiled_kernel(const uint16_t* __restrict__ W, uint32_t R,
+__global__ void __launch_bounds__(256, 4) compress_2of4_tiled_kernel(const uint16_t* __restrict__ W, uint32_t R,
                                                                   uint32_t K, int64_t ldw,
                                                                   uint16_t* __restrict__ V,
                                                                   uint32_t* __restrict__ meta, uint32_t cblocks,
