@@ -362,11 +362,16 @@ def run_ours(args, rank: int, world: int, dist):
     bytes_all = sum(b["gemm_bytes"] for b in bufs)
     gsec = gemm_ms.sum() * 1e-3
     tensor_bound = flops_all / (tc_peak * 1e12) >= bytes_all / (hbm_peak * 1e9)
+    # DRAM bytes (read + write) of the GEMM call's kernels per layer, from one ncu capture
+    # (profiles/<workload>_gemm_traffic.json); summed over the step like `achieved`.
     traffic = None
     tfile = os.path.join(ROOT, "profiles", f"{args.workload}_gemm_traffic.json")
-    if os.path.exists(tfile):
+    if os.path.exists(tfile) and args.algo == "auto":
         with open(tfile) as f:
-            traffic = json.load(f).get("bytes_per_launch")
+            per = json.load(f).get("bytes_per_launch", {})
+        names = [f"{b['L'].R}x{b['L'].K}" for b in bufs]
+        if all(n in per for n in names):
+            traffic = sum(sum(per[n].get(k, 0) for k in ("spmm_pair_kernel", "gather_rows_kernel")) for n in names)
     if tensor_bound:
         achieved, peak, unit = flops_all / gsec / 1e12, tc_peak, "TFLOP/s"
         src = (f"{peak_src} bf16 {'sustained' if sustained else 'burst'} dense peak; useful 2:4 FLOPs run at "
@@ -375,7 +380,8 @@ def run_ours(args, rank: int, world: int, dist):
         achieved, peak, unit = bytes_all / gsec / 1e9, hbm_peak, "GB/s"
         src = f"{peak_src} HBM copy bandwidth"
     roofline = {"bound": "tensor" if tensor_bound else "hbm", "achieved": achieved, "peak": peak, "unit": unit,
-                "frac": achieved / peak, "traffic": traffic, "kernel": "spmm_kernel (tcgen05 GEMM)",
+                "frac": achieved / peak, "traffic": traffic,
+                "kernel": "nm_spmm_permuted call: gather_rows_kernel + spmm_pair_kernel (tcgen05 2-SM GEMM)",
                 "peak_source": src,
                 "algorithmic_per_launch": [b["flops"] if tensor_bound else b["gemm_bytes"] for b in bufs]}
 
