@@ -28,12 +28,13 @@
  *              bit b*(j mod S), S = floor(32/b); unused bits 0.
  *  - Every pointer is DEVICE memory owned by the caller (none is freed or
  *    retained).  The library allocates no device memory, except the staging
- *    buffer of nm_spmm_permuted (see there).
+ *    buffers of the GEMM calls on the two-SM path (see nm_spmm and
+ *    nm_spmm_permuted).
  *  - Calls are asynchronous on `stream` (a cudaStream_t; NULL = the legacy
  *    default stream).  Argument errors are detected on the host and returned
  *    before anything is launched.  Each successful call launches one kernel
- *    (none when the output is empty), except nm_spmm_permuted on the two-SM
- *    path, which launches two.
+ *    (none when the output is empty), except the GEMM calls that stage an
+ *    operand first (a re-encoding and/or a gather pass; see nm_spmm).
  *  - Device pointers given to the GEMMs must be 16-byte aligned, and leading
  *    dimensions of X and Y must keep every row 16-byte aligned
  *    (NM_ERR_MISALIGNED otherwise).
@@ -133,6 +134,13 @@ NM_API nm_status nm_decompress(const uint16_t* values, const uint32_t* meta, int
  *   values, meta [in] compressed R x K weights, pattern n:m
  *   X            [in] K x T bf16, row stride ldx >= T, ldx % 8 == 0
  *   Y            [out] R x T, bf16 or fp32 (y_dtype), row stride ldy >= T
+ * Kernel choice: shapes with K % 128 == 0, T >= 192 and T % 8 == 0 run on two
+ * SMs per 256 x 256 tile.  2:4 reads the caller's operand directly.  1:2, 1:4,
+ * 1:8 and 2:8 (at most two survivors per aligned group of four) are first
+ * re-encoded as 2:4 into a staging buffer (R*K bytes of values plus R*K/8
+ * bytes of metadata) from the library's pool (see nm_spmm_permuted and
+ * nm_release_staging), one extra launch.  Every other case runs on one SM per
+ * 128-row tile and stages nothing.
  * Errors: NM_ERR_INVALID_ARG, NM_ERR_MISALIGNED, NM_ERR_CUDA.
  */
 NM_API nm_status nm_spmm(const uint16_t* values, const uint32_t* meta, int n, int m, int64_t R, int64_t K,
@@ -144,14 +152,15 @@ NM_API nm_status nm_spmm(const uint16_t* values, const uint32_t* meta, int n, in
  * as an index map: row k of the permuted input is X[idx[k]], so
  * y[r][t] = sum_k W'[r][k] * X[idx[k]][t].  The FLOP count is that of
  * nm_spmm, and an identity map gives nm_spmm's result.  How X is read:
- *  - 2:4 weights with K % 128 == 0, T >= 192 and T % 8 == 0 (the two-SM
- *    path): a gather pass first writes Xp[k] = X[idx[k]] into a staging
- *    buffer of K x ceil8(T) bf16, which the GEMM then streams like X.  The
+ *  - the two-SM path (see nm_spmm): a gather pass first writes
+ *    Xp[k] = X[idx[k]] into a staging buffer of K x ceil8(T) bf16, which the
+ *    GEMM then streams like X.  The
  *    buffer comes from a stream-ordered pool that the library owns (one per
  *    device) and goes back to it, on `stream`, when the call's kernels are
  *    done; the pool keeps its memory for later calls (high-water mark: the
- *    largest K x ceil8(T) x 2 bytes, times the calls in flight on different
- *    streams) until nm_release_staging().  A failed allocation returns
+ *    largest staged bytes of one call, K x ceil8(T) x 2 plus a re-encoded
+ *    operand if any, times the calls in flight on different streams) until
+ *    nm_release_staging().  A failed allocation returns
  *    NM_ERR_CUDA.
  *  - every other shape: the GEMM kernel reads the mapped rows of X while it
  *    stages its tiles; there is no separate pass and no allocation.
@@ -222,8 +231,10 @@ NM_API nm_status nm_release_staging(void);
  *    that may overlap on the GPU (different streams, or other host threads)
  *    race and must be serialised by the caller.  Nothing in the array needs to
  *    start at zero: each chunk writes every element it later reads.
- * Shapes that the two-SM path does not take (not 2:4, K % 128 != 0, T < 192,
- * T % 8 != 0) stage nothing and run exactly as nm_spmm_permuted.
+ * Every other case (patterns other than 2:4, K % 128 != 0, T < 192,
+ * T % 8 != 0) runs on the one-SM kernel, which reads the mapped rows of X
+ * itself and stages nothing (patterns other than 2:4 are not re-encoded
+ * here, unlike nm_spmm_permuted).
  */
 NM_API nm_status nm_spmm_permuted_noalloc(const uint16_t* values, const uint32_t* meta, int n, int m, int64_t R,
                                           int64_t K, const int32_t* idx, const uint16_t* X, int64_t ldx, int64_t T,

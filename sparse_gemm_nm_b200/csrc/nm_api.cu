@@ -192,6 +192,9 @@ struct GemmRequest {
   int64_t ldw;
   const uint8_t* tile_map;
   int tile;
+  // false: never stage anything (no re-encoded operand); used by the
+  // allocation-free entry point for shapes it does not chunk itself
+  bool allow_staging = true;
 };
 
 static nm_status run_gemm(const GemmRequest& q, cudaStream_t stream) {
@@ -267,23 +270,66 @@ static nm_status run_gemm(const GemmRequest& q, cudaStream_t stream) {
   if (!p.status) return fail(NM_ERR_CUDA, "device status word is unavailable");
 
   // Two SMs per 256 x 256 tile when the shape allows it (2:4 from TMA, K % 128 == 0).
-  if (q.algo != NM_ALGO_DENSE_TC && pair_kernel_fits(p) && al16(q.meta)) {
+  // Other patterns that fit the 2:4 MMA take the same kernel on shapes it
+  // serves, after a re-encoding pass into a staged 2:4 operand.
+  const bool pair_shape = q.K % 128 == 0 && q.T >= 192 && q.T % 8 == 0;
+  const bool reencode =
+      q.allow_staging && !q.hybrid && p.a_mode == A_BUILD_SPARSE && !(q.n == 2 && q.m == 4) && pair_shape;
+  if (reencode || (q.algo != NM_ALGO_DENSE_TC && pair_kernel_fits(p) && al16(q.meta))) {
+    cudaMemPool_t pool = nullptr;
+    cudaError_t e = cudaSuccess;
+    const uint16_t* vals = q.values;
+    const uint32_t* meta = q.meta;
+    void* staged_a = nullptr;  // re-encoded values, then tiled metadata
+    if (reencode) {
+      e = staging_pool(&pool);
+      if (e != cudaSuccess) return cuda_fail(e, "staging pool");
+      const size_t vbytes = (size_t)(q.R * (q.K / 2) * 2 + 255) / 256 * 256;
+      const size_t mbytes = (size_t)meta_words(q.R, q.K, 2, 4) * 4;
+      e = cudaMallocFromPoolAsync(&staged_a, vbytes + mbytes, pool, stream);
+      if (e != cudaSuccess) return cuda_fail(e, "staging buffer for the re-encoded weights");
+      uint16_t* v2 = static_cast<uint16_t*>(staged_a);
+      uint32_t* m2 = reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(staged_a) + vbytes);
+      e = launch_reencode_2of4(q.values, q.meta, q.R, q.K, q.n, q.m, v2, m2, stream);
+      if (e != cudaSuccess) {
+        cudaFreeAsync(staged_a, stream);
+        return cuda_fail(e, "re-encode launch");
+      }
+      vals = v2;
+      meta = m2;
+      p.n = 2;
+      p.m = 4;
+      p.pattern = PAT_2_4;
+      p.a_mode = A_TMA_SPARSE;
+      p.vcols = q.K / 2;
+      p.mcols = 0;
+    }
     // With an index map, one gather pass stages Xp[k] = X[idx[k]] in a
     // stream-ordered buffer from the staging pool and the pair kernel streams
     // Xp with TMA boxes.
     const uint16_t* xsrc = q.X;
     int64_t ldsrc = q.ldx;
     void* staged = nullptr;
+    auto release = [&]() {
+      if (staged) cudaFreeAsync(staged, stream);
+      if (staged_a) cudaFreeAsync(staged_a, stream);
+    };
     if (p.permuted) {
       const int64_t ldp = (q.T + 7) / 8 * 8;
-      cudaMemPool_t pool = nullptr;
-      cudaError_t e = staging_pool(&pool);
-      if (e != cudaSuccess) return cuda_fail(e, "staging pool");
+      if (!pool) e = staging_pool(&pool);
+      if (e != cudaSuccess) {
+        release();
+        return cuda_fail(e, "staging pool");
+      }
       e = cudaMallocFromPoolAsync(&staged, (size_t)(q.K * ldp * 2), pool, stream);
-      if (e != cudaSuccess) return cuda_fail(e, "staging buffer for the permuted input");
+      if (e != cudaSuccess) {
+        staged = nullptr;
+        release();
+        return cuda_fail(e, "staging buffer for the permuted input");
+      }
       e = launch_gather_rows(q.X, q.ldx, q.idx, q.K, q.T, static_cast<uint16_t*>(staged), ldp, stream);
       if (e != cudaSuccess) {
-        cudaFreeAsync(staged, stream);
+        release();
         return cuda_fail(e, "gather launch");
       }
       xsrc = static_cast<const uint16_t*>(staged);
@@ -292,17 +338,19 @@ static nm_status run_gemm(const GemmRequest& q, cudaStream_t stream) {
     }
     p.tiles_m = (int)((q.R + 255) / 256);
     p.tiles_n = (int)((q.T + 255) / 256);
-    if ((int64_t)p.tiles_m * p.tiles_n >= (1ll << 31)) return fail(NM_ERR_UNSUPPORTED, "too many tiles");
+    if ((int64_t)p.tiles_m * p.tiles_n >= (1ll << 31)) {
+      release();
+      return fail(NM_ERR_UNSUPPORTED, "too many tiles");
+    }
     p.num_tiles = p.tiles_m * p.tiles_n;
     p.k_tiles = q.K / 128;
     st = make_tmap(&p.tm_x, xsrc, (uint64_t)q.T, (uint64_t)q.K, (uint64_t)ldsrc * 2, 64, kPairBoxRows, 128, "X");
     if (st == NM_OK)
-      st = make_tmap(&p.tm_vals, q.values, (uint64_t)p.vcols, (uint64_t)q.R, (uint64_t)p.vcols * 2, 64, kPairBoxRows, 128,
-                     "values");
-    if (st == NM_OK) st = make_meta_tmap(&p.tm_meta, q.meta, p.meta_rblocks, p.meta_cblocks);
-    cudaError_t e = cudaSuccess;
+      st = make_tmap(&p.tm_vals, vals, (uint64_t)p.vcols, (uint64_t)q.R, (uint64_t)p.vcols * 2, 64, kPairBoxRows,
+                     128, "values");
+    if (st == NM_OK) st = make_meta_tmap(&p.tm_meta, meta, p.meta_rblocks, p.meta_cblocks);
     if (st == NM_OK) e = launch_spmm_pair(p, stream);
-    if (staged) cudaFreeAsync(staged, stream);
+    release();
     if (st != NM_OK) return st;
     return e == cudaSuccess ? NM_OK : cuda_fail(e, "spmm pair launch");
   }
@@ -334,6 +382,32 @@ static nm_status run_gemm(const GemmRequest& q, cudaStream_t stream) {
 
 // ---- helpers for entry points defined in other files (additive) ----
 void set_last_error(const char* msg) { t_last_error = msg ? msg : ""; }
+
+// nm_spmm_permuted for shapes the allocation-free call does not stage itself:
+// the same kernels, but never a staged (re-encoded) operand.
+nm_status spmm_permuted_unstaged(const uint16_t* values, const uint32_t* meta, int n, int m, int64_t R, int64_t K,
+                                 const int32_t* idx, const uint16_t* X, int64_t ldx, int64_t T, void* Y,
+                                 int64_t ldy, nm_out_dtype y_dtype, cudaStream_t stream) {
+  if (!idx && R > 0 && K > 0 && T > 0) return fail(NM_ERR_INVALID_ARG, "idx is null");
+  GemmRequest q{};
+  q.values = values;
+  q.meta = meta;
+  q.n = n;
+  q.m = m;
+  q.R = R;
+  q.K = K;
+  q.T = T;
+  q.idx = idx;
+  q.X = X;
+  q.ldx = ldx;
+  q.Y = Y;
+  q.ldy = ldy;
+  q.y_dtype = (int)y_dtype;
+  q.algo = NM_ALGO_AUTO;
+  q.hybrid = false;
+  q.allow_staging = false;
+  return run_gemm(q, stream);
+}
 
 bool pair_path_for(int n, int m, int64_t R, int64_t K, int64_t T, const void* values, const void* meta) {
   SpmmParams p;

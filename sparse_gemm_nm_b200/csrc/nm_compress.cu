@@ -309,6 +309,66 @@ __global__ void __launch_bounds__(256) gather_rows_kernel(const uint16_t* __rest
   }
 }
 
+// Re-encoding of an N:M operand whose survivors never exceed two per aligned
+// group of four (1:2, 1:4, 2:4, 1:8, 2:8) as a 2:4 operand with tiled
+// metadata, so that the two-SM sparse GEMM can run it.  A group of four keeps
+// its survivors (ascending); one survivor is paired with a +0.0 at the lowest
+// other position, none gives (0, 1) with two zeros.  One thread per row and
+// 16-column chunk (one 16-bit half of a tiled metadata word); rows and
+// columns of the padded blocks get the padding nibbles 0x4.
+template <int M>
+__global__ void __launch_bounds__(256) reencode_2of4_kernel(const uint16_t* __restrict__ V,
+                                                            const uint32_t* __restrict__ meta, uint32_t R,
+                                                            uint32_t K, int n, uint32_t vcols, uint32_t mcols,
+                                                            uint16_t* __restrict__ V2, uint16_t* __restrict__ meta2,
+                                                            uint32_t cblocks, uint32_t total) {
+  constexpr int B = M == 2 ? 1 : M == 4 ? 2 : 3;
+  constexpr int S = 32 / B;
+  const uint32_t chunks = cblocks * 8;
+  for (uint32_t t = blockIdx.x * blockDim.x + threadIdx.x; t < total; t += gridDim.x * blockDim.x) {
+    const uint32_t r = t / chunks, c = t - r * chunks;
+    const uint32_t cb = c >> 3, qh = c & 7u;  // block column 16*qh = 32q + 16h
+    const uint32_t k0 = cb * 128 + 16 * qh;
+    const uint32_t word = ((r >> 4) * cblocks + cb) * 64 + 4 * ((r & 7u) + 8 * (qh & 1u)) + (qh >> 1);
+    uint32_t nib16 = 0x4444u;
+    if (r < R && k0 < K) {
+      nib16 = 0;
+      uint32_t out[4];
+      for (int g4 = 0; g4 < 4; ++g4) {
+        const uint32_t c4 = k0 + 4 * g4;  // first column of this group of four
+        uint32_t pos[2] = {0, 1}, val[2] = {0, 0};
+        int cnt = 0;
+        if (c4 < K) {
+          const uint32_t g_first = c4 / M, g_last = (c4 + 3) / M;  // N:M groups overlapping [c4, c4 + 4)
+          for (uint32_t g = g_first; g <= g_last; ++g) {
+            for (int s = 0; s < n; ++s) {
+              const uint32_t j = g * n + s;
+              const uint32_t pw = __ldg(meta + (int64_t)r * mcols + j / S);
+              const uint32_t col = g * M + ((pw >> (B * (j % S))) & ((1u << B) - 1u));
+              if (col >= c4 && col < c4 + 4 && cnt < 2) {
+                pos[cnt] = col - c4;
+                val[cnt] = V[(int64_t)r * vcols + j];
+                ++cnt;
+              }
+            }
+          }
+        }
+        uint32_t p0 = pos[0], p1 = pos[1], v0 = val[0], v1 = val[1];
+        if (cnt == 1) {  // pair the survivor with a zero at the lowest other position
+          if (pos[0] == 0) { p0 = 0; p1 = 1; v0 = val[0]; v1 = 0; }
+          else { p0 = 0; p1 = pos[0]; v0 = 0; v1 = val[0]; }
+        }
+        nib16 |= (p0 | (p1 << 2)) << (4 * g4);
+        out[g4] = v0 | (v1 << 16);
+      }
+      uint32_t* vrow = reinterpret_cast<uint32_t*>(V2 + (int64_t)r * (K >> 1) + k0 / 2);
+      for (int g4 = 0; g4 < 4; ++g4)
+        if (k0 + 4 * g4 < K) vrow[g4] = out[g4];
+    }
+    meta2[2 * (int64_t)word + ((r >> 3) & 1u)] = (uint16_t)nib16;
+  }
+}
+
 static int grid_for(int64_t work, int threads) {
   const int64_t want = (work + threads - 1) / threads;
   const int64_t cap = (int64_t)sm_count_current() * 16;
@@ -373,6 +433,27 @@ cudaError_t launch_fill_zero(void* Y, int64_t R, int64_t T, int64_t ldy, int esi
   const int threads = 256;
   fill_zero_kernel<<<grid_for(R * T * esize, threads), threads, 0, s>>>(static_cast<uint8_t*>(Y), R, T * esize,
                                                                          ldy * esize);
+  count_launch();
+  return cudaGetLastError();
+}
+
+cudaError_t launch_reencode_2of4(const uint16_t* values, const uint32_t* meta, int64_t R, int64_t K, int n, int m,
+                                 uint16_t* values2, uint32_t* meta2, cudaStream_t s) {
+  const int threads = 256;
+  const int64_t cblocks = meta_col_blocks(K);
+  const int64_t total = meta_row_blocks(R) * 16 * cblocks * 8;
+  const int grid = grid_for(total, threads);
+  const uint32_t vcols = (uint32_t)value_cols(K, n, m), mcols = (uint32_t)meta_cols(K, n, m);
+  uint16_t* m16 = reinterpret_cast<uint16_t*>(meta2);
+  switch (m) {
+    case 2: reencode_2of4_kernel<2><<<grid, threads, 0, s>>>(values, meta, (uint32_t)R, (uint32_t)K, n, vcols, mcols,
+                                                                values2, m16, (uint32_t)cblocks, (uint32_t)total); break;
+    case 4: reencode_2of4_kernel<4><<<grid, threads, 0, s>>>(values, meta, (uint32_t)R, (uint32_t)K, n, vcols, mcols,
+                                                                values2, m16, (uint32_t)cblocks, (uint32_t)total); break;
+    case 8: reencode_2of4_kernel<8><<<grid, threads, 0, s>>>(values, meta, (uint32_t)R, (uint32_t)K, n, vcols, mcols,
+                                                                values2, m16, (uint32_t)cblocks, (uint32_t)total); break;
+    default: return cudaErrorInvalidValue;
+  }
   count_launch();
   return cudaGetLastError();
 }

@@ -37,6 +37,8 @@ cudaError_t launch_decompress(const uint16_t* values, const uint32_t* meta, int6
                               uint16_t* W_out, int64_t ldw, cudaStream_t s);
 cudaError_t launch_gather_rows(const uint16_t* X, int64_t ldx, const int32_t* idx, int64_t K, int64_t T,
                                uint16_t* Xp, int64_t ldp, cudaStream_t s);
+cudaError_t launch_reencode_2of4(const uint16_t* values, const uint32_t* meta, int64_t R, int64_t K, int n, int m,
+                                 uint16_t* values2, uint32_t* meta2, cudaStream_t s);
 cudaError_t launch_fill_zero(void* Y, int64_t R, int64_t T, int64_t ldy, int esize, cudaStream_t s);
 
 }  // namespace nmk

@@ -25,6 +25,9 @@ namespace nmk {
 
 void set_last_error(const char* msg);
 bool pair_path_for(int n, int m, int64_t R, int64_t K, int64_t T, const void* values, const void* meta);
+nm_status spmm_permuted_unstaged(const uint16_t* values, const uint32_t* meta, int n, int m, int64_t R, int64_t K,
+                                 const int32_t* idx, const uint16_t* X, int64_t ldx, int64_t T, void* Y,
+                                 int64_t ldy, nm_out_dtype y_dtype, cudaStream_t stream);
 nm_status build_pair_params(SpmmParams& p, const uint16_t* values, const uint32_t* meta, int64_t R, int64_t K,
                             const uint16_t* X, int64_t ldx, int64_t T, void* Y, int64_t ldy, bool out_f32);
 
@@ -72,10 +75,11 @@ extern "C" NM_API nm_status nm_spmm_permuted_noalloc(const uint16_t* values, con
                                                      int64_t R, int64_t K, const int32_t* idx, const uint16_t* X,
                                                      int64_t ldx, int64_t T, void* Y, int64_t ldy,
                                                      nm_out_dtype y_dtype, void* stream) {
-  // Shapes that the two-SM path does not take never stage anything: the
-  // one-SM kernel gathers X rows itself, so the ordinary call allocates nothing.
+  // Other shapes and patterns run on the one-SM kernel, which gathers X rows
+  // itself and stages nothing (no re-encoded operand either).
   if (!pair_path_for(n, m, R, K, T, values, meta) || R <= 0 || K <= 0 || T <= 0)
-    return nm_spmm_permuted(values, meta, n, m, R, K, idx, X, ldx, T, Y, ldy, y_dtype, stream);
+    return spmm_permuted_unstaged(values, meta, n, m, R, K, idx, X, ldx, T, Y, ldy, y_dtype,
+                                  static_cast<cudaStream_t>(stream));
   set_last_error("");
   if (!idx || !X || !Y || !values || !meta) {
     set_last_error("null pointer");

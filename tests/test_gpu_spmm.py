@@ -314,3 +314,28 @@ def test_permuted_pair_path_after_release_staging():
     assert torch.equal(first, second)
     ref, mag = reference(W, X, 2, 4, idx)
     assert_gemm_close(values_f64(second), ref, mag, "permuted after release")
+
+
+# ----------------------------------------------------------------------------
+# 1:2 / 1:4 / 1:8 / 2:8 on two-SM shapes: re-encoded as 2:4, then the pair kernel
+# ----------------------------------------------------------------------------
+@pytest.mark.parametrize("n,m", [(1, 2), (1, 4), (1, 8), (2, 8)])
+@pytest.mark.parametrize("permuted", [False, True])
+def test_reencoded_pair_path(n, m, permuted):
+    R, K, T = 300, 512, 264
+    W = wl.normal_bf16((R, K), 0.02, seed=131 + m + n)
+    X = wl.normal_bf16((K, T), 1.0, seed=132)
+    idx = wl.permutation(K, 133) if permuted else None
+    before = nm.nm_launch_count()
+    check(W, X, n, m, idx=idx, what=f"re-encoded {n}:{m}")
+    # prune_compress, re-encode, [gather,] pair GEMM
+    assert nm.nm_launch_count() - before == (4 if permuted else 3)
+
+
+def test_reencoded_pair_path_integer_exact():
+    R, K, T = 256, 384, 256
+    W = wl.integer_bf16((R, K), -8, 8, seed=141)
+    X = wl.integer_bf16((K, T), -8, 8, seed=142)
+    ref, _ = reference(W, X, 1, 8)
+    Y = run_spmm(W, X, 1, 8, out_dtype=torch.float32)
+    assert np.array_equal(Y.cpu().numpy().astype(np.float64), ref)

@@ -72,3 +72,27 @@ def test_noalloc_rejects_k_beyond_the_array():
         nm.nm_spmm_permuted_noalloc(vals, meta, 2, 4, R, K, idx, X, T, T, Y, T)
     assert e.value.status == nm.NM_ERR_UNSUPPORTED
     assert "staging array" in str(e.value)
+
+
+def test_noalloc_other_patterns_stage_nothing():
+    """1:8 on a two-SM shape: nm_spmm_permuted re-encodes it into a staged
+    operand; the allocation-free call must run the one-SM kernel instead (one
+    launch) and give the same result within the tolerance."""
+    R, K, T = 256, 512, 256
+    W = wl.normal_bf16((R, K), 0.02, seed=8)
+    X = wl.normal_bf16((K, T), 1.0, seed=9)
+    idx = wl.permutation(K, 10)
+    vals, meta = nm.prune_compress(to_dev(W), 1, 8)
+    Xd, idxd = to_dev(X), to_dev_i32(idx)
+    y_ref = torch.empty((R, T), dtype=torch.bfloat16, device=DEV)
+    y_new = torch.empty((R, T), dtype=torch.bfloat16, device=DEV)
+    nm.nm_spmm_permuted(vals, meta, 1, 8, R, K, idxd, Xd, T, T, y_ref, T)
+    before = nm.nm_launch_count()
+    nm.nm_spmm_permuted_noalloc(vals, meta, 1, 8, R, K, idxd, Xd, T, T, y_new, T)
+    assert nm.nm_launch_count() - before == 1
+    torch.cuda.synchronize()
+    nm.nm_device_status()
+    vals_o, meta_o = oracle.compress(W, 1, 8)
+    Wd = wl.bf16_to_f32(oracle.decompress(vals_o, meta_o, K, 1, 8)).astype(np.float64)
+    Xp = wl.bf16_to_f32(np.ascontiguousarray(X[idx])).astype(np.float64)
+    assert_gemm_close(values_f64(y_new), values_f64(y_ref), np.abs(Wd) @ np.abs(Xp), "1:8 no-alloc")
