@@ -139,8 +139,12 @@ NM_API nm_status nm_decompress(const uint16_t* values, const uint32_t* meta, int
  * 1:8 and 2:8 (at most two survivors per aligned group of four) are first
  * re-encoded as 2:4 into a staging buffer (R*K bytes of values plus R*K/8
  * bytes of metadata) from the library's pool (see nm_spmm_permuted and
- * nm_release_staging), one extra launch.  Every other case runs on one SM per
- * 128-row tile and stages nothing.
+ * nm_release_staging), one extra launch.  Shapes with K % 128 == 0 and
+ * T <= 64 run a split-K kernel (one 128-row tile and one range of K per work
+ * unit, persistent over the SMs); when K is split into s > 1 ranges it stages
+ * s*R*bn*4 bytes of fp32 partials (bn = T rounded up to 16, 32 or 64) and a
+ * second launch sums them in range order.  Every other case runs on one SM
+ * per 128-row tile and stages nothing.
  * Errors: NM_ERR_INVALID_ARG, NM_ERR_MISALIGNED, NM_ERR_CUDA.
  */
 NM_API nm_status nm_spmm(const uint16_t* values, const uint32_t* meta, int n, int m, int64_t R, int64_t K,

@@ -197,6 +197,30 @@ struct GemmRequest {
   bool allow_staging = true;
 };
 
+// Split of the K stages for the skinny kernel: the number of ranges that
+// keeps the persistent CTAs best balanced (units per CTA / its ceiling), each
+// range at least two stages, fewest ranges on ties.  Every range is non-empty.
+static void choose_splits(SpmmParams& p, int sms) {
+  const int64_t kt = p.k_tiles;
+  int best_s = 1, best_kps = (int)kt;
+  double best = -1.0;
+  for (int s = 1; s <= 16 && s <= kt; ++s) {
+    const int64_t kps = (kt + s - 1) / s;
+    if (kps < 2 && s > 1) break;
+    const int64_t se = (kt + kps - 1) / kps;  // ranges actually used
+    const int64_t units = (int64_t)p.tiles_m * se;
+    const int64_t waves = (units + sms - 1) / sms;
+    const double eff = (double)units / (double)(waves * sms);
+    if (eff > best + 1e-9) {
+      best = eff;
+      best_s = (int)se;
+      best_kps = (int)kps;
+    }
+  }
+  p.splits = best_s;
+  p.kt_per_split = best_kps;
+}
+
 static nm_status run_gemm(const GemmRequest& q, cudaStream_t stream) {
   t_last_error.clear();
   if (q.R < 0 || q.K < 0 || q.T < 0) return fail(NM_ERR_INVALID_ARG, "negative dimension");
@@ -272,10 +296,14 @@ static nm_status run_gemm(const GemmRequest& q, cudaStream_t stream) {
   // Two SMs per 256 x 256 tile when the shape allows it (2:4 from TMA, K % 128 == 0).
   // Other patterns that fit the 2:4 MMA take the same kernel on shapes it
   // serves, after a re-encoding pass into a staged 2:4 operand.
+  // Few columns (T <= 64): the split-K skinny kernel on the same staged operands.
   const bool pair_shape = q.K % 128 == 0 && q.T >= 192 && q.T % 8 == 0;
-  const bool reencode =
-      q.allow_staging && !q.hybrid && p.a_mode == A_BUILD_SPARSE && !(q.n == 2 && q.m == 4) && pair_shape;
-  if (reencode || (q.algo != NM_ALGO_DENSE_TC && pair_kernel_fits(p) && al16(q.meta))) {
+  const bool skinny_shape = q.K % 128 == 0 && skinny_kernel_fits(q.T) && q.allow_staging;
+  const bool tma_2of4 = p.a_mode == A_TMA_SPARSE && al16(q.meta) && q.algo != NM_ALGO_DENSE_TC;
+  const bool reencode = q.allow_staging && !q.hybrid && p.a_mode == A_BUILD_SPARSE && !(q.n == 2 && q.m == 4) &&
+                        (pair_shape || skinny_shape);
+  const bool use_skinny = skinny_shape && (tma_2of4 || reencode);
+  if (reencode || use_skinny || (q.algo != NM_ALGO_DENSE_TC && pair_kernel_fits(p) && al16(q.meta))) {
     cudaMemPool_t pool = nullptr;
     cudaError_t e = cudaSuccess;
     const uint16_t* vals = q.values;
@@ -336,23 +364,51 @@ static nm_status run_gemm(const GemmRequest& q, cudaStream_t stream) {
       ldsrc = ldp;
       p.permuted = 0;
     }
-    p.tiles_m = (int)((q.R + 255) / 256);
-    p.tiles_n = (int)((q.T + 255) / 256);
-    if ((int64_t)p.tiles_m * p.tiles_n >= (1ll << 31)) {
-      release();
-      return fail(NM_ERR_UNSUPPORTED, "too many tiles");
-    }
-    p.num_tiles = p.tiles_m * p.tiles_n;
     p.k_tiles = q.K / 128;
-    st = make_tmap(&p.tm_x, xsrc, (uint64_t)q.T, (uint64_t)q.K, (uint64_t)ldsrc * 2, 64, kPairBoxRows, 128, "X");
+    void* ws = nullptr;
+    if (use_skinny) {
+      p.bn = skinny_bn(q.T);
+      p.kd = skinny_kd(q.K, q.T);
+      p.k_tiles = q.K / p.kd;
+      p.tiles_m = (int)((q.R + 127) / 128);
+      if ((int64_t)p.tiles_m * p.k_tiles >= (1ll << 31)) {
+        release();
+        return fail(NM_ERR_UNSUPPORTED, "too many tiles");
+      }
+      choose_splits(p, sm_count_current());
+      p.tiles_n = 1;
+      p.num_tiles = p.tiles_m;
+      if (p.splits > 1) {
+        if (!pool) e = staging_pool(&pool);
+        if (e == cudaSuccess) e = cudaMallocFromPoolAsync(&ws, (size_t)p.splits * q.R * p.bn * 4, pool, stream);
+        if (e != cudaSuccess) {
+          ws = nullptr;
+          release();
+          return cuda_fail(e, "split-K workspace");
+        }
+        p.ws = static_cast<float*>(ws);
+      }
+      st = make_tmap(&p.tm_x, xsrc, (uint64_t)q.T, (uint64_t)q.K, (uint64_t)ldsrc * 2, (uint32_t)p.bn,
+                     (uint32_t)p.kd, p.bn * 2, "X");
+    } else {
+      p.tiles_m = (int)((q.R + 255) / 256);
+      p.tiles_n = (int)((q.T + 255) / 256);
+      if ((int64_t)p.tiles_m * p.tiles_n >= (1ll << 31)) {
+        release();
+        return fail(NM_ERR_UNSUPPORTED, "too many tiles");
+      }
+      p.num_tiles = p.tiles_m * p.tiles_n;
+      st = make_tmap(&p.tm_x, xsrc, (uint64_t)q.T, (uint64_t)q.K, (uint64_t)ldsrc * 2, 64, kPairBoxRows, 128, "X");
+    }
     if (st == NM_OK)
       st = make_tmap(&p.tm_vals, vals, (uint64_t)p.vcols, (uint64_t)q.R, (uint64_t)p.vcols * 2, 64, kPairBoxRows,
                      128, "values");
     if (st == NM_OK) st = make_meta_tmap(&p.tm_meta, meta, p.meta_rblocks, p.meta_cblocks);
-    if (st == NM_OK) e = launch_spmm_pair(p, stream);
+    if (st == NM_OK) e = use_skinny ? launch_spmm_skinny(p, stream) : launch_spmm_pair(p, stream);
+    if (ws) cudaFreeAsync(ws, stream);
     release();
     if (st != NM_OK) return st;
-    return e == cudaSuccess ? NM_OK : cuda_fail(e, "spmm pair launch");
+    return e == cudaSuccess ? NM_OK : cuda_fail(e, use_skinny ? "spmm skinny launch" : "spmm pair launch");
   }
 
   const int bn = pick_bn(q.T);

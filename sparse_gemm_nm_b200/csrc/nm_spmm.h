@@ -46,6 +46,13 @@ struct SpmmParams {
   int hyb_tiles_k;
   int stages;
   uint32_t a_slot_bytes;
+  // skinny (small T) split-K kernel: K tiles of 128 split into `splits`
+  // ranges of `kt_per_split`; fp32 partials in ws[splits][R][bn] when splits > 1
+  int splits;
+  int kt_per_split;
+  int bn;
+  int kd;  // skinny stage depth (logical K per stage: 128 or 256)
+  float* ws;
 };
 
 int spmm_max_stages(int bn, uint32_t a_slot);
@@ -54,5 +61,9 @@ cudaError_t read_and_clear_status(uint32_t* out);
 uint32_t* status_word_ptr();
 bool pair_kernel_fits(const SpmmParams& p);
 cudaError_t launch_spmm_pair(SpmmParams& p, cudaStream_t stream);
+bool skinny_kernel_fits(int64_t T);
+int skinny_bn(int64_t T);
+int skinny_kd(int64_t K, int64_t T);
+cudaError_t launch_spmm_skinny(SpmmParams& p, cudaStream_t stream);
 
 }  // namespace nmk

@@ -339,3 +339,35 @@ def test_reencoded_pair_path_integer_exact():
     ref, _ = reference(W, X, 1, 8)
     Y = run_spmm(W, X, 1, 8, out_dtype=torch.float32)
     assert np.array_equal(Y.cpu().numpy().astype(np.float64), ref)
+
+
+# ----------------------------------------------------------------------------
+# Few columns (T <= 64, K % 128 == 0): the split-K skinny kernel
+# ----------------------------------------------------------------------------
+@pytest.mark.parametrize("R,K,T", [(200, 1024, 16), (128, 512, 8), (333, 2048, 40), (1000, 256, 64),
+                                   (64, 128, 8), (13824 // 8, 5120, 24)])
+def test_skinny_kernel(R, K, T):
+    W = wl.normal_bf16((R, K), 0.02, seed=R + K + T)
+    X = wl.normal_bf16((K, T), 1.0, seed=T + 7)
+    check(W, X, 2, 4, what=f"skinny {R}x{K}x{T}")
+
+
+@pytest.mark.parametrize("n,m", [(2, 4), (1, 8)])
+def test_skinny_kernel_permuted(n, m):
+    R, K, T = 300, 1024, 16
+    W = wl.normal_bf16((R, K), 0.02, seed=151)
+    X = wl.normal_bf16((K, T), 1.0, seed=152)
+    check(W, X, n, m, idx=wl.permutation(K, 153), what=f"skinny permuted {n}:{m}")
+
+
+@pytest.mark.parametrize("out", [torch.bfloat16, torch.float32])
+def test_skinny_kernel_integer_exact(out):
+    R, K, T = 384, 4096, 16  # several K ranges: partial sums are exact integers
+    W = wl.integer_bf16((R, K), -8, 8, seed=161)
+    X = wl.integer_bf16((K, T), -8, 8, seed=162)
+    ref, _ = reference(W, X, 2, 4)
+    Y = run_spmm(W, X, 2, 4, out_dtype=out)
+    if out == torch.float32:
+        assert np.array_equal(Y.cpu().numpy().astype(np.float64), ref)
+    else:
+        assert np.array_equal(bits(Y), bf16_rne_of(ref))
