@@ -404,6 +404,8 @@ static nm_status run_gemm(const GemmRequest& q, cudaStream_t stream) {
       st = make_tmap(&p.tm_vals, vals, (uint64_t)p.vcols, (uint64_t)q.R, (uint64_t)p.vcols * 2, 64, kPairBoxRows,
                      128, "values");
     if (st == NM_OK) st = make_meta_tmap(&p.tm_meta, meta, p.meta_rblocks, p.meta_cblocks);
+    if (st == NM_OK && !use_skinny && !p.out_f32)
+      st = make_tmap(&p.tm_y, q.Y, (uint64_t)q.T, (uint64_t)q.R, (uint64_t)q.ldy * 2, 64, 32, 128, "Y");
     if (st == NM_OK) e = use_skinny ? launch_spmm_skinny(p, stream) : launch_spmm_pair(p, stream);
     if (ws) cudaFreeAsync(ws, stream);
     release();
@@ -507,6 +509,8 @@ nm_status build_pair_params(SpmmParams& p, const uint16_t* values, const uint32_
     st = make_tmap(&p.tm_vals, values, (uint64_t)p.vcols, (uint64_t)R, (uint64_t)p.vcols * 2, 64, kPairBoxRows, 128,
                    "values");
   if (st == NM_OK) st = make_meta_tmap(&p.tm_meta, meta, p.meta_rblocks, p.meta_cblocks);
+  if (st == NM_OK && !out_f32)
+    st = make_tmap(&p.tm_y, Y, (uint64_t)T, (uint64_t)R, (uint64_t)ldy * 2, 64, 32, 128, "Y");
   return st;
 }
 

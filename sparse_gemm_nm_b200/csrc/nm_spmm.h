@@ -23,6 +23,7 @@ struct SpmmParams {
   CUtensorMap tm_vals;  // compressed values R x K*n/m, box {32, 128} 64B swizzle (one SM) or {64, kPairBoxRows} 128B (SM pair)
   CUtensorMap tm_w;     // dense W R x K, box {64, 128}, 128B swizzle (hybrid)
   CUtensorMap tm_x;     // X K x T, box {strip, 64} (one SM) or {64, kPairBoxRows} (SM pair)
+  CUtensorMap tm_y;     // Y R x T bf16, box {64, 32}, 128B swizzle (SM-pair epilogue stores)
   CUtensorMap tm_meta;  // tiled 2:4 metadata {64 words, col blocks, row blocks}, box {64, 1, 8} (SM pair)
   const uint16_t* vals;
   const uint32_t* meta;

@@ -46,12 +46,13 @@ constexpr uint64_t kWaitNs = 2000000000ull;
 constexpr uint32_t kTxPerStage = 2u * (kA + kB + kE);  // both CTAs' A, B and E bytes
 constexpr uint32_t kIdesc = idesc_bf16(256, true, 256);
 
+constexpr uint32_t kEpi = 4096;  // per epilogue warp: 32 rows x 64 bf16 columns, 128-byte swizzle
 struct Layout {
-  uint32_t a, b, e, bar, total;
+  uint32_t a, b, e, epi, bar, total;
 };
 __host__ __device__ constexpr Layout layout() {
-  return Layout{0u, kStages * kA, kStages * (kA + kB), kStages * (kA + kB + kE),
-                kStages * (kA + kB + kE) + (2 * kStages + 4) * 8 + 64};
+  return Layout{0u, kStages * kA, kStages * (kA + kB), kStages * (kA + kB + kE), kStages * (kA + kB + kE) + 4 * kEpi,
+                kStages * (kA + kB + kE) + 4 * kEpi + (2 * kStages + 4) * 8 + 64};
 }
 }  // namespace pair
 
@@ -188,7 +189,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pair::kThreads, 1)
       tc_fence_after();
       const uint32_t t_addr = tmem_base + ((uint32_t)(quarter * 32) << 16);
       const bool row_ok = row < p.R;
-      if (!p.out_f32 && n0 + 256 <= p.T) {
+      if (!p.out_f32) {
+        // Whole accumulator row into registers (bf16), release TMEM, then four
+        // 64-column chunks through this warp's swizzled staging buffer and a
+        // TMA store each: every store writes whole lines, and parts of the box
+        // beyond R or T are not written.
         uint32_t pk[128];
 #pragma unroll
         for (int c = 0; c < 8; ++c) {
@@ -202,11 +207,22 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pair::kThreads, 1)
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive_cluster(lead_acc_empty);
-        if (row_ok) {
-          uint4* yrow = reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.Y) + row * p.ldy + n0);
+        const int32_t wrow0 = (int32_t)(tm * 256 + 128 * rank + quarter * 32);
+        uint8_t* ebuf = smem + L.epi + quarter * kEpi;
 #pragma unroll
-          for (int c8 = 0; c8 < 32; ++c8)
-            yrow[c8] = make_uint4(pk[4 * c8], pk[4 * c8 + 1], pk[4 * c8 + 2], pk[4 * c8 + 3]);
+        for (int c = 0; c < 4; ++c) {
+          if (lane == 0) bulk_wait_group_read<0>();  // the previous store has read the buffer
+          __syncwarp();
+#pragma unroll
+          for (int j = 0; j < 8; ++j)
+            *reinterpret_cast<uint4*>(ebuf + lane * 128 + ((j ^ (lane & 7)) << 4)) =
+                make_uint4(pk[32 * c + 4 * j], pk[32 * c + 4 * j + 1], pk[32 * c + 4 * j + 2], pk[32 * c + 4 * j + 3]);
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0 && n0 + 64 * c < p.T && wrow0 < p.R) {
+            tma_store_2d(&p.tm_y, ebuf, (int32_t)(n0 + 64 * c), wrow0);
+            bulk_commit_group();
+          }
         }
       } else {
 #pragma unroll 1
@@ -237,6 +253,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pair::kThreads, 1)
       }
       aph ^= 1u;
     }
+    if (lane == 0) bulk_wait_group<0>();  // every store of this warp has landed
   }
 
   // -------------------------------------------------------------- teardown
