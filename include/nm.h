@@ -190,6 +190,10 @@ NM_API nm_status nm_spmm_permuted(const uint16_t* values, const uint32_t* meta, 
  *   values, meta [in] nm_prune_compress(W, 2, 4) (2:4 tiles)
  *   tile_map [in] ceil(R/tile) x ceil(K/tile) uint8, 0 = dense, 1 = 2:4
  *   tile     [in] must be 128
+ * Shapes with K % 128 == 0, T >= 192 and T % 8 == 0 run on SM pairs: a K
+ * stage of a 256-row tile uses the 2:4 MMA when both 128-row tiles are 2:4,
+ * else dense MMAs; the 2:4 tiles of such stages come from a staged copy of W
+ * under the mask (R*K*2 bytes from the library's pool, one extra launch).
  * Other arguments as nm_spmm.  Errors: as nm_spmm, NM_ERR_UNSUPPORTED for
  * tile != 128 or K % 16 != 0.
  */

@@ -296,6 +296,44 @@ static nm_status run_gemm(const GemmRequest& q, cudaStream_t stream) {
   // Two SMs per 256 x 256 tile when the shape allows it (2:4 from TMA, K % 128 == 0).
   // Other patterns that fit the 2:4 MMA take the same kernel on shapes it
   // serves, after a re-encoding pass into a staged 2:4 operand.
+  // PATCH hybrid on SM pairs: a stage runs the sparse MMA when both CTAs' 128 x 128
+  // tiles are 2:4, else the dense MMA on W, with the 2:4 tiles taken from a staged
+  // copy of W under the mask (one tile-filtered decompress pass).
+  if (q.hybrid && q.allow_staging && q.K % 128 == 0 && q.T >= 192 && q.T % 8 == 0 && al16(q.meta)) {
+    cudaMemPool_t pool = nullptr;
+    cudaError_t e = staging_pool(&pool);
+    if (e != cudaSuccess) return cuda_fail(e, "staging pool");
+    void* wm = nullptr;
+    e = cudaMallocFromPoolAsync(&wm, (size_t)(q.R * q.K * 2), pool, stream);
+    if (e != cudaSuccess) return cuda_fail(e, "staging buffer for the masked 2:4 tiles");
+    e = launch_decompress_tiles(q.values, q.meta, q.R, q.K, q.tile_map, static_cast<uint16_t*>(wm), q.K, stream);
+    if (e != cudaSuccess) {
+      cudaFreeAsync(wm, stream);
+      return cuda_fail(e, "masked-tile decompress launch");
+    }
+    p.tiles_m = (int)((q.R + 255) / 256);
+    p.tiles_n = (int)((q.T + 255) / 256);
+    p.num_tiles = p.tiles_m * p.tiles_n;
+    p.k_tiles = q.K / 128;
+    p.hyb_tiles_k = (int)(q.K / 128);
+    p.hyb_rows = (int)((q.R + 127) / 128);
+    st = make_tmap(&p.tm_x, q.X, (uint64_t)q.T, (uint64_t)q.K, (uint64_t)q.ldx * 2, 64, kPairBoxRows, 128, "X");
+    if (st == NM_OK)
+      st = make_tmap(&p.tm_vals, q.values, (uint64_t)p.vcols, (uint64_t)q.R, (uint64_t)p.vcols * 2, 64,
+                     kPairBoxRows, 128, "values");
+    if (st == NM_OK) st = make_meta_tmap(&p.tm_meta, q.meta, p.meta_rblocks, p.meta_cblocks);
+    if (st == NM_OK)
+      st = make_tmap(&p.tm_w, q.W, (uint64_t)q.K, (uint64_t)q.R, (uint64_t)q.ldw * 2, 64, kPairBoxRows, 128, "W");
+    if (st == NM_OK)
+      st = make_tmap(&p.tm_wm, wm, (uint64_t)q.K, (uint64_t)q.R, (uint64_t)q.K * 2, 64, kPairBoxRows, 128, "W masked");
+    if (st == NM_OK && !p.out_f32)
+      st = make_tmap(&p.tm_y, q.Y, (uint64_t)q.T, (uint64_t)q.R, (uint64_t)q.ldy * 2, 64, 32, 128, "Y");
+    if (st == NM_OK) e = launch_spmm_pair_hybrid(p, stream);
+    cudaFreeAsync(wm, stream);
+    if (st != NM_OK) return st;
+    return e == cudaSuccess ? NM_OK : cuda_fail(e, "hybrid pair launch");
+  }
+
   // Few columns (T <= 64): the split-K skinny kernel on the same staged operands.
   const bool pair_shape = q.K % 128 == 0 && q.T >= 192 && q.T % 8 == 0;
   const bool skinny_shape = q.K % 128 == 0 && skinny_kernel_fits(q.T) && q.allow_staging;

@@ -218,7 +218,7 @@ __global__ void __launch_bounds__(256) decompress_2of4_tiled_kernel(const uint16
                                                                     const uint32_t* __restrict__ meta, uint32_t R,
                                                                     uint32_t K, uint16_t* __restrict__ W,
                                                                     int64_t ldw, uint32_t cblocks, uint32_t total,
-                                                                    bool vec) {
+                                                                    bool vec, const uint8_t* __restrict__ tile_map) {
   for (uint32_t w = blockIdx.x * blockDim.x + threadIdx.x; w < total; w += gridDim.x * blockDim.x) {
     const uint32_t blk = w >> 6, wi = w & 63u;
     const uint32_t l = wi >> 2, q = wi & 3u;
@@ -226,6 +226,8 @@ __global__ void __launch_bounds__(256) decompress_2of4_tiled_kernel(const uint16
     const uint32_t r_lo = rb * 16 + (l & 7u);
     const uint32_t k0 = cb * 128 + q * 32 + (l >> 3) * 16;
     if (k0 >= K) continue;
+    // with a tile map (128 x 128 tiles, one column block each): 2:4 tiles only
+    if (tile_map && __ldg(tile_map + (int64_t)(r_lo >> 7) * cblocks + cb) == 0) continue;
     const uint32_t word = __ldg(meta + w);
     if (r_lo < R)
       decompress_half16(V + (int64_t)r_lo * (K >> 1), W + (int64_t)r_lo * ldw, word & 0xFFFFu, k0, K, vec);
@@ -406,7 +408,8 @@ cudaError_t launch_decompress(const uint16_t* values, const uint32_t* meta, int6
     const int64_t total = meta_words(R, K, n, m);
     const bool vec = K % 16 == 0 && ldw % 8 == 0 && aligned16(W_out) && aligned16(values);
     decompress_2of4_tiled_kernel<<<grid_for(total, threads), threads, 0, s>>>(
-        values, meta, (uint32_t)R, (uint32_t)K, W_out, ldw, (uint32_t)meta_col_blocks(K), (uint32_t)total, vec);
+        values, meta, (uint32_t)R, (uint32_t)K, W_out, ldw, (uint32_t)meta_col_blocks(K), (uint32_t)total, vec,
+        nullptr);
   } else {
     const int64_t work = R * (K / m);
     const int grid = grid_for(work, threads);
@@ -417,6 +420,18 @@ cudaError_t launch_decompress(const uint16_t* values, const uint32_t* meta, int6
       default: decompress_generic_kernel<16><<<grid, threads, 0, s>>>(values, meta, R, K, n, W_out, ldw); break;
     }
   }
+  count_launch();
+  return cudaGetLastError();
+}
+
+cudaError_t launch_decompress_tiles(const uint16_t* values, const uint32_t* meta, int64_t R, int64_t K,
+                                    const uint8_t* tile_map, uint16_t* W_out, int64_t ldw, cudaStream_t s) {
+  const int threads = 256;
+  const int64_t total = meta_words(R, K, 2, 4);
+  const bool vec = K % 16 == 0 && ldw % 8 == 0 && aligned16(W_out) && aligned16(values);
+  decompress_2of4_tiled_kernel<<<grid_for(total, threads), threads, 0, s>>>(
+      values, meta, (uint32_t)R, (uint32_t)K, W_out, ldw, (uint32_t)meta_col_blocks(K), (uint32_t)total, vec,
+      tile_map);
   count_launch();
   return cudaGetLastError();
 }

@@ -35,6 +35,10 @@ cudaError_t launch_compress(const uint16_t* W, int64_t R, int64_t K, int64_t ldw
                             uint32_t* meta, cudaStream_t s);
 cudaError_t launch_decompress(const uint16_t* values, const uint32_t* meta, int64_t R, int64_t K, int n, int m,
                               uint16_t* W_out, int64_t ldw, cudaStream_t s);
+// 2:4 decompress of the 128 x 128 tiles whose tile_map entry is non-zero
+// (tile map ceil(R/128) x ceil(K/128)); other tiles of W_out are not written.
+cudaError_t launch_decompress_tiles(const uint16_t* values, const uint32_t* meta, int64_t R, int64_t K,
+                                    const uint8_t* tile_map, uint16_t* W_out, int64_t ldw, cudaStream_t s);
 cudaError_t launch_gather_rows(const uint16_t* X, int64_t ldx, const int32_t* idx, int64_t K, int64_t T,
                                uint16_t* Xp, int64_t ldp, cudaStream_t s);
 cudaError_t launch_reencode_2of4(const uint16_t* values, const uint32_t* meta, int64_t R, int64_t K, int n, int m,

@@ -23,6 +23,7 @@ struct SpmmParams {
   CUtensorMap tm_vals;  // compressed values R x K*n/m, box {32, 128} 64B swizzle (one SM) or {64, kPairBoxRows} 128B (SM pair)
   CUtensorMap tm_w;     // dense W R x K, box {64, 128}, 128B swizzle (hybrid)
   CUtensorMap tm_x;     // X K x T, box {strip, 64} (one SM) or {64, kPairBoxRows} (SM pair)
+  CUtensorMap tm_wm;    // W under the 2:4 mask (staged), box {64, 64}, 128B swizzle (SM-pair hybrid)
   CUtensorMap tm_y;     // Y R x T bf16, box {64, 32}, 128B swizzle (SM-pair epilogue stores)
   CUtensorMap tm_meta;  // tiled 2:4 metadata {64 words, col blocks, row blocks}, box {64, 1, 8} (SM pair)
   const uint16_t* vals;
@@ -45,6 +46,7 @@ struct SpmmParams {
   int out_f32;
   int tiles_m, tiles_n, num_tiles;
   int hyb_tiles_k;
+  int hyb_rows;  // tile-map rows, ceil(R / 128)
   int stages;
   uint32_t a_slot_bytes;
   // skinny (small T) split-K kernel: K tiles of 128 split into `splits`
@@ -62,6 +64,7 @@ cudaError_t read_and_clear_status(uint32_t* out);
 uint32_t* status_word_ptr();
 bool pair_kernel_fits(const SpmmParams& p);
 cudaError_t launch_spmm_pair(SpmmParams& p, cudaStream_t stream);
+cudaError_t launch_spmm_pair_hybrid(SpmmParams& p, cudaStream_t stream);
 bool skinny_kernel_fits(int64_t T);
 int skinny_bn(int64_t T);
 int skinny_kd(int64_t K, int64_t T);

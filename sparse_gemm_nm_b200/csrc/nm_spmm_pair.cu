@@ -38,30 +38,43 @@ namespace nmk {
 
 namespace pair {
 constexpr int kThreads = 384;  // warps 0,2-5,10,11 copies; 1 MMA; 6-9 epilogue
-constexpr int kStages = 4;
-constexpr uint32_t kA = 16384, kB = 32768, kE = 2048;
+constexpr uint32_t kB = 32768, kE = 2048;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kECol = 256;
 constexpr uint64_t kWaitNs = 2000000000ull;
-constexpr uint32_t kTxPerStage = 2u * (kA + kB + kE);  // both CTAs' A, B and E bytes
 constexpr uint32_t kIdesc = idesc_bf16(256, true, 256);
-
+constexpr uint32_t kIdescDense = idesc_bf16(256, false, 256);
 constexpr uint32_t kEpi = 4096;  // per epilogue warp: 32 rows x 64 bf16 columns, 128-byte swizzle
+
 struct Layout {
   uint32_t a, b, e, epi, bar, total;
 };
-__host__ __device__ constexpr Layout layout() {
-  return Layout{0u, kStages * kA, kStages * (kA + kB), kStages * (kA + kB + kE), kStages * (kA + kB + kE) + 4 * kEpi,
-                kStages * (kA + kB + kE) + 4 * kEpi + (2 * kStages + 4) * 8 + 64};
-}
+// HYB = false: 2:4 only, A slots of 16 KB (compressed values), four stages.
+// HYB = true (PATCH hybrid): A slots of 32 KB so that a stage can hold the
+// dense 128 x 128 tile instead, three stages.
+template <bool HYB>
+struct Cfg {
+  static constexpr int kStages = HYB ? 3 : 4;
+  static constexpr uint32_t kA = HYB ? 32768u : 16384u;
+  static constexpr uint32_t kTxSparse = 2u * (16384u + kB + kE);  // both CTAs' A, B and E bytes
+  static constexpr uint32_t kTxDense = 2u * (32768u + kB);        // both CTAs' dense A and B bytes
+  __host__ __device__ static constexpr Layout layout() {
+    return Layout{0u, kStages * kA, kStages * (kA + kB), kStages * (kA + kB + kE),
+                  kStages * (kA + kB + kE) + 4 * kEpi, kStages * (kA + kB + kE) + 4 * kEpi + (2 * kStages + 4) * 8 + 64};
+  }
+};
 }  // namespace pair
 
+template <bool HYB>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pair::kThreads, 1)
     spmm_pair_kernel(const __grid_constant__ SpmmParams p) {
   using namespace pair;
+  using C = Cfg<HYB>;
+  constexpr int kStages = C::kStages;
+  constexpr uint32_t kA = C::kA;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  constexpr Layout L = layout();
+  constexpr Layout L = C::layout();
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + L.bar);
   uint64_t* empty = full + kStages;
   uint64_t* acc_full = empty + kStages;
@@ -107,6 +120,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pair::kThreads, 1)
   const uint32_t lead_full0 = map_to_cta(smem_u32(&full[0]), 0);
   const uint32_t lead_acc_empty = map_to_cta(smem_u32(acc_empty), 0);
   bool ok = true;
+  // Hybrid: is the 128 x 128 weight tile (row block 2*tm + rr, k block kt) 2:4?
+  // A stage runs the sparse MMA only when both CTAs' tiles are 2:4; otherwise
+  // both CTAs stage dense tiles (W, or W with the 2:4 mask applied).
+  auto tile_sparse = [&](int tm, int64_t kt, int rr) -> bool {
+    if (!HYB) return true;
+    int rb = 2 * tm + rr;
+    if (rb >= p.hyb_rows) rb = 2 * tm;
+    return __ldg(p.tile_map + (int64_t)rb * p.hyb_tiles_k + kt) != 0;
+  };
 
   if (warp < 6 || warp >= 10) {
     if (warp == 1) {
@@ -115,6 +137,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pair::kThreads, 1)
         int s = 0;
         uint32_t ph = 0, aph = 0;
         for (int tile = pair_id; tile < p.num_tiles && ok; tile += npairs) {
+          const int tm = tile % p.tiles_m;
           ok = mbar_wait(acc_empty, aph ^ 1u, abort_flag, p.status, kWaitNs);
           if (!ok) break;
           tc_fence_after();
@@ -125,13 +148,22 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pair::kThreads, 1)
             const uint32_t a_addr = smem_u32(smem + L.a + s * kA);
             const uint32_t b_addr = smem_u32(smem + L.b + s * kB);
             const uint32_t e_tmem = tmem_base + kECol + 4u * s;
-            tc_cp_128x128b_pair(e_tmem, smem_desc(smem_u32(smem + L.e + s * kE), 2048, 128, SWZ_NONE));
+            if (tile_sparse(tm, kt, 0) && tile_sparse(tm, kt, 1)) {
+              tc_cp_128x128b_pair(e_tmem, smem_desc(smem_u32(smem + L.e + s * kE), 2048, 128, SWZ_NONE));
 #pragma unroll
-            for (int kk = 0; kk < 4; ++kk) {
-              const uint64_t ad = smem_desc(a_addr + kk * 32, 16, 1024, SWZ_128B);
-              const uint64_t bd = smem_desc(b_addr + kk * 4096, 16384, 1024, SWZ_128B);
-              tc_mma_sp_pair(tmem_base, ad, bd, e_tmem + (uint32_t)(kk & 2), kIdesc | (uint32_t)(kk & 1),
-                             (kt > 0 || kk > 0) ? 1u : 0u);
+              for (int kk = 0; kk < 4; ++kk) {
+                const uint64_t ad = smem_desc(a_addr + kk * 32, 16, 1024, SWZ_128B);
+                const uint64_t bd = smem_desc(b_addr + kk * 4096, 16384, 1024, SWZ_128B);
+                tc_mma_sp_pair(tmem_base, ad, bd, e_tmem + (uint32_t)(kk & 2), kIdesc | (uint32_t)(kk & 1),
+                               (kt > 0 || kk > 0) ? 1u : 0u);
+              }
+            } else if (HYB) {  // dense A tile: [K half][128 rows][128 B], eight K = 16 MMAs
+#pragma unroll
+              for (int kk = 0; kk < 8; ++kk) {
+                const uint64_t ad = smem_desc(a_addr + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024, SWZ_128B);
+                const uint64_t bd = smem_desc(b_addr + kk * 2048, 16384, 1024, SWZ_128B);
+                tc_mma_pair(tmem_base, ad, bd, kIdescDense, (kt > 0 || kk > 0) ? 1u : 0u);
+              }
             }
             tc_commit_pair(&empty[s], 0x3);
             if (++s == kStages) { s = 0; ph ^= 1u; }
@@ -159,16 +191,25 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pair::kThreads, 1)
             ok = mbar_wait(&empty[s], ph ^ 1u, abort_flag, p.status, kWaitNs);
             if (!ok) break;
             const uint32_t lead_full = lead_full0 + 8u * s;
+            const bool sparse = tile_sparse(tm, kt, 0) && tile_sparse(tm, kt, 1);
             if (warp == 0 || warp == 10) {
               const int h = warp == 10;
-              if (rank == 0 && h == 0) mbar_arrive_expect_tx(&full[s], kTxPerStage);
-              tma_load_2d_pair(smem + L.a + s * kA + h * (kA / 2), &p.tm_vals, lead_full, (int32_t)(kt * 64),
-                               row0 + 64 * h);
+              if (rank == 0 && h == 0) mbar_arrive_expect_tx(&full[s], sparse ? C::kTxSparse : C::kTxDense);
+              if (sparse) {
+                tma_load_2d_pair(smem + L.a + s * kA + h * 8192, &p.tm_vals, lead_full, (int32_t)(kt * 64),
+                                 row0 + 64 * h);
+              } else if (HYB) {  // this CTA's dense tile: W, or W under the 2:4 mask if the tile is 2:4
+                const CUtensorMap* src = tile_sparse(tm, kt, (int)rank) ? &p.tm_wm : &p.tm_w;
+#pragma unroll
+                for (int kh = 0; kh < 2; ++kh)
+                  tma_load_2d_pair(smem + L.a + s * kA + kh * 16384 + h * 8192, src, lead_full,
+                                   (int32_t)(kt * 128 + 64 * kh), row0 + 64 * h);
+              }
             } else if (warp <= 5) {  // box (strip j, K half h): 64 columns x 64 rows of X
               const int j = (warp - 2) >> 1, h = (warp - 2) & 1;
               tma_load_2d_pair(smem + L.b + s * kB + j * 16384 + h * 8192, &p.tm_x, lead_full, col0 + 64 * j,
                                (int32_t)(kt * 128 + 64 * h));
-            } else {  // eight 16-row metadata blocks of column block kt
+            } else if (sparse) {  // eight 16-row metadata blocks of column block kt
               tma_load_3d_pair(smem + L.e + s * kE, &p.tm_meta, lead_full, 0, (int32_t)kt, row0 / 16);
             }
             if (++s == kStages) { s = 0; ph ^= 1u; }
@@ -274,22 +315,27 @@ bool pair_kernel_fits(const SpmmParams& p) {
   return p.a_mode == A_TMA_SPARSE && p.K % 128 == 0 && p.K > 0 && p.T >= 192 && p.R >= 1 && p.T % 8 == 0;
 }
 
-cudaError_t launch_spmm_pair(SpmmParams& p, cudaStream_t stream) {
-  constexpr pair::Layout L = pair::layout();
+template <bool HYB>
+static cudaError_t launch_pair(SpmmParams& p, cudaStream_t stream) {
+  constexpr pair::Layout L = pair::Cfg<HYB>::layout();
   const size_t bytes = L.total + 1024;
   static bool configured[64] = {};
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 64 && !configured[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(spmm_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+    cudaError_t e = cudaFuncSetAttribute(spmm_pair_kernel<HYB>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
     if (e != cudaSuccess) return e;
     configured[dev] = true;
   }
   const int pairs_avail = sm_count_current() / 2;
   const int pairs = p.num_tiles < pairs_avail ? p.num_tiles : pairs_avail;
-  spmm_pair_kernel<<<2 * pairs, pair::kThreads, bytes, stream>>>(p);
+  spmm_pair_kernel<HYB><<<2 * pairs, pair::kThreads, bytes, stream>>>(p);
   count_launch();
   return cudaGetLastError();
 }
+
+cudaError_t launch_spmm_pair(SpmmParams& p, cudaStream_t stream) { return launch_pair<false>(p, stream); }
+
+cudaError_t launch_spmm_pair_hybrid(SpmmParams& p, cudaStream_t stream) { return launch_pair<true>(p, stream); }
 
 }  // namespace nmk

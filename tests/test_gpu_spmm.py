@@ -371,3 +371,27 @@ def test_skinny_kernel_integer_exact(out):
         assert np.array_equal(Y.cpu().numpy().astype(np.float64), ref)
     else:
         assert np.array_equal(bits(Y), bf16_rne_of(ref))
+
+
+# ----------------------------------------------------------------------------
+# PATCH hybrid on SM pairs (K % 128 == 0, T >= 192): mixed stages run dense
+# ----------------------------------------------------------------------------
+@pytest.mark.parametrize("p", [0.25, 0.75])
+def test_hybrid_pair_ragged(p):
+    R, K, T = 300, 384, 264
+    W = wl.normal_bf16((R, K), 0.02, seed=171)
+    X = wl.normal_bf16((K, T), 1.0, seed=172)
+    tm = wl.tile_map(3, 3, p, seed=173)
+    Y = run_hybrid(W, X, tm)
+    ref, mag = oracle.hybrid_spmm(W, tm, X, 128, with_abs=True)
+    assert_gemm_close(values_f64(Y), ref, mag, f"hybrid pair p={p}")
+
+
+def test_hybrid_pair_integer_exact():
+    R, K, T = 512, 512, 256
+    W = wl.integer_bf16((R, K), -8, 8, seed=181)
+    X = wl.integer_bf16((K, T), -8, 8, seed=182)
+    tm = wl.tile_map(4, 4, 0.5, seed=183)
+    Y = run_hybrid(W, X, tm)
+    ref = oracle.hybrid_spmm(W, tm, X, 128)
+    assert np.array_equal(bits(Y), bf16_rne_of(ref))
