@@ -290,6 +290,7 @@ __global__ void __launch_bounds__(256) gather_rows_kernel(const uint16_t* __rest
   const int64_t warp = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) >> 5;
   const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
   const int64_t pieces = T >> 3;  // 16-byte pieces per row
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");  // the GEMM may start its setup
   for (int64_t k = warp; k < K; k += nwarps) {
     const int32_t src = __ldg(idx + k);
     const bool valid = src >= 0 && (int64_t)src < K;
@@ -327,6 +328,7 @@ __global__ void __launch_bounds__(256) reencode_2of4_kernel(const uint16_t* __re
   constexpr int B = M == 2 ? 1 : M == 4 ? 2 : 3;
   constexpr int S = 32 / B;
   const uint32_t chunks = cblocks * 8;
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");  // the GEMM may start its setup
   for (uint32_t t = blockIdx.x * blockDim.x + threadIdx.x; t < total; t += gridDim.x * blockDim.x) {
     const uint32_t r = t / chunks, c = t - r * chunks;
     const uint32_t cb = c >> 3, qh = c & 7u;  // block column 16*qh = 32q + 16h

@@ -181,6 +181,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pair::kThreads, 1)
     } else {
       // ------ copy issuers: warps 0/10 A halves, warps 2-5 B boxes, warp 11 metadata (E)
       if (lane == 0) {
+        // When launched as a programmatic dependent of a staging pass (gather or
+        // re-encode), its outputs are visible only after this wait; otherwise a no-op.
+        asm volatile("griddepcontrol.wait;" ::: "memory");
         int s = 0;
         uint32_t ph = 0;
         for (int tile = pair_id; tile < p.num_tiles && ok; tile += npairs) {
@@ -316,7 +319,7 @@ bool pair_kernel_fits(const SpmmParams& p) {
 }
 
 template <bool HYB>
-static cudaError_t launch_pair(SpmmParams& p, cudaStream_t stream) {
+static cudaError_t launch_pair(SpmmParams& p, cudaStream_t stream, bool pdl) {
   constexpr pair::Layout L = pair::Cfg<HYB>::layout();
   const size_t bytes = L.total + 1024;
   static bool configured[64] = {};
@@ -329,13 +332,23 @@ static cudaError_t launch_pair(SpmmParams& p, cudaStream_t stream) {
   }
   const int pairs_avail = sm_count_current() / 2;
   const int pairs = p.num_tiles < pairs_avail ? p.num_tiles : pairs_avail;
-  spmm_pair_kernel<HYB><<<2 * pairs, pair::kThreads, bytes, stream>>>(p);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2 * pairs);
+  cfg.blockDim = dim3(pair::kThreads);
+  cfg.dynamicSmemBytes = bytes;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, spmm_pair_kernel<HYB>, p);
   count_launch();
-  return cudaGetLastError();
+  return e != cudaSuccess ? e : cudaGetLastError();
 }
 
-cudaError_t launch_spmm_pair(SpmmParams& p, cudaStream_t stream) { return launch_pair<false>(p, stream); }
+cudaError_t launch_spmm_pair(SpmmParams& p, cudaStream_t stream, bool pdl) { return launch_pair<false>(p, stream, pdl); }
 
-cudaError_t launch_spmm_pair_hybrid(SpmmParams& p, cudaStream_t stream) { return launch_pair<true>(p, stream); }
+cudaError_t launch_spmm_pair_hybrid(SpmmParams& p, cudaStream_t stream) { return launch_pair<true>(p, stream, true); }
 
 }  // namespace nmk
