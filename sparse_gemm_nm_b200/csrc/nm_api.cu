@@ -445,7 +445,7 @@ static nm_status run_gemm(const GemmRequest& q, cudaStream_t stream) {
     if (st == NM_OK && !use_skinny && !p.out_f32)
       st = make_tmap(&p.tm_y, q.Y, (uint64_t)q.T, (uint64_t)q.R, (uint64_t)q.ldy * 2, 64, 32, 128, "Y");
     if (st == NM_OK)
-      e = use_skinny ? launch_spmm_skinny(p, stream) : launch_spmm_pair(p, stream, staged || staged_a);
+      e = use_skinny ? launch_spmm_skinny(p, stream) : launch_spmm_pair(p, stream);
     if (ws) cudaFreeAsync(ws, stream);
     release();
     if (st != NM_OK) return st;

@@ -64,6 +64,7 @@ __global__ void __launch_bounds__(256, 4) compress_2of4_tiled_kernel(const uint1
                                                                   uint16_t* __restrict__ V,
                                                                   uint32_t* __restrict__ meta, uint32_t cblocks,
                                                                   uint32_t nblocks, bool vec) {
+  pdl_gate();
   const uint32_t lane = threadIdx.x & 31u;
   const uint32_t warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const uint32_t nwarps = (gridDim.x * blockDim.x) >> 5;
@@ -141,6 +142,7 @@ __global__ void __launch_bounds__(256) compress_generic_kernel(const uint16_t* _
                                                                int64_t K, int64_t ldw, int n,
                                                                uint16_t* __restrict__ V,
                                                                uint32_t* __restrict__ meta) {
+  pdl_gate();
   constexpr int B = M == 2 ? 1 : M == 4 ? 2 : M == 8 ? 3 : 4;
   constexpr int S = 32 / B;
   const int64_t vcols = K / M * n;
@@ -219,6 +221,7 @@ __global__ void __launch_bounds__(256) decompress_2of4_tiled_kernel(const uint16
                                                                     uint32_t K, uint16_t* __restrict__ W,
                                                                     int64_t ldw, uint32_t cblocks, uint32_t total,
                                                                     bool vec, const uint8_t* __restrict__ tile_map) {
+  pdl_gate();
   for (uint32_t w = blockIdx.x * blockDim.x + threadIdx.x; w < total; w += gridDim.x * blockDim.x) {
     const uint32_t blk = w >> 6, wi = w & 63u;
     const uint32_t l = wi >> 2, q = wi & 3u;
@@ -242,6 +245,7 @@ __global__ void __launch_bounds__(256) decompress_generic_kernel(const uint16_t*
                                                                  const uint32_t* __restrict__ meta, int64_t R,
                                                                  int64_t K, int n, uint16_t* __restrict__ W,
                                                                  int64_t ldw) {
+  pdl_gate();
   constexpr int B = M == 2 ? 1 : M == 4 ? 2 : M == 8 ? 3 : 4;
   constexpr int S = 32 / B;
   const int64_t groups = K / M;
@@ -271,6 +275,7 @@ __global__ void __launch_bounds__(256) decompress_generic_kernel(const uint16_t*
 }
 
 __global__ void fill_zero_kernel(uint8_t* Y, int64_t R, int64_t row_bytes, int64_t ld_bytes) {
+  pdl_gate();
   const int64_t total = R * row_bytes;
   for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < total;
        i += (int64_t)gridDim.x * blockDim.x) {
@@ -279,35 +284,43 @@ __global__ void fill_zero_kernel(uint8_t* Y, int64_t R, int64_t row_bytes, int64
   }
 }
 
-// Row gather Xp[k][0..T) = X[idx[k]][0..T): one warp per row, 16-byte pieces,
-// all of a lane's pieces loaded before any is stored.  Entries of idx outside
-// [0, K) give zero rows.  X and Xp rows are 16-byte aligned (T % 8 == 0 on
-// the vector path).
+// Row gather Xp[k][0..T) = X[idx[k]][0..T).  Work items are (row, 4 KB chunk)
+// pairs so that long rows (large T) spread over many warps; a warp loads its
+// chunk as 8 x 16 bytes per lane, all in flight, then stores it.  Entries of
+// idx outside [0, K) give zero rows.  X and Xp rows are 16-byte aligned
+// (T % 8 == 0).  Persistent grid of kGatherCtasPerSm CTAs per SM (the dynamic
+// shared memory it requests, unused, caps residency there): as a programmatic
+// dependent the kernel is placed on SMs while the previous kernel drains, and
+// without the cap all of it could land on the first few SMs to free up.
+constexpr int kGatherCtasPerSm = 4;
+constexpr size_t kGatherSmemCap = 56 * 1024;
+
 __global__ void __launch_bounds__(256) gather_rows_kernel(const uint16_t* __restrict__ X, int64_t ldx,
                                                           const int32_t* __restrict__ idx, int64_t K, int64_t T,
                                                           uint16_t* __restrict__ Xp, int64_t ldp) {
+  pdl_gate();
   const int lane = threadIdx.x & 31;
   const int64_t warp = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) >> 5;
   const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
-  const int64_t pieces = T >> 3;  // 16-byte pieces per row
-  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");  // the GEMM may start its setup
-  for (int64_t k = warp; k < K; k += nwarps) {
+  const int64_t pieces = T >> 3;                    // 16-byte pieces per row
+  const int64_t chunks = (pieces + 255) / 256;      // 4 KB chunks per row
+  const int64_t items = K * chunks;
+  for (int64_t it = warp; it < items; it += nwarps) {
+    const int64_t k = it / chunks, c0 = (it - k * chunks) * 256;
     const int32_t src = __ldg(idx + k);
     const bool valid = src >= 0 && (int64_t)src < K;
     const uint4* in = reinterpret_cast<const uint4*>(X + (valid ? (int64_t)src : 0) * ldx);
     uint4* out = reinterpret_cast<uint4*>(Xp + k * ldp);
-    for (int64_t c0 = 0; c0 < pieces; c0 += 32 * 8) {
-      uint4 v[8];
+    uint4 v[8];
 #pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        const int64_t c = c0 + u * 32 + lane;
-        v[u] = (valid && c < pieces) ? __ldg(in + c) : make_uint4(0, 0, 0, 0);
-      }
+    for (int u = 0; u < 8; ++u) {
+      const int64_t c = c0 + u * 32 + lane;
+      v[u] = (valid && c < pieces) ? __ldg(in + c) : make_uint4(0, 0, 0, 0);
+    }
 #pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        const int64_t c = c0 + u * 32 + lane;
-        if (c < pieces) out[c] = v[u];
-      }
+    for (int u = 0; u < 8; ++u) {
+      const int64_t c = c0 + u * 32 + lane;
+      if (c < pieces) out[c] = v[u];
     }
   }
 }
@@ -325,10 +338,10 @@ __global__ void __launch_bounds__(256) reencode_2of4_kernel(const uint16_t* __re
                                                             uint32_t K, int n, uint32_t vcols, uint32_t mcols,
                                                             uint16_t* __restrict__ V2, uint16_t* __restrict__ meta2,
                                                             uint32_t cblocks, uint32_t total) {
+  pdl_gate();
   constexpr int B = M == 2 ? 1 : M == 4 ? 2 : 3;
   constexpr int S = 32 / B;
   const uint32_t chunks = cblocks * 8;
-  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");  // the GEMM may start its setup
   for (uint32_t t = blockIdx.x * blockDim.x + threadIdx.x; t < total; t += gridDim.x * blockDim.x) {
     const uint32_t r = t / chunks, c = t - r * chunks;
     const uint32_t cb = c >> 3, qh = c & 7u;  // block column 16*qh = 32q + 16h
@@ -387,16 +400,16 @@ cudaError_t launch_compress(const uint16_t* W, int64_t R, int64_t K, int64_t ldw
   if (tiled_meta(n, m)) {
     const int64_t nblocks = meta_row_blocks(R) * meta_col_blocks(K);
     const bool vec = K % 8 == 0 && ldw % 8 == 0 && aligned16(W) && aligned16(values);
-    compress_2of4_tiled_kernel<<<grid_for(nblocks * 32, threads), threads, 0, s>>>(
+    launch_pdl(compress_2of4_tiled_kernel, grid_for(nblocks * 32, threads), threads, 0, s,
         W, (uint32_t)R, (uint32_t)K, ldw, values, meta, (uint32_t)meta_col_blocks(K), (uint32_t)nblocks, vec);
   } else {
     const int64_t work = R * meta_cols(K, n, m);
     const int grid = grid_for(work, threads);
     switch (m) {
-      case 2: compress_generic_kernel<2><<<grid, threads, 0, s>>>(W, R, K, ldw, n, values, meta); break;
-      case 4: compress_generic_kernel<4><<<grid, threads, 0, s>>>(W, R, K, ldw, n, values, meta); break;
-      case 8: compress_generic_kernel<8><<<grid, threads, 0, s>>>(W, R, K, ldw, n, values, meta); break;
-      default: compress_generic_kernel<16><<<grid, threads, 0, s>>>(W, R, K, ldw, n, values, meta); break;
+      case 2: launch_pdl(compress_generic_kernel<2>, grid, threads, 0, s, W, R, K, ldw, n, values, meta); break;
+      case 4: launch_pdl(compress_generic_kernel<4>, grid, threads, 0, s, W, R, K, ldw, n, values, meta); break;
+      case 8: launch_pdl(compress_generic_kernel<8>, grid, threads, 0, s, W, R, K, ldw, n, values, meta); break;
+      default: launch_pdl(compress_generic_kernel<16>, grid, threads, 0, s, W, R, K, ldw, n, values, meta); break;
     }
   }
   count_launch();
@@ -409,17 +422,17 @@ cudaError_t launch_decompress(const uint16_t* values, const uint32_t* meta, int6
   if (tiled_meta(n, m)) {
     const int64_t total = meta_words(R, K, n, m);
     const bool vec = K % 16 == 0 && ldw % 8 == 0 && aligned16(W_out) && aligned16(values);
-    decompress_2of4_tiled_kernel<<<grid_for(total, threads), threads, 0, s>>>(
+    launch_pdl(decompress_2of4_tiled_kernel, grid_for(total, threads), threads, 0, s,
         values, meta, (uint32_t)R, (uint32_t)K, W_out, ldw, (uint32_t)meta_col_blocks(K), (uint32_t)total, vec,
         nullptr);
   } else {
     const int64_t work = R * (K / m);
     const int grid = grid_for(work, threads);
     switch (m) {
-      case 2: decompress_generic_kernel<2><<<grid, threads, 0, s>>>(values, meta, R, K, n, W_out, ldw); break;
-      case 4: decompress_generic_kernel<4><<<grid, threads, 0, s>>>(values, meta, R, K, n, W_out, ldw); break;
-      case 8: decompress_generic_kernel<8><<<grid, threads, 0, s>>>(values, meta, R, K, n, W_out, ldw); break;
-      default: decompress_generic_kernel<16><<<grid, threads, 0, s>>>(values, meta, R, K, n, W_out, ldw); break;
+      case 2: launch_pdl(decompress_generic_kernel<2>, grid, threads, 0, s, values, meta, R, K, n, W_out, ldw); break;
+      case 4: launch_pdl(decompress_generic_kernel<4>, grid, threads, 0, s, values, meta, R, K, n, W_out, ldw); break;
+      case 8: launch_pdl(decompress_generic_kernel<8>, grid, threads, 0, s, values, meta, R, K, n, W_out, ldw); break;
+      default: launch_pdl(decompress_generic_kernel<16>, grid, threads, 0, s, values, meta, R, K, n, W_out, ldw); break;
     }
   }
   count_launch();
@@ -431,7 +444,7 @@ cudaError_t launch_decompress_tiles(const uint16_t* values, const uint32_t* meta
   const int threads = 256;
   const int64_t total = meta_words(R, K, 2, 4);
   const bool vec = K % 16 == 0 && ldw % 8 == 0 && aligned16(W_out) && aligned16(values);
-  decompress_2of4_tiled_kernel<<<grid_for(total, threads), threads, 0, s>>>(
+  launch_pdl(decompress_2of4_tiled_kernel, grid_for(total, threads), threads, 0, s,
       values, meta, (uint32_t)R, (uint32_t)K, W_out, ldw, (uint32_t)meta_col_blocks(K), (uint32_t)total, vec,
       tile_map);
   count_launch();
@@ -441,14 +454,27 @@ cudaError_t launch_decompress_tiles(const uint16_t* values, const uint32_t* meta
 cudaError_t launch_gather_rows(const uint16_t* X, int64_t ldx, const int32_t* idx, int64_t K, int64_t T,
                                uint16_t* Xp, int64_t ldp, cudaStream_t s) {
   const int threads = 256;
-  gather_rows_kernel<<<grid_for(K * 32, threads), threads, 0, s>>>(X, ldx, idx, K, T, Xp, ldp);
+  static bool configured[64] = {};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev >= 0 && dev < 64 && !configured[dev]) {
+    cudaError_t e = cudaFuncSetAttribute(gather_rows_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)kGatherSmemCap);
+    if (e != cudaSuccess) return e;
+    configured[dev] = true;
+  }
+  const int64_t items = K * ((T / 8 + 255) / 256);
+  const int64_t want = (items + 7) / 8;  // 8 warps per CTA
+  const int64_t cap = (int64_t)sm_count_current() * kGatherCtasPerSm;
+  const int grid = (int)(want < cap ? (want > 0 ? want : 1) : cap);
+  cudaError_t e = launch_pdl(gather_rows_kernel, grid, threads, kGatherSmemCap, s, X, ldx, idx, K, T, Xp, ldp);
   count_launch();
-  return cudaGetLastError();
+  return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 cudaError_t launch_fill_zero(void* Y, int64_t R, int64_t T, int64_t ldy, int esize, cudaStream_t s) {
   const int threads = 256;
-  fill_zero_kernel<<<grid_for(R * T * esize, threads), threads, 0, s>>>(static_cast<uint8_t*>(Y), R, T * esize,
+  launch_pdl(fill_zero_kernel, grid_for(R * T * esize, threads), threads, 0, s, static_cast<uint8_t*>(Y), R, T * esize,
                                                                          ldy * esize);
   count_launch();
   return cudaGetLastError();
@@ -463,11 +489,11 @@ cudaError_t launch_reencode_2of4(const uint16_t* values, const uint32_t* meta, i
   const uint32_t vcols = (uint32_t)value_cols(K, n, m), mcols = (uint32_t)meta_cols(K, n, m);
   uint16_t* m16 = reinterpret_cast<uint16_t*>(meta2);
   switch (m) {
-    case 2: reencode_2of4_kernel<2><<<grid, threads, 0, s>>>(values, meta, (uint32_t)R, (uint32_t)K, n, vcols, mcols,
+    case 2: launch_pdl(reencode_2of4_kernel<2>, grid, threads, 0, s, values, meta, (uint32_t)R, (uint32_t)K, n, vcols, mcols,
                                                                 values2, m16, (uint32_t)cblocks, (uint32_t)total); break;
-    case 4: reencode_2of4_kernel<4><<<grid, threads, 0, s>>>(values, meta, (uint32_t)R, (uint32_t)K, n, vcols, mcols,
+    case 4: launch_pdl(reencode_2of4_kernel<4>, grid, threads, 0, s, values, meta, (uint32_t)R, (uint32_t)K, n, vcols, mcols,
                                                                 values2, m16, (uint32_t)cblocks, (uint32_t)total); break;
-    case 8: reencode_2of4_kernel<8><<<grid, threads, 0, s>>>(values, meta, (uint32_t)R, (uint32_t)K, n, vcols, mcols,
+    case 8: launch_pdl(reencode_2of4_kernel<8>, grid, threads, 0, s, values, meta, (uint32_t)R, (uint32_t)K, n, vcols, mcols,
                                                                 values2, m16, (uint32_t)cblocks, (uint32_t)total); break;
     default: return cudaErrorInvalidValue;
   }

@@ -2,6 +2,7 @@
 // kernel launchers of libnm_b200 (not part of the public ABI).
 #pragma once
 #include <cstdint>
+#include <utility>
 #include <cuda_runtime.h>
 
 namespace nmk {
@@ -27,6 +28,35 @@ inline int64_t meta_words(int64_t R, int64_t K, int n, int m) {
 // Patterns whose survivors never exceed two per aligned group of four, so a
 // tile of them can be re-encoded as 2:4 for the sparse MMA.
 inline bool fits_2of4(int n, int m) { return (m == 2 && n == 1) || ((m == 4 || m == 8) && n <= 2); }
+
+// Every kernel of the library is launched as a programmatic dependent of the
+// previous kernel in its stream and starts with pdl_gate(): it waits until
+// that kernel has completed and its writes are visible (griddepcontrol.wait),
+// touching no global memory before, then lets its own successor be scheduled.
+// Stream order is unchanged; the successor's launch and setup overlap the tail
+// of the kernel before it.
+#ifdef __CUDACC__
+__device__ __forceinline__ void pdl_gate() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+#endif
+
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                              Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
 
 int sm_count_current();
 void count_launch();

@@ -273,6 +273,7 @@ __global__ void __launch_bounds__(kThreads, 1) spmm_kernel(const __grid_constant
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  pdl_gate();  // no global memory touched before this point
 
   const int64_t k_tiles = p.k_tiles;
   bool ok = true;
@@ -578,8 +579,8 @@ static cudaError_t launch_bn(const SpmmParams& p, int grid, cudaStream_t stream)
     if (e != cudaSuccess) return e;
     configured[dev] = true;
   }
-  spmm_kernel<BN><<<grid, kThreads, bytes, stream>>>(p);
-  return cudaGetLastError();
+  cudaError_t e = launch_pdl(spmm_kernel<BN>, dim3(grid), dim3(kThreads), bytes, stream, p);
+  return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 int spmm_max_stages(int bn, uint32_t a_slot) {

@@ -63,9 +63,7 @@ cudaError_t launch_spmm(SpmmParams& p, int bn, cudaStream_t stream);
 cudaError_t read_and_clear_status(uint32_t* out);
 uint32_t* status_word_ptr();
 bool pair_kernel_fits(const SpmmParams& p);
-// pdl: launch as a programmatic dependent of the previous kernel (a staging pass
-// of the same call), so that launch and setup overlap its tail.
-cudaError_t launch_spmm_pair(SpmmParams& p, cudaStream_t stream, bool pdl = false);
+cudaError_t launch_spmm_pair(SpmmParams& p, cudaStream_t stream);
 cudaError_t launch_spmm_pair_hybrid(SpmmParams& p, cudaStream_t stream);
 bool skinny_kernel_fits(int64_t T);
 int skinny_bn(int64_t T);

@@ -115,6 +115,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pair::kThreads, 1)
   cluster_sync();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  pdl_gate();  // no global memory touched before this point
 
   const int64_t k_tiles = p.K / 128;
   const uint32_t lead_full0 = map_to_cta(smem_u32(&full[0]), 0);
@@ -181,9 +182,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pair::kThreads, 1)
     } else {
       // ------ copy issuers: warps 0/10 A halves, warps 2-5 B boxes, warp 11 metadata (E)
       if (lane == 0) {
-        // When launched as a programmatic dependent of a staging pass (gather or
-        // re-encode), its outputs are visible only after this wait; otherwise a no-op.
-        asm volatile("griddepcontrol.wait;" ::: "memory");
         int s = 0;
         uint32_t ph = 0;
         for (int tile = pair_id; tile < p.num_tiles && ok; tile += npairs) {
@@ -319,7 +317,7 @@ bool pair_kernel_fits(const SpmmParams& p) {
 }
 
 template <bool HYB>
-static cudaError_t launch_pair(SpmmParams& p, cudaStream_t stream, bool pdl) {
+static cudaError_t launch_pair(SpmmParams& p, cudaStream_t stream) {
   constexpr pair::Layout L = pair::Cfg<HYB>::layout();
   const size_t bytes = L.total + 1024;
   static bool configured[64] = {};
@@ -332,23 +330,13 @@ static cudaError_t launch_pair(SpmmParams& p, cudaStream_t stream, bool pdl) {
   }
   const int pairs_avail = sm_count_current() / 2;
   const int pairs = p.num_tiles < pairs_avail ? p.num_tiles : pairs_avail;
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(2 * pairs);
-  cfg.blockDim = dim3(pair::kThreads);
-  cfg.dynamicSmemBytes = bytes;
-  cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = pdl ? 1 : 0;
-  cudaError_t e = cudaLaunchKernelEx(&cfg, spmm_pair_kernel<HYB>, p);
+  cudaError_t e = launch_pdl(spmm_pair_kernel<HYB>, dim3(2 * pairs), dim3(pair::kThreads), bytes, stream, p);
   count_launch();
   return e != cudaSuccess ? e : cudaGetLastError();
 }
 
-cudaError_t launch_spmm_pair(SpmmParams& p, cudaStream_t stream, bool pdl) { return launch_pair<false>(p, stream, pdl); }
+cudaError_t launch_spmm_pair(SpmmParams& p, cudaStream_t stream) { return launch_pair<false>(p, stream); }
 
-cudaError_t launch_spmm_pair_hybrid(SpmmParams& p, cudaStream_t stream) { return launch_pair<true>(p, stream, true); }
+cudaError_t launch_spmm_pair_hybrid(SpmmParams& p, cudaStream_t stream) { return launch_pair<true>(p, stream); }
 
 }  // namespace nmk

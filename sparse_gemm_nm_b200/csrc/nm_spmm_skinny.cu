@@ -106,9 +106,7 @@ __global__ void __launch_bounds__(skinny::kThreads, 1) spmm_skinny_kernel(const 
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
   bool ok = true;
-  // The reduce kernel that follows (when K is split) may be scheduled now; it
-  // waits for this grid to finish before it reads anything.
-  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  pdl_gate();  // no global memory touched before this point
 
   auto unit_range = [&](int u, int& tm, int64_t& kt0, int64_t& kt1) {
     tm = u % p.tiles_m;
@@ -263,7 +261,7 @@ __global__ void __launch_bounds__(skinny::kThreads, 1) spmm_skinny_kernel(const 
 // and waits (griddepcontrol.wait) for the GEMM's writes before reading ws.
 __global__ void __launch_bounds__(256) skinny_reduce_kernel(const float* __restrict__ ws, int splits, int64_t R,
                                                             int bn, int64_t T, void* Y, int64_t ldy, int out_f32) {
-  asm volatile("griddepcontrol.wait;" ::: "memory");
+  pdl_gate();
   const int64_t total = R * T;
   for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < total; i += (int64_t)gridDim.x * blockDim.x) {
     const int64_t r = i / T, t = i - r * T;
@@ -293,9 +291,10 @@ static cudaError_t launch_bn(SpmmParams& p, cudaStream_t stream) {
   }
   const int units = p.tiles_m * p.splits;
   const int sms = sm_count_current();
-  spmm_skinny_kernel<BN, KD><<<units < sms ? units : sms, kThreads, bytes, stream>>>(p);
+  cudaError_t e = launch_pdl(spmm_skinny_kernel<BN, KD>, dim3(units < sms ? units : sms), dim3(kThreads), bytes,
+                             stream, p);
   count_launch();
-  cudaError_t e = cudaGetLastError();
+  if (e == cudaSuccess) e = cudaGetLastError();
   if (e != cudaSuccess || p.splits == 1) return e;
   const int64_t total = p.R * p.T;
   const int64_t want = (total + 255) / 256;
