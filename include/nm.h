@@ -221,6 +221,19 @@ NM_API nm_status nm_spmm_algo(const uint16_t* values, const uint32_t* meta, int 
 NM_API nm_status nm_release_staging(void);
 
 /*
+ * nm_selftest_wait_timeout -- exercise the failure-reporting path.  The pages
+ * have no counterpart to this call; it exists so that the bounded waits of the
+ * kernels can be tested without a fault.  It launches one block on `stream`
+ * in which a thread waits, with the same bounded wait the GEMM kernels use, on
+ * a barrier that nothing completes; after limit_us microseconds (1..1000000)
+ * the wait gives up and records a timeout in the device status word, and the
+ * kernel returns.  The next nm_device_status(stream) returns NM_ERR_TIMEOUT
+ * (and clears the word); the context stays usable.
+ * Errors: NM_ERR_INVALID_ARG (limit out of range), NM_ERR_NO_DEVICE, NM_ERR_CUDA.
+ */
+NM_API nm_status nm_selftest_wait_timeout(uint32_t limit_us, void* stream);
+
+/*
  * nm_spmm_permuted_noalloc -- nm_spmm_permuted without any device allocation.
  * The pages have no counterpart to this call; it exists for callers that
  * cannot let a library allocate device memory: runtimes that budget every

@@ -51,6 +51,7 @@ SIGNATURES = {
     "nm_spmm_algo": ([_P, _P, _I, _I, _I64, _I64, _P, _P, _I64, _I64, _P, _I64, _I, _I, _P], _I),
     "nm_spmm_permuted_noalloc": ([_P, _P, _I, _I, _I64, _I64, _P, _P, _I64, _I64, _P, _I64, _I, _P], _I),
     "nm_release_staging": ([], _I),
+    "nm_selftest_wait_timeout": ([ctypes.c_uint32, _P], _I),
     "nm_device_status": ([_P], _I),
     "nm_status_string": ([_I], ctypes.c_char_p),
     "nm_last_error": ([], ctypes.c_char_p),
@@ -164,6 +165,10 @@ def nm_spmm_permuted_noalloc(values, meta, n, m, R, K, idx, X, ldx, T, Y, ldy, y
                              stream=None) -> None:
     _check(lib().nm_spmm_permuted_noalloc(_ptr(values), _ptr(meta), n, m, R, K, _ptr(idx), _ptr(X), ldx, T,
                                           _ptr(Y), ldy, y_dtype, _stream(stream)), "nm_spmm_permuted_noalloc")
+
+
+def nm_selftest_wait_timeout(limit_us: int, stream=None) -> None:
+    _check(lib().nm_selftest_wait_timeout(limit_us, _stream(stream)), "nm_selftest_wait_timeout")
 
 
 def nm_release_staging() -> None:

@@ -695,6 +695,15 @@ uint64_t nm_launch_count(void) { return g_launches.load(std::memory_order_relaxe
 
 int nm_version(void) { return 100; }
 
+nm_status nm_selftest_wait_timeout(uint32_t limit_us, void* stream) {
+  t_last_error.clear();
+  if (limit_us < 1 || limit_us > 1000000) return fail(NM_ERR_INVALID_ARG, "limit_us must be in [1, 1000000]");
+  nm_status st = require_device();
+  if (st != NM_OK) return st;
+  cudaError_t e = launch_selftest_wait((uint64_t)limit_us * 1000ull, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? NM_OK : cuda_fail(e, "self-test launch");
+}
+
 nm_status nm_release_staging(void) {
   set_last_error("");
   std::lock_guard<std::mutex> lk(g_pool_mu);

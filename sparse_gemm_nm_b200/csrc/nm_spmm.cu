@@ -617,6 +617,29 @@ cudaError_t launch_spmm(SpmmParams& p, int bn, cudaStream_t stream) {
   return e;
 }
 
+// Self-test of the failure path: one thread waits, with the library's bounded
+// wait, on a barrier that nothing completes; the wait gives up after limit_ns
+// and records the timeout in the status word.  Nothing else is touched.
+__global__ void selftest_wait_kernel(uint32_t* status, uint64_t limit_ns) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    abort_flag = 0;
+    fence_barrier_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) mbar_wait(&bar, 0, &abort_flag, status, limit_ns);
+}
+
+cudaError_t launch_selftest_wait(uint64_t limit_ns, cudaStream_t stream) {
+  uint32_t* st = status_word_ptr();
+  if (!st) return cudaErrorInvalidSymbol;
+  selftest_wait_kernel<<<1, 32, 0, stream>>>(st, limit_ns);
+  count_launch();
+  return cudaGetLastError();
+}
+
 cudaError_t read_and_clear_status(uint32_t* out) {
   uint32_t zero = 0;
   cudaError_t e = cudaMemcpyFromSymbol(out, g_status, sizeof(uint32_t));

@@ -61,6 +61,7 @@ struct SpmmParams {
 int spmm_max_stages(int bn, uint32_t a_slot);
 cudaError_t launch_spmm(SpmmParams& p, int bn, cudaStream_t stream);
 cudaError_t read_and_clear_status(uint32_t* out);
+cudaError_t launch_selftest_wait(uint64_t limit_ns, cudaStream_t stream);
 uint32_t* status_word_ptr();
 bool pair_kernel_fits(const SpmmParams& p);
 cudaError_t launch_spmm_pair(SpmmParams& p, cudaStream_t stream);

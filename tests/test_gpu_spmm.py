@@ -395,3 +395,20 @@ def test_hybrid_pair_integer_exact():
     Y = run_hybrid(W, X, tm)
     ref = oracle.hybrid_spmm(W, tm, X, 128)
     assert np.array_equal(bits(Y), bf16_rne_of(ref))
+
+
+# ----------------------------------------------------------------------------
+# Failure path: a bounded wait that runs out is reported, the context stays usable
+# ----------------------------------------------------------------------------
+def test_bounded_wait_timeout_is_reported():
+    nm.nm_device_status()  # start from a clear status word
+    nm.nm_selftest_wait_timeout(20000)  # 20 ms on a barrier that nothing completes
+    with pytest.raises(nm.NmError) as e:
+        nm.nm_device_status()
+    assert e.value.status == nm.NM_ERR_TIMEOUT
+    nm.nm_device_status()  # the word was cleared by the read
+    # the context still runs kernels correctly
+    R, K, T = 256, 512, 256
+    W = wl.normal_bf16((R, K), 0.02, seed=191)
+    X = wl.normal_bf16((K, T), 1.0, seed=192)
+    check(W, X, 2, 4, what="after a reported timeout")
