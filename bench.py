@@ -168,6 +168,24 @@ def cpu_baseline(data, target_s: float):
                       f"single thread)"}
 
 
+# ----------------------------------------------------------------------------
+# Multi-rank plumbing (one process per GPU; replicas, no data-path collective)
+# ----------------------------------------------------------------------------
+def rank_barrier(dist) -> None:
+    if dist is not None:
+        dist.barrier()
+
+
+def max_over_ranks_on(ms: float, dist, device) -> float:
+    """The slowest rank's time: all-reduce MAX of one float64 (NCCL on the GPU, gloo on the CPU)."""
+    if dist is None:
+        return ms
+    import torch
+    t = torch.tensor([ms], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
 def run_reference(args, rank: int, world: int):
     if rank != 0:
         return
@@ -283,15 +301,10 @@ def run_ours(args, rank: int, world: int, dist):
             evs[2 * len(bufs)].record(stream)
 
     def barrier():
-        if dist is not None:
-            dist.barrier()
+        rank_barrier(dist)
 
     def max_over_ranks(ms):
-        if dist is None:
-            return ms
-        t = torch.tensor([ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+        return max_over_ranks_on(ms, dist, dev)
 
     useful = sum(b["flops"] for b in bufs)
 
