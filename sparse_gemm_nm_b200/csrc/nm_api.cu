@@ -123,9 +123,47 @@ static cudaError_t staging_pool(cudaMemPool_t* out) {
   return cudaSuccess;
 }
 
+// Per-thread cache of encoded tensor maps: a call that repeats the previous
+// calls' buffers and shapes (an inference loop) skips cuTensorMapEncodeTiled.
+// The key is every encode argument; a map depends on nothing else.
+struct TmapKey {
+  const void* base;
+  uint64_t d0, d1, d2, s0, s1;
+  uint32_t b0, b1, b2;
+  int swizzle, dtype, rank;
+  bool operator==(const TmapKey& o) const {
+    return base == o.base && d0 == o.d0 && d1 == o.d1 && d2 == o.d2 && s0 == o.s0 && s1 == o.s1 && b0 == o.b0 &&
+           b1 == o.b1 && b2 == o.b2 && swizzle == o.swizzle && dtype == o.dtype && rank == o.rank;
+  }
+};
+struct TmapCache {
+  static constexpr int kEntries = 32;
+  TmapKey key[kEntries];
+  CUtensorMap map[kEntries];
+  bool used[kEntries] = {};
+  int next = 0;
+  bool find(const TmapKey& k, CUtensorMap* out) const {
+    for (int i = 0; i < kEntries; ++i)
+      if (used[i] && key[i] == k) {
+        *out = map[i];
+        return true;
+      }
+    return false;
+  }
+  void put(const TmapKey& k, const CUtensorMap& m) {
+    key[next] = k;
+    map[next] = m;
+    used[next] = true;
+    next = (next + 1) % kEntries;
+  }
+};
+static thread_local TmapCache t_tmaps;
+
 static nm_status make_tmap(CUtensorMap* tm, const void* base, uint64_t inner, uint64_t outer,
                            uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer, int swizzle_bytes,
                            const char* what, CUtensorMapDataType dtype = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16) {
+  const TmapKey key{base, inner, outer, 0, row_bytes, 0, box_inner, box_outer, 0, swizzle_bytes, (int)dtype, 2};
+  if (t_tmaps.find(key, tm)) return NM_OK;
   EncodeTiledFn fn = encode_fn();
   if (!fn) return fail(NM_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
   cuuint64_t dims[2] = {inner, outer};
@@ -139,11 +177,15 @@ static nm_status make_tmap(CUtensorMap* tm, const void* base, uint64_t inner, ui
   CUresult r = fn(tm, dtype, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                   swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return fail(NM_ERR_CUDA, "cuTensorMapEncodeTiled(%s) failed with %d", what, (int)r);
+  t_tmaps.put(key, *tm);
   return NM_OK;
 }
 
 // 3-D map of the tiled 2:4 metadata: {64 words of a block, column blocks, row blocks}.
 static nm_status make_meta_tmap(CUtensorMap* tm, const void* meta, int64_t rblocks, int64_t cblocks) {
+  const TmapKey key{meta, 64, (uint64_t)cblocks, (uint64_t)rblocks, 256, (uint64_t)cblocks * 256, 64, 1, 8, 0,
+                    (int)CU_TENSOR_MAP_DATA_TYPE_UINT32, 3};
+  if (t_tmaps.find(key, tm)) return NM_OK;
   EncodeTiledFn fn = encode_fn();
   if (!fn) return fail(NM_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
   cuuint64_t dims[3] = {64, (cuuint64_t)cblocks, (cuuint64_t)rblocks};
@@ -154,6 +196,7 @@ static nm_status make_meta_tmap(CUtensorMap* tm, const void* meta, int64_t rbloc
                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return fail(NM_ERR_CUDA, "cuTensorMapEncodeTiled(meta) failed with %d", (int)r);
+  t_tmaps.put(key, *tm);
   return NM_OK;
 }
 
