@@ -139,7 +139,10 @@ NM_API nm_status nm_decompress(const uint16_t* values, const uint32_t* meta, int
  * 1:8 and 2:8 (at most two survivors per aligned group of four) are first
  * re-encoded as 2:4 into a staging buffer (R*K bytes of values plus R*K/8
  * bytes of metadata) from the library's pool (see nm_spmm_permuted and
- * nm_release_staging), one extra launch.  Shapes with K % 128 == 0 and
+ * nm_release_staging), one extra launch.  On the same shapes, the dense
+ * design (NM_ALGO_DENSE_TC, or any pattern the 2:4 MMA cannot take under
+ * NM_ALGO_AUTO) decompresses the operand into a staged dense copy (R*K*2
+ * bytes) and runs dense MMAs on SM pairs.  Shapes with K % 128 == 0 and
  * T <= 64 run a split-K kernel (one 128-row tile and one range of K per work
  * unit, persistent over the SMs); when K is split into s > 1 ranges it stages
  * s*R*bn*4 bytes of fp32 partials (bn = T rounded up to 16, 32 or 64) and a

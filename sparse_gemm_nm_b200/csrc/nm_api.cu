@@ -384,13 +384,27 @@ static nm_status run_gemm(const GemmRequest& q, cudaStream_t stream) {
   const bool reencode = q.allow_staging && !q.hybrid && p.a_mode == A_BUILD_SPARSE && !(q.n == 2 && q.m == 4) &&
                         (pair_shape || skinny_shape);
   const bool use_skinny = skinny_shape && (tma_2of4 || reencode);
-  if (reencode || use_skinny || (q.algo != NM_ALGO_DENSE_TC && pair_kernel_fits(p) && al16(q.meta))) {
+  // Dense design on SM pairs (NM_ALGO_DENSE_TC, or a pattern the 2:4 MMA cannot
+  // take): decompress into a staged dense operand, then the pair kernel's dense stages.
+  const bool dense_pair = q.allow_staging && !q.hybrid && p.a_mode == A_BUILD_DENSE && pair_shape;
+  if (dense_pair || reencode || use_skinny || (q.algo != NM_ALGO_DENSE_TC && pair_kernel_fits(p) && al16(q.meta))) {
     cudaMemPool_t pool = nullptr;
     cudaError_t e = cudaSuccess;
     const uint16_t* vals = q.values;
     const uint32_t* meta = q.meta;
     void* staged_a = nullptr;  // re-encoded values, then tiled metadata
-    if (reencode) {
+    if (dense_pair) {
+      e = staging_pool(&pool);
+      if (e != cudaSuccess) return cuda_fail(e, "staging pool");
+      e = cudaMallocFromPoolAsync(&staged_a, (size_t)(q.R * q.K * 2), pool, stream);
+      if (e != cudaSuccess) return cuda_fail(e, "staging buffer for the decompressed weights");
+      e = launch_decompress(q.values, q.meta, q.R, q.K, q.n, q.m, static_cast<uint16_t*>(staged_a), q.K, stream);
+      if (e != cudaSuccess) {
+        cudaFreeAsync(staged_a, stream);
+        return cuda_fail(e, "decompress launch");
+      }
+      p.tile_map = nullptr;
+    } else if (reencode) {
       e = staging_pool(&pool);
       if (e != cudaSuccess) return cuda_fail(e, "staging pool");
       const size_t vbytes = (size_t)(q.R * (q.K / 2) * 2 + 255) / 256 * 256;
@@ -481,14 +495,19 @@ static nm_status run_gemm(const GemmRequest& q, cudaStream_t stream) {
       p.num_tiles = p.tiles_m * p.tiles_n;
       st = make_tmap(&p.tm_x, xsrc, (uint64_t)q.T, (uint64_t)q.K, (uint64_t)ldsrc * 2, 64, kPairBoxRows, 128, "X");
     }
-    if (st == NM_OK)
+    if (st == NM_OK && dense_pair)
+      st = make_tmap(&p.tm_w, staged_a, (uint64_t)q.K, (uint64_t)q.R, (uint64_t)q.K * 2, 64, kPairBoxRows, 128,
+                     "decompressed W");
+    if (st == NM_OK && !dense_pair)
       st = make_tmap(&p.tm_vals, vals, (uint64_t)p.vcols, (uint64_t)q.R, (uint64_t)p.vcols * 2, 64, kPairBoxRows,
                      128, "values");
-    if (st == NM_OK) st = make_meta_tmap(&p.tm_meta, meta, p.meta_rblocks, p.meta_cblocks);
+    if (st == NM_OK && !dense_pair) st = make_meta_tmap(&p.tm_meta, meta, p.meta_rblocks, p.meta_cblocks);
     if (st == NM_OK && !use_skinny && !p.out_f32)
       st = make_tmap(&p.tm_y, q.Y, (uint64_t)q.T, (uint64_t)q.R, (uint64_t)q.ldy * 2, 64, 32, 128, "Y");
     if (st == NM_OK)
-      e = use_skinny ? launch_spmm_skinny(p, stream) : launch_spmm_pair(p, stream);
+      e = use_skinny   ? launch_spmm_skinny(p, stream)
+          : dense_pair ? launch_spmm_pair_hybrid(p, stream)
+                       : launch_spmm_pair(p, stream);
     if (ws) cudaFreeAsync(ws, stream);
     release();
     if (st != NM_OK) return st;

@@ -126,6 +126,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pair::kThreads, 1)
   // both CTAs stage dense tiles (W, or W with the 2:4 mask applied).
   auto tile_sparse = [&](int tm, int64_t kt, int rr) -> bool {
     if (!HYB) return true;
+    if (!p.tile_map) return false;  // dense design: every stage dense (W is the staged decompressed operand)
     int rb = 2 * tm + rr;
     if (rb >= p.hyb_rows) rb = 2 * tm;
     return __ldg(p.tile_map + (int64_t)rb * p.hyb_tiles_k + kt) != 0;

@@ -412,3 +412,26 @@ def test_bounded_wait_timeout_is_reported():
     W = wl.normal_bf16((R, K), 0.02, seed=191)
     X = wl.normal_bf16((K, T), 1.0, seed=192)
     check(W, X, 2, 4, what="after a reported timeout")
+
+
+# ----------------------------------------------------------------------------
+# Dense design on SM pairs: decompress into a staged dense operand, dense stages
+# ----------------------------------------------------------------------------
+@pytest.mark.parametrize("n,m,algo", [(2, 4, nm.NM_ALGO_DENSE_TC), (1, 8, nm.NM_ALGO_DENSE_TC),
+                                      (3, 4, nm.NM_ALGO_AUTO), (5, 8, nm.NM_ALGO_AUTO)])
+@pytest.mark.parametrize("permuted", [False, True])
+def test_dense_design_pair_path(n, m, algo, permuted):
+    R, K, T = 300, 512, 264
+    W = wl.normal_bf16((R, K), 0.02, seed=201 + m)
+    X = wl.normal_bf16((K, T), 1.0, seed=202)
+    idx = wl.permutation(K, 203) if permuted else None
+    check(W, X, n, m, idx=idx, algo=algo, what=f"dense design {n}:{m}")
+
+
+def test_dense_design_pair_integer_exact():
+    R, K, T = 256, 512, 256
+    W = wl.integer_bf16((R, K), -8, 8, seed=211)
+    X = wl.integer_bf16((K, T), -8, 8, seed=212)
+    ref, _ = reference(W, X, 3, 4)
+    Y = run_spmm(W, X, 3, 4, out_dtype=torch.float32)
+    assert np.array_equal(Y.cpu().numpy().astype(np.float64), ref)
