@@ -646,7 +646,18 @@ nm_status nm_prune_compress(const uint16_t* W, int64_t R, int64_t K, int64_t ldw
     return fail(NM_ERR_UNSUPPORTED, "matrix too large for one call");
   nm_status st = require_device();
   if (st != NM_OK) return st;
-  cudaError_t e = launch_compress(W, R, K, ldw, n, m, values, meta, static_cast<cudaStream_t>(stream));
+  cudaError_t e;
+  if (tiled_meta(n, m) && K % 8 == 0 && ldw % 8 == 0 && al16(W) && al16(values) && al16(meta)) {
+    // 2:4 on aligned rows: the TMA-fed stream kernel (16-row x 128-column boxes)
+    CUtensorMap tm;
+    st = make_tmap(&tm, W, (uint64_t)K, (uint64_t)R, (uint64_t)ldw * 2, 128, 16, 0, "W");
+    if (st != NM_OK) return st;
+    uint32_t* status = status_word_ptr();
+    if (!status) return fail(NM_ERR_CUDA, "device status word is unavailable");
+    e = launch_compress_stream(tm, R, K, values, meta, status, static_cast<cudaStream_t>(stream));
+  } else {
+    e = launch_compress(W, R, K, ldw, n, m, values, meta, static_cast<cudaStream_t>(stream));
+  }
   return e == cudaSuccess ? NM_OK : cuda_fail(e, "compress launch");
 }
 

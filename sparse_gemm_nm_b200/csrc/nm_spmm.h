@@ -70,5 +70,7 @@ bool skinny_kernel_fits(int64_t T);
 int skinny_bn(int64_t T);
 int skinny_kd(int64_t K, int64_t T);
 cudaError_t launch_spmm_skinny(SpmmParams& p, cudaStream_t stream);
+cudaError_t launch_compress_stream(const CUtensorMap& tm_w, int64_t R, int64_t K, uint16_t* values, uint32_t* meta,
+                                   uint32_t* status, cudaStream_t s);
 
 }  // namespace nmk
