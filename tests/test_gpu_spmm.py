@@ -322,7 +322,7 @@ def test_permuted_pair_path_after_release_staging():
 @pytest.mark.parametrize("n,m", [(1, 2), (1, 4), (1, 8), (2, 8)])
 @pytest.mark.parametrize("permuted", [False, True])
 def test_reencoded_pair_path(n, m, permuted):
-    R, K, T = 300, 512, 264
+    R, K, T = 600, 1024, 264
     W = wl.normal_bf16((R, K), 0.02, seed=131 + m + n)
     X = wl.normal_bf16((K, T), 1.0, seed=132)
     idx = wl.permutation(K, 133) if permuted else None
@@ -332,8 +332,9 @@ def test_reencoded_pair_path(n, m, permuted):
     assert nm.nm_launch_count() - before == (4 if permuted else 3)
 
 
+
 def test_reencoded_pair_path_integer_exact():
-    R, K, T = 256, 384, 256
+    R, K, T = 512, 1024, 256
     W = wl.integer_bf16((R, K), -8, 8, seed=141)
     X = wl.integer_bf16((K, T), -8, 8, seed=142)
     ref, _ = reference(W, X, 1, 8)
@@ -421,7 +422,7 @@ def test_bounded_wait_timeout_is_reported():
                                       (3, 4, nm.NM_ALGO_AUTO), (5, 8, nm.NM_ALGO_AUTO)])
 @pytest.mark.parametrize("permuted", [False, True])
 def test_dense_design_pair_path(n, m, algo, permuted):
-    R, K, T = 300, 512, 264
+    R, K, T = 600, 1024, 264
     W = wl.normal_bf16((R, K), 0.02, seed=201 + m)
     X = wl.normal_bf16((K, T), 1.0, seed=202)
     idx = wl.permutation(K, 203) if permuted else None
@@ -429,7 +430,7 @@ def test_dense_design_pair_path(n, m, algo, permuted):
 
 
 def test_dense_design_pair_integer_exact():
-    R, K, T = 256, 512, 256
+    R, K, T = 512, 1024, 256
     W = wl.integer_bf16((R, K), -8, 8, seed=211)
     X = wl.integer_bf16((K, T), -8, 8, seed=212)
     ref, _ = reference(W, X, 3, 4)
