@@ -16,6 +16,7 @@
 #include <cuda_runtime.h>
 
 #include "nm_internal.h"
+#include "nm_select.cuh"
 
 namespace nmk {
 
@@ -31,34 +32,8 @@ __device__ __forceinline__ uint32_t mag_key(uint32_t bits16) {
 // eight rows, every load and every value store of the warp covers whole
 // 128-byte lines, and each lane keeps one byte of nibbles per row (rows
 // 2k + l/16: k = 0..3 in `lo8`, k = 4..7 in `hi8`).  The block's 64 words are
-// assembled with shuffles, two per lane.
-//
-// Selection of one group.  Composite keys c_i = (magnitude field of e_i) * 4
-// + (3 - i), NaNs folded to one key just above +Inf: all four are distinct,
-// and a larger key means a larger magnitude or, on equal magnitudes, a lower
-// index.  The two largest keys come from a four-input network (max/min of
-// each pair, then the larger maximum and the larger of the smaller maximum and
-// the larger minimum); their low bits give the positions.
-__device__ __forceinline__ uint32_t ckey(uint32_t shifted_by2, uint32_t tie) {
-  return min((shifted_by2 & 0x1FFFCu) | tie, 0x1FE04u | tie);  // 0x1FE04 = (0x7F81 << 2)
-}
-
-// Group of four in (lo, hi) = (e0 | e1 << 16, e2 | e3 << 16): returns the
-// nibble p0 | p1 << 2 (p0 < p1), and in `pk` the two survivors (first in the
-// low half).
-__device__ __forceinline__ uint32_t select_pair(uint32_t lo, uint32_t hi, uint32_t& pk) {
-  const uint32_t c0 = ckey(lo << 2, 3u), c1 = ckey(lo >> 14, 2u);
-  const uint32_t c2 = ckey(hi << 2, 1u), c3 = ckey(hi >> 14, 0u);
-  const uint32_t m01 = max(c0, c1), n01 = min(c0, c1);
-  const uint32_t m23 = max(c2, c3), n23 = min(c2, c3);
-  const uint32_t top = max(m01, m23);
-  const uint32_t second = max(min(m01, m23), max(n01, n23));
-  const uint32_t pa = (top & 3u) ^ 3u, pb = (second & 3u) ^ 3u;
-  const uint32_t p0 = min(pa, pb), p1 = max(pa, pb);
-  pk = __byte_perm(lo, hi, 0x1010u + p0 * 0x22u + p1 * 0x2200u);
-  return p0 | (p1 << 2);
-}
-
+// assembled with shuffles, two per lane.  The group selection is select_pair
+// (nm_select.cuh).
 __global__ void __launch_bounds__(256, 4) compress_2of4_tiled_kernel(const uint16_t* __restrict__ W, uint32_t R,
                                                                   uint32_t K, int64_t ldw,
                                                                   uint16_t* __restrict__ V,

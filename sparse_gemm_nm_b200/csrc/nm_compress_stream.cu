@@ -16,6 +16,7 @@
 
 #include "nm_internal.h"
 #include "nm_ptx.cuh"
+#include "nm_select.cuh"
 
 namespace nmk {
 
@@ -33,26 +34,6 @@ constexpr uint64_t kWaitNs = 2000000000ull;
 constexpr size_t kSmem = 100 * 1024;
 static_assert(kSlots * kBlockBytes + 2 * kSlots * 8 + 64 + 1024 <= kSmem, "ring does not fit");
 }  // namespace cstream
-
-// Selection of one group of four, (lo, hi) = (e0 | e1 << 16, e2 | e3 << 16):
-// composite keys (magnitude field * 4 + (3 - index), NaNs folded just above
-// +Inf) through a four-input max/min network; returns the nibble p0 | p1 << 2
-// and the two survivors in `pk` (first in the low half).
-__device__ __forceinline__ uint32_t stream_ckey(uint32_t shifted_by2, uint32_t tie) {
-  return min((shifted_by2 & 0x1FFFCu) | tie, 0x1FE04u | tie);
-}
-__device__ __forceinline__ uint32_t stream_select(uint32_t lo, uint32_t hi, uint32_t& pk) {
-  const uint32_t c0 = stream_ckey(lo << 2, 3u), c1 = stream_ckey(lo >> 14, 2u);
-  const uint32_t c2 = stream_ckey(hi << 2, 1u), c3 = stream_ckey(hi >> 14, 0u);
-  const uint32_t m01 = max(c0, c1), n01 = min(c0, c1);
-  const uint32_t m23 = max(c2, c3), n23 = min(c2, c3);
-  const uint32_t top = max(m01, m23);
-  const uint32_t second = max(min(m01, m23), max(n01, n23));
-  const uint32_t pa = (top & 3u) ^ 3u, pb = (second & 3u) ^ 3u;
-  const uint32_t p0 = min(pa, pb), p1 = max(pa, pb);
-  pk = __byte_perm(lo, hi, 0x1010u + p0 * 0x22u + p1 * 0x2200u);
-  return p0 | (p1 << 2);
-}
 
 __global__ void __launch_bounds__(cstream::kThreads, 2)
     compress_2of4_stream_kernel(const __grid_constant__ CUtensorMap tm_w, uint32_t R, uint32_t K,
@@ -106,7 +87,7 @@ __global__ void __launch_bounds__(cstream::kThreads, 2)
     uint32_t pk[16], by[8];
 #pragma unroll
     for (int i = 0; i < 8; ++i)
-      by[i] = stream_select(in[i].x, in[i].y, pk[2 * i]) | (stream_select(in[i].z, in[i].w, pk[2 * i + 1]) << 4);
+      by[i] = select_pair(in[i].x, in[i].y, pk[2 * i]) | (select_pair(in[i].z, in[i].w, pk[2 * i + 1]) << 4);
     __syncwarp();
     if (lane == 0) mbar_arrive(&empty[slot]);  // the block's registers are consumed
     const uint32_t col = cb * 128 + 8 * piece;
