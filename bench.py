@@ -54,6 +54,9 @@ def parse_args(argv=None):
     ap.add_argument("--algo", choices=["auto", "sparse", "dense"], default="auto",
                     help="kernel design for 1:4 / 1:8 (nm_spmm_algo)")
     ap.add_argument("--plain", action="store_true", help="ignore the workload's index map (y = W x)")
+    ap.add_argument("--fused", action="store_true",
+                    help="one nm_prune_spmm call per layer (prune + compress + GEMM, same outputs) instead of "
+                         "nm_prune_compress followed by the GEMM call")
     ap.add_argument("--quick", action="store_true",
                     help="timed region only: no clock sampling, end-to-end pass, oracle baseline or extras")
     return ap.parse_args(argv)
@@ -248,6 +251,8 @@ def run_ours(args, rank: int, world: int, dist):
     def up(bits):
         return torch.from_numpy(bits.view(np.int16)).to(dev).view(torch.bfloat16)
 
+    if args.fused and any(d.tmap is not None for d in data):
+        raise SystemExit("--fused covers the n:m pruned GEMM, not the hybrid workloads")
     bufs = []
     for d in data:
         L = d.layer
@@ -258,7 +263,7 @@ def run_ours(args, rank: int, world: int, dist):
              "meta": torch.empty((max(nm.nm_meta_words(L.R, L.K, L.n, L.m), 0),), dtype=torch.int32, device=dev),
              "Y": torch.empty((L.R, L.T), dtype=torch.bfloat16, device=dev)}
         b["flops"] = float(wl.hybrid_useful_flops(d) if d.tmap is not None else L.useful_flops)
-        b["gemm_bytes"] = gemm_bytes(L, d)
+        b["gemm_bytes"] = gemm_bytes(L, d) + (2.0 * L.R * L.K if args.fused else 0.0)  # fused: W read once
         b["comp_bytes"] = 2.0 * L.R * L.K + 2.0 * b["vals"].numel() + 4.0 * b["meta"].numel()
         bufs.append(b)
     torch.cuda.synchronize()
@@ -289,10 +294,22 @@ def run_ours(args, rank: int, world: int, dist):
             check(L_.nm_spmm(b["vals"].data_ptr(), b["meta"].data_ptr(), L.n, L.m, L.R, L.K, b["X"].data_ptr(),
                              L.T, L.T, b["Y"].data_ptr(), L.T, 0, sp), "nm_spmm")
 
+    def launch_fused(b, permuted=True):
+        L = b["L"]
+        idx = b["idx"].data_ptr() if b["idx"] is not None and permuted else None
+        check(L_.nm_prune_spmm(b["W"].data_ptr(), L.K, L.n, L.m, L.R, L.K, idx, b["X"].data_ptr(), L.T, L.T,
+                               b["Y"].data_ptr(), L.T, 0, b["vals"].data_ptr(), b["meta"].data_ptr(), sp),
+              "nm_prune_spmm")
+
     def step(evs=None, permuted=True):
         for i, b in enumerate(bufs):
             if evs is not None:
                 evs[2 * i].record(stream)
+            if args.fused:  # the whole call is timed as the GEMM; the compress slot stays empty
+                if evs is not None:
+                    evs[2 * i + 1].record(stream)
+                launch_fused(b, permuted)
+                continue
             launch_compress(b)
             if evs is not None:
                 evs[2 * i + 1].record(stream)
@@ -374,9 +391,10 @@ def run_ours(args, rank: int, world: int, dist):
             "gemm_gbs": b["gemm_bytes"] / (gemm_ms[i] * 1e-3) / 1e9,
             "gemm_bound": "tensor" if t_tc >= t_hbm else "hbm",
             "gemm_frac": max(t_tc, t_hbm) / (gemm_ms[i] * 1e-3),
-            "compress_us": 1e3 * comp_ms[i],
-            "compress_gbs": b["comp_bytes"] / (comp_ms[i] * 1e-3) / 1e9,
-            "compress_frac": b["comp_bytes"] / (comp_ms[i] * 1e-3) / 1e9 / hbm_peak}
+            "compress_us": 1e3 * comp_ms[i]}
+        if not args.fused:
+            kernels[L.name]["compress_gbs"] = b["comp_bytes"] / (comp_ms[i] * 1e-3) / 1e9
+            kernels[L.name]["compress_frac"] = kernels[L.name]["compress_gbs"] / hbm_peak
 
     # dominant kernel: the GEMM (all launches of the step together)
     flops_all = sum(b["flops"] for b in bufs)
@@ -387,7 +405,7 @@ def run_ours(args, rank: int, world: int, dist):
     # (profiles/<workload>_gemm_traffic.json); summed over the step like `achieved`.
     traffic = None
     tfile = os.path.join(ROOT, "profiles", f"{args.workload}_gemm_traffic.json")
-    if os.path.exists(tfile) and args.algo == "auto":
+    if os.path.exists(tfile) and args.algo == "auto" and not args.fused:
         with open(tfile) as f:
             per = json.load(f).get("bytes_per_launch", {})
         names = [f"{b['L'].R}x{b['L'].K}" for b in bufs]
@@ -402,14 +420,16 @@ def run_ours(args, rank: int, world: int, dist):
         src = f"{peak_src} HBM copy bandwidth"
     roofline = {"bound": "tensor" if tensor_bound else "hbm", "achieved": achieved, "peak": peak, "unit": unit,
                 "frac": achieved / peak, "traffic": traffic,
-                "kernel": "nm_spmm_permuted call: gather_rows_kernel + spmm_pair_kernel (tcgen05 2-SM GEMM)",
+                "kernel": ("nm_prune_spmm call: prune_spmm_skinny_kernel (+ gather, split-K reduction)" if args.fused
+                           else "nm_spmm_permuted call: gather_rows_kernel + spmm_pair_kernel (tcgen05 2-SM GEMM)"),
                 "peak_source": src,
                 "algorithmic_per_launch": [b["flops"] if tensor_bound else b["gemm_bytes"] for b in bufs]}
 
     cfg = {"workload": args.workload, "shapes": [[b["L"].R, b["L"].K] for b in bufs],
            "T": [b["L"].T for b in bufs], "pattern": [f"{b['L'].n}:{b['L'].m}" for b in bufs],
            "permuted": any(b["idx"] is not None for b in bufs), "algo": args.algo,
-           "step": "prune+compress, then the sparse GEMM, for every layer",
+           "step": ("one fused prune+compress+GEMM call (nm_prune_spmm) per layer" if args.fused
+                    else "prune+compress, then the sparse GEMM, for every layer"),
            "kernel_timing": "per-kernel CUDA events in a second timed pass of the same K steps",
            "l2": "inputs larger than L2 (126 MB) per step" if sum(
                b["W"].numel() * 2 + b["X"].numel() * 2 + b["Y"].numel() * 2 for b in bufs) > 126e6
@@ -474,8 +494,11 @@ def run_ours(args, rank: int, world: int, dist):
                 stream.wait_event(copied[i])
                 if started[i]:
                     stream.wait_event(returned[i])  # Y of the previous step has been read back
-                launch_compress(b)
-                launch_gemm(b)
+                if args.fused:
+                    launch_fused(b)
+                else:
+                    launch_compress(b)
+                    launch_gemm(b)
                 computed[i].record(stream)
                 with torch.cuda.stream(s_d2h):
                     s_d2h.wait_event(computed[i])

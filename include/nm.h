@@ -205,7 +205,36 @@ NM_API nm_status nm_hybrid_spmm(const uint16_t* W, int64_t ldw, const uint16_t* 
                          int64_t ldx, int64_t T, void* Y, int64_t ldy, nm_out_dtype y_dtype, void* stream);
 
 /*
- * nm_spmm_algo -- nm_spmm / nm_spmm_permuted (idx may be NULL) with the kernel
+ * nm_prune_spmm -- prune and multiply in one call, for masks that change from
+ * call to call (weights re-pruned during training): Y = (W' Pi) X where W' is
+ * W under the n:m magnitude mask of nm_prune_compress, and Pi is the index
+ * map of nm_spmm_permuted (idx may be NULL for none).  The result equals
+ * nm_prune_compress followed by nm_spmm_permuted on its output.
+ * Source: "Structured Sparsity" topic cards, RNM-TD3 abstract (N:M structured
+ * sparsity kept through the whole of training, so the mask is recomputed as
+ * the weights move) and "M:N sparsity on NVIDIA tensor cores" (the mask).
+ *   W      [in]  R x K bf16, row stride ldw >= K
+ *   values, meta [out, optional] both NULL, or both set: they receive
+ *          exactly what nm_prune_compress(W, n, m) writes
+ *   other arguments as nm_spmm_permuted.
+ * 2:4 with K % 128 == 0, T <= 64, ldw % 8 == 0 and 16-byte aligned W (and
+ * values/meta when given) runs one fused kernel: each 128 x 128 tile of W is
+ * read once by TMA, selected in shared memory and fed to the sparse MMA, so
+ * W is read from HBM once and the compressed form is only written when
+ * asked for; split-K partials and the gather of permuted rows are staged as
+ * in nm_spmm_permuted (a second launch sums the partials).  Every other case
+ * runs nm_prune_compress into `values`/`meta` (or, when those are NULL, into
+ * a staging buffer of R*K*9/16 bytes for 2:4 from the library's pool) and
+ * then the nm_spmm_permuted path.
+ * Errors: as nm_prune_compress and nm_spmm_permuted; NM_ERR_INVALID_ARG when
+ * only one of values and meta is given.
+ */
+NM_API nm_status nm_prune_spmm(const uint16_t* W, int64_t ldw, int n, int m, int64_t R, int64_t K,
+                               const int32_t* idx, const uint16_t* X, int64_t ldx, int64_t T, void* Y, int64_t ldy,
+                               nm_out_dtype y_dtype, uint16_t* values, uint32_t* meta, void* stream);
+
+/*
+ * nm_spmm_algo --nm_spmm / nm_spmm_permuted (idx may be NULL) with the kernel
  * design chosen explicitly, to compare the sparse tensor-core path with the
  * dense expansion on the same pattern.  NM_ERR_UNSUPPORTED when the pattern
  * does not fit the requested design (NM_ALGO_SPARSE_TC with 3:4, say).

@@ -3,11 +3,11 @@
 Python binding of the C ABI in ``include/nm.h`` (library ``libnm_b200.so``).
 The functions named like the C entry points (``nm_prune_compress``,
 ``nm_decompress``, ``nm_spmm``, ``nm_spmm_permuted``, ``nm_hybrid_spmm``,
-``nm_spmm_algo``) only marshal arguments: tensors become device pointers, the
+``nm_spmm_algo``, ``nm_prune_spmm``) only marshal arguments: tensors become device pointers, the
 stream defaults to torch's current stream, and a non-zero status raises
 :class:`NmError`.  Every step of the computation runs in the library's CUDA
 kernels; there is no fallback of any kind.  The convenience wrappers
-(``prune_compress``, ``decompress``, ``spmm``, ``hybrid_spmm``) also allocate
+(``prune_compress``, ``decompress``, ``spmm``, ``hybrid_spmm``, ``prune_spmm``) also allocate
 the outputs with torch.
 
 bf16 data is accepted as ``torch.bfloat16`` tensors (or int16/uint16 views of
@@ -48,6 +48,7 @@ SIGNATURES = {
     "nm_spmm": ([_P, _P, _I, _I, _I64, _I64, _P, _I64, _I64, _P, _I64, _I, _P], _I),
     "nm_spmm_permuted": ([_P, _P, _I, _I, _I64, _I64, _P, _P, _I64, _I64, _P, _I64, _I, _P], _I),
     "nm_hybrid_spmm": ([_P, _I64, _P, _P, _P, _I, _I64, _I64, _P, _I64, _I64, _P, _I64, _I, _P], _I),
+    "nm_prune_spmm": ([_P, _I64, _I, _I, _I64, _I64, _P, _P, _I64, _I64, _P, _I64, _I, _P, _P, _P], _I),
     "nm_spmm_algo": ([_P, _P, _I, _I, _I64, _I64, _P, _P, _I64, _I64, _P, _I64, _I, _I, _P], _I),
     "nm_spmm_permuted_noalloc": ([_P, _P, _I, _I, _I64, _I64, _P, _P, _I64, _I64, _P, _I64, _I, _P], _I),
     "nm_release_staging": ([], _I),
@@ -155,6 +156,12 @@ def nm_hybrid_spmm(W, ldw, values, meta, tile_map, tile, R, K, X, ldx, T, Y, ldy
                                 ldx, T, _ptr(Y), ldy, y_dtype, _stream(stream)), "nm_hybrid_spmm")
 
 
+def nm_prune_spmm(W, ldw, n, m, R, K, idx, X, ldx, T, Y, ldy, y_dtype=NM_OUT_BF16, values=None, meta=None,
+                  stream=None) -> None:
+    _check(lib().nm_prune_spmm(_ptr(W), ldw, n, m, R, K, _ptr(idx), _ptr(X), ldx, T, _ptr(Y), ldy, y_dtype,
+                               _ptr(values), _ptr(meta), _stream(stream)), "nm_prune_spmm")
+
+
 def nm_spmm_algo(values, meta, n, m, R, K, idx, X, ldx, T, Y, ldy, y_dtype=NM_OUT_BF16, algo=NM_ALGO_AUTO,
                  stream=None) -> None:
     _check(lib().nm_spmm_algo(_ptr(values), _ptr(meta), n, m, R, K, _ptr(idx), _ptr(X), ldx, T, _ptr(Y), ldy,
@@ -246,3 +253,29 @@ def hybrid_spmm(W, values, meta, tile_map, X, tile: int = 128, out_dtype=None, s
     yt = NM_OUT_F32 if out_dtype == torch.float32 else NM_OUT_BF16
     nm_hybrid_spmm(W, W.stride(0), values, meta, tile_map, tile, R, K, X, X.stride(0), T, Y, T, yt, stream)
     return Y
+
+
+def prune_spmm(W, n: int, m: int, X, idx=None, out_dtype=None, keep_compressed: bool = False, stream=None):
+    """Y = (W' Pi) X with W' the n:m magnitude-pruned W, from the dense W in one call.
+
+    With keep_compressed=True also returns (values, meta) as prune_compress would.
+    Y's rows are padded to 16 bytes; the returned tensor is the R x T view.
+    """
+    import torch
+    _require_cuda(W, X, idx)
+    out_dtype = out_dtype or torch.bfloat16
+    R, K = W.shape
+    T = X.shape[1]
+    per16 = 4 if out_dtype == torch.float32 else 8
+    ldy = max((T + per16 - 1) // per16 * per16, per16)
+    Y = torch.empty((R, ldy), dtype=out_dtype, device=X.device)
+    yt = NM_OUT_F32 if out_dtype == torch.float32 else NM_OUT_BF16
+    vals = meta = None
+    if keep_compressed:
+        if nm_value_cols(K, n, m) < 0:
+            _check(lib().nm_prune_compress(None, R, K, K, n, m, None, None, None), "nm_prune_spmm")
+        vals = torch.empty((R, nm_value_cols(K, n, m)), dtype=torch.bfloat16, device=W.device)
+        meta = torch.empty((max(nm_meta_words(R, K, n, m), 0),), dtype=torch.int32, device=W.device)
+    nm_prune_spmm(W, W.stride(0), n, m, R, K, idx, X, X.stride(0), T, Y, ldy, yt, vals, meta, stream)
+    Y = Y[:, :T]
+    return (Y, vals, meta) if keep_compressed else Y

@@ -615,6 +615,137 @@ nm_status build_pair_params(SpmmParams& p, const uint16_t* values, const uint32_
   return st;
 }
 
+
+// Prune + GEMM.  2:4 on skinny shapes: one fused kernel selects each W tile in
+// shared memory and feeds the sparse MMA (W read from HBM once).  Otherwise:
+// compress (into the caller's buffers or a staged pair), then the GEMM path.
+static nm_status run_prune_gemm(const uint16_t* W, int64_t ldw, int n, int m, int64_t R, int64_t K,
+                                const int32_t* idx, const uint16_t* X, int64_t ldx, int64_t T, void* Y, int64_t ldy,
+                                nm_out_dtype y_dtype, uint16_t* values, uint32_t* meta, cudaStream_t stream) {
+  t_last_error.clear();
+  if (R < 0 || K < 0 || T < 0) return fail(NM_ERR_INVALID_ARG, "negative dimension");
+  if (!pattern_ok(n, m)) return fail(NM_ERR_INVALID_ARG, "pattern %d:%d not supported", n, m);
+  if (K % m != 0) return fail(NM_ERR_INVALID_ARG, "K=%lld is not a multiple of M=%d", (long long)K, m);
+  if ((values == nullptr) != (meta == nullptr)) return fail(NM_ERR_INVALID_ARG, "values and meta: give both or neither");
+  if (ldw < K) return fail(NM_ERR_INVALID_ARG, "ldw < K");
+  if (y_dtype != NM_OUT_BF16 && y_dtype != NM_OUT_F32) return fail(NM_ERR_INVALID_ARG, "bad output dtype");
+  if (R == 0) return NM_OK;
+  if (K > 0 && !W) return fail(NM_ERR_INVALID_ARG, "W is null");
+  if (T == 0 || K == 0) {
+    nm_status st = values ? nm_prune_compress(W, R, K, ldw, n, m, values, meta, stream) : NM_OK;
+    if (st != NM_OK || T == 0) return st;
+    return nm_spmm_algo(nullptr, nullptr, n, m, R, K, nullptr, X, ldx, T, Y, ldy, y_dtype, NM_ALGO_AUTO, stream);
+  }
+  if (!X) return fail(NM_ERR_INVALID_ARG, "X is null");
+  const bool fused = n == 2 && m == 4 && K % 128 == 0 && skinny_kernel_fits(T) && ldw % 8 == 0 && al16(W) &&
+                     (!values || (al16(values) && al16(meta))) && R < (1ll << 31) && K < (1ll << 31);
+  if (!fused) {
+    void* staged = nullptr;
+    uint16_t* v = values;
+    uint32_t* mt = meta;
+    if (!values) {
+      cudaMemPool_t pool = nullptr;
+      cudaError_t e = staging_pool(&pool);
+      if (e != cudaSuccess) return cuda_fail(e, "staging pool");
+      const size_t vbytes = (size_t)(R * value_cols(K, n, m) * 2 + 255) / 256 * 256;
+      const size_t mbytes = (size_t)meta_words(R, K, n, m) * 4;
+      e = cudaMallocFromPoolAsync(&staged, vbytes + mbytes, pool, stream);
+      if (e != cudaSuccess) return cuda_fail(e, "staging buffer for the compressed weights");
+      v = static_cast<uint16_t*>(staged);
+      mt = reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(staged) + vbytes);
+    }
+    nm_status st = nm_prune_compress(W, R, K, ldw, n, m, v, mt, stream);
+    if (st == NM_OK) st = nm_spmm_algo(v, mt, n, m, R, K, idx, X, ldx, T, Y, ldy, y_dtype, NM_ALGO_AUTO, stream);
+    if (staged) cudaFreeAsync(staged, stream);
+    return st;
+  }
+
+  // fused kernel: same argument rules as the GEMM calls
+  if (!Y) return fail(NM_ERR_INVALID_ARG, "Y is null");
+  if (ldy < T) return fail(NM_ERR_INVALID_ARG, "ldy < T");
+  const int esize = y_dtype == NM_OUT_F32 ? 4 : 2;
+  if (!al16(Y) || (ldy * esize) % 16 != 0) return fail(NM_ERR_MISALIGNED, "Y rows must be 16-byte aligned");
+  if (!X) return fail(NM_ERR_INVALID_ARG, "X is null");
+  if (ldx < T) return fail(NM_ERR_INVALID_ARG, "ldx < T");
+  if (!al16(X) || ldx % 8 != 0) return fail(NM_ERR_MISALIGNED, "X rows must be 16-byte aligned");
+  nm_status st = require_device();
+  if (st != NM_OK) return st;
+
+  SpmmParams p;
+  std::memset(&p, 0, sizeof p);
+  p.Y = Y;
+  p.ldy = ldy;
+  p.R = R;
+  p.K = K;
+  p.T = T;
+  p.n = 2;
+  p.m = 4;
+  p.pattern = PAT_2_4;
+  p.vcols = K / 2;
+  p.meta_rblocks = meta_row_blocks(R);
+  p.meta_cblocks = meta_col_blocks(K);
+  p.out_f32 = y_dtype == NM_OUT_F32;
+  p.out_vals = values;
+  p.out_meta = meta;
+  p.status = status_word_ptr();
+  if (!p.status) return fail(NM_ERR_CUDA, "device status word is unavailable");
+  p.bn = skinny_bn(T);
+  p.kd = 128;
+  p.k_tiles = K / 128;
+  p.tiles_m = (int)((R + 127) / 128);
+  if ((int64_t)p.tiles_m * p.k_tiles >= (1ll << 31)) return fail(NM_ERR_UNSUPPORTED, "too many tiles");
+  choose_splits(p, sm_count_current());
+  p.tiles_n = 1;
+  p.num_tiles = p.tiles_m;
+
+  cudaMemPool_t pool = nullptr;
+  cudaError_t e = cudaSuccess;
+  void* staged = nullptr;
+  void* ws = nullptr;
+  auto release = [&]() {
+    if (staged) cudaFreeAsync(staged, stream);
+    if (ws) cudaFreeAsync(ws, stream);
+  };
+  const uint16_t* xsrc = X;
+  int64_t ldsrc = ldx;
+  if (idx || p.splits > 1) {
+    e = staging_pool(&pool);
+    if (e != cudaSuccess) return cuda_fail(e, "staging pool");
+  }
+  if (idx) {
+    const int64_t ldp = (T + 7) / 8 * 8;
+    e = cudaMallocFromPoolAsync(&staged, (size_t)(K * ldp * 2), pool, stream);
+    if (e != cudaSuccess) {
+      staged = nullptr;
+      return cuda_fail(e, "staging buffer for the permuted input");
+    }
+    e = launch_gather_rows(X, ldx, idx, K, T, static_cast<uint16_t*>(staged), ldp, stream);
+    if (e != cudaSuccess) {
+      release();
+      return cuda_fail(e, "gather launch");
+    }
+    xsrc = static_cast<const uint16_t*>(staged);
+    ldsrc = ldp;
+  }
+  if (p.splits > 1) {
+    e = cudaMallocFromPoolAsync(&ws, (size_t)p.splits * R * p.bn * 4, pool, stream);
+    if (e != cudaSuccess) {
+      ws = nullptr;
+      release();
+      return cuda_fail(e, "split-K workspace");
+    }
+    p.ws = static_cast<float*>(ws);
+  }
+  // W: one 128 x 128 box per stage, unswizzled (256-byte rows in shared memory)
+  st = make_tmap(&p.tm_w, W, (uint64_t)K, (uint64_t)R, (uint64_t)ldw * 2, 128, 128, 0, "W");
+  if (st == NM_OK)
+    st = make_tmap(&p.tm_x, xsrc, (uint64_t)T, (uint64_t)K, (uint64_t)ldsrc * 2, (uint32_t)p.bn, 128, p.bn * 2, "X");
+  if (st == NM_OK) e = launch_prune_spmm_skinny(p, stream);
+  release();
+  if (st != NM_OK) return st;
+  return e == cudaSuccess ? NM_OK : cuda_fail(e, "fused prune + GEMM launch");
+}
+
 }  // namespace nmk
 
 using namespace nmk;
@@ -737,6 +868,13 @@ nm_status nm_hybrid_spmm(const uint16_t* W, int64_t ldw, const uint16_t* values,
   q.tile_map = tile_map;
   q.tile = tile;
   return run_gemm(q, static_cast<cudaStream_t>(stream));
+}
+
+nm_status nm_prune_spmm(const uint16_t* W, int64_t ldw, int n, int m, int64_t R, int64_t K, const int32_t* idx,
+                        const uint16_t* X, int64_t ldx, int64_t T, void* Y, int64_t ldy, nm_out_dtype y_dtype,
+                        uint16_t* values, uint32_t* meta, void* stream) {
+  return run_prune_gemm(W, ldw, n, m, R, K, idx, X, ldx, T, Y, ldy, y_dtype, values, meta,
+                        static_cast<cudaStream_t>(stream));
 }
 
 nm_status nm_device_status(void* stream) {

@@ -277,20 +277,27 @@ __global__ void __launch_bounds__(256) gather_rows_kernel(const uint16_t* __rest
   const int lane = threadIdx.x & 31;
   const int64_t warp = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) >> 5;
   const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
-  const int64_t pieces = T >> 3;                    // 16-byte pieces per row
+  const int64_t whole = T >> 3;                     // 16-byte pieces inside the row's T columns
+  const int64_t pieces = (T + 7) >> 3;              // + a partial last piece when T % 8 != 0
   const int64_t chunks = (pieces + 255) / 256;      // 4 KB chunks per row
   const int64_t items = K * chunks;
   for (int64_t it = warp; it < items; it += nwarps) {
     const int64_t k = it / chunks, c0 = (it - k * chunks) * 256;
     const int32_t src = __ldg(idx + k);
     const bool valid = src >= 0 && (int64_t)src < K;
-    const uint4* in = reinterpret_cast<const uint4*>(X + (valid ? (int64_t)src : 0) * ldx);
+    const uint16_t* row = X + (valid ? (int64_t)src : 0) * ldx;
+    const uint4* in = reinterpret_cast<const uint4*>(row);
     uint4* out = reinterpret_cast<uint4*>(Xp + k * ldp);
     uint4 v[8];
 #pragma unroll
     for (int u = 0; u < 8; ++u) {
       const int64_t c = c0 + u * 32 + lane;
-      v[u] = (valid && c < pieces) ? __ldg(in + c) : make_uint4(0, 0, 0, 0);
+      v[u] = (valid && c < whole) ? __ldg(in + c) : make_uint4(0, 0, 0, 0);
+      if (valid && c == whole && c < pieces) {  // columns 8c .. T-1 one by one, zeros after them
+        uint32_t w[4] = {0, 0, 0, 0};
+        for (int64_t j = 0; 8 * c + j < T; ++j) w[j >> 1] |= (uint32_t)__ldg(row + 8 * c + j) << (16 * (j & 1));
+        v[u] = make_uint4(w[0], w[1], w[2], w[3]);
+      }
     }
 #pragma unroll
     for (int u = 0; u < 8; ++u) {
@@ -438,7 +445,7 @@ cudaError_t launch_gather_rows(const uint16_t* X, int64_t ldx, const int32_t* id
     if (e != cudaSuccess) return e;
     configured[dev] = true;
   }
-  const int64_t items = K * ((T / 8 + 255) / 256);
+  const int64_t items = K * (((T + 7) / 8 + 255) / 256);
   const int64_t want = (items + 7) / 8;  // 8 warps per CTA
   const int64_t cap = (int64_t)sm_count_current() * kGatherCtasPerSm;
   const int grid = (int)(want < cap ? (want > 0 ? want : 1) : cap);

@@ -56,6 +56,9 @@ struct SpmmParams {
   int bn;
   int kd;  // skinny stage depth (logical K per stage: 128 or 256)
   float* ws;
+  // fused prune + compress + GEMM: optional outputs of the compressed operand
+  uint16_t* out_vals;
+  uint32_t* out_meta;
 };
 
 int spmm_max_stages(int bn, uint32_t a_slot);
@@ -70,6 +73,8 @@ bool skinny_kernel_fits(int64_t T);
 int skinny_bn(int64_t T);
 int skinny_kd(int64_t K, int64_t T);
 cudaError_t launch_spmm_skinny(SpmmParams& p, cudaStream_t stream);
+cudaError_t launch_skinny_reduce(const SpmmParams& p, cudaStream_t stream);
+cudaError_t launch_prune_spmm_skinny(SpmmParams& p, cudaStream_t stream);
 cudaError_t launch_compress_stream(const CUtensorMap& tm_w, int64_t R, int64_t K, uint16_t* values, uint32_t* meta,
                                    uint32_t* status, cudaStream_t s);
 

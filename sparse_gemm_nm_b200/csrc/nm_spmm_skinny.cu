@@ -276,6 +276,18 @@ bool skinny_kernel_fits(int64_t T) { return T >= 1 && T <= 64; }
 
 int skinny_bn(int64_t T) { return T <= 16 ? 16 : T <= 32 ? 32 : 64; }
 
+// Sum of the K ranges' fp32 partials into Y (when the skinny kernels split K).
+cudaError_t launch_skinny_reduce(const SpmmParams& p, cudaStream_t stream) {
+  const int sms = sm_count_current();
+  const int64_t total = p.R * p.T;
+  const int64_t want = (total + 255) / 256;
+  const int grid = (int)(want < (int64_t)sms * 8 ? want : (int64_t)sms * 8);
+  cudaError_t e = launch_pdl(skinny_reduce_kernel, dim3(grid), dim3(256), 0, stream, (const float*)p.ws, p.splits,
+                             p.R, p.bn, p.T, p.Y, p.ldy, p.out_f32);
+  count_launch();
+  return e != cudaSuccess ? e : cudaGetLastError();
+}
+
 template <int BN, int KD>
 static cudaError_t launch_bn(SpmmParams& p, cudaStream_t stream) {
   using namespace skinny;
@@ -296,21 +308,7 @@ static cudaError_t launch_bn(SpmmParams& p, cudaStream_t stream) {
   count_launch();
   if (e == cudaSuccess) e = cudaGetLastError();
   if (e != cudaSuccess || p.splits == 1) return e;
-  const int64_t total = p.R * p.T;
-  const int64_t want = (total + 255) / 256;
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)(want < (int64_t)sms * 8 ? want : (int64_t)sms * 8));
-  cfg.blockDim = dim3(256);
-  cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  e = cudaLaunchKernelEx(&cfg, skinny_reduce_kernel, (const float*)p.ws, p.splits, p.R, BN, p.T, p.Y, p.ldy,
-                         p.out_f32);
-  count_launch();
-  return e != cudaSuccess ? e : cudaGetLastError();
+  return launch_skinny_reduce(p, stream);
 }
 
 int skinny_kd(int64_t K, int64_t T) { (void)T; return K % 128 == 0 ? 128 : 0; }

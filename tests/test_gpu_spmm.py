@@ -361,6 +361,25 @@ def test_skinny_kernel_permuted(n, m):
     check(W, X, n, m, idx=wl.permutation(K, 153), what=f"skinny permuted {n}:{m}")
 
 
+@pytest.mark.parametrize("T", [1, 13, 33])
+def test_skinny_kernel_permuted_ragged_columns(T):
+    """T % 8 != 0: X rows padded to 16 bytes; the gathered copy must carry the partial last piece."""
+    R, K = 200, 512
+    W = wl.normal_bf16((R, K), 0.02, seed=155 + T)
+    X = wl.normal_bf16((K, T), 1.0, seed=156)
+    idx = wl.permutation(K, 157)
+    ld = (T + 7) // 8 * 8
+    Xbuf = np.zeros((K, ld), np.uint16)
+    Xbuf[:, :T] = X
+    vals, meta = nm.prune_compress(to_dev(W), 2, 4)
+    Y = torch.empty((R, ld), dtype=torch.bfloat16, device=DEV)
+    nm.nm_spmm_permuted(vals, meta, 2, 4, R, K, to_dev_i32(idx), to_dev(Xbuf), ld, T, Y, ld)
+    torch.cuda.synchronize()
+    nm.nm_device_status()
+    ref, mag = reference(W, X, 2, 4, idx)
+    assert_gemm_close(values_f64(Y[:, :T]), ref, mag, f"skinny permuted T={T}")
+
+
 @pytest.mark.parametrize("out", [torch.bfloat16, torch.float32])
 def test_skinny_kernel_integer_exact(out):
     R, K, T = 384, 4096, 16  # several K ranges: partial sums are exact integers
