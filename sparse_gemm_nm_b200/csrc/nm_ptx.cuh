@@ -18,6 +18,30 @@ __device__ __forceinline__ uint64_t global_timer_ns() {
   return t;
 }
 
+// Wall time spent in a wait, robust to steps of %globaltimer (the driver may
+// adjust it; a backward step read as `now - start` would be a huge interval):
+// each reading adds only its forward step since the previous one, at most 1 ms.
+struct WaitClock {
+  uint64_t prev, waited;
+  __device__ __forceinline__ void start() {
+    prev = global_timer_ns();
+    waited = 0;
+  }
+  __device__ __forceinline__ uint64_t tick() {
+    const uint64_t now = global_timer_ns();
+    if (now > prev) waited += (now - prev) < 1000000ull ? (now - prev) : 1000000ull;
+    prev = now;
+    return waited;
+  }
+};
+
+// Sleep about `ns` nanoseconds (bounded also by an iteration count).
+__device__ __forceinline__ void sleep_about_ns(uint64_t ns) {
+  WaitClock c;
+  c.start();
+  for (uint32_t it = 0; c.tick() < ns && it < (uint32_t)(ns / 500u) + 1u; ++it) __nanosleep(1000);
+}
+
 // ---------------------------------------------------------------- mbarrier
 __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
@@ -59,12 +83,15 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 // on an already completed phase; ~142 with this split).
 static __device__ __noinline__ bool mbar_wait_slow(uint64_t* bar, uint32_t parity, volatile int* abort, uint32_t* status,
                                                    uint64_t limit_ns) {
-  const uint64_t t0 = global_timer_ns();
-  for (uint32_t it = 1;; ++it) {
+  WaitClock clock;
+  clock.start();
+  // Backstop for a timer that stops: an iteration takes well over 4 ns.
+  const uint64_t max_iters = (limit_ns >> 2) + 64u;
+  for (uint64_t it = 1;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
     if ((it & 63u) == 0u) {
       if (*abort) return false;
-      if (global_timer_ns() - t0 > limit_ns) {
+      if (clock.tick() > limit_ns || it > max_iters) {
         *abort = 1;
         atomicOr(status, 1u);
         return false;

@@ -553,8 +553,7 @@ __global__ void __launch_bounds__(kThreads, 1) spmm_kernel(const __grid_constant
   __syncthreads();
   if (*abort_flag && threadIdx.x == 0) {
     // give TMA copies that were already issued time to land (bounded)
-    const uint64_t t0 = global_timer_ns();
-    while (global_timer_ns() - t0 < 200000ull) __nanosleep(1000);
+    sleep_about_ns(200000ull);
   }
   __syncthreads();
   if (warp == 1) {

@@ -301,8 +301,7 @@ __global__ void __launch_bounds__(fused::kThreads, 1) prune_spmm_skinny_kernel(c
   // ------------------------------------------------------------- teardown
   __syncthreads();
   if (*abort_flag && threadIdx.x == 0) {
-    const uint64_t t0 = global_timer_ns();
-    while (global_timer_ns() - t0 < 200000ull) __nanosleep(1000);
+    sleep_about_ns(200000ull);
   }
   if (warp == 1) {
     __syncwarp();

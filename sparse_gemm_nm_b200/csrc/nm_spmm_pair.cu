@@ -302,8 +302,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pair::kThreads, 1)
   // -------------------------------------------------------------- teardown
   __syncthreads();
   if (*abort_flag && threadIdx.x == 0) {
-    const uint64_t t0 = global_timer_ns();
-    while (global_timer_ns() - t0 < 200000ull) __nanosleep(1000);
+    sleep_about_ns(200000ull);
   }
   cluster_sync();
   if (warp == 1) {

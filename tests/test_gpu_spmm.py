@@ -163,6 +163,28 @@ def test_permuted_identity_equals_plain_and_host_permuted():
     assert torch.equal(perm, host)  # same tiles, same MMA order: bitwise equal
 
 
+@pytest.mark.parametrize("T", [256, 16, 100])  # gather pass + SM-pair kernel, gather pass + skinny, one SM
+def test_permuted_out_of_range_entries_read_zero_rows(T):
+    R, K = 300, 512
+    W = wl.normal_bf16((R, K), 0.02, seed=74)
+    X = wl.normal_bf16((K, T), 1.0, seed=75)
+    idx = wl.permutation(K, 76).astype(np.int32)
+    idx[[0, 5, 130, 257, 511]] = [-1, K, K + 1000, -(2 ** 31), 2 ** 31 - 1]
+    ld = (T + 7) // 8 * 8
+    Xbuf = np.zeros((K, ld), np.uint16)
+    Xbuf[:, :T] = X
+    vals, meta = nm.prune_compress(to_dev(W), 2, 4)
+    Y = torch.empty((R, ld), dtype=torch.bfloat16, device=DEV)
+    nm.nm_spmm_permuted(vals, meta, 2, 4, R, K, to_dev_i32(idx), to_dev(Xbuf), ld, T, Y, ld)
+    torch.cuda.synchronize()
+    nm.nm_device_status()
+    Xp = np.zeros((K, T), np.uint16)  # the permuted input by its definition, zero rows for the bad entries
+    ok = (idx >= 0) & (idx < K)
+    Xp[ok] = X[idx[ok]]
+    ref, mag = reference(W, Xp, 2, 4)
+    assert_gemm_close(values_f64(Y[:, :T]), ref, mag, f"out-of-range idx, T={T}")
+
+
 def test_permuted_ragged_k():
     R, K, T = 130, 1040, 64
     W = wl.normal_bf16((R, K), 0.02, seed=71)

@@ -1,10 +1,10 @@
-"""The allocation-free permuted GEMM (nm_spmm_permuted_noalloc) against nm_spmm_permuted.
+"""The allocation-free permuted GEMM (nm_spmm_permuted_noalloc) against the oracle.
 
 nm_spmm_permuted_noalloc is for callers that cannot let the library take
 device memory; it stages the gathered input in a fixed array inside the
-library instead of a pool allocation.  Each case calls it twice in a row
-with different inputs (the array keeps the previous call's contents) and
-compares both outputs with the ordinary entry point's, within the acceptance
+library instead of a pool allocation.  Each case calls
+it twice in a row with different inputs (the array keeps the previous call's
+contents) and compares both outputs with the oracle, within the acceptance
 rule the other GEMM tests use.  This file is collected last on purpose.
 """
 import numpy as np
@@ -27,29 +27,28 @@ def _bound(W, X, idx):
     return np.abs(Wd) @ np.abs(Xp)
 
 
-def _run_both(W, X, idx):
+def _run_noalloc(W, X, idx):
     R, K = W.shape
     T = X.shape[1]
     vals, meta = nm.prune_compress(to_dev(W), 2, 4)
-    Xd, idxd = to_dev(X), to_dev_i32(idx)
-    y_ref = torch.empty((R, T), dtype=torch.bfloat16, device=DEV)
-    y_new = torch.full((R, T), 5.0, dtype=torch.bfloat16, device=DEV)
-    nm.nm_spmm_permuted(vals, meta, 2, 4, R, K, idxd, Xd, T, T, y_ref, T)
-    nm.nm_spmm_permuted_noalloc(vals, meta, 2, 4, R, K, idxd, Xd, T, T, y_new, T)
+    y = torch.full((R, T), 5.0, dtype=torch.bfloat16, device=DEV)
+    nm.nm_spmm_permuted_noalloc(vals, meta, 2, 4, R, K, to_dev_i32(idx), to_dev(X), T, T, y, T)
     torch.cuda.synchronize()
     nm.nm_device_status()
-    return values_f64(y_ref), values_f64(y_new)
+    ov, om = oracle.compress(W, 2, 4)
+    ref = oracle.dense_gemm(oracle.decompress(ov, om, K, 2, 4), X, idx)
+    return values_f64(y), ref
 
 
 @pytest.mark.parametrize("R,K,T", [(512, 1024, 512),     # one chunk
                                    (128, 8192, 2304)])   # two chunks of the 32 MiB array, the second ragged
-def test_noalloc_matches_permuted_twice(R, K, T):
+def test_noalloc_matches_oracle_twice(R, K, T):
     for call in range(2):  # second call: new inputs, array still holds the first call's chunks
         W = wl.normal_bf16((R, K), 0.02, seed=1000 + 10 * call + K)
         X = wl.normal_bf16((K, T), 1.0, seed=2000 + 10 * call + T)
         idx = wl.permutation(K, 3000 + call)
-        y_ref, y_new = _run_both(W, X, idx)
-        assert_gemm_close(y_new, y_ref, _bound(W, X, idx), f"no-alloc call {call + 1}")
+        y, ref = _run_noalloc(W, X, idx)
+        assert_gemm_close(y, ref, _bound(W, X, idx), f"no-alloc call {call + 1}")
 
 
 def test_noalloc_other_shapes_run_as_permuted():
@@ -57,8 +56,8 @@ def test_noalloc_other_shapes_run_as_permuted():
     W = wl.normal_bf16((R, K), 0.02, seed=5)
     X = wl.normal_bf16((K, T), 1.0, seed=6)
     idx = wl.permutation(K, 7)
-    y_ref, y_new = _run_both(W, X, idx)
-    assert_gemm_close(y_new, y_ref, _bound(W, X, idx), "delegated shape")
+    y, ref = _run_noalloc(W, X, idx)
+    assert_gemm_close(y, ref, _bound(W, X, idx), "delegated shape")
 
 
 def test_noalloc_rejects_k_beyond_the_array():
