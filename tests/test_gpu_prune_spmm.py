@@ -179,3 +179,35 @@ def test_edge_cases():
     # only one of values / meta
     with pytest.raises(nm.NmError):
         nm.nm_prune_spmm(W, 128, 2, 4, 64, 128, None, X, 8, 8, Y, 8, values=vals)
+
+
+# ----------------------------------------------------------------------------
+# CUDA graphs: the calls (staging allocations and gather passes included)
+# capture and replay
+# ----------------------------------------------------------------------------
+def test_graph_capture_replays_permuted_calls():
+    R, K, T = 512, 1024, 256
+    W = wl.normal_bf16((R, K), 0.02, seed=271)
+    X = wl.normal_bf16((K, T), 1.0, seed=272)
+    idx = wl.permutation(K, 273)
+    Wd, Xd, idxd = to_dev(W), to_dev(X), to_dev_i32(idx)
+    direct, vals, meta = nm.prune_spmm(Wd, 2, 4, Xd, idx=idxd, keep_compressed=True)
+    torch.cuda.synchronize()
+    Y1 = torch.empty((R, T), dtype=torch.bfloat16, device=DEV)
+    Y2 = torch.empty_like(Y1)
+    v = torch.empty_like(vals)
+    mt = torch.empty_like(meta)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        nm.nm_prune_spmm(Wd, K, 2, 4, R, K, idxd, Xd, T, T, Y1, T, values=v, meta=mt)
+        nm.nm_spmm_permuted(vals, meta, 2, 4, R, K, idxd, Xd, T, T, Y2, T)
+    for _ in range(2):
+        Y1.zero_()
+        Y2.zero_()
+        g.replay()
+        torch.cuda.synchronize()
+        nm.nm_device_status()
+        assert torch.equal(Y1, direct) and torch.equal(Y2, direct)
+        assert torch.equal(v, vals) and torch.equal(mt, meta)
+    ref, mag, _, _ = reference(W, X, 2, 4, idx)
+    assert_gemm_close(values_f64(Y1), ref, mag, "graph replay")
