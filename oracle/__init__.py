@@ -17,6 +17,9 @@ Sources, by page title and passage:
   * "Technische Samenvatting: SHUFFLESPARSE", "2. Methodologie": y = (W Pi) x
     with Pi applied as an index map on the input read.
   * "Structured Sparsity" topic cards, PATCH abstract: per-tile dense / 2:4.
+  * "Structured Sparsity" topic cards, RNM-TD3 abstract, and the DynaDiag
+    page's abstract: N:M structure kept through training, sparse forward and
+    backward passes (the gradients :func:`spmm_t` and :func:`sddmm`).
 """
 from __future__ import annotations
 
@@ -64,6 +67,8 @@ def _load():
                 "oracle_dense_gemm": ([P, I64, I64, I64, P, I64, I64, P, P, P, I64], I),
                 "oracle_hybrid_weights": ([P, I64, I64, I64, P, I64, P], I),
                 "oracle_hybrid_spmm": ([P, I64, I64, I64, P, I64, P, I64, I64, P, P, I64], I),
+                "oracle_spmm_t": ([P, P, I, I, I64, I64, P, I64, I64, P, P, P, I64], I),
+                "oracle_sddmm": ([P, I, I, I64, I64, P, I64, P, I64, I64, P, P, P], I),
             }
             for name, (args, res) in sig.items():
                 fn = getattr(lib, name)
@@ -217,3 +222,33 @@ def hybrid_spmm(W, tile_map, X, tile=128, with_abs=False):
     _check(_load().oracle_hybrid_spmm(_ptr(W), R, K, K, _ptr(tile_map), tile, _ptr(X), T, T,
                                       _ptr(Y), _ptr(A), T), "hybrid_spmm")
     return (Y, A) if with_abs else Y
+
+
+def spmm_t(values, meta, n, m, K, dY, idx=None, with_abs=False):
+    """fp64 input gradient of y = (W' Pi) X: dX (K x T) from dY (R x T), the adjoint of the gather."""
+    values = _u16(values)
+    meta = np.ascontiguousarray(meta, dtype=np.uint32)
+    dY = _u16(dY)
+    R, T = dY.shape
+    if idx is not None:
+        idx = np.ascontiguousarray(idx, dtype=np.int32)
+    dX = np.zeros((K, T), np.float64)
+    A = np.zeros((K, T), np.float64) if with_abs else None
+    _check(_load().oracle_spmm_t(_ptr(values), _ptr(meta), n, m, R, K, _ptr(dY), T, T, _ptr(idx), _ptr(dX),
+                                 _ptr(A), T), "spmm_t")
+    return (dX, A) if with_abs else dX
+
+
+def sddmm(meta, n, m, R, K, dY, X, idx=None, with_abs=False):
+    """fp64 gradient of the stored values: dV[r][j] = sum_t dY[r][t] X[pi(k_j)][t] (R x K*n/m)."""
+    meta = np.ascontiguousarray(meta, dtype=np.uint32)
+    dY = _u16(dY)
+    X = _u16(X)
+    T = dY.shape[1]
+    if idx is not None:
+        idx = np.ascontiguousarray(idx, dtype=np.int32)
+    dV = np.zeros((R, value_cols(K, n, m)), np.float64)
+    A = np.zeros_like(dV) if with_abs else None
+    _check(_load().oracle_sddmm(_ptr(meta), n, m, R, K, _ptr(dY), T, _ptr(X), X.shape[1], T, _ptr(idx),
+                                _ptr(dV), _ptr(A)), "sddmm")
+    return (dV, A) if with_abs else dV

@@ -36,6 +36,10 @@
  *             its input at the permuted addresses (same FLOP count).
  *  [PATCH]    "Structured Sparsity" topic cards, the PATCH abstract: weight
  *             matrices are split into tiles, each tile either dense or 2:4.
+ *  [TRAIN]    "Structured Sparsity" topic cards, RNM-TD3 abstract (N:M
+ *             sparsity kept through the whole of training) and the
+ *             DynaDiag page's abstract (sparse computation in the forward
+ *             and the backward pass): the gradients of y = (W' Pi) x.
  *
  * Readings where the pages are silent (each listed in the design notes):
  *  - ties in magnitude go to the lower index inside the group;
@@ -53,7 +57,12 @@
  *    a B200 sparse tensor-core instruction reads them ("tiled" packing, see
  *    meta_slot_2of4 below); groups past R or K in the padded tiles hold the
  *    nibble of an all-zero group, positions (0,1);
- *  - the permutation is applied as X_perm[k][t] = X[idx[k]][t];
+ *  - the permutation is applied as X_perm[k][t] = X[idx[k]][t]; an entry of
+ *    idx outside [0, K) reads a zero row;
+ *  - backward: dX is the adjoint of that gather (row k of W'^T dY is added to
+ *    row idx[k] of dX; entries outside [0, K) drop their row, repeated
+ *    entries add up), and the gradient of the stored values is
+ *    dV[r][j] = sum_t dY[r][t] * X_perm[k_j][t] for the survivor's column k_j;
  *  - W (dense, R x K) and the compressed values hold bf16 bit patterns
  *    (uint16); X is K x T row-major; Y is R x T (double here).
  */
@@ -282,6 +291,7 @@ int oracle_spmm(const uint16_t *values, const uint32_t *meta, int n, int m,
             for (int64_t j = 0; j < vcols; j++) {
                 int64_t k = (j / n) * m + position_of(meta, K, r, j, n, m);
                 int64_t src = idx ? (int64_t)idx[k] : k;
+                if (src < 0 || src >= K) continue; /* a zero row */
                 acc += bf16_value(values[r * vcols + j]) * bf16_value(X[src * ldx + t]);
             }
             Y[r * ldy + t] = acc;
@@ -307,7 +317,7 @@ int oracle_spmm_sampled(const uint16_t *values, const uint32_t *meta, int n, int
             int64_t k = (j / n) * m + position_of(meta, K, r, j, n, m);
             int64_t src = idx ? (int64_t)idx[k] : k;
             double w = bf16_value(values[r * vcols + j]);
-            double x = bf16_value(X[src * ldx + t]);
+            double x = (src < 0 || src >= K) ? 0.0 : bf16_value(X[src * ldx + t]);
             acc += w * x;
             mag += fabs(w) * fabs(x);
         }
@@ -335,7 +345,7 @@ int oracle_dense_gemm(const uint16_t *W, int64_t R, int64_t K, int64_t ldw,
             for (int64_t k = 0; k < K; k++) {
                 int64_t src = idx ? (int64_t)idx[k] : k;
                 double w = bf16_value(W[r * ldw + k]);
-                double x = bf16_value(X[src * ldx + t]);
+                double x = (src < 0 || src >= K) ? 0.0 : bf16_value(X[src * ldx + t]);
                 acc += w * x;
                 mag += fabs(w) * fabs(x);
             }
@@ -382,4 +392,72 @@ int oracle_hybrid_spmm(const uint16_t *W, int64_t R, int64_t K, int64_t ldw,
     if (rc == 0) rc = oracle_dense_gemm(W_eff, R, K, K, X, ldx, T, NULL, Y, Y_abs, ldy);
     free(W_eff);
     return rc;
+}
+
+/* ------------------------------------------------------------------ */
+/* Backward products of y = (W' Pi) x [TRAIN], [SS-perm], [MN-gemm].    */
+/* dY is R x T (the gradient of y).                                     */
+/*                                                                      */
+/* Input gradient: with Xp[k] = X[pi(k)], y = W' Xp gives               */
+/*   dXp[k][t] = sum_r W'[r][k] * dY[r][t],  and dX[pi(k)] += dXp[k].    */
+/* Only survivors are non-zero in W', so the sum runs over the stored   */
+/* values: survivor j of row r sits in column k = (j/N)*M + pos_j.      */
+/* dX (K x T) is overwritten; dX_abs (optional) gets the sums of        */
+/* |products|.  Entries of idx outside [0, K) drop their row.           */
+/* ------------------------------------------------------------------ */
+int oracle_spmm_t(const uint16_t *values, const uint32_t *meta, int n, int m,
+                  int64_t R, int64_t K, const uint16_t *dY, int64_t lddy, int64_t T,
+                  const int32_t *idx, double *dX, double *dX_abs, int64_t lddx)
+{
+    if (!pattern_ok(n, m) || K % m != 0 || lddy < T || lddx < T) return 1;
+    int64_t vcols = oracle_value_cols(K, n, m);
+    for (int64_t k = 0; k < K; k++)
+        for (int64_t t = 0; t < T; t++) {
+            dX[k * lddx + t] = 0.0;
+            if (dX_abs) dX_abs[k * lddx + t] = 0.0;
+        }
+    for (int64_t r = 0; r < R; r++) {
+        for (int64_t j = 0; j < vcols; j++) {
+            int64_t k = (j / n) * m + position_of(meta, K, r, j, n, m);
+            int64_t dst = idx ? (int64_t)idx[k] : k;
+            if (dst < 0 || dst >= K) continue;
+            double w = bf16_value(values[r * vcols + j]);
+            for (int64_t t = 0; t < T; t++) {
+                double g = bf16_value(dY[r * lddy + t]);
+                dX[dst * lddx + t] += w * g;
+                if (dX_abs) dX_abs[dst * lddx + t] += fabs(w) * fabs(g);
+            }
+        }
+    }
+    return 0;
+}
+
+/* Gradient of the stored values: dV[r][j] = sum_t dY[r][t] * Xp[k_j][t], */
+/* the entries of dY Xp^T at the survivors' columns only (a sampled      */
+/* dense-dense product).  dV is R x K*N/M; dV_abs (optional) gets the     */
+/* sums of |products|.                                                    */
+int oracle_sddmm(const uint32_t *meta, int n, int m, int64_t R, int64_t K,
+                 const uint16_t *dY, int64_t lddy, const uint16_t *X, int64_t ldx, int64_t T,
+                 const int32_t *idx, double *dV, double *dV_abs)
+{
+    if (!pattern_ok(n, m) || K % m != 0 || lddy < T || ldx < T) return 1;
+    int64_t vcols = oracle_value_cols(K, n, m);
+    for (int64_t r = 0; r < R; r++) {
+        for (int64_t j = 0; j < vcols; j++) {
+            int64_t k = (j / n) * m + position_of(meta, K, r, j, n, m);
+            int64_t src = idx ? (int64_t)idx[k] : k;
+            double acc = 0.0, mag = 0.0;
+            if (src >= 0 && src < K) {
+                for (int64_t t = 0; t < T; t++) {
+                    double g = bf16_value(dY[r * lddy + t]);
+                    double x = bf16_value(X[src * ldx + t]);
+                    acc += g * x;
+                    mag += fabs(g) * fabs(x);
+                }
+            }
+            dV[r * vcols + j] = acc;
+            if (dV_abs) dV_abs[r * vcols + j] = mag;
+        }
+    }
+    return 0;
 }
