@@ -233,6 +233,50 @@ NM_API nm_status nm_prune_spmm(const uint16_t* W, int64_t ldw, int n, int m, int
                                const int32_t* idx, const uint16_t* X, int64_t ldx, int64_t T, void* Y, int64_t ldy,
                                nm_out_dtype y_dtype, uint16_t* values, uint32_t* meta, void* stream);
 
+/* ------------------------------------------------------------- backward */
+/*
+ * nm_spmm_t -- input gradient of y = (W' Pi) x: dX = (W' Pi)^T dY, i.e.
+ * dXp = W'^T dY (K x T) and dX[idx[k]] = dXp[k] (dX = dXp when idx is NULL).
+ * Source: "Structured Sparsity" topic cards, RNM-TD3 abstract (N:M sparsity
+ * kept through training), and the DynaDiag page's abstract (sparse forward
+ * and backward passes); the gather of nm_spmm_permuted, whose adjoint this is.
+ * W'^T is N:M along its output axis, not along the reduction axis R, so the
+ * sparse MMA cannot take it: W' is decompressed into a staging buffer
+ * (R x ceil8(K) bf16 from the library's pool, one launch) and a dense
+ * tcgen05 GEMM on SM pairs reads it transposed (a second launch).
+ *   values, meta [in] compressed R x K weights, pattern n:m
+ *   idx  [in] NULL, or a permutation of [0, K) (the forward's index map):
+ *        row k of W'^T dY is written to row idx[k] of dX; entries outside
+ *        [0, K) drop their row; repeated entries are not supported (their
+ *        rows race), and rows of dX that no entry names are not written
+ *   dY   [in]  R x T bf16, row stride lddy >= T, lddy % 8 == 0
+ *   dX   [out] K x T, bf16 or fp32 (dtype), row stride lddx >= T, 16-byte rows
+ * Errors: as nm_spmm.
+ */
+NM_API nm_status nm_spmm_t(const uint16_t* values, const uint32_t* meta, int n, int m, int64_t R, int64_t K,
+                           const int32_t* idx, const uint16_t* dY, int64_t lddy, int64_t T, void* dX, int64_t lddx,
+                           nm_out_dtype dtype, void* stream);
+
+/*
+ * nm_sddmm -- gradient of the stored values of y = (W' Pi) x:
+ * dV[r][j] = sum_t dY[r][t] * X[idx[k_j]][t], with k_j the column of
+ * survivor j of row r (group j / n, position from meta; X[idx[k]] = X[k]
+ * when idx is NULL, a zero row for an entry outside [0, K)).  These are the
+ * entries of dY Xp^T at the survivors, in the layout of `values`.
+ * Source: same passages as nm_spmm_t.
+ * The full product dY Xp^T runs as a dense tcgen05 GEMM on SM pairs and the
+ * epilogue stores only the survivor entries.  With idx, one gather pass first
+ * stages Xp (K x ceil8(T) bf16 from the library's pool).
+ *   meta [in]  metadata of the compressed R x K weights, pattern n:m
+ *   dY   [in]  R x T bf16, row stride lddy >= T, lddy % 8 == 0
+ *   X    [in]  K x T bf16, row stride ldx >= T, ldx % 8 == 0
+ *   dV   [out] R x nm_value_cols(K,n,m), bf16 or fp32 (dtype), contiguous rows
+ * Errors: as nm_spmm.
+ */
+NM_API nm_status nm_sddmm(const uint32_t* meta, int n, int m, int64_t R, int64_t K, const int32_t* idx,
+                          const uint16_t* dY, int64_t lddy, const uint16_t* X, int64_t ldx, int64_t T, void* dV,
+                          nm_out_dtype dtype, void* stream);
+
 /*
  * nm_spmm_algo --nm_spmm / nm_spmm_permuted (idx may be NULL) with the kernel
  * design chosen explicitly, to compare the sparse tensor-core path with the

@@ -3,11 +3,12 @@
 Python binding of the C ABI in ``include/nm.h`` (library ``libnm_b200.so``).
 The functions named like the C entry points (``nm_prune_compress``,
 ``nm_decompress``, ``nm_spmm``, ``nm_spmm_permuted``, ``nm_hybrid_spmm``,
-``nm_spmm_algo``, ``nm_prune_spmm``) only marshal arguments: tensors become device pointers, the
+``nm_spmm_algo``, ``nm_prune_spmm``, ``nm_spmm_t``, ``nm_sddmm``) only marshal arguments: tensors become device pointers, the
 stream defaults to torch's current stream, and a non-zero status raises
 :class:`NmError`.  Every step of the computation runs in the library's CUDA
 kernels; there is no fallback of any kind.  The convenience wrappers
-(``prune_compress``, ``decompress``, ``spmm``, ``hybrid_spmm``, ``prune_spmm``) also allocate
+(``prune_compress``, ``decompress``, ``spmm``, ``hybrid_spmm``, ``prune_spmm``, ``spmm_t``,
+``sddmm``) also allocate
 the outputs with torch.
 
 bf16 data is accepted as ``torch.bfloat16`` tensors (or int16/uint16 views of
@@ -49,6 +50,8 @@ SIGNATURES = {
     "nm_spmm_permuted": ([_P, _P, _I, _I, _I64, _I64, _P, _P, _I64, _I64, _P, _I64, _I, _P], _I),
     "nm_hybrid_spmm": ([_P, _I64, _P, _P, _P, _I, _I64, _I64, _P, _I64, _I64, _P, _I64, _I, _P], _I),
     "nm_prune_spmm": ([_P, _I64, _I, _I, _I64, _I64, _P, _P, _I64, _I64, _P, _I64, _I, _P, _P, _P], _I),
+    "nm_spmm_t": ([_P, _P, _I, _I, _I64, _I64, _P, _P, _I64, _I64, _P, _I64, _I, _P], _I),
+    "nm_sddmm": ([_P, _I, _I, _I64, _I64, _P, _P, _I64, _P, _I64, _I64, _P, _I, _P], _I),
     "nm_spmm_algo": ([_P, _P, _I, _I, _I64, _I64, _P, _P, _I64, _I64, _P, _I64, _I, _I, _P], _I),
     "nm_spmm_permuted_noalloc": ([_P, _P, _I, _I, _I64, _I64, _P, _P, _I64, _I64, _P, _I64, _I, _P], _I),
     "nm_release_staging": ([], _I),
@@ -160,6 +163,16 @@ def nm_prune_spmm(W, ldw, n, m, R, K, idx, X, ldx, T, Y, ldy, y_dtype=NM_OUT_BF1
                   stream=None) -> None:
     _check(lib().nm_prune_spmm(_ptr(W), ldw, n, m, R, K, _ptr(idx), _ptr(X), ldx, T, _ptr(Y), ldy, y_dtype,
                                _ptr(values), _ptr(meta), _stream(stream)), "nm_prune_spmm")
+
+
+def nm_spmm_t(values, meta, n, m, R, K, idx, dY, lddy, T, dX, lddx, dtype=NM_OUT_BF16, stream=None) -> None:
+    _check(lib().nm_spmm_t(_ptr(values), _ptr(meta), n, m, R, K, _ptr(idx), _ptr(dY), lddy, T, _ptr(dX), lddx,
+                           dtype, _stream(stream)), "nm_spmm_t")
+
+
+def nm_sddmm(meta, n, m, R, K, idx, dY, lddy, X, ldx, T, dV, dtype=NM_OUT_BF16, stream=None) -> None:
+    _check(lib().nm_sddmm(_ptr(meta), n, m, R, K, _ptr(idx), _ptr(dY), lddy, _ptr(X), ldx, T, _ptr(dV), dtype,
+                          _stream(stream)), "nm_sddmm")
 
 
 def nm_spmm_algo(values, meta, n, m, R, K, idx, X, ldx, T, Y, ldy, y_dtype=NM_OUT_BF16, algo=NM_ALGO_AUTO,
@@ -279,3 +292,29 @@ def prune_spmm(W, n: int, m: int, X, idx=None, out_dtype=None, keep_compressed: 
     nm_prune_spmm(W, W.stride(0), n, m, R, K, idx, X, X.stride(0), T, Y, ldy, yt, vals, meta, stream)
     Y = Y[:, :T]
     return (Y, vals, meta) if keep_compressed else Y
+
+
+def spmm_t(values, meta, n: int, m: int, K: int, dY, idx=None, out_dtype=None, stream=None):
+    """dX = (W' Pi)^T dY (K x T) from the compressed operand; idx=None means Pi = I."""
+    import torch
+    _require_cuda(values, meta, dY, idx)
+    out_dtype = out_dtype or torch.bfloat16
+    R, T = dY.shape
+    per16 = 4 if out_dtype == torch.float32 else 8
+    ld = max((T + per16 - 1) // per16 * per16, per16)
+    dX = torch.empty((K, ld), dtype=out_dtype, device=dY.device)
+    yt = NM_OUT_F32 if out_dtype == torch.float32 else NM_OUT_BF16
+    nm_spmm_t(values, meta, n, m, R, K, idx, dY, dY.stride(0), T, dX, ld, yt, stream)
+    return dX[:, :T]
+
+
+def sddmm(meta, n: int, m: int, R: int, K: int, dY, X, idx=None, out_dtype=None, stream=None):
+    """dV[r][j] = sum_t dY[r][t] X[idx[k_j]][t] (R x K*n/m), the gradient of the stored values."""
+    import torch
+    _require_cuda(meta, dY, X, idx)
+    out_dtype = out_dtype or torch.bfloat16
+    T = dY.shape[1]
+    dV = torch.empty((R, max(nm_value_cols(K, n, m), 0)), dtype=out_dtype, device=dY.device)
+    yt = NM_OUT_F32 if out_dtype == torch.float32 else NM_OUT_BF16
+    nm_sddmm(meta, n, m, R, K, idx, dY, dY.stride(0), X, X.stride(0), T, dV, yt, stream)
+    return dV

@@ -746,6 +746,141 @@ static nm_status run_prune_gemm(const uint16_t* W, int64_t ldw, int n, int m, in
   return e == cudaSuccess ? NM_OK : cuda_fail(e, "fused prune + GEMM launch");
 }
 
+
+// Backward products of y = (W' Pi) x on the dense SM-pair GEMM.
+static nm_status check_bwd_common(int n, int m, int64_t R, int64_t K, int64_t T, nm_out_dtype dtype) {
+  if (R < 0 || K < 0 || T < 0) return fail(NM_ERR_INVALID_ARG, "negative dimension");
+  if (!pattern_ok(n, m)) return fail(NM_ERR_INVALID_ARG, "pattern %d:%d not supported", n, m);
+  if (K % m != 0) return fail(NM_ERR_INVALID_ARG, "K=%lld is not a multiple of M=%d", (long long)K, m);
+  if (dtype != NM_OUT_BF16 && dtype != NM_OUT_F32) return fail(NM_ERR_INVALID_ARG, "bad output dtype");
+  if (R >= (1ll << 31) || K >= (1ll << 31) || T >= (1ll << 31))
+    return fail(NM_ERR_UNSUPPORTED, "dimensions must stay below 2^31");
+  return NM_OK;
+}
+
+static nm_status run_spmm_t(const uint16_t* values, const uint32_t* meta, int n, int m, int64_t R, int64_t K,
+                            const int32_t* idx, const uint16_t* dY, int64_t lddy, int64_t T, void* dX, int64_t lddx,
+                            nm_out_dtype dtype, cudaStream_t stream) {
+  t_last_error.clear();
+  nm_status st = check_bwd_common(n, m, R, K, T, dtype);
+  if (st != NM_OK) return st;
+  if (K == 0 || T == 0) return NM_OK;
+  if (!dX) return fail(NM_ERR_INVALID_ARG, "dX is null");
+  if (lddx < T) return fail(NM_ERR_INVALID_ARG, "lddx < T");
+  const int esize = dtype == NM_OUT_F32 ? 4 : 2;
+  if (!al16(dX) || (lddx * esize) % 16 != 0) return fail(NM_ERR_MISALIGNED, "dX rows must be 16-byte aligned");
+  st = require_device();
+  if (st != NM_OK) return st;
+  if (R == 0) {  // no rows of W': the gradient is zero
+    cudaError_t e = launch_fill_zero(dX, K, T, lddx, esize, stream);
+    return e == cudaSuccess ? NM_OK : cuda_fail(e, "zero fill");
+  }
+  if (!values || !meta || !dY) return fail(NM_ERR_INVALID_ARG, "null operand");
+  if (lddy < T) return fail(NM_ERR_INVALID_ARG, "lddy < T");
+  if (!al16(dY) || lddy % 8 != 0) return fail(NM_ERR_MISALIGNED, "dY rows must be 16-byte aligned");
+  // W' written out densely (R x ldk bf16, rows padded to 16 bytes) in a staging buffer
+  cudaMemPool_t pool = nullptr;
+  cudaError_t e = staging_pool(&pool);
+  if (e != cudaSuccess) return cuda_fail(e, "staging pool");
+  const int64_t ldk = (K + 7) / 8 * 8;
+  void* wd = nullptr;
+  e = cudaMallocFromPoolAsync(&wd, (size_t)(R * ldk * 2), pool, stream);
+  if (e != cudaSuccess) return cuda_fail(e, "staging buffer for the decompressed weights");
+  e = launch_decompress(values, meta, R, K, n, m, static_cast<uint16_t*>(wd), ldk, stream);
+  DenseParams p;
+  std::memset(&p, 0, sizeof p);
+  p.M = K;
+  p.N = T;
+  p.Kr = R;
+  p.k_tiles = (R + 127) / 128;
+  p.tiles_m = (int)((K + 255) / 256);
+  p.tiles_n = (int)((T + 255) / 256);
+  p.num_tiles = p.tiles_m * p.tiles_n;
+  p.status = status_word_ptr();
+  p.out = dX;
+  p.ldo = lddx;
+  p.out_f32 = dtype == NM_OUT_F32;
+  p.row_map = idx;
+  p.rows_out = K;
+  if (e == cudaSuccess && !p.status) e = cudaErrorInvalidSymbol;
+  if ((int64_t)p.tiles_m * p.tiles_n >= (1ll << 31)) st = fail(NM_ERR_UNSUPPORTED, "too many tiles");
+  if (e == cudaSuccess && st == NM_OK)
+    st = make_tmap(&p.tm_a, wd, (uint64_t)K, (uint64_t)R, (uint64_t)ldk * 2, 64, 64, 128, "W' (dense)");
+  if (e == cudaSuccess && st == NM_OK)
+    st = make_tmap(&p.tm_b, dY, (uint64_t)T, (uint64_t)R, (uint64_t)lddy * 2, 64, 64, 128, "dY");
+  if (e == cudaSuccess && st == NM_OK) e = launch_dense_pair(p, true, true, EPI_STORE, stream);
+  cudaFreeAsync(wd, stream);
+  if (st != NM_OK) return st;
+  return e == cudaSuccess ? NM_OK : cuda_fail(e, "transposed GEMM launch");
+}
+
+static nm_status run_sddmm(const uint32_t* meta, int n, int m, int64_t R, int64_t K, const int32_t* idx,
+                           const uint16_t* dY, int64_t lddy, const uint16_t* X, int64_t ldx, int64_t T, void* dV,
+                           nm_out_dtype dtype, cudaStream_t stream) {
+  t_last_error.clear();
+  nm_status st = check_bwd_common(n, m, R, K, T, dtype);
+  if (st != NM_OK) return st;
+  if (R == 0 || K == 0) return NM_OK;
+  if (!dV || !meta) return fail(NM_ERR_INVALID_ARG, "null operand");
+  const int esize = dtype == NM_OUT_F32 ? 4 : 2;
+  if ((reinterpret_cast<uintptr_t>(dV) & (uintptr_t)(esize - 1)) != 0) return fail(NM_ERR_MISALIGNED, "dV misaligned");
+  st = require_device();
+  if (st != NM_OK) return st;
+  const int64_t vcols = value_cols(K, n, m);
+  if (T == 0) {  // an empty reduction: every gradient entry is zero
+    cudaError_t e = launch_fill_zero(dV, R, vcols, vcols, esize, stream);
+    return e == cudaSuccess ? NM_OK : cuda_fail(e, "zero fill");
+  }
+  if (!dY || !X) return fail(NM_ERR_INVALID_ARG, "null operand");
+  if (lddy < T || ldx < T) return fail(NM_ERR_INVALID_ARG, "leading dimension < T");
+  if (!al16(dY) || lddy % 8 != 0 || !al16(X) || ldx % 8 != 0)
+    return fail(NM_ERR_MISALIGNED, "dY and X rows must be 16-byte aligned");
+  cudaError_t e = cudaSuccess;
+  void* staged = nullptr;
+  const uint16_t* xsrc = X;
+  int64_t ldsrc = ldx;
+  if (idx) {  // Xp[k] = X[idx[k]] staged once, then read as the K-major B operand
+    cudaMemPool_t pool = nullptr;
+    e = staging_pool(&pool);
+    if (e != cudaSuccess) return cuda_fail(e, "staging pool");
+    const int64_t ldp = (T + 7) / 8 * 8;
+    e = cudaMallocFromPoolAsync(&staged, (size_t)(K * ldp * 2), pool, stream);
+    if (e != cudaSuccess) return cuda_fail(e, "staging buffer for the permuted input");
+    e = launch_gather_rows(X, ldx, idx, K, T, static_cast<uint16_t*>(staged), ldp, stream);
+    xsrc = static_cast<const uint16_t*>(staged);
+    ldsrc = ldp;
+  }
+  DenseParams p;
+  std::memset(&p, 0, sizeof p);
+  p.M = R;
+  p.N = K;
+  p.Kr = T;
+  p.k_tiles = (T + 127) / 128;
+  p.tiles_m = (int)((R + 255) / 256);
+  p.tiles_n = (int)((K + 255) / 256);
+  p.num_tiles = p.tiles_m * p.tiles_n;
+  p.status = status_word_ptr();
+  p.out = dV;
+  p.ldo = vcols;
+  p.out_f32 = dtype == NM_OUT_F32;
+  p.meta = meta;
+  p.n = n;
+  p.m = m;
+  p.vcols = vcols;
+  p.mcols = meta_cols(K, n, m);
+  p.meta_cblocks = meta_col_blocks(K);
+  if (e == cudaSuccess && !p.status) e = cudaErrorInvalidSymbol;
+  if ((int64_t)p.tiles_m * p.tiles_n >= (1ll << 31)) st = fail(NM_ERR_UNSUPPORTED, "too many tiles");
+  if (e == cudaSuccess && st == NM_OK)
+    st = make_tmap(&p.tm_a, dY, (uint64_t)T, (uint64_t)R, (uint64_t)lddy * 2, 64, 64, 128, "dY");
+  if (e == cudaSuccess && st == NM_OK)
+    st = make_tmap(&p.tm_b, xsrc, (uint64_t)T, (uint64_t)K, (uint64_t)ldsrc * 2, 64, 64, 128, "X");
+  if (e == cudaSuccess && st == NM_OK) e = launch_dense_pair(p, false, false, EPI_SURVIVORS, stream);
+  if (staged) cudaFreeAsync(staged, stream);
+  if (st != NM_OK) return st;
+  return e == cudaSuccess ? NM_OK : cuda_fail(e, "value-gradient GEMM launch");
+}
+
 }  // namespace nmk
 
 using namespace nmk;
@@ -875,6 +1010,18 @@ nm_status nm_prune_spmm(const uint16_t* W, int64_t ldw, int n, int m, int64_t R,
                         uint16_t* values, uint32_t* meta, void* stream) {
   return run_prune_gemm(W, ldw, n, m, R, K, idx, X, ldx, T, Y, ldy, y_dtype, values, meta,
                         static_cast<cudaStream_t>(stream));
+}
+
+nm_status nm_spmm_t(const uint16_t* values, const uint32_t* meta, int n, int m, int64_t R, int64_t K,
+                    const int32_t* idx, const uint16_t* dY, int64_t lddy, int64_t T, void* dX, int64_t lddx,
+                    nm_out_dtype dtype, void* stream) {
+  return run_spmm_t(values, meta, n, m, R, K, idx, dY, lddy, T, dX, lddx, dtype, static_cast<cudaStream_t>(stream));
+}
+
+nm_status nm_sddmm(const uint32_t* meta, int n, int m, int64_t R, int64_t K, const int32_t* idx, const uint16_t* dY,
+                   int64_t lddy, const uint16_t* X, int64_t ldx, int64_t T, void* dV, nm_out_dtype dtype,
+                   void* stream) {
+  return run_sddmm(meta, n, m, R, K, idx, dY, lddy, X, ldx, T, dV, dtype, static_cast<cudaStream_t>(stream));
 }
 
 nm_status nm_device_status(void* stream) {

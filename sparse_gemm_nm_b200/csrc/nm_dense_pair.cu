@@ -1,0 +1,304 @@
+// nm_dense_pair.cu -- dense bf16 GEMMs on SM pairs for the backward pass of an N:M layer.
+//
+// Training keeps the N:M structure of W' through every step ("Structured
+// Sparsity" topic cards, RNM-TD3 abstract; the DynaDiag page's abstract asks
+// for sparse forward and backward passes).  The forward product y = (W' Pi) x
+// runs on the sparse tensor cores because W' is N:M along its reduction axis K.
+// The two gradients are not of that form:
+//   dX = (W' Pi)^T dY  reduces over R, and W'^T is N:M along its output axis;
+//   dV = the survivor entries of dY Xp^T, a product sampled at the survivors.
+// The sparse MMA takes sparsity only on A along the reduction axis, so both
+// run here as dense MMAs: dX on the decompressed W' (A = W'^T read MN-major
+// from the R x K matrix), dV as the full product with only the survivor
+// entries stored.
+//
+// Layout per CTA of the pair (cta_group::2, M = 256 = 2 x 128 rows, N = 256):
+// three stages of 128 reduction steps, A 128 rows x 128 (32 KB) and B 128 x
+// this CTA's 128 columns (32 KB), each as four TMA boxes of 64 x 64 with the
+// 128-byte swizzle.  A K-major stage is [K half][128 rows][128 B]; an MN-major
+// stage is [64-wide M (or N) strip][128 reduction rows][128 B].  The leader's
+// MMA thread issues eight tcgen05.mma (K = 16) per stage; its commits release
+// the stage in both CTAs.  Each CTA drains its own 128 x 256 fp32 accumulator.
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include "nm_internal.h"
+#include "nm_ptx.cuh"
+#include "nm_spmm.h"
+
+namespace nmk {
+
+namespace dpair {
+constexpr int kThreads = 256;  // warp 0 copies, 1 MMA, 4-7 epilogue
+constexpr int kStages = 3;
+constexpr uint32_t kA = 32768, kB = 32768;
+constexpr uint32_t kTx = 2u * (kA + kB);  // both CTAs' bytes of a stage
+constexpr uint32_t kTmemCols = 256;
+constexpr uint32_t kRowPad = 33;          // epilogue row buffer: 32 floats + 1 (no bank conflicts)
+constexpr uint32_t kEpiBuf = 32 * kRowPad * 4;
+constexpr uint64_t kWaitNs = 2000000000ull;
+constexpr uint32_t kOffBuf = kStages * (kA + kB);
+constexpr uint32_t kOffBar = kOffBuf + 4 * kEpiBuf;
+constexpr uint32_t kSmemBytes = kOffBar + (2 * kStages + 3) * 8 + 16 + 1024;
+static_assert(kSmemBytes <= 227 * 1024, "shared memory");
+}  // namespace dpair
+
+// Column of survivor j of weight row r (stored position read from the
+// metadata): 2:4 tiled metadata or the row-wise packing of other patterns.
+__device__ __forceinline__ int64_t survivor_col(const DenseParams& p, int64_t r, int64_t j) {
+  const int64_t g = j / p.n;
+  if (p.n == 2 && p.m == 4) {
+    const int64_t k = 4 * g, c = k & 127;
+    const int64_t word = ((r >> 4) * p.meta_cblocks + (k >> 7)) * 64 + 4 * ((r & 7) + 8 * ((c >> 4) & 1)) + (c >> 5);
+    const uint32_t nib = (__ldg(p.meta + word) >> (16 * ((r >> 3) & 1) + 4 * ((c >> 2) & 3))) & 0xFu;
+    return k + ((j & 1) ? (nib >> 2) : (nib & 3u));
+  }
+  const int b = p.m == 2 ? 1 : p.m == 4 ? 2 : p.m == 8 ? 3 : 4;
+  const int S = 32 / b;
+  const uint32_t w = __ldg(p.meta + r * p.mcols + j / S);
+  return g * p.m + ((w >> (b * (int)(j % S))) & ((1u << b) - 1u));
+}
+
+template <bool A_MN, bool B_MN, int EPI>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dpair::kThreads, 1)
+    dense_pair_kernel(const __grid_constant__ DenseParams p) {
+  using namespace dpair;
+  constexpr uint32_t kIdesc = idesc_bf16_major(256, 256, A_MN, B_MN);
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kOffBar);
+  uint64_t* empty = full + kStages;
+  uint64_t* acc_full = empty + kStages;
+  uint64_t* acc_empty = acc_full + 1;
+  uint64_t* spare = acc_empty + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(spare + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const uint32_t rank = cluster_ctarank();  // 0: leader (issues the MMAs)
+  const int pair_id = blockIdx.x >> 1;
+  const int npairs = gridDim.x >> 1;
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    mbar_init(acc_full, 1);
+    mbar_init(acc_empty, 8);  // four epilogue warps in each CTA
+    mbar_init(spare, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+    fence_proxy_async_smem();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&p.tm_a);
+    tma_prefetch_desc(&p.tm_b);
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(tmem_slot, kTmemCols);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  pdl_gate();  // no global memory touched before this point
+
+  const uint32_t lead_full0 = map_to_cta(smem_u32(&full[0]), 0);
+  const uint32_t lead_acc_empty = map_to_cta(smem_u32(acc_empty), 0);
+  bool ok = true;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------- copies
+    if (lane == 0) {
+      int s = 0;
+      uint32_t ph = 0;
+      for (int tile = pair_id; tile < p.num_tiles && ok; tile += npairs) {
+        const int tm = tile % p.tiles_m, tn = tile / p.tiles_m;
+        const int32_t m0 = tm * 256 + 128 * (int)rank;  // this CTA's 128 rows of C
+        const int32_t n0 = tn * 256 + 128 * (int)rank;  // this CTA's 128 columns of B
+        for (int64_t kt = 0; kt < p.k_tiles; ++kt) {
+          ok = mbar_wait(&empty[s], ph ^ 1u, abort_flag, p.status, kWaitNs);
+          if (!ok) break;
+          const uint32_t bar = lead_full0 + 8u * s;
+          if (rank == 0) mbar_arrive_expect_tx(&full[s], kTx);
+          uint8_t* a = smem + s * (kA + kB);
+          uint8_t* b = a + kA;
+          const int32_t k0 = (int32_t)(kt * 128);
+#pragma unroll
+          for (int i = 0; i < 2; ++i) {
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+              // A: MN-major box (64 M columns at m0 + 64 i, reduction rows k0 + 64 h) or K-major box
+              // (reduction columns k0 + 64 i, rows m0 + 64 h); same smem slot either way.
+              if (A_MN)
+                tma_load_2d_pair(a + i * 16384 + h * 8192, &p.tm_a, bar, m0 + 64 * i, k0 + 64 * h);
+              else
+                tma_load_2d_pair(a + i * 16384 + h * 8192, &p.tm_a, bar, k0 + 64 * i, m0 + 64 * h);
+              if (B_MN)
+                tma_load_2d_pair(b + i * 16384 + h * 8192, &p.tm_b, bar, n0 + 64 * i, k0 + 64 * h);
+              else
+                tma_load_2d_pair(b + i * 16384 + h * 8192, &p.tm_b, bar, k0 + 64 * i, n0 + 64 * h);
+            }
+          }
+          if (++s == kStages) { s = 0; ph ^= 1u; }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------------------------------------------------- MMA (leader)
+    if (rank == 0 && lane == 0) {
+      int s = 0;
+      uint32_t ph = 0, aph = 0;
+      for (int tile = pair_id; tile < p.num_tiles && ok; tile += npairs) {
+        ok = mbar_wait(acc_empty, aph ^ 1u, abort_flag, p.status, kWaitNs);
+        if (!ok) break;
+        tc_fence_after();
+        for (int64_t kt = 0; kt < p.k_tiles; ++kt) {
+          ok = mbar_wait(&full[s], ph, abort_flag, p.status, kWaitNs);
+          if (!ok) break;
+          tc_fence_after();
+          const uint32_t a_addr = smem_u32(smem + s * (kA + kB));
+          const uint32_t b_addr = a_addr + kA;
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk) {
+            // K = 16 step kk: K-major operands advance 32 B inside a 64-wide half (halves 16 KB
+            // apart); MN-major operands advance 16 rows of 128 B (strips 16 KB apart).
+            const uint64_t ad = A_MN ? smem_desc(a_addr + kk * 2048, 16384, 1024, SWZ_128B)
+                                     : smem_desc(a_addr + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024, SWZ_128B);
+            const uint64_t bd = B_MN ? smem_desc(b_addr + kk * 2048, 16384, 1024, SWZ_128B)
+                                     : smem_desc(b_addr + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024, SWZ_128B);
+            tc_mma_pair(tmem_base, ad, bd, kIdesc, (kt > 0 || kk > 0) ? 1u : 0u);
+          }
+          tc_commit_pair(&empty[s], 0x3);
+          if (++s == kStages) { s = 0; ph ^= 1u; }
+        }
+        if (!ok) break;
+        tc_commit_pair(acc_full, 0x3);
+        aph ^= 1u;
+      }
+      if (!ok) {
+        tc_commit_pair(spare, 0x1);
+        volatile int dummy = 0;
+        mbar_wait(spare, 0, &dummy, p.status, 100000000ull);
+      }
+    }
+  } else if (warp >= 4) {
+    // ------------------------------------------------------------- epilogue
+    const int quarter = warp & 3;  // TMEM lanes 32*quarter .. +31
+    float* buf = reinterpret_cast<float*>(smem + kOffBuf + (warp - 4) * kEpiBuf) + lane * kRowPad;
+    uint32_t aph = 0;
+    for (int tile = pair_id; tile < p.num_tiles && ok; tile += npairs) {
+      const int tm = tile % p.tiles_m, tn = tile / p.tiles_m;
+      const int64_t row = (int64_t)tm * 256 + 128 * rank + quarter * 32 + lane;
+      const int64_t n0 = (int64_t)tn * 256;
+      ok = mbar_wait(acc_full, aph, abort_flag, p.status, kWaitNs);
+      if (!ok) break;
+      tc_fence_after();
+      const uint32_t t_addr = tmem_base + ((uint32_t)(quarter * 32) << 16);
+      bool row_ok = row < p.M;
+      int64_t orow = row;
+      if (EPI == EPI_STORE && row_ok && p.row_map) {
+        const int32_t v = __ldg(p.row_map + row);
+        row_ok = v >= 0 && (int64_t)v < p.rows_out;
+        orow = v;
+      }
+#pragma unroll 1
+      for (int c = 0; c < 8; ++c) {
+        uint32_t v[32];
+        tmem_ld_32x32b_x32(t_addr + c * 32, v);
+        tc_wait_ld();
+        const int64_t col0 = n0 + 32 * c;
+        if (!row_ok || col0 >= p.N) continue;
+        if (EPI == EPI_STORE) {
+          if (p.out_f32) {
+            float* y = static_cast<float*>(p.out) + orow * p.ldo + col0;
+            if (col0 + 32 <= p.N) {
+#pragma unroll
+              for (int q = 0; q < 8; ++q)
+                reinterpret_cast<float4*>(y)[q] = make_float4(__uint_as_float(v[4 * q]), __uint_as_float(v[4 * q + 1]),
+                                                              __uint_as_float(v[4 * q + 2]), __uint_as_float(v[4 * q + 3]));
+            } else {
+#pragma unroll
+              for (int e = 0; e < 32; ++e)
+                if (col0 + e < p.N) y[e] = __uint_as_float(v[e]);
+            }
+          } else {
+            uint16_t* y = static_cast<uint16_t*>(p.out) + orow * p.ldo + col0;
+            uint32_t pk[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) pk[i] = pack_bf16x2(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1]));
+            if (col0 + 32 <= p.N) {
+#pragma unroll
+              for (int q = 0; q < 4; ++q)
+                reinterpret_cast<uint4*>(y)[q] = make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
+            } else {
+#pragma unroll
+              for (int e = 0; e < 32; ++e)
+                if (col0 + e < p.N) y[e] = (uint16_t)(pk[e >> 1] >> (16 * (e & 1)));
+            }
+          }
+        } else {
+          // survivors of weight row `row` among columns col0 .. col0 + 31 (M divides 32)
+#pragma unroll
+          for (int e = 0; e < 32; ++e) buf[e] = __uint_as_float(v[e]);
+          const int64_t cend = col0 + 32 < p.N ? col0 + 32 : p.N;
+          const int64_t j0 = col0 / p.m * p.n, j1 = cend / p.m * p.n;
+          for (int64_t j = j0; j < j1; ++j) {
+            const float val = buf[survivor_col(p, row, j) - col0];
+            if (p.out_f32)
+              static_cast<float*>(p.out)[row * p.ldo + j] = val;
+            else
+              static_cast<uint16_t*>(p.out)[row * p.ldo + j] = (uint16_t)(pack_bf16x2(val, 0.0f) & 0xFFFFu);
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(lead_acc_empty);
+      aph ^= 1u;
+    }
+  }
+
+  // -------------------------------------------------------------- teardown
+  __syncthreads();
+  if (*abort_flag && threadIdx.x == 0) sleep_about_ns(200000ull);
+  cluster_sync();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc_pair(tmem_base, dpair::kTmemCols);
+  }
+}
+
+template <bool A_MN, bool B_MN, int EPI>
+static cudaError_t launch_dp(const DenseParams& p, cudaStream_t stream) {
+  static bool configured[64] = {};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev >= 0 && dev < 64 && !configured[dev]) {
+    cudaError_t e = cudaFuncSetAttribute(dense_pair_kernel<A_MN, B_MN, EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)dpair::kSmemBytes);
+    if (e != cudaSuccess) return e;
+    configured[dev] = true;
+  }
+  const int pairs_avail = sm_count_current() / 2;
+  const int pairs = p.num_tiles < pairs_avail ? p.num_tiles : pairs_avail;
+  cudaError_t e = launch_pdl(dense_pair_kernel<A_MN, B_MN, EPI>, dim3(2 * pairs), dim3(dpair::kThreads),
+                             (size_t)dpair::kSmemBytes, stream, p);
+  count_launch();
+  return e != cudaSuccess ? e : cudaGetLastError();
+}
+
+cudaError_t launch_dense_pair(const DenseParams& p, bool a_mn, bool b_mn, int epi, cudaStream_t stream) {
+  if (p.num_tiles <= 0) return cudaSuccess;
+  if (a_mn && b_mn && epi == EPI_STORE) return launch_dp<true, true, EPI_STORE>(p, stream);
+  if (!a_mn && !b_mn && epi == EPI_SURVIVORS) return launch_dp<false, false, EPI_SURVIVORS>(p, stream);
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace nmk

@@ -372,6 +372,13 @@ __host__ __device__ constexpr uint32_t idesc_bf16(uint32_t n, bool sparse, uint3
          ((m >> 4) << 24);
 }
 
+// Dense kind::f16 descriptor with the operand majors given: a_mn / b_mn set bits
+// 15 / 16 (the operand is MN-major: M or N is the contiguous axis).
+__host__ __device__ constexpr uint32_t idesc_bf16_major(uint32_t n, uint32_t m, bool a_mn, bool b_mn) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | (a_mn ? (1u << 15) : 0u) | (b_mn ? (1u << 16) : 0u) |
+         ((n >> 3) << 17) | ((m >> 4) << 24);
+}
+
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   uint32_t r;
   asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));

@@ -61,6 +61,30 @@ struct SpmmParams {
   uint32_t* out_meta;
 };
 
+// Dense bf16 GEMM on SM pairs for the backward products: C (M x N) = A (M x Kr) B (Kr x N),
+// fp32 accumulation.  A and B are read with TMA boxes of 64 x 64 (128-byte swizzle), K-major
+// (the reduction axis contiguous) or MN-major.  Epilogue 0 stores C, row m of C going to row
+// row_map[m] of `out` when row_map is set (rows mapped outside [0, rows_out) are dropped);
+// epilogue 1 stores only the entries at the survivor columns of an N:M pattern of an
+// M x N weight (meta), as out[m][j] for survivor j of row m.
+struct DenseParams {
+  CUtensorMap tm_a, tm_b;
+  int64_t M, N, Kr;
+  int64_t k_tiles;
+  int tiles_m, tiles_n, num_tiles;
+  uint32_t* status;
+  void* out;
+  int64_t ldo;
+  int out_f32;
+  const int32_t* row_map;
+  int64_t rows_out;
+  const uint32_t* meta;
+  int n, m;
+  int64_t vcols, mcols, meta_cblocks;
+};
+enum DenseEpi : int { EPI_STORE = 0, EPI_SURVIVORS = 1 };
+cudaError_t launch_dense_pair(const DenseParams& p, bool a_mn, bool b_mn, int epi, cudaStream_t stream);
+
 int spmm_max_stages(int bn, uint32_t a_slot);
 cudaError_t launch_spmm(SpmmParams& p, int bn, cudaStream_t stream);
 cudaError_t read_and_clear_status(uint32_t* out);
