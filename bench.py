@@ -462,6 +462,45 @@ def run_ours(args, rank: int, world: int, dist):
                           "plain_frac": max(b["flops"] / (tc_peak * 1e12), b["gemm_bytes"] / (hbm_peak * 1e9))
                           / (plain_ms[i] * 1e-3)} for i, b in enumerate(bufs)}
 
+    if not args.quick and not args.fused and all(b["tmap"] is None for b in bufs) and all(
+            b["L"].n == 2 and b["L"].m == 4 for b in bufs):
+        # backward products of each layer (training): dX = (W' Pi)^T dY and the value gradient dV,
+        # timed in event-free loops of the same calls; dense tensor-core FLOPs 2 R K T per call
+        reps = max(10, min(50, args.steps))
+        back = {}
+        for i, b in enumerate(bufs):
+            L = b["L"]
+            dY = up(wl.normal_bf16((L.R, L.T), 1.0, seed=100 + i))
+            dX = torch.empty((L.K, L.T), dtype=torch.bfloat16, device=dev)
+            dV = torch.empty((L.R, L.K // 2), dtype=torch.bfloat16, device=dev)
+            idx = b["idx"].data_ptr() if b["idx"] is not None else None
+            calls = {
+                "spmm_t": lambda: check(L_.nm_spmm_t(b["vals"].data_ptr(), b["meta"].data_ptr(), 2, 4, L.R, L.K, idx,
+                                                     dY.data_ptr(), L.T, L.T, dX.data_ptr(), L.T, 0, sp), "nm_spmm_t"),
+                "sddmm": lambda: check(L_.nm_sddmm(b["meta"].data_ptr(), 2, 4, L.R, L.K, idx, dY.data_ptr(), L.T,
+                                                   b["X"].data_ptr(), L.T, L.T, dV.data_ptr(), 0, sp), "nm_sddmm")}
+            res = {}
+            for name, fn in calls.items():
+                for _ in range(3):
+                    fn()
+                torch.cuda.synchronize()
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record(stream)
+                for _ in range(reps):
+                    fn()
+                e1.record(stream)
+                torch.cuda.synchronize()
+                us = e0.elapsed_time(e1) / reps * 1e3
+                tflops = 2.0 * L.R * L.K * L.T / (us * 1e-6) / 1e12
+                res[name] = {"us": us, "dense_tflops": tflops, "frac": tflops / tc_peak}
+            back[L.name] = res
+        nm.nm_device_status(sp)
+        line["backward"] = {"calls": back, "timing": f"event-free loops of {reps} calls per product",
+                            "roofline": "dense tcgen05 FLOPs 2*R*K*T per call against the same dense bf16 peak "
+                                        "as `roofline` (the useful, survivor-only FLOPs are half of these)",
+                            "spmm_t": "includes the decompression of W' into the staged dense operand",
+                            "permuted": any(b["idx"] is not None for b in bufs)}
+
     # end-to-end through the public API with host buffers
     if not args.quick and not args.no_e2e:
         hW = [torch.from_numpy(b["d"].W.view(np.int16)).pin_memory() for b in bufs]

@@ -869,6 +869,7 @@ static nm_status run_sddmm(const uint32_t* meta, int n, int m, int64_t R, int64_
   p.vcols = vcols;
   p.mcols = meta_cols(K, n, m);
   p.meta_cblocks = meta_col_blocks(K);
+  p.vec_out = n == 2 && m == 4 && K % 16 == 0 && al16(dV);
   if (e == cudaSuccess && !p.status) e = cudaErrorInvalidSymbol;
   if ((int64_t)p.tiles_m * p.tiles_n >= (1ll << 31)) st = fail(NM_ERR_UNSUPPORTED, "too many tiles");
   if (e == cudaSuccess && st == NM_OK)

@@ -18,7 +18,8 @@
 // 128-byte swizzle.  A K-major stage is [K half][128 rows][128 B]; an MN-major
 // stage is [64-wide M (or N) strip][128 reduction rows][128 B].  The leader's
 // MMA thread issues eight tcgen05.mma (K = 16) per stage; its commits release
-// the stage in both CTAs.  Each CTA drains its own 128 x 256 fp32 accumulator.
+// the stage in both CTAs.  Each CTA drains its own 128 x 256 fp32 accumulator;
+// two accumulators (512 TMEM columns) let the next tile's MMAs run meanwhile.
 #include <cstdint>
 #include <cuda.h>
 #include <cuda_runtime.h>
@@ -34,13 +35,13 @@ constexpr int kThreads = 256;  // warp 0 copies, 1 MMA, 4-7 epilogue
 constexpr int kStages = 3;
 constexpr uint32_t kA = 32768, kB = 32768;
 constexpr uint32_t kTx = 2u * (kA + kB);  // both CTAs' bytes of a stage
-constexpr uint32_t kTmemCols = 256;
+constexpr uint32_t kTmemCols = 512;  // two 256-column accumulators
 constexpr uint32_t kRowPad = 33;          // epilogue row buffer: 32 floats + 1 (no bank conflicts)
 constexpr uint32_t kEpiBuf = 32 * kRowPad * 4;
 constexpr uint64_t kWaitNs = 2000000000ull;
 constexpr uint32_t kOffBuf = kStages * (kA + kB);
 constexpr uint32_t kOffBar = kOffBuf + 4 * kEpiBuf;
-constexpr uint32_t kSmemBytes = kOffBar + (2 * kStages + 3) * 8 + 16 + 1024;
+constexpr uint32_t kSmemBytes = kOffBar + (2 * kStages + 5) * 8 + 16 + 1024;
 static_assert(kSmemBytes <= 227 * 1024, "shared memory");
 }  // namespace dpair
 
@@ -69,9 +70,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dpair::kThreads, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + kOffBar);
   uint64_t* empty = full + kStages;
-  uint64_t* acc_full = empty + kStages;
-  uint64_t* acc_empty = acc_full + 1;
-  uint64_t* spare = acc_empty + 1;
+  uint64_t* acc_full = empty + kStages;  // [2]
+  uint64_t* acc_empty = acc_full + 2;    // [2]
+  uint64_t* spare = acc_empty + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(spare + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -86,8 +87,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dpair::kThreads, 1)
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
-    mbar_init(acc_full, 1);
-    mbar_init(acc_empty, 8);  // four epilogue warps in each CTA
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&acc_full[a], 1);
+      mbar_init(&acc_empty[a], 8);  // four epilogue warps in each CTA
+    }
     mbar_init(spare, 1);
     *abort_flag = 0;
     fence_barrier_init();
@@ -109,7 +112,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dpair::kThreads, 1)
   pdl_gate();  // no global memory touched before this point
 
   const uint32_t lead_full0 = map_to_cta(smem_u32(&full[0]), 0);
-  const uint32_t lead_acc_empty = map_to_cta(smem_u32(acc_empty), 0);
+  const uint32_t lead_acc_empty0 = map_to_cta(smem_u32(acc_empty), 0);
   bool ok = true;
 
   if (warp == 0) {
@@ -153,11 +156,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dpair::kThreads, 1)
     // ---------------------------------------------------------- MMA (leader)
     if (rank == 0 && lane == 0) {
       int s = 0;
-      uint32_t ph = 0, aph = 0;
-      for (int tile = pair_id; tile < p.num_tiles && ok; tile += npairs) {
-        ok = mbar_wait(acc_empty, aph ^ 1u, abort_flag, p.status, kWaitNs);
+      uint32_t ph = 0;
+      int i = 0;  // tile counter: accumulator i % 2, its use i / 2
+      for (int tile = pair_id; tile < p.num_tiles && ok; tile += npairs, ++i) {
+        const int ab = i & 1;
+        ok = mbar_wait(&acc_empty[ab], ((uint32_t)(i >> 1) & 1u) ^ 1u, abort_flag, p.status, kWaitNs);
         if (!ok) break;
         tc_fence_after();
+        const uint32_t d_tmem = tmem_base + 256u * (uint32_t)ab;
         for (int64_t kt = 0; kt < p.k_tiles; ++kt) {
           ok = mbar_wait(&full[s], ph, abort_flag, p.status, kWaitNs);
           if (!ok) break;
@@ -172,14 +178,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dpair::kThreads, 1)
                                      : smem_desc(a_addr + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024, SWZ_128B);
             const uint64_t bd = B_MN ? smem_desc(b_addr + kk * 2048, 16384, 1024, SWZ_128B)
                                      : smem_desc(b_addr + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024, SWZ_128B);
-            tc_mma_pair(tmem_base, ad, bd, kIdesc, (kt > 0 || kk > 0) ? 1u : 0u);
+            tc_mma_pair(d_tmem, ad, bd, kIdesc, (kt > 0 || kk > 0) ? 1u : 0u);
           }
           tc_commit_pair(&empty[s], 0x3);
           if (++s == kStages) { s = 0; ph ^= 1u; }
         }
         if (!ok) break;
-        tc_commit_pair(acc_full, 0x3);
-        aph ^= 1u;
+        tc_commit_pair(&acc_full[ab], 0x3);
       }
       if (!ok) {
         tc_commit_pair(spare, 0x1);
@@ -191,15 +196,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dpair::kThreads, 1)
     // ------------------------------------------------------------- epilogue
     const int quarter = warp & 3;  // TMEM lanes 32*quarter .. +31
     float* buf = reinterpret_cast<float*>(smem + kOffBuf + (warp - 4) * kEpiBuf) + lane * kRowPad;
-    uint32_t aph = 0;
-    for (int tile = pair_id; tile < p.num_tiles && ok; tile += npairs) {
+    int i = 0;
+    for (int tile = pair_id; tile < p.num_tiles && ok; tile += npairs, ++i) {
+      const int ab = i & 1;
       const int tm = tile % p.tiles_m, tn = tile / p.tiles_m;
       const int64_t row = (int64_t)tm * 256 + 128 * rank + quarter * 32 + lane;
       const int64_t n0 = (int64_t)tn * 256;
-      ok = mbar_wait(acc_full, aph, abort_flag, p.status, kWaitNs);
+      ok = mbar_wait(&acc_full[ab], (uint32_t)(i >> 1) & 1u, abort_flag, p.status, kWaitNs);
       if (!ok) break;
       tc_fence_after();
-      const uint32_t t_addr = tmem_base + ((uint32_t)(quarter * 32) << 16);
+      const uint32_t t_addr = tmem_base + ((uint32_t)(quarter * 32) << 16) + 256u * (uint32_t)ab;
       bool row_ok = row < p.M;
       int64_t orow = row;
       if (EPI == EPI_STORE && row_ok && p.row_map) {
@@ -242,6 +248,35 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dpair::kThreads, 1)
                 if (col0 + e < p.N) y[e] = (uint16_t)(pk[e >> 1] >> (16 * (e & 1)));
             }
           }
+        } else if (p.vec_out && col0 + 32 <= p.N) {
+          // 2:4: the chunk's eight groups take their nibbles from two tiled metadata words (column
+          // halves h = 0, 1 of the chunk's 32-column quarter q); the sixteen survivors are picked from
+          // registers and stored as 32 (bf16) or 64 (fp32) contiguous bytes of the row.
+          const uint32_t* mb =
+              p.meta + ((row >> 4) * p.meta_cblocks + (col0 >> 7)) * 64 + 4 * (row & 7) + ((col0 >> 5) & 3);
+          const uint32_t wh[2] = {__ldg(mb), __ldg(mb + 32)};
+          const int sh = 16 * (int)((row >> 3) & 1);
+          float o[16];
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const uint32_t nib = (wh[i >> 2] >> (sh + 4 * (i & 3))) & 0xFu;
+            const uint32_t p0 = nib & 3u, p1 = nib >> 2;
+            const float a0 = __uint_as_float(v[4 * i]), a1 = __uint_as_float(v[4 * i + 1]);
+            const float a2 = __uint_as_float(v[4 * i + 2]), a3 = __uint_as_float(v[4 * i + 3]);
+            o[2 * i] = p0 == 0 ? a0 : (p0 == 1 ? a1 : a2);
+            o[2 * i + 1] = p1 == 3 ? a3 : (p1 == 2 ? a2 : a1);
+          }
+          if (p.out_f32) {
+            float4* y = reinterpret_cast<float4*>(static_cast<float*>(p.out) + row * p.ldo + (col0 >> 1));
+#pragma unroll
+            for (int q = 0; q < 4; ++q) y[q] = make_float4(o[4 * q], o[4 * q + 1], o[4 * q + 2], o[4 * q + 3]);
+          } else {
+            uint4* y = reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.out) + row * p.ldo + (col0 >> 1));
+            y[0] = make_uint4(pack_bf16x2(o[0], o[1]), pack_bf16x2(o[2], o[3]), pack_bf16x2(o[4], o[5]),
+                              pack_bf16x2(o[6], o[7]));
+            y[1] = make_uint4(pack_bf16x2(o[8], o[9]), pack_bf16x2(o[10], o[11]), pack_bf16x2(o[12], o[13]),
+                              pack_bf16x2(o[14], o[15]));
+          }
         } else {
           // survivors of weight row `row` among columns col0 .. col0 + 31 (M divides 32)
 #pragma unroll
@@ -259,8 +294,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dpair::kThreads, 1)
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive_cluster(lead_acc_empty);
-      aph ^= 1u;
+      if (lane == 0) mbar_arrive_cluster(lead_acc_empty0 + 8u * (uint32_t)ab);
     }
   }
 

@@ -81,6 +81,7 @@ struct DenseParams {
   const uint32_t* meta;
   int n, m;
   int64_t vcols, mcols, meta_cblocks;
+  int vec_out;  // epilogue 1, 2:4: K % 16 == 0 and `out` 16-byte aligned (vector stores of whole chunks)
 };
 enum DenseEpi : int { EPI_STORE = 0, EPI_SURVIVORS = 1 };
 cudaError_t launch_dense_pair(const DenseParams& p, bool a_mn, bool b_mn, int epi, cudaStream_t stream);
