@@ -54,9 +54,10 @@ def parse_args(argv=None):
     ap.add_argument("--algo", choices=["auto", "sparse", "dense"], default="auto",
                     help="kernel design for 1:4 / 1:8 (nm_spmm_algo)")
     ap.add_argument("--plain", action="store_true", help="ignore the workload's index map (y = W x)")
-    ap.add_argument("--fused", action="store_true",
-                    help="one nm_prune_spmm call per layer (prune + compress + GEMM, same outputs) instead of "
-                         "nm_prune_compress followed by the GEMM call")
+    ap.add_argument("--step", choices=["one-call", "two-calls"], default="one-call",
+                    help="one-call: nm_prune_spmm per layer (prune + compress + GEMM in one library call, the "
+                         "compressed form written too); two-calls: nm_prune_compress, then the GEMM call.  The "
+                         "hybrid workloads and --algo other than auto always use two calls")
     ap.add_argument("--quick", action="store_true",
                     help="timed region only: no clock sampling, end-to-end pass, oracle baseline or extras")
     return ap.parse_args(argv)
@@ -251,8 +252,7 @@ def run_ours(args, rank: int, world: int, dist):
     def up(bits):
         return torch.from_numpy(bits.view(np.int16)).to(dev).view(torch.bfloat16)
 
-    if args.fused and any(d.tmap is not None for d in data):
-        raise SystemExit("--fused covers the n:m pruned GEMM, not the hybrid workloads")
+    one_call = args.step == "one-call" and all(d.tmap is None for d in data) and args.algo == "auto"
     bufs = []
     for d in data:
         L = d.layer
@@ -263,8 +263,24 @@ def run_ours(args, rank: int, world: int, dist):
              "meta": torch.empty((max(nm.nm_meta_words(L.R, L.K, L.n, L.m), 0),), dtype=torch.int32, device=dev),
              "Y": torch.empty((L.R, L.T), dtype=torch.bfloat16, device=dev)}
         b["flops"] = float(wl.hybrid_useful_flops(d) if d.tmap is not None else L.useful_flops)
-        b["gemm_bytes"] = gemm_bytes(L, d) + (2.0 * L.R * L.K if args.fused else 0.0)  # fused: W read once
         b["comp_bytes"] = 2.0 * L.R * L.K + 2.0 * b["vals"].numel() + 4.0 * b["meta"].numel()
+        # How nm_prune_spmm runs the layer (mirrors the library's dispatch), and what the kernel-timing
+        # pass brackets with events: "fused" the whole call (prune_spmm_skinny_kernel + reduction);
+        # "combined" the pair GEMM on the gathered input, the same launch the call makes after its
+        # compress-and-gather grid; "split" the GEMM call after a separate compress.
+        b["mode"] = "split"
+        if one_call and L.n == 2 and L.m == 4 and L.K % 128 == 0:
+            if 1 <= L.T <= 64:
+                b["mode"] = "fused"
+            elif b["idx"] is not None and L.T >= 192 and L.T % 8 == 0:
+                b["mode"] = "combined"
+                b["Xp"] = b["X"][b["idx"].long()].contiguous()  # input of the timed GEMM launch (setup only)
+        if b["mode"] == "fused":  # W read once, compressed form written, X read, Y written
+            b["gemm_bytes"] = b["comp_bytes"] + 2.0 * L.K * L.T + 2.0 * L.R * L.T
+        elif b["mode"] == "combined":  # the GEMM reads the gathered input: no index map
+            b["gemm_bytes"] = gemm_bytes(L, d) - 4.0 * L.K
+        else:
+            b["gemm_bytes"] = gemm_bytes(L, d)
         bufs.append(b)
     torch.cuda.synchronize()
 
@@ -301,19 +317,35 @@ def run_ours(args, rank: int, world: int, dist):
                                b["Y"].data_ptr(), L.T, 0, b["vals"].data_ptr(), b["meta"].data_ptr(), sp),
               "nm_prune_spmm")
 
-    def step(evs=None, permuted=True):
+    def launch_gemm_xp(b):
+        L = b["L"]
+        check(L_.nm_spmm(b["vals"].data_ptr(), b["meta"].data_ptr(), 2, 4, L.R, L.K, b["Xp"].data_ptr(), L.T, L.T,
+                         b["Y"].data_ptr(), L.T, 0, sp), "nm_spmm")
+
+    def launch_layer(b):  # one layer of the timed step
+        if one_call:
+            launch_fused(b)
+        else:
+            launch_compress(b)
+            launch_gemm(b)
+
+    def step(evs=None):
+        """The step; with events, the kernel-timing form of it (see b["mode"])."""
         for i, b in enumerate(bufs):
-            if evs is not None:
-                evs[2 * i].record(stream)
-            if args.fused:  # the whole call is timed as the GEMM; the compress slot stays empty
-                if evs is not None:
-                    evs[2 * i + 1].record(stream)
-                launch_fused(b, permuted)
+            if evs is None:
+                launch_layer(b)
+                continue
+            evs[2 * i].record(stream)
+            if b["mode"] == "fused":  # the whole call; the compress slot stays empty
+                evs[2 * i + 1].record(stream)
+                launch_fused(b)
                 continue
             launch_compress(b)
-            if evs is not None:
-                evs[2 * i + 1].record(stream)
-            launch_gemm(b, permuted)
+            evs[2 * i + 1].record(stream)
+            if b["mode"] == "combined":
+                launch_gemm_xp(b)
+            else:
+                launch_gemm(b)
         if evs is not None:
             evs[2 * len(bufs)].record(stream)
 
@@ -391,8 +423,10 @@ def run_ours(args, rank: int, world: int, dist):
             "gemm_gbs": b["gemm_bytes"] / (gemm_ms[i] * 1e-3) / 1e9,
             "gemm_bound": "tensor" if t_tc >= t_hbm else "hbm",
             "gemm_frac": max(t_tc, t_hbm) / (gemm_ms[i] * 1e-3),
-            "compress_us": 1e3 * comp_ms[i]}
-        if not args.fused:
+            "compress_us": 1e3 * comp_ms[i], "timed": {
+                "fused": "the nm_prune_spmm call", "combined": "spmm_pair_kernel on the gathered input",
+                "split": "the GEMM call"}[b["mode"]]}
+        if b["mode"] != "fused":
             kernels[L.name]["compress_gbs"] = b["comp_bytes"] / (comp_ms[i] * 1e-3) / 1e9
             kernels[L.name]["compress_frac"] = kernels[L.name]["compress_gbs"] / hbm_peak
 
@@ -405,12 +439,14 @@ def run_ours(args, rank: int, world: int, dist):
     # (profiles/<workload>_gemm_traffic.json); summed over the step like `achieved`.
     traffic = None
     tfile = os.path.join(ROOT, "profiles", f"{args.workload}_gemm_traffic.json")
-    if os.path.exists(tfile) and args.algo == "auto" and not args.fused:
+    if os.path.exists(tfile) and args.algo == "auto" and all(b["mode"] != "fused" for b in bufs):
         with open(tfile) as f:
             per = json.load(f).get("bytes_per_launch", {})
         names = [f"{b['L'].R}x{b['L'].K}" for b in bufs]
-        if all(n in per for n in names):
-            traffic = sum(sum(per[n].get(k, 0) for k in ("spmm_pair_kernel", "gather_rows_kernel")) for n in names)
+        kinds = [("spmm_pair_kernel",) if b["mode"] == "combined" else ("spmm_pair_kernel", "gather_rows_kernel")
+                 for b in bufs]
+        if all(n in per and all(k in per[n] for k in ks) for n, ks in zip(names, kinds)):
+            traffic = sum(sum(per[n][k] for k in ks) for n, ks in zip(names, kinds))
     if tensor_bound:
         achieved, peak, unit = flops_all / gsec / 1e12, tc_peak, "TFLOP/s"
         src = (f"{peak_src} bf16 {'sustained' if sustained else 'burst'} dense peak; useful 2:4 FLOPs run at "
@@ -420,17 +456,24 @@ def run_ours(args, rank: int, world: int, dist):
         src = f"{peak_src} HBM copy bandwidth"
     roofline = {"bound": "tensor" if tensor_bound else "hbm", "achieved": achieved, "peak": peak, "unit": unit,
                 "frac": achieved / peak, "traffic": traffic,
-                "kernel": ("nm_prune_spmm call: prune_spmm_skinny_kernel (+ gather, split-K reduction)" if args.fused
-                           else "nm_spmm_permuted call: gather_rows_kernel + spmm_pair_kernel (tcgen05 2-SM GEMM)"),
+                "kernel": ("nm_prune_spmm call: prune_spmm_skinny_kernel + split-K reduction"
+                           if all(b["mode"] == "fused" for b in bufs) else
+                           "spmm_pair_kernel (tcgen05 2-SM GEMM) on the gathered input, as launched by nm_prune_spmm"
+                           if all(b["mode"] == "combined" for b in bufs) else
+                           "the GEMM call (nm_spmm_permuted: gather_rows_kernel + spmm_pair_kernel, or nm_spmm / "
+                           "nm_hybrid_spmm)"),
                 "peak_source": src,
                 "algorithmic_per_launch": [b["flops"] if tensor_bound else b["gemm_bytes"] for b in bufs]}
 
     cfg = {"workload": args.workload, "shapes": [[b["L"].R, b["L"].K] for b in bufs],
            "T": [b["L"].T for b in bufs], "pattern": [f"{b['L'].n}:{b['L'].m}" for b in bufs],
            "permuted": any(b["idx"] is not None for b in bufs), "algo": args.algo,
-           "step": ("one fused prune+compress+GEMM call (nm_prune_spmm) per layer" if args.fused
-                    else "prune+compress, then the sparse GEMM, for every layer"),
-           "kernel_timing": "per-kernel CUDA events in a second timed pass of the same K steps",
+           "step": ("one nm_prune_spmm call per layer: prune + compress (the compressed form written) + the sparse "
+                    "GEMM" if one_call else "nm_prune_compress, then the sparse GEMM call, for every layer"),
+           "layer_paths": {b["L"].name: b["mode"] for b in bufs},
+           "kernel_timing": ("CUDA events in a second pass of K steps: per layer the compress and the GEMM launch "
+                             "(\"combined\": the pair GEMM on the gathered input, the launch nm_prune_spmm makes "
+                             "after its compress-and-gather grid; \"fused\": the whole call)"),
            "l2": "inputs larger than L2 (126 MB) per step" if sum(
                b["W"].numel() * 2 + b["X"].numel() * 2 + b["Y"].numel() * 2 for b in bufs) > 126e6
            else "working set below L2 size (small config)",
@@ -442,27 +485,34 @@ def run_ours(args, rank: int, world: int, dist):
             "config": cfg, "roofline": roofline, "kernels": kernels, "gpu_launches": launches,
             "clocks": sampler.summary() if sampler else None}
 
-    if not args.quick and any(b["idx"] is not None for b in bufs):
-        # cost of the index-map read: the same steps with the plain GEMM (nm_spmm), timed the same way
+    if not args.quick and any(b["idx"] is not None for b in bufs) and all(b["tmap"] is None for b in bufs):
+        # cost of the index-map read: per layer the GEMM call with the map (nm_spmm_permuted: gather pass +
+        # GEMM) and without it (nm_spmm), each in an event-bracketed loop on the compressed operand
         reps = max(10, min(200, args.steps))
-        for _ in range(3):
-            step(permuted=False)
-        pevs = [[torch.cuda.Event(enable_timing=True) for _ in range(nev)] for _ in range(reps)]
-        torch.cuda.synchronize()
-        for k in range(reps):
-            step(pevs[k], permuted=False)
-        torch.cuda.synchronize()
-        plain_ms = [sum(pevs[k][2 * i + 1].elapsed_time(pevs[k][2 * i + 2]) for k in range(reps)) / reps
-                    for i in range(len(bufs))]
-        # plain_frac: the plain GEMM (nm_spmm) against the same roofline as `roofline`
-        line["permutation_overhead"] = {
-            b["L"].name: {"plain_us": 1e3 * plain_ms[i], "permuted_us": 1e3 * gemm_ms[i],
-                          "overhead": gemm_ms[i] / plain_ms[i] - 1.0,
-                          "plain_tflops": b["flops"] / (plain_ms[i] * 1e-3) / 1e12,
-                          "plain_frac": max(b["flops"] / (tc_peak * 1e12), b["gemm_bytes"] / (hbm_peak * 1e9))
-                          / (plain_ms[i] * 1e-3)} for i, b in enumerate(bufs)}
+        over = {}
+        for b in bufs:
+            L = b["L"]
+            res = {}
+            for name, permuted in (("permuted", True), ("plain", False)):
+                for _ in range(3):
+                    launch_gemm(b, permuted)
+                torch.cuda.synchronize()
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record(stream)
+                for _ in range(reps):
+                    launch_gemm(b, permuted)
+                e1.record(stream)
+                torch.cuda.synchronize()
+                res[name] = e0.elapsed_time(e1) / reps
+            t_bound = max(b["flops"] / (tc_peak * 1e12), gemm_bytes(L, b["d"]) / (hbm_peak * 1e9))
+            over[L.name] = {"plain_us": 1e3 * res["plain"], "permuted_us": 1e3 * res["permuted"],
+                            "overhead": res["permuted"] / res["plain"] - 1.0,
+                            "plain_tflops": b["flops"] / (res["plain"] * 1e-3) / 1e12,
+                            "plain_frac": t_bound / (res["plain"] * 1e-3)}
+        nm.nm_device_status(sp)
+        line["permutation_overhead"] = over
 
-    if not args.quick and not args.fused and all(b["tmap"] is None for b in bufs) and all(
+    if not args.quick and all(b["tmap"] is None for b in bufs) and all(
             b["L"].n == 2 and b["L"].m == 4 for b in bufs):
         # backward products of each layer (training): dX = (W' Pi)^T dY and the value gradient dV,
         # timed in event-free loops of the same calls; dense tensor-core FLOPs 2 R K T per call
@@ -533,11 +583,7 @@ def run_ours(args, rank: int, world: int, dist):
                 stream.wait_event(copied[i])
                 if started[i]:
                     stream.wait_event(returned[i])  # Y of the previous step has been read back
-                if args.fused:
-                    launch_fused(b)
-                else:
-                    launch_compress(b)
-                    launch_gemm(b)
+                launch_layer(b)
                 computed[i].record(stream)
                 with torch.cuda.stream(s_d2h):
                     s_d2h.wait_event(computed[i])

@@ -654,8 +654,43 @@ static nm_status run_prune_gemm(const uint16_t* W, int64_t ldw, int n, int m, in
       v = static_cast<uint16_t*>(staged);
       mt = reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(staged) + vbytes);
     }
-    nm_status st = nm_prune_compress(W, R, K, ldw, n, m, v, mt, stream);
-    if (st == NM_OK) st = nm_spmm_algo(v, mt, n, m, R, K, idx, X, ldx, T, Y, ldy, y_dtype, NM_ALGO_AUTO, stream);
+    // 2:4 on SM-pair shapes with an index map: the compress grid also gathers
+    // Xp[k] = X[idx[k]] (its selection is integer-bound and leaves HBM
+    // bandwidth over), then the GEMM reads Xp like an unpermuted input.
+    const bool combined = idx && X && n == 2 && m == 4 && K % 128 == 0 && T >= 192 && T % 8 == 0 &&
+                          ldw % 8 == 0 && al16(W) && al16(v) && al16(mt) && al16(X) && ldx % 8 == 0 && ldx >= T &&
+                          R < (1ll << 31) && K < (1ll << 31);
+    nm_status st = NM_OK;
+    if (combined) {
+      st = require_device();
+      void* xp = nullptr;
+      cudaError_t e = cudaSuccess;
+      if (st == NM_OK) {
+        cudaMemPool_t pool = nullptr;
+        e = staging_pool(&pool);
+        if (e == cudaSuccess) e = cudaMallocFromPoolAsync(&xp, (size_t)(K * T * 2), pool, stream);
+        if (e != cudaSuccess) {
+          xp = nullptr;
+          st = cuda_fail(e, "staging buffer for the permuted input");
+        }
+      }
+      CUtensorMap tm;
+      if (st == NM_OK) st = make_tmap(&tm, W, (uint64_t)K, (uint64_t)R, (uint64_t)ldw * 2, 128, 16, 0, "W");
+      uint32_t* status = status_word_ptr();
+      if (st == NM_OK && !status) st = fail(NM_ERR_CUDA, "device status word is unavailable");
+      if (st == NM_OK) {
+        const GatherJob g{X, ldx, idx, K, T, static_cast<uint16_t*>(xp), T};
+        e = launch_compress_stream(tm, R, K, v, mt, status, stream, &g);
+        if (e != cudaSuccess) st = cuda_fail(e, "compress + gather launch");
+      }
+      if (st == NM_OK)
+        st = nm_spmm_algo(v, mt, 2, 4, R, K, nullptr, static_cast<const uint16_t*>(xp), T, T, Y, ldy, y_dtype,
+                          NM_ALGO_AUTO, stream);
+      if (xp) cudaFreeAsync(xp, stream);
+    } else {
+      st = nm_prune_compress(W, R, K, ldw, n, m, v, mt, stream);
+      if (st == NM_OK) st = nm_spmm_algo(v, mt, n, m, R, K, idx, X, ldx, T, Y, ldy, y_dtype, NM_ALGO_AUTO, stream);
+    }
     if (staged) cudaFreeAsync(staged, stream);
     return st;
   }

@@ -270,41 +270,11 @@ __global__ void fill_zero_kernel(uint8_t* Y, int64_t R, int64_t row_bytes, int64
 constexpr int kGatherCtasPerSm = 4;
 constexpr size_t kGatherSmemCap = 56 * 1024;
 
-__global__ void __launch_bounds__(256) gather_rows_kernel(const uint16_t* __restrict__ X, int64_t ldx,
-                                                          const int32_t* __restrict__ idx, int64_t K, int64_t T,
-                                                          uint16_t* __restrict__ Xp, int64_t ldp) {
+__global__ void __launch_bounds__(256) gather_rows_kernel(const GatherJob g) {
   pdl_gate();
-  const int lane = threadIdx.x & 31;
   const int64_t warp = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) >> 5;
   const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
-  const int64_t whole = T >> 3;                     // 16-byte pieces inside the row's T columns
-  const int64_t pieces = (T + 7) >> 3;              // + a partial last piece when T % 8 != 0
-  const int64_t chunks = (pieces + 255) / 256;      // 4 KB chunks per row
-  const int64_t items = K * chunks;
-  for (int64_t it = warp; it < items; it += nwarps) {
-    const int64_t k = it / chunks, c0 = (it - k * chunks) * 256;
-    const int32_t src = __ldg(idx + k);
-    const bool valid = src >= 0 && (int64_t)src < K;
-    const uint16_t* row = X + (valid ? (int64_t)src : 0) * ldx;
-    const uint4* in = reinterpret_cast<const uint4*>(row);
-    uint4* out = reinterpret_cast<uint4*>(Xp + k * ldp);
-    uint4 v[8];
-#pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      const int64_t c = c0 + u * 32 + lane;
-      v[u] = (valid && c < whole) ? __ldg(in + c) : make_uint4(0, 0, 0, 0);
-      if (valid && c == whole && c < pieces) {  // columns 8c .. T-1 one by one, zeros after them
-        uint32_t w[4] = {0, 0, 0, 0};
-        for (int64_t j = 0; 8 * c + j < T; ++j) w[j >> 1] |= (uint32_t)__ldg(row + 8 * c + j) << (16 * (j & 1));
-        v[u] = make_uint4(w[0], w[1], w[2], w[3]);
-      }
-    }
-#pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      const int64_t c = c0 + u * 32 + lane;
-      if (c < pieces) out[c] = v[u];
-    }
-  }
+  gather_rows_items(g, warp, nwarps, threadIdx.x & 31);
 }
 
 // Re-encoding of an N:M operand whose survivors never exceed two per aligned
@@ -449,7 +419,8 @@ cudaError_t launch_gather_rows(const uint16_t* X, int64_t ldx, const int32_t* id
   const int64_t want = (items + 7) / 8;  // 8 warps per CTA
   const int64_t cap = (int64_t)sm_count_current() * kGatherCtasPerSm;
   const int grid = (int)(want < cap ? (want > 0 ? want : 1) : cap);
-  cudaError_t e = launch_pdl(gather_rows_kernel, grid, threads, kGatherSmemCap, s, X, ldx, idx, K, T, Xp, ldp);
+  const GatherJob g{X, ldx, idx, K, T, Xp, ldp};
+  cudaError_t e = launch_pdl(gather_rows_kernel, grid, threads, kGatherSmemCap, s, g);
   count_launch();
   return e != cudaSuccess ? e : cudaGetLastError();
 }

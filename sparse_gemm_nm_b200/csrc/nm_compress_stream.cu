@@ -9,7 +9,8 @@
 // ring, and eight consumer warps select from shared memory and store values and
 // metadata while the next blocks are in flight.  Blocks past R or K arrive
 // zero-filled, which selects positions (0, 1): exactly the padding nibble 0x4;
-// values are stored only inside R x K.
+// values are stored only inside R x K.  Optionally the same grid also gathers
+// the permuted rows of a GEMM input (see kGatherWarps).
 #include <cstdint>
 #include <cuda.h>
 #include <cuda_runtime.h>
@@ -23,6 +24,11 @@ namespace nmk {
 namespace cstream {
 constexpr int kConsumers = 8;
 constexpr int kThreads = 32 * (kConsumers + 1);  // warps 0..7 consume, warp 8 produces
+// With a gather job the CTA also runs kGatherWarps warps (9 ..) that copy the
+// permuted rows of an input X: integer-bound selection leaves HBM bandwidth
+// to spare, which the copy uses.
+constexpr int kGatherWarps = 4;
+constexpr int kThreadsGather = kThreads + 32 * kGatherWarps;
 constexpr int kSlots = 16;
 constexpr uint32_t kBlockBytes = 16 * 128 * 2;
 constexpr uint64_t kWaitNs = 2000000000ull;
@@ -35,10 +41,11 @@ constexpr size_t kSmem = 100 * 1024;
 static_assert(kSlots * kBlockBytes + 2 * kSlots * 8 + 64 + 1024 <= kSmem, "ring does not fit");
 }  // namespace cstream
 
-__global__ void __launch_bounds__(cstream::kThreads, 2)
+template <bool GATHER>
+__global__ void __launch_bounds__(GATHER ? cstream::kThreadsGather : cstream::kThreads, 2)
     compress_2of4_stream_kernel(const __grid_constant__ CUtensorMap tm_w, uint32_t R, uint32_t K,
                                 uint16_t* __restrict__ V, uint32_t* __restrict__ meta, uint32_t cblocks,
-                                uint32_t nblocks, uint32_t* status) {
+                                uint32_t nblocks, uint32_t* status, const __grid_constant__ GatherJob gj) {
   using namespace cstream;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* ring = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -60,6 +67,11 @@ __global__ void __launch_bounds__(cstream::kThreads, 2)
 
   // this CTA's blocks: blockIdx.x + j * gridDim.x, j = 0, 1, ...; slot j % kSlots; consumer j % kConsumers
   const uint32_t nmine = blockIdx.x < nblocks ? (nblocks - 1 - blockIdx.x) / gridDim.x + 1 : 0;
+  if (GATHER && warp > kConsumers) {
+    gather_rows_items(gj, (int64_t)blockIdx.x * kGatherWarps + (warp - kConsumers - 1),
+                      (int64_t)gridDim.x * kGatherWarps, lane);
+    return;
+  }
   if (warp == kConsumers) {
     if (lane == 0) {
       for (uint32_t j = 0; j < nmine; ++j) {
@@ -117,22 +129,31 @@ __global__ void __launch_bounds__(cstream::kThreads, 2)
 }
 
 cudaError_t launch_compress_stream(const CUtensorMap& tm_w, int64_t R, int64_t K, uint16_t* values, uint32_t* meta,
-                                   uint32_t* status, cudaStream_t s) {
+                                   uint32_t* status, cudaStream_t s, const GatherJob* gather) {
   using namespace cstream;
-  static bool configured[64] = {};
+  static bool configured[2][64] = {};
   int dev = 0;
   cudaGetDevice(&dev);
-  if (dev >= 0 && dev < 64 && !configured[dev]) {
-    cudaError_t e =
-        cudaFuncSetAttribute(compress_2of4_stream_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmem);
+  const int gi = gather ? 1 : 0;
+  if (dev >= 0 && dev < 64 && !configured[gi][dev]) {
+    cudaError_t e = gather ? cudaFuncSetAttribute(compress_2of4_stream_kernel<true>,
+                                                  cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmem)
+                           : cudaFuncSetAttribute(compress_2of4_stream_kernel<false>,
+                                                  cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmem);
     if (e != cudaSuccess) return e;
-    configured[dev] = true;
+    configured[gi][dev] = true;
   }
   const int64_t nblocks = meta_row_blocks(R) * meta_col_blocks(K);
   const int64_t cap = (int64_t)sm_count_current() * 2;
-  const int grid = (int)(nblocks < cap ? nblocks : cap);
-  cudaError_t e = launch_pdl(compress_2of4_stream_kernel, dim3(grid), dim3(kThreads), kSmem, s, tm_w, (uint32_t)R,
-                             (uint32_t)K, values, meta, (uint32_t)meta_col_blocks(K), (uint32_t)nblocks, status);
+  // with a gather job every CTA of the persistent grid also copies rows
+  const int grid = gather ? (int)cap : (int)(nblocks < cap ? nblocks : cap);
+  const GatherJob none{};
+  cudaError_t e =
+      gather ? launch_pdl(compress_2of4_stream_kernel<true>, dim3(grid), dim3(kThreadsGather), kSmem, s, tm_w,
+                          (uint32_t)R, (uint32_t)K, values, meta, (uint32_t)meta_col_blocks(K), (uint32_t)nblocks,
+                          status, *gather)
+             : launch_pdl(compress_2of4_stream_kernel<false>, dim3(grid), dim3(kThreads), kSmem, s, tm_w, (uint32_t)R,
+                          (uint32_t)K, values, meta, (uint32_t)meta_col_blocks(K), (uint32_t)nblocks, status, none);
   count_launch();
   return e != cudaSuccess ? e : cudaGetLastError();
 }

@@ -35,10 +35,55 @@ inline bool fits_2of4(int n, int m) { return (m == 2 && n == 1) || ((m == 4 || m
 // touching no global memory before, then lets its own successor be scheduled.
 // Stream order is unchanged; the successor's launch and setup overlap the tail
 // of the kernel before it.
+// Gather of permuted input rows, Xp[k] = X[idx[k]] (K x T bf16; an entry of idx
+// outside [0, K) gives a zero row).  Work items are (row, 4 KB chunk).
+struct GatherJob {
+  const uint16_t* X;
+  int64_t ldx;
+  const int32_t* idx;
+  int64_t K, T;
+  uint16_t* Xp;
+  int64_t ldp;
+};
+
 #ifdef __CUDACC__
 __device__ __forceinline__ void pdl_gate() {
   asm volatile("griddepcontrol.wait;" ::: "memory");
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// Items warp, warp + nwarps, ... of a gather: each lane moves 16-byte pieces of
+// one row; when T % 8 != 0 the partial last piece is read element by element,
+// so the reads stay inside the row's T columns.
+__device__ __forceinline__ void gather_rows_items(const GatherJob& g, int64_t warp, int64_t nwarps, int lane) {
+  const int64_t whole = g.T >> 3;         // 16-byte pieces inside the row's T columns
+  const int64_t pieces = (g.T + 7) >> 3;  // + a partial last piece when T % 8 != 0
+  const int64_t chunks = (pieces + 255) / 256;
+  const int64_t items = g.K * chunks;
+  for (int64_t it = warp; it < items; it += nwarps) {
+    const int64_t k = it / chunks, c0 = (it - k * chunks) * 256;
+    const int32_t src = __ldg(g.idx + k);
+    const bool valid = src >= 0 && (int64_t)src < g.K;
+    const uint16_t* row = g.X + (valid ? (int64_t)src : 0) * g.ldx;
+    const uint4* in = reinterpret_cast<const uint4*>(row);
+    uint4* out = reinterpret_cast<uint4*>(g.Xp + k * g.ldp);
+    uint4 v[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int64_t c = c0 + u * 32 + lane;
+      v[u] = (valid && c < whole) ? __ldg(in + c) : make_uint4(0, 0, 0, 0);
+      if (valid && c == whole && c < pieces) {  // columns 8c .. T-1 one by one, zeros after them
+        uint32_t w[4] = {0, 0, 0, 0};
+        for (int64_t j = 0; 8 * c + j < g.T; ++j) w[j >> 1] |= (uint32_t)__ldg(row + 8 * c + j) << (16 * (j & 1));
+        v[u] = make_uint4(w[0], w[1], w[2], w[3]);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int64_t c = c0 + u * 32 + lane;
+      if (c < pieces) out[c] = v[u];
+    }
+  }
 }
 #endif
 

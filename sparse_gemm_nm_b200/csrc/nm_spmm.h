@@ -4,6 +4,8 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include "nm_internal.h"
+
 namespace nmk {
 
 enum AMode : int {
@@ -101,6 +103,6 @@ cudaError_t launch_spmm_skinny(SpmmParams& p, cudaStream_t stream);
 cudaError_t launch_skinny_reduce(const SpmmParams& p, cudaStream_t stream);
 cudaError_t launch_prune_spmm_skinny(SpmmParams& p, cudaStream_t stream);
 cudaError_t launch_compress_stream(const CUtensorMap& tm_w, int64_t R, int64_t K, uint16_t* values, uint32_t* meta,
-                                   uint32_t* status, cudaStream_t s);
+                                   uint32_t* status, cudaStream_t s, const GatherJob* gather = nullptr);
 
 }  // namespace nmk

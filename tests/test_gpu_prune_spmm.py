@@ -146,7 +146,8 @@ def test_decode_full_size_sampled():
 # compress-then-GEMM route of the same call
 # ----------------------------------------------------------------------------
 @pytest.mark.parametrize("n,m,R,K,T", [(2, 4, 200, 1024, 100), (2, 4, 130, 96, 16), (1, 4, 300, 1024, 16),
-                                       (1, 8, 256, 512, 264), (3, 4, 70, 256, 24)])
+                                       (1, 8, 256, 512, 264), (3, 4, 70, 256, 24), (2, 4, 300, 1024, 264),
+                                       (2, 4, 600, 384, 520)])
 @pytest.mark.parametrize("keep", [False, True])
 def test_unfused_routes(n, m, R, K, T, keep):
     W = wl.normal_bf16((R, K), 0.02, seed=R + K + T + n + m)
@@ -211,3 +212,25 @@ def test_graph_capture_replays_permuted_calls():
         assert torch.equal(v, vals) and torch.equal(mt, meta)
     ref, mag, _, _ = reference(W, X, 2, 4, idx)
     assert_gemm_close(values_f64(Y1), ref, mag, "graph replay")
+
+
+def test_compress_and_gather_in_one_grid():
+    """2:4, two-SM shape, index map: one compress grid that also gathers Xp, then the GEMM (two launches)."""
+    R, K, T = 512, 1024, 256
+    W = wl.normal_bf16((R, K), 0.02, seed=281)
+    X = wl.normal_bf16((K, T), 1.0, seed=282)
+    idx = wl.permutation(K, 283).astype(np.int32)
+    idx[[4, 9]] = [-1, K]  # zero rows
+    Wd, Xd, idxd = to_dev(W), to_dev(X), to_dev_i32(idx)
+    vals = torch.empty((R, K // 2), dtype=torch.bfloat16, device=DEV)
+    meta = torch.empty((nm.nm_meta_words(R, K, 2, 4),), dtype=torch.int32, device=DEV)
+    Y = torch.empty((R, T), dtype=torch.bfloat16, device=DEV)
+    torch.cuda.synchronize()
+    c0 = nm.nm_launch_count()
+    nm.nm_prune_spmm(Wd, K, 2, 4, R, K, idxd, Xd, T, T, Y, T, values=vals, meta=meta)
+    assert nm.nm_launch_count() - c0 == 2
+    torch.cuda.synchronize()
+    nm.nm_device_status()
+    ref, mag, ov, om = reference(W, X, 2, 4, idx)
+    assert_gemm_close(values_f64(Y), ref, mag, "compress + gather grid")
+    assert np.array_equal(bits(vals), ov) and np.array_equal(words(meta), om)
