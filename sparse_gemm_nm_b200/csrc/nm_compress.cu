@@ -32,8 +32,8 @@ __device__ __forceinline__ uint32_t mag_key(uint32_t bits16) {
 // eight rows, every load and every value store of the warp covers whole
 // 128-byte lines, and each lane keeps one byte of nibbles per row (rows
 // 2k + l/16: k = 0..3 in `lo8`, k = 4..7 in `hi8`).  The block's 64 words are
-// assembled with shuffles, two per lane.  The group selection is select_pair
-// (nm_select.cuh).
+// assembled with shuffles, two per lane.  The group selection is select_quad
+// (two groups per call, nm_select.cuh); select_pair for a lone group at a ragged edge.
 __global__ void __launch_bounds__(256, 4) compress_2of4_tiled_kernel(const uint16_t* __restrict__ W, uint32_t R,
                                                                   uint32_t K, int64_t ldw,
                                                                   uint16_t* __restrict__ V,
@@ -61,7 +61,7 @@ __global__ void __launch_bounds__(256, 4) compress_2of4_tiled_kernel(const uint1
         uint32_t byte = 0x44u;
         if (row < R && col < K) {
           uint32_t v0, v1;
-          byte = select_pair(in[i].x, in[i].y, v0) | (select_pair(in[i].z, in[i].w, v1) << 4);
+          byte = select_quad(in[i], v0, v1);
           *reinterpret_cast<uint2*>(V + (int64_t)row * (K >> 1) + col / 2) = make_uint2(v0, v1);
         }
         if (i < 4) lo8 = (lo8 & ~(0xFFu << (8 * i))) | (byte << (8 * i));

@@ -99,7 +99,7 @@ __global__ void __launch_bounds__(GATHER ? cstream::kThreadsGather : cstream::kT
     uint32_t pk[16], by[8];
 #pragma unroll
     for (int i = 0; i < 8; ++i)
-      by[i] = select_pair(in[i].x, in[i].y, pk[2 * i]) | (select_pair(in[i].z, in[i].w, pk[2 * i + 1]) << 4);
+      by[i] = select_quad(in[i], pk[2 * i], pk[2 * i + 1]);
     __syncwarp();
     if (lane == 0) mbar_arrive(&empty[slot]);  // the block's registers are consumed
     const uint32_t col = cb * 128 + 8 * piece;

@@ -208,7 +208,7 @@ __global__ void __launch_bounds__(fused::kThreads, 1) prune_spmm_skinny_kernel(c
         uint32_t pk[16], by[8];
 #pragma unroll
         for (int i = 0; i < 8; ++i)
-          by[i] = select_pair(in[i].x, in[i].y, pk[2 * i]) | (select_pair(in[i].z, in[i].w, pk[2 * i + 1]) << 4);
+          by[i] = select_quad(in[i], pk[2 * i], pk[2 * i + 1]);
         // compressed values into the A slot: tile row r, 128 bytes, 16-byte chunks swizzled by r % 8
         uint8_t* at = a_base + s * kA;
 #pragma unroll

@@ -112,3 +112,23 @@ def test_empty_shapes():
     assert v.shape == (0, 32) and mt.shape == (0,)
     with pytest.raises(nm.NmError):
         nm.prune_compress(torch.zeros((4, 10), dtype=torch.bfloat16, device=DEV), 2, 4)
+
+
+def test_selection_exhaustive_alphabet():
+    """Every group of four over a 12-value alphabet (+-0, +-1, 1 + ulp, +-Inf, NaNs with different payloads and
+    signs, denormals): the stream kernel (aligned rows), the other compress path (ldw % 8 != 0) and the fused
+    prune + GEMM all select exactly as the oracle."""
+    import itertools
+    alphabet = [0x0000, 0x8000, 0x3F80, 0xBF80, 0x3F81, 0x7F80, 0xFF80, 0x7FC0, 0xFFC1, 0x7F81, 0x0001, 0x8001]
+    groups = np.array(list(itertools.product(alphabet, repeat=4)), np.uint16)  # 20736 groups
+    W = groups.reshape(-1, 128)  # 648 rows of 32 groups
+    R, K = W.shape
+    ov, om = oracle.compress(W, 2, 4)
+    v, mt = gpu_compress(W, 2, 4)
+    assert np.array_equal(v, ov) and np.array_equal(mt, om)
+    v, mt = gpu_compress(W, 2, 4, ldw=132)
+    assert np.array_equal(v, ov) and np.array_equal(mt, om)
+    X = torch.zeros((K, 16), dtype=torch.bfloat16, device=DEV)
+    _, fv, fm = nm.prune_spmm(to_dev(W), 2, 4, X, keep_compressed=True)
+    torch.cuda.synchronize()
+    assert np.array_equal(bits(fv), ov) and np.array_equal(words(fm), om)
