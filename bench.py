@@ -390,6 +390,31 @@ def run_ours(args, rank: int, world: int, dist):
         step(evs[k])
     torch.cuda.synchronize()
     barrier()
+
+    # Third pass, for `roofline`: the GEMM launches of the step alone, back to back, no events between them
+    # (the step's layers together exceed L2, so every launch reads its operands from HBM).
+    def gemm_only():
+        for b in bufs:
+            if b["mode"] == "fused":
+                launch_fused(b)
+            elif b["mode"] == "combined":
+                launch_gemm_xp(b)
+            else:
+                launch_gemm(b)
+
+    greps = max(10, min(args.steps, 200))
+    for _ in range(2):
+        gemm_only()
+    torch.cuda.synchronize()
+    barrier()
+    g0, g1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    g0.record(stream)
+    for _ in range(greps):
+        gemm_only()
+    g1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    gemm_only_ms = max_over_ranks(g0.elapsed_time(g1)) / greps
     if sampler:
         sampler.stop()
     nm.nm_device_status(sp)
@@ -433,7 +458,7 @@ def run_ours(args, rank: int, world: int, dist):
     # dominant kernel: the GEMM (all launches of the step together)
     flops_all = sum(b["flops"] for b in bufs)
     bytes_all = sum(b["gemm_bytes"] for b in bufs)
-    gsec = gemm_ms.sum() * 1e-3
+    gsec = gemm_only_ms * 1e-3  # the GEMM launches of one step, timed back to back (third pass)
     tensor_bound = flops_all / (tc_peak * 1e12) >= bytes_all / (hbm_peak * 1e9)
     # DRAM bytes (read + write) of the GEMM call's kernels per layer, from one ncu capture
     # (profiles/<workload>_gemm_traffic.json); summed over the step like `achieved`.
@@ -463,7 +488,11 @@ def run_ours(args, rank: int, world: int, dist):
                            "the GEMM call (nm_spmm_permuted: gather_rows_kernel + spmm_pair_kernel, or nm_spmm / "
                            "nm_hybrid_spmm)"),
                 "peak_source": src,
-                "algorithmic_per_launch": [b["flops"] if tensor_bound else b["gemm_bytes"] for b in bufs]}
+                "algorithmic_per_launch": [b["flops"] if tensor_bound else b["gemm_bytes"] for b in bufs],
+                "timing": (f"CUDA events around {greps} back-to-back repetitions of the step's GEMM launches "
+                           "(one per layer, no events between them); per-layer event-bracketed times are in "
+                           "`kernels`"),
+                "gemm_step_us": 1e3 * gemm_only_ms}
 
     cfg = {"workload": args.workload, "shapes": [[b["L"].R, b["L"].K] for b in bufs],
            "T": [b["L"].T for b in bufs], "pattern": [f"{b['L'].n}:{b['L'].m}" for b in bufs],
