@@ -17,6 +17,8 @@ Sources, by page title and passage:
   * "Technische Samenvatting: SHUFFLESPARSE", "2. Methodologie": y = (W Pi) x
     with Pi applied as an index map on the input read.
   * "Structured Sparsity" topic cards, PATCH abstract: per-tile dense / 2:4.
+  * "M:N sparsity on NVIDIA tensor cores", the formats the sparse tensor cores
+    take (INT8 among them) and the INT8 storage arithmetic: the ``*_i8`` functions.
   * "Structured Sparsity" topic cards, RNM-TD3 abstract, and the DynaDiag
     page's abstract: N:M structure kept through training, sparse forward and
     backward passes (the gradients :func:`spmm_t` and :func:`sddmm`).
@@ -68,6 +70,10 @@ def _load():
                 "oracle_hybrid_weights": ([P, I64, I64, I64, P, I64, P], I),
                 "oracle_hybrid_spmm": ([P, I64, I64, I64, P, I64, P, I64, I64, P, P, I64], I),
                 "oracle_spmm_t": ([P, P, I, I, I64, I64, P, I64, I64, P, P, P, I64], I),
+                "oracle_prune_mask_i8": ([P, I64, I64, I64, I, I, P], I),
+                "oracle_compress_i8": ([P, I64, I64, I64, I, I, P, P], I),
+                "oracle_decompress_i8": ([P, P, I64, I64, I, I, P, I64], I),
+                "oracle_spmm_i8": ([P, P, I, I, I64, I64, P, I64, I64, P, I64], I),
                 "oracle_sddmm": ([P, I, I, I64, I64, P, I64, P, I64, I64, P, P, P], I),
             }
             for name, (args, res) in sig.items():
@@ -252,3 +258,49 @@ def sddmm(meta, n, m, R, K, dY, X, idx=None, with_abs=False):
     _check(_load().oracle_sddmm(_ptr(meta), n, m, R, K, _ptr(dY), T, _ptr(X), X.shape[1], T, _ptr(idx),
                                 _ptr(dV), _ptr(A)), "sddmm")
     return (dV, A) if with_abs else dV
+
+
+def _i8(a):
+    a = np.ascontiguousarray(a)
+    assert a.dtype == np.int8, "int8 data"
+    return a
+
+
+def prune_mask_i8(W, n, m):
+    W = _i8(W)
+    R, K = W.shape
+    mask = np.zeros((R, K), np.uint8)
+    _check(_load().oracle_prune_mask_i8(_ptr(W), R, K, K, n, m, _ptr(mask)), "prune_mask_i8")
+    return mask
+
+
+def compress_i8(W, n=2, m=4):
+    """(values R x K*n/m int8, meta uint32) of int8 W, same metadata packing as compress()."""
+    W = _i8(W)
+    R, K = W.shape
+    if K % m or not (1 <= n < m) or m not in (2, 4, 8, 16):
+        raise ValueError(f"oracle compress_i8 rejected its arguments (K={K}, {n}:{m})")
+    vals = np.zeros((R, value_cols(K, n, m)), np.int8)
+    meta = np.zeros(meta_words(R, K, n, m), np.uint32)
+    _check(_load().oracle_compress_i8(_ptr(W), R, K, K, n, m, _ptr(vals), _ptr(meta)), "compress_i8")
+    return vals, meta
+
+
+def decompress_i8(values, meta, K, n=2, m=4):
+    values = _i8(values)
+    meta = np.ascontiguousarray(meta, dtype=np.uint32)
+    R = values.shape[0]
+    out = np.zeros((R, K), np.int8)
+    _check(_load().oracle_decompress_i8(_ptr(values), _ptr(meta), R, K, n, m, _ptr(out), K), "decompress_i8")
+    return out
+
+
+def spmm_i8(values, meta, K, X, n=2, m=4):
+    """Exact int64 y = W' X for int8 compressed W' and int8 X (K x T)."""
+    values = _i8(values)
+    meta = np.ascontiguousarray(meta, dtype=np.uint32)
+    X = _i8(X)
+    R, T = values.shape[0], X.shape[1]
+    Y = np.zeros((R, T), np.int64)
+    _check(_load().oracle_spmm_i8(_ptr(values), _ptr(meta), n, m, R, K, _ptr(X), T, T, _ptr(Y), T), "spmm_i8")
+    return Y

@@ -36,6 +36,10 @@
  *             its input at the permuted addresses (same FLOP count).
  *  [PATCH]    "Structured Sparsity" topic cards, the PATCH abstract: weight
  *             matrices are split into tiles, each tile either dense or 2:4.
+ *  [MN-int8]  "M:N sparsity on NVIDIA tensor cores", passage on the formats
+ *             the sparse tensor cores accept (2:4 for FP16, BF16 and INT8
+ *             weights) and the storage paragraphs (a 2-bit index per stored
+ *             value: 25 % of an INT8 value, so INT8 2:4 saves 37.5 %).
  *  [TRAIN]    "Structured Sparsity" topic cards, RNM-TD3 abstract (N:M
  *             sparsity kept through the whole of training) and the
  *             DynaDiag page's abstract (sparse computation in the forward
@@ -457,6 +461,103 @@ int oracle_sddmm(const uint32_t *meta, int n, int m, int64_t R, int64_t K,
             }
             dV[r * vcols + j] = acc;
             if (dV_abs) dV_abs[r * vcols + j] = mag;
+        }
+    }
+    return 0;
+}
+
+/* ------------------------------------------------------------------ */
+/* INT8 weights [MN-int8].  The same rule on int8 values: the larger    */
+/* |w| wins (|-128| = 128 ranks above 127), equal magnitudes go to the  */
+/* lower index; values are pushed left and the positions use the same   */
+/* metadata packing as bf16 (tiled for 2:4).  The GEMM is exact integer */
+/* arithmetic: y[r][t] = sum_j V[r][j] * X[k_j][t] in 64 bits.           */
+/* ------------------------------------------------------------------ */
+int oracle_prune_mask_i8(const int8_t *W, int64_t R, int64_t K, int64_t ldw, int n, int m, uint8_t *mask)
+{
+    if (!pattern_ok(n, m) || K % m != 0 || ldw < K) return 1;
+    for (int64_t r = 0; r < R; r++) {
+        for (int64_t g = 0; g < K / m; g++) {
+            const int8_t *grp = W + r * ldw + g * m;
+            for (int i = 0; i < m; i++) {
+                int rank = 0, mi = abs((int)grp[i]);
+                for (int j = 0; j < m; j++) {
+                    int mj = abs((int)grp[j]);
+                    if (j != i && (mj > mi || (mj == mi && j < i))) rank++;
+                }
+                mask[r * K + g * m + i] = (uint8_t)(rank < n);
+            }
+        }
+    }
+    return 0;
+}
+
+int oracle_compress_i8(const int8_t *W, int64_t R, int64_t K, int64_t ldw, int n, int m, int8_t *values,
+                       uint32_t *meta)
+{
+    if (!pattern_ok(n, m) || K % m != 0 || ldw < K) return 1;
+    int64_t vcols = oracle_value_cols(K, n, m);
+    int64_t mcols = oracle_meta_cols(K, n, m);
+    int b = oracle_index_bits(m);
+    int s = oracle_positions_per_word(m);
+    uint8_t *mask = (uint8_t *)malloc((size_t)(R * K > 0 ? R * K : 1));
+    if (!mask) return 2;
+    oracle_prune_mask_i8(W, R, K, ldw, n, m, mask);
+    int tiled = (n == 2 && m == 4);
+    int64_t words = oracle_meta_words(R, K, n, m);
+    for (int64_t i = 0; i < words; i++) meta[i] = tiled ? 0x44444444u : 0u;
+    for (int64_t r = 0; r < R; r++) {
+        int64_t j = 0;
+        for (int64_t g = 0; g < K / m; g++) {
+            uint32_t nib = 0;
+            int seen = 0;
+            for (int p = 0; p < m; p++) {
+                if (!mask[r * K + g * m + p]) continue;
+                values[r * vcols + j] = W[r * ldw + g * m + p];
+                if (tiled)
+                    nib |= (uint32_t)p << (2 * seen);
+                else
+                    meta[r * mcols + j / s] |= (uint32_t)p << (b * (j % s));
+                seen++;
+                j++;
+            }
+            if (tiled) {
+                int bit;
+                int64_t w = meta_slot_2of4(r, g, K, &bit);
+                meta[w] = (meta[w] & ~(0xFu << bit)) | (nib << bit);
+            }
+        }
+    }
+    free(mask);
+    return 0;
+}
+
+int oracle_decompress_i8(const int8_t *values, const uint32_t *meta, int64_t R, int64_t K, int n, int m,
+                         int8_t *W_out, int64_t ldw)
+{
+    if (!pattern_ok(n, m) || K % m != 0 || ldw < K) return 1;
+    int64_t vcols = oracle_value_cols(K, n, m);
+    for (int64_t r = 0; r < R; r++) {
+        for (int64_t k = 0; k < K; k++) W_out[r * ldw + k] = 0;
+        for (int64_t j = 0; j < vcols; j++)
+            W_out[r * ldw + (j / n) * m + position_of(meta, K, r, j, n, m)] = values[r * vcols + j];
+    }
+    return 0;
+}
+
+int oracle_spmm_i8(const int8_t *values, const uint32_t *meta, int n, int m, int64_t R, int64_t K,
+                   const int8_t *X, int64_t ldx, int64_t T, int64_t *Y, int64_t ldy)
+{
+    if (!pattern_ok(n, m) || K % m != 0 || ldx < T || ldy < T) return 1;
+    int64_t vcols = oracle_value_cols(K, n, m);
+    for (int64_t r = 0; r < R; r++) {
+        for (int64_t t = 0; t < T; t++) {
+            int64_t acc = 0;
+            for (int64_t j = 0; j < vcols; j++) {
+                int64_t k = (j / n) * m + position_of(meta, K, r, j, n, m);
+                acc += (int64_t)values[r * vcols + j] * (int64_t)X[k * ldx + t];
+            }
+            Y[r * ldy + t] = acc;
         }
     }
     return 0;

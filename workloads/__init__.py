@@ -65,6 +65,17 @@ def integer_bf16(shape, lo: int, hi: int, seed: int) -> np.ndarray:
     return bf16_bits(_rng(seed).integers(lo, hi + 1, size=shape).astype(np.float32))
 
 
+def integer_i8(shape, lo: int, hi: int, seed: int) -> np.ndarray:
+    """int8 values drawn uniformly from [lo, hi] (-128 <= lo <= hi <= 127)."""
+    return _rng(seed).integers(lo, hi + 1, size=shape).astype(np.int8)
+
+
+def normal_i8(shape, std: float, seed: int) -> np.ndarray:
+    """int8 values: a normal draw scaled by std, rounded to nearest and clipped to [-128, 127]."""
+    x = np.rint(_rng(seed).standard_normal(shape, dtype=np.float32) * np.float32(std))
+    return np.clip(x, -128, 127).astype(np.int8)
+
+
 def permutation(K: int, seed: int) -> np.ndarray:
     return _rng(seed).permutation(K).astype(np.int32)
 
