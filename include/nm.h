@@ -233,6 +233,36 @@ NM_API nm_status nm_prune_spmm(const uint16_t* W, int64_t ldw, int n, int m, int
                                const int32_t* idx, const uint16_t* X, int64_t ldx, int64_t T, void* Y, int64_t ldy,
                                nm_out_dtype y_dtype, uint16_t* values, uint32_t* meta, void* stream);
 
+/* ----------------------------------------------------------------- INT8 */
+/*
+ * INT8 2:4 weights.  Source: "M:N sparsity on NVIDIA tensor cores" -- the
+ * sparse tensor cores take 2:4 for FP16, BF16 and INT8 weights; with a 2-bit
+ * index per stored value INT8 2:4 keeps 62.5 % of the dense bytes (a 37.5 %
+ * saving).  Same selection rule as nm_prune_compress on int8 magnitudes
+ * (|-128| = 128 ranks above 127, equal magnitudes to the lower index), values
+ * pushed left (R x K/2 int8), and the same tiled 2:4 metadata
+ * (nm_meta_words(R, K, 2, 4) words).  All three need K % 16 == 0
+ * (NM_ERR_UNSUPPORTED otherwise).
+ *
+ * nm_prune_compress_i8: W R x K int8 (row stride ldw >= K, ldw % 8 == 0,
+ *   8-byte aligned); values 4-byte and meta 8-byte aligned.
+ * nm_decompress_i8: W_out R x K int8 (ldw % 16 == 0, 16-byte aligned), 0 at
+ *   the pruned positions.
+ * nm_spmm_i8: Y = W' X exactly in int32, X K x T int8 (ldx % 16 == 0, 16-byte
+ *   aligned), Y R x T int32 (ldy % 4 == 0, 16-byte aligned).  The operand is
+ *   decompressed into a staging buffer (R x K bytes from the library's pool,
+ *   one launch), then a dense tcgen05 kind::i8 GEMM on SM pairs (a second
+ *   launch).  |W'| <= 128 and |X| <= 128, so a sum overflows int32 only for
+ *   K > 131072; the call does not check.
+ * Errors: NM_ERR_INVALID_ARG, NM_ERR_UNSUPPORTED, NM_ERR_MISALIGNED, NM_ERR_CUDA.
+ */
+NM_API nm_status nm_prune_compress_i8(const int8_t* W, int64_t R, int64_t K, int64_t ldw, int8_t* values,
+                                      uint32_t* meta, void* stream);
+NM_API nm_status nm_decompress_i8(const int8_t* values, const uint32_t* meta, int64_t R, int64_t K, int8_t* W_out,
+                                  int64_t ldw, void* stream);
+NM_API nm_status nm_spmm_i8(const int8_t* values, const uint32_t* meta, int64_t R, int64_t K, const int8_t* X,
+                            int64_t ldx, int64_t T, int32_t* Y, int64_t ldy, void* stream);
+
 /* ------------------------------------------------------------- backward */
 /*
  * nm_spmm_t -- input gradient of y = (W' Pi) x: dX = (W' Pi)^T dY, i.e.

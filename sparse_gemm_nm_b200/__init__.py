@@ -51,6 +51,9 @@ SIGNATURES = {
     "nm_hybrid_spmm": ([_P, _I64, _P, _P, _P, _I, _I64, _I64, _P, _I64, _I64, _P, _I64, _I, _P], _I),
     "nm_prune_spmm": ([_P, _I64, _I, _I, _I64, _I64, _P, _P, _I64, _I64, _P, _I64, _I, _P, _P, _P], _I),
     "nm_spmm_t": ([_P, _P, _I, _I, _I64, _I64, _P, _P, _I64, _I64, _P, _I64, _I, _P], _I),
+    "nm_prune_compress_i8": ([_P, _I64, _I64, _I64, _P, _P, _P], _I),
+    "nm_decompress_i8": ([_P, _P, _I64, _I64, _P, _I64, _P], _I),
+    "nm_spmm_i8": ([_P, _P, _I64, _I64, _P, _I64, _I64, _P, _I64, _P], _I),
     "nm_sddmm": ([_P, _I, _I, _I64, _I64, _P, _P, _I64, _P, _I64, _I64, _P, _I, _P], _I),
     "nm_spmm_algo": ([_P, _P, _I, _I, _I64, _I64, _P, _P, _I64, _I64, _P, _I64, _I, _I, _P], _I),
     "nm_spmm_permuted_noalloc": ([_P, _P, _I, _I, _I64, _I64, _P, _P, _I64, _I64, _P, _I64, _I, _P], _I),
@@ -173,6 +176,21 @@ def nm_spmm_t(values, meta, n, m, R, K, idx, dY, lddy, T, dX, lddx, dtype=NM_OUT
 def nm_sddmm(meta, n, m, R, K, idx, dY, lddy, X, ldx, T, dV, dtype=NM_OUT_BF16, stream=None) -> None:
     _check(lib().nm_sddmm(_ptr(meta), n, m, R, K, _ptr(idx), _ptr(dY), lddy, _ptr(X), ldx, T, _ptr(dV), dtype,
                           _stream(stream)), "nm_sddmm")
+
+
+def nm_prune_compress_i8(W, R, K, ldw, values, meta, stream=None) -> None:
+    _check(lib().nm_prune_compress_i8(_ptr(W), R, K, ldw, _ptr(values), _ptr(meta), _stream(stream)),
+           "nm_prune_compress_i8")
+
+
+def nm_decompress_i8(values, meta, R, K, W_out, ldw, stream=None) -> None:
+    _check(lib().nm_decompress_i8(_ptr(values), _ptr(meta), R, K, _ptr(W_out), ldw, _stream(stream)),
+           "nm_decompress_i8")
+
+
+def nm_spmm_i8(values, meta, R, K, X, ldx, T, Y, ldy, stream=None) -> None:
+    _check(lib().nm_spmm_i8(_ptr(values), _ptr(meta), R, K, _ptr(X), ldx, T, _ptr(Y), ldy, _stream(stream)),
+           "nm_spmm_i8")
 
 
 def nm_spmm_algo(values, meta, n, m, R, K, idx, X, ldx, T, Y, ldy, y_dtype=NM_OUT_BF16, algo=NM_ALGO_AUTO,
@@ -318,3 +336,34 @@ def sddmm(meta, n: int, m: int, R: int, K: int, dY, X, idx=None, out_dtype=None,
     yt = NM_OUT_F32 if out_dtype == torch.float32 else NM_OUT_BF16
     nm_sddmm(meta, n, m, R, K, idx, dY, dY.stride(0), X, X.stride(0), T, dV, yt, stream)
     return dV
+
+
+def prune_compress_i8(W, stream=None):
+    """2:4 (values R x K/2 int8, meta uint32 as int32) of int8 W (R x K)."""
+    import torch
+    _require_cuda(W)
+    R, K = W.shape
+    vals = torch.empty((R, K // 2), dtype=torch.int8, device=W.device)
+    meta = torch.empty((max(nm_meta_words(R, K, 2, 4), 0),), dtype=torch.int32, device=W.device)
+    nm_prune_compress_i8(W, R, K, W.stride(0), vals, meta, stream)
+    return vals, meta
+
+
+def decompress_i8(values, meta, K: int, stream=None):
+    import torch
+    _require_cuda(values, meta)
+    R = values.shape[0]
+    out = torch.empty((R, K), dtype=torch.int8, device=values.device)
+    nm_decompress_i8(values, meta, R, K, out, K, stream)
+    return out
+
+
+def spmm_i8(values, meta, K: int, X, stream=None):
+    """Y = W' X (int32, exact) from the int8 2:4 operand and int8 X (K x T)."""
+    import torch
+    _require_cuda(values, meta, X)
+    R, T = values.shape[0], X.shape[1]
+    ld = max((T + 3) // 4 * 4, 4)
+    Y = torch.empty((R, ld), dtype=torch.int32, device=X.device)
+    nm_spmm_i8(values, meta, R, K, X, X.stride(0), T, Y, ld, stream)
+    return Y[:, :T]

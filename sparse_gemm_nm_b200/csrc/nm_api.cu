@@ -917,6 +917,104 @@ static nm_status run_sddmm(const uint32_t* meta, int n, int m, int64_t R, int64_
   return e == cudaSuccess ? NM_OK : cuda_fail(e, "value-gradient GEMM launch");
 }
 
+
+// INT8 2:4 (compress, decompress, GEMM on the decompressed operand).
+static bool aligned_to(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+
+static nm_status check_i8_shape(int64_t R, int64_t K) {
+  if (R < 0 || K < 0) return fail(NM_ERR_INVALID_ARG, "negative dimension");
+  if (K % 16 != 0) return fail(NM_ERR_UNSUPPORTED, "int8 calls need K %% 16 == 0 (K = %lld)", (long long)K);
+  if (R >= (1ll << 31) || K >= (1ll << 31)) return fail(NM_ERR_UNSUPPORTED, "matrix too large for one call");
+  return NM_OK;
+}
+
+static nm_status run_compress_i8(const int8_t* W, int64_t R, int64_t K, int64_t ldw, int8_t* values, uint32_t* meta,
+                                 cudaStream_t stream) {
+  t_last_error.clear();
+  nm_status st = check_i8_shape(R, K);
+  if (st != NM_OK) return st;
+  if (ldw < K) return fail(NM_ERR_INVALID_ARG, "ldw < K");
+  if (R == 0 || K == 0) return NM_OK;
+  if (!W || !values || !meta) return fail(NM_ERR_INVALID_ARG, "null pointer");
+  if (!aligned_to(W, 8) || ldw % 8 != 0 || !aligned_to(values, 4) || !aligned_to(meta, 8))
+    return fail(NM_ERR_MISALIGNED, "int8 compress: W rows 8-byte aligned, values 4-byte, meta 8-byte");
+  st = require_device();
+  if (st != NM_OK) return st;
+  cudaError_t e = launch_compress_i8(W, R, K, ldw, values, meta, stream);
+  return e == cudaSuccess ? NM_OK : cuda_fail(e, "int8 compress launch");
+}
+
+static nm_status run_decompress_i8(const int8_t* values, const uint32_t* meta, int64_t R, int64_t K, int8_t* W_out,
+                                   int64_t ldw, cudaStream_t stream) {
+  t_last_error.clear();
+  nm_status st = check_i8_shape(R, K);
+  if (st != NM_OK) return st;
+  if (ldw < K) return fail(NM_ERR_INVALID_ARG, "ldw < K");
+  if (R == 0 || K == 0) return NM_OK;
+  if (!W_out || !values || !meta) return fail(NM_ERR_INVALID_ARG, "null pointer");
+  if (!aligned_to(W_out, 16) || ldw % 16 != 0 || !aligned_to(values, 8) || !aligned_to(meta, 4))
+    return fail(NM_ERR_MISALIGNED, "int8 decompress: W_out rows 16-byte aligned, values 8-byte");
+  st = require_device();
+  if (st != NM_OK) return st;
+  cudaError_t e = launch_decompress_i8(values, meta, R, K, W_out, ldw, stream);
+  return e == cudaSuccess ? NM_OK : cuda_fail(e, "int8 decompress launch");
+}
+
+static nm_status run_spmm_i8(const int8_t* values, const uint32_t* meta, int64_t R, int64_t K, const int8_t* X,
+                             int64_t ldx, int64_t T, int32_t* Y, int64_t ldy, cudaStream_t stream) {
+  t_last_error.clear();
+  nm_status st = check_i8_shape(R, K);
+  if (st != NM_OK) return st;
+  if (T < 0) return fail(NM_ERR_INVALID_ARG, "negative dimension");
+  if (R == 0 || T == 0) return NM_OK;
+  if (!Y) return fail(NM_ERR_INVALID_ARG, "Y is null");
+  if (ldy < T) return fail(NM_ERR_INVALID_ARG, "ldy < T");
+  if (!al16(Y) || ldy % 4 != 0) return fail(NM_ERR_MISALIGNED, "Y rows must be 16-byte aligned");
+  if (T >= (1ll << 31)) return fail(NM_ERR_UNSUPPORTED, "dimensions must stay below 2^31");
+  st = require_device();
+  if (st != NM_OK) return st;
+  if (K == 0) {
+    cudaError_t e = launch_fill_zero(Y, R, T, ldy, 4, stream);
+    return e == cudaSuccess ? NM_OK : cuda_fail(e, "zero fill");
+  }
+  if (!values || !meta || !X) return fail(NM_ERR_INVALID_ARG, "null operand");
+  if (ldx < T) return fail(NM_ERR_INVALID_ARG, "ldx < T");
+  if (!al16(X) || ldx % 16 != 0) return fail(NM_ERR_MISALIGNED, "X rows must be 16-byte aligned");
+  if (!aligned_to(values, 8) || !aligned_to(meta, 4)) return fail(NM_ERR_MISALIGNED, "values must be 8-byte aligned");
+  cudaMemPool_t pool = nullptr;
+  cudaError_t e = staging_pool(&pool);
+  if (e != cudaSuccess) return cuda_fail(e, "staging pool");
+  void* wd = nullptr;
+  e = cudaMallocFromPoolAsync(&wd, (size_t)(R * K), pool, stream);
+  if (e != cudaSuccess) return cuda_fail(e, "staging buffer for the decompressed int8 weights");
+  e = launch_decompress_i8(values, meta, R, K, static_cast<int8_t*>(wd), K, stream);
+  DenseParams p;
+  std::memset(&p, 0, sizeof p);
+  p.M = R;
+  p.N = T;
+  p.Kr = K;
+  p.k_tiles = (K + 255) / 256;
+  p.tiles_m = (int)((R + 255) / 256);
+  p.tiles_n = (int)((T + 255) / 256);
+  p.num_tiles = p.tiles_m * p.tiles_n;
+  p.status = status_word_ptr();
+  p.out = Y;
+  p.ldo = ldy;
+  p.out_f32 = 1;  // the int32 accumulator bits, stored unchanged
+  if (e == cudaSuccess && !p.status) e = cudaErrorInvalidSymbol;
+  if ((int64_t)p.tiles_m * p.tiles_n >= (1ll << 31)) st = fail(NM_ERR_UNSUPPORTED, "too many tiles");
+  if (e == cudaSuccess && st == NM_OK)
+    st = make_tmap(&p.tm_a, wd, (uint64_t)K, (uint64_t)R, (uint64_t)K, 128, 64, 128, "W' (int8, dense)",
+                   CU_TENSOR_MAP_DATA_TYPE_UINT8);
+  if (e == cudaSuccess && st == NM_OK)
+    st = make_tmap(&p.tm_b, X, (uint64_t)T, (uint64_t)K, (uint64_t)ldx, 128, 64, 128, "X (int8)",
+                   CU_TENSOR_MAP_DATA_TYPE_UINT8);
+  if (e == cudaSuccess && st == NM_OK) e = launch_dense_pair_i8(p, stream);
+  cudaFreeAsync(wd, stream);
+  if (st != NM_OK) return st;
+  return e == cudaSuccess ? NM_OK : cuda_fail(e, "int8 GEMM launch");
+}
+
 }  // namespace nmk
 
 using namespace nmk;
@@ -1058,6 +1156,21 @@ nm_status nm_sddmm(const uint32_t* meta, int n, int m, int64_t R, int64_t K, con
                    int64_t lddy, const uint16_t* X, int64_t ldx, int64_t T, void* dV, nm_out_dtype dtype,
                    void* stream) {
   return run_sddmm(meta, n, m, R, K, idx, dY, lddy, X, ldx, T, dV, dtype, static_cast<cudaStream_t>(stream));
+}
+
+nm_status nm_prune_compress_i8(const int8_t* W, int64_t R, int64_t K, int64_t ldw, int8_t* values, uint32_t* meta,
+                               void* stream) {
+  return run_compress_i8(W, R, K, ldw, values, meta, static_cast<cudaStream_t>(stream));
+}
+
+nm_status nm_decompress_i8(const int8_t* values, const uint32_t* meta, int64_t R, int64_t K, int8_t* W_out,
+                           int64_t ldw, void* stream) {
+  return run_decompress_i8(values, meta, R, K, W_out, ldw, static_cast<cudaStream_t>(stream));
+}
+
+nm_status nm_spmm_i8(const int8_t* values, const uint32_t* meta, int64_t R, int64_t K, const int8_t* X, int64_t ldx,
+                     int64_t T, int32_t* Y, int64_t ldy, void* stream) {
+  return run_spmm_i8(values, meta, R, K, X, ldx, T, Y, ldy, static_cast<cudaStream_t>(stream));
 }
 
 nm_status nm_device_status(void* stream) {

@@ -61,11 +61,14 @@ __device__ __forceinline__ int64_t survivor_col(const DenseParams& p, int64_t r,
   return g * p.m + ((w >> (b * (int)(j % S))) & ((1u << b) - 1u));
 }
 
-template <bool A_MN, bool B_MN, int EPI>
+// I8: signed int8 operands and int32 accumulation (kind::i8).  A stage then holds 256 reduction steps in
+// the same bytes: A K-major as two 128-byte halves, B MN-major as one 128-column strip of 256 rows.
+template <bool A_MN, bool B_MN, int EPI, bool I8 = false>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dpair::kThreads, 1)
     dense_pair_kernel(const __grid_constant__ DenseParams p) {
   using namespace dpair;
-  constexpr uint32_t kIdesc = idesc_bf16_major(256, 256, A_MN, B_MN);
+  static_assert(!I8 || (!A_MN && B_MN), "int8: K-major A and MN-major B");
+  constexpr uint32_t kIdesc = I8 ? idesc_s8_major(256, 256, A_MN, B_MN) : idesc_bf16_major(256, 256, A_MN, B_MN);
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + kOffBar);
@@ -131,6 +134,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dpair::kThreads, 1)
           if (rank == 0) mbar_arrive_expect_tx(&full[s], kTx);
           uint8_t* a = smem + s * (kA + kB);
           uint8_t* b = a + kA;
+          if (I8) {  // A: two 128-step halves x two 64-row halves; B: four 64-row boxes of one 128-column strip
+            const int32_t k0 = (int32_t)(kt * 256);
+#pragma unroll
+            for (int i = 0; i < 2; ++i)
+#pragma unroll
+              for (int h = 0; h < 2; ++h)
+                tma_load_2d_pair(a + i * 16384 + h * 8192, &p.tm_a, bar, k0 + 128 * i, m0 + 64 * h);
+#pragma unroll
+            for (int j = 0; j < 4; ++j) tma_load_2d_pair(b + j * 8192, &p.tm_b, bar, n0, k0 + 64 * j);
+            if (++s == kStages) { s = 0; ph ^= 1u; }
+            continue;
+          }
           const int32_t k0 = (int32_t)(kt * 128);
 #pragma unroll
           for (int i = 0; i < 2; ++i) {
@@ -176,9 +191,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dpair::kThreads, 1)
             // apart); MN-major operands advance 16 rows of 128 B (strips 16 KB apart).
             const uint64_t ad = A_MN ? smem_desc(a_addr + kk * 2048, 16384, 1024, SWZ_128B)
                                      : smem_desc(a_addr + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024, SWZ_128B);
-            const uint64_t bd = B_MN ? smem_desc(b_addr + kk * 2048, 16384, 1024, SWZ_128B)
-                                     : smem_desc(b_addr + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024, SWZ_128B);
-            tc_mma_pair(d_tmem, ad, bd, kIdesc, (kt > 0 || kk > 0) ? 1u : 0u);
+            // int8 MN-major B: K = 32 step kk advances 32 rows of 128 B
+            const uint64_t bd = I8 ? smem_desc(b_addr + kk * 4096, 32768, 1024, SWZ_128B)
+                                : B_MN ? smem_desc(b_addr + kk * 2048, 16384, 1024, SWZ_128B)
+                                       : smem_desc(b_addr + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024, SWZ_128B);
+            if (I8)
+              tc_mma_pair_i8(d_tmem, ad, bd, kIdesc, (kt > 0 || kk > 0) ? 1u : 0u);
+            else
+              tc_mma_pair(d_tmem, ad, bd, kIdesc, (kt > 0 || kk > 0) ? 1u : 0u);
           }
           tc_commit_pair(&empty[s], 0x3);
           if (++s == kStages) { s = 0; ph ^= 1u; }
@@ -309,20 +329,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dpair::kThreads, 1)
   }
 }
 
-template <bool A_MN, bool B_MN, int EPI>
+template <bool A_MN, bool B_MN, int EPI, bool I8 = false>
 static cudaError_t launch_dp(const DenseParams& p, cudaStream_t stream) {
   static bool configured[64] = {};
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev >= 0 && dev < 64 && !configured[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(dense_pair_kernel<A_MN, B_MN, EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaError_t e = cudaFuncSetAttribute(dense_pair_kernel<A_MN, B_MN, EPI, I8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)dpair::kSmemBytes);
     if (e != cudaSuccess) return e;
     configured[dev] = true;
   }
   const int pairs_avail = sm_count_current() / 2;
   const int pairs = p.num_tiles < pairs_avail ? p.num_tiles : pairs_avail;
-  cudaError_t e = launch_pdl(dense_pair_kernel<A_MN, B_MN, EPI>, dim3(2 * pairs), dim3(dpair::kThreads),
+  cudaError_t e = launch_pdl(dense_pair_kernel<A_MN, B_MN, EPI, I8>, dim3(2 * pairs), dim3(dpair::kThreads),
                              (size_t)dpair::kSmemBytes, stream, p);
   count_launch();
   return e != cudaSuccess ? e : cudaGetLastError();
@@ -333,6 +353,13 @@ cudaError_t launch_dense_pair(const DenseParams& p, bool a_mn, bool b_mn, int ep
   if (a_mn && b_mn && epi == EPI_STORE) return launch_dp<true, true, EPI_STORE>(p, stream);
   if (!a_mn && !b_mn && epi == EPI_SURVIVORS) return launch_dp<false, false, EPI_SURVIVORS>(p, stream);
   return cudaErrorInvalidValue;
+}
+
+// int8 forward GEMM on the decompressed operand: A K-major, B MN-major, int32 stored through the 32-bit path
+// (p.out_f32 = 1 moves the accumulator bits unchanged).
+cudaError_t launch_dense_pair_i8(const DenseParams& p, cudaStream_t stream) {
+  if (p.num_tiles <= 0) return cudaSuccess;
+  return launch_dp<false, true, EPI_STORE, true>(p, stream);
 }
 
 }  // namespace nmk

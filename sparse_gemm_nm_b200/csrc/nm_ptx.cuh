@@ -246,6 +246,17 @@ __device__ __forceinline__ void tc_mma_pair(uint32_t d_tmem, uint64_t a_desc, ui
       : "memory");
 }
 
+// The same for kind::i8: signed 8-bit A and B, int32 accumulator.
+__device__ __forceinline__ void tc_mma_pair_i8(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                               uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::i8 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
 // Arrive once on the mbarrier at this shared offset in every CTA of cta_mask
 // when all previously issued pair tcgen05 operations have completed.
 __device__ __forceinline__ void tc_commit_pair(uint64_t* bar, uint16_t cta_mask) {
@@ -376,6 +387,12 @@ __host__ __device__ constexpr uint32_t idesc_bf16(uint32_t n, bool sparse, uint3
 // 15 / 16 (the operand is MN-major: M or N is the contiguous axis).
 __host__ __device__ constexpr uint32_t idesc_bf16_major(uint32_t n, uint32_t m, bool a_mn, bool b_mn) {
   return (1u << 4) | (1u << 7) | (1u << 10) | (a_mn ? (1u << 15) : 0u) | (b_mn ? (1u << 16) : 0u) |
+         ((n >> 3) << 17) | ((m >> 4) << 24);
+}
+
+// kind::i8 descriptor: signed 8-bit A and B, int32 D (c_format 2), operand majors as above.
+__host__ __device__ constexpr uint32_t idesc_s8_major(uint32_t n, uint32_t m, bool a_mn, bool b_mn) {
+  return (2u << 4) | (1u << 7) | (1u << 10) | (a_mn ? (1u << 15) : 0u) | (b_mn ? (1u << 16) : 0u) |
          ((n >> 3) << 17) | ((m >> 4) << 24);
 }
 
