@@ -54,6 +54,9 @@ def parse_args(argv=None):
     ap.add_argument("--algo", choices=["auto", "sparse", "dense"], default="auto",
                     help="kernel design for 1:4 / 1:8 (nm_spmm_algo)")
     ap.add_argument("--plain", action="store_true", help="ignore the workload's index map (y = W x)")
+    ap.add_argument("--dtype", choices=["bf16", "i8"], default="bf16",
+                    help="i8: INT8 2:4 weights and int8 inputs on the workload's shapes (nm_prune_compress_i8, then "
+                         "nm_spmm_i8; no index map), useful TOP/s against the int8 dense peak")
     ap.add_argument("--step", choices=["one-call", "two-calls"], default="one-call",
                     help="one-call: nm_prune_spmm per layer (prune + compress + GEMM in one library call, the "
                          "compressed form written too); two-calls: nm_prune_compress, then the GEMM call.  The "
@@ -647,6 +650,103 @@ def run_ours(args, rank: int, world: int, dist):
         print(json.dumps(line), flush=True)
 
 
+def run_i8(args, rank: int, world: int, dist):
+    """INT8 2:4 step on the workload's shapes: per layer nm_prune_compress_i8 then nm_spmm_i8 (exact int32)."""
+    import torch
+    import sparse_gemm_nm_b200 as nm
+
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    stream = torch.cuda.current_stream(dev)
+    sp = stream.cuda_stream
+    L_ = nm.lib()
+    layers = wl.workload(args.workload)
+    if args.layers:
+        layers = [layers[int(i)] for i in args.layers.split(",")]
+    if any(L.n != 2 or L.m != 4 or L.K % 16 for L in layers):
+        raise SystemExit("--dtype i8 needs 2:4 layers with K % 16 == 0")
+    bufs = []
+    for i, L in enumerate(layers):
+        T16 = (L.T + 15) // 16 * 16
+        Xb = np.zeros((L.K, T16), np.int8)
+        Xb[:, :L.T] = wl.integer_i8((L.K, L.T), -128, 127, seed=10 * i + 2)
+        b = {"L": L, "W": torch.from_numpy(wl.normal_i8((L.R, L.K), 32.0, seed=10 * i + 1)).to(dev),
+             "X": torch.from_numpy(Xb).to(dev), "ldx": T16,
+             "vals": torch.empty((L.R, L.K // 2), dtype=torch.int8, device=dev),
+             "meta": torch.empty((nm.nm_meta_words(L.R, L.K, 2, 4),), dtype=torch.int32, device=dev),
+             "Y": torch.empty((L.R, (L.T + 3) // 4 * 4), dtype=torch.int32, device=dev)}
+        b["ops"] = 2.0 * L.R * L.T * L.K / 2  # useful: survivors only
+        bufs.append(b)
+    torch.cuda.synchronize()
+
+    def check(st, what):
+        if st != 0:
+            raise RuntimeError(f"{what}: {L_.nm_last_error().decode()}")
+
+    def compress(b):
+        L = b["L"]
+        check(L_.nm_prune_compress_i8(b["W"].data_ptr(), L.R, L.K, L.K, b["vals"].data_ptr(), b["meta"].data_ptr(),
+                                      sp), "nm_prune_compress_i8")
+
+    def gemm(b):
+        L = b["L"]
+        check(L_.nm_spmm_i8(b["vals"].data_ptr(), b["meta"].data_ptr(), L.R, L.K, b["X"].data_ptr(), b["ldx"], L.T,
+                            b["Y"].data_ptr(), b["Y"].shape[1], sp), "nm_spmm_i8")
+
+    def step():
+        for b in bufs:
+            compress(b)
+            gemm(b)
+
+    def timed(fn, reps):
+        rank_barrier(dist)
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(reps):
+            fn()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        rank_barrier(dist)
+        return max_over_ranks_on(e0.elapsed_time(e1), dist, dev) / reps
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    props = torch.cuda.get_device_properties(dev)
+    sampler = None if args.quick else ClockSampler(f"GPU-{props.uuid}" if getattr(props, "uuid", None) else "")
+    if sampler:
+        sampler.start()
+    launches0 = nm.nm_launch_count()
+    ms_per_step = timed(step, args.steps)
+    launches = nm.nm_launch_count() - launches0
+    gemm_ms = timed(lambda: [gemm(b) for b in bufs], max(10, min(args.steps, 200)))
+    if sampler:
+        sampler.stop()
+    nm.nm_device_status(sp)
+    peaks, peak_src = load_peaks()
+    i8_peak = 2.0 * peaks["bf16_tflops"]
+    useful = sum(b["ops"] for b in bufs)
+    achieved = useful / (gemm_ms * 1e-3) / 1e12
+    line = {"metric": METRIC, "value": world * useful / (ms_per_step * 1e-3) / 1e12, "unit": "TOP/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "s8",
+            "data": "synthetic int8: W rounded N(0, 32^2) clipped to [-128, 127], X uniform int8",
+            "config": {"workload": args.workload + " (INT8 2:4)", "shapes": [[b["L"].R, b["L"].K] for b in bufs],
+                       "T": [b["L"].T for b in bufs], "step": "nm_prune_compress_i8, then nm_spmm_i8, per layer",
+                       "parallelism": f"replicas x{world}"},
+            "roofline": {"bound": "tensor", "achieved": achieved, "peak": i8_peak, "unit": "TOP/s",
+                         "frac": achieved / i8_peak, "traffic": None,
+                         "kernel": "nm_spmm_i8 calls: decompress_2of4_i8_kernel + dense_pair_kernel (kind::i8)",
+                         "peak_source": f"{peak_src} bf16 burst dense peak x 2 (the nominal int8 / bf16 dense ratio); "
+                                        "useful (survivor) operations, half of the dense ones",
+                         "timing": "CUDA events around back-to-back repetitions of the step's GEMM calls"},
+            "gpu_launches": launches, "clocks": sampler.summary() if sampler else None, "cpu_baseline": None}
+    if rank == 0:
+        print(json.dumps(line))
+
+
 def main(argv=None):
     args = parse_args(argv)
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -664,7 +764,7 @@ def main(argv=None):
         tdist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
         dist = tdist
     try:
-        run_ours(args, rank, world, dist)
+        (run_i8 if args.dtype == "i8" else run_ours)(args, rank, world, dist)
     finally:
         if dist is not None:
             dist.destroy_process_group()
