@@ -19,6 +19,9 @@ Sources, by page title and passage:
   * "Structured Sparsity" topic cards, PATCH abstract: per-tile dense / 2:4.
   * "M:N sparsity on NVIDIA tensor cores", the formats the sparse tensor cores
     take (INT8 among them) and the INT8 storage arithmetic: the ``*_i8`` functions.
+  * SHUFFLESPARSE's contributions (block, N:M and diagonal patterns under one
+    permutation) and the DynaDiag abstract: the ``diag_*`` functions (the pages
+    give no format; see the readings in nm_oracle.c).
   * "Structured Sparsity" topic cards, RNM-TD3 abstract, and the DynaDiag
     page's abstract: N:M structure kept through training, sparse forward and
     backward passes (the gradients :func:`spmm_t` and :func:`sddmm`).
@@ -71,6 +74,11 @@ def _load():
                 "oracle_hybrid_spmm": ([P, I64, I64, I64, P, I64, P, I64, I64, P, P, I64], I),
                 "oracle_spmm_t": ([P, P, I, I, I64, I64, P, I64, I64, P, P, P, I64], I),
                 "oracle_prune_mask_i8": ([P, I64, I64, I64, I, I, P], I),
+                "oracle_diag_scores": ([P, I64, I64, I64, P], I),
+                "oracle_diag_select": ([P, I64, I64, I64, I64, P], I),
+                "oracle_diag_compress": ([P, I64, I64, I64, I64, P, P], I),
+                "oracle_diag_expand": ([P, P, I64, I64, I64, P, I64], I),
+                "oracle_diag_spmm": ([P, P, I64, I64, I64, P, I64, I64, P, P, P, I64], I),
                 "oracle_compress_i8": ([P, I64, I64, I64, I, I, P, P], I),
                 "oracle_decompress_i8": ([P, P, I64, I64, I, I, P, I64], I),
                 "oracle_spmm_i8": ([P, P, I, I, I64, I64, P, I64, I64, P, I64], I),
@@ -304,3 +312,54 @@ def spmm_i8(values, meta, K, X, n=2, m=4):
     Y = np.zeros((R, T), np.int64)
     _check(_load().oracle_spmm_i8(_ptr(values), _ptr(meta), n, m, R, K, _ptr(X), T, T, _ptr(Y), T), "spmm_i8")
     return Y
+
+
+def diag_scores(W):
+    W = _u16(W)
+    R, K = W.shape
+    out = np.zeros(K, np.float32)
+    _check(_load().oracle_diag_scores(_ptr(W), R, K, K, _ptr(out)), "diag_scores")
+    return out
+
+
+def diag_select(W, D):
+    """Ascending int32 offsets of the D diagonals with the largest fp32 scores (ties to the lower offset)."""
+    W = _u16(W)
+    R, K = W.shape
+    out = np.zeros(D, np.int32)
+    _check(_load().oracle_diag_select(_ptr(W), R, K, K, D, _ptr(out)), "diag_select")
+    return out
+
+
+def diag_compress(W, offsets):
+    """V (D x R uint16): V[d][r] = W[r][(r + o_d) mod K]."""
+    W = _u16(W)
+    R, K = W.shape
+    offsets = np.ascontiguousarray(offsets, dtype=np.int32)
+    V = np.zeros((len(offsets), R), np.uint16)
+    _check(_load().oracle_diag_compress(_ptr(W), R, K, K, len(offsets), _ptr(offsets), _ptr(V)), "diag_compress")
+    return V
+
+
+def diag_expand(values, offsets, K):
+    values = _u16(values)
+    offsets = np.ascontiguousarray(offsets, dtype=np.int32)
+    D, R = values.shape
+    out = np.zeros((R, K), np.uint16)
+    _check(_load().oracle_diag_expand(_ptr(values), _ptr(offsets), D, R, K, _ptr(out), K), "diag_expand")
+    return out
+
+
+def diag_spmm(values, offsets, K, X, idx=None, with_abs=False):
+    values = _u16(values)
+    offsets = np.ascontiguousarray(offsets, dtype=np.int32)
+    X = _u16(X)
+    D, R = values.shape
+    T = X.shape[1]
+    if idx is not None:
+        idx = np.ascontiguousarray(idx, dtype=np.int32)
+    Y = np.zeros((R, T), np.float64)
+    A = np.zeros((R, T), np.float64) if with_abs else None
+    _check(_load().oracle_diag_spmm(_ptr(values), _ptr(offsets), D, R, K, _ptr(X), T, T, _ptr(idx), _ptr(Y),
+                                    _ptr(A), T), "diag_spmm")
+    return (Y, A) if with_abs else Y

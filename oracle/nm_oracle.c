@@ -40,6 +40,12 @@
  *             the sparse tensor cores accept (2:4 for FP16, BF16 and INT8
  *             weights) and the storage paragraphs (a 2-bit index per stored
  *             value: 25 % of an INT8 value, so INT8 2:4 saves 37.5 %).
+ *  [DIAG]     SHUFFLESPARSE (the technical summary's contributions and the
+ *             author page's abstract): one permutation primitive over block,
+ *             N:M and diagonal patterns; the DynaDiag abstract on the same
+ *             author page: a diagonal sparsity pattern kept through training,
+ *             90 % sparse ViT linears.  The pages give no format; the
+ *             readings are below.
  *  [TRAIN]    "Structured Sparsity" topic cards, RNM-TD3 abstract (N:M
  *             sparsity kept through the whole of training) and the
  *             DynaDiag page's abstract (sparse computation in the forward
@@ -63,6 +69,12 @@
  *    nibble of an all-zero group, positions (0,1);
  *  - the permutation is applied as X_perm[k][t] = X[idx[k]][t]; an entry of
  *    idx outside [0, K) reads a zero row;
+ *  - diagonal pattern: diagonal o (0 <= o < K) of an R x K matrix is the set
+ *    {(r, (r + o) mod K)}, one entry per row (wrapping); a diagonally sparse
+ *    weight keeps D distinct offsets (ascending) and stores V[d][r] =
+ *    W[r][(r + o_d) mod K] (D x R); one-shot selection keeps the D diagonals
+ *    of largest score s(o) = sum_r |W[r][(r + o) mod K]| (an fp32 sum in
+ *    ascending r, NaN above every number), ties to the lower offset;
  *  - backward: dX is the adjoint of that gather (row k of W'^T dY is added to
  *    row idx[k] of dX; entries outside [0, K) drop their row, repeated
  *    entries add up), and the gradient of the stored values is
@@ -558,6 +570,98 @@ int oracle_spmm_i8(const int8_t *values, const uint32_t *meta, int n, int m, int
                 acc += (int64_t)values[r * vcols + j] * (int64_t)X[k * ldx + t];
             }
             Y[r * ldy + t] = acc;
+        }
+    }
+    return 0;
+}
+
+/* ------------------------------------------------------------------ */
+/* Diagonal sparsity [DIAG] (readings in the header).                   */
+/* ------------------------------------------------------------------ */
+/* s(o) = sum_r |W[r][(r + o) mod K]| in float32, r ascending. */
+int oracle_diag_scores(const uint16_t *W, int64_t R, int64_t K, int64_t ldw, float *scores)
+{
+    if (K <= 0 || ldw < K) return 1;
+    for (int64_t o = 0; o < K; o++) {
+        float acc = 0.0f;
+        for (int64_t r = 0; r < R; r++) acc += (float)fabs(bf16_value(W[r * ldw + (r + o) % K]));
+        scores[o] = acc;
+    }
+    return 0;
+}
+
+/* Does offset a (score sa) rank above offset b (score sb)? */
+static int diag_beats(float sa, int64_t a, float sb, int64_t b)
+{
+    int na = isnan(sa), nb = isnan(sb);
+    if (na || nb) {
+        if (na && !nb) return 1;
+        if (nb && !na) return 0;
+        return a < b;
+    }
+    if (sa != sb) return sa > sb;
+    return a < b;
+}
+
+/* The D best offsets by score, written in ascending order. */
+int oracle_diag_select(const uint16_t *W, int64_t R, int64_t K, int64_t ldw, int64_t D, int32_t *offsets)
+{
+    if (K <= 0 || D < 0 || D > K || ldw < K) return 1;
+    float *s = (float *)malloc((size_t)K * sizeof(float));
+    if (!s) return 2;
+    oracle_diag_scores(W, R, K, ldw, s);
+    int64_t n = 0;
+    for (int64_t o = 0; o < K; o++) {
+        int64_t rank = 0;
+        for (int64_t p = 0; p < K; p++)
+            if (p != o && diag_beats(s[p], p, s[o], o)) rank++;
+        if (rank < D) offsets[n++] = (int32_t)o;
+    }
+    free(s);
+    return n == D ? 0 : 3;
+}
+
+/* V[d][r] = W[r][(r + o_d) mod K]. */
+int oracle_diag_compress(const uint16_t *W, int64_t R, int64_t K, int64_t ldw, int64_t D, const int32_t *offsets,
+                         uint16_t *values)
+{
+    if (K <= 0 || ldw < K) return 1;
+    for (int64_t d = 0; d < D; d++)
+        for (int64_t r = 0; r < R; r++) values[d * R + r] = W[r * ldw + (r + offsets[d]) % K];
+    return 0;
+}
+
+/* The dense R x K matrix of a diagonal operand: +0 off the kept diagonals. */
+int oracle_diag_expand(const uint16_t *values, const int32_t *offsets, int64_t D, int64_t R, int64_t K,
+                       uint16_t *W_out, int64_t ldw)
+{
+    if (K <= 0 || ldw < K) return 1;
+    for (int64_t r = 0; r < R; r++)
+        for (int64_t k = 0; k < K; k++) W_out[r * ldw + k] = 0;
+    for (int64_t d = 0; d < D; d++)
+        for (int64_t r = 0; r < R; r++) W_out[r * ldw + (r + offsets[d]) % K] = values[d * R + r];
+    return 0;
+}
+
+/* y[r][t] = sum_d V[d][r] * X[pi((r + o_d) mod K)][t] in double; y_abs gets the sums of |products|. */
+int oracle_diag_spmm(const uint16_t *values, const int32_t *offsets, int64_t D, int64_t R, int64_t K,
+                     const uint16_t *X, int64_t ldx, int64_t T, const int32_t *idx, double *Y, double *Y_abs,
+                     int64_t ldy)
+{
+    if (K <= 0 || ldx < T || ldy < T) return 1;
+    for (int64_t r = 0; r < R; r++) {
+        for (int64_t t = 0; t < T; t++) {
+            double acc = 0.0, mag = 0.0;
+            for (int64_t d = 0; d < D; d++) {
+                int64_t k = (r + offsets[d]) % K;
+                int64_t src = idx ? (int64_t)idx[k] : k;
+                double w = bf16_value(values[d * R + r]);
+                double x = (src < 0 || src >= K) ? 0.0 : bf16_value(X[src * ldx + t]);
+                acc += w * x;
+                mag += fabs(w) * fabs(x);
+            }
+            Y[r * ldy + t] = acc;
+            if (Y_abs) Y_abs[r * ldy + t] = mag;
         }
     }
     return 0;
