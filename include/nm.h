@@ -263,6 +263,40 @@ NM_API nm_status nm_decompress_i8(const int8_t* values, const uint32_t* meta, in
 NM_API nm_status nm_spmm_i8(const int8_t* values, const uint32_t* meta, int64_t R, int64_t K, const int8_t* X,
                             int64_t ldx, int64_t T, int32_t* Y, int64_t ldy, void* stream);
 
+/* ------------------------------------------------------------- diagonal */
+/*
+ * Diagonal sparsity under the index map.  Source: the SHUFFLESPARSE technical
+ * summary, section "3. Belangrijkste Bijdragen" (one permutation primitive
+ * over block, N:M and diagonal patterns), and the DynaDiag abstract on the
+ * SHUFFLESPARSE author page (a diagonal pattern kept through training, 90 %
+ * sparse ViT linears).  The pages give no format; this library reads it as:
+ * diagonal o (0 <= o < K) of an R x K matrix is {(r, (r + o) mod K)}, one
+ * entry per row; a diagonal operand is D distinct offsets (int32, ascending)
+ * and values V (D x R bf16), V[d][r] = W[r][(r + o_d) mod K].
+ *
+ * nm_diag_prune_compress: keep the D diagonals of largest score
+ *   s(o) = sum_r |W[r][(r + o) mod K]| (fp32, summed in ascending r; NaN
+ *   ranks above every number; ties to the lower offset); writes offsets[D]
+ *   and values (D x R).  Stages K*5 bytes from the library's pool; four
+ *   launches (scores, ranks, placement, gather).
+ * nm_diag_expand: the dense R x K copy (+0 off the kept diagonals), row
+ *   stride ldw >= K; offsets outside [0, K) place nothing.
+ * nm_diag_spmm: y[r][t] = sum_d V[d][r] * X[idx[(r + o_d) mod K]][t]
+ *   (X[k] when idx is NULL; idx entries outside [0, K) read zero rows).
+ *   Offsets must be distinct.  The operand is expanded into a staged dense
+ *   copy (R x ceil8(K) bf16) and multiplied by a dense tcgen05 GEMM on SM
+ *   pairs; with idx one gather pass stages X[idx] first.  X, Y as nm_spmm.
+ * Errors: NM_ERR_INVALID_ARG (D > K, ld too small, null), NM_ERR_MISALIGNED,
+ *   NM_ERR_UNSUPPORTED, NM_ERR_CUDA.
+ */
+NM_API nm_status nm_diag_prune_compress(const uint16_t* W, int64_t R, int64_t K, int64_t ldw, int64_t D,
+                                        int32_t* offsets, uint16_t* values, void* stream);
+NM_API nm_status nm_diag_expand(const uint16_t* values, const int32_t* offsets, int64_t D, int64_t R, int64_t K,
+                                uint16_t* W_out, int64_t ldw, void* stream);
+NM_API nm_status nm_diag_spmm(const uint16_t* values, const int32_t* offsets, int64_t D, int64_t R, int64_t K,
+                              const int32_t* idx, const uint16_t* X, int64_t ldx, int64_t T, void* Y, int64_t ldy,
+                              nm_out_dtype dtype, void* stream);
+
 /* ------------------------------------------------------------- backward */
 /*
  * nm_spmm_t -- input gradient of y = (W' Pi) x: dX = (W' Pi)^T dY, i.e.

@@ -52,6 +52,9 @@ SIGNATURES = {
     "nm_prune_spmm": ([_P, _I64, _I, _I, _I64, _I64, _P, _P, _I64, _I64, _P, _I64, _I, _P, _P, _P], _I),
     "nm_spmm_t": ([_P, _P, _I, _I, _I64, _I64, _P, _P, _I64, _I64, _P, _I64, _I, _P], _I),
     "nm_prune_compress_i8": ([_P, _I64, _I64, _I64, _P, _P, _P], _I),
+    "nm_diag_prune_compress": ([_P, _I64, _I64, _I64, _I64, _P, _P, _P], _I),
+    "nm_diag_expand": ([_P, _P, _I64, _I64, _I64, _P, _I64, _P], _I),
+    "nm_diag_spmm": ([_P, _P, _I64, _I64, _I64, _P, _P, _I64, _I64, _P, _I64, _I, _P], _I),
     "nm_decompress_i8": ([_P, _P, _I64, _I64, _P, _I64, _P], _I),
     "nm_spmm_i8": ([_P, _P, _I64, _I64, _P, _I64, _I64, _P, _I64, _P], _I),
     "nm_sddmm": ([_P, _I, _I, _I64, _I64, _P, _P, _I64, _P, _I64, _I64, _P, _I, _P], _I),
@@ -191,6 +194,21 @@ def nm_decompress_i8(values, meta, R, K, W_out, ldw, stream=None) -> None:
 def nm_spmm_i8(values, meta, R, K, X, ldx, T, Y, ldy, stream=None) -> None:
     _check(lib().nm_spmm_i8(_ptr(values), _ptr(meta), R, K, _ptr(X), ldx, T, _ptr(Y), ldy, _stream(stream)),
            "nm_spmm_i8")
+
+
+def nm_diag_prune_compress(W, R, K, ldw, D, offsets, values, stream=None) -> None:
+    _check(lib().nm_diag_prune_compress(_ptr(W), R, K, ldw, D, _ptr(offsets), _ptr(values), _stream(stream)),
+           "nm_diag_prune_compress")
+
+
+def nm_diag_expand(values, offsets, D, R, K, W_out, ldw, stream=None) -> None:
+    _check(lib().nm_diag_expand(_ptr(values), _ptr(offsets), D, R, K, _ptr(W_out), ldw, _stream(stream)),
+           "nm_diag_expand")
+
+
+def nm_diag_spmm(values, offsets, D, R, K, idx, X, ldx, T, Y, ldy, y_dtype=NM_OUT_BF16, stream=None) -> None:
+    _check(lib().nm_diag_spmm(_ptr(values), _ptr(offsets), D, R, K, _ptr(idx), _ptr(X), ldx, T, _ptr(Y), ldy,
+                              y_dtype, _stream(stream)), "nm_diag_spmm")
 
 
 def nm_spmm_algo(values, meta, n, m, R, K, idx, X, ldx, T, Y, ldy, y_dtype=NM_OUT_BF16, algo=NM_ALGO_AUTO,
@@ -366,4 +384,29 @@ def spmm_i8(values, meta, K: int, X, stream=None):
     ld = max((T + 3) // 4 * 4, 4)
     Y = torch.empty((R, ld), dtype=torch.int32, device=X.device)
     nm_spmm_i8(values, meta, R, K, X, X.stride(0), T, Y, ld, stream)
+    return Y[:, :T]
+
+
+def diag_prune_compress(W, D: int, stream=None):
+    """(offsets int32[D] ascending, values D x R bf16) of the D highest-scoring diagonals of bf16 W (R x K)."""
+    import torch
+    _require_cuda(W)
+    R, K = W.shape
+    offsets = torch.empty((D,), dtype=torch.int32, device=W.device)
+    values = torch.empty((D, R), dtype=torch.bfloat16, device=W.device)
+    nm_diag_prune_compress(W, R, K, W.stride(0), D, offsets, values, stream)
+    return offsets, values
+
+
+def diag_spmm(values, offsets, K: int, X, idx=None, out_dtype=None, stream=None):
+    import torch
+    _require_cuda(values, offsets, X, idx)
+    out_dtype = out_dtype or torch.bfloat16
+    D, R = values.shape
+    T = X.shape[1]
+    per16 = 4 if out_dtype == torch.float32 else 8
+    ld = max((T + per16 - 1) // per16 * per16, per16)
+    Y = torch.empty((R, ld), dtype=out_dtype, device=X.device)
+    yt = NM_OUT_F32 if out_dtype == torch.float32 else NM_OUT_BF16
+    nm_diag_spmm(values, offsets, D, R, K, idx, X, X.stride(0), T, Y, ld, yt, stream)
     return Y[:, :T]

@@ -1015,6 +1015,112 @@ static nm_status run_spmm_i8(const int8_t* values, const uint32_t* meta, int64_t
   return e == cudaSuccess ? NM_OK : cuda_fail(e, "int8 GEMM launch");
 }
 
+
+// Diagonal sparsity: selection + gather, dense copy, GEMM on the dense copy.
+static nm_status run_diag_prune_compress(const uint16_t* W, int64_t R, int64_t K, int64_t ldw, int64_t D,
+                                         int32_t* offsets, uint16_t* values, cudaStream_t stream) {
+  t_last_error.clear();
+  if (R < 0 || K < 0 || D < 0) return fail(NM_ERR_INVALID_ARG, "negative dimension");
+  if (D > K) return fail(NM_ERR_INVALID_ARG, "D > K");
+  if (ldw < K) return fail(NM_ERR_INVALID_ARG, "ldw < K");
+  if (K == 0 || D == 0) return NM_OK;
+  if (!W || !offsets || (R > 0 && !values)) return fail(NM_ERR_INVALID_ARG, "null pointer");
+  if (R >= (1ll << 31) || K >= (1ll << 31)) return fail(NM_ERR_UNSUPPORTED, "matrix too large for one call");
+  nm_status st = require_device();
+  if (st != NM_OK) return st;
+  cudaMemPool_t pool = nullptr;
+  cudaError_t e = staging_pool(&pool);
+  if (e != cudaSuccess) return cuda_fail(e, "staging pool");
+  void* buf = nullptr;
+  const size_t sbytes = (size_t)((K * 4 + 255) / 256 * 256);
+  e = cudaMallocFromPoolAsync(&buf, sbytes + (size_t)K, pool, stream);
+  if (e != cudaSuccess) return cuda_fail(e, "staging buffer for the diagonal scores");
+  e = launch_diag_select(W, R, K, ldw, D, static_cast<float*>(buf), static_cast<uint8_t*>(buf) + sbytes, offsets,
+                         values, stream);
+  cudaFreeAsync(buf, stream);
+  return e == cudaSuccess ? NM_OK : cuda_fail(e, "diagonal selection launch");
+}
+
+static nm_status run_diag_expand(const uint16_t* values, const int32_t* offsets, int64_t D, int64_t R, int64_t K,
+                                 uint16_t* W_out, int64_t ldw, cudaStream_t stream) {
+  t_last_error.clear();
+  if (R < 0 || K < 0 || D < 0) return fail(NM_ERR_INVALID_ARG, "negative dimension");
+  if (D > K || ldw < K) return fail(NM_ERR_INVALID_ARG, "D > K or ldw < K");
+  if (R == 0 || K == 0) return NM_OK;
+  if (!W_out || (D > 0 && (!values || !offsets))) return fail(NM_ERR_INVALID_ARG, "null pointer");
+  nm_status st = require_device();
+  if (st != NM_OK) return st;
+  cudaError_t e = launch_diag_expand(values, offsets, D, R, K, W_out, ldw, stream);
+  return e == cudaSuccess ? NM_OK : cuda_fail(e, "diagonal expand launch");
+}
+
+static nm_status run_diag_spmm(const uint16_t* values, const int32_t* offsets, int64_t D, int64_t R, int64_t K,
+                               const int32_t* idx, const uint16_t* X, int64_t ldx, int64_t T, void* Y, int64_t ldy,
+                               nm_out_dtype dtype, cudaStream_t stream) {
+  t_last_error.clear();
+  if (R < 0 || K < 0 || D < 0 || T < 0) return fail(NM_ERR_INVALID_ARG, "negative dimension");
+  if (D > K) return fail(NM_ERR_INVALID_ARG, "D > K");
+  if (dtype != NM_OUT_BF16 && dtype != NM_OUT_F32) return fail(NM_ERR_INVALID_ARG, "bad output dtype");
+  if (R == 0 || T == 0) return NM_OK;
+  if (!Y) return fail(NM_ERR_INVALID_ARG, "Y is null");
+  if (ldy < T) return fail(NM_ERR_INVALID_ARG, "ldy < T");
+  const int esize = dtype == NM_OUT_F32 ? 4 : 2;
+  if (!al16(Y) || (ldy * esize) % 16 != 0) return fail(NM_ERR_MISALIGNED, "Y rows must be 16-byte aligned");
+  if (R >= (1ll << 31) || K >= (1ll << 31) || T >= (1ll << 31))
+    return fail(NM_ERR_UNSUPPORTED, "dimensions must stay below 2^31");
+  nm_status st = require_device();
+  if (st != NM_OK) return st;
+  if (K == 0 || D == 0) {
+    cudaError_t e = launch_fill_zero(Y, R, T, ldy, esize, stream);
+    return e == cudaSuccess ? NM_OK : cuda_fail(e, "zero fill");
+  }
+  if (!values || !offsets || !X) return fail(NM_ERR_INVALID_ARG, "null operand");
+  if (ldx < T) return fail(NM_ERR_INVALID_ARG, "ldx < T");
+  if (!al16(X) || ldx % 8 != 0) return fail(NM_ERR_MISALIGNED, "X rows must be 16-byte aligned");
+  cudaMemPool_t pool = nullptr;
+  cudaError_t e = staging_pool(&pool);
+  if (e != cudaSuccess) return cuda_fail(e, "staging pool");
+  const int64_t ldk = (K + 7) / 8 * 8;
+  void* wd = nullptr;
+  void* xp = nullptr;
+  e = cudaMallocFromPoolAsync(&wd, (size_t)(R * ldk * 2), pool, stream);
+  if (e != cudaSuccess) return cuda_fail(e, "staging buffer for the dense diagonal operand");
+  e = launch_diag_expand(values, offsets, D, R, K, static_cast<uint16_t*>(wd), ldk, stream);
+  const uint16_t* xsrc = X;
+  int64_t ldsrc = ldx;
+  if (e == cudaSuccess && idx) {
+    const int64_t ldp = (T + 7) / 8 * 8;
+    e = cudaMallocFromPoolAsync(&xp, (size_t)(K * ldp * 2), pool, stream);
+    if (e == cudaSuccess) e = launch_gather_rows(X, ldx, idx, K, T, static_cast<uint16_t*>(xp), ldp, stream);
+    xsrc = static_cast<const uint16_t*>(xp);
+    ldsrc = ldp;
+  }
+  DenseParams p;
+  std::memset(&p, 0, sizeof p);
+  p.M = R;
+  p.N = T;
+  p.Kr = K;
+  p.k_tiles = (K + 127) / 128;
+  p.tiles_m = (int)((R + 255) / 256);
+  p.tiles_n = (int)((T + 255) / 256);
+  p.num_tiles = p.tiles_m * p.tiles_n;
+  p.status = status_word_ptr();
+  p.out = Y;
+  p.ldo = ldy;
+  p.out_f32 = dtype == NM_OUT_F32;
+  if (e == cudaSuccess && !p.status) e = cudaErrorInvalidSymbol;
+  if ((int64_t)p.tiles_m * p.tiles_n >= (1ll << 31)) st = fail(NM_ERR_UNSUPPORTED, "too many tiles");
+  if (e == cudaSuccess && st == NM_OK)
+    st = make_tmap(&p.tm_a, wd, (uint64_t)K, (uint64_t)R, (uint64_t)ldk * 2, 64, 64, 128, "diagonal operand (dense)");
+  if (e == cudaSuccess && st == NM_OK)
+    st = make_tmap(&p.tm_b, xsrc, (uint64_t)T, (uint64_t)K, (uint64_t)ldsrc * 2, 64, 64, 128, "X");
+  if (e == cudaSuccess && st == NM_OK) e = launch_dense_pair(p, false, true, EPI_STORE, stream);
+  cudaFreeAsync(wd, stream);
+  if (xp) cudaFreeAsync(xp, stream);
+  if (st != NM_OK) return st;
+  return e == cudaSuccess ? NM_OK : cuda_fail(e, "diagonal GEMM launch");
+}
+
 }  // namespace nmk
 
 using namespace nmk;
@@ -1171,6 +1277,22 @@ nm_status nm_decompress_i8(const int8_t* values, const uint32_t* meta, int64_t R
 nm_status nm_spmm_i8(const int8_t* values, const uint32_t* meta, int64_t R, int64_t K, const int8_t* X, int64_t ldx,
                      int64_t T, int32_t* Y, int64_t ldy, void* stream) {
   return run_spmm_i8(values, meta, R, K, X, ldx, T, Y, ldy, static_cast<cudaStream_t>(stream));
+}
+
+nm_status nm_diag_prune_compress(const uint16_t* W, int64_t R, int64_t K, int64_t ldw, int64_t D, int32_t* offsets,
+                                 uint16_t* values, void* stream) {
+  return run_diag_prune_compress(W, R, K, ldw, D, offsets, values, static_cast<cudaStream_t>(stream));
+}
+
+nm_status nm_diag_expand(const uint16_t* values, const int32_t* offsets, int64_t D, int64_t R, int64_t K,
+                         uint16_t* W_out, int64_t ldw, void* stream) {
+  return run_diag_expand(values, offsets, D, R, K, W_out, ldw, static_cast<cudaStream_t>(stream));
+}
+
+nm_status nm_diag_spmm(const uint16_t* values, const int32_t* offsets, int64_t D, int64_t R, int64_t K,
+                       const int32_t* idx, const uint16_t* X, int64_t ldx, int64_t T, void* Y, int64_t ldy,
+                       nm_out_dtype dtype, void* stream) {
+  return run_diag_spmm(values, offsets, D, R, K, idx, X, ldx, T, Y, ldy, dtype, static_cast<cudaStream_t>(stream));
 }
 
 nm_status nm_device_status(void* stream) {

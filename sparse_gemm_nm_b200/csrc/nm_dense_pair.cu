@@ -352,6 +352,7 @@ cudaError_t launch_dense_pair(const DenseParams& p, bool a_mn, bool b_mn, int ep
   if (p.num_tiles <= 0) return cudaSuccess;
   if (a_mn && b_mn && epi == EPI_STORE) return launch_dp<true, true, EPI_STORE>(p, stream);
   if (!a_mn && !b_mn && epi == EPI_SURVIVORS) return launch_dp<false, false, EPI_SURVIVORS>(p, stream);
+  if (!a_mn && b_mn && epi == EPI_STORE) return launch_dp<false, true, EPI_STORE>(p, stream);
   return cudaErrorInvalidValue;
 }
 

@@ -1,0 +1,91 @@
+"""GPU diagonal sparsity (selection, gather, dense copy, GEMM) against the oracle."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import sparse_gemm_nm_b200 as nm
+import workloads as wl
+from gpu_helpers import DEV, assert_gemm_close, bf16_rne_of, bits, to_dev, to_dev_i32, values_f64
+
+pytestmark = pytest.mark.gpu
+
+
+def padded(X):
+    K, T = X.shape
+    buf = np.zeros((K, (T + 7) // 8 * 8), np.uint16)
+    buf[:, :T] = X
+    return to_dev(buf)[:, :T]
+
+
+@pytest.mark.parametrize("R,K,D", [(64, 64, 7), (300, 128, 13), (128, 300, 30), (3072, 768, 77), (768, 3072, 307)])
+def test_selection_and_values_match_oracle(R, K, D):
+    W = wl.normal_bf16((R, K), 0.02, seed=R + K + D)
+    offs, V = nm.diag_prune_compress(to_dev(W), D)
+    torch.cuda.synchronize()
+    oo = oracle.diag_select(W, D)
+    assert np.array_equal(offs.cpu().numpy(), oo)
+    assert np.array_equal(bits(V), oracle.diag_compress(W, oo))
+    Wd = torch.empty((R, K), dtype=torch.bfloat16, device=DEV)
+    nm.nm_diag_expand(V, offs, D, R, K, Wd, K)
+    torch.cuda.synchronize()
+    assert np.array_equal(bits(Wd), oracle.diag_expand(oracle.diag_compress(W, oo), oo, K))
+
+
+def test_selection_ties_and_nan():
+    W = wl.bf16_bits(np.ones((40, 24), np.float32))  # all diagonals tie
+    offs, _ = nm.diag_prune_compress(to_dev(W), 5)
+    torch.cuda.synchronize()
+    assert np.array_equal(offs.cpu().numpy(), np.arange(5))
+    W[3, (3 + 17) % 24] = 0x7FC0
+    offs, _ = nm.diag_prune_compress(to_dev(W), 1)
+    torch.cuda.synchronize()
+    assert offs.cpu().numpy().tolist() == [17]
+
+
+@pytest.mark.parametrize("R,K,D,T", [(300, 128, 13, 264), (128, 300, 30, 100), (256, 512, 51, 256), (64, 64, 64, 8)])
+@pytest.mark.parametrize("permuted", [False, True])
+def test_diag_spmm_matches_oracle(R, K, D, T, permuted):
+    W = wl.normal_bf16((R, K), 0.02, seed=R * 3 + K)
+    X = wl.normal_bf16((K, T), 1.0, seed=T + 1)
+    idx = wl.permutation(K, R + 2) if permuted else None
+    offs, V = nm.diag_prune_compress(to_dev(W), D)
+    Y = nm.diag_spmm(V, offs, K, padded(X), idx=None if idx is None else to_dev_i32(idx))
+    torch.cuda.synchronize()
+    nm.nm_device_status()
+    oo = oracle.diag_select(W, D)
+    ref, mag = oracle.diag_spmm(oracle.diag_compress(W, oo), oo, K, X, idx, with_abs=True)
+    assert_gemm_close(values_f64(Y), ref, mag, f"diag {R}x{K} D={D} T={T} permuted={permuted}")
+
+
+@pytest.mark.parametrize("out", [torch.bfloat16, torch.float32])
+def test_diag_spmm_integer_exact(out):
+    R, K, D, T = 384, 512, 64, 256
+    W = wl.integer_bf16((R, K), -8, 8, seed=401)
+    X = wl.integer_bf16((K, T), -8, 8, seed=402)
+    offs, V = nm.diag_prune_compress(to_dev(W), D)
+    Y = nm.diag_spmm(V, offs, K, to_dev(X), out_dtype=out)
+    torch.cuda.synchronize()
+    oo = oracle.diag_select(W, D)
+    ref = oracle.diag_spmm(oracle.diag_compress(W, oo), oo, K, X)
+    if out == torch.float32:
+        assert np.array_equal(Y.contiguous().cpu().numpy().astype(np.float64), ref)
+    else:
+        assert np.array_equal(bits(Y), bf16_rne_of(ref))
+
+
+def test_vit_size_sampled():
+    R, K, D, T = 3072, 768, 77, 197 * 256  # 90 % sparse ViT-B linear, 197 tokens x 256 images
+    W = wl.normal_bf16((R, K), 0.02, seed=411)
+    X = wl.normal_bf16((K, T), 1.0, seed=412)
+    idx = wl.permutation(K, 413)
+    offs, V = nm.diag_prune_compress(to_dev(W), D)
+    Y = nm.diag_spmm(V, offs, K, to_dev(X), idx=to_dev_i32(idx))
+    torch.cuda.synchronize()
+    nm.nm_device_status()
+    oo = oracle.diag_select(W, D)
+    assert np.array_equal(offs.cpu().numpy(), oo)
+    cols = np.array([0, 1, 999, 30000, T - 1])
+    ref, mag = oracle.diag_spmm(oracle.diag_compress(W, oo), oo, K, np.ascontiguousarray(X[:, cols]), idx,
+                                with_abs=True)
+    assert_gemm_close(values_f64(Y)[:, cols], ref, mag, "diag ViT sampled")
