@@ -275,10 +275,12 @@ NM_API nm_status nm_spmm_i8(const int8_t* values, const uint32_t* meta, int64_t 
  * and values V (D x R bf16), V[d][r] = W[r][(r + o_d) mod K].
  *
  * nm_diag_prune_compress: keep the D diagonals of largest score
- *   s(o) = sum_r |W[r][(r + o) mod K]| (fp32, summed in ascending r; NaN
- *   ranks above every number; ties to the lower offset); writes offsets[D]
- *   and values (D x R).  Stages K*5 bytes from the library's pool; four
- *   launches (scores, ranks, placement, gather).
+ *   s(o) = sum_r |W[r][(r + o) mod K]| (fp32 in a fixed order: 32-row chunk
+ *   sums with r ascending, then the chunk sums in ascending order; NaN ranks
+ *   above every number; ties to the lower offset); writes offsets[D] and
+ *   values (D x R).  Stages ceil(R/32)*K*4 + K*8 bytes from the library's
+ *   pool; a memset and five launches (partial sums, scores, ranks,
+ *   placement, gather).
  * nm_diag_expand: the dense R x K copy (+0 off the kept diagonals), row
  *   stride ldw >= K; offsets outside [0, K) place nothing.
  * nm_diag_spmm: y[r][t] = sum_d V[d][r] * X[idx[(r + o_d) mod K]][t]

@@ -73,8 +73,9 @@
  *    {(r, (r + o) mod K)}, one entry per row (wrapping); a diagonally sparse
  *    weight keeps D distinct offsets (ascending) and stores V[d][r] =
  *    W[r][(r + o_d) mod K] (D x R); one-shot selection keeps the D diagonals
- *    of largest score s(o) = sum_r |W[r][(r + o) mod K]| (an fp32 sum in
- *    ascending r, NaN above every number), ties to the lower offset;
+ *    of largest score s(o) = sum_r |W[r][(r + o) mod K]| (fp32: 32-row chunk
+ *    sums in ascending r, then the chunk sums in ascending order; NaN above
+ *    every number), ties to the lower offset;
  *  - backward: dX is the adjoint of that gather (row k of W'^T dY is added to
  *    row idx[k] of dX; entries outside [0, K) drop their row, repeated
  *    entries add up), and the gradient of the stored values is
@@ -578,14 +579,21 @@ int oracle_spmm_i8(const int8_t *values, const uint32_t *meta, int n, int m, int
 /* ------------------------------------------------------------------ */
 /* Diagonal sparsity [DIAG] (readings in the header).                   */
 /* ------------------------------------------------------------------ */
-/* s(o) = sum_r |W[r][(r + o) mod K]| in float32, r ascending. */
+/* s(o) = sum_r |W[r][(r + o) mod K]| in float32, in a fixed order: the rows
+ * in chunks of 32, each chunk summed in ascending r, then the chunk sums in
+ * ascending chunk order. */
 int oracle_diag_scores(const uint16_t *W, int64_t R, int64_t K, int64_t ldw, float *scores)
 {
     if (K <= 0 || ldw < K) return 1;
     for (int64_t o = 0; o < K; o++) {
-        float acc = 0.0f;
-        for (int64_t r = 0; r < R; r++) acc += (float)fabs(bf16_value(W[r * ldw + (r + o) % K]));
-        scores[o] = acc;
+        float total = 0.0f;
+        for (int64_t c = 0; c * 32 < R; c++) {
+            float part = 0.0f;
+            for (int64_t r = 32 * c; r < R && r < 32 * c + 32; r++)
+                part += (float)fabs(bf16_value(W[r * ldw + (r + o) % K]));
+            total += part;
+        }
+        scores[o] = total;
     }
     return 0;
 }

@@ -1032,11 +1032,13 @@ static nm_status run_diag_prune_compress(const uint16_t* W, int64_t R, int64_t K
   cudaError_t e = staging_pool(&pool);
   if (e != cudaSuccess) return cuda_fail(e, "staging pool");
   void* buf = nullptr;
+  const size_t pbytes = (size_t)(((R + 31) / 32 * K * 4 + 255) / 256 * 256);
   const size_t sbytes = (size_t)((K * 4 + 255) / 256 * 256);
-  e = cudaMallocFromPoolAsync(&buf, sbytes + (size_t)K, pool, stream);
+  e = cudaMallocFromPoolAsync(&buf, pbytes + sbytes + (size_t)K * 4, pool, stream);
   if (e != cudaSuccess) return cuda_fail(e, "staging buffer for the diagonal scores");
-  e = launch_diag_select(W, R, K, ldw, D, static_cast<float*>(buf), static_cast<uint8_t*>(buf) + sbytes, offsets,
-                         values, stream);
+  uint8_t* b8 = static_cast<uint8_t*>(buf);
+  e = launch_diag_select(W, R, K, ldw, D, reinterpret_cast<float*>(b8), reinterpret_cast<float*>(b8 + pbytes),
+                         b8 + pbytes + sbytes, offsets, values, stream);
   cudaFreeAsync(buf, stream);
   return e == cudaSuccess ? NM_OK : cuda_fail(e, "diagonal selection launch");
 }

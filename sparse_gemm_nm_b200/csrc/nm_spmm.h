@@ -88,8 +88,8 @@ struct DenseParams {
 enum DenseEpi : int { EPI_STORE = 0, EPI_SURVIVORS = 1 };
 cudaError_t launch_dense_pair(const DenseParams& p, bool a_mn, bool b_mn, int epi, cudaStream_t stream);
 cudaError_t launch_dense_pair_i8(const DenseParams& p, cudaStream_t stream);
-cudaError_t launch_diag_select(const uint16_t* W, int64_t R, int64_t K, int64_t ldw, int64_t D, float* scores,
-                               uint8_t* keep, int32_t* offsets, uint16_t* values, cudaStream_t s);
+cudaError_t launch_diag_select(const uint16_t* W, int64_t R, int64_t K, int64_t ldw, int64_t D, float* part,
+                               float* scores, uint8_t* keep, int32_t* offsets, uint16_t* values, cudaStream_t s);
 cudaError_t launch_diag_expand(const uint16_t* V, const int32_t* offsets, int64_t D, int64_t R, int64_t K,
                                uint16_t* W_out, int64_t ldw, cudaStream_t s);
 cudaError_t launch_compress_i8(const int8_t* W, int64_t R, int64_t K, int64_t ldw, int8_t* values, uint32_t* meta,
