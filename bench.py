@@ -54,6 +54,9 @@ def parse_args(argv=None):
     ap.add_argument("--algo", choices=["auto", "sparse", "dense"], default="auto",
                     help="kernel design for 1:4 / 1:8 (nm_spmm_algo)")
     ap.add_argument("--plain", action="store_true", help="ignore the workload's index map (y = W x)")
+    ap.add_argument("--diag", action="store_true",
+                    help="diagonal pattern at 90 %% sparsity (D = K/10 kept diagonals) on the workload's shapes: "
+                         "nm_diag_prune_compress, then nm_diag_spmm with the index map, per layer")
     ap.add_argument("--dtype", choices=["bf16", "i8"], default="bf16",
                     help="i8: INT8 2:4 weights and int8 inputs on the workload's shapes (nm_prune_compress_i8, then "
                          "nm_spmm_i8; no index map), useful TOP/s against the int8 dense peak")
@@ -747,6 +750,107 @@ def run_i8(args, rank: int, world: int, dist):
         print(json.dumps(line))
 
 
+def run_diag(args, rank: int, world: int, dist):
+    """Diagonal-pattern step: per layer nm_diag_prune_compress (D = K/10) then nm_diag_spmm with the index map."""
+    import torch
+    import sparse_gemm_nm_b200 as nm
+
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    stream = torch.cuda.current_stream(dev)
+    sp = stream.cuda_stream
+    L_ = nm.lib()
+    layers = wl.workload(args.workload)
+    if args.layers:
+        layers = [layers[int(i)] for i in args.layers.split(",")]
+    up = lambda bits: torch.from_numpy(bits.view(np.int16)).to(dev).view(torch.bfloat16)
+    bufs = []
+    for i, L in enumerate(layers):
+        d = wl.make_layer(L)
+        D = max(1, round(L.K / 10))
+        T8 = (L.T + 7) // 8 * 8
+        Xb = np.zeros((L.K, T8), np.uint16)
+        Xb[:, :L.T] = d.X
+        idx = d.idx if d.idx is not None else wl.permutation(L.K, 100 + i)
+        b = {"L": L, "D": D, "W": up(d.W), "X": up(Xb), "ldx": T8, "idx": torch.from_numpy(idx).to(dev),
+             "offs": torch.empty((D,), dtype=torch.int32, device=dev),
+             "V": torch.empty((D, L.R), dtype=torch.bfloat16, device=dev),
+             "Y": torch.empty((L.R, T8), dtype=torch.bfloat16, device=dev)}
+        b["flops"] = 2.0 * L.R * D * L.T  # useful: kept entries only
+        bufs.append(b)
+    torch.cuda.synchronize()
+
+    def check(st, what):
+        if st != 0:
+            raise RuntimeError(f"{what}: {L_.nm_last_error().decode()}")
+
+    def select(b):
+        L = b["L"]
+        check(L_.nm_diag_prune_compress(b["W"].data_ptr(), L.R, L.K, L.K, b["D"], b["offs"].data_ptr(),
+                                        b["V"].data_ptr(), sp), "nm_diag_prune_compress")
+
+    def gemm(b):
+        L = b["L"]
+        check(L_.nm_diag_spmm(b["V"].data_ptr(), b["offs"].data_ptr(), b["D"], L.R, L.K, b["idx"].data_ptr(),
+                              b["X"].data_ptr(), b["ldx"], L.T, b["Y"].data_ptr(), b["ldx"], 0, sp), "nm_diag_spmm")
+
+    def step():
+        for b in bufs:
+            select(b)
+            gemm(b)
+
+    def timed(fn, reps):
+        rank_barrier(dist)
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(reps):
+            fn()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        rank_barrier(dist)
+        return max_over_ranks_on(e0.elapsed_time(e1), dist, dev) / reps
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    props = torch.cuda.get_device_properties(dev)
+    sampler = None if args.quick else ClockSampler(f"GPU-{props.uuid}" if getattr(props, "uuid", None) else "")
+    if sampler:
+        sampler.start()
+    launches0 = nm.nm_launch_count()
+    ms_per_step = timed(step, args.steps)
+    launches = nm.nm_launch_count() - launches0
+    gemm_ms = timed(lambda: [gemm(b) for b in bufs], max(10, min(args.steps, 200)))
+    if sampler:
+        sampler.stop()
+    nm.nm_device_status(sp)
+    peaks, peak_src = load_peaks()
+    useful = sum(b["flops"] for b in bufs)
+    dense = sum(2.0 * b["L"].R * b["L"].K * b["L"].T for b in bufs)
+    line = {"metric": METRIC, "value": world * useful / (ms_per_step * 1e-3) / 1e12, "unit": "TFLOP/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded numpy PCG64 draws rounded to bf16; the workload's shapes)",
+            "config": {"workload": args.workload + " (diagonal, 90 % sparse)",
+                       "shapes": [[b["L"].R, b["L"].K] for b in bufs], "T": [b["L"].T for b in bufs],
+                       "kept_diagonals": [b["D"] for b in bufs], "permuted": True,
+                       "step": "nm_diag_prune_compress, then nm_diag_spmm with the index map, per layer",
+                       "parallelism": f"replicas x{world}"},
+            "roofline": {"bound": "tensor", "achieved": dense / (gemm_ms * 1e-3) / 1e12,
+                         "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                         "frac": dense / (gemm_ms * 1e-3) / 1e12 / peaks["bf16_tflops"], "traffic": None,
+                         "kernel": "nm_diag_spmm calls: dense copy + gather pass + dense_pair_kernel",
+                         "peak_source": f"{peak_src} bf16 burst dense peak; executed dense FLOPs 2 R K T (the "
+                                        "useful ones, 2 R D T, are what `value` counts)",
+                         "useful_tflops_in_gemm": useful / (gemm_ms * 1e-3) / 1e12,
+                         "timing": "CUDA events around back-to-back repetitions of the step's GEMM calls"},
+            "gpu_launches": launches, "clocks": sampler.summary() if sampler else None, "cpu_baseline": None}
+    if rank == 0:
+        print(json.dumps(line))
+
+
 def main(argv=None):
     args = parse_args(argv)
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -764,7 +868,7 @@ def main(argv=None):
         tdist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
         dist = tdist
     try:
-        (run_i8 if args.dtype == "i8" else run_ours)(args, rank, world, dist)
+        (run_i8 if args.dtype == "i8" else run_diag if args.diag else run_ours)(args, rank, world, dist)
     finally:
         if dist is not None:
             dist.destroy_process_group()
