@@ -421,6 +421,24 @@ def run_ours(args, rank: int, world: int, dist):
     torch.cuda.synchronize()
     barrier()
     gemm_only_ms = max_over_ranks(g0.elapsed_time(g1)) / greps
+
+    # Fourth pass, for `compress_roofline`: the step's compress calls (nm_prune_compress) alone, back to back.
+    def compress_only():
+        for b in bufs:
+            launch_compress(b)
+
+    for _ in range(2):
+        compress_only()
+    torch.cuda.synchronize()
+    barrier()
+    c0, c1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    c0.record(stream)
+    for _ in range(greps):
+        compress_only()
+    c1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    compress_only_ms = max_over_ranks(c0.elapsed_time(c1)) / greps
     if sampler:
         sampler.stop()
     nm.nm_device_status(sp)
@@ -517,11 +535,19 @@ def run_ours(args, rank: int, world: int, dist):
                b["W"].numel() * 2 + b["X"].numel() * 2 + b["Y"].numel() * 2 for b in bufs) > 126e6
            else "working set below L2 size (small config)",
            "parallelism": f"replicas x{world}"}
+    comp_bytes_all = sum(b["comp_bytes"] for b in bufs)
+    comp_gbs = comp_bytes_all / (compress_only_ms * 1e-3) / 1e9
+    compress_roofline = {"bound": "hbm", "achieved": comp_gbs, "peak": hbm_peak, "unit": "GB/s",
+                         "frac": comp_gbs / hbm_peak, "kernel": "nm_prune_compress on the step's weights",
+                         "algorithmic_per_launch": [b["comp_bytes"] for b in bufs],
+                         "timing": f"CUDA events around {greps} back-to-back repetitions of the step's compress calls",
+                         "compress_step_us": 1e3 * compress_only_ms}
     line = {"metric": METRIC, "value": world * useful / (ms_per_step * 1e-3) / 1e12, "unit": "TFLOP/s",
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic (seeded numpy PCG64 draws rounded to bf16; shapes and distributions of the workload)",
-            "config": cfg, "roofline": roofline, "kernels": kernels, "gpu_launches": launches,
+            "config": cfg, "roofline": roofline, "compress_roofline": compress_roofline, "kernels": kernels,
+            "gpu_launches": launches,
             "clocks": sampler.summary() if sampler else None}
 
     if not args.quick and any(b["idx"] is not None for b in bufs) and all(b["tmap"] is None for b in bufs):
