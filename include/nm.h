@@ -282,12 +282,19 @@ NM_API nm_status nm_spmm_i8(const int8_t* values, const uint32_t* meta, int64_t 
  *   pool; a memset and five launches (partial sums, scores, ranks,
  *   placement, gather).
  * nm_diag_expand: the dense R x K copy (+0 off the kept diagonals), row
- *   stride ldw >= K; offsets outside [0, K) place nothing.
+ *   stride ldw >= K (columns K..ldw-1 are not written); offsets outside
+ *   [0, K) place nothing.  Every element is written once, by lookup in a
+ *   K-entry table staged from the library's pool (K*4 bytes).
  * nm_diag_spmm: y[r][t] = sum_d V[d][r] * X[idx[(r + o_d) mod K]][t]
  *   (X[k] when idx is NULL; idx entries outside [0, K) read zero rows).
  *   Offsets must be distinct.  The operand is expanded into a staged dense
  *   copy (R x ceil8(K) bf16) and multiplied by a dense tcgen05 GEMM on SM
- *   pairs; with idx one gather pass stages X[idx] first.  X, Y as nm_spmm.
+ *   pairs.  With idx the device checks whether idx is a permutation of
+ *   [0, K): if so, the copy's columns are placed through idx (column idx[k]
+ *   holds the entries of column k) and the GEMM reads X itself; otherwise a
+ *   gather pass stages X[idx] and the GEMM reads that.  Staging: the copy,
+ *   (3K+1)*4 bytes of tables, and K x ceil8(T) bf16 for the gather (reserved
+ *   in both cases).  X, Y as nm_spmm.
  * Errors: NM_ERR_INVALID_ARG (D > K, ld too small, null), NM_ERR_MISALIGNED,
  *   NM_ERR_UNSUPPORTED, NM_ERR_CUDA.
  */

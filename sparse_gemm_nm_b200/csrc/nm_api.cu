@@ -1026,6 +1026,7 @@ static nm_status run_diag_prune_compress(const uint16_t* W, int64_t R, int64_t K
   if (K == 0 || D == 0) return NM_OK;
   if (!W || !offsets || (R > 0 && !values)) return fail(NM_ERR_INVALID_ARG, "null pointer");
   if (R >= (1ll << 31) || K >= (1ll << 31)) return fail(NM_ERR_UNSUPPORTED, "matrix too large for one call");
+  if (K > 65535ll * 256) return fail(NM_ERR_UNSUPPORTED, "K > 16776960 (the rank grid's offset tiles)");
   nm_status st = require_device();
   if (st != NM_OK) return st;
   cudaMemPool_t pool = nullptr;
@@ -1050,9 +1051,21 @@ static nm_status run_diag_expand(const uint16_t* values, const int32_t* offsets,
   if (D > K || ldw < K) return fail(NM_ERR_INVALID_ARG, "D > K or ldw < K");
   if (R == 0 || K == 0) return NM_OK;
   if (!W_out || (D > 0 && (!values || !offsets))) return fail(NM_ERR_INVALID_ARG, "null pointer");
+  if (R >= (1ll << 31) || K >= (1ll << 31)) return fail(NM_ERR_UNSUPPORTED, "matrix too large for one call");
   nm_status st = require_device();
   if (st != NM_OK) return st;
-  cudaError_t e = launch_diag_expand(values, offsets, D, R, K, W_out, ldw, stream);
+  if (D == 0) {
+    cudaError_t e = launch_fill_zero(W_out, R, K, ldw, 2, stream);
+    return e == cudaSuccess ? NM_OK : cuda_fail(e, "zero fill");
+  }
+  cudaMemPool_t pool = nullptr;
+  cudaError_t e = staging_pool(&pool);
+  if (e != cudaSuccess) return cuda_fail(e, "staging pool");
+  void* tables = nullptr;
+  e = cudaMallocFromPoolAsync(&tables, (size_t)diag_table_words(K, false) * 4, pool, stream);
+  if (e != cudaSuccess) return cuda_fail(e, "staging buffer for the diagonal table");
+  e = launch_diag_dense(values, offsets, D, R, K, nullptr, static_cast<int32_t*>(tables), W_out, ldw, stream, nullptr);
+  cudaFreeAsync(tables, stream);
   return e == cudaSuccess ? NM_OK : cuda_fail(e, "diagonal expand launch");
 }
 
@@ -1082,18 +1095,26 @@ static nm_status run_diag_spmm(const uint16_t* values, const int32_t* offsets, i
   cudaMemPool_t pool = nullptr;
   cudaError_t e = staging_pool(&pool);
   if (e != cudaSuccess) return cuda_fail(e, "staging pool");
+  // Staging: the dense copy (R x ceil8(K)) with its lookup tables, and with idx
+  // a gathered X[idx] that the gather pass fills only when idx is not a
+  // permutation (otherwise the copy's columns are placed through idx and the
+  // GEMM reads X itself; the device-side check decides at run time).
   const int64_t ldk = (K + 7) / 8 * 8;
+  const size_t wbytes = (size_t)((R * ldk * 2 + 255) / 256 * 256);
   void* wd = nullptr;
   void* xp = nullptr;
-  e = cudaMallocFromPoolAsync(&wd, (size_t)(R * ldk * 2), pool, stream);
+  e = cudaMallocFromPoolAsync(&wd, wbytes + (size_t)diag_table_words(K, idx != nullptr) * 4, pool, stream);
   if (e != cudaSuccess) return cuda_fail(e, "staging buffer for the dense diagonal operand");
-  e = launch_diag_expand(values, offsets, D, R, K, static_cast<uint16_t*>(wd), ldk, stream);
+  const uint32_t* is_perm = nullptr;
+  e = launch_diag_dense(values, offsets, D, R, K, idx, reinterpret_cast<int32_t*>(static_cast<uint8_t*>(wd) + wbytes),
+                        static_cast<uint16_t*>(wd), ldk, stream, &is_perm);
   const uint16_t* xsrc = X;
   int64_t ldsrc = ldx;
   if (e == cudaSuccess && idx) {
     const int64_t ldp = (T + 7) / 8 * 8;
     e = cudaMallocFromPoolAsync(&xp, (size_t)(K * ldp * 2), pool, stream);
-    if (e == cudaSuccess) e = launch_gather_rows(X, ldx, idx, K, T, static_cast<uint16_t*>(xp), ldp, stream);
+    if (e == cudaSuccess)
+      e = launch_gather_rows(X, ldx, idx, K, T, static_cast<uint16_t*>(xp), ldp, stream, is_perm);
     xsrc = static_cast<const uint16_t*>(xp);
     ldsrc = ldp;
   }
@@ -1116,6 +1137,10 @@ static nm_status run_diag_spmm(const uint16_t* values, const int32_t* offsets, i
     st = make_tmap(&p.tm_a, wd, (uint64_t)K, (uint64_t)R, (uint64_t)ldk * 2, 64, 64, 128, "diagonal operand (dense)");
   if (e == cudaSuccess && st == NM_OK)
     st = make_tmap(&p.tm_b, xsrc, (uint64_t)T, (uint64_t)K, (uint64_t)ldsrc * 2, 64, 64, 128, "X");
+  if (e == cudaSuccess && st == NM_OK && idx) {
+    st = make_tmap(&p.tm_b_alt, X, (uint64_t)T, (uint64_t)K, (uint64_t)ldx * 2, 64, 64, 128, "X (direct)");
+    p.use_alt = is_perm;
+  }
   if (e == cudaSuccess && st == NM_OK) e = launch_dense_pair(p, false, true, EPI_STORE, stream);
   cudaFreeAsync(wd, stream);
   if (xp) cudaFreeAsync(xp, stream);

@@ -272,6 +272,7 @@ constexpr size_t kGatherSmemCap = 56 * 1024;
 
 __global__ void __launch_bounds__(256) gather_rows_kernel(const GatherJob g) {
   pdl_gate();
+  if (g.skip_if && *reinterpret_cast<const volatile uint32_t*>(g.skip_if)) return;
   const int64_t warp = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) >> 5;
   const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
   gather_rows_items(g, warp, nwarps, threadIdx.x & 31);
@@ -404,7 +405,7 @@ cudaError_t launch_decompress_tiles(const uint16_t* values, const uint32_t* meta
 }
 
 cudaError_t launch_gather_rows(const uint16_t* X, int64_t ldx, const int32_t* idx, int64_t K, int64_t T,
-                               uint16_t* Xp, int64_t ldp, cudaStream_t s) {
+                               uint16_t* Xp, int64_t ldp, cudaStream_t s, const uint32_t* skip_if) {
   const int threads = 256;
   static bool configured[64] = {};
   int dev = 0;
@@ -419,7 +420,7 @@ cudaError_t launch_gather_rows(const uint16_t* X, int64_t ldx, const int32_t* id
   const int64_t want = (items + 7) / 8;  // 8 warps per CTA
   const int64_t cap = (int64_t)sm_count_current() * kGatherCtasPerSm;
   const int grid = (int)(want < cap ? (want > 0 ? want : 1) : cap);
-  const GatherJob g{X, ldx, idx, K, T, Xp, ldp};
+  const GatherJob g{X, ldx, idx, K, T, Xp, ldp, skip_if};
   cudaError_t e = launch_pdl(gather_rows_kernel, grid, threads, kGatherSmemCap, s, g);
   count_launch();
   return e != cudaSuccess ? e : cudaGetLastError();

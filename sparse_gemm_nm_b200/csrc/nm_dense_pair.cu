@@ -102,6 +102,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dpair::kThreads, 1)
   if (warp == 0 && lane == 0) {
     tma_prefetch_desc(&p.tm_a);
     tma_prefetch_desc(&p.tm_b);
+    if (p.use_alt) tma_prefetch_desc(&p.tm_b_alt);
   }
   if (warp == 1) {
     tmem_alloc_pair(tmem_slot, kTmemCols);
@@ -121,6 +122,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dpair::kThreads, 1)
   if (warp == 0) {
     // ------------------------------------------------------------- copies
     if (lane == 0) {
+      const CUtensorMap* tmb =
+          (p.use_alt && *reinterpret_cast<const volatile uint32_t*>(p.use_alt)) ? &p.tm_b_alt : &p.tm_b;
       int s = 0;
       uint32_t ph = 0;
       for (int tile = pair_id; tile < p.num_tiles && ok; tile += npairs) {
@@ -142,7 +145,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dpair::kThreads, 1)
               for (int h = 0; h < 2; ++h)
                 tma_load_2d_pair(a + i * 16384 + h * 8192, &p.tm_a, bar, k0 + 128 * i, m0 + 64 * h);
 #pragma unroll
-            for (int j = 0; j < 4; ++j) tma_load_2d_pair(b + j * 8192, &p.tm_b, bar, n0, k0 + 64 * j);
+            for (int j = 0; j < 4; ++j) tma_load_2d_pair(b + j * 8192, tmb, bar, n0, k0 + 64 * j);
             if (++s == kStages) { s = 0; ph ^= 1u; }
             continue;
           }
@@ -158,9 +161,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dpair::kThreads, 1)
               else
                 tma_load_2d_pair(a + i * 16384 + h * 8192, &p.tm_a, bar, k0 + 64 * i, m0 + 64 * h);
               if (B_MN)
-                tma_load_2d_pair(b + i * 16384 + h * 8192, &p.tm_b, bar, n0 + 64 * i, k0 + 64 * h);
+                tma_load_2d_pair(b + i * 16384 + h * 8192, tmb, bar, n0 + 64 * i, k0 + 64 * h);
               else
-                tma_load_2d_pair(b + i * 16384 + h * 8192, &p.tm_b, bar, k0 + 64 * i, n0 + 64 * h);
+                tma_load_2d_pair(b + i * 16384 + h * 8192, tmb, bar, k0 + 64 * i, n0 + 64 * h);
             }
           }
           if (++s == kStages) { s = 0; ph ^= 1u; }

@@ -44,6 +44,7 @@ struct GatherJob {
   int64_t K, T;
   uint16_t* Xp;
   int64_t ldp;
+  const uint32_t* skip_if;  // gather_rows_kernel does nothing when this word is set and nonzero at run time
 };
 
 #ifdef __CUDACC__
@@ -114,8 +115,10 @@ cudaError_t launch_decompress(const uint16_t* values, const uint32_t* meta, int6
 // (tile map ceil(R/128) x ceil(K/128)); other tiles of W_out are not written.
 cudaError_t launch_decompress_tiles(const uint16_t* values, const uint32_t* meta, int64_t R, int64_t K,
                                     const uint8_t* tile_map, uint16_t* W_out, int64_t ldw, cudaStream_t s);
+// Xp[k] = X[idx[k]] (zero rows for idx outside [0, K)); with skip_if set, the
+// launch does nothing when that device word is nonzero when it runs.
 cudaError_t launch_gather_rows(const uint16_t* X, int64_t ldx, const int32_t* idx, int64_t K, int64_t T,
-                               uint16_t* Xp, int64_t ldp, cudaStream_t s);
+                               uint16_t* Xp, int64_t ldp, cudaStream_t s, const uint32_t* skip_if = nullptr);
 cudaError_t launch_reencode_2of4(const uint16_t* values, const uint32_t* meta, int64_t R, int64_t K, int n, int m,
                                  uint16_t* values2, uint32_t* meta2, cudaStream_t s);
 cudaError_t launch_fill_zero(void* Y, int64_t R, int64_t T, int64_t ldy, int esize, cudaStream_t s);

@@ -71,6 +71,8 @@ struct SpmmParams {
 // M x N weight (meta), as out[m][j] for survivor j of row m.
 struct DenseParams {
   CUtensorMap tm_a, tm_b;
+  CUtensorMap tm_b_alt;     // read instead of tm_b when use_alt is set and *use_alt is nonzero at run time
+  const uint32_t* use_alt;
   int64_t M, N, Kr;
   int64_t k_tiles;
   int tiles_m, tiles_n, num_tiles;
@@ -90,8 +92,16 @@ cudaError_t launch_dense_pair(const DenseParams& p, bool a_mn, bool b_mn, int ep
 cudaError_t launch_dense_pair_i8(const DenseParams& p, cudaStream_t stream);
 cudaError_t launch_diag_select(const uint16_t* W, int64_t R, int64_t K, int64_t ldw, int64_t D, float* part,
                                float* scores, uint8_t* keep, int32_t* offsets, uint16_t* values, cudaStream_t s);
-cudaError_t launch_diag_expand(const uint16_t* V, const int32_t* offsets, int64_t D, int64_t R, int64_t K,
-                               uint16_t* W_out, int64_t ldw, cudaStream_t s);
+// Dense copy of a diagonal operand, columns [0, K) of rows [0, R) of W_out.
+// `tables` is device scratch of diag_table_words(K, idx != nullptr) words.
+// With idx: when idx is a permutation of [0, K) the copy's columns are placed
+// through it (column idx[k] holds what column k would), so that the product
+// with X equals the product of the plain copy with X[idx]; the word returned
+// in *is_perm (inside `tables`) is nonzero exactly then.
+int64_t diag_table_words(int64_t K, bool with_idx);
+cudaError_t launch_diag_dense(const uint16_t* V, const int32_t* offsets, int64_t D, int64_t R, int64_t K,
+                              const int32_t* idx, int32_t* tables, uint16_t* W_out, int64_t ldw, cudaStream_t s,
+                              const uint32_t** is_perm);
 cudaError_t launch_compress_i8(const int8_t* W, int64_t R, int64_t K, int64_t ldw, int8_t* values, uint32_t* meta,
                                cudaStream_t s);
 cudaError_t launch_decompress_i8(const int8_t* values, const uint32_t* meta, int64_t R, int64_t K, int8_t* W_out,

@@ -89,3 +89,54 @@ def test_vit_size_sampled():
     ref, mag = oracle.diag_spmm(oracle.diag_compress(W, oo), oo, K, np.ascontiguousarray(X[:, cols]), idx,
                                 with_abs=True)
     assert_gemm_close(values_f64(Y)[:, cols], ref, mag, "diag ViT sampled")
+
+
+@pytest.mark.parametrize("kind", ["permutation", "repeats", "out_of_range"])
+@pytest.mark.parametrize("out", [torch.bfloat16, torch.float32])
+def test_diag_spmm_index_maps_integer_exact(kind, out):
+    # A permutation takes the route that places the dense copy's columns through idx (the GEMM reads X
+    # itself); any other map takes the gather of X[idx].  Both are exact on small integers.
+    R, K, D, T = 320, 384, 40, 264
+    W = wl.integer_bf16((R, K), -8, 8, seed=421)
+    X = wl.integer_bf16((K, T), -8, 8, seed=422)
+    rng = np.random.default_rng(423)
+    idx = rng.permutation(K).astype(np.int32)
+    if kind == "repeats":
+        idx[[5, 77, 200]] = idx[[6, 6, 300]]
+    elif kind == "out_of_range":
+        idx[[0, 383]] = [-1, K]
+    offs, V = nm.diag_prune_compress(to_dev(W), D)
+    Y = nm.diag_spmm(V, offs, K, padded(X), idx=to_dev_i32(idx), out_dtype=out)
+    torch.cuda.synchronize()
+    nm.nm_device_status()
+    oo = oracle.diag_select(W, D)
+    ref = oracle.diag_spmm(oracle.diag_compress(W, oo), oo, K, X, idx)
+    if out == torch.float32:
+        assert np.array_equal(Y.contiguous().cpu().numpy().astype(np.float64), ref)
+    else:
+        assert np.array_equal(bits(Y), bf16_rne_of(ref))
+
+
+def test_diag_expand_strides_and_foreign_offsets():
+    R, K, D = 70, 45, 6
+    W = wl.normal_bf16((R, K), 1.0, seed=431)
+    oo = np.array([0, 3, 9, 20, 33, 44], np.int32)
+    V = oracle.diag_compress(W, oo)
+    ref = oracle.diag_expand(V, oo, K)
+    for ldw in (K, K + 3, 56):  # rows that are not 16-byte multiples, and ones that are
+        buf = torch.full((R, ldw), 5.0, dtype=torch.bfloat16, device=DEV)
+        nm.nm_diag_expand(to_dev(V), to_dev_i32(oo), D, R, K, buf, ldw)
+        torch.cuda.synchronize()
+        got = bits(buf)
+        assert np.array_equal(got[:, :K], ref)
+        assert np.all(got[:, K:] == bits(torch.tensor([5.0], dtype=torch.bfloat16))[0])  # padding untouched
+    bad = oo.copy()
+    bad[2] = K + 7  # an offset outside [0, K) places nothing
+    buf = torch.full((R, K), 5.0, dtype=torch.bfloat16, device=DEV)
+    nm.nm_diag_expand(to_dev(V), to_dev_i32(bad), D, R, K, buf, K)
+    torch.cuda.synchronize()
+    keep = np.array([0, 1, 3, 4, 5])
+    assert np.array_equal(bits(buf), oracle.diag_expand(V[keep], oo[keep], K))
+    nm.nm_diag_expand(to_dev(V), to_dev_i32(oo), 0, R, K, buf, K)  # D = 0: all zero
+    torch.cuda.synchronize()
+    assert torch.count_nonzero(buf).item() == 0
