@@ -19,6 +19,8 @@ Sources, by page title and passage:
   * "Structured Sparsity" topic cards, PATCH abstract: per-tile dense / 2:4.
   * "M:N sparsity on NVIDIA tensor cores", the formats the sparse tensor cores
     take (INT8 among them) and the INT8 storage arithmetic: the ``*_i8`` functions.
+  * The same passage: for TF32 the block halves to 1:2 -- the ``*_f32`` functions
+    (float32 weights, 1:2 on the TF32 path).
   * SHUFFLESPARSE's contributions (block, N:M and diagonal patterns under one
     permutation) and the DynaDiag abstract: the ``diag_*`` functions (the pages
     give no format; see the readings in nm_oracle.c).
@@ -83,6 +85,10 @@ def _load():
                 "oracle_decompress_i8": ([P, P, I64, I64, I, I, P, I64], I),
                 "oracle_spmm_i8": ([P, P, I, I, I64, I64, P, I64, I64, P, I64], I),
                 "oracle_sddmm": ([P, I, I, I64, I64, P, I64, P, I64, I64, P, P, P], I),
+                "oracle_prune_mask_f32": ([P, I64, I64, I64, I, I, P], I),
+                "oracle_compress_f32": ([P, I64, I64, I64, I, I, P, P], I),
+                "oracle_decompress_f32": ([P, P, I64, I64, I, I, P, I64], I),
+                "oracle_spmm_f32": ([P, P, I, I, I64, I64, P, I64, I64, P, P, I64], I),
             }
             for name, (args, res) in sig.items():
                 fn = getattr(lib, name)
@@ -312,6 +318,58 @@ def spmm_i8(values, meta, K, X, n=2, m=4):
     Y = np.zeros((R, T), np.int64)
     _check(_load().oracle_spmm_i8(_ptr(values), _ptr(meta), n, m, R, K, _ptr(X), T, T, _ptr(Y), T), "spmm_i8")
     return Y
+
+
+def _u32(a):
+    """float32 data as its uint32 bit patterns (float32 or uint32 arrays)."""
+    a = np.ascontiguousarray(a)
+    if a.dtype == np.float32:
+        return a.view(np.uint32)
+    assert a.dtype == np.uint32, "float32 data or its uint32 bits"
+    return a
+
+
+def prune_mask_f32(W, n=1, m=2):
+    """uint8 R x K mask of the N:M survivors of float32 W (TF32 path: 1:2)."""
+    W = _u32(W)
+    R, K = W.shape
+    mask = np.zeros((R, K), np.uint8)
+    _check(_load().oracle_prune_mask_f32(_ptr(W), R, K, K, n, m, _ptr(mask)), "prune_mask_f32")
+    return mask
+
+
+def compress_f32(W, n=1, m=2):
+    """(values R x K*n/m as uint32 float32 bits, meta uint32) of float32 W; same packing as compress()."""
+    W = _u32(W)
+    R, K = W.shape
+    if K % m or not (1 <= n < m) or m not in (2, 4, 8, 16):
+        raise ValueError(f"oracle compress_f32 rejected its arguments (K={K}, {n}:{m})")
+    vals = np.zeros((R, value_cols(K, n, m)), np.uint32)
+    meta = np.zeros(meta_words(R, K, n, m), np.uint32)
+    _check(_load().oracle_compress_f32(_ptr(W), R, K, K, n, m, _ptr(vals), _ptr(meta)), "compress_f32")
+    return vals, meta
+
+
+def decompress_f32(values, meta, K, n=1, m=2):
+    values = _u32(values)
+    meta = np.ascontiguousarray(meta, dtype=np.uint32)
+    R = values.shape[0]
+    out = np.zeros((R, K), np.uint32)
+    _check(_load().oracle_decompress_f32(_ptr(values), _ptr(meta), R, K, n, m, _ptr(out), K), "decompress_f32")
+    return out
+
+
+def spmm_f32(values, meta, K, X, n=1, m=2, with_abs=False):
+    """y = W' X in fp64 for float32 compressed W' and float32 X (K x T); optionally sum |w||x|."""
+    values = _u32(values)
+    meta = np.ascontiguousarray(meta, dtype=np.uint32)
+    X = _u32(X)
+    R, T = values.shape[0], X.shape[1]
+    Y = np.zeros((R, T), np.float64)
+    A = np.zeros((R, T), np.float64) if with_abs else None
+    _check(_load().oracle_spmm_f32(_ptr(values), _ptr(meta), n, m, R, K, _ptr(X), T, T, _ptr(Y), _ptr(A), T),
+           "spmm_f32")
+    return (Y, A) if with_abs else Y
 
 
 def diag_scores(W):

@@ -40,6 +40,8 @@
  *             the sparse tensor cores accept (2:4 for FP16, BF16 and INT8
  *             weights) and the storage paragraphs (a 2-bit index per stored
  *             value: 25 % of an INT8 value, so INT8 2:4 saves 37.5 %).
+ *  [MN-tf32]  "M:N sparsity on NVIDIA tensor cores", the same passage on the
+ *             formats: for TF32 the block halves to 1:2, still 50 percent.
  *  [DIAG]     SHUFFLESPARSE (the technical summary's contributions and the
  *             author page's abstract): one permutation primitive over block,
  *             N:M and diagonal patterns; the DynaDiag abstract on the same
@@ -80,6 +82,9 @@
  *    row idx[k] of dX; entries outside [0, K) drop their row, repeated
  *    entries add up), and the gradient of the stored values is
  *    dV[r][j] = sum_t dY[r][t] * X_perm[k_j][t] for the survivor's column k_j;
+ *  - TF32: 1:2 selection compares the float32 values (the same rules); the
+ *    values and W hold float32 bit patterns (uint32); the oracle's GEMM is
+ *    exact in double and the TF32 device path is held to the GEMM tolerance;
  *  - W (dense, R x K) and the compressed values hold bf16 bit patterns
  *    (uint16); X is K x T row-major; Y is R x T (double here).
  */
@@ -571,6 +576,116 @@ int oracle_spmm_i8(const int8_t *values, const uint32_t *meta, int n, int m, int
                 acc += (int64_t)values[r * vcols + j] * (int64_t)X[k * ldx + t];
             }
             Y[r * ldy + t] = acc;
+        }
+    }
+    return 0;
+}
+
+/* ------------------------------------------------------------------ */
+/* FP32 weights for the TF32 tensor cores [MN-tf32]: the block halves   */
+/* to 1:2 for TF32.  The same selection rule on the float32 value       */
+/* (converted to double exactly; NaN above every number, equal          */
+/* magnitudes to the lower index), the same push-left values (float32   */
+/* bits, copied) and the same metadata packing as bf16.  The GEMM is    */
+/* the exact sum of the exact products of the stored float32 values, in */
+/* double; a device that rounds its inputs to TF32 is held to the GEMM  */
+/* tolerance, not to bit equality.                                      */
+/* ------------------------------------------------------------------ */
+static double f32_value(uint32_t bits)
+{
+    float f;
+    memcpy(&f, &bits, sizeof f);
+    return (double)f;
+}
+
+int oracle_prune_mask_f32(const uint32_t *W, int64_t R, int64_t K, int64_t ldw, int n, int m, uint8_t *mask)
+{
+    if (!pattern_ok(n, m) || K % m != 0 || ldw < K) return 1;
+    for (int64_t r = 0; r < R; r++) {
+        for (int64_t g = 0; g < K / m; g++) {
+            const uint32_t *grp = W + r * ldw + g * m;
+            for (int i = 0; i < m; i++) {
+                int rank = 0;
+                for (int j = 0; j < m; j++)
+                    if (j != i && beats(f32_value(grp[j]), j, f32_value(grp[i]), i)) rank++;
+                mask[r * K + g * m + i] = (uint8_t)(rank < n);
+            }
+        }
+    }
+    return 0;
+}
+
+int oracle_compress_f32(const uint32_t *W, int64_t R, int64_t K, int64_t ldw, int n, int m, uint32_t *values,
+                        uint32_t *meta)
+{
+    if (!pattern_ok(n, m) || K % m != 0 || ldw < K) return 1;
+    int64_t vcols = oracle_value_cols(K, n, m);
+    int64_t mcols = oracle_meta_cols(K, n, m);
+    int b = oracle_index_bits(m);
+    int s = oracle_positions_per_word(m);
+    uint8_t *mask = (uint8_t *)malloc((size_t)(R * K > 0 ? R * K : 1));
+    if (!mask) return 2;
+    oracle_prune_mask_f32(W, R, K, ldw, n, m, mask);
+    int tiled = (n == 2 && m == 4);
+    int64_t words = oracle_meta_words(R, K, n, m);
+    for (int64_t i = 0; i < words; i++) meta[i] = tiled ? 0x44444444u : 0u;
+    for (int64_t r = 0; r < R; r++) {
+        int64_t j = 0;
+        for (int64_t g = 0; g < K / m; g++) {
+            uint32_t nib = 0;
+            int seen = 0;
+            for (int p = 0; p < m; p++) {
+                if (!mask[r * K + g * m + p]) continue;
+                values[r * vcols + j] = W[r * ldw + g * m + p];
+                if (tiled)
+                    nib |= (uint32_t)p << (2 * seen);
+                else
+                    meta[r * mcols + j / s] |= (uint32_t)p << (b * (j % s));
+                seen++;
+                j++;
+            }
+            if (tiled) {
+                int bit;
+                int64_t w = meta_slot_2of4(r, g, K, &bit);
+                meta[w] = (meta[w] & ~(0xFu << bit)) | (nib << bit);
+            }
+        }
+    }
+    free(mask);
+    return 0;
+}
+
+int oracle_decompress_f32(const uint32_t *values, const uint32_t *meta, int64_t R, int64_t K, int n, int m,
+                          uint32_t *W_out, int64_t ldw)
+{
+    if (!pattern_ok(n, m) || K % m != 0 || ldw < K) return 1;
+    int64_t vcols = oracle_value_cols(K, n, m);
+    for (int64_t r = 0; r < R; r++) {
+        for (int64_t k = 0; k < K; k++) W_out[r * ldw + k] = 0u; /* +0.0 */
+        for (int64_t j = 0; j < vcols; j++)
+            W_out[r * ldw + (j / n) * m + position_of(meta, K, r, j, n, m)] = values[r * vcols + j];
+    }
+    return 0;
+}
+
+/* y[r][t] = sum_j V[r][j] * X[k_j][t] (float32 values, double sums);    */
+/* Y_abs (optional) receives sum_j |V[r][j]| |X[k_j][t]|.                */
+int oracle_spmm_f32(const uint32_t *values, const uint32_t *meta, int n, int m, int64_t R, int64_t K,
+                    const uint32_t *X, int64_t ldx, int64_t T, double *Y, double *Y_abs, int64_t ldy)
+{
+    if (!pattern_ok(n, m) || K % m != 0 || ldx < T || ldy < T) return 1;
+    int64_t vcols = oracle_value_cols(K, n, m);
+    for (int64_t r = 0; r < R; r++) {
+        for (int64_t t = 0; t < T; t++) {
+            double acc = 0.0, mag = 0.0;
+            for (int64_t j = 0; j < vcols; j++) {
+                int64_t k = (j / n) * m + position_of(meta, K, r, j, n, m);
+                double w = f32_value(values[r * vcols + j]), x = f32_value(X[k * ldx + t]);
+                acc += w * x;
+                mag += fabs(w) * fabs(x);
+            }
+            Y[r * ldy + t] = acc;
+            if (Y_abs) Y_abs[r * ldy + t] = mag;
         }
     }
     return 0;

@@ -76,6 +76,15 @@ def normal_i8(shape, std: float, seed: int) -> np.ndarray:
     return np.clip(x, -128, 127).astype(np.int8)
 
 
+def normal_f32(shape, std: float, seed: int) -> np.ndarray:
+    return _rng(seed).standard_normal(shape, dtype=np.float32) * np.float32(std)
+
+
+def integer_f32(shape, lo: int, hi: int, seed: int) -> np.ndarray:
+    """Small integers as float32 (exact in TF32 too) drawn uniformly from [lo, hi]."""
+    return _rng(seed).integers(lo, hi + 1, size=shape).astype(np.float32)
+
+
 def permutation(K: int, seed: int) -> np.ndarray:
     return _rng(seed).permutation(K).astype(np.int32)
 
