@@ -57,9 +57,11 @@ def parse_args(argv=None):
     ap.add_argument("--diag", action="store_true",
                     help="diagonal pattern at 90 %% sparsity (D = K/10 kept diagonals) on the workload's shapes: "
                          "nm_diag_prune_compress, then nm_diag_spmm with the index map, per layer")
-    ap.add_argument("--dtype", choices=["bf16", "i8"], default="bf16",
+    ap.add_argument("--dtype", choices=["bf16", "i8", "tf32"], default="bf16",
                     help="i8: INT8 2:4 weights and int8 inputs on the workload's shapes (nm_prune_compress_i8, then "
-                         "nm_spmm_i8; no index map), useful TOP/s against the int8 dense peak")
+                         "nm_spmm_i8; no index map), useful TOP/s against the int8 dense peak; tf32: 1:2 float32 "
+                         "weights and float32 inputs (nm_prune_compress_tf32, then nm_spmm_tf32 with fp32 output), "
+                         "useful TFLOP/s against the tf32 dense peak")
     ap.add_argument("--step", choices=["one-call", "two-calls"], default="one-call",
                     help="one-call: nm_prune_spmm per layer (prune + compress + GEMM in one library call, the "
                          "compressed form written too); two-calls: nm_prune_compress, then the GEMM call.  The "
@@ -780,6 +782,104 @@ def run_i8(args, rank: int, world: int, dist):
         print(json.dumps(line))
 
 
+def run_tf32(args, rank: int, world: int, dist):
+    """TF32 1:2 step on the workload's shapes: per layer nm_prune_compress_tf32 then nm_spmm_tf32 (fp32 out)."""
+    import torch
+    import sparse_gemm_nm_b200 as nm
+
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    stream = torch.cuda.current_stream(dev)
+    sp = stream.cuda_stream
+    L_ = nm.lib()
+    layers = wl.workload(args.workload)
+    if args.layers:
+        layers = [layers[int(i)] for i in args.layers.split(",")]
+    if any(L.K % 2 for L in layers):
+        raise SystemExit("--dtype tf32 needs even K")
+    bufs = []
+    for i, L in enumerate(layers):
+        T4 = (L.T + 3) // 4 * 4
+        Xb = np.zeros((L.K, T4), np.float32)
+        Xb[:, :L.T] = wl.normal_f32((L.K, L.T), 1.0, seed=10 * i + 2)
+        b = {"L": L, "W": torch.from_numpy(wl.normal_f32((L.R, L.K), 0.02, seed=10 * i + 1)).to(dev),
+             "X": torch.from_numpy(Xb).to(dev), "ldx": T4,
+             "vals": torch.empty((L.R, L.K // 2), dtype=torch.float32, device=dev),
+             "meta": torch.empty((nm.nm_meta_words(L.R, L.K, 1, 2),), dtype=torch.int32, device=dev),
+             "Y": torch.empty((L.R, T4), dtype=torch.float32, device=dev)}
+        b["flops"] = 2.0 * L.R * L.T * L.K / 2  # useful: survivors only
+        bufs.append(b)
+    torch.cuda.synchronize()
+
+    def check(st, what):
+        if st != 0:
+            raise RuntimeError(f"{what}: {L_.nm_last_error().decode()}")
+
+    def compress(b):
+        L = b["L"]
+        check(L_.nm_prune_compress_tf32(b["W"].data_ptr(), L.R, L.K, L.K, b["vals"].data_ptr(),
+                                        b["meta"].data_ptr(), sp), "nm_prune_compress_tf32")
+
+    def gemm(b):
+        L = b["L"]
+        check(L_.nm_spmm_tf32(b["vals"].data_ptr(), b["meta"].data_ptr(), L.R, L.K, b["X"].data_ptr(), b["ldx"],
+                              L.T, b["Y"].data_ptr(), b["Y"].shape[1], 1, sp), "nm_spmm_tf32")
+
+    def step():
+        for b in bufs:
+            compress(b)
+            gemm(b)
+
+    def timed(fn, reps):
+        rank_barrier(dist)
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(reps):
+            fn()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        rank_barrier(dist)
+        return max_over_ranks_on(e0.elapsed_time(e1), dist, dev) / reps
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    props = torch.cuda.get_device_properties(dev)
+    sampler = None if args.quick else ClockSampler(f"GPU-{props.uuid}" if getattr(props, "uuid", None) else "")
+    if sampler:
+        sampler.start()
+    launches0 = nm.nm_launch_count()
+    ms_per_step = timed(step, args.steps)
+    launches = nm.nm_launch_count() - launches0
+    gemm_ms = timed(lambda: [gemm(b) for b in bufs], max(10, min(args.steps, 200)))
+    if sampler:
+        sampler.stop()
+    nm.nm_device_status(sp)
+    peaks, peak_src = load_peaks()
+    tf32_peak = 0.5 * peaks["bf16_tflops"]
+    useful = sum(b["flops"] for b in bufs)
+    achieved = useful / (gemm_ms * 1e-3) / 1e12
+    line = {"metric": METRIC, "value": world * useful / (ms_per_step * 1e-3) / 1e12, "unit": "TFLOP/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "tf32",
+            "data": "synthetic float32: W ~ N(0, 0.02^2), X ~ N(0, 1) (seeded PCG64)",
+            "config": {"workload": args.workload + " (TF32 1:2)", "shapes": [[b["L"].R, b["L"].K] for b in bufs],
+                       "T": [b["L"].T for b in bufs],
+                       "step": "nm_prune_compress_tf32, then nm_spmm_tf32 (fp32 out), per layer",
+                       "parallelism": f"replicas x{world}"},
+            "roofline": {"bound": "tensor", "achieved": achieved, "peak": tf32_peak, "unit": "TFLOP/s",
+                         "frac": achieved / tf32_peak, "traffic": None,
+                         "kernel": "nm_spmm_tf32 calls: decompress_1of2_f32_kernel + dense_pair_kernel (kind::tf32)",
+                         "peak_source": f"{peak_src} bf16 burst dense peak x 0.5 (the nominal tf32 / bf16 dense "
+                                        "ratio); useful (survivor) FLOPs, half of the dense ones",
+                         "timing": "CUDA events around back-to-back repetitions of the step's GEMM calls"},
+            "gpu_launches": launches, "clocks": sampler.summary() if sampler else None, "cpu_baseline": None}
+    if rank == 0:
+        print(json.dumps(line))
+
+
 def run_diag(args, rank: int, world: int, dist):
     """Diagonal-pattern step: per layer nm_diag_prune_compress (D = K/10) then nm_diag_spmm with the index map."""
     import torch
@@ -898,7 +998,7 @@ def main(argv=None):
         tdist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
         dist = tdist
     try:
-        (run_i8 if args.dtype == "i8" else run_diag if args.diag else run_ours)(args, rank, world, dist)
+        (run_i8 if args.dtype == "i8" else run_tf32 if args.dtype == "tf32" else run_diag if args.diag else run_ours)(args, rank, world, dist)
     finally:
         if dist is not None:
             dist.destroy_process_group()

@@ -263,6 +263,38 @@ NM_API nm_status nm_decompress_i8(const int8_t* values, const uint32_t* meta, in
 NM_API nm_status nm_spmm_i8(const int8_t* values, const uint32_t* meta, int64_t R, int64_t K, const int8_t* X,
                             int64_t ldx, int64_t T, int32_t* Y, int64_t ldy, void* stream);
 
+/* ----------------------------------------------------------------- TF32 */
+/*
+ * 1:2 sparsity of float32 weights for the TF32 tensor cores.  Source: "M:N
+ * sparsity on NVIDIA tensor cores", the passage on the formats the sparse
+ * tensor cores take (for TF32 the block halves to 1:2, still 50 percent).
+ *
+ * nm_prune_compress_tf32: W float32 R x K (row stride ldw >= K, K even),
+ *   4-byte aligned.  Of each pair (W[r][2p], W[r][2p+1]) the larger
+ *   magnitude survives; equal magnitudes go to the first; a NaN ranks above
+ *   every number (NaNs tie).  values: R x K/2 float32, the survivors' bits.
+ *   meta: R x ceil(K/64) words (nm_meta_words(R, K, 1, 2)); survivor p of a
+ *   row is bit p % 32 of word p / 32: its position in the pair (0 or 1);
+ *   unused bits 0.  One launch.
+ * nm_decompress_tf32: W_out[r][2p + bit] = values[r][p], +0.0 at the other
+ *   position (row stride ldw >= K).
+ * nm_spmm_tf32: Y = W' X, X float32 K x T (row stride ldx >= T, ldx % 4 == 0,
+ *   16-byte aligned), Y R x T bf16 or fp32 (y_dtype) as nm_spmm.  The
+ *   operand is decompressed into a staged dense copy (R x ceil4(K) float32
+ *   from the library's pool) and multiplied by a dense tcgen05 kind::tf32
+ *   GEMM on SM pairs: the tensor cores read W' and X as TF32 (10 explicit
+ *   mantissa bits) and accumulate in fp32, so Y meets the GEMM tolerance
+ *   (|y - y_ref| <= 2^-7 sum |w||x|), not bit equality with an fp32 product.
+ * Errors: NM_ERR_INVALID_ARG (odd K, negative sizes, ld too small, null),
+ *   NM_ERR_MISALIGNED, NM_ERR_UNSUPPORTED (a dimension >= 2^31), NM_ERR_CUDA.
+ */
+NM_API nm_status nm_prune_compress_tf32(const float* W, int64_t R, int64_t K, int64_t ldw, float* values,
+                                        uint32_t* meta, void* stream);
+NM_API nm_status nm_decompress_tf32(const float* values, const uint32_t* meta, int64_t R, int64_t K, float* W_out,
+                                    int64_t ldw, void* stream);
+NM_API nm_status nm_spmm_tf32(const float* values, const uint32_t* meta, int64_t R, int64_t K, const float* X,
+                              int64_t ldx, int64_t T, void* Y, int64_t ldy, nm_out_dtype y_dtype, void* stream);
+
 /* ------------------------------------------------------------- diagonal */
 /*
  * Diagonal sparsity under the index map.  Source: the SHUFFLESPARSE technical

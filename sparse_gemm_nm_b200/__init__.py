@@ -57,6 +57,9 @@ SIGNATURES = {
     "nm_diag_spmm": ([_P, _P, _I64, _I64, _I64, _P, _P, _I64, _I64, _P, _I64, _I, _P], _I),
     "nm_decompress_i8": ([_P, _P, _I64, _I64, _P, _I64, _P], _I),
     "nm_spmm_i8": ([_P, _P, _I64, _I64, _P, _I64, _I64, _P, _I64, _P], _I),
+    "nm_prune_compress_tf32": ([_P, _I64, _I64, _I64, _P, _P, _P], _I),
+    "nm_decompress_tf32": ([_P, _P, _I64, _I64, _P, _I64, _P], _I),
+    "nm_spmm_tf32": ([_P, _P, _I64, _I64, _P, _I64, _I64, _P, _I64, _I, _P], _I),
     "nm_sddmm": ([_P, _I, _I, _I64, _I64, _P, _P, _I64, _P, _I64, _I64, _P, _I, _P], _I),
     "nm_spmm_algo": ([_P, _P, _I, _I, _I64, _I64, _P, _P, _I64, _I64, _P, _I64, _I, _I, _P], _I),
     "nm_spmm_permuted_noalloc": ([_P, _P, _I, _I, _I64, _I64, _P, _P, _I64, _I64, _P, _I64, _I, _P], _I),
@@ -194,6 +197,21 @@ def nm_decompress_i8(values, meta, R, K, W_out, ldw, stream=None) -> None:
 def nm_spmm_i8(values, meta, R, K, X, ldx, T, Y, ldy, stream=None) -> None:
     _check(lib().nm_spmm_i8(_ptr(values), _ptr(meta), R, K, _ptr(X), ldx, T, _ptr(Y), ldy, _stream(stream)),
            "nm_spmm_i8")
+
+
+def nm_prune_compress_tf32(W, R, K, ldw, values, meta, stream=None) -> None:
+    _check(lib().nm_prune_compress_tf32(_ptr(W), R, K, ldw, _ptr(values), _ptr(meta), _stream(stream)),
+           "nm_prune_compress_tf32")
+
+
+def nm_decompress_tf32(values, meta, R, K, W_out, ldw, stream=None) -> None:
+    _check(lib().nm_decompress_tf32(_ptr(values), _ptr(meta), R, K, _ptr(W_out), ldw, _stream(stream)),
+           "nm_decompress_tf32")
+
+
+def nm_spmm_tf32(values, meta, R, K, X, ldx, T, Y, ldy, y_dtype=NM_OUT_F32, stream=None) -> None:
+    _check(lib().nm_spmm_tf32(_ptr(values), _ptr(meta), R, K, _ptr(X), ldx, T, _ptr(Y), ldy, y_dtype,
+                              _stream(stream)), "nm_spmm_tf32")
 
 
 def nm_diag_prune_compress(W, R, K, ldw, D, offsets, values, stream=None) -> None:
@@ -384,6 +402,40 @@ def spmm_i8(values, meta, K: int, X, stream=None):
     ld = max((T + 3) // 4 * 4, 4)
     Y = torch.empty((R, ld), dtype=torch.int32, device=X.device)
     nm_spmm_i8(values, meta, R, K, X, X.stride(0), T, Y, ld, stream)
+    return Y[:, :T]
+
+
+def prune_compress_tf32(W, stream=None):
+    """1:2 (values R x K/2 float32, meta uint32 as int32) of float32 W (R x K), for the TF32 path."""
+    import torch
+    _require_cuda(W)
+    R, K = W.shape
+    vals = torch.empty((R, K // 2), dtype=torch.float32, device=W.device)
+    meta = torch.empty((max(nm_meta_words(R, K, 1, 2), 0),), dtype=torch.int32, device=W.device)
+    nm_prune_compress_tf32(W, R, K, W.stride(0), vals, meta, stream)
+    return vals, meta
+
+
+def decompress_tf32(values, meta, K: int, stream=None):
+    import torch
+    _require_cuda(values, meta)
+    R = values.shape[0]
+    out = torch.empty((R, K), dtype=torch.float32, device=values.device)
+    nm_decompress_tf32(values, meta, R, K, out, K, stream)
+    return out
+
+
+def spmm_tf32(values, meta, K: int, X, out_dtype=None, stream=None):
+    """Y = W' X from the 1:2 float32 operand and float32 X (K x T) on the TF32 tensor cores (fp32 by default)."""
+    import torch
+    _require_cuda(values, meta, X)
+    out_dtype = torch.float32 if out_dtype is None else out_dtype
+    R, T = values.shape[0], X.shape[1]
+    per = 4 if out_dtype == torch.float32 else 8
+    ld = max((T + per - 1) // per * per, per)
+    Y = torch.empty((R, ld), dtype=out_dtype, device=X.device)
+    nm_spmm_tf32(values, meta, R, K, X, X.stride(0), T, Y, ld,
+                 NM_OUT_F32 if out_dtype == torch.float32 else NM_OUT_BF16, stream)
     return Y[:, :T]
 
 

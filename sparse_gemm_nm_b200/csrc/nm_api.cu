@@ -159,6 +159,9 @@ struct TmapCache {
 };
 static thread_local TmapCache t_tmaps;
 
+// swizzle_bytes code of the 128-byte swizzle with 32-byte units (MN-major tf32 operands of the MMA).
+constexpr int kSwizzle128Atom32B = -32;
+
 static nm_status make_tmap(CUtensorMap* tm, const void* base, uint64_t inner, uint64_t outer,
                            uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer, int swizzle_bytes,
                            const char* what, CUtensorMapDataType dtype = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16) {
@@ -170,8 +173,9 @@ static nm_status make_tmap(CUtensorMap* tm, const void* base, uint64_t inner, ui
   cuuint64_t strides[1] = {row_bytes};
   cuuint32_t box[2] = {box_inner, box_outer};
   cuuint32_t estr[2] = {1, 1};
-  CUtensorMapSwizzle swz = swizzle_bytes == 128  ? CU_TENSOR_MAP_SWIZZLE_128B
-                           : swizzle_bytes == 64 ? CU_TENSOR_MAP_SWIZZLE_64B
+  CUtensorMapSwizzle swz = swizzle_bytes == 128                 ? CU_TENSOR_MAP_SWIZZLE_128B
+                           : swizzle_bytes == kSwizzle128Atom32B ? CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B
+                           : swizzle_bytes == 64                ? CU_TENSOR_MAP_SWIZZLE_64B
                            : swizzle_bytes == 32 ? CU_TENSOR_MAP_SWIZZLE_32B
                                                  : CU_TENSOR_MAP_SWIZZLE_NONE;
   CUresult r = fn(tm, dtype, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
@@ -179,6 +183,15 @@ static nm_status make_tmap(CUtensorMap* tm, const void* base, uint64_t inner, ui
   if (r != CUDA_SUCCESS) return fail(NM_ERR_CUDA, "cuTensorMapEncodeTiled(%s) failed with %d", what, (int)r);
   t_tmaps.put(key, *tm);
   return NM_OK;
+}
+
+// Whole-line TMA stores for the dense pair kernel's plain epilogue: C is rows x cols with row stride ldo
+// elements (bf16, or four-byte values when wide); the caller has checked 16-byte rows.
+static nm_status set_store_map(DenseParams& p, void* out, int64_t rows, int64_t cols, int64_t ldo, bool wide) {
+  p.tma_store = 1;
+  return wide ? make_tmap(&p.tm_out, out, (uint64_t)cols, (uint64_t)rows, (uint64_t)ldo * 4, 32, 32, 128,
+                          "C (four-byte)", CU_TENSOR_MAP_DATA_TYPE_FLOAT32)
+              : make_tmap(&p.tm_out, out, (uint64_t)cols, (uint64_t)rows, (uint64_t)ldo * 2, 64, 32, 128, "C (bf16)");
 }
 
 // 3-D map of the tiled 2:4 metadata: {64 words of a block, column blocks, row blocks}.
@@ -843,6 +856,7 @@ static nm_status run_spmm_t(const uint16_t* values, const uint32_t* meta, int n,
     st = make_tmap(&p.tm_a, wd, (uint64_t)K, (uint64_t)R, (uint64_t)ldk * 2, 64, 64, 128, "W' (dense)");
   if (e == cudaSuccess && st == NM_OK)
     st = make_tmap(&p.tm_b, dY, (uint64_t)T, (uint64_t)R, (uint64_t)lddy * 2, 64, 64, 128, "dY");
+  if (e == cudaSuccess && st == NM_OK && !idx) st = set_store_map(p, dX, K, T, lddx, p.out_f32 != 0);
   if (e == cudaSuccess && st == NM_OK) e = launch_dense_pair(p, true, true, EPI_STORE, stream);
   cudaFreeAsync(wd, stream);
   if (st != NM_OK) return st;
@@ -1009,12 +1023,112 @@ static nm_status run_spmm_i8(const int8_t* values, const uint32_t* meta, int64_t
   if (e == cudaSuccess && st == NM_OK)
     st = make_tmap(&p.tm_b, X, (uint64_t)T, (uint64_t)K, (uint64_t)ldx, 128, 64, 128, "X (int8)",
                    CU_TENSOR_MAP_DATA_TYPE_UINT8);
+  if (e == cudaSuccess && st == NM_OK) st = set_store_map(p, Y, R, T, ldy, true);
   if (e == cudaSuccess && st == NM_OK) e = launch_dense_pair_i8(p, stream);
   cudaFreeAsync(wd, stream);
   if (st != NM_OK) return st;
   return e == cudaSuccess ? NM_OK : cuda_fail(e, "int8 GEMM launch");
 }
 
+
+// TF32 path: 1:2 float32 weights, GEMM on a staged dense copy with the kind::tf32 pair kernel.
+static nm_status check_tf32_shape(int64_t R, int64_t K) {
+  if (R < 0 || K < 0) return fail(NM_ERR_INVALID_ARG, "negative dimension");
+  if (K % 2 != 0) return fail(NM_ERR_INVALID_ARG, "K must be even (1:2)");
+  if (R >= (1ll << 31) || K >= (1ll << 31)) return fail(NM_ERR_UNSUPPORTED, "dimensions must stay below 2^31");
+  return NM_OK;
+}
+
+static nm_status run_compress_tf32(const float* W, int64_t R, int64_t K, int64_t ldw, float* values, uint32_t* meta,
+                                   cudaStream_t stream) {
+  t_last_error.clear();
+  nm_status st = check_tf32_shape(R, K);
+  if (st != NM_OK) return st;
+  if (ldw < K) return fail(NM_ERR_INVALID_ARG, "ldw < K");
+  if (R == 0 || K == 0) return NM_OK;
+  if (!W || !values || !meta) return fail(NM_ERR_INVALID_ARG, "null pointer");
+  if (!aligned_to(W, 4) || !aligned_to(values, 4) || !aligned_to(meta, 4))
+    return fail(NM_ERR_MISALIGNED, "float32 operands must be 4-byte aligned");
+  st = require_device();
+  if (st != NM_OK) return st;
+  cudaError_t e = launch_compress_tf32(W, R, K, ldw, values, meta, stream);
+  return e == cudaSuccess ? NM_OK : cuda_fail(e, "tf32 compress launch");
+}
+
+static nm_status run_decompress_tf32(const float* values, const uint32_t* meta, int64_t R, int64_t K, float* W_out,
+                                     int64_t ldw, cudaStream_t stream) {
+  t_last_error.clear();
+  nm_status st = check_tf32_shape(R, K);
+  if (st != NM_OK) return st;
+  if (ldw < K) return fail(NM_ERR_INVALID_ARG, "ldw < K");
+  if (R == 0 || K == 0) return NM_OK;
+  if (!W_out || !values || !meta) return fail(NM_ERR_INVALID_ARG, "null pointer");
+  if (!aligned_to(W_out, 4) || !aligned_to(values, 4) || !aligned_to(meta, 4))
+    return fail(NM_ERR_MISALIGNED, "float32 operands must be 4-byte aligned");
+  st = require_device();
+  if (st != NM_OK) return st;
+  cudaError_t e = launch_decompress_tf32(values, meta, R, K, W_out, ldw, stream);
+  return e == cudaSuccess ? NM_OK : cuda_fail(e, "tf32 decompress launch");
+}
+
+static nm_status run_spmm_tf32(const float* values, const uint32_t* meta, int64_t R, int64_t K, const float* X,
+                               int64_t ldx, int64_t T, void* Y, int64_t ldy, nm_out_dtype dtype, cudaStream_t stream) {
+  t_last_error.clear();
+  nm_status st = check_tf32_shape(R, K);
+  if (st != NM_OK) return st;
+  if (T < 0) return fail(NM_ERR_INVALID_ARG, "negative dimension");
+  if (dtype != NM_OUT_BF16 && dtype != NM_OUT_F32) return fail(NM_ERR_INVALID_ARG, "bad output dtype");
+  if (R == 0 || T == 0) return NM_OK;
+  if (!Y) return fail(NM_ERR_INVALID_ARG, "Y is null");
+  if (ldy < T) return fail(NM_ERR_INVALID_ARG, "ldy < T");
+  const int esize = dtype == NM_OUT_F32 ? 4 : 2;
+  if (!al16(Y) || (ldy * esize) % 16 != 0) return fail(NM_ERR_MISALIGNED, "Y rows must be 16-byte aligned");
+  if (T >= (1ll << 31)) return fail(NM_ERR_UNSUPPORTED, "dimensions must stay below 2^31");
+  st = require_device();
+  if (st != NM_OK) return st;
+  if (K == 0) {
+    cudaError_t e = launch_fill_zero(Y, R, T, ldy, esize, stream);
+    return e == cudaSuccess ? NM_OK : cuda_fail(e, "zero fill");
+  }
+  if (!values || !meta || !X) return fail(NM_ERR_INVALID_ARG, "null operand");
+  if (ldx < T) return fail(NM_ERR_INVALID_ARG, "ldx < T");
+  if (!al16(X) || ldx % 4 != 0) return fail(NM_ERR_MISALIGNED, "X rows must be 16-byte aligned");
+  if (!aligned_to(values, 4) || !aligned_to(meta, 4)) return fail(NM_ERR_MISALIGNED, "values must be 4-byte aligned");
+  cudaMemPool_t pool = nullptr;
+  cudaError_t e = staging_pool(&pool);
+  if (e != cudaSuccess) return cuda_fail(e, "staging pool");
+  const int64_t ldk = (K + 3) / 4 * 4;  // 16-byte rows for the TMA
+  void* wd = nullptr;
+  e = cudaMallocFromPoolAsync(&wd, (size_t)(R * ldk * 4), pool, stream);
+  if (e != cudaSuccess) return cuda_fail(e, "staging buffer for the decompressed float32 weights");
+  e = launch_decompress_tf32(values, meta, R, K, static_cast<float*>(wd), ldk, stream);
+  DenseParams p;
+  std::memset(&p, 0, sizeof p);
+  p.M = R;
+  p.N = T;
+  p.Kr = K;
+  p.k_tiles = (K + 63) / 64;
+  p.tiles_m = (int)((R + 255) / 256);
+  p.tiles_n = (int)((T + 255) / 256);
+  p.num_tiles = p.tiles_m * p.tiles_n;
+  p.status = status_word_ptr();
+  p.out = Y;
+  p.ldo = ldy;
+  p.out_f32 = dtype == NM_OUT_F32;
+  if (e == cudaSuccess && !p.status) e = cudaErrorInvalidSymbol;
+  if ((int64_t)p.tiles_m * p.tiles_n >= (1ll << 31)) st = fail(NM_ERR_UNSUPPORTED, "too many tiles");
+  if (e == cudaSuccess && st == NM_OK)
+    st = make_tmap(&p.tm_a, wd, (uint64_t)K, (uint64_t)R, (uint64_t)ldk * 4, 32, 64, 128, "W' (float32, dense)",
+                   CU_TENSOR_MAP_DATA_TYPE_FLOAT32);
+  if (e == cudaSuccess && st == NM_OK)
+    st = make_tmap(&p.tm_b, X, (uint64_t)T, (uint64_t)K, (uint64_t)ldx * 4, 32, 64, kSwizzle128Atom32B,
+                   "X (float32)", CU_TENSOR_MAP_DATA_TYPE_FLOAT32);
+  if (e == cudaSuccess && st == NM_OK) st = set_store_map(p, Y, R, T, ldy, p.out_f32 != 0);
+  if (e == cudaSuccess && st == NM_OK) e = launch_dense_pair_tf32(p, stream);
+  cudaFreeAsync(wd, stream);
+  if (st != NM_OK) return st;
+  return e == cudaSuccess ? NM_OK : cuda_fail(e, "tf32 GEMM launch");
+}
 
 // Diagonal sparsity: selection + gather, dense copy, GEMM on the dense copy.
 static nm_status run_diag_prune_compress(const uint16_t* W, int64_t R, int64_t K, int64_t ldw, int64_t D,
@@ -1141,6 +1255,7 @@ static nm_status run_diag_spmm(const uint16_t* values, const int32_t* offsets, i
     st = make_tmap(&p.tm_b_alt, X, (uint64_t)T, (uint64_t)K, (uint64_t)ldx * 2, 64, 64, 128, "X (direct)");
     p.use_alt = is_perm;
   }
+  if (e == cudaSuccess && st == NM_OK) st = set_store_map(p, Y, R, T, ldy, p.out_f32 != 0);
   if (e == cudaSuccess && st == NM_OK) e = launch_dense_pair(p, false, true, EPI_STORE, stream);
   cudaFreeAsync(wd, stream);
   if (xp) cudaFreeAsync(xp, stream);
@@ -1304,6 +1419,21 @@ nm_status nm_decompress_i8(const int8_t* values, const uint32_t* meta, int64_t R
 nm_status nm_spmm_i8(const int8_t* values, const uint32_t* meta, int64_t R, int64_t K, const int8_t* X, int64_t ldx,
                      int64_t T, int32_t* Y, int64_t ldy, void* stream) {
   return run_spmm_i8(values, meta, R, K, X, ldx, T, Y, ldy, static_cast<cudaStream_t>(stream));
+}
+
+nm_status nm_prune_compress_tf32(const float* W, int64_t R, int64_t K, int64_t ldw, float* values, uint32_t* meta,
+                                 void* stream) {
+  return run_compress_tf32(W, R, K, ldw, values, meta, static_cast<cudaStream_t>(stream));
+}
+
+nm_status nm_decompress_tf32(const float* values, const uint32_t* meta, int64_t R, int64_t K, float* W_out, int64_t ldw,
+                             void* stream) {
+  return run_decompress_tf32(values, meta, R, K, W_out, ldw, static_cast<cudaStream_t>(stream));
+}
+
+nm_status nm_spmm_tf32(const float* values, const uint32_t* meta, int64_t R, int64_t K, const float* X, int64_t ldx,
+                       int64_t T, void* Y, int64_t ldy, nm_out_dtype y_dtype, void* stream) {
+  return run_spmm_tf32(values, meta, R, K, X, ldx, T, Y, ldy, y_dtype, static_cast<cudaStream_t>(stream));
 }
 
 nm_status nm_diag_prune_compress(const uint16_t* W, int64_t R, int64_t K, int64_t ldw, int64_t D, int32_t* offsets,

@@ -37,7 +37,8 @@ constexpr uint32_t kA = 32768, kB = 32768;
 constexpr uint32_t kTx = 2u * (kA + kB);  // both CTAs' bytes of a stage
 constexpr uint32_t kTmemCols = 512;  // two 256-column accumulators
 constexpr uint32_t kRowPad = 33;          // epilogue row buffer: 32 floats + 1 (no bank conflicts)
-constexpr uint32_t kEpiBuf = 32 * kRowPad * 4;
+constexpr uint32_t kEpiBuf = 5120;        // per epilogue warp: the row buffer, or a 4 KB TMA-store tile (1024-aligned)
+static_assert(kEpiBuf >= 32 * kRowPad * 4 && kEpiBuf % 1024 == 0, "epilogue buffer");
 constexpr uint64_t kWaitNs = 2000000000ull;
 constexpr uint32_t kOffBuf = kStages * (kA + kB);
 constexpr uint32_t kOffBar = kOffBuf + 4 * kEpiBuf;
@@ -63,12 +64,15 @@ __device__ __forceinline__ int64_t survivor_col(const DenseParams& p, int64_t r,
 
 // I8: signed int8 operands and int32 accumulation (kind::i8).  A stage then holds 256 reduction steps in
 // the same bytes: A K-major as two 128-byte halves, B MN-major as one 128-column strip of 256 rows.
-template <bool A_MN, bool B_MN, int EPI, bool I8 = false>
+template <bool A_MN, bool B_MN, int EPI, bool I8 = false, bool TF32 = false>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dpair::kThreads, 1)
     dense_pair_kernel(const __grid_constant__ DenseParams p) {
   using namespace dpair;
   static_assert(!I8 || (!A_MN && B_MN), "int8: K-major A and MN-major B");
-  constexpr uint32_t kIdesc = I8 ? idesc_s8_major(256, 256, A_MN, B_MN) : idesc_bf16_major(256, 256, A_MN, B_MN);
+  static_assert(!TF32 || (!A_MN && B_MN && !I8), "tf32: K-major A and MN-major B");
+  constexpr uint32_t kIdesc = I8     ? idesc_s8_major(256, 256, A_MN, B_MN)
+                              : TF32 ? idesc_tf32_major(256, 256, A_MN, B_MN)
+                                     : idesc_bf16_major(256, 256, A_MN, B_MN);
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + kOffBar);
@@ -137,6 +141,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dpair::kThreads, 1)
           if (rank == 0) mbar_arrive_expect_tx(&full[s], kTx);
           uint8_t* a = smem + s * (kA + kB);
           uint8_t* b = a + kA;
+          if (TF32) {  // A: two 32-step halves x two 64-row halves; B: four 32-column strips of 64 rows (their
+                       // tensor map swizzles 128-byte rows in 32-byte units, the layout the MMA reads)
+            const int32_t k0 = (int32_t)(kt * 64);
+#pragma unroll
+            for (int i = 0; i < 2; ++i)
+#pragma unroll
+              for (int h = 0; h < 2; ++h)
+                tma_load_2d_pair(a + i * 16384 + h * 8192, &p.tm_a, bar, k0 + 32 * i, m0 + 64 * h);
+#pragma unroll
+            for (int j = 0; j < 4; ++j) tma_load_2d_pair(b + j * 8192, tmb, bar, n0 + 32 * j, k0);
+            if (++s == kStages) { s = 0; ph ^= 1u; }
+            continue;
+          }
           if (I8) {  // A: two 128-step halves x two 64-row halves; B: four 64-row boxes of one 128-column strip
             const int32_t k0 = (int32_t)(kt * 256);
 #pragma unroll
@@ -194,12 +211,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dpair::kThreads, 1)
             // apart); MN-major operands advance 16 rows of 128 B (strips 16 KB apart).
             const uint64_t ad = A_MN ? smem_desc(a_addr + kk * 2048, 16384, 1024, SWZ_128B)
                                      : smem_desc(a_addr + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024, SWZ_128B);
-            // int8 MN-major B: K = 32 step kk advances 32 rows of 128 B
-            const uint64_t bd = I8 ? smem_desc(b_addr + kk * 4096, 32768, 1024, SWZ_128B)
+            // int8 MN-major B: K = 32 step kk advances 32 rows of 128 B.  tf32 (K = 8 steps of 32 B for A):
+            // B is MN-major in the 128-byte / 32-byte-unit swizzle (four-row atoms 512 B apart), advances
+            // 8 rows of 128 B, and its four 32-column strips are 8 KB apart
+            const uint64_t bd = I8     ? smem_desc(b_addr + kk * 4096, 32768, 1024, SWZ_128B)
+                                : TF32 ? smem_desc(b_addr + kk * 1024, 8192, 512, SWZ_128B_BASE32B)
                                 : B_MN ? smem_desc(b_addr + kk * 2048, 16384, 1024, SWZ_128B)
                                        : smem_desc(b_addr + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024, SWZ_128B);
             if (I8)
               tc_mma_pair_i8(d_tmem, ad, bd, kIdesc, (kt > 0 || kk > 0) ? 1u : 0u);
+            else if (TF32)
+              tc_mma_pair_tf32(d_tmem, ad, bd, kIdesc, (kt > 0 || kk > 0) ? 1u : 0u);
             else
               tc_mma_pair(d_tmem, ad, bd, kIdesc, (kt > 0 || kk > 0) ? 1u : 0u);
           }
@@ -229,6 +251,53 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dpair::kThreads, 1)
       if (!ok) break;
       tc_fence_after();
       const uint32_t t_addr = tmem_base + ((uint32_t)(quarter * 32) << 16) + 256u * (uint32_t)ab;
+      if (EPI == EPI_STORE && p.tma_store) {
+        // Whole-line stores: each chunk (64 bf16 or 32 four-byte columns = 128-byte rows) goes through
+        // this warp's 128-byte-swizzled staging tile and one TMA store of 32 rows; parts of the box past
+        // M or N are not written.  The accumulator is released after its last TMEM load.
+        const bool wide = p.out_f32 != 0;
+        const int chunks = wide ? 8 : 4;
+        const int32_t wrow0 = (int32_t)(tm * 256 + 128 * rank + quarter * 32);
+        uint8_t* sbuf = smem + kOffBuf + (warp - 4) * kEpiBuf;
+#pragma unroll 1
+        for (int c = 0; c < chunks; ++c) {
+          uint32_t w[32];
+          if (wide) {
+            tmem_ld_32x32b_x32(t_addr + c * 32, w);
+            tc_wait_ld();
+          } else {
+            uint32_t v[32];
+            tmem_ld_32x32b_x32(t_addr + c * 64, v);
+            tc_wait_ld();
+#pragma unroll
+            for (int j = 0; j < 16; ++j) w[j] = pack_bf16x2(__uint_as_float(v[2 * j]), __uint_as_float(v[2 * j + 1]));
+            tmem_ld_32x32b_x32(t_addr + c * 64 + 32, v);
+            tc_wait_ld();
+#pragma unroll
+            for (int j = 0; j < 16; ++j)
+              w[16 + j] = pack_bf16x2(__uint_as_float(v[2 * j]), __uint_as_float(v[2 * j + 1]));
+          }
+          if (c == chunks - 1) {
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive_cluster(lead_acc_empty0 + 8u * (uint32_t)ab);
+          }
+          const int64_t col0 = n0 + (wide ? 32 : 64) * c;
+          if (lane == 0) bulk_wait_group_read<0>();  // the previous store has read the tile
+          __syncwarp();
+#pragma unroll
+          for (int j = 0; j < 8; ++j)
+            *reinterpret_cast<uint4*>(sbuf + lane * 128 + ((j ^ (lane & 7)) << 4)) =
+                make_uint4(w[4 * j], w[4 * j + 1], w[4 * j + 2], w[4 * j + 3]);
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0 && col0 < p.N && (int64_t)wrow0 < p.M) {
+            tma_store_2d(&p.tm_out, sbuf, (int32_t)col0, wrow0);
+            bulk_commit_group();
+          }
+        }
+        continue;
+      }
       bool row_ok = row < p.M;
       int64_t orow = row;
       if (EPI == EPI_STORE && row_ok && p.row_map) {
@@ -319,6 +388,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dpair::kThreads, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(lead_acc_empty0 + 8u * (uint32_t)ab);
     }
+    if (lane == 0) bulk_wait_group<0>();  // every TMA store of this warp has landed
   }
 
   // -------------------------------------------------------------- teardown
@@ -332,20 +402,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dpair::kThreads, 1)
   }
 }
 
-template <bool A_MN, bool B_MN, int EPI, bool I8 = false>
+template <bool A_MN, bool B_MN, int EPI, bool I8 = false, bool TF32 = false>
 static cudaError_t launch_dp(const DenseParams& p, cudaStream_t stream) {
   static bool configured[64] = {};
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev >= 0 && dev < 64 && !configured[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(dense_pair_kernel<A_MN, B_MN, EPI, I8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaError_t e = cudaFuncSetAttribute(dense_pair_kernel<A_MN, B_MN, EPI, I8, TF32>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)dpair::kSmemBytes);
     if (e != cudaSuccess) return e;
     configured[dev] = true;
   }
   const int pairs_avail = sm_count_current() / 2;
   const int pairs = p.num_tiles < pairs_avail ? p.num_tiles : pairs_avail;
-  cudaError_t e = launch_pdl(dense_pair_kernel<A_MN, B_MN, EPI, I8>, dim3(2 * pairs), dim3(dpair::kThreads),
+  cudaError_t e = launch_pdl(dense_pair_kernel<A_MN, B_MN, EPI, I8, TF32>, dim3(2 * pairs), dim3(dpair::kThreads),
                              (size_t)dpair::kSmemBytes, stream, p);
   count_launch();
   return e != cudaSuccess ? e : cudaGetLastError();
@@ -364,6 +434,13 @@ cudaError_t launch_dense_pair(const DenseParams& p, bool a_mn, bool b_mn, int ep
 cudaError_t launch_dense_pair_i8(const DenseParams& p, cudaStream_t stream) {
   if (p.num_tiles <= 0) return cudaSuccess;
   return launch_dp<false, true, EPI_STORE, true>(p, stream);
+}
+
+// tf32 forward GEMM on the decompressed 1:2 operand: A (float32) K-major, B (float32) MN-major, a stage of
+// 64 reduction steps in the same bytes as a bf16 stage.
+cudaError_t launch_dense_pair_tf32(const DenseParams& p, cudaStream_t stream) {
+  if (p.num_tiles <= 0) return cudaSuccess;
+  return launch_dp<false, true, EPI_STORE, false, true>(p, stream);
 }
 
 }  // namespace nmk

@@ -247,6 +247,16 @@ __device__ __forceinline__ void tc_mma_pair(uint32_t d_tmem, uint64_t a_desc, ui
 }
 
 // The same for kind::i8: signed 8-bit A and B, int32 accumulator.
+__device__ __forceinline__ void tc_mma_pair_tf32(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                                 uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::tf32 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
 __device__ __forceinline__ void tc_mma_pair_i8(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
                                                uint32_t accumulate) {
   asm volatile(
@@ -363,7 +373,10 @@ __device__ __forceinline__ void tmem_ld_32x32b_x16(uint32_t taddr, uint32_t (&r)
 
 // Shared-memory matrix descriptor (sm_100 layout): start, leading and stride
 // byte offsets (16-byte units), descriptor version 1, swizzle mode in [61,64).
-enum : uint32_t { SWZ_NONE = 0, SWZ_128B = 2, SWZ_64B = 4, SWZ_32B = 6 };
+// Layout type of a shared-memory matrix descriptor (bits 61-63).  SWZ_128B_BASE32B is the 128-byte
+// swizzle with 32-byte units (XOR of address bits 7-8 into bits 5-6), the MN-major layout of 32-bit
+// (tf32) operands; its swizzle atom is four 128-byte rows.
+enum : uint32_t { SWZ_NONE = 0, SWZ_128B_BASE32B = 1, SWZ_128B = 2, SWZ_64B = 4, SWZ_32B = 6 };
 
 __device__ __forceinline__ uint64_t smem_desc(uint32_t saddr, uint32_t lbo_bytes, uint32_t sbo_bytes,
                                               uint32_t swizzle) {
@@ -391,6 +404,12 @@ __host__ __device__ constexpr uint32_t idesc_bf16_major(uint32_t n, uint32_t m, 
 }
 
 // kind::i8 descriptor: signed 8-bit A and B, int32 D (c_format 2), operand majors as above.
+// kind::tf32 descriptor: TF32 A and B (type 2), F32 D, operand majors as above.
+__host__ __device__ constexpr uint32_t idesc_tf32_major(uint32_t n, uint32_t m, bool a_mn, bool b_mn) {
+  return (1u << 4) | (2u << 7) | (2u << 10) | (a_mn ? (1u << 15) : 0u) | (b_mn ? (1u << 16) : 0u) |
+         ((n >> 3) << 17) | ((m >> 4) << 24);
+}
+
 __host__ __device__ constexpr uint32_t idesc_s8_major(uint32_t n, uint32_t m, bool a_mn, bool b_mn) {
   return (2u << 4) | (1u << 7) | (1u << 10) | (a_mn ? (1u << 15) : 0u) | (b_mn ? (1u << 16) : 0u) |
          ((n >> 3) << 17) | ((m >> 4) << 24);

@@ -72,7 +72,9 @@ struct SpmmParams {
 struct DenseParams {
   CUtensorMap tm_a, tm_b;
   CUtensorMap tm_b_alt;     // read instead of tm_b when use_alt is set and *use_alt is nonzero at run time
+  CUtensorMap tm_out;       // epilogue 0 with tma_store: C (M x N), box {64 bf16 | 32 four-byte, 32 rows}, 128B swizzle
   const uint32_t* use_alt;
+  int tma_store;            // epilogue 0 without row_map: whole-line TMA stores through tm_out
   int64_t M, N, Kr;
   int64_t k_tiles;
   int tiles_m, tiles_n, num_tiles;
@@ -90,6 +92,12 @@ struct DenseParams {
 enum DenseEpi : int { EPI_STORE = 0, EPI_SURVIVORS = 1 };
 cudaError_t launch_dense_pair(const DenseParams& p, bool a_mn, bool b_mn, int epi, cudaStream_t stream);
 cudaError_t launch_dense_pair_i8(const DenseParams& p, cudaStream_t stream);
+cudaError_t launch_dense_pair_tf32(const DenseParams& p, cudaStream_t stream);
+// 1:2 float32 operand for the TF32 path (values R x K/2, metadata R x ceil(K/64) words, one bit per survivor).
+cudaError_t launch_compress_tf32(const float* W, int64_t R, int64_t K, int64_t ldw, float* values, uint32_t* meta,
+                                 cudaStream_t s);
+cudaError_t launch_decompress_tf32(const float* values, const uint32_t* meta, int64_t R, int64_t K, float* W_out,
+                                   int64_t ldw, cudaStream_t s);
 cudaError_t launch_diag_select(const uint16_t* W, int64_t R, int64_t K, int64_t ldw, int64_t D, float* part,
                                float* scores, uint8_t* keep, int32_t* offsets, uint16_t* values, cudaStream_t s);
 // Dense copy of a diagonal operand, columns [0, K) of rows [0, R) of W_out.
