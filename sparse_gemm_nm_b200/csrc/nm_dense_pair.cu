@@ -1,4 +1,6 @@
-// nm_dense_pair.cu -- dense bf16 GEMMs on SM pairs for the backward pass of an N:M layer.
+// nm_dense_pair.cu -- dense GEMMs on SM pairs: the backward pass of an N:M layer,
+// and the forward GEMM of the formats run on a staged dense copy (the diagonal
+// pattern in bf16, INT8 2:4 as kind::i8, TF32 1:2 as kind::tf32).
 //
 // Training keeps the N:M structure of W' through every step ("Structured
 // Sparsity" topic cards, RNM-TD3 abstract; the DynaDiag page's abstract asks
@@ -20,6 +22,10 @@
 // MMA thread issues eight tcgen05.mma (K = 16) per stage; its commits release
 // the stage in both CTAs.  Each CTA drains its own 128 x 256 fp32 accumulator;
 // two accumulators (512 TMEM columns) let the next tile's MMAs run meanwhile.
+// The int8 and tf32 forms keep the stage bytes (256 and 64 reduction steps),
+// with K = 32 and K = 8 per MMA.  The plain store epilogue sends whole
+// 128-byte row chunks through a swizzled staging tile and TMA stores; with a
+// row map (dX under an index map) rows are stored one per lane.
 #include <cstdint>
 #include <cuda.h>
 #include <cuda_runtime.h>
