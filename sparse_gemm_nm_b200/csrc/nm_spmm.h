@@ -78,6 +78,7 @@ struct DenseParams {
   int64_t M, N, Kr;
   int64_t k_tiles;
   int tiles_m, tiles_n, num_tiles;
+  int n_major;  // tile order: column tiles fastest, so pairs running together share A's row block (A larger than B)
   uint32_t* status;
   void* out;
   int64_t ldo;
