@@ -94,3 +94,25 @@ def test_product_package_does_not_touch_the_oracle():
             if f.endswith((".py", ".cu", ".cuh", ".h", ".cpp")):
                 text = open(os.path.join(dirpath, f)).read()
                 assert "oracle" not in text.replace("oracle as the", ""), f
+
+
+def test_host_argument_checks_of_the_format_calls(lib):
+    """The TF32, INT8 and diagonal calls refuse bad shapes, leading dimensions and nulls before any launch."""
+    L = lib
+    I = nm.NM_ERR_INVALID_ARG
+    assert L.nm_prune_compress_tf32(None, 4, 5, 6, None, None, None) == I          # odd K (1:2)
+    assert L.nm_prune_compress_tf32(None, 4, 8, 6, None, None, None) == I          # ldw < K
+    assert L.nm_prune_compress_tf32(None, 4, 8, 8, None, None, None) == I          # null pointers
+    assert L.nm_prune_compress_tf32(None, 0, 8, 8, None, None, None) == nm.NM_OK   # empty
+    assert L.nm_decompress_tf32(None, None, 4, 7, None, 8, None) == I
+    assert L.nm_spmm_tf32(None, None, 4, 8, None, 8, 8, None, 8, 7, None) == I     # bad output dtype
+    assert L.nm_spmm_tf32(None, None, 4, 8, None, 8, 8, None, 4, 0, None) == I     # ldy < T
+    assert L.nm_spmm_tf32(None, None, 4, 8, None, 8, 8, None, 8, 0, None) == I     # Y null
+    assert L.nm_spmm_tf32(None, None, 0, 8, None, 8, 8, None, 8, 0, None) == nm.NM_OK
+    assert L.nm_diag_prune_compress(None, 4, 8, 8, 9, None, None, None) == I       # D > K
+    assert L.nm_diag_prune_compress(None, 4, 8, 6, 2, None, None, None) == I       # ldw < K
+    assert L.nm_diag_expand(None, None, 9, 4, 8, None, 8, None) == I               # D > K
+    assert L.nm_diag_spmm(None, None, 9, 4, 8, None, None, 8, 8, None, 8, 0, None) == I
+    assert L.nm_diag_spmm(None, None, 2, 4, 8, None, None, 8, 8, None, 4, 0, None) == I  # ldy < T
+    assert L.nm_prune_compress_i8(None, 4, 16, 8, None, None, None) == I           # ldw < K
+    assert L.nm_spmm_i8(None, None, 4, 16, None, 16, 16, None, 8, None) == I       # ldy < T
