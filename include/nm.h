@@ -315,7 +315,8 @@ NM_API nm_status nm_spmm_tf32(const float* values, const uint32_t* meta, int64_t
  *   placement, gather).
  * nm_diag_expand: the dense R x K copy (+0 off the kept diagonals), row
  *   stride ldw >= K (columns K..ldw-1 are not written); offsets outside
- *   [0, K) place nothing.  Every element is written once, by lookup in a
+ *   [0, K) place nothing; offsets must be distinct (of a repeated offset,
+ *   one of its diagonals is placed).  Every element is written once, by lookup in a
  *   K-entry table staged from the library's pool (K*4 bytes).
  * nm_diag_spmm: y[r][t] = sum_d V[d][r] * X[idx[(r + o_d) mod K]][t]
  *   (X[k] when idx is NULL; idx entries outside [0, K) read zero rows).
