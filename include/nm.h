@@ -2,7 +2,9 @@
  * nm.h -- C ABI of libnm_b200, N:M structured weight sparsity on NVIDIA B200
  * (sm_100a): magnitude prune + push-left compression, decompression, and the
  * sparse x dense GEMM y = (W Pi) x in plain, column-permuted and PATCH-style
- * hybrid forms.
+ * hybrid forms; further down, the one-call prune + GEMM, the two backward
+ * products, INT8 2:4, TF32 1:2 (float32 data) and the diagonal pattern, each
+ * with its own conventions where they differ from the ones below.
  *
  * Conventions shared by every call
  *  - bf16 data is passed as its 16-bit pattern (uint16_t).  All matrices are
@@ -27,9 +29,9 @@
  *              (b = ceil(log2 M) bits) in word r*ceil(K*N/M/S) + floor(j/S) at
  *              bit b*(j mod S), S = floor(32/b); unused bits 0.
  *  - Every pointer is DEVICE memory owned by the caller (none is freed or
- *    retained).  The library allocates no device memory, except the staging
- *    buffers of the GEMM calls on the two-SM path (see nm_spmm and
- *    nm_spmm_permuted).
+ *    retained).  The library allocates no device memory, except stream-ordered
+ *    staging buffers from its own pool in the calls that document them (the
+ *    GEMMs on the two-SM path, the backward, INT8, TF32 and diagonal calls).
  *  - Calls are asynchronous on `stream` (a cudaStream_t; NULL = the legacy
  *    default stream).  Argument errors are detected on the host and returned
  *    before anything is launched.  Each successful call launches one kernel
