@@ -309,10 +309,14 @@ NM_API nm_status nm_spmm_tf32(const float* values, const uint32_t* meta, int64_t
  * and values V (D x R bf16), V[d][r] = W[r][(r + o_d) mod K].
  *
  * nm_diag_prune_compress: keep the D diagonals of largest score
- *   s(o) = sum_r |W[r][(r + o) mod K]| (fp32 in a fixed order: 32-row chunk
- *   sums with r ascending, then the chunk sums in ascending order; NaN ranks
- *   above every number; ties to the lower offset); writes offsets[D] and
- *   values (D x R).  Stages ceil(R/32)*K*4 + K*8 bytes from the library's
+ *   s(o) = sum_r |W[r][(r + o) mod K]| (NaN ranks above every number; ties
+ *   to the lower offset); writes offsets[D] and values (D x R).  The device
+ *   adds the scores in float32 (32-row chunk sums with r ascending, then the
+ *   chunk sums in ascending order), so where two diagonals' exact scores
+ *   differ by less than the rounding of R float32 additions, either one may
+ *   be kept: the set is one that a float32 evaluation of s ranks first, and
+ *   no dropped diagonal's exact score exceeds a kept one's by more than
+ *   that rounding.  Stages ceil(R/32)*K*4 + K*8 bytes from the library's
  *   pool; a memset and five launches (partial sums, scores, ranks,
  *   placement, gather).
  * nm_diag_expand: the dense R x K copy (+0 off the kept diagonals), row

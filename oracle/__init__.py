@@ -373,15 +373,71 @@ def spmm_f32(values, meta, K, X, n=1, m=2, with_abs=False):
 
 
 def diag_scores(W):
+    """float64 scores s(o) = sum_r |W[r][(r + o) mod K]| (r ascending; NaN if the diagonal holds one)."""
     W = _u16(W)
     R, K = W.shape
-    out = np.zeros(K, np.float32)
+    out = np.zeros(K, np.float64)
     _check(_load().oracle_diag_scores(_ptr(W), R, K, K, _ptr(out)), "diag_scores")
     return out
 
 
+def diag_selection_errors(W, D, offsets, terms_exact=False):
+    """Why ``offsets`` is not a valid choice of the D highest-scoring diagonals of W (empty list: it is).
+
+    Several selections are correct when a device adds the scores in float32:
+    two diagonals whose exact scores differ by less than the float32 rounding
+    error may come out in either order.  A selection is accepted when
+    * it holds D distinct offsets in [0, K), ascending;
+    * every diagonal holding a NaN is kept before any other (NaNs tie among
+      themselves: lower offsets first);
+    * no dropped diagonal beats a kept one by more than the rounding error:
+      min over kept of s*(1 + g) >= max over dropped of s*(1 - g), where s is
+      the exact score (``diag_scores``) and g = (n - 1) u / (1 - (n - 1) u),
+      u = 2^-24, bounds the relative error of ANY float32 summation order of
+      n = R non-negative terms that are exact in float32 (Higham, "Accuracy
+      and Stability of Numerical Algorithms", recursive summation bound).
+    With ``terms_exact`` (every partial sum is exact in float32, e.g. small
+    integers) g = 0 and equal scores must go to the lower offset.  The bound
+    assumes the float32 sums do not overflow.
+    """
+    W = _u16(W)
+    R, K = W.shape
+    offs = np.asarray(offsets)
+    errs = []
+    if offs.shape != (D,):
+        return [f"expected {D} offsets, got shape {offs.shape}"]
+    if D and (offs.min() < 0 or offs.max() >= K):
+        return ["offset outside [0, K)"]
+    if np.any(np.diff(offs.astype(np.int64)) <= 0):
+        return ["offsets not strictly ascending"]
+    s = diag_scores(W)
+    kept = np.zeros(K, bool)
+    kept[offs] = True
+    nan = np.isnan(s)
+    if np.any(nan & ~kept) and np.any(~nan & kept):
+        errs.append("a diagonal without NaN kept while one with NaN was dropped")
+    kn, dn = np.flatnonzero(nan & kept), np.flatnonzero(nan & ~kept)
+    if kn.size and dn.size and kn.max() > dn.min():
+        errs.append("NaN diagonals not kept in offset order")
+    fk, fd = np.flatnonzero(~nan & kept), np.flatnonzero(~nan & ~kept)
+    if fk.size and fd.size:
+        if terms_exact:
+            a = fk[np.lexsort((-fk, s[fk]))[0]]        # weakest kept: lowest score, then highest offset
+            b = fd[np.lexsort((fd, -s[fd]))[0]]        # strongest dropped: highest score, then lowest offset
+            if s[a] < s[b] or (s[a] == s[b] and a > b):
+                errs.append(f"dropped offset {b} (score {s[b]!r}) beats kept offset {a} (score {s[a]!r})")
+        else:
+            u = 2.0 ** -24
+            g = (R - 1) * u / (1.0 - (R - 1) * u)
+            lo, hi = s[fk].min() * (1.0 + g), s[fd].max() * (1.0 - g)
+            if lo < hi:
+                errs.append(f"a dropped score {s[fd].max()!r} beats the lowest kept score {s[fk].min()!r} by more "
+                            f"than the float32 bound (relative {g:.3g})")
+    return errs
+
+
 def diag_select(W, D):
-    """Ascending int32 offsets of the D diagonals with the largest fp32 scores (ties to the lower offset)."""
+    """Ascending int32 offsets of the D diagonals with the largest scores (ties to the lower offset)."""
     W = _u16(W)
     R, K = W.shape
     out = np.zeros(D, np.int32)
