@@ -236,20 +236,26 @@ def test_hybrid_integer_exact():
 # ----------------------------------------------------------------------------
 # Full workload sizes, sampled outputs
 # ----------------------------------------------------------------------------
-def sampled_check(vals, meta, n, m, W_unused, X, Y, idx=None, count=3000, seed=0):
+def sampled_check(vals, meta, n, m, W, X, Y, idx=None, count=3000, seed=0):
+    """Compare sampled outputs of Y with the oracle's product of ITS OWN compressed
+    form of W (oracle.compress), after asserting that the device's compressed
+    operand (vals, meta) equals that form bit for bit."""
     R, T = Y.shape
     K = X.shape[0]
+    ov, om = oracle.compress(W, n, m)
+    assert np.array_equal(bits(vals), ov), "compressed values differ from the oracle's"
+    assert np.array_equal(meta.cpu().numpy().view(np.uint32), om), "metadata differs from the oracle's"
     rng = np.random.default_rng(seed)
     rows = np.concatenate([rng.integers(0, R, count), [0, R - 1, 0, R - 1]])
     cols = np.concatenate([rng.integers(0, T, count), [0, T - 1, T - 1, 0]])
-    ref, mag = oracle.spmm_sampled(bits(vals), meta.cpu().numpy().view(np.uint32), n, m, K, X, rows, cols, idx)
+    ref, mag = oracle.spmm_sampled(ov, om, n, m, K, X, rows, cols, idx)
     got = values_f64(Y)[rows, cols]
     assert_gemm_close(got, ref, mag, "sampled")
 
 
 @pytest.mark.parametrize("li", [0, 1, 2])
 def test_llama_full_size_sampled(li):
-    L = wl.workload("llama7b")[li]
+    L = wl.workload("llama7b")[li]  # layer seeds 0, 10, 20
     d = wl.make_layer(L)
     Wd, Xd, idxd = to_dev(d.W), to_dev(d.X), to_dev_i32(d.idx)
     vals, meta = nm.prune_compress(Wd, 2, 4)
@@ -273,7 +279,7 @@ def test_decode_full_size_sampled():
 
 @pytest.mark.parametrize("li", [0, 1])
 def test_vit_full_size_sampled(li):
-    L = wl.workload("vit")[li]
+    L = wl.workload("vit")[li]  # layer seeds 0, 10
     d = wl.make_layer(L)
     vals, meta = nm.prune_compress(to_dev(d.W), 1, 8)
     Y = nm.spmm(vals, meta, 1, 8, L.K, to_dev(d.X))

@@ -166,6 +166,69 @@ def test_tiled_2of4_every_group_once():
     assert np.all(pos_wide[R:] == np.tile([0, 1], 64))
 
 
+# The 64 words of one tiled 2:4 metadata block (16 rows x 128 columns), written
+# out by hand from the layout description: lane l = 0..15 holds rows l mod 8
+# (bits 0-15) and 8 + l mod 8 (bits 16-31); its word q = 0..3 covers the
+# 16 columns starting at 32q + 16 (l / 8); four nibbles per row half, in column
+# order.  Entry: (row in bits 0-15, row in bits 16-31, first column).
+TILED_BLOCK_WORDS = [
+    (0, 8, 0), (0, 8, 32), (0, 8, 64), (0, 8, 96),           # words 0-3, lane 0
+    (1, 9, 0), (1, 9, 32), (1, 9, 64), (1, 9, 96),           # words 4-7, lane 1
+    (2, 10, 0), (2, 10, 32), (2, 10, 64), (2, 10, 96),       # words 8-11, lane 2
+    (3, 11, 0), (3, 11, 32), (3, 11, 64), (3, 11, 96),       # words 12-15, lane 3
+    (4, 12, 0), (4, 12, 32), (4, 12, 64), (4, 12, 96),       # words 16-19, lane 4
+    (5, 13, 0), (5, 13, 32), (5, 13, 64), (5, 13, 96),       # words 20-23, lane 5
+    (6, 14, 0), (6, 14, 32), (6, 14, 64), (6, 14, 96),       # words 24-27, lane 6
+    (7, 15, 0), (7, 15, 32), (7, 15, 64), (7, 15, 96),       # words 28-31, lane 7
+    (0, 8, 16), (0, 8, 48), (0, 8, 80), (0, 8, 112),         # words 32-35, lane 8
+    (1, 9, 16), (1, 9, 48), (1, 9, 80), (1, 9, 112),         # words 36-39, lane 9
+    (2, 10, 16), (2, 10, 48), (2, 10, 80), (2, 10, 112),     # words 40-43, lane 10
+    (3, 11, 16), (3, 11, 48), (3, 11, 80), (3, 11, 112),     # words 44-47, lane 11
+    (4, 12, 16), (4, 12, 48), (4, 12, 80), (4, 12, 112),     # words 48-51, lane 12
+    (5, 13, 16), (5, 13, 48), (5, 13, 80), (5, 13, 112),     # words 52-55, lane 13
+    (6, 14, 16), (6, 14, 48), (6, 14, 80), (6, 14, 112),     # words 56-59, lane 14
+    (7, 15, 16), (7, 15, 48), (7, 15, 80), (7, 15, 112),     # words 60-63, lane 15
+]
+
+
+def _slot_from_table(r, g):
+    """(word, bit) of group g (columns 4g..4g+3) of row r inside one block, by table lookup."""
+    hits = [(w, 16 * (r == hi) + 4 * ((4 * g - c) // 4))
+            for w, (lo, hi, c) in enumerate(TILED_BLOCK_WORDS) if r in (lo, hi) and c <= 4 * g < c + 16]
+    assert len(hits) == 1
+    return hits[0]
+
+
+def _planted_slot(R, K, r, g):
+    """Compress a matrix that is zero except group g of row r = [0, 0, 1, 1]
+    (positions 2, 3: nibble 0xE); every other group is all-zero (nibble 0x4).
+    Returns the (word, bit) of the only 0xE nibble."""
+    W = np.zeros((R, K), np.uint16)
+    W[r, 4 * g + 2:4 * g + 4] = bits_of([1.0, 1.0])
+    _, meta = oracle.compress(W, 2, 4)
+    nib = (meta[:, None] >> (4 * np.arange(8))) & 0xF
+    assert np.count_nonzero(nib == 0xE) == 1 and np.count_nonzero(nib == 0x4) == nib.size - 1
+    w, j = np.argwhere(nib == 0xE)[0]
+    return int(w), int(4 * j)
+
+
+def test_tiled_2of4_slot_map_matches_hand_table():
+    """Every (row, group) of one block lands at the word and bit of the hand-written table."""
+    for r in range(16):
+        for g in range(32):
+            assert _planted_slot(16, 128, r, g) == _slot_from_table(r, g), (r, g)
+
+
+@pytest.mark.parametrize("r,g", [(21, 67), (16, 0), (31, 95), (3, 40), (30, 33)])
+def test_tiled_2of4_block_order(r, g):
+    """Blocks follow one another row block by row block: block (rb, cb) of a
+    32 x 384 matrix (three 128-column blocks per row block) starts at word
+    (3 rb + cb) * 64."""
+    rb, cb = r // 16, g // 32
+    w, bit = _slot_from_table(r % 16, g % 32)
+    assert _planted_slot(32, 384, r, g) == ((3 * rb + cb) * 64 + w, bit)
+
+
 # ---------------------------------------------------------------------------
 # Decompression
 # ---------------------------------------------------------------------------
