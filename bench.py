@@ -48,6 +48,8 @@ def parse_args(argv=None):
     ap.add_argument("--cpu-seconds", type=float, default=10.0, help="target length of the oracle baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-configs", action="store_true",
+                    help="skip the pass over the other configurations (decode, ViT, PATCH, RL-MLP, tiny)")
     ap.add_argument("--workload", default=WORKLOAD, choices=wl.ALL_WORKLOADS,
                     help="llama7b (default, the headline), decode, vit, patch_p25/p50/p75, tiny, rl_mlp_*")
     ap.add_argument("--layers", default=None, help="comma-separated subset of the workload's layers")
@@ -150,34 +152,67 @@ class ClockSampler:
 
 
 # ----------------------------------------------------------------------------
-# Oracle baseline (CPU)
+# Oracle baseline (CPU): the oracle as it stands, its rows spread over threads
 # ----------------------------------------------------------------------------
-def oracle_sample(d, rows: int, cols: int):
-    """Oracle compress of `rows` weight rows and its permuted GEMM over `cols` tokens."""
+def host_threads() -> int:
+    """Host cores this process may run on."""
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+def cpu_model() -> str:
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
+def oracle_sample(d, r0: int, r1: int, cols: int):
+    """Oracle compress of weight rows r0..r1-1 and their permuted GEMM over the first `cols` tokens."""
     import oracle
     L = d.layer
     Xs = np.ascontiguousarray(d.X[:, :cols])
-    t0 = time.perf_counter()
-    vals, meta = oracle.compress(np.ascontiguousarray(d.W[:rows]), 2, 4)
+    vals, meta = oracle.compress(np.ascontiguousarray(d.W[r0:r1]), 2, 4)
     oracle.spmm(vals, meta, 2, 4, L.K, Xs, d.idx)
-    dt = time.perf_counter() - t0
-    flops = 2.0 * rows * cols * (L.K // 2)
-    return flops, dt
+    return 2.0 * (r1 - r0) * cols * (L.K // 2)
+
+
+def oracle_parallel(d, rows: int, cols: int, threads: int):
+    """Rows 0..rows-1 split into `threads` contiguous blocks, one oracle call pair per thread (the
+    oracle's C functions run without the GIL).  Returns (useful FLOPs, seconds)."""
+    from concurrent.futures import ThreadPoolExecutor
+    bounds = np.linspace(0, rows, threads + 1).astype(int)
+    blocks = [(int(a), int(b)) for a, b in zip(bounds[:-1], bounds[1:]) if b > a]
+    t0 = time.perf_counter()
+    with ThreadPoolExecutor(max_workers=len(blocks)) as ex:
+        flops = sum(ex.map(lambda ab: oracle_sample(d, ab[0], ab[1], cols), blocks))
+    return flops, time.perf_counter() - t0
 
 
 def cpu_baseline(data, target_s: float):
+    """The oracle on all of this host's cores, on a sample of the first layer sized for ~target_s seconds."""
     d = data[0]
-    f0, t0 = oracle_sample(d, 16, 16)
-    rate = f0 / max(t0, 1e-9)
-    # scale the sample to about target_s seconds of single-thread oracle work
-    side = int(np.sqrt(max(target_s * rate / (2.0 * (d.layer.K // 2)), 256.0)))
-    rows = int(min(max(side, 16), d.layer.R))
-    cols = int(min(max(side, 16), d.layer.T))
-    flops, dt = oracle_sample(d, rows, cols)
-    return {"value": flops / dt / 1e12, "unit": "TFLOP/s", "cores": 1, "kind": "oracle",
-            "sample": f"{d.layer.name}: oracle compress of {rows} weight rows + permuted spmm of those rows "
-                      f"over {cols} of {d.layer.T} tokens ({flops / 1e9:.2f} useful GFLOP, {dt:.1f} s, "
-                      f"single thread)"}
+    L = d.layer
+    threads = host_threads()
+    f0, t0 = oracle_parallel(d, 16, 16, 1)
+    rate = f0 / max(t0, 1e-9)                      # one thread
+    want = target_s * rate * threads               # FLOPs for about target_s seconds on every core
+    cols = int(min(L.T, 512))
+    rows = int(min(L.R, max(threads, want / (2.0 * cols * (L.K // 2)))))
+    if rows == L.R:
+        cols = int(min(L.T, max(cols, want / (2.0 * rows * (L.K // 2)))))
+    flops, dt = oracle_parallel(d, rows, cols, threads)
+    return {"value": flops / dt / 1e12, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+            "cpu_model": cpu_model(),
+            "sample": f"{L.name}: oracle compress of {rows} weight rows + permuted spmm of those rows over "
+                      f"{cols} of {L.T} tokens ({flops / 1e9:.2f} useful GFLOP, {dt:.1f} s wall, rows split "
+                      f"over {threads} threads)"}
 
 
 # ----------------------------------------------------------------------------
@@ -198,29 +233,68 @@ def max_over_ranks_on(ms: float, dist, device) -> float:
     return float(t.item())
 
 
+def layer_mode(L, step_mode: str, algo: str, permuted: bool) -> str:
+    """How a layer of the step runs (mirrors the library's dispatch for nm_prune_spmm), and what the
+    kernel-timing pass brackets: "fused" the whole call (prune_spmm_skinny_kernel + reduction);
+    "combined" the pair GEMM on the gathered input, the launch the call makes after its compress-and-gather
+    grid; "split" the GEMM call after a separate compress."""
+    one_call = step_mode == "one-call" and L.tile_p is None and algo == "auto"
+    if one_call and L.n == 2 and L.m == 4 and L.K % 128 == 0:
+        if 1 <= L.T <= 64:
+            return "fused"
+        if permuted and L.T >= 192 and L.T % 8 == 0:
+            return "combined"
+    return "split"
+
+
+def step_config(workload: str, layers, step_mode: str, algo: str, plain: bool, world: int) -> dict:
+    """The `config` object of a bench line (the same for both arms)."""
+    permuted = [L.permuted and not plain for L in layers]
+    one_call = step_mode == "one-call" and all(L.tile_p is None for L in layers) and algo == "auto"
+    ws = sum(2 * L.R * L.K + 2 * L.K * L.T + 2 * L.R * L.T for L in layers)
+    return {"workload": workload, "shapes": [[L.R, L.K] for L in layers], "T": [L.T for L in layers],
+            "pattern": [f"{L.n}:{L.m}" if L.tile_p is None else f"dense/2:4 tiles p={L.tile_p}" for L in layers],
+            "permuted": any(permuted), "algo": algo,
+            "step": ("one nm_prune_spmm call per layer: prune + compress (the compressed form written) + the sparse "
+                     "GEMM" if one_call else "nm_prune_compress, then the sparse GEMM call, for every layer"),
+            "layer_paths": {L.name: layer_mode(L, step_mode, algo, p) for L, p in zip(layers, permuted)},
+            "kernel_timing": ("CUDA events in a second pass of K steps: per layer the compress and the GEMM launch "
+                              "(\"combined\": the pair GEMM on the gathered input, the launch nm_prune_spmm makes "
+                              "after its compress-and-gather grid; \"fused\": the whole call)"),
+            "l2": ("inputs larger than L2 (126 MB) per step" if ws > 126e6
+                   else "working set below L2 size (small config)"),
+            "parallelism": f"replicas x{world}"}
+
+
 def run_reference(args, rank: int, world: int):
+    """The oracle on the host's cores: each step a bounded sample of the workload's first layer."""
     if rank != 0:
         return
-    data = [wl.make_layer(L) for L in wl.workload(WORKLOAD)]
-    d = data[0]
-    rows, cols = 48, 64  # bounded sample per step
+    layers = wl.workload(args.workload)
+    if args.layers:
+        layers = [layers[int(i)] for i in args.layers.split(",")]
+    d = wl.make_layer(layers[0])
+    threads = host_threads()
+    rows, cols = int(min(d.layer.R, 8 * threads)), 64  # bounded sample per step
     for _ in range(args.warmup):
-        oracle_sample(d, rows, cols)
+        oracle_parallel(d, rows, cols, threads)
     t = 0.0
     flops = 0.0
     for _ in range(args.steps):
-        f, dt = oracle_sample(d, rows, cols)
+        f, dt = oracle_parallel(d, rows, cols, threads)
         t += dt
         flops += f
     value = flops / t / 1e12
-    cfg = {"workload": f"{WORKLOAD}_2of4_permuted", "shapes": [[L.layer.R, L.layer.K] for L in data],
-           "T": d.layer.T, "pattern": "2:4", "sample_per_step": f"{rows} rows x {cols} tokens of {d.layer.name}"}
+    cfg = step_config(args.workload, layers, args.step, args.algo, args.plain, world)
+    sample = (f"per step {rows} weight rows x {cols} tokens of {d.layer.name}: oracle compress + permuted spmm, "
+              f"rows split over {threads} threads")
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * t / args.steps,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-            "data": "synthetic", "config": cfg,
-            "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": 1, "kind": "oracle",
-                             "sample": cfg["sample_per_step"]},
+            "data": "synthetic (seeded numpy PCG64 draws rounded to bf16; shapes and distributions of the workload)",
+            "config": cfg,
+            "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+                             "cpu_model": cpu_model(), "sample": sample},
             "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
@@ -240,6 +314,259 @@ def gemm_bytes(L, d) -> float:
     return b
 
 
+class Runner:
+    """Device buffers and library calls (through the C ABI) of one workload's step."""
+
+    def __init__(self, workload, dev, stream, nm, algo="auto", layers=None, plain=False, step_mode="one-call"):
+        import torch
+        self.torch, self.nm, self.L_ = torch, nm, nm.lib()
+        self.dev, self.stream, self.sp = dev, stream, stream.cuda_stream
+        self.algo_name = algo
+        self.algo = {"auto": nm.NM_ALGO_AUTO, "sparse": nm.NM_ALGO_SPARSE_TC, "dense": nm.NM_ALGO_DENSE_TC}[algo]
+        lay = wl.workload(workload)
+        if layers:
+            lay = [lay[int(i)] for i in layers.split(",")]
+        self.layers = lay
+        self.data = [wl.make_layer(L) for L in lay]
+        self.one_call = step_mode == "one-call" and all(d.tmap is None for d in self.data) and algo == "auto"
+        self.bufs = []
+        for d in self.data:
+            L = d.layer
+            b = {"L": L, "d": d, "W": self.up(d.W), "X": self.up(d.X),
+                 "idx": torch.from_numpy(d.idx).to(dev) if d.idx is not None and not plain else None,
+                 "tmap": torch.from_numpy(d.tmap).to(dev) if d.tmap is not None else None,
+                 "vals": torch.empty((L.R, max(nm.nm_value_cols(L.K, L.n, L.m), 0)), dtype=torch.bfloat16,
+                                     device=dev),
+                 "meta": torch.empty((max(nm.nm_meta_words(L.R, L.K, L.n, L.m), 0),), dtype=torch.int32, device=dev),
+                 "Y": torch.empty((L.R, L.T), dtype=torch.bfloat16, device=dev)}
+            b["flops"] = float(wl.hybrid_useful_flops(d) if d.tmap is not None else L.useful_flops)
+            b["comp_bytes"] = 2.0 * L.R * L.K + 2.0 * b["vals"].numel() + 4.0 * b["meta"].numel()
+            b["mode"] = layer_mode(L, step_mode, algo, b["idx"] is not None)
+            if b["mode"] == "combined":
+                b["Xp"] = b["X"][b["idx"].long()].contiguous()  # input of the timed GEMM launch (setup only)
+            if b["mode"] == "fused":  # W read once, compressed form written, X read, Y written
+                b["gemm_bytes"] = b["comp_bytes"] + 2.0 * L.K * L.T + 2.0 * L.R * L.T
+            elif b["mode"] == "combined":  # the GEMM reads the gathered input: no index map
+                b["gemm_bytes"] = gemm_bytes(L, d) - 4.0 * L.K
+            else:
+                b["gemm_bytes"] = gemm_bytes(L, d)
+            self.bufs.append(b)
+        torch.cuda.synchronize()
+        self.useful = sum(b["flops"] for b in self.bufs)
+
+    def up(self, bits):
+        return self.torch.from_numpy(bits.view(np.int16)).to(self.dev).view(self.torch.bfloat16)
+
+    def check(self, st, what):
+        if st != 0:
+            raise RuntimeError(f"{what}: {self.L_.nm_last_error().decode()}")
+
+    def launch_compress(self, b):
+        L = b["L"]
+        self.check(self.L_.nm_prune_compress(b["W"].data_ptr(), L.R, L.K, L.K, L.n, L.m, b["vals"].data_ptr(),
+                                             b["meta"].data_ptr(), self.sp), "nm_prune_compress")
+
+    def launch_gemm(self, b, permuted=True):
+        L, L_, sp = b["L"], self.L_, self.sp
+        if b["tmap"] is not None:
+            self.check(L_.nm_hybrid_spmm(b["W"].data_ptr(), L.K, b["vals"].data_ptr(), b["meta"].data_ptr(),
+                                         b["tmap"].data_ptr(), L.tile, L.R, L.K, b["X"].data_ptr(), L.T, L.T,
+                                         b["Y"].data_ptr(), L.T, 0, sp), "nm_hybrid_spmm")
+        elif b["idx"] is not None and permuted:
+            self.check(L_.nm_spmm_permuted(b["vals"].data_ptr(), b["meta"].data_ptr(), L.n, L.m, L.R, L.K,
+                                           b["idx"].data_ptr(), b["X"].data_ptr(), L.T, L.T, b["Y"].data_ptr(), L.T,
+                                           0, sp), "nm_spmm_permuted")
+        elif self.algo != self.nm.NM_ALGO_AUTO:
+            self.check(L_.nm_spmm_algo(b["vals"].data_ptr(), b["meta"].data_ptr(), L.n, L.m, L.R, L.K, None,
+                                       b["X"].data_ptr(), L.T, L.T, b["Y"].data_ptr(), L.T, 0, self.algo, sp),
+                       "nm_spmm_algo")
+        else:
+            self.check(L_.nm_spmm(b["vals"].data_ptr(), b["meta"].data_ptr(), L.n, L.m, L.R, L.K, b["X"].data_ptr(),
+                                  L.T, L.T, b["Y"].data_ptr(), L.T, 0, sp), "nm_spmm")
+
+    def launch_fused(self, b, permuted=True):
+        L = b["L"]
+        idx = b["idx"].data_ptr() if b["idx"] is not None and permuted else None
+        self.check(self.L_.nm_prune_spmm(b["W"].data_ptr(), L.K, L.n, L.m, L.R, L.K, idx, b["X"].data_ptr(), L.T,
+                                         L.T, b["Y"].data_ptr(), L.T, 0, b["vals"].data_ptr(), b["meta"].data_ptr(),
+                                         self.sp), "nm_prune_spmm")
+
+    def launch_gemm_xp(self, b):
+        L = b["L"]
+        self.check(self.L_.nm_spmm(b["vals"].data_ptr(), b["meta"].data_ptr(), 2, 4, L.R, L.K, b["Xp"].data_ptr(),
+                                   L.T, L.T, b["Y"].data_ptr(), L.T, 0, self.sp), "nm_spmm")
+
+    def launch_layer(self, b):  # one layer of the timed step
+        if self.one_call:
+            self.launch_fused(b)
+        else:
+            self.launch_compress(b)
+            self.launch_gemm(b)
+
+    def step(self, evs=None):
+        """The step; with events, the kernel-timing form of it (see layer_mode)."""
+        for i, b in enumerate(self.bufs):
+            if evs is None:
+                self.launch_layer(b)
+                continue
+            evs[2 * i].record(self.stream)
+            if b["mode"] == "fused":  # the whole call; the compress slot stays empty
+                evs[2 * i + 1].record(self.stream)
+                self.launch_fused(b)
+                continue
+            self.launch_compress(b)
+            evs[2 * i + 1].record(self.stream)
+            if b["mode"] == "combined":
+                self.launch_gemm_xp(b)
+            else:
+                self.launch_gemm(b)
+        if evs is not None:
+            evs[2 * len(self.bufs)].record(self.stream)
+
+    def gemm_only(self):
+        """The step's GEMM launches alone (the dominant kernel of every workload)."""
+        for b in self.bufs:
+            if b["mode"] == "fused":
+                self.launch_fused(b)
+            elif b["mode"] == "combined":
+                self.launch_gemm_xp(b)
+            else:
+                self.launch_gemm(b)
+
+    def compress_only(self):
+        for b in self.bufs:
+            self.launch_compress(b)
+
+    def timed(self, fn, reps, warm=2):
+        """Milliseconds per call of fn(), CUDA events on the launching stream around `reps` back-to-back calls."""
+        torch = self.torch
+        for _ in range(warm):
+            fn()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(self.stream)
+        for _ in range(reps):
+            fn()
+        e1.record(self.stream)
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / reps
+
+    def kernels(self, comp_ms, gemm_ms, tc_peak, hbm_peak):
+        out = {}
+        for i, b in enumerate(self.bufs):
+            L = b["L"]
+            t_tc = b["flops"] / (tc_peak * 1e12)
+            t_hbm = b["gemm_bytes"] / (hbm_peak * 1e9)
+            k = {"gemm_us": 1e3 * gemm_ms[i],
+                 "gemm_tflops": b["flops"] / (gemm_ms[i] * 1e-3) / 1e12,
+                 "gemm_gbs": b["gemm_bytes"] / (gemm_ms[i] * 1e-3) / 1e9,
+                 "gemm_bound": "tensor" if t_tc >= t_hbm else "hbm",
+                 "gemm_frac": max(t_tc, t_hbm) / (gemm_ms[i] * 1e-3),
+                 "timed": {"fused": "the nm_prune_spmm call", "combined": "spmm_pair_kernel on the gathered input",
+                           "split": "the GEMM call"}[b["mode"]]}
+            if comp_ms is not None:
+                k["compress_us"] = 1e3 * comp_ms[i]
+                if b["mode"] != "fused":
+                    k["compress_gbs"] = b["comp_bytes"] / (comp_ms[i] * 1e-3) / 1e9
+                    k["compress_frac"] = k["compress_gbs"] / hbm_peak
+            out[L.name] = k
+        return out
+
+    def roofline(self, gemm_step_ms, tc_peak, hbm_peak, peak_note):
+        """Roofline of the step's GEMM launches together: useful FLOPs against the dense bf16 peak (2:4 useful
+        FLOPs run at half the sparse-MMA rate, i.e. at most at the dense rate) or algorithmic bytes against the
+        HBM copy bandwidth, whichever bound is slower."""
+        flops_all = sum(b["flops"] for b in self.bufs)
+        bytes_all = sum(b["gemm_bytes"] for b in self.bufs)
+        gsec = gemm_step_ms * 1e-3
+        tensor_bound = flops_all / (tc_peak * 1e12) >= bytes_all / (hbm_peak * 1e9)
+        if tensor_bound:
+            achieved, peak, unit = flops_all / gsec / 1e12, tc_peak, "TFLOP/s"
+        else:
+            achieved, peak, unit = bytes_all / gsec / 1e9, hbm_peak, "GB/s"
+        modes = {b["mode"] for b in self.bufs}
+        kernel = ("nm_prune_spmm call: prune_spmm_skinny_kernel + split-K reduction" if modes == {"fused"} else
+                  "spmm_pair_kernel (tcgen05 2-SM GEMM) on the gathered input, as launched by nm_prune_spmm"
+                  if modes == {"combined"} else
+                  "the GEMM call (nm_spmm_permuted: gather_rows_kernel + spmm_pair_kernel, or nm_spmm / "
+                  "nm_hybrid_spmm)")
+        return {"bound": "tensor" if tensor_bound else "hbm", "achieved": achieved, "peak": peak, "unit": unit,
+                "frac": achieved / peak, "traffic": None, "kernel": kernel,
+                "peak_source": peak_note if tensor_bound else "measured HBM copy bandwidth",
+                "algorithmic_per_launch": [b["flops"] if tensor_bound else b["gemm_bytes"] for b in self.bufs],
+                "gemm_step_us": 1e3 * gemm_step_ms}
+
+
+EXTRA_CONFIGS = ["decode", "vit", "patch_p25", "patch_p50", "patch_p75", "rl_mlp_2of4", "rl_mlp_1of4",
+                 "rl_mlp_1of8", "tiny"]
+
+
+def measure_config(name, args, dev, stream, nm, peaks, world):
+    """One further configuration of the pages' workloads: the step timed back to back (CUDA events around
+    enough steps for >= 20 ms), the GEMM launches alone for `roofline`, the compress calls alone, and the
+    per-layer event pass.  Inputs stay resident in HBM."""
+    torch = __import__("torch")
+    r = Runner(name, dev, stream, nm)
+    tc_peak, hbm_peak = peaks["bf16_tflops"], peaks["hbm_gbs"]
+    est = r.timed(r.step, 3, warm=3)
+    reps = int(min(2000, max(args.steps, 20.0 / max(est, 1e-4))))
+    launches0 = nm.nm_launch_count()
+    ms = r.timed(r.step, reps, warm=0)
+    launches = (nm.nm_launch_count() - launches0) / reps
+    greps = int(min(2000, max(args.steps, 20.0 / max(r.timed(r.gemm_only, 3), 1e-4))))
+    gemm_step_ms = r.timed(r.gemm_only, greps)
+    comp_ms_step = None if r.one_call and all(b["mode"] == "fused" for b in r.bufs) else \
+        r.timed(r.compress_only, greps)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(2 * len(r.bufs) + 1)] for _ in range(20)]
+    for e in evs:
+        r.step(e)
+    torch.cuda.synchronize()
+    comp_ms = np.zeros(len(r.bufs))
+    gemm_ms = np.zeros(len(r.bufs))
+    for e in evs:
+        for i in range(len(r.bufs)):
+            comp_ms[i] += e[2 * i].elapsed_time(e[2 * i + 1]) / len(evs)
+            gemm_ms[i] += e[2 * i + 1].elapsed_time(e[2 * i + 2]) / len(evs)
+    nm.nm_device_status(r.sp)
+    roof = r.roofline(gemm_step_ms, tc_peak, hbm_peak, "measured bf16 burst dense peak")
+    roof["timing"] = f"CUDA events around {greps} back-to-back repetitions of the step's GEMM launches"
+    out = {"value": world * r.useful / (ms * 1e-3) / 1e12, "unit": "TFLOP/s", "ms_per_step": ms,
+           "steps": reps, "gpu_launches_per_step": launches,
+           "config": step_config(name, r.layers, "one-call", "auto", False, world),
+           "roofline": roof, "kernels": r.kernels(comp_ms if comp_ms_step is not None else None, gemm_ms,
+                                                  tc_peak, hbm_peak)}
+    if comp_ms_step is not None:
+        cb = sum(b["comp_bytes"] for b in r.bufs)
+        out["compress_roofline"] = {"bound": "hbm", "achieved": cb / (comp_ms_step * 1e-3) / 1e9, "peak": hbm_peak,
+                                    "unit": "GB/s", "frac": cb / (comp_ms_step * 1e-3) / 1e9 / hbm_peak,
+                                    "compress_step_us": 1e3 * comp_ms_step}
+    if name in ("tiny",) or name.startswith("rl_mlp"):
+        out["latency_us"] = 1e3 * ms
+        out["note"] = ("launch-latency-bound: the roofline bound is well under a microsecond; the step time is "
+                       "host call overhead and launch latency")
+    if any(b["mode"] == "fused" for b in r.bufs):
+        # the two-call design's GEMM (nm_spmm on the compressed operand, the split-K skinny kernel): the
+        # decode-batch GEMM whose HBM fraction the pages' shape targets
+        two = r.timed(lambda: [r.launch_gemm(b) for b in r.bufs], greps)
+        gb = sum(gemm_bytes(b["L"], b["d"]) for b in r.bufs)
+        out["gemm_call_roofline"] = {"bound": "hbm", "achieved": gb / (two * 1e-3) / 1e9, "peak": hbm_peak,
+                                     "unit": "GB/s", "frac": gb / (two * 1e-3) / 1e9 / hbm_peak,
+                                     "kernel": "nm_spmm: spmm_skinny_kernel + split-K reduction",
+                                     "call_us": 1e3 * two}
+    if name == "vit":
+        # executed MACs of the re-encoded 2:4 design: every 1:8 survivor rides in a 2:4 pair, 4x the useful
+        # products at the sparse rate (2x the dense rate)
+        ex = sum(4.0 * b["flops"] for b in r.bufs)
+        t_exec = max(ex / 2.0 / (tc_peak * 1e12), sum(b["gemm_bytes"] for b in r.bufs) / (hbm_peak * 1e9))
+        out["roofline_reencoded"] = {"t_bound_us": 1e6 * t_exec, "frac": t_exec / (gemm_step_ms * 1e-3),
+                                     "note": "max(executed 2:4 MACs at the sparse rate, algorithmic bytes at "
+                                             "the HBM rate) over the step's GEMM launches"}
+    del r
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+    return out
+
+
 def run_ours(args, rank: int, world: int, dist):
     import torch
     import sparse_gemm_nm_b200 as nm
@@ -248,114 +575,9 @@ def run_ours(args, rank: int, world: int, dist):
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
     stream = torch.cuda.current_stream(dev)
-    sp = stream.cuda_stream
-    L_ = nm.lib()
-    algo = {"auto": nm.NM_ALGO_AUTO, "sparse": nm.NM_ALGO_SPARSE_TC, "dense": nm.NM_ALGO_DENSE_TC}[args.algo]
-
-    layers = wl.workload(args.workload)
-    if args.layers:
-        layers = [layers[int(i)] for i in args.layers.split(",")]
-    data = [wl.make_layer(L) for L in layers]
-
-    def up(bits):
-        return torch.from_numpy(bits.view(np.int16)).to(dev).view(torch.bfloat16)
-
-    one_call = args.step == "one-call" and all(d.tmap is None for d in data) and args.algo == "auto"
-    bufs = []
-    for d in data:
-        L = d.layer
-        b = {"L": L, "d": d, "W": up(d.W), "X": up(d.X),
-             "idx": torch.from_numpy(d.idx).to(dev) if d.idx is not None and not args.plain else None,
-             "tmap": torch.from_numpy(d.tmap).to(dev) if d.tmap is not None else None,
-             "vals": torch.empty((L.R, max(nm.nm_value_cols(L.K, L.n, L.m), 0)), dtype=torch.bfloat16, device=dev),
-             "meta": torch.empty((max(nm.nm_meta_words(L.R, L.K, L.n, L.m), 0),), dtype=torch.int32, device=dev),
-             "Y": torch.empty((L.R, L.T), dtype=torch.bfloat16, device=dev)}
-        b["flops"] = float(wl.hybrid_useful_flops(d) if d.tmap is not None else L.useful_flops)
-        b["comp_bytes"] = 2.0 * L.R * L.K + 2.0 * b["vals"].numel() + 4.0 * b["meta"].numel()
-        # How nm_prune_spmm runs the layer (mirrors the library's dispatch), and what the kernel-timing
-        # pass brackets with events: "fused" the whole call (prune_spmm_skinny_kernel + reduction);
-        # "combined" the pair GEMM on the gathered input, the same launch the call makes after its
-        # compress-and-gather grid; "split" the GEMM call after a separate compress.
-        b["mode"] = "split"
-        if one_call and L.n == 2 and L.m == 4 and L.K % 128 == 0:
-            if 1 <= L.T <= 64:
-                b["mode"] = "fused"
-            elif b["idx"] is not None and L.T >= 192 and L.T % 8 == 0:
-                b["mode"] = "combined"
-                b["Xp"] = b["X"][b["idx"].long()].contiguous()  # input of the timed GEMM launch (setup only)
-        if b["mode"] == "fused":  # W read once, compressed form written, X read, Y written
-            b["gemm_bytes"] = b["comp_bytes"] + 2.0 * L.K * L.T + 2.0 * L.R * L.T
-        elif b["mode"] == "combined":  # the GEMM reads the gathered input: no index map
-            b["gemm_bytes"] = gemm_bytes(L, d) - 4.0 * L.K
-        else:
-            b["gemm_bytes"] = gemm_bytes(L, d)
-        bufs.append(b)
-    torch.cuda.synchronize()
-
-    def check(st, what):
-        if st != 0:
-            raise RuntimeError(f"{what}: {L_.nm_last_error().decode()}")
-
-    def launch_compress(b):
-        L = b["L"]
-        check(L_.nm_prune_compress(b["W"].data_ptr(), L.R, L.K, L.K, L.n, L.m, b["vals"].data_ptr(),
-                                   b["meta"].data_ptr(), sp), "nm_prune_compress")
-
-    def launch_gemm(b, permuted=True):
-        L = b["L"]
-        if b["tmap"] is not None:
-            check(L_.nm_hybrid_spmm(b["W"].data_ptr(), L.K, b["vals"].data_ptr(), b["meta"].data_ptr(),
-                                    b["tmap"].data_ptr(), L.tile, L.R, L.K, b["X"].data_ptr(), L.T, L.T,
-                                    b["Y"].data_ptr(), L.T, 0, sp), "nm_hybrid_spmm")
-        elif b["idx"] is not None and permuted:
-            check(L_.nm_spmm_permuted(b["vals"].data_ptr(), b["meta"].data_ptr(), L.n, L.m, L.R, L.K,
-                                      b["idx"].data_ptr(), b["X"].data_ptr(), L.T, L.T, b["Y"].data_ptr(), L.T, 0,
-                                      sp), "nm_spmm_permuted")
-        elif algo != nm.NM_ALGO_AUTO:
-            check(L_.nm_spmm_algo(b["vals"].data_ptr(), b["meta"].data_ptr(), L.n, L.m, L.R, L.K, None,
-                                  b["X"].data_ptr(), L.T, L.T, b["Y"].data_ptr(), L.T, 0, algo, sp), "nm_spmm_algo")
-        else:
-            check(L_.nm_spmm(b["vals"].data_ptr(), b["meta"].data_ptr(), L.n, L.m, L.R, L.K, b["X"].data_ptr(),
-                             L.T, L.T, b["Y"].data_ptr(), L.T, 0, sp), "nm_spmm")
-
-    def launch_fused(b, permuted=True):
-        L = b["L"]
-        idx = b["idx"].data_ptr() if b["idx"] is not None and permuted else None
-        check(L_.nm_prune_spmm(b["W"].data_ptr(), L.K, L.n, L.m, L.R, L.K, idx, b["X"].data_ptr(), L.T, L.T,
-                               b["Y"].data_ptr(), L.T, 0, b["vals"].data_ptr(), b["meta"].data_ptr(), sp),
-              "nm_prune_spmm")
-
-    def launch_gemm_xp(b):
-        L = b["L"]
-        check(L_.nm_spmm(b["vals"].data_ptr(), b["meta"].data_ptr(), 2, 4, L.R, L.K, b["Xp"].data_ptr(), L.T, L.T,
-                         b["Y"].data_ptr(), L.T, 0, sp), "nm_spmm")
-
-    def launch_layer(b):  # one layer of the timed step
-        if one_call:
-            launch_fused(b)
-        else:
-            launch_compress(b)
-            launch_gemm(b)
-
-    def step(evs=None):
-        """The step; with events, the kernel-timing form of it (see b["mode"])."""
-        for i, b in enumerate(bufs):
-            if evs is None:
-                launch_layer(b)
-                continue
-            evs[2 * i].record(stream)
-            if b["mode"] == "fused":  # the whole call; the compress slot stays empty
-                evs[2 * i + 1].record(stream)
-                launch_fused(b)
-                continue
-            launch_compress(b)
-            evs[2 * i + 1].record(stream)
-            if b["mode"] == "combined":
-                launch_gemm_xp(b)
-            else:
-                launch_gemm(b)
-        if evs is not None:
-            evs[2 * len(bufs)].record(stream)
+    r = Runner(args.workload, dev, stream, nm, algo=args.algo, layers=args.layers, plain=args.plain,
+               step_mode=args.step)
+    bufs, sp = r.bufs, r.sp
 
     def barrier():
         rank_barrier(dist)
@@ -363,10 +585,9 @@ def run_ours(args, rank: int, world: int, dist):
     def max_over_ranks(ms):
         return max_over_ranks_on(ms, dist, dev)
 
-    useful = sum(b["flops"] for b in bufs)
-
+    useful = r.useful
     for _ in range(args.warmup):
-        step()
+        r.step()
     torch.cuda.synchronize()
     nm.nm_device_status(sp)
 
@@ -389,60 +610,45 @@ def run_ours(args, rank: int, world: int, dist):
     t_end = torch.cuda.Event(enable_timing=True)
     t_start.record(stream)
     for k in range(args.steps):
-        step()
+        r.step()
     t_end.record(stream)
     torch.cuda.synchronize()
     barrier()
     launches = nm.nm_launch_count() - launches0
     for k in range(args.steps):  # second pass: per-kernel events
-        step(evs[k])
+        r.step(evs[k])
     torch.cuda.synchronize()
     barrier()
 
     # Third pass, for `roofline`: the GEMM launches of the step alone, back to back, no events between them
     # (the step's layers together exceed L2, so every launch reads its operands from HBM).
-    def gemm_only():
-        for b in bufs:
-            if b["mode"] == "fused":
-                launch_fused(b)
-            elif b["mode"] == "combined":
-                launch_gemm_xp(b)
-            else:
-                launch_gemm(b)
-
     greps = max(10, min(args.steps, 200))
     for _ in range(2):
-        gemm_only()
+        r.gemm_only()
     torch.cuda.synchronize()
     barrier()
     g0, g1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     g0.record(stream)
     for _ in range(greps):
-        gemm_only()
+        r.gemm_only()
     g1.record(stream)
     torch.cuda.synchronize()
     barrier()
     gemm_only_ms = max_over_ranks(g0.elapsed_time(g1)) / greps
 
     # Fourth pass, for `compress_roofline`: the step's compress calls (nm_prune_compress) alone, back to back.
-    def compress_only():
-        for b in bufs:
-            launch_compress(b)
-
     for _ in range(2):
-        compress_only()
+        r.compress_only()
     torch.cuda.synchronize()
     barrier()
     c0, c1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     c0.record(stream)
     for _ in range(greps):
-        compress_only()
+        r.compress_only()
     c1.record(stream)
     torch.cuda.synchronize()
     barrier()
     compress_only_ms = max_over_ranks(c0.elapsed_time(c1)) / greps
-    if sampler:
-        sampler.stop()
     nm.nm_device_status(sp)
 
     elapsed_ms = max_over_ranks(t_start.elapsed_time(t_end))
@@ -466,32 +672,17 @@ def run_ours(args, rank: int, world: int, dist):
     sustained = loaded_ms > 1000.0
     tc_peak = peaks["bf16_tflops_sustained" if sustained else "bf16_tflops"]
     hbm_peak = peaks["hbm_gbs"]
-    kernels = {}
-    for i, b in enumerate(bufs):
-        L = b["L"]
-        t_tc = b["flops"] / (tc_peak * 1e12)
-        t_hbm = b["gemm_bytes"] / (hbm_peak * 1e9)
-        kernels[L.name] = {
-            "gemm_us": 1e3 * gemm_ms[i],
-            "gemm_tflops": b["flops"] / (gemm_ms[i] * 1e-3) / 1e12,
-            "gemm_gbs": b["gemm_bytes"] / (gemm_ms[i] * 1e-3) / 1e9,
-            "gemm_bound": "tensor" if t_tc >= t_hbm else "hbm",
-            "gemm_frac": max(t_tc, t_hbm) / (gemm_ms[i] * 1e-3),
-            "compress_us": 1e3 * comp_ms[i], "timed": {
-                "fused": "the nm_prune_spmm call", "combined": "spmm_pair_kernel on the gathered input",
-                "split": "the GEMM call"}[b["mode"]]}
-        if b["mode"] != "fused":
-            kernels[L.name]["compress_gbs"] = b["comp_bytes"] / (comp_ms[i] * 1e-3) / 1e9
-            kernels[L.name]["compress_frac"] = kernels[L.name]["compress_gbs"] / hbm_peak
-
-    # dominant kernel: the GEMM (all launches of the step together)
-    flops_all = sum(b["flops"] for b in bufs)
-    bytes_all = sum(b["gemm_bytes"] for b in bufs)
-    gsec = gemm_only_ms * 1e-3  # the GEMM launches of one step, timed back to back (third pass)
-    tensor_bound = flops_all / (tc_peak * 1e12) >= bytes_all / (hbm_peak * 1e9)
+    kernels = r.kernels(comp_ms, gemm_ms, tc_peak, hbm_peak)
+    roofline = r.roofline(gemm_only_ms, tc_peak, hbm_peak,
+                          f"{peak_src} bf16 {'sustained' if sustained else 'burst'} dense peak ({loaded_ms:.0f} ms "
+                          "of unbroken load up to the end of the roofline pass); useful 2:4 FLOPs run at half the "
+                          "sparse-MMA rate, i.e. at the dense rate")
+    roofline["timing"] = (f"CUDA events around {greps} back-to-back repetitions of the step's GEMM launches "
+                          "(one per layer, no events between them); per-layer event-bracketed times are in `kernels`")
+    if roofline["bound"] == "hbm":
+        roofline["peak_source"] = f"{peak_src} HBM copy bandwidth"
     # DRAM bytes (read + write) of the GEMM call's kernels per layer, from one ncu capture
     # (profiles/<workload>_gemm_traffic.json); summed over the step like `achieved`.
-    traffic = None
     tfile = os.path.join(ROOT, "profiles", f"{args.workload}_gemm_traffic.json")
     if os.path.exists(tfile) and args.algo == "auto" and all(b["mode"] != "fused" for b in bufs):
         with open(tfile) as f:
@@ -500,43 +691,9 @@ def run_ours(args, rank: int, world: int, dist):
         kinds = [("spmm_pair_kernel",) if b["mode"] == "combined" else ("spmm_pair_kernel", "gather_rows_kernel")
                  for b in bufs]
         if all(n in per and all(k in per[n] for k in ks) for n, ks in zip(names, kinds)):
-            traffic = sum(sum(per[n][k] for k in ks) for n, ks in zip(names, kinds))
-    if tensor_bound:
-        achieved, peak, unit = flops_all / gsec / 1e12, tc_peak, "TFLOP/s"
-        src = (f"{peak_src} bf16 {'sustained' if sustained else 'burst'} dense peak ({loaded_ms:.0f} ms of "
-               "unbroken load up to the end of the roofline pass); useful 2:4 FLOPs run at half the sparse-MMA "
-               "rate, i.e. at the dense rate")
-    else:
-        achieved, peak, unit = bytes_all / gsec / 1e9, hbm_peak, "GB/s"
-        src = f"{peak_src} HBM copy bandwidth"
-    roofline = {"bound": "tensor" if tensor_bound else "hbm", "achieved": achieved, "peak": peak, "unit": unit,
-                "frac": achieved / peak, "traffic": traffic,
-                "kernel": ("nm_prune_spmm call: prune_spmm_skinny_kernel + split-K reduction"
-                           if all(b["mode"] == "fused" for b in bufs) else
-                           "spmm_pair_kernel (tcgen05 2-SM GEMM) on the gathered input, as launched by nm_prune_spmm"
-                           if all(b["mode"] == "combined" for b in bufs) else
-                           "the GEMM call (nm_spmm_permuted: gather_rows_kernel + spmm_pair_kernel, or nm_spmm / "
-                           "nm_hybrid_spmm)"),
-                "peak_source": src,
-                "algorithmic_per_launch": [b["flops"] if tensor_bound else b["gemm_bytes"] for b in bufs],
-                "timing": (f"CUDA events around {greps} back-to-back repetitions of the step's GEMM launches "
-                           "(one per layer, no events between them); per-layer event-bracketed times are in "
-                           "`kernels`"),
-                "gemm_step_us": 1e3 * gemm_only_ms}
+            roofline["traffic"] = sum(sum(per[n][k] for k in ks) for n, ks in zip(names, kinds))
 
-    cfg = {"workload": args.workload, "shapes": [[b["L"].R, b["L"].K] for b in bufs],
-           "T": [b["L"].T for b in bufs], "pattern": [f"{b['L'].n}:{b['L'].m}" for b in bufs],
-           "permuted": any(b["idx"] is not None for b in bufs), "algo": args.algo,
-           "step": ("one nm_prune_spmm call per layer: prune + compress (the compressed form written) + the sparse "
-                    "GEMM" if one_call else "nm_prune_compress, then the sparse GEMM call, for every layer"),
-           "layer_paths": {b["L"].name: b["mode"] for b in bufs},
-           "kernel_timing": ("CUDA events in a second pass of K steps: per layer the compress and the GEMM launch "
-                             "(\"combined\": the pair GEMM on the gathered input, the launch nm_prune_spmm makes "
-                             "after its compress-and-gather grid; \"fused\": the whole call)"),
-           "l2": "inputs larger than L2 (126 MB) per step" if sum(
-               b["W"].numel() * 2 + b["X"].numel() * 2 + b["Y"].numel() * 2 for b in bufs) > 126e6
-           else "working set below L2 size (small config)",
-           "parallelism": f"replicas x{world}"}
+    cfg = step_config(args.workload, r.layers, args.step, args.algo, args.plain, world)
     comp_bytes_all = sum(b["comp_bytes"] for b in bufs)
     comp_gbs = comp_bytes_all / (compress_only_ms * 1e-3) / 1e9
     compress_roofline = {"bound": "hbm", "achieved": comp_gbs, "peak": hbm_peak, "unit": "GB/s",
@@ -549,8 +706,7 @@ def run_ours(args, rank: int, world: int, dist):
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic (seeded numpy PCG64 draws rounded to bf16; shapes and distributions of the workload)",
             "config": cfg, "roofline": roofline, "compress_roofline": compress_roofline, "kernels": kernels,
-            "gpu_launches": launches,
-            "clocks": sampler.summary() if sampler else None}
+            "gpu_launches": launches}
 
     if not args.quick and any(b["idx"] is not None for b in bufs) and all(b["tmap"] is None for b in bufs):
         # cost of the index-map read: per layer the GEMM call with the map (nm_spmm_permuted: gather pass +
@@ -559,18 +715,8 @@ def run_ours(args, rank: int, world: int, dist):
         over = {}
         for b in bufs:
             L = b["L"]
-            res = {}
-            for name, permuted in (("permuted", True), ("plain", False)):
-                for _ in range(3):
-                    launch_gemm(b, permuted)
-                torch.cuda.synchronize()
-                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-                e0.record(stream)
-                for _ in range(reps):
-                    launch_gemm(b, permuted)
-                e1.record(stream)
-                torch.cuda.synchronize()
-                res[name] = e0.elapsed_time(e1) / reps
+            res = {name: r.timed(lambda: r.launch_gemm(b, permuted), reps, warm=3)
+                   for name, permuted in (("permuted", True), ("plain", False))}
             t_bound = max(b["flops"] / (tc_peak * 1e12), gemm_bytes(L, b["d"]) / (hbm_peak * 1e9))
             over[L.name] = {"plain_us": 1e3 * res["plain"], "permuted_us": 1e3 * res["permuted"],
                             "overhead": res["permuted"] / res["plain"] - 1.0,
@@ -585,29 +731,22 @@ def run_ours(args, rank: int, world: int, dist):
         # timed in event-free loops of the same calls; dense tensor-core FLOPs 2 R K T per call
         reps = max(10, min(50, args.steps))
         back = {}
+        L_ = r.L_
         for i, b in enumerate(bufs):
             L = b["L"]
-            dY = up(wl.normal_bf16((L.R, L.T), 1.0, seed=100 + i))
+            dY = r.up(wl.normal_bf16((L.R, L.T), 1.0, seed=100 + i))
             dX = torch.empty((L.K, L.T), dtype=torch.bfloat16, device=dev)
             dV = torch.empty((L.R, L.K // 2), dtype=torch.bfloat16, device=dev)
             idx = b["idx"].data_ptr() if b["idx"] is not None else None
             calls = {
-                "spmm_t": lambda: check(L_.nm_spmm_t(b["vals"].data_ptr(), b["meta"].data_ptr(), 2, 4, L.R, L.K, idx,
-                                                     dY.data_ptr(), L.T, L.T, dX.data_ptr(), L.T, 0, sp), "nm_spmm_t"),
-                "sddmm": lambda: check(L_.nm_sddmm(b["meta"].data_ptr(), 2, 4, L.R, L.K, idx, dY.data_ptr(), L.T,
-                                                   b["X"].data_ptr(), L.T, L.T, dV.data_ptr(), 0, sp), "nm_sddmm")}
+                "spmm_t": lambda: r.check(L_.nm_spmm_t(b["vals"].data_ptr(), b["meta"].data_ptr(), 2, 4, L.R, L.K,
+                                                       idx, dY.data_ptr(), L.T, L.T, dX.data_ptr(), L.T, 0, sp),
+                                          "nm_spmm_t"),
+                "sddmm": lambda: r.check(L_.nm_sddmm(b["meta"].data_ptr(), 2, 4, L.R, L.K, idx, dY.data_ptr(), L.T,
+                                                     b["X"].data_ptr(), L.T, L.T, dV.data_ptr(), 0, sp), "nm_sddmm")}
             res = {}
             for name, fn in calls.items():
-                for _ in range(3):
-                    fn()
-                torch.cuda.synchronize()
-                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-                e0.record(stream)
-                for _ in range(reps):
-                    fn()
-                e1.record(stream)
-                torch.cuda.synchronize()
-                us = e0.elapsed_time(e1) / reps * 1e3
+                us = r.timed(fn, reps, warm=3) * 1e3
                 tflops = 2.0 * L.R * L.K * L.T / (us * 1e-6) / 1e12
                 res[name] = {"us": us, "dense_tflops": tflops, "frac": tflops / tc_peak}
             back[L.name] = res
@@ -650,7 +789,7 @@ def run_ours(args, rank: int, world: int, dist):
                 stream.wait_event(copied[i])
                 if started[i]:
                     stream.wait_event(returned[i])  # Y of the previous step has been read back
-                launch_layer(b)
+                r.launch_layer(b)
                 computed[i].record(stream)
                 with torch.cuda.stream(s_d2h):
                     s_d2h.wait_event(computed[i])
@@ -677,8 +816,26 @@ def run_ours(args, rank: int, world: int, dist):
                        "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                        "ms_per_step": e_ms / args.e2e_steps,
                        "overlap": "per-layer H2D / compute / D2H on three streams, chained by events"}
+
+    # The pages' other configurations, each measured on its own (same clocks sampler), each with its
+    # own roofline.  Every rank measures them (identical collective-free work); rank 0 reports.
+    if not args.quick and not args.no_configs and args.workload == WORKLOAD and args.algo == "auto" \
+            and not args.layers and not args.plain and args.step == "one-call":
+        data_host = r.data
+        del r, bufs
+        torch.cuda.empty_cache()
+        configs = {}
+        for name in EXTRA_CONFIGS:
+            barrier()
+            configs[name] = measure_config(name, args, dev, stream, nm, peaks, world)
+        line["configs"] = configs
+    else:
+        data_host = r.data
+    if sampler:
+        sampler.stop()
+    line["clocks"] = sampler.summary() if sampler else None
     if rank == 0 and world == 1 and not args.quick and not args.no_cpu_baseline and args.workload == "llama7b":
-        line["cpu_baseline"] = cpu_baseline(data, args.cpu_seconds)
+        line["cpu_baseline"] = cpu_baseline(data_host, args.cpu_seconds)
     elif rank == 0:
         line["cpu_baseline"] = None
     if rank == 0:

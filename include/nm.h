@@ -430,12 +430,19 @@ NM_API nm_status nm_selftest_wait_timeout(uint32_t limit_us, void* stream);
  * the gathered input X[idx[k]] in a buffer taken from a library-owned memory
  * pool on `stream`; this call stages it instead in a fixed 32 MiB array inside the
  * library, which every device that loads the library holds until the process
- * exits, and works through the columns of X in chunks that fit it.  Results
- * match nm_spmm_permuted.  Arguments and errors as nm_spmm_permuted, plus:
+ * exits, and works through the columns of X in chunks that fit it (chunks of
+ * floor(16 Mi / K / 256) * 256 columns, one gather and one GEMM launch each).
+ * For 2:4, columns that a two-SM chunk serves are bit-identical to
+ * nm_spmm_permuted's; a last chunk of fewer than 192 columns runs on the one-SM
+ * kernel, and other patterns always do, so those agree with nm_spmm_permuted
+ * within the GEMM tolerance (different summation order).  Arguments and
+ * errors as nm_spmm_permuted (the same checks), plus:
  *  - NM_ERR_UNSUPPORTED when K > 65536 on the two-SM path (a 256-column chunk
  *    of K rows must fit the array);
  *  - the first call on each device looks up the array's device address
- *    (cudaGetSymbolAddress); make that first call before any stream capture;
+ *    (cudaGetSymbolAddress) and keeps it for the life of the process; make
+ *    that first call before any stream capture, and do not use the call
+ *    after cudaDeviceReset on that device (the kept address would be stale);
  *  - all calls share the one array and each leaves its last chunk in it: calls
  *    that may overlap on the GPU (different streams, or other host threads)
  *    race and must be serialised by the caller.  Nothing in the array needs to

@@ -109,6 +109,111 @@ __global__ void __launch_bounds__(256, 4) compress_2of4_tiled_kernel(const uint1
   }
 }
 
+// Row-wise patterns with whole 16-byte pieces (K % 8 == 0, 16-byte aligned
+// rows): 1:2, 1:4, 3:4, 1:8, 2:8, 3:8, 4:8.  Lanes read consecutive 16-byte
+// pieces of one row (a warp load is 512 contiguous bytes); a piece is 8/M
+// groups for M <= 8.  Each group keeps its N largest combined keys
+// (magnitude key, then the lower index: key << log2(M) | (M - 1 - i), all
+// distinct), found by N rounds of a max over the group; the kept positions
+// are then emitted in ascending order.  A work unit is one row and one span of
+// groups whose survivors fill whole metadata words (UNITS pieces per lane);
+// every lane parks its survivors' position codes in shared memory, and after
+// a warp barrier each lane ORs the codes of its own words (S codes of b bits)
+// and stores them.  Value stores are 2-byte per survivor, contiguous across the
+// warp.
+template <int M, int N>
+struct RowwisePlan {
+  static constexpr int B = M == 2 ? 1 : M == 4 ? 2 : 3;        // position bits
+  static constexpr int S = 32 / B;                              // positions per word
+  static constexpr int G = 8 / M;                               // groups per 16-byte piece
+  static constexpr int PER_PIECE = G * N;                       // survivors per piece
+  static constexpr int gcd(int a, int b) { return b == 0 ? a : gcd(b, a % b); }
+  static constexpr int BASE = S / gcd(S, 32 * PER_PIECE);       // pieces per lane to fill whole words
+  static constexpr int UNITS = BASE >= 4 ? BASE : BASE * ((4 + BASE - 1) / BASE);  // >= 4 loads in flight
+  static constexpr int SURV = 32 * PER_PIECE * UNITS;           // survivors per work unit
+  static constexpr int WORDS = SURV / S;                        // metadata words per work unit
+  static constexpr int GROUPS = 32 * G * UNITS;                 // groups per work unit
+};
+
+template <int M, int N>
+__global__ void __launch_bounds__(256) compress_rowwise_warp_kernel(const uint16_t* __restrict__ W, int64_t R,
+                                                                    int64_t K, int64_t ldw,
+                                                                    uint16_t* __restrict__ V,
+                                                                    uint32_t* __restrict__ meta) {
+  using P = RowwisePlan<M, N>;
+  static_assert(P::SURV % P::S == 0, "a work unit must fill whole words");
+  constexpr int LOGM = M == 2 ? 1 : M == 4 ? 2 : 3;
+  __shared__ uint8_t codes[8][P::SURV];
+  pdl_gate();
+  const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
+  const int64_t ngroups = K / M;
+  const int64_t vcols = ngroups * N;
+  const int64_t mcols = (vcols + P::S - 1) / P::S;
+  const int64_t units_per_row = (ngroups + P::GROUPS - 1) / P::GROUPS;
+  const int64_t units = R * units_per_row;
+  const int64_t nwarps = (int64_t)gridDim.x * (blockDim.x >> 5);
+  uint8_t* my = codes[wib];
+  for (int64_t u = (int64_t)blockIdx.x * (blockDim.x >> 5) + wib; u < units; u += nwarps) {
+    const int64_t row = u / units_per_row;
+    const int64_t g0 = (u - row * units_per_row) * P::GROUPS;  // first group of the unit
+    const uint16_t* wrow = W + row * ldw;
+    uint4 in[P::UNITS];
+#pragma unroll
+    for (int i = 0; i < P::UNITS; ++i) {
+      const int64_t g = g0 + (int64_t)(i * 32 + lane) * P::G;
+      in[i] = g < ngroups ? __ldg(reinterpret_cast<const uint4*>(wrow + g * M)) : make_uint4(0, 0, 0, 0);
+    }
+#pragma unroll
+    for (int i = 0; i < P::UNITS; ++i) {
+      const int piece = i * 32 + lane;
+      const int64_t gp = g0 + (int64_t)piece * P::G;
+      const uint32_t w4[4] = {in[i].x, in[i].y, in[i].z, in[i].w};
+#pragma unroll
+      for (int gg = 0; gg < P::G; ++gg) {
+        uint32_t ck[M];
+#pragma unroll
+        for (int e = 0; e < M; ++e) {
+          const int flat = gg * M + e;  // element of the piece
+          const uint32_t b16 = (w4[flat >> 1] >> (16 * (flat & 1))) & 0xFFFFu;
+          ck[e] = (mag_key(b16) << LOGM) | (uint32_t)(M - 1 - e);
+        }
+        uint32_t keep = 0;  // bit e: element e survives
+#pragma unroll
+        for (int t = 0; t < N; ++t) {
+          uint32_t best = 0;
+#pragma unroll
+          for (int e = 0; e < M; ++e) best = max(best, (keep >> e) & 1u ? 0u : ck[e]);
+          keep |= 1u << (M - 1 - (best & (M - 1)));
+        }
+        const bool valid = gp + gg < ngroups;
+        const int64_t j0 = (gp + gg) * N;  // first survivor of the group in the row
+        const int sc0 = (piece * P::G + gg) * N;  // its slot in the unit
+#pragma unroll
+        for (int t = 0; t < N; ++t) {
+          const uint32_t p = __ffs(keep) - 1u;
+          keep &= keep - 1u;
+          const int flat = gg * M + (int)p;
+          const uint32_t word = (flat >> 1) == 0 ? w4[0] : (flat >> 1) == 1 ? w4[1] : (flat >> 1) == 2 ? w4[2] : w4[3];
+          if (valid) V[row * vcols + j0 + t] = (uint16_t)((word >> (16 * (flat & 1))) & 0xFFFFu);
+          my[sc0 + t] = valid ? (uint8_t)p : (uint8_t)0;
+        }
+      }
+    }
+    __syncwarp();
+    const int64_t w0 = (g0 * N) / P::S;  // first word of the unit (units start on word boundaries)
+#pragma unroll
+    for (int w = lane; w < P::WORDS; w += 32) {
+      if (w0 + w < mcols) {
+        uint32_t word = 0;
+#pragma unroll
+        for (int j = 0; j < P::S; ++j) word |= (uint32_t)my[w * P::S + j] << (P::B * j);
+        meta[row * mcols + w0 + w] = word;
+      }
+    }
+    __syncwarp();
+  }
+}
+
 // Generic path: one thread per metadata word.  The thread re-derives the
 // selection of every group its survivors belong to (a group may straddle two
 // words when S is not a multiple of N) and writes only its own survivors.
@@ -347,6 +452,11 @@ static int grid_for(int64_t work, int threads) {
 
 static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+// Row-wise patterns served by compress_rowwise_warp_kernel.
+static bool rowwise_warp_pattern(int n, int m) {
+  return (m == 2 && n == 1) || (m == 4 && (n == 1 || n == 3)) || (m == 8 && n >= 1 && n <= 4);
+}
+
 cudaError_t launch_compress(const uint16_t* W, int64_t R, int64_t K, int64_t ldw, int n, int m, uint16_t* values,
                             uint32_t* meta, cudaStream_t s) {
   const int threads = 256;
@@ -355,6 +465,21 @@ cudaError_t launch_compress(const uint16_t* W, int64_t R, int64_t K, int64_t ldw
     const bool vec = K % 8 == 0 && ldw % 8 == 0 && aligned16(W) && aligned16(values);
     launch_pdl(compress_2of4_tiled_kernel, grid_for(nblocks * 32, threads), threads, 0, s,
         W, (uint32_t)R, (uint32_t)K, ldw, values, meta, (uint32_t)meta_col_blocks(K), (uint32_t)nblocks, vec);
+  } else if (K % 8 == 0 && ldw % 8 == 0 && aligned16(W) && rowwise_warp_pattern(n, m)) {
+    // one warp per work unit (a row's span of groups filling whole words); 8 warps per block
+    auto units = [&](int groups) { return R * ((K / m + groups - 1) / groups); };
+    auto go = [&](auto kernel, int groups) {
+      const int64_t want = (units(groups) + 7) / 8;
+      const int64_t cap = (int64_t)sm_count_current() * 8;
+      launch_pdl(kernel, (int)(want < cap ? (want > 0 ? want : 1) : cap), threads, 0, s, W, R, K, ldw, values, meta);
+    };
+    if (n == 1 && m == 2) go(compress_rowwise_warp_kernel<2, 1>, RowwisePlan<2, 1>::GROUPS);
+    else if (n == 1 && m == 4) go(compress_rowwise_warp_kernel<4, 1>, RowwisePlan<4, 1>::GROUPS);
+    else if (n == 3 && m == 4) go(compress_rowwise_warp_kernel<4, 3>, RowwisePlan<4, 3>::GROUPS);
+    else if (n == 1 && m == 8) go(compress_rowwise_warp_kernel<8, 1>, RowwisePlan<8, 1>::GROUPS);
+    else if (n == 2 && m == 8) go(compress_rowwise_warp_kernel<8, 2>, RowwisePlan<8, 2>::GROUPS);
+    else if (n == 3 && m == 8) go(compress_rowwise_warp_kernel<8, 3>, RowwisePlan<8, 3>::GROUPS);
+    else go(compress_rowwise_warp_kernel<8, 4>, RowwisePlan<8, 4>::GROUPS);
   } else {
     const int64_t work = R * meta_cols(K, n, m);
     const int grid = grid_for(work, threads);

@@ -25,6 +25,9 @@ namespace nmk {
 
 void set_last_error(const char* msg);
 bool pair_path_for(int n, int m, int64_t R, int64_t K, int64_t T, const void* values, const void* meta);
+nm_status check_permuted_args(const uint16_t* values, const uint32_t* meta, int n, int m, int64_t R, int64_t K,
+                              const int32_t* idx, const uint16_t* X, int64_t ldx, int64_t T, void* Y, int64_t ldy,
+                              nm_out_dtype y_dtype);
 nm_status spmm_permuted_unstaged(const uint16_t* values, const uint32_t* meta, int n, int m, int64_t R, int64_t K,
                                  const int32_t* idx, const uint16_t* X, int64_t ldx, int64_t T, void* Y,
                                  int64_t ldy, nm_out_dtype y_dtype, cudaStream_t stream);
@@ -80,25 +83,10 @@ extern "C" NM_API nm_status nm_spmm_permuted_noalloc(const uint16_t* values, con
   if (!pair_path_for(n, m, R, K, T, values, meta) || R <= 0 || K <= 0 || T <= 0)
     return spmm_permuted_unstaged(values, meta, n, m, R, K, idx, X, ldx, T, Y, ldy, y_dtype,
                                   static_cast<cudaStream_t>(stream));
-  set_last_error("");
-  if (!idx || !X || !Y || !values || !meta) {
-    set_last_error("null pointer");
-    return NM_ERR_INVALID_ARG;
-  }
-  if (y_dtype != NM_OUT_BF16 && y_dtype != NM_OUT_F32) {
-    set_last_error("bad output dtype");
-    return NM_ERR_INVALID_ARG;
-  }
+  // The same checks, statuses and texts as nm_spmm_permuted.
+  nm_status st = check_permuted_args(values, meta, n, m, R, K, idx, X, ldx, T, Y, ldy, y_dtype);
+  if (st != NM_OK) return st;
   const int esize = y_dtype == NM_OUT_F32 ? 4 : 2;
-  if (ldx < T || ldy < T) {
-    set_last_error("leading dimension smaller than T");
-    return NM_ERR_INVALID_ARG;
-  }
-  if ((reinterpret_cast<uintptr_t>(X) & 15u) || ldx % 8 || (reinterpret_cast<uintptr_t>(Y) & 15u) ||
-      (ldy * esize) % 16) {
-    set_last_error("X and Y rows must be 16-byte aligned");
-    return NM_ERR_MISALIGNED;
-  }
   // Each chunk stages K rows x `chunk` columns; chunks are multiples of 256
   // columns, so at least one 256-column chunk must fit.
   const int64_t chunk = kNoAllocScratchElems / K / 256 * 256;
@@ -111,21 +99,30 @@ extern "C" NM_API nm_status nm_spmm_permuted_noalloc(const uint16_t* values, con
     return NM_ERR_UNSUPPORTED;
   }
   uint16_t* scratch = nullptr;
-  nm_status st = scratch_for_current_device(&scratch);
+  st = scratch_for_current_device(&scratch);
   if (st != NM_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   // The array keeps whatever the previous call left; every element a chunk
   // reads is written by that chunk's gather first, so nothing is cleared.
   for (int64_t t0 = 0; t0 < T; t0 += chunk) {
     const int64_t tc = (T - t0 < chunk) ? T - t0 : chunk;
+    uint8_t* y0 = static_cast<uint8_t*>(Y) + t0 * esize;
+    if (!pair_path_for(n, m, R, K, tc, values, meta)) {
+      // A last chunk too narrow for the two-SM kernel (fewer than 192
+      // columns): the one-SM kernel reads its mapped rows of X itself and
+      // stages nothing.  t0 is a multiple of 256, so X + t0 and y0 stay
+      // 16-byte aligned.
+      st = spmm_permuted_unstaged(values, meta, n, m, R, K, idx, X + t0, ldx, tc, y0, ldy, y_dtype, s);
+      if (st != NM_OK) return st;
+      continue;
+    }
     cudaError_t e = launch_gather_rows(X + t0, ldx, idx, K, tc, scratch, tc, s);
     if (e != cudaSuccess) {
       set_last_error(cudaGetErrorString(e));
       return NM_ERR_CUDA;
     }
     SpmmParams p;
-    st = build_pair_params(p, values, meta, R, K, scratch, tc, tc, static_cast<uint8_t*>(Y) + t0 * esize, ldy,
-                           y_dtype == NM_OUT_F32);
+    st = build_pair_params(p, values, meta, R, K, scratch, tc, tc, y0, ldy, y_dtype == NM_OUT_F32);
     if (st != NM_OK) return st;
     e = launch_spmm_pair(p, s);
     if (e != cudaSuccess) {

@@ -132,3 +132,53 @@ def test_selection_exhaustive_alphabet():
     _, fv, fm = nm.prune_spmm(to_dev(W), 2, 4, X, keep_compressed=True)
     torch.cuda.synchronize()
     assert np.array_equal(bits(fv), ov) and np.array_equal(words(fm), om)
+
+
+# ----------------------------------------------------------------------------
+# Row-wise patterns (warp kernel on aligned rows, per-word kernel otherwise)
+# ----------------------------------------------------------------------------
+def _alphabet_rows(alphabet, m, groups_per_row):
+    import itertools
+    groups = np.array(list(itertools.product(alphabet, repeat=m)), np.uint16)
+    pad = (-len(groups)) % groups_per_row
+    groups = np.concatenate([groups, np.zeros((pad, m), np.uint16)])
+    return groups.reshape(-1, groups_per_row * m)
+
+
+ALPHA12 = [0x0000, 0x8000, 0x3F80, 0xBF80, 0x3F81, 0x7F80, 0xFF80, 0x7FC0, 0xFFC1, 0x7F81, 0x0001, 0x8001]
+ZERO_ONE_TWO = [0x0000, 0x3F80, 0x4000]       # {0, 1, 2}
+ZERO_MINUS_ONE_TWO = [0x0000, 0xBF80, 0x4000]  # {0, -1, 2}
+
+
+@pytest.mark.parametrize("n,m,alphabet", [(1, 8, ZERO_ONE_TWO), (2, 8, ZERO_ONE_TWO), (3, 8, ZERO_ONE_TWO),
+                                          (4, 8, ZERO_ONE_TWO), (1, 8, ZERO_MINUS_ONE_TWO),
+                                          (2, 8, ZERO_MINUS_ONE_TWO), (1, 4, ALPHA12), (3, 4, ALPHA12),
+                                          (1, 2, ALPHA12)])
+def test_rowwise_selection_exhaustive_alphabet(n, m, alphabet):
+    """Every group of M over the alphabet ({0,1,2}^8 = 6561 groups of eight with their ties; the 12-value
+    alphabet with NaN payloads, +-0, +-Inf and denormals for M = 4 and 2): the warp kernel (aligned rows) and
+    the per-word kernel (row stride not a multiple of 8) both select exactly as the oracle."""
+    W = _alphabet_rows(alphabet, m, 81 if m == 8 else 32)
+    ov, om = oracle.compress(W, n, m)
+    v, mt = gpu_compress(W, n, m)
+    assert np.array_equal(v, ov) and np.array_equal(mt, om)
+    v, mt = gpu_compress(W, n, m, ldw=W.shape[1] + 4)
+    assert np.array_equal(v, ov) and np.array_equal(mt, om)
+
+
+@pytest.mark.parametrize("n,m", [(1, 8), (2, 8), (1, 4)])
+@pytest.mark.parametrize("R,K", [(7, 8), (3, 1032), (2, 10 * 8 * 33), (200, 5128)])
+def test_rowwise_unit_tails(n, m, R, K):
+    """Rows whose group count leaves a partial work unit and a partial last metadata word."""
+    W = wl.normal_bf16((R, K), 1.0, seed=K + n)
+    ov, om = oracle.compress(W, n, m)
+    v, mt = gpu_compress(W, n, m)
+    assert np.array_equal(v, ov) and np.array_equal(mt, om)
+
+
+def test_compress_1of8_large_weight():
+    """A 13824 x 5120 weight (141.6 MB) at 1:8, whole arrays compared."""
+    W = wl.normal_bf16((13824, 5120), 0.02, seed=30)
+    ov, om = oracle.compress(W, 1, 8)
+    v, mt = gpu_compress(W, 1, 8)
+    assert np.array_equal(v, ov) and np.array_equal(mt, om)
