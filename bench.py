@@ -18,6 +18,7 @@ times the fp64 CPU oracle on a bounded sample of the same workload.
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import json
 import os
 import statistics
@@ -56,6 +57,8 @@ def parse_args(argv=None):
     ap.add_argument("--algo", choices=["auto", "sparse", "dense"], default="auto",
                     help="kernel design for 1:4 / 1:8 (nm_spmm_algo)")
     ap.add_argument("--plain", action="store_true", help="ignore the workload's index map (y = W x)")
+    ap.add_argument("--pattern", default=None,
+                    help="N:M to use instead of the workload's own pattern (e.g. --workload decode --pattern 1:8)")
     ap.add_argument("--diag", action="store_true",
                     help="diagonal pattern at 90 %% sparsity (D = K/10 kept diagonals) on the workload's shapes: "
                          "nm_diag_prune_compress, then nm_diag_spmm with the index map, per layer")
@@ -317,7 +320,8 @@ def gemm_bytes(L, d) -> float:
 class Runner:
     """Device buffers and library calls (through the C ABI) of one workload's step."""
 
-    def __init__(self, workload, dev, stream, nm, algo="auto", layers=None, plain=False, step_mode="one-call"):
+    def __init__(self, workload, dev, stream, nm, algo="auto", layers=None, plain=False, step_mode="one-call",
+                 pattern=None):
         import torch
         self.torch, self.nm, self.L_ = torch, nm, nm.lib()
         self.dev, self.stream, self.sp = dev, stream, stream.cuda_stream
@@ -326,6 +330,9 @@ class Runner:
         lay = wl.workload(workload)
         if layers:
             lay = [lay[int(i)] for i in layers.split(",")]
+        if pattern:
+            n, m = (int(x) for x in pattern.split(":"))
+            lay = [dataclasses.replace(L, n=n, m=m) for L in lay]
         self.layers = lay
         self.data = [wl.make_layer(L) for L in lay]
         self.one_call = step_mode == "one-call" and all(d.tmap is None for d in self.data) and algo == "auto"
@@ -576,7 +583,7 @@ def run_ours(args, rank: int, world: int, dist):
     dev = torch.device("cuda", local)
     stream = torch.cuda.current_stream(dev)
     r = Runner(args.workload, dev, stream, nm, algo=args.algo, layers=args.layers, plain=args.plain,
-               step_mode=args.step)
+               step_mode=args.step, pattern=args.pattern)
     bufs, sp = r.bufs, r.sp
 
     def barrier():
@@ -820,7 +827,7 @@ def run_ours(args, rank: int, world: int, dist):
     # The pages' other configurations, each measured on its own (same clocks sampler), each with its
     # own roofline.  Every rank measures them (identical collective-free work); rank 0 reports.
     if not args.quick and not args.no_configs and args.workload == WORKLOAD and args.algo == "auto" \
-            and not args.layers and not args.plain and args.step == "one-call":
+            and not args.layers and not args.plain and args.step == "one-call" and not args.pattern:
         data_host = r.data
         del r, bufs
         torch.cuda.empty_cache()
@@ -834,7 +841,8 @@ def run_ours(args, rank: int, world: int, dist):
     if sampler:
         sampler.stop()
     line["clocks"] = sampler.summary() if sampler else None
-    if rank == 0 and world == 1 and not args.quick and not args.no_cpu_baseline and args.workload == "llama7b":
+    if rank == 0 and world == 1 and not args.quick and not args.no_cpu_baseline and args.workload == "llama7b" \
+            and not args.pattern:
         line["cpu_baseline"] = cpu_baseline(data_host, args.cpu_seconds)
     elif rank == 0:
         line["cpu_baseline"] = None

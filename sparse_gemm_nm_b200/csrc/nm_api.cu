@@ -2,7 +2,6 @@
 // checks on the host, tensor-map encoding, choice of kernel variant, launch.
 #include <atomic>
 #include <cstdarg>
-#include <cmath>
 #include <cstdint>
 #include <cstdio>
 #include <cstring>
@@ -308,49 +307,6 @@ static nm_status check_gemm_operands(const GemmRequest& q) {
   return NM_OK;
 }
 
-// Stream-K for the SM-pair kernel.  With whole tiles per pair, a last wave of
-// num_tiles % pairs tiles leaves the other pairs idle (LLaMA 4096 x 11008 x 2048:
-// 128 tiles of 86 stages on 74 pairs run as two waves, 86 % busy).  Stream-K
-// gives every pair the same number of (tile, stage) units instead, at the cost
-// of one more accumulator hand-over per pair and the fp32 sum of split tiles.
-// Measured on B200: ~0.45 us per 128-deep stage and ~2 us per hand-over, so
-// the schedule is taken only where that model predicts at least 5 % less time
-// (long tiles; never for 4096 x 4096 x 2048, where the hand-overs eat the
-// gain), and only with at least one tile per pair (a tile then spans at most
-// two ranges).  `buf` receives the pool buffer to free after the launch.
-static nm_status setup_stream_k(SpmmParams& p, cudaMemPool_t& pool, void** buf, cudaStream_t stream) {
-  *buf = nullptr;
-  const int pairs = sm_count_current() / 2;
-  if (pairs < 2 || p.num_tiles < pairs || p.num_tiles % pairs == 0) return NM_OK;
-  const double k = (double)p.k_tiles, handover = 4.5;  // in stages
-  const double waves = (double)((p.num_tiles + pairs - 1) / pairs);
-  const double t_dp = waves * (k + handover);
-  const double per = (double)p.num_tiles * k / pairs;
-  const double t_sk = per + (std::ceil(per / k) + 2.0) * handover;
-  if (t_sk > 0.95 * t_dp) return NM_OK;
-  cudaError_t e = cudaSuccess;
-  if (!pool) e = staging_pool(&pool);
-  if (e != cudaSuccess) return cuda_fail(e, "staging pool");
-  const size_t ws_bytes = (size_t)pairs * 2 * 2 * 128 * 256 * 4;
-  const size_t cnt_bytes = (size_t)p.num_tiles * 2 * 4;
-  e = cudaMallocFromPoolAsync(buf, ws_bytes + cnt_bytes, pool, stream);
-  if (e != cudaSuccess) {
-    *buf = nullptr;
-    return cuda_fail(e, "stream-K workspace");
-  }
-  p.sk = 1;
-  p.sk_ws = static_cast<float*>(*buf);
-  p.sk_cnt = reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(*buf) + ws_bytes);
-  e = launch_fill_zero(p.sk_cnt, 1, p.num_tiles * 2, p.num_tiles * 2, 4, stream);
-  if (e != cudaSuccess) {
-    cudaFreeAsync(*buf, stream);
-    *buf = nullptr;
-    p.sk = 0;
-    return cuda_fail(e, "stream-K counter reset");
-  }
-  return NM_OK;
-}
-
 static nm_status run_gemm(const GemmRequest& q, cudaStream_t stream) {
   t_last_error.clear();
   nm_status st = check_gemm_shape(q);
@@ -448,10 +404,7 @@ static nm_status run_gemm(const GemmRequest& q, cudaStream_t stream) {
       st = make_tmap(&p.tm_wm, wm, (uint64_t)q.K, (uint64_t)q.R, (uint64_t)q.K * 2, 64, kPairBoxRows, 128, "W masked");
     if (st == NM_OK && !p.out_f32)
       st = make_tmap(&p.tm_y, q.Y, (uint64_t)q.T, (uint64_t)q.R, (uint64_t)q.ldy * 2, 64, 32, 128, "Y");
-    void* skbuf = nullptr;
-    if (st == NM_OK) st = setup_stream_k(p, pool, &skbuf, stream);
     if (st == NM_OK) e = launch_spmm_pair_hybrid(p, stream);
-    if (skbuf) cudaFreeAsync(skbuf, stream);
     cudaFreeAsync(wm, stream);
     if (st != NM_OK) return st;
     return e == cudaSuccess ? NM_OK : cuda_fail(e, "hybrid pair launch");
@@ -584,13 +537,10 @@ static nm_status run_gemm(const GemmRequest& q, cudaStream_t stream) {
     if (st == NM_OK && !dense_pair) st = make_meta_tmap(&p.tm_meta, meta, p.meta_rblocks, p.meta_cblocks);
     if (st == NM_OK && !use_skinny && !p.out_f32)
       st = make_tmap(&p.tm_y, q.Y, (uint64_t)q.T, (uint64_t)q.R, (uint64_t)q.ldy * 2, 64, 32, 128, "Y");
-    void* skbuf = nullptr;
-    if (st == NM_OK && !use_skinny) st = setup_stream_k(p, pool, &skbuf, stream);
     if (st == NM_OK)
       e = use_skinny   ? launch_spmm_skinny(p, stream)
           : dense_pair ? launch_spmm_pair_hybrid(p, stream)
                        : launch_spmm_pair(p, stream);
-    if (skbuf) cudaFreeAsync(skbuf, stream);
     if (ws) cudaFreeAsync(ws, stream);
     release();
     if (st != NM_OK) return st;

@@ -61,12 +61,6 @@ struct SpmmParams {
   // fused prune + compress + GEMM: optional outputs of the compressed operand
   uint16_t* out_vals;
   uint32_t* out_meta;
-  // SM-pair kernel, stream-K schedule: equal runs of (tile, 128-deep stage) units per
-  // pair; fp32 partials in sk_ws (2 slots per pair x 2 CTAs x 128 x 256), one arrival
-  // counter per (tile, CTA) in sk_cnt (zeroed before the launch)
-  int sk;
-  float* sk_ws;
-  uint32_t* sk_cnt;
 };
 
 // Dense bf16 GEMM on SM pairs for the backward products: C (M x N) = A (M x Kr) B (Kr x N),

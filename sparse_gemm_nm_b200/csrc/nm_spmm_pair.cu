@@ -26,6 +26,18 @@
 // copies E into TMEM (tcgen05.cp, both CTAs) and issues four tcgen05.mma.sp
 // (M = 256, N = 256, K = 32) per stage; its commits release the stage in both
 // CTAs.  Each CTA drains its own 128 x 256 fp32 accumulator.
+//
+// Short tiles (DB): a tile of few stages spends about as long handing its
+// accumulator over (MMA completion, TMEM drain, release) as computing it; on a
+// six-stage ViT tile a trace showed ~2.3 us of MMAs and ~1.6 us until the next
+// tile's first MMA.  Two accumulators let the next tile's MMAs run while the
+// epilogue drains, but two 256-column fp32 accumulators fill all 512 TMEM
+// columns and leave none for the sparse metadata.  So the DB form uses 256 x 192
+// tiles (each CTA supplies 96 columns of X: its first 64-column strip and half of
+// its second) and two 192-column accumulators (TMEM columns 0 and 256, metadata
+// from column 448).  It keeps four stages: a trace of the three-stage form on the
+// ViT shape showed the MMA thread waiting ~240 ns of each ~600 ns stage for data
+// (X rows 100 KB apart, a third of them from HBM).
 #include <cstdint>
 #include <cuda.h>
 #include <cuda_runtime.h>
@@ -40,9 +52,7 @@ namespace pair {
 constexpr int kThreads = 384;  // warps 0,2-5,10,11 copies; 1 MMA; 6-9 epilogue
 constexpr uint32_t kB = 32768, kE = 2048;
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kECol = 256;
 constexpr uint64_t kWaitNs = 2000000000ull;
-constexpr uint32_t kIdesc = idesc_bf16(256, true, 256);
 constexpr uint32_t kIdescDense = idesc_bf16(256, false, 256);
 constexpr uint32_t kEpi = 4096;  // per epilogue warp: 32 rows x 64 bf16 columns, 128-byte swizzle
 
@@ -52,85 +62,33 @@ struct Layout {
 // HYB = false: 2:4 only, A slots of 16 KB (compressed values), four stages.
 // HYB = true (PATCH hybrid): A slots of 32 KB so that a stage can hold the
 // dense 128 x 128 tile instead, three stages.
-// SHORT (2:4, few stages per tile): three stages, and four 4 KB staging
-// buffers per epilogue warp instead of one.  A warp's 32 x 256 bf16 output is
-// then written to shared memory while the accumulator drains and leaves as
-// four TMA stores issued together; with one buffer each 4 KB chunk waited for
-// the previous store to read it, a chain (~4 us) that a long tile hides behind
-// its MMAs but a six-stage tile (~2.8 us of MMAs) does not.
-template <bool HYB, bool SHORT = false>
+// DB = true (2:4, short tiles): 256 x 192 tiles, two accumulators, four stages.
+template <bool HYB, bool DB = false>
 struct Cfg {
-  static constexpr int kStages = (HYB || SHORT) ? 3 : 4;
-  static constexpr int kEpiBufs = SHORT ? 4 : 1;
+  static constexpr int kStages = HYB ? 3 : 4;
+  static constexpr uint32_t kN = DB ? 192u : 256u;  // pair tile columns (per CTA: kN / 2 of X)
+  static constexpr int kAcc = DB ? 2 : 1;           // accumulators, 256 TMEM columns apart
+  static constexpr uint32_t kECol = DB ? 448u : 256u;
+  static constexpr int kEpiBufs = 1;
+  static constexpr uint32_t kIdesc = idesc_bf16(kN, true, 256);
   static constexpr uint32_t kA = HYB ? 32768u : 16384u;
   static constexpr uint32_t kTxSparse = 2u * (16384u + kB + kE);  // both CTAs' A, B and E bytes
   static constexpr uint32_t kTxDense = 2u * (32768u + kB);        // both CTAs' dense A and B bytes
+  static constexpr uint32_t kBars = (2 * kStages + 6) * 8;        // full, empty, acc_full[2], acc_empty[2], spare[2]
   __host__ __device__ static constexpr Layout layout() {
     return Layout{0u, kStages * kA, kStages * (kA + kB), kStages * (kA + kB + kE),
                   kStages * (kA + kB + kE) + 4 * kEpiBufs * kEpi,
-                  kStages * (kA + kB + kE) + 4 * kEpiBufs * kEpi + (2 * kStages + 4) * 8 + 64};
+                  kStages * (kA + kB + kE) + 4 * kEpiBufs * kEpi + kBars + 64};
   }
-  static_assert(kStages * (kA + kB + kE) + 4 * kEpiBufs * kEpi + (2 * kStages + 4) * 8 + 64 + 1024 <= 232448,
-                "shared memory");
+  static_assert(kStages * (kA + kB + kE) + 4 * kEpiBufs * kEpi + kBars + 64 + 1024 <= 232448, "shared memory");
 };
 }  // namespace pair
 
-// Work of one SM pair.  Data-parallel: whole tiles pair_id, pair_id + npairs,
-// ...  Stream-K (p.sk): the num_tiles * k_tiles (tile, 128-deep stage) units in
-// tile-major order are cut into npairs contiguous ranges of equal length, so
-// every pair gets the same number of stages; a tile whose stages fall in two
-// ranges is finished by whichever of its pairs completes last (epilogue).
-__device__ __forceinline__ int64_t sk_begin(int64_t units, int npairs, int q) { return units * q / npairs; }
-
-__device__ __forceinline__ int sk_pair_of(int64_t u, int64_t units, int npairs) {
-  int q = (int)((u * npairs) / units);
-  while (q + 1 < npairs && sk_begin(units, npairs, q + 1) <= u) ++q;
-  while (q > 0 && sk_begin(units, npairs, q) > u) --q;
-  return q;
-}
-
-struct PairWork {
-  int64_t u, end, k_tiles;
-  int tile, npairs, num_tiles;
-  bool sk;
-  __device__ PairWork(const SpmmParams& p, int pair_id, int npairs_)
-      : k_tiles(p.k_tiles), tile(pair_id), npairs(npairs_), num_tiles(p.num_tiles), sk(p.sk != 0) {
-    const int64_t units = (int64_t)p.num_tiles * p.k_tiles;
-    u = sk ? sk_begin(units, npairs, pair_id) : 0;
-    end = sk ? sk_begin(units, npairs, pair_id + 1) : 0;
-  }
-  // next (tile, stages [kt0, kt1)) of this pair
-  __device__ bool next(int& t, int64_t& kt0, int64_t& kt1) {
-    if (!sk) {
-      if (tile >= num_tiles) return false;
-      t = tile;
-      kt0 = 0;
-      kt1 = k_tiles;
-      tile += npairs;
-      return true;
-    }
-    if (u >= end) return false;
-    t = (int)(u / k_tiles);
-    kt0 = u - (int64_t)t * k_tiles;
-    kt1 = kt0 + (end - u) < k_tiles ? kt0 + (end - u) : k_tiles;
-    u += kt1 - kt0;
-    return true;
-  }
-};
-
-// Stream-K partial accumulator of one CTA: 128 rows x 256 fp32 columns, stored
-// as [column quad][row] float4s so that a warp's access to one quad of its 32
-// rows covers 512 contiguous bytes.  Slot 2q holds the first segment of pair
-// q's range, 2q + 1 its last.
-__device__ __forceinline__ float4* sk_slot(const SpmmParams& p, int q, bool later, uint32_t rank) {
-  return reinterpret_cast<float4*>(p.sk_ws) + ((int64_t)(2 * q + (later ? 1 : 0)) * 2 + rank) * (128 * 64);
-}
-
-template <bool HYB, bool SHORT>
+template <bool HYB, bool DB>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pair::kThreads, 1)
     spmm_pair_kernel(const __grid_constant__ SpmmParams p) {
   using namespace pair;
-  using C = Cfg<HYB, SHORT>;
+  using C = Cfg<HYB, DB>;
   constexpr int kStages = C::kStages;
   constexpr uint32_t kA = C::kA;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -138,9 +96,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pair::kThreads, 1)
   constexpr Layout L = C::layout();
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + L.bar);
   uint64_t* empty = full + kStages;
-  uint64_t* acc_full = empty + kStages;
-  uint64_t* acc_empty = acc_full + 1;
-  uint64_t* spare = acc_empty + 1;
+  uint64_t* acc_full = empty + kStages;  // [2]
+  uint64_t* acc_empty = acc_full + 2;    // [2]
+  uint64_t* spare = acc_empty + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(spare + 2);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -155,10 +113,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pair::kThreads, 1)
       mbar_init(&full[s], 1);  // the leader's expect_tx; bytes from both CTAs
       mbar_init(&empty[s], 1);
     }
-    mbar_init(acc_full, 1);
-    mbar_init(acc_empty, 8);
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&acc_full[a], 1);
+      mbar_init(&acc_empty[a], 8);
+    }
     mbar_init(spare, 1);
-    mbar_init(spare + 1, 4);  // the four epilogue warps (stream-K hand-off)
     *abort_flag = 0;
     fence_barrier_init();
     fence_proxy_async_smem();
@@ -179,8 +138,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pair::kThreads, 1)
   const uint32_t tmem_base = *tmem_slot;
   pdl_gate();  // no global memory touched before this point
 
+  const int64_t k_tiles = p.K / 128;
   const uint32_t lead_full0 = map_to_cta(smem_u32(&full[0]), 0);
-  const uint32_t lead_acc_empty = map_to_cta(smem_u32(acc_empty), 0);
+  const uint32_t lead_acc_empty0 = map_to_cta(smem_u32(acc_empty), 0);
   bool ok = true;
   // Hybrid: is the 128 x 128 weight tile (row block 2*tm + rr, k block kt) 2:4?
   // A stage runs the sparse MMA only when both CTAs' tiles are 2:4; otherwise
@@ -197,46 +157,45 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pair::kThreads, 1)
     if (warp == 1) {
       // ---------------------------------------------------------- MMA (leader)
       if (rank == 0 && lane == 0) {
-        int s = 0;
-        uint32_t ph = 0, aph = 0;
-        PairWork work(p, pair_id, npairs);
-        int tile;
-        int64_t kt0, kt1;
-        while (ok && work.next(tile, kt0, kt1)) {
+        int s = 0, acc = 0;
+        uint32_t ph = 0, aph = 0;  // aph bit a: phase of accumulator a
+        for (int tile = pair_id; tile < p.num_tiles && ok; tile += npairs) {
           const int tm = tile % p.tiles_m;
-          ok = mbar_wait(acc_empty, aph ^ 1u, abort_flag, p.status, kWaitNs);
+          ok = mbar_wait(&acc_empty[acc], ((aph >> acc) & 1u) ^ 1u, abort_flag, p.status, kWaitNs);
           if (!ok) break;
           tc_fence_after();
-          for (int64_t kt = kt0; kt < kt1; ++kt) {
+          const uint32_t d_tmem = tmem_base + 256u * (uint32_t)acc;
+          for (int64_t kt = 0; kt < k_tiles; ++kt) {
             ok = mbar_wait(&full[s], ph, abort_flag, p.status, kWaitNs);
             if (!ok) break;
             tc_fence_after();
             const uint32_t a_addr = smem_u32(smem + L.a + s * kA);
             const uint32_t b_addr = smem_u32(smem + L.b + s * kB);
-            const uint32_t e_tmem = tmem_base + kECol + 4u * s;
+            const uint32_t e_tmem = tmem_base + C::kECol + 4u * s;
             if (tile_sparse(tm, kt, 0) && tile_sparse(tm, kt, 1)) {
               tc_cp_128x128b_pair(e_tmem, smem_desc(smem_u32(smem + L.e + s * kE), 2048, 128, SWZ_NONE));
 #pragma unroll
               for (int kk = 0; kk < 4; ++kk) {
                 const uint64_t ad = smem_desc(a_addr + kk * 32, 16, 1024, SWZ_128B);
                 const uint64_t bd = smem_desc(b_addr + kk * 4096, 16384, 1024, SWZ_128B);
-                tc_mma_sp_pair(tmem_base, ad, bd, e_tmem + (uint32_t)(kk & 2), kIdesc | (uint32_t)(kk & 1),
-                               (kt > kt0 || kk > 0) ? 1u : 0u);
+                tc_mma_sp_pair(d_tmem, ad, bd, e_tmem + (uint32_t)(kk & 2), C::kIdesc | (uint32_t)(kk & 1),
+                               (kt > 0 || kk > 0) ? 1u : 0u);
               }
             } else if (HYB) {  // dense A tile: [K half][128 rows][128 B], eight K = 16 MMAs
 #pragma unroll
               for (int kk = 0; kk < 8; ++kk) {
                 const uint64_t ad = smem_desc(a_addr + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024, SWZ_128B);
                 const uint64_t bd = smem_desc(b_addr + kk * 2048, 16384, 1024, SWZ_128B);
-                tc_mma_pair(tmem_base, ad, bd, kIdescDense, (kt > kt0 || kk > 0) ? 1u : 0u);
+                tc_mma_pair(d_tmem, ad, bd, kIdescDense, (kt > 0 || kk > 0) ? 1u : 0u);
               }
             }
             tc_commit_pair(&empty[s], 0x3);
             if (++s == kStages) { s = 0; ph ^= 1u; }
           }
           if (!ok) break;
-          tc_commit_pair(acc_full, 0x3);
-          aph ^= 1u;
+          tc_commit_pair(&acc_full[acc], 0x3);
+          aph ^= 1u << acc;
+          if (C::kAcc == 2) acc ^= 1;
         }
         if (!ok) {
           tc_commit_pair(spare, 0x1);
@@ -249,14 +208,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pair::kThreads, 1)
       if (lane == 0) {
         int s = 0;
         uint32_t ph = 0;
-        PairWork work(p, pair_id, npairs);
-        int tile;
-        int64_t kt0, kt1;
-        while (ok && work.next(tile, kt0, kt1)) {
+        for (int tile = pair_id; tile < p.num_tiles && ok; tile += npairs) {
           const int tm = tile % p.tiles_m, tn = tile / p.tiles_m;
           const int32_t row0 = tm * 256 + 128 * (int)rank;
-          const int32_t col0 = tn * 256 + 128 * (int)rank;
-          for (int64_t kt = kt0; kt < kt1; ++kt) {
+          const int32_t col0 = tn * (int32_t)C::kN + (int32_t)(C::kN / 2) * (int)rank;
+          for (int64_t kt = 0; kt < k_tiles; ++kt) {
             ok = mbar_wait(&empty[s], ph ^ 1u, abort_flag, p.status, kWaitNs);
             if (!ok) break;
             const uint32_t lead_full = lead_full0 + 8u * s;
@@ -289,259 +245,122 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pair::kThreads, 1)
   } else {
     // -------------------------------------------------------------- epilogue
     const int quarter = warp & 3;
-    uint32_t aph = 0, ephase = 0;
-    uint64_t* epi_bar = spare + 1;
-    volatile uint32_t* sk_flag = reinterpret_cast<volatile uint32_t*>(tmem_slot + 2);
-    const int64_t units = (int64_t)p.num_tiles * p.k_tiles;
-    const int64_t my_beg = p.sk ? sk_begin(units, npairs, pair_id) : 0;
-    // all four epilogue warps meet (bounded wait; orders the shared flag and, with the
-    // fences before it, this CTA's workspace stores)
-    auto epi_sync = [&]() -> bool {
-      __syncwarp();
-      if (lane == 0) mbar_arrive(epi_bar);
-      const bool r = mbar_wait(epi_bar, ephase, abort_flag, p.status, kWaitNs);
-      ephase ^= 1u;
-      return r;
-    };
-    PairWork work(p, pair_id, npairs);
-    int tile;
-    int64_t kt0, kt1;
-    while (ok && work.next(tile, kt0, kt1)) {
+    uint32_t aph = 0;  // bit a: phase of accumulator a
+    int acc = 0;
+    for (int tile = pair_id; tile < p.num_tiles && ok; tile += npairs) {
       const int tm = tile % p.tiles_m, tn = tile / p.tiles_m;
       const int64_t row = (int64_t)tm * 256 + 128 * rank + quarter * 32 + lane;
-      const int64_t n0 = (int64_t)tn * 256;
-      ok = mbar_wait(acc_full, aph, abort_flag, p.status, kWaitNs);
+      const int64_t n0 = (int64_t)tn * C::kN;
+      ok = mbar_wait(&acc_full[acc], (aph >> acc) & 1u, abort_flag, p.status, kWaitNs);
       if (!ok) break;
       tc_fence_after();
-      const uint32_t t_addr = tmem_base + ((uint32_t)(quarter * 32) << 16);
+      const uint32_t t_addr = tmem_base + 256u * (uint32_t)acc + ((uint32_t)(quarter * 32) << 16);
+      const uint32_t lead_acc_empty = lead_acc_empty0 + 8u * (uint32_t)acc;
       const bool row_ok = row < p.R;
-      if (kt0 == 0 && kt1 == p.k_tiles) {
-        if (C::kEpiBufs == 4 && !p.out_f32) {
-          // 64-column chunk c of the warp's 32 rows: two TMEM loads, bf16 pairs
-          // into staging buffer c (128-byte swizzled rows); TMEM released after
-          // the last load, then the four stores leave together.
-          const int32_t wrow0 = (int32_t)(tm * 256 + 128 * rank + quarter * 32);
-          uint8_t* ebuf = smem + L.epi + quarter * (C::kEpiBufs * kEpi);
-          if (lane == 0) bulk_wait_group_read<0>();  // the previous tile's stores have read the buffers
-          __syncwarp();
+      if (DB && !p.out_f32) {
+        // Three 64-column chunks through the warp's staging buffer, one TMA
+        // store each.  The accumulator is released after the last TMEM load; the
+        // next tile's MMAs run in the other accumulator meanwhile, so this
+        // epilogue has a whole tile period to finish.
+        const int32_t wrow0 = (int32_t)(tm * 256 + 128 * rank + quarter * 32);
+        uint8_t* ebuf = smem + L.epi + quarter * kEpi;
 #pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            uint32_t v0[32], v1[32];
-            tmem_ld_32x32b_x32(t_addr + c * 64, v0);
-            tmem_ld_32x32b_x32(t_addr + c * 64 + 32, v1);
-            tc_wait_ld();
-            uint8_t* buf = ebuf + c * kEpi;
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-              *reinterpret_cast<uint4*>(buf + lane * 128 + ((j ^ (lane & 7)) << 4)) =
-                  make_uint4(pack_bf16x2(__uint_as_float(v0[8 * j]), __uint_as_float(v0[8 * j + 1])),
-                             pack_bf16x2(__uint_as_float(v0[8 * j + 2]), __uint_as_float(v0[8 * j + 3])),
-                             pack_bf16x2(__uint_as_float(v0[8 * j + 4]), __uint_as_float(v0[8 * j + 5])),
-                             pack_bf16x2(__uint_as_float(v0[8 * j + 6]), __uint_as_float(v0[8 * j + 7])));
-              *reinterpret_cast<uint4*>(buf + lane * 128 + (((j + 4) ^ (lane & 7)) << 4)) =
-                  make_uint4(pack_bf16x2(__uint_as_float(v1[8 * j]), __uint_as_float(v1[8 * j + 1])),
-                             pack_bf16x2(__uint_as_float(v1[8 * j + 2]), __uint_as_float(v1[8 * j + 3])),
-                             pack_bf16x2(__uint_as_float(v1[8 * j + 4]), __uint_as_float(v1[8 * j + 5])),
-                             pack_bf16x2(__uint_as_float(v1[8 * j + 6]), __uint_as_float(v1[8 * j + 7])));
-            }
+        for (int c = 0; c < 3; ++c) {
+          uint32_t v0[32], v1[32];
+          tmem_ld_32x32b_x32(t_addr + c * 64, v0);
+          tmem_ld_32x32b_x32(t_addr + c * 64 + 32, v1);
+          tc_wait_ld();
+          if (c == 2) {
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive_cluster(lead_acc_empty);
           }
-          tc_fence_before();
+          if (lane == 0) bulk_wait_group_read<0>();  // the previous store has read the buffer
           __syncwarp();
-          if (lane == 0) mbar_arrive_cluster(lead_acc_empty);
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            *reinterpret_cast<uint4*>(ebuf + lane * 128 + ((j ^ (lane & 7)) << 4)) =
+                make_uint4(pack_bf16x2(__uint_as_float(v0[8 * j]), __uint_as_float(v0[8 * j + 1])),
+                           pack_bf16x2(__uint_as_float(v0[8 * j + 2]), __uint_as_float(v0[8 * j + 3])),
+                           pack_bf16x2(__uint_as_float(v0[8 * j + 4]), __uint_as_float(v0[8 * j + 5])),
+                           pack_bf16x2(__uint_as_float(v0[8 * j + 6]), __uint_as_float(v0[8 * j + 7])));
+            *reinterpret_cast<uint4*>(ebuf + lane * 128 + (((j + 4) ^ (lane & 7)) << 4)) =
+                make_uint4(pack_bf16x2(__uint_as_float(v1[8 * j]), __uint_as_float(v1[8 * j + 1])),
+                           pack_bf16x2(__uint_as_float(v1[8 * j + 2]), __uint_as_float(v1[8 * j + 3])),
+                           pack_bf16x2(__uint_as_float(v1[8 * j + 4]), __uint_as_float(v1[8 * j + 5])),
+                           pack_bf16x2(__uint_as_float(v1[8 * j + 6]), __uint_as_float(v1[8 * j + 7])));
+          }
           fence_proxy_async_smem();
           __syncwarp();
-          if (lane == 0 && wrow0 < p.R) {
-#pragma unroll
-            for (int c = 0; c < 4; ++c)
-              if (n0 + 64 * c < p.T) tma_store_2d(&p.tm_y, ebuf + c * kEpi, (int32_t)(n0 + 64 * c), wrow0);
+          if (lane == 0 && n0 + 64 * c < p.T && wrow0 < p.R) {
+            tma_store_2d(&p.tm_y, ebuf, (int32_t)(n0 + 64 * c), wrow0);
             bulk_commit_group();
           }
-        } else if (C::kEpiBufs == 1 && !p.out_f32) {
-          // Whole accumulator row into registers (bf16), release TMEM, then four
-          // 64-column chunks through this warp's swizzled staging buffer and a
-          // TMA store each: every store writes whole lines, and parts of the box
-          // beyond R or T are not written.
-          uint32_t pk[128];
+        }
+      } else if (!DB && !p.out_f32) {
+        // Whole accumulator row into registers (bf16), release TMEM, then four
+        // 64-column chunks through this warp's swizzled staging buffer and a
+        // TMA store each: every store writes whole lines, and parts of the box
+        // beyond R or T are not written.
+        uint32_t pk[128];
 #pragma unroll
-          for (int c = 0; c < 8; ++c) {
-            uint32_t v[32];
-            tmem_ld_32x32b_x32(t_addr + c * 32, v);
-            tc_wait_ld();
+        for (int c = 0; c < 8; ++c) {
+          uint32_t v[32];
+          tmem_ld_32x32b_x32(t_addr + c * 32, v);
+          tc_wait_ld();
 #pragma unroll
-            for (int i = 0; i < 16; ++i)
-              pk[c * 16 + i] = pack_bf16x2(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1]));
-          }
-          tc_fence_before();
+          for (int i = 0; i < 16; ++i)
+            pk[c * 16 + i] = pack_bf16x2(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1]));
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_cluster(lead_acc_empty);
+        const int32_t wrow0 = (int32_t)(tm * 256 + 128 * rank + quarter * 32);
+        uint8_t* ebuf = smem + L.epi + quarter * kEpi;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          if (lane == 0) bulk_wait_group_read<0>();  // the previous store has read the buffer
           __syncwarp();
-          if (lane == 0) mbar_arrive_cluster(lead_acc_empty);
-          const int32_t wrow0 = (int32_t)(tm * 256 + 128 * rank + quarter * 32);
-          uint8_t* ebuf = smem + L.epi + quarter * (C::kEpiBufs * kEpi);
 #pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            if (lane == 0) bulk_wait_group_read<0>();  // the previous store has read the buffer
-            __syncwarp();
-#pragma unroll
-            for (int j = 0; j < 8; ++j)
-              *reinterpret_cast<uint4*>(ebuf + lane * 128 + ((j ^ (lane & 7)) << 4)) =
-                  make_uint4(pk[32 * c + 4 * j], pk[32 * c + 4 * j + 1], pk[32 * c + 4 * j + 2], pk[32 * c + 4 * j + 3]);
-            fence_proxy_async_smem();
-            __syncwarp();
-            if (lane == 0 && n0 + 64 * c < p.T && wrow0 < p.R) {
-              tma_store_2d(&p.tm_y, ebuf, (int32_t)(n0 + 64 * c), wrow0);
-              bulk_commit_group();
-            }
-          }
-        } else {
-#pragma unroll 1
-          for (int c = 0; c < 16; ++c) {
-            uint32_t v[16];
-            tmem_ld_32x32b_x16(t_addr + c * 16, v);
-            tc_wait_ld();
-            if (!row_ok) continue;
-            const int64_t col0 = n0 + c * 16;
-            if (p.out_f32) {
-              float* yrow = static_cast<float*>(p.Y) + row * p.ldy;
-#pragma unroll
-              for (int e = 0; e < 16; ++e)
-                if (col0 + e < p.T) yrow[col0 + e] = __uint_as_float(v[e]);
-            } else {
-              uint16_t* yrow = static_cast<uint16_t*>(p.Y) + row * p.ldy;
-#pragma unroll
-              for (int e = 0; e < 16; e += 2) {
-                const uint32_t pk = pack_bf16x2(__uint_as_float(v[e]), __uint_as_float(v[e + 1]));
-                if (col0 + e < p.T) yrow[col0 + e] = (uint16_t)(pk & 0xFFFFu);
-                if (col0 + e + 1 < p.T) yrow[col0 + e + 1] = (uint16_t)(pk >> 16);
-              }
-            }
-          }
-          tc_fence_before();
+          for (int j = 0; j < 8; ++j)
+            *reinterpret_cast<uint4*>(ebuf + lane * 128 + ((j ^ (lane & 7)) << 4)) =
+                make_uint4(pk[32 * c + 4 * j], pk[32 * c + 4 * j + 1], pk[32 * c + 4 * j + 2], pk[32 * c + 4 * j + 3]);
+          fence_proxy_async_smem();
           __syncwarp();
-          if (lane == 0) mbar_arrive_cluster(lead_acc_empty);
+          if (lane == 0 && n0 + 64 * c < p.T && wrow0 < p.R) {
+            tma_store_2d(&p.tm_y, ebuf, (int32_t)(n0 + 64 * c), wrow0);
+            bulk_commit_group();
+          }
         }
       } else {
-        // Stream-K segment of a split tile.  If the tile's other segments are
-        // already in the workspace, this CTA adds them to its accumulator as it
-        // drains TMEM and stores the tile.  Otherwise its partial goes to its
-        // workspace slot, and the last segment to arrive adds all partials in
-        // range order.  Either way the sum runs over the segments in range
-        // order, so the result does not depend on which pair finishes last.
-        const int rr = quarter * 32 + lane;  // row within this CTA's 128
-        const int64_t tu0 = (int64_t)tile * p.k_tiles;
-        const int q0 = sk_pair_of(tu0, units, npairs);
-        const int q1 = sk_pair_of(tu0 + p.k_tiles - 1, units, npairs);
-        const bool q0_later = tu0 > sk_begin(units, npairs, q0);
-        const int32_t wrow0 = (int32_t)(tm * 256 + 128 * rank + quarter * 32);
-        uint8_t* ebuf = smem + L.epi + quarter * (C::kEpiBufs * kEpi);
-        uint32_t* cnt = p.sk_cnt + 2 * tile + (int)rank;
-        // Only a tile's first segment, which ends its pair's range, checks first:
-        // the other segment starts a later range and is usually long finished.
-        if (kt0 == 0) {
-          if (warp == 6 && lane == 0) {
-            *sk_flag = atomicAdd(cnt, 0u);
-            __threadfence();
-          }
-          ok = epi_sync();
-          if (!ok) break;
-        }
-        // 64-column chunk c of this warp's rows to the output (staging + TMA store, or fp32 rows)
-        auto emit = [&](int c, const float* a) {
-          if (!p.out_f32) {
-            uint8_t* buf = ebuf + (C::kEpiBufs == 4 ? c * kEpi : 0);
-            if (C::kEpiBufs == 1 || c == 0) {
-              if (lane == 0) bulk_wait_group_read<0>();  // earlier stores have read the buffer(s)
-              __syncwarp();
-            }
-#pragma unroll
-            for (int j = 0; j < 8; ++j)
-              *reinterpret_cast<uint4*>(buf + lane * 128 + ((j ^ (lane & 7)) << 4)) =
-                  make_uint4(pack_bf16x2(a[8 * j], a[8 * j + 1]), pack_bf16x2(a[8 * j + 2], a[8 * j + 3]),
-                             pack_bf16x2(a[8 * j + 4], a[8 * j + 5]), pack_bf16x2(a[8 * j + 6], a[8 * j + 7]));
-            fence_proxy_async_smem();
-            __syncwarp();
-            if (lane == 0 && n0 + 64 * c < p.T && wrow0 < p.R) {
-              tma_store_2d(&p.tm_y, buf, (int32_t)(n0 + 64 * c), wrow0);
-              bulk_commit_group();
-            }
-          } else if (row_ok) {
+#pragma unroll 1
+        for (int c = 0; c < (int)(C::kN / 16); ++c) {
+          uint32_t v[16];
+          tmem_ld_32x32b_x16(t_addr + c * 16, v);
+          tc_wait_ld();
+          if (!row_ok) continue;
+          const int64_t col0 = n0 + c * 16;
+          if (p.out_f32) {
             float* yrow = static_cast<float*>(p.Y) + row * p.ldy;
 #pragma unroll
-            for (int j = 0; j < 64; ++j)
-              if (n0 + 64 * c + j < p.T) yrow[n0 + 64 * c + j] = a[j];
-          }
-        };
-        if (kt0 == 0 && *sk_flag == (uint32_t)(q1 - q0)) {
-          // every other segment is in the workspace (nseg <= 2 here: the host
-          // enables stream-K only with at least one tile per pair)
-          const int qo = pair_id == q0 ? q1 : q0;
-          const float4* other = sk_slot(p, qo, qo == q0 && q0_later, rank);
-          __threadfence();
-#pragma unroll 1
-          for (int c = 0; c < 4; ++c) {
-            uint32_t v[64];
-            tmem_ld_32x32b_x32(t_addr + c * 64, *reinterpret_cast<uint32_t(*)[32]>(v));
-            tmem_ld_32x32b_x32(t_addr + c * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(v + 32));
-            tc_wait_ld();
-            float a[64];
+            for (int e = 0; e < 16; ++e)
+              if (col0 + e < p.T) yrow[col0 + e] = __uint_as_float(v[e]);
+          } else {
+            uint16_t* yrow = static_cast<uint16_t*>(p.Y) + row * p.ldy;
 #pragma unroll
-            for (int g = 0; g < 16; ++g) {
-              const float4 o = __ldcg(other + (16 * c + g) * 128 + rr);
-              a[4 * g] = __uint_as_float(v[4 * g]) + o.x;
-              a[4 * g + 1] = __uint_as_float(v[4 * g + 1]) + o.y;
-              a[4 * g + 2] = __uint_as_float(v[4 * g + 2]) + o.z;
-              a[4 * g + 3] = __uint_as_float(v[4 * g + 3]) + o.w;
-            }
-            if (c == 3) {
-              tc_fence_before();
-              __syncwarp();
-              if (lane == 0) mbar_arrive_cluster(lead_acc_empty);
-            }
-            emit(c, a);
-          }
-        } else {
-          float4* mine = sk_slot(p, pair_id, tu0 + kt0 > my_beg, rank);
-#pragma unroll 1
-          for (int c = 0; c < 8; ++c) {
-            uint32_t v[32];
-            tmem_ld_32x32b_x32(t_addr + c * 32, v);
-            tc_wait_ld();
-#pragma unroll
-            for (int g = 0; g < 8; ++g)
-              mine[(8 * c + g) * 128 + rr] = make_float4(__uint_as_float(v[4 * g]), __uint_as_float(v[4 * g + 1]),
-                                                         __uint_as_float(v[4 * g + 2]), __uint_as_float(v[4 * g + 3]));
-          }
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive_cluster(lead_acc_empty);
-          __threadfence();
-          ok = epi_sync();
-          if (!ok) break;
-          if (warp == 6 && lane == 0) *sk_flag = atomicAdd(cnt, 1u);
-          ok = epi_sync();
-          if (!ok) break;
-          if (*sk_flag == (uint32_t)(q1 - q0)) {
-            __threadfence();
-#pragma unroll 1
-            for (int c = 0; c < 4; ++c) {
-              float a[64];
-#pragma unroll
-              for (int j = 0; j < 64; ++j) a[j] = 0.0f;
-              for (int q = q0; q <= q1; ++q) {
-                const float4* src = sk_slot(p, q, q == q0 && q0_later, rank);
-#pragma unroll
-                for (int g = 0; g < 16; ++g) {
-                  const float4 o = __ldcg(src + (16 * c + g) * 128 + rr);
-                  a[4 * g] += o.x;
-                  a[4 * g + 1] += o.y;
-                  a[4 * g + 2] += o.z;
-                  a[4 * g + 3] += o.w;
-                }
-              }
-              emit(c, a);
+            for (int e = 0; e < 16; e += 2) {
+              const uint32_t pk = pack_bf16x2(__uint_as_float(v[e]), __uint_as_float(v[e + 1]));
+              if (col0 + e < p.T) yrow[col0 + e] = (uint16_t)(pk & 0xFFFFu);
+              if (col0 + e + 1 < p.T) yrow[col0 + e + 1] = (uint16_t)(pk >> 16);
             }
           }
         }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_cluster(lead_acc_empty);
       }
-      aph ^= 1u;
+      aph ^= 1u << acc;
+      if (C::kAcc == 2) acc ^= 1;
     }
     if (lane == 0) bulk_wait_group<0>();  // every store of this warp has landed
   }
@@ -563,30 +382,41 @@ bool pair_kernel_fits(const SpmmParams& p) {
   return p.a_mode == A_TMA_SPARSE && p.K % 128 == 0 && p.K > 0 && p.T >= 192 && p.R >= 1 && p.T % 8 == 0;
 }
 
-template <bool HYB, bool SHORT>
+template <bool HYB, bool DB>
 static cudaError_t launch_pair(SpmmParams& p, cudaStream_t stream) {
-  constexpr pair::Layout L = pair::Cfg<HYB, SHORT>::layout();
+  constexpr pair::Layout L = pair::Cfg<HYB, DB>::layout();
   const size_t bytes = L.total + 1024;
   static bool configured[64] = {};
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 64 && !configured[dev]) {
     cudaError_t e =
-        cudaFuncSetAttribute(spmm_pair_kernel<HYB, SHORT>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+        cudaFuncSetAttribute(spmm_pair_kernel<HYB, DB>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
     if (e != cudaSuccess) return e;
     configured[dev] = true;
   }
   const int pairs_avail = sm_count_current() / 2;
   const int pairs = p.num_tiles < pairs_avail ? p.num_tiles : pairs_avail;
-  cudaError_t e = launch_pdl(spmm_pair_kernel<HYB, SHORT>, dim3(2 * pairs), dim3(pair::kThreads), bytes, stream, p);
+  cudaError_t e = launch_pdl(spmm_pair_kernel<HYB, DB>, dim3(2 * pairs), dim3(pair::kThreads), bytes, stream, p);
   count_launch();
   return e != cudaSuccess ? e : cudaGetLastError();
 }
 
-// Tiles of at most eight 128-deep stages take the short-tile configuration
-// (three stages, four staging buffers per epilogue warp).
+// Tiles of at most kDbMaxStages 128-deep stages take the double-buffered
+// 256 x 192 form.  Measured on B200 (nm_spmm, event-timed loops): ViT
+// 3072 x 768 x 50432 at 1:8 (6 stages) 174 -> 166 us; at 24 stages (768 x 3072)
+// 125 -> 143 us, at 32 (4096 x 4096 x 2048) 33 -> 44 us.  A 192-column stage
+// costs about as much as a 256-column one, so the narrower tile pays only where
+// the hidden hand-over is a large part of a tile.
+constexpr int64_t kDbMaxStages = 8;
+
 cudaError_t launch_spmm_pair(SpmmParams& p, cudaStream_t stream) {
-  return p.k_tiles <= 8 ? launch_pair<false, true>(p, stream) : launch_pair<false, false>(p, stream);
+  if (p.k_tiles <= kDbMaxStages) {
+    p.tiles_n = (int)((p.T + 191) / 192);
+    p.num_tiles = p.tiles_m * p.tiles_n;
+    return launch_pair<false, true>(p, stream);
+  }
+  return launch_pair<false, false>(p, stream);
 }
 
 cudaError_t launch_spmm_pair_hybrid(SpmmParams& p, cudaStream_t stream) { return launch_pair<true, false>(p, stream); }

@@ -486,62 +486,50 @@ def test_dense_design_pair_integer_exact():
 
 
 # ----------------------------------------------------------------------------
-# Stream-K schedule of the SM-pair kernel (tile counts that leave a partial
-# last wave: ranges of equal length per pair, split tiles summed in fp32)
+# SM-pair kernel tile forms: 256 x 256 tiles with one accumulator (more than 8
+# stages per tile) and 256 x 192 tiles with two accumulators (at most 8)
 # ----------------------------------------------------------------------------
-@pytest.mark.parametrize("R,K,T", [(2560, 8192, 2048),   # 80 tiles of 64 stages on 74 pairs: stream-K
-                                   (4096, 11008, 2048),  # the LLaMA 4096 x 11008 layer: 128 tiles of 86 stages
-                                   (1280, 512, 4096),    # 80 tiles of 4 stages: whole tiles (short-tile kernel)
-                                   (2304, 768, 2560)])   # 90 tiles of 6 stages: whole tiles
+@pytest.mark.parametrize("R,K,T", [(2560, 8192, 2048),   # 64 stages: 256 x 256 tiles
+                                   (4096, 11008, 2048),  # the LLaMA 4096 x 11008 layer
+                                   (1280, 512, 4096),    # 4 stages: 256 x 192 tiles, 22 column tiles
+                                   (2304, 768, 2560),    # 6 stages (the ViT depth), last column tile partial
+                                   (300, 1024, 200)])    # 8 stages, one partial 192-column tile, ragged rows
 @pytest.mark.parametrize("out", [torch.bfloat16, torch.float32])
-def test_stream_k_integer_exact(R, K, T, out):
-    """Small integers keep every fp32 partial sum exact, so a tile summed from two
-    ranges must equal the oracle bit for bit."""
+def test_pair_tile_forms_integer_exact(R, K, T, out):
+    """Small integers keep every fp32 sum exact: sampled rows equal the oracle bit for bit."""
     W = wl.integer_bf16((R, K), -8, 8, seed=R + 7)
     X = wl.integer_bf16((K, T), -8, 8, seed=T + 9)
     Y = run_spmm(W, X, 2, 4, out_dtype=out)
     ov, om = oracle.compress(W, 2, 4)
     rng = np.random.default_rng(3)
-    rows = np.unique(np.concatenate([rng.integers(0, R, 96), [0, 127, 128, 255, 256, R - 1]]))
+    rows = np.unique(np.concatenate([rng.integers(0, R, 96), [0, 127, 128, 255, R - 1]]))
+    rows = rows[rows < R]
     Wd = oracle.decompress(ov, om, K, 2, 4)
     ref = oracle.dense_gemm(np.ascontiguousarray(Wd[rows]), X)
-    got = Y.contiguous().cpu().float().numpy().astype(np.float64)[rows] if out == torch.float32 else None
     if out == torch.float32:
-        assert np.array_equal(got, ref)
+        assert np.array_equal(Y.contiguous().cpu().numpy().astype(np.float64)[rows], ref)
     else:
         assert np.array_equal(bits(Y)[rows], bf16_rne_of(ref))
 
 
-def test_stream_k_permuted_tolerance():
-    R, K, T = 2560, 8192, 2048
+def test_pair_double_buffered_permuted_tolerance():
+    """ViT-depth tiles (6 stages, two accumulators) with an index map, sampled at full width."""
+    R, K, T = 3072, 768, 6144
     W = wl.normal_bf16((R, K), 0.02, seed=41)
     X = wl.normal_bf16((K, T), 1.0, seed=42)
     idx = wl.permutation(K, 43)
-    Wd_, Xd, idxd = to_dev(W), to_dev(X), to_dev_i32(idx)
-    vals, meta = nm.prune_compress(Wd_, 2, 4)
-    Y = nm.spmm(vals, meta, 2, 4, K, Xd, idx=idxd)
+    vals, meta = nm.prune_compress(to_dev(W), 2, 4)
+    Y = nm.spmm(vals, meta, 2, 4, K, to_dev(X), idx=to_dev_i32(idx))
     torch.cuda.synchronize()
     nm.nm_device_status()
     sampled_check(vals, meta, 2, 4, W, X, Y, idx=idx, count=4000)
 
 
-def test_stream_k_hybrid_integer_exact():
-    R, K, T = 1280, 8192, 4096  # 80 pair tiles of 64 stages on the hybrid kernel: stream-K
-    W = wl.integer_bf16((R, K), -8, 8, seed=51)
-    X = wl.integer_bf16((K, T), -8, 8, seed=52)
-    tm = wl.tile_map(10, 64, 0.5, seed=53)
-    Y = run_hybrid(W, X, tm)
-    rows = np.arange(0, R, 5)
-    Weff = oracle.hybrid_weights(W, tm, 128)
-    ref = oracle.dense_gemm(np.ascontiguousarray(Weff[rows]), X)
-    assert np.array_equal(bits(Y)[rows], bf16_rne_of(ref))
-
-
-def test_stream_k_repeatable():
-    """The split tiles' partials are added in a fixed order: two runs agree bit for bit."""
-    R, K, T = 2560, 8192, 2048
-    W = wl.normal_bf16((R, K), 0.02, seed=61)
-    X = wl.normal_bf16((K, T), 1.0, seed=62)
-    a = run_spmm(W, X, 2, 4)
-    b = run_spmm(W, X, 2, 4)
-    assert torch.equal(a, b)
+def test_pair_repeatable():
+    """Two runs of the same GEMM agree bit for bit (both tile forms)."""
+    for R, K, T in ((2560, 8192, 2048), (1280, 768, 4096)):
+        W = wl.normal_bf16((R, K), 0.02, seed=61)
+        X = wl.normal_bf16((K, T), 1.0, seed=62)
+        a = run_spmm(W, X, 2, 4)
+        b = run_spmm(W, X, 2, 4)
+        assert torch.equal(a, b)
