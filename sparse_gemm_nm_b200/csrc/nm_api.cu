@@ -1046,6 +1046,49 @@ static nm_status run_spmm_i8(const int8_t* values, const uint32_t* meta, int64_t
   cudaMemPool_t pool = nullptr;
   cudaError_t e = staging_pool(&pool);
   if (e != cudaSuccess) return cuda_fail(e, "staging pool");
+  // The sparse tensor cores (kind::i8 on SM pairs) when the shape fills pair tiles: the tiled metadata is
+  // re-laid out per row (R x K / 8 bytes staged) and the compressed values are read as they are.
+  if (T >= 192 && K % 32 == 0 && al16(values) && R < (1ll << 31) && K < (1ll << 31)) {
+    const int64_t rblocks128 = (R + 255) / 256 * 2, kblocks = (K + 255) / 256;
+    void* em = nullptr;
+    e = cudaMallocFromPoolAsync(&em, (size_t)(rblocks128 * kblocks * 4096), pool, stream);
+    if (e != cudaSuccess) return cuda_fail(e, "staging buffer for the int8 metadata");
+    e = launch_relayout_meta_i8(meta, R, K, static_cast<uint32_t*>(em), rblocks128, stream);
+    SpmmParams p;
+    std::memset(&p, 0, sizeof p);
+    p.R = R;
+    p.K = K;
+    p.T = T;
+    p.n = 2;
+    p.m = 4;
+    p.Y = Y;
+    p.ldy = ldy;
+    p.out_f32 = 1;  // the int32 accumulator bits, stored unchanged
+    p.a_mode = A_TMA_SPARSE;
+    p.pattern = PAT_2_4;
+    p.vcols = K / 2;
+    p.meta_cblocks = kblocks;
+    p.k_tiles = kblocks;
+    p.tiles_m = (int)((R + 255) / 256);
+    p.tiles_n = (int)((T + 255) / 256);
+    p.num_tiles = p.tiles_m * p.tiles_n;
+    p.status = status_word_ptr();
+    if (e == cudaSuccess && !p.status) e = cudaErrorInvalidSymbol;
+    if ((int64_t)p.tiles_m * p.tiles_n >= (1ll << 31)) st = fail(NM_ERR_UNSUPPORTED, "too many tiles");
+    if (e == cudaSuccess && st == NM_OK)
+      st = make_tmap(&p.tm_vals, values, (uint64_t)(K / 2), (uint64_t)R, (uint64_t)(K / 2), 128, kPairBoxRows, 128,
+                     "values (int8)", CU_TENSOR_MAP_DATA_TYPE_UINT8);
+    if (e == cudaSuccess && st == NM_OK)
+      st = make_tmap(&p.tm_x, X, (uint64_t)T, (uint64_t)K, (uint64_t)ldx, 128, kPairBoxRows, 128, "X (int8)",
+                     CU_TENSOR_MAP_DATA_TYPE_UINT8);
+    if (e == cudaSuccess && st == NM_OK)
+      st = make_tmap(&p.tm_meta, em, 256, (uint64_t)(rblocks128 * kblocks * 16), 256, 256, 16, 0,
+                     "metadata (int8 order)", CU_TENSOR_MAP_DATA_TYPE_UINT8);
+    if (e == cudaSuccess && st == NM_OK) e = launch_spmm_pair_i8(p, stream);
+    cudaFreeAsync(em, stream);
+    if (st != NM_OK) return st;
+    return e == cudaSuccess ? NM_OK : cuda_fail(e, "int8 sparse GEMM launch");
+  }
   void* wd = nullptr;
   e = cudaMallocFromPoolAsync(&wd, (size_t)(R * K), pool, stream);
   if (e != cudaSuccess) return cuda_fail(e, "staging buffer for the decompressed int8 weights");

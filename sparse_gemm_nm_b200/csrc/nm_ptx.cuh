@@ -267,6 +267,20 @@ __device__ __forceinline__ void tc_mma_pair_i8(uint32_t d_tmem, uint64_t a_desc,
       : "memory");
 }
 
+// Sparse kind::i8 on SM pairs: 2:4 A (signed 8-bit, 32 stored bytes per row for K = 64), signed 8-bit B,
+// int32 accumulator.  Its metadata is read per row in plain K order: TMEM lane = row, the 16 groups of
+// the K = 64 step in two consecutive columns (group g at column g / 8, bits 4 (g % 8)); the sparsity
+// selector must be 0.
+__device__ __forceinline__ void tc_mma_sp_pair_i8(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t e_tmem,
+                                                  uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %5, 0;\n\t"
+      "tcgen05.mma.sp.cta_group::2.kind::i8 [%0], %1, %2, [%3], %4, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(e_tmem), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
 // Arrive once on the mbarrier at this shared offset in every CTA of cta_mask
 // when all previously issued pair tcgen05 operations have completed.
 __device__ __forceinline__ void tc_commit_pair(uint64_t* bar, uint16_t cta_mask) {
@@ -279,6 +293,11 @@ __device__ __forceinline__ void tc_commit_pair(uint64_t* bar, uint16_t cta_mask)
 
 __device__ __forceinline__ void tc_cp_128x128b_pair(uint32_t taddr, uint64_t s_desc) {
   asm volatile("tcgen05.cp.cta_group::2.128x128b [%0], %1;" ::"r"(taddr), "l"(s_desc) : "memory");
+}
+
+// 128 lanes x 256 bits (8 columns) from shared memory into TMEM, both CTAs of the pair.
+__device__ __forceinline__ void tc_cp_128x256b_pair(uint32_t taddr, uint64_t s_desc) {
+  asm volatile("tcgen05.cp.cta_group::2.128x256b [%0], %1;" ::"r"(taddr), "l"(s_desc) : "memory");
 }
 
 __device__ __forceinline__ void tmem_alloc(uint32_t* smem_result, uint32_t ncols) {

@@ -124,6 +124,12 @@ uint32_t* status_word_ptr();
 bool pair_kernel_fits(const SpmmParams& p);
 cudaError_t launch_spmm_pair(SpmmParams& p, cudaStream_t stream);
 cudaError_t launch_spmm_pair_hybrid(SpmmParams& p, cudaStream_t stream);
+// INT8 2:4 on SM pairs (sparse kind::i8): tm_vals int8 values R x K/2 (box {128, 64}), tm_x int8 X (box
+// {128, 64}), tm_meta the re-laid-out metadata as rows of 256 bytes (box {256, 16}), meta_cblocks = its
+// 256-column K blocks; int32 results through the fp32 store path (out_f32 = 1).
+cudaError_t launch_spmm_pair_i8(SpmmParams& p, cudaStream_t stream);
+cudaError_t launch_relayout_meta_i8(const uint32_t* meta, int64_t R, int64_t K, uint32_t* out, int64_t rblocks128,
+                                    cudaStream_t s);
 bool skinny_kernel_fits(int64_t T);
 int skinny_bn(int64_t T);
 int skinny_kd(int64_t K, int64_t T);

@@ -38,6 +38,12 @@
 // from column 448).  It keeps four stages: a trace of the three-stage form on the
 // ViT shape showed the MMA thread waiting ~240 ns of each ~600 ns stage for data
 // (X rows 100 KB apart, a third of them from HBM).
+//
+// INT8 (I8): the same pipeline on the sparse kind::i8 MMA.  A stage covers 256
+// logical K: A is 128 rows x 128 stored bytes (16 KB), B 256 rows x this CTA's
+// 128 int8 columns (32 KB, four 64-row boxes), and the metadata 4 KB per CTA in
+// the per-row order that MMA reads (relayout_meta_i8_kernel), copied into 8
+// TMEM columns; four K = 64 MMAs per stage, int32 accumulators stored as such.
 #include <cstdint>
 #include <cuda.h>
 #include <cuda_runtime.h>
@@ -50,7 +56,7 @@ namespace nmk {
 
 namespace pair {
 constexpr int kThreads = 384;  // warps 0,2-5,10,11 copies; 1 MMA; 6-9 epilogue
-constexpr uint32_t kB = 32768, kE = 2048;
+constexpr uint32_t kB = 32768;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint64_t kWaitNs = 2000000000ull;
 constexpr uint32_t kIdescDense = idesc_bf16(256, false, 256);
@@ -63,14 +69,18 @@ struct Layout {
 // HYB = true (PATCH hybrid): A slots of 32 KB so that a stage can hold the
 // dense 128 x 128 tile instead, three stages.
 // DB = true (2:4, short tiles): 256 x 192 tiles, two accumulators, four stages.
-template <bool HYB, bool DB = false>
+template <bool HYB, bool DB = false, bool I8 = false>
 struct Cfg {
+  static_assert(!(I8 && (HYB || DB)), "int8 runs the 256 x 256 sparse form only");
   static constexpr int kStages = HYB ? 3 : 4;
   static constexpr uint32_t kN = DB ? 192u : 256u;  // pair tile columns (per CTA: kN / 2 of X)
   static constexpr int kAcc = DB ? 2 : 1;           // accumulators, 256 TMEM columns apart
   static constexpr uint32_t kECol = DB ? 448u : 256u;
+  static constexpr uint32_t kE = I8 ? 4096u : 2048u;  // metadata bytes per stage and CTA
+  static constexpr uint32_t kECols = I8 ? 8u : 4u;    // its TMEM columns
   static constexpr int kEpiBufs = 1;
-  static constexpr uint32_t kIdesc = idesc_bf16(kN, true, 256);
+  static constexpr uint32_t kIdesc = I8 ? (idesc_s8_major(256, 256, false, true) | (1u << 2))
+                                        : idesc_bf16(kN, true, 256);
   static constexpr uint32_t kA = HYB ? 32768u : 16384u;
   static constexpr uint32_t kTxSparse = 2u * (16384u + kB + kE);  // both CTAs' A, B and E bytes
   static constexpr uint32_t kTxDense = 2u * (32768u + kB);        // both CTAs' dense A and B bytes
@@ -84,11 +94,12 @@ struct Cfg {
 };
 }  // namespace pair
 
-template <bool HYB, bool DB>
+template <bool HYB, bool DB, bool I8>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pair::kThreads, 1)
     spmm_pair_kernel(const __grid_constant__ SpmmParams p) {
   using namespace pair;
-  using C = Cfg<HYB, DB>;
+  using C = Cfg<HYB, DB, I8>;
+  constexpr uint32_t kE = C::kE;
   constexpr int kStages = C::kStages;
   constexpr uint32_t kA = C::kA;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -171,8 +182,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pair::kThreads, 1)
             tc_fence_after();
             const uint32_t a_addr = smem_u32(smem + L.a + s * kA);
             const uint32_t b_addr = smem_u32(smem + L.b + s * kB);
-            const uint32_t e_tmem = tmem_base + C::kECol + 4u * s;
-            if (tile_sparse(tm, kt, 0) && tile_sparse(tm, kt, 1)) {
+            const uint32_t e_tmem = tmem_base + C::kECol + C::kECols * s;
+            if (I8) {  // four K = 64 steps: 32 stored bytes of A and 64 rows (8 KB) of B each
+              tc_cp_128x256b_pair(e_tmem, smem_desc(smem_u32(smem + L.e + s * kE), 128, 256, SWZ_NONE));
+#pragma unroll
+              for (int kk = 0; kk < 4; ++kk) {
+                const uint64_t ad = smem_desc(a_addr + kk * 32, 16, 1024, SWZ_128B);
+                const uint64_t bd = smem_desc(b_addr + kk * 8192, 32768, 1024, SWZ_128B);
+                tc_mma_sp_pair_i8(d_tmem, ad, bd, e_tmem + 2u * (uint32_t)kk, C::kIdesc,
+                                  (kt > 0 || kk > 0) ? 1u : 0u);
+              }
+            } else if (tile_sparse(tm, kt, 0) && tile_sparse(tm, kt, 1)) {
               tc_cp_128x128b_pair(e_tmem, smem_desc(smem_u32(smem + L.e + s * kE), 2048, 128, SWZ_NONE));
 #pragma unroll
               for (int kk = 0; kk < 4; ++kk) {
@@ -221,8 +241,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pair::kThreads, 1)
               const int h = warp == 10;
               if (rank == 0 && h == 0) mbar_arrive_expect_tx(&full[s], sparse ? C::kTxSparse : C::kTxDense);
               if (sparse) {
-                tma_load_2d_pair(smem + L.a + s * kA + h * 8192, &p.tm_vals, lead_full, (int32_t)(kt * 64),
-                                 row0 + 64 * h);
+                tma_load_2d_pair(smem + L.a + s * kA + h * 8192, &p.tm_vals, lead_full,
+                                 (int32_t)(kt * (I8 ? 128 : 64)), row0 + 64 * h);
               } else if (HYB) {  // this CTA's dense tile: W, or W under the 2:4 mask if the tile is 2:4
                 const CUtensorMap* src = tile_sparse(tm, kt, (int)rank) ? &p.tm_wm : &p.tm_w;
 #pragma unroll
@@ -230,10 +250,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pair::kThreads, 1)
                   tma_load_2d_pair(smem + L.a + s * kA + kh * 16384 + h * 8192, src, lead_full,
                                    (int32_t)(kt * 128 + 64 * kh), row0 + 64 * h);
               }
-            } else if (warp <= 5) {  // box (strip j, K half h): 64 columns x 64 rows of X
-              const int j = (warp - 2) >> 1, h = (warp - 2) & 1;
-              tma_load_2d_pair(smem + L.b + s * kB + j * 16384 + h * 8192, &p.tm_x, lead_full, col0 + 64 * j,
-                               (int32_t)(kt * 128 + 64 * h));
+            } else if (warp <= 5) {
+              if (I8) {  // box K quarter q: 128 int8 columns x 64 rows of X
+                const int q = warp - 2;
+                tma_load_2d_pair(smem + L.b + s * kB + q * 8192, &p.tm_x, lead_full, col0,
+                                 (int32_t)(kt * 256 + 64 * q));
+              } else {  // box (strip j, K half h): 64 columns x 64 rows of X
+                const int j = (warp - 2) >> 1, h = (warp - 2) & 1;
+                tma_load_2d_pair(smem + L.b + s * kB + j * 16384 + h * 8192, &p.tm_x, lead_full, col0 + 64 * j,
+                                 (int32_t)(kt * 128 + 64 * h));
+              }
+            } else if (I8) {  // the 4 KB chunk (128-row block, K block kt): 16 rows of 256 bytes
+              tma_load_2d_pair(smem + L.e + s * kE, &p.tm_meta, lead_full, 0,
+                               (int32_t)(((int64_t)(row0 / 128) * p.meta_cblocks + kt) * 16));
             } else if (sparse) {  // eight 16-row metadata blocks of column block kt
               tma_load_3d_pair(smem + L.e + s * kE, &p.tm_meta, lead_full, 0, (int32_t)kt, row0 / 16);
             }
@@ -382,22 +411,23 @@ bool pair_kernel_fits(const SpmmParams& p) {
   return p.a_mode == A_TMA_SPARSE && p.K % 128 == 0 && p.K > 0 && p.T >= 192 && p.R >= 1 && p.T % 8 == 0;
 }
 
-template <bool HYB, bool DB>
+template <bool HYB, bool DB, bool I8 = false>
 static cudaError_t launch_pair(SpmmParams& p, cudaStream_t stream) {
-  constexpr pair::Layout L = pair::Cfg<HYB, DB>::layout();
+  constexpr pair::Layout L = pair::Cfg<HYB, DB, I8>::layout();
   const size_t bytes = L.total + 1024;
   static bool configured[64] = {};
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 64 && !configured[dev]) {
     cudaError_t e =
-        cudaFuncSetAttribute(spmm_pair_kernel<HYB, DB>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+        cudaFuncSetAttribute(spmm_pair_kernel<HYB, DB, I8>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
     if (e != cudaSuccess) return e;
     configured[dev] = true;
   }
   const int pairs_avail = sm_count_current() / 2;
   const int pairs = p.num_tiles < pairs_avail ? p.num_tiles : pairs_avail;
-  cudaError_t e = launch_pdl(spmm_pair_kernel<HYB, DB>, dim3(2 * pairs), dim3(pair::kThreads), bytes, stream, p);
+  cudaError_t e =
+      launch_pdl(spmm_pair_kernel<HYB, DB, I8>, dim3(2 * pairs), dim3(pair::kThreads), bytes, stream, p);
   count_launch();
   return e != cudaSuccess ? e : cudaGetLastError();
 }
@@ -420,5 +450,7 @@ cudaError_t launch_spmm_pair(SpmmParams& p, cudaStream_t stream) {
 }
 
 cudaError_t launch_spmm_pair_hybrid(SpmmParams& p, cudaStream_t stream) { return launch_pair<true, false>(p, stream); }
+
+cudaError_t launch_spmm_pair_i8(SpmmParams& p, cudaStream_t stream) { return launch_pair<false, false, true>(p, stream); }
 
 }  // namespace nmk
