@@ -938,9 +938,10 @@ def run_i8(args, rank: int, world: int, dist):
                        "parallelism": f"replicas x{world}"},
             "roofline": {"bound": "tensor", "achieved": achieved, "peak": i8_peak, "unit": "TOP/s",
                          "frac": achieved / i8_peak, "traffic": None,
-                         "kernel": "nm_spmm_i8 calls: decompress_2of4_i8_kernel + dense_pair_kernel (kind::i8)",
+                         "kernel": "nm_spmm_i8 calls: relayout_meta_i8_kernel + spmm_pair_kernel (sparse kind::i8)",
                          "peak_source": f"{peak_src} bf16 burst dense peak x 2 (the nominal int8 / bf16 dense ratio); "
-                                        "useful (survivor) operations, half of the dense ones",
+                                        "useful (survivor) operations, which the sparse MMA executes at twice the "
+                                        "dense rate",
                          "timing": "CUDA events around back-to-back repetitions of the step's GEMM calls"},
             "gpu_launches": launches, "clocks": sampler.summary() if sampler else None, "cpu_baseline": None}
     if rank == 0:

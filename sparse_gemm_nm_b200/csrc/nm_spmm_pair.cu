@@ -149,7 +149,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pair::kThreads, 1)
   const uint32_t tmem_base = *tmem_slot;
   pdl_gate();  // no global memory touched before this point
 
-  const int64_t k_tiles = p.K / 128;
+  const int64_t k_tiles = p.k_tiles;  // 128-deep stages (bf16) or 256-deep (int8), set by the host
   const uint32_t lead_full0 = map_to_cta(smem_u32(&full[0]), 0);
   const uint32_t lead_acc_empty0 = map_to_cta(smem_u32(acc_empty), 0);
   bool ok = true;
@@ -278,21 +278,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pair::kThreads, 1)
     int acc = 0;
     for (int tile = pair_id; tile < p.num_tiles && ok; tile += npairs) {
       const int tm = tile % p.tiles_m, tn = tile / p.tiles_m;
-      const int64_t row = (int64_t)tm * 256 + 128 * rank + quarter * 32 + lane;
       const int64_t n0 = (int64_t)tn * C::kN;
       ok = mbar_wait(&acc_full[acc], (aph >> acc) & 1u, abort_flag, p.status, kWaitNs);
       if (!ok) break;
       tc_fence_after();
       const uint32_t t_addr = tmem_base + 256u * (uint32_t)acc + ((uint32_t)(quarter * 32) << 16);
       const uint32_t lead_acc_empty = lead_acc_empty0 + 8u * (uint32_t)acc;
-      const bool row_ok = row < p.R;
       if (DB && !p.out_f32) {
         // Three 64-column chunks through the warp's staging buffer, one TMA
         // store each.  The accumulator is released after the last TMEM load; the
         // next tile's MMAs run in the other accumulator meanwhile, so this
         // epilogue has a whole tile period to finish.
         const int32_t wrow0 = (int32_t)(tm * 256 + 128 * rank + quarter * 32);
-        uint8_t* ebuf = smem + L.epi + quarter * kEpi;
+        uint8_t* ebuf = smem + L.epi + quarter * (C::kEpiBufs * kEpi);
 #pragma unroll
         for (int c = 0; c < 3; ++c) {
           uint32_t v0[32], v1[32];
@@ -345,7 +343,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pair::kThreads, 1)
         __syncwarp();
         if (lane == 0) mbar_arrive_cluster(lead_acc_empty);
         const int32_t wrow0 = (int32_t)(tm * 256 + 128 * rank + quarter * 32);
-        uint8_t* ebuf = smem + L.epi + quarter * kEpi;
+        uint8_t* ebuf = smem + L.epi + quarter * (C::kEpiBufs * kEpi);
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
           if (lane == 0) bulk_wait_group_read<0>();  // the previous store has read the buffer
@@ -362,31 +360,42 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pair::kThreads, 1)
           }
         }
       } else {
+        // 32-bit results (fp32, or the int32 accumulator bits): 32-column chunks
+        // (128-byte rows) through the warp's 128-byte-swizzled staging buffer, one
+        // TMA store each (tm_y encodes 4-byte elements, box 32 x 32).  The next
+        // chunk's TMEM load is issued before waiting for the previous store to
+        // read the buffer; the accumulator is released after the last load.
+        const int32_t wrow0 = (int32_t)(tm * 256 + 128 * rank + quarter * 32);
+        uint8_t* ebufs = smem + L.epi + quarter * (C::kEpiBufs * kEpi);
+        constexpr int kChunks = (int)(C::kN / 32);
+        uint32_t v[32];
+        tmem_ld_32x32b_x32(t_addr, v);
+        tc_wait_ld();
 #pragma unroll 1
-        for (int c = 0; c < (int)(C::kN / 16); ++c) {
-          uint32_t v[16];
-          tmem_ld_32x32b_x16(t_addr + c * 16, v);
-          tc_wait_ld();
-          if (!row_ok) continue;
-          const int64_t col0 = n0 + c * 16;
-          if (p.out_f32) {
-            float* yrow = static_cast<float*>(p.Y) + row * p.ldy;
+        for (int c = 0; c < kChunks; ++c) {
+          uint8_t* ebuf = ebufs + (c % C::kEpiBufs) * kEpi;
+          if (lane == 0) bulk_wait_group_read<C::kEpiBufs - 1>();  // this buffer's last store has read it
+          __syncwarp();
 #pragma unroll
-            for (int e = 0; e < 16; ++e)
-              if (col0 + e < p.T) yrow[col0 + e] = __uint_as_float(v[e]);
-          } else {
-            uint16_t* yrow = static_cast<uint16_t*>(p.Y) + row * p.ldy;
-#pragma unroll
-            for (int e = 0; e < 16; e += 2) {
-              const uint32_t pk = pack_bf16x2(__uint_as_float(v[e]), __uint_as_float(v[e + 1]));
-              if (col0 + e < p.T) yrow[col0 + e] = (uint16_t)(pk & 0xFFFFu);
-              if (col0 + e + 1 < p.T) yrow[col0 + e + 1] = (uint16_t)(pk >> 16);
-            }
+          for (int j = 0; j < 8; ++j)
+            *reinterpret_cast<uint4*>(ebuf + lane * 128 + ((j ^ (lane & 7)) << 4)) =
+                make_uint4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0 && n0 + 32 * c < p.T && wrow0 < p.R) {
+            tma_store_2d(&p.tm_y, ebuf, (int32_t)(n0 + 32 * c), wrow0);
+            bulk_commit_group();
+          }
+          if (c + 1 < kChunks) {
+            tmem_ld_32x32b_x32(t_addr + (c + 1) * 32, v);
+            tc_wait_ld();
+          }
+          if (c + 2 == kChunks || kChunks == 1) {  // the last TMEM load is done
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive_cluster(lead_acc_empty);
           }
         }
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive_cluster(lead_acc_empty);
       }
       aph ^= 1u << acc;
       if (C::kAcc == 2) acc ^= 1;
