@@ -1194,6 +1194,51 @@ static nm_status run_spmm_tf32(const float* values, const uint32_t* meta, int64_
   cudaMemPool_t pool = nullptr;
   cudaError_t e = staging_pool(&pool);
   if (e != cudaSuccess) return cuda_fail(e, "staging pool");
+  // The sparse tensor cores (kind::tf32 on SM pairs) when the shape fills pair tiles: the 1-bit row-wise
+  // positions are re-laid out into the MMA's metadata order (R x K / 8 bytes staged) and the compressed
+  // values are read as they are.
+  if (T >= 192 && K % 8 == 0 && al16(values)) {
+    const int64_t rblocks128 = (R + 255) / 256 * 2, kblocks = (K + 63) / 64;
+    void* em = nullptr;
+    e = cudaMallocFromPoolAsync(&em, (size_t)(rblocks128 * kblocks * 4096), pool, stream);
+    if (e != cudaSuccess) return cuda_fail(e, "staging buffer for the tf32 metadata");
+    e = launch_relayout_meta_tf32(meta, R, K, static_cast<uint32_t*>(em), rblocks128, stream);
+    SpmmParams p;
+    std::memset(&p, 0, sizeof p);
+    p.R = R;
+    p.K = K;
+    p.T = T;
+    p.n = 1;
+    p.m = 2;
+    p.Y = Y;
+    p.ldy = ldy;
+    p.out_f32 = dtype == NM_OUT_F32;
+    p.a_mode = A_TMA_SPARSE;
+    p.pattern = PAT_1_2;
+    p.vcols = K / 2;
+    p.meta_cblocks = kblocks;
+    p.k_tiles = kblocks;
+    p.tiles_m = (int)((R + 255) / 256);
+    p.tiles_n = (int)((T + 255) / 256);
+    p.num_tiles = p.tiles_m * p.tiles_n;
+    p.status = status_word_ptr();
+    if (e == cudaSuccess && !p.status) e = cudaErrorInvalidSymbol;
+    if ((int64_t)p.tiles_m * p.tiles_n >= (1ll << 31)) st = fail(NM_ERR_UNSUPPORTED, "too many tiles");
+    if (e == cudaSuccess && st == NM_OK)
+      st = make_tmap(&p.tm_vals, values, (uint64_t)(K / 2), (uint64_t)R, (uint64_t)(K / 2) * 4, 32, kPairBoxRows, 128,
+                     "values (float32)", CU_TENSOR_MAP_DATA_TYPE_FLOAT32);
+    if (e == cudaSuccess && st == NM_OK)
+      st = make_tmap(&p.tm_x, X, (uint64_t)T, (uint64_t)K, (uint64_t)ldx * 4, 32, kPairBoxRows, kSwizzle128Atom32B,
+                     "X (float32)", CU_TENSOR_MAP_DATA_TYPE_FLOAT32);
+    if (e == cudaSuccess && st == NM_OK)
+      st = make_tmap(&p.tm_meta, em, 256, (uint64_t)(rblocks128 * kblocks * 16), 256, 256, 16, 0,
+                     "metadata (tf32 order)", CU_TENSOR_MAP_DATA_TYPE_UINT8);
+    if (e == cudaSuccess && st == NM_OK) st = make_pair_store_map(&p.tm_y, Y, R, T, ldy, p.out_f32 != 0);
+    if (e == cudaSuccess && st == NM_OK) e = launch_spmm_pair_tf32(p, stream);
+    cudaFreeAsync(em, stream);
+    if (st != NM_OK) return st;
+    return e == cudaSuccess ? NM_OK : cuda_fail(e, "tf32 sparse GEMM launch");
+  }
   const int64_t ldk = (K + 3) / 4 * 4;  // 16-byte rows for the TMA
   void* wd = nullptr;
   e = cudaMallocFromPoolAsync(&wd, (size_t)(R * ldk * 4), pool, stream);

@@ -281,6 +281,21 @@ __device__ __forceinline__ void tc_mma_sp_pair_i8(uint32_t d_tmem, uint64_t a_de
       : "memory");
 }
 
+// Sparse kind::tf32 on SM pairs: 1:2 A (32 stored bytes per row for K = 16), TF32 B, fp32 accumulator.  Its
+// metadata takes one TMEM column per K = 16 step, in the kind::f16 order with a group of four 16-bit slots
+// standing for one pair of TF32 elements: lane l of a 16-row block holds rows l % 8 (bits 0-15) and
+// 8 + l % 8 (bits 16-31), pairs 4 (l / 8) .. 4 (l / 8) + 3, the nibble 0x4 keeping a pair's first element
+// and 0xE its second; sparsity selector 0.
+__device__ __forceinline__ void tc_mma_sp_pair_tf32(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                                    uint32_t e_tmem, uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %5, 0;\n\t"
+      "tcgen05.mma.sp.cta_group::2.kind::tf32 [%0], %1, %2, [%3], %4, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(e_tmem), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
 // Arrive once on the mbarrier at this shared offset in every CTA of cta_mask
 // when all previously issued pair tcgen05 operations have completed.
 __device__ __forceinline__ void tc_commit_pair(uint64_t* bar, uint16_t cta_mask) {

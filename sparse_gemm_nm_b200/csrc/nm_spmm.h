@@ -130,6 +130,12 @@ cudaError_t launch_spmm_pair_hybrid(SpmmParams& p, cudaStream_t stream);
 cudaError_t launch_spmm_pair_i8(SpmmParams& p, cudaStream_t stream);
 cudaError_t launch_relayout_meta_i8(const uint32_t* meta, int64_t R, int64_t K, uint32_t* out, int64_t rblocks128,
                                     cudaStream_t s);
+// TF32 1:2 on SM pairs (sparse kind::tf32): tm_vals fp32 values R x K/2 (box {32, 64}), tm_x fp32 X (box {32, 64},
+// 128-byte swizzle in 32-byte units), tm_meta the re-laid-out metadata (box {256, 16}), meta_cblocks = its 64-deep
+// K blocks; Y bf16 or fp32.
+cudaError_t launch_spmm_pair_tf32(SpmmParams& p, cudaStream_t stream);
+cudaError_t launch_relayout_meta_tf32(const uint32_t* meta, int64_t R, int64_t K, uint32_t* out, int64_t rblocks128,
+                                      cudaStream_t s);
 bool skinny_kernel_fits(int64_t T);
 int skinny_bn(int64_t T);
 int skinny_kd(int64_t K, int64_t T);

@@ -44,6 +44,11 @@
 // 128 int8 columns (32 KB, four 64-row boxes), and the metadata 4 KB per CTA in
 // the per-row order that MMA reads (relayout_meta_i8_kernel), copied into 8
 // TMEM columns; four K = 64 MMAs per stage, int32 accumulators stored as such.
+// TF32 1:2 (TF32): the same on the sparse kind::tf32 MMA.  A stage covers 64
+// logical K: A 128 rows x 32 stored fp32, B 64 rows x 128 fp32 columns (four
+// 32-column strips in the 32-byte-unit swizzle the MMA reads for MN-major
+// 32-bit operands), 4 KB of metadata (relayout_meta_tf32_kernel); four K = 16
+// MMAs per stage, each with its own even TMEM metadata column.
 #include <cstdint>
 #include <cuda.h>
 #include <cuda_runtime.h>
@@ -69,18 +74,20 @@ struct Layout {
 // HYB = true (PATCH hybrid): A slots of 32 KB so that a stage can hold the
 // dense 128 x 128 tile instead, three stages.
 // DB = true (2:4, short tiles): 256 x 192 tiles, two accumulators, four stages.
-template <bool HYB, bool DB = false, bool I8 = false>
+template <bool HYB, bool DB = false, bool I8 = false, bool TF32 = false>
 struct Cfg {
-  static_assert(!(I8 && (HYB || DB)), "int8 runs the 256 x 256 sparse form only");
+  static_assert(!((I8 || TF32) && (HYB || DB)) && !(I8 && TF32), "int8 / tf32 run the 256 x 256 sparse form only");
+  static constexpr bool kWideE = I8 || TF32;  // 4 KB metadata chunks staged per row block and stage
   static constexpr int kStages = HYB ? 3 : 4;
   static constexpr uint32_t kN = DB ? 192u : 256u;  // pair tile columns (per CTA: kN / 2 of X)
   static constexpr int kAcc = DB ? 2 : 1;           // accumulators, 256 TMEM columns apart
   static constexpr uint32_t kECol = DB ? 448u : 256u;
-  static constexpr uint32_t kE = I8 ? 4096u : 2048u;  // metadata bytes per stage and CTA
-  static constexpr uint32_t kECols = I8 ? 8u : 4u;    // its TMEM columns
+  static constexpr uint32_t kE = kWideE ? 4096u : 2048u;  // metadata bytes per stage and CTA
+  static constexpr uint32_t kECols = kWideE ? 8u : 4u;    // its TMEM columns
   static constexpr int kEpiBufs = 1;
-  static constexpr uint32_t kIdesc = I8 ? (idesc_s8_major(256, 256, false, true) | (1u << 2))
-                                        : idesc_bf16(kN, true, 256);
+  static constexpr uint32_t kIdesc = I8     ? (idesc_s8_major(256, 256, false, true) | (1u << 2))
+                                     : TF32 ? (idesc_tf32_major(256, 256, false, true) | (1u << 2))
+                                            : idesc_bf16(kN, true, 256);
   static constexpr uint32_t kA = HYB ? 32768u : 16384u;
   static constexpr uint32_t kTxSparse = 2u * (16384u + kB + kE);  // both CTAs' A, B and E bytes
   static constexpr uint32_t kTxDense = 2u * (32768u + kB);        // both CTAs' dense A and B bytes
@@ -94,11 +101,11 @@ struct Cfg {
 };
 }  // namespace pair
 
-template <bool HYB, bool DB, bool I8>
+template <bool HYB, bool DB, bool I8, bool TF32>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pair::kThreads, 1)
     spmm_pair_kernel(const __grid_constant__ SpmmParams p) {
   using namespace pair;
-  using C = Cfg<HYB, DB, I8>;
+  using C = Cfg<HYB, DB, I8, TF32>;
   constexpr uint32_t kE = C::kE;
   constexpr int kStages = C::kStages;
   constexpr uint32_t kA = C::kA;
@@ -192,6 +199,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pair::kThreads, 1)
                 tc_mma_sp_pair_i8(d_tmem, ad, bd, e_tmem + 2u * (uint32_t)kk, C::kIdesc,
                                   (kt > 0 || kk > 0) ? 1u : 0u);
               }
+            } else if (TF32) {  // four K = 16 steps: 32 bytes of A and 16 rows (2 KB per strip) of B each
+              tc_cp_128x256b_pair(e_tmem, smem_desc(smem_u32(smem + L.e + s * kE), 128, 256, SWZ_NONE));
+#pragma unroll
+              for (int kk = 0; kk < 4; ++kk) {
+                const uint64_t ad = smem_desc(a_addr + kk * 32, 16, 1024, SWZ_128B);
+                const uint64_t bd = smem_desc(b_addr + kk * 2048, 8192, 512, SWZ_128B_BASE32B);
+                tc_mma_sp_pair_tf32(d_tmem, ad, bd, e_tmem + 2u * (uint32_t)kk, C::kIdesc,
+                                    (kt > 0 || kk > 0) ? 1u : 0u);
+              }
             } else if (tile_sparse(tm, kt, 0) && tile_sparse(tm, kt, 1)) {
               tc_cp_128x128b_pair(e_tmem, smem_desc(smem_u32(smem + L.e + s * kE), 2048, 128, SWZ_NONE));
 #pragma unroll
@@ -242,7 +258,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pair::kThreads, 1)
               if (rank == 0 && h == 0) mbar_arrive_expect_tx(&full[s], sparse ? C::kTxSparse : C::kTxDense);
               if (sparse) {
                 tma_load_2d_pair(smem + L.a + s * kA + h * 8192, &p.tm_vals, lead_full,
-                                 (int32_t)(kt * (I8 ? 128 : 64)), row0 + 64 * h);
+                                 (int32_t)(kt * (I8 ? 128 : TF32 ? 32 : 64)), row0 + 64 * h);
               } else if (HYB) {  // this CTA's dense tile: W, or W under the 2:4 mask if the tile is 2:4
                 const CUtensorMap* src = tile_sparse(tm, kt, (int)rank) ? &p.tm_wm : &p.tm_w;
 #pragma unroll
@@ -255,12 +271,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pair::kThreads, 1)
                 const int q = warp - 2;
                 tma_load_2d_pair(smem + L.b + s * kB + q * 8192, &p.tm_x, lead_full, col0,
                                  (int32_t)(kt * 256 + 64 * q));
+              } else if (TF32) {  // strip j: 32 fp32 columns x 64 rows of X
+                const int j = warp - 2;
+                tma_load_2d_pair(smem + L.b + s * kB + j * 8192, &p.tm_x, lead_full, col0 + 32 * j,
+                                 (int32_t)(kt * 64));
               } else {  // box (strip j, K half h): 64 columns x 64 rows of X
                 const int j = (warp - 2) >> 1, h = (warp - 2) & 1;
                 tma_load_2d_pair(smem + L.b + s * kB + j * 16384 + h * 8192, &p.tm_x, lead_full, col0 + 64 * j,
                                  (int32_t)(kt * 128 + 64 * h));
               }
-            } else if (I8) {  // the 4 KB chunk (128-row block, K block kt): 16 rows of 256 bytes
+            } else if (C::kWideE) {  // the 4 KB chunk (128-row block, K block kt): 16 rows of 256 bytes
               tma_load_2d_pair(smem + L.e + s * kE, &p.tm_meta, lead_full, 0,
                                (int32_t)(((int64_t)(row0 / 128) * p.meta_cblocks + kt) * 16));
             } else if (sparse) {  // eight 16-row metadata blocks of column block kt
@@ -420,23 +440,23 @@ bool pair_kernel_fits(const SpmmParams& p) {
   return p.a_mode == A_TMA_SPARSE && p.K % 128 == 0 && p.K > 0 && p.T >= 192 && p.R >= 1 && p.T % 8 == 0;
 }
 
-template <bool HYB, bool DB, bool I8 = false>
+template <bool HYB, bool DB, bool I8 = false, bool TF32 = false>
 static cudaError_t launch_pair(SpmmParams& p, cudaStream_t stream) {
-  constexpr pair::Layout L = pair::Cfg<HYB, DB, I8>::layout();
+  constexpr pair::Layout L = pair::Cfg<HYB, DB, I8, TF32>::layout();
   const size_t bytes = L.total + 1024;
   static bool configured[64] = {};
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 64 && !configured[dev]) {
-    cudaError_t e =
-        cudaFuncSetAttribute(spmm_pair_kernel<HYB, DB, I8>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+    cudaError_t e = cudaFuncSetAttribute(spmm_pair_kernel<HYB, DB, I8, TF32>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
     if (e != cudaSuccess) return e;
     configured[dev] = true;
   }
   const int pairs_avail = sm_count_current() / 2;
   const int pairs = p.num_tiles < pairs_avail ? p.num_tiles : pairs_avail;
   cudaError_t e =
-      launch_pdl(spmm_pair_kernel<HYB, DB, I8>, dim3(2 * pairs), dim3(pair::kThreads), bytes, stream, p);
+      launch_pdl(spmm_pair_kernel<HYB, DB, I8, TF32>, dim3(2 * pairs), dim3(pair::kThreads), bytes, stream, p);
   count_launch();
   return e != cudaSuccess ? e : cudaGetLastError();
 }
@@ -461,5 +481,9 @@ cudaError_t launch_spmm_pair(SpmmParams& p, cudaStream_t stream) {
 cudaError_t launch_spmm_pair_hybrid(SpmmParams& p, cudaStream_t stream) { return launch_pair<true, false>(p, stream); }
 
 cudaError_t launch_spmm_pair_i8(SpmmParams& p, cudaStream_t stream) { return launch_pair<false, false, true>(p, stream); }
+
+cudaError_t launch_spmm_pair_tf32(SpmmParams& p, cudaStream_t stream) {
+  return launch_pair<false, false, false, true>(p, stream);
+}
 
 }  // namespace nmk

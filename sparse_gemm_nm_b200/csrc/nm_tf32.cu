@@ -104,6 +104,51 @@ __global__ void __launch_bounds__(256) decompress_1of2_f32_kernel(const uint32_t
   }
 }
 
+// Metadata of the sparse kind::tf32 MMA (TMEM order in tc_mma_sp_pair_tf32): per 128-row block and
+// 64-deep K stage (32 pairs: one stored word per row), one 4 KB chunk that tcgen05.cp (128 lanes x 256
+// bits, no swizzle) moves into 8 TMEM columns; the four K = 16 steps of the stage take columns 0, 2, 4, 6
+// (odd columns stay 0).  Lane L of the chunk: rows 16 (L / 16) + L % 8 and + 8, pairs 4 ((L % 16) / 8) ..
+// + 3 of each step.  Pairs or rows outside R x K/2 get the nibble 0x4 (their values are zero).  Chunk
+// layout as the int8 one: half c of lanes 8j .. 8j + 7 at 256 j + 128 c, 16 bytes per lane.
+__global__ void __launch_bounds__(256) relayout_meta_tf32_kernel(const uint32_t* __restrict__ meta, int64_t R,
+                                                                int64_t npairs, int64_t mcols, uint32_t kblocks,
+                                                                uint32_t* __restrict__ out, uint32_t total) {
+  pdl_gate();
+  for (uint32_t i = blockIdx.x * blockDim.x + threadIdx.x; i < total; i += gridDim.x * blockDim.x) {
+    const uint32_t chunk = i >> 10, within = i & 1023u;
+    const uint32_t L = within >> 3, w = within & 7u;  // lane, word (TMEM column) of the lane
+    const uint32_t rb128 = chunk / kblocks, kb = chunk - rb128 * kblocks;
+    uint32_t word = 0u;
+    if ((w & 1u) == 0u) {
+      const uint32_t kk = w >> 1, l = L & 15u, h = l >> 3;
+      const int64_t r0 = (int64_t)rb128 * 128 + 16 * (L >> 4) + (l & 7u);
+      word = 0x44444444u;
+      for (int half = 0; half < 2; ++half) {
+        const int64_t r = r0 + 8 * half;
+        if (r >= R) continue;
+        const int64_t p0 = (int64_t)kb * 32 + kk * 8 + 4 * h;  // first of the four pairs
+        const uint32_t bits = p0 < npairs ? (__ldg(meta + r * mcols + kb) >> (kk * 8 + 4 * h)) & 0xFu : 0u;
+        for (int t = 0; t < 4; ++t) {
+          const bool second = p0 + t < npairs && ((bits >> t) & 1u);
+          if (second) word = (word & ~(0xFu << (16 * half + 4 * t))) | (0xEu << (16 * half + 4 * t));
+        }
+      }
+    }
+    out[(int64_t)chunk * 1024 + (L >> 3) * 64 + (w >> 2) * 32 + (L & 7u) * 4 + (w & 3u)] = word;
+  }
+}
+
+cudaError_t launch_relayout_meta_tf32(const uint32_t* meta, int64_t R, int64_t K, uint32_t* out, int64_t rblocks128,
+                                      cudaStream_t s) {
+  const int64_t kblocks = (K + 63) / 64;
+  const int64_t total = rblocks128 * kblocks * 1024;
+  const int64_t npairs = K / 2, mcols = (npairs + 31) / 32;
+  cudaError_t e = launch_pdl(relayout_meta_tf32_kernel, dim3(grid_of(total, 256)), dim3(256), 0, s, meta, R, npairs,
+                             mcols, (uint32_t)kblocks, out, (uint32_t)total);
+  count_launch();
+  return e != cudaSuccess ? e : cudaGetLastError();
+}
+
 static int aligned16_rows(const void* p, int64_t ld) { return (reinterpret_cast<uintptr_t>(p) % 16 == 0 && ld % 4 == 0) ? 1 : 0; }
 static int aligned8_rows(const void* p, int64_t ld) { return (reinterpret_cast<uintptr_t>(p) % 8 == 0 && ld % 2 == 0) ? 1 : 0; }
 
