@@ -251,11 +251,15 @@ NM_API nm_status nm_prune_spmm(const uint16_t* W, int64_t ldw, int n, int m, int
  * nm_decompress_i8: W_out R x K int8 (ldw % 16 == 0, 16-byte aligned), 0 at
  *   the pruned positions.
  * nm_spmm_i8: Y = W' X exactly in int32, X K x T int8 (ldx % 16 == 0, 16-byte
- *   aligned), Y R x T int32 (ldy % 4 == 0, 16-byte aligned).  The operand is
- *   decompressed into a staging buffer (R x K bytes from the library's pool,
- *   one launch), then a dense tcgen05 kind::i8 GEMM on SM pairs (a second
- *   launch).  |W'| <= 128 and |X| <= 128, so a sum overflows int32 only for
- *   K > 131072; the call does not check.
+ *   aligned), Y R x T int32 (ldy % 4 == 0, 16-byte aligned).  With T >= 192,
+ *   K % 32 == 0 and 16-byte aligned values it runs on the sparse tensor cores
+ *   (tcgen05 kind::i8 on SM pairs): the tiled metadata is first re-laid out
+ *   into the order that MMA reads (one launch, 4 KB per 128 rows and 256
+ *   columns staged from the library's pool), then the GEMM (a second
+ *   launch).  Other shapes: the operand is decompressed into a staging buffer
+ *   (R x K bytes) and multiplied by a dense kind::i8 GEMM.  |W'| <= 128 and
+ *   |X| <= 128, so a sum overflows int32 only for K > 131072; the call does
+ *   not check.
  * Errors: NM_ERR_INVALID_ARG, NM_ERR_UNSUPPORTED, NM_ERR_MISALIGNED, NM_ERR_CUDA.
  */
 NM_API nm_status nm_prune_compress_i8(const int8_t* W, int64_t R, int64_t K, int64_t ldw, int8_t* values,
@@ -281,12 +285,16 @@ NM_API nm_status nm_spmm_i8(const int8_t* values, const uint32_t* meta, int64_t 
  * nm_decompress_tf32: W_out[r][2p + bit] = values[r][p], +0.0 at the other
  *   position (row stride ldw >= K).
  * nm_spmm_tf32: Y = W' X, X float32 K x T (row stride ldx >= T, ldx % 4 == 0,
- *   16-byte aligned), Y R x T bf16 or fp32 (y_dtype) as nm_spmm.  The
- *   operand is decompressed into a staged dense copy (R x ceil4(K) float32
- *   from the library's pool) and multiplied by a dense tcgen05 kind::tf32
- *   GEMM on SM pairs: the tensor cores read W' and X as TF32 (10 explicit
- *   mantissa bits) and accumulate in fp32, so Y meets the GEMM tolerance
- *   (|y - y_ref| <= 2^-7 sum |w||x|), not bit equality with an fp32 product.
+ *   16-byte aligned), Y R x T bf16 or fp32 (y_dtype) as nm_spmm.  With
+ *   T >= 192, K % 8 == 0 and 16-byte aligned values it runs on the sparse
+ *   tensor cores (tcgen05 kind::tf32 on SM pairs) after one pass that re-lays
+ *   the positions out into that MMA's metadata order (4 KB per 128 rows and
+ *   64 columns staged from the library's pool).  Other shapes: the operand
+ *   is decompressed into a staged dense copy (R x ceil4(K) float32) and
+ *   multiplied by a dense kind::tf32 GEMM.  Either way the tensor cores read
+ *   W' and X as TF32 (10 explicit mantissa bits) and accumulate in fp32, so Y
+ *   meets the GEMM tolerance (|y - y_ref| <= 2^-7 sum |w||x|), not bit
+ *   equality with an fp32 product.
  * Errors: NM_ERR_INVALID_ARG (odd K, negative sizes, ld too small, null),
  *   NM_ERR_MISALIGNED, NM_ERR_UNSUPPORTED (a dimension >= 2^31), NM_ERR_CUDA.
  */
