@@ -215,6 +215,12 @@ static nm_status make_meta_tmap(CUtensorMap* tm, const void* meta, int64_t rbloc
 
 static bool al16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+// Tile order of the SM-pair kernel: column tiles fastest when the compressed weights (R x vcols) exceed
+// 1.5x the dense input (K x T; same element size), so that the weights stream from HBM about once.
+static int pair_n_major(int64_t R, int64_t vcols, int64_t K, int64_t T) {
+  return (double)R * (double)vcols > 1.5 * (double)K * (double)T ? 1 : 0;
+}
+
 // Store map of the SM-pair kernel's epilogue: bf16 Y in 64-column x 32-row boxes, 32-bit Y (fp32,
 // or int32 accumulator bits) in 32 x 32 boxes; both 128-byte rows with the 128-byte swizzle.
 static nm_status make_pair_store_map(CUtensorMap* tm, void* Y, int64_t R, int64_t T, int64_t ldy, bool out32) {
@@ -543,6 +549,7 @@ static nm_status run_gemm(const GemmRequest& q, cudaStream_t stream) {
                      128, "values");
     if (st == NM_OK && !dense_pair) st = make_meta_tmap(&p.tm_meta, meta, p.meta_rblocks, p.meta_cblocks);
     if (st == NM_OK && !use_skinny) st = make_pair_store_map(&p.tm_y, q.Y, q.R, q.T, q.ldy, p.out_f32 != 0);
+    if (!use_skinny && !dense_pair) p.n_major = pair_n_major(q.R, p.vcols, q.K, q.T);
     if (st == NM_OK)
       e = use_skinny   ? launch_spmm_skinny(p, stream)
           : dense_pair ? launch_spmm_pair_hybrid(p, stream)
@@ -678,6 +685,7 @@ nm_status build_pair_params(SpmmParams& p, const uint16_t* values, const uint32_
                    "values");
   if (st == NM_OK) st = make_meta_tmap(&p.tm_meta, meta, p.meta_rblocks, p.meta_cblocks);
   if (st == NM_OK) st = make_pair_store_map(&p.tm_y, Y, R, T, ldy, out_f32);
+  p.n_major = pair_n_major(R, p.vcols, K, T);
   return st;
 }
 
@@ -1090,6 +1098,7 @@ static nm_status run_spmm_i8(const int8_t* values, const uint32_t* meta, int64_t
       st = make_tmap(&p.tm_meta, em, 256, (uint64_t)(rblocks128 * kblocks * 16), 256, 256, 16, 0,
                      "metadata (int8 order)", CU_TENSOR_MAP_DATA_TYPE_UINT8);
     if (e == cudaSuccess && st == NM_OK) st = make_pair_store_map(&p.tm_y, Y, R, T, ldy, true);
+    p.n_major = pair_n_major(R, K / 2, K, T);
     if (e == cudaSuccess && st == NM_OK) e = launch_spmm_pair_i8(p, stream);
     cudaFreeAsync(em, stream);
     if (st != NM_OK) return st;
@@ -1234,6 +1243,7 @@ static nm_status run_spmm_tf32(const float* values, const uint32_t* meta, int64_
       st = make_tmap(&p.tm_meta, em, 256, (uint64_t)(rblocks128 * kblocks * 16), 256, 256, 16, 0,
                      "metadata (tf32 order)", CU_TENSOR_MAP_DATA_TYPE_UINT8);
     if (e == cudaSuccess && st == NM_OK) st = make_pair_store_map(&p.tm_y, Y, R, T, ldy, p.out_f32 != 0);
+    p.n_major = pair_n_major(R, K / 2, K, T);
     if (e == cudaSuccess && st == NM_OK) e = launch_spmm_pair_tf32(p, stream);
     cudaFreeAsync(em, stream);
     if (st != NM_OK) return st;

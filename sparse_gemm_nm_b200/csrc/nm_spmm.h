@@ -47,6 +47,7 @@ struct SpmmParams {
   int permuted;
   int out_f32;
   int tiles_m, tiles_n, num_tiles;
+  int n_major;  // SM-pair kernel: column tiles go fastest (set when the compressed weights are larger than X)
   int hyb_tiles_k;
   int hyb_rows;  // tile-map rows, ceil(R / 128)
   int stages;

@@ -114,34 +114,48 @@ __global__ void __launch_bounds__(256) relayout_meta_tf32_kernel(const uint32_t*
                                                                 int64_t npairs, int64_t mcols, uint32_t kblocks,
                                                                 uint32_t* __restrict__ out, uint32_t total) {
   pdl_gate();
+  // one thread per (chunk, lane L): its four metadata words (even columns) and four zeros, two 16-byte stores
   for (uint32_t i = blockIdx.x * blockDim.x + threadIdx.x; i < total; i += gridDim.x * blockDim.x) {
-    const uint32_t chunk = i >> 10, within = i & 1023u;
-    const uint32_t L = within >> 3, w = within & 7u;  // lane, word (TMEM column) of the lane
+    const uint32_t chunk = i >> 7, L = i & 127u;
     const uint32_t rb128 = chunk / kblocks, kb = chunk - rb128 * kblocks;
-    uint32_t word = 0u;
-    if ((w & 1u) == 0u) {
-      const uint32_t kk = w >> 1, l = L & 15u, h = l >> 3;
-      const int64_t r0 = (int64_t)rb128 * 128 + 16 * (L >> 4) + (l & 7u);
-      word = 0x44444444u;
-      for (int half = 0; half < 2; ++half) {
-        const int64_t r = r0 + 8 * half;
-        if (r >= R) continue;
-        const int64_t p0 = (int64_t)kb * 32 + kk * 8 + 4 * h;  // first of the four pairs
-        const uint32_t bits = p0 < npairs ? (__ldg(meta + r * mcols + kb) >> (kk * 8 + 4 * h)) & 0xFu : 0u;
-        for (int t = 0; t < 4; ++t) {
-          const bool second = p0 + t < npairs && ((bits >> t) & 1u);
-          if (second) word = (word & ~(0xFu << (16 * half + 4 * t))) | (0xEu << (16 * half + 4 * t));
-        }
+    const uint32_t l = L & 15u, h = l >> 3;
+    const int64_t r0 = (int64_t)rb128 * 128 + 16 * (L >> 4) + (l & 7u);
+    uint32_t m[2] = {0u, 0u};  // the stage's stored word of rows r0 and r0 + 8 (bit p: position of pair p)
+    int64_t valid[2] = {0, 0};  // pairs of the stage inside K / 2
+    const int64_t p0 = (int64_t)kb * 32;
+    const int64_t inside = npairs - p0 < 32 ? npairs - p0 : 32;
+#pragma unroll
+    for (int half = 0; half < 2; ++half) {
+      const int64_t r = r0 + 8 * half;
+      if (r < R && inside > 0) {
+        m[half] = __ldg(meta + r * mcols + kb);
+        valid[half] = inside;
       }
     }
-    out[(int64_t)chunk * 1024 + (L >> 3) * 64 + (w >> 2) * 32 + (L & 7u) * 4 + (w & 3u)] = word;
+    uint32_t w[4];
+#pragma unroll
+    for (int kk = 0; kk < 4; ++kk) {
+      uint32_t word = 0x44444444u;
+#pragma unroll
+      for (int half = 0; half < 2; ++half)
+#pragma unroll
+        for (int t = 0; t < 4; ++t) {
+          const int q = kk * 8 + 4 * (int)h + t;  // pair of the stage
+          if (q < valid[half] && ((m[half] >> q) & 1u)) word ^= 0xAu << (16 * half + 4 * t);  // 0x4 -> 0xE
+        }
+      w[kk] = word;
+    }
+    // words 0..7 of lane L: half c (words 4c .. 4c + 3) at 256 (L / 8) + 128 c + 16 (L % 8) bytes
+    uint4* dst = reinterpret_cast<uint4*>(out + (int64_t)chunk * 1024 + (L >> 3) * 64 + (L & 7u) * 4);
+    dst[0] = make_uint4(w[0], 0u, w[1], 0u);
+    dst[8] = make_uint4(w[2], 0u, w[3], 0u);
   }
 }
 
 cudaError_t launch_relayout_meta_tf32(const uint32_t* meta, int64_t R, int64_t K, uint32_t* out, int64_t rblocks128,
                                       cudaStream_t s) {
   const int64_t kblocks = (K + 63) / 64;
-  const int64_t total = rblocks128 * kblocks * 1024;
+  const int64_t total = rblocks128 * kblocks * 128;  // one thread per chunk lane
   const int64_t npairs = K / 2, mcols = (npairs + 31) / 32;
   cudaError_t e = launch_pdl(relayout_meta_tf32_kernel, dim3(grid_of(total, 256)), dim3(256), 0, s, meta, R, npairs,
                              mcols, (uint32_t)kblocks, out, (uint32_t)total);
