@@ -150,8 +150,9 @@ def test_permuted_matches_oracle(n, m):
     check(W, X, n, m, idx=idx, what="permuted")
 
 
-def test_permuted_identity_equals_plain_and_host_permuted():
-    R, K, T = 256, 768, 256
+@pytest.mark.parametrize("K", [768, 2048])  # SM-pair kernel: 256 x 192 tiles (6 stages), 256 x 256 tiles (16)
+def test_permuted_identity_equals_plain_and_host_permuted(K):
+    R, T = 256, 256
     W = wl.normal_bf16((R, K), 0.02, seed=61)
     X = wl.normal_bf16((K, T), 1.0, seed=62)
     plain = run_spmm(W, X, 2, 4)
@@ -163,13 +164,16 @@ def test_permuted_identity_equals_plain_and_host_permuted():
     assert torch.equal(perm, host)  # same tiles, same MMA order: bitwise equal
 
 
-@pytest.mark.parametrize("T", [256, 16, 100])  # gather pass + SM-pair kernel, gather pass + skinny, one SM
-def test_permuted_out_of_range_entries_read_zero_rows(T):
-    R, K = 300, 512
+@pytest.mark.parametrize("K,T", [(512, 256),    # gather pass + SM-pair kernel, 256 x 192 tiles
+                                 (1280, 264),   # the same with 256 x 256 tiles and a ragged column tile
+                                 (512, 16),     # gather pass + split-K skinny kernel
+                                 (512, 100)])   # one-SM kernel gathering its own rows
+def test_permuted_out_of_range_entries_read_zero_rows(K, T):
+    R = 300
     W = wl.normal_bf16((R, K), 0.02, seed=74)
     X = wl.normal_bf16((K, T), 1.0, seed=75)
     idx = wl.permutation(K, 76).astype(np.int32)
-    idx[[0, 5, 130, 257, 511]] = [-1, K, K + 1000, -(2 ** 31), 2 ** 31 - 1]
+    idx[[0, 5, 130, 257, K - 1]] = [-1, K, K + 1000, -(2 ** 31), 2 ** 31 - 1]
     ld = (T + 7) // 8 * 8
     Xbuf = np.zeros((K, ld), np.uint16)
     Xbuf[:, :T] = X
@@ -328,19 +332,21 @@ def test_pair_kernel_integer_exact(out):
         assert np.array_equal(bits(Y), bf16_rne_of(ref))
 
 
-def test_permuted_pair_path_after_release_staging():
-    """The two-SM permuted path stages Xp in a library pool; handing the pool's
-    memory back between calls must not change the result."""
+@pytest.mark.parametrize("n,m", [(2, 4), (1, 8)])
+def test_permuted_pair_path_after_release_staging(n, m):
+    """The two-SM permuted path stages Xp (and for 1:8 a re-encoded 2:4
+    operand) in a library pool; handing the pool's memory back between calls
+    must not change the result."""
     R, K, T = 512, 1024, 512
     W = wl.normal_bf16((R, K), 0.02, seed=121)
     X = wl.normal_bf16((K, T), 1.0, seed=122)
     idx = wl.permutation(K, 123)
-    first = run_spmm(W, X, 2, 4, idx=idx)
+    first = run_spmm(W, X, n, m, idx=idx)
     nm.nm_release_staging()
-    second = run_spmm(W, X, 2, 4, idx=idx)
+    second = run_spmm(W, X, n, m, idx=idx)
     nm.nm_release_staging()
     assert torch.equal(first, second)
-    ref, mag = reference(W, X, 2, 4, idx)
+    ref, mag = reference(W, X, n, m, idx)
     assert_gemm_close(values_f64(second), ref, mag, "permuted after release")
 
 
@@ -506,6 +512,32 @@ def test_pair_tile_forms_integer_exact(R, K, T, out):
     rows = rows[rows < R]
     Wd = oracle.decompress(ov, om, K, 2, 4)
     ref = oracle.dense_gemm(np.ascontiguousarray(Wd[rows]), X)
+    if out == torch.float32:
+        assert np.array_equal(Y.contiguous().cpu().numpy().astype(np.float64)[rows], ref)
+    else:
+        assert np.array_equal(bits(Y)[rows], bf16_rne_of(ref))
+
+
+@pytest.mark.parametrize("R,K,T", [(2560, 8192, 2048),   # 256 x 256 tiles, row tiles fastest
+                                   (4096, 11008, 2048),  # 256 x 256 tiles, column tiles fastest
+                                   (1280, 512, 4096),    # 256 x 192 tiles
+                                   (2304, 768, 2568),    # 256 x 192 tiles, last column tile partial
+                                   (300, 1024, 200)])    # one partial 192-column tile, ragged rows
+@pytest.mark.parametrize("out", [torch.bfloat16, torch.float32])
+def test_pair_permuted_integer_exact(R, K, T, out):
+    """The permuted two-SM path (gather pass, then the pair kernel) on small
+    integers (every fp32 sum exact): sampled rows equal the oracle's permuted
+    product bit for bit."""
+    W = wl.integer_bf16((R, K), -8, 8, seed=R + 17)
+    X = wl.integer_bf16((K, T), -8, 8, seed=T + 19)
+    idx = wl.permutation(K, K + 23)
+    Y = run_spmm(W, X, 2, 4, idx=idx, out_dtype=out)
+    ov, om = oracle.compress(W, 2, 4)
+    rng = np.random.default_rng(5)
+    rows = np.unique(np.concatenate([rng.integers(0, R, 96), [0, 127, 128, 255, R - 1]]))
+    rows = rows[rows < R]
+    Wd = oracle.decompress(ov, om, K, 2, 4)
+    ref = oracle.dense_gemm(np.ascontiguousarray(Wd[rows]), X, idx)
     if out == torch.float32:
         assert np.array_equal(Y.contiguous().cpu().numpy().astype(np.float64)[rows], ref)
     else:
