@@ -1037,9 +1037,10 @@ def run_tf32(args, rank: int, world: int, dist):
                        "parallelism": f"replicas x{world}"},
             "roofline": {"bound": "tensor", "achieved": achieved, "peak": tf32_peak, "unit": "TFLOP/s",
                          "frac": achieved / tf32_peak, "traffic": None,
-                         "kernel": "nm_spmm_tf32 calls: decompress_1of2_f32_kernel + dense_pair_kernel (kind::tf32)",
+                         "kernel": "nm_spmm_tf32 calls: relayout_meta_tf32_kernel + spmm_pair_kernel (sparse kind::tf32)",
                          "peak_source": f"{peak_src} bf16 burst dense peak x 0.5 (the nominal tf32 / bf16 dense "
-                                        "ratio); useful (survivor) FLOPs, half of the dense ones",
+                                        "ratio); useful (survivor) FLOPs, which the sparse MMA executes at twice "
+                                        "the dense rate",
                          "timing": "CUDA events around back-to-back repetitions of the step's GEMM calls"},
             "gpu_launches": launches, "clocks": sampler.summary() if sampler else None, "cpu_baseline": None}
     if rank == 0:

@@ -120,41 +120,51 @@ __global__ void __launch_bounds__(256) decompress_2of4_i8_kernel(const int8_t* _
 // TMEM columns: row r's 32 bytes (64 groups, two per byte, low nibble first)
 // as two 16-byte halves, half c of rows 8j .. 8j + 7 at 256 j + 128 c.
 // Groups or rows outside the tiled words (padding) get the nibble 0x4.
-// One thread per output 32-bit word (row r, word w: groups 8w .. 8w + 7).
+// One thread per output 16-byte half (row r, half c: words 4c .. 4c + 3, groups
+// 32c .. 32c + 31 of the chunk's 64): they are the 16-bit row halves of four
+// consecutive tiled words (lo) and of the four 32 words later (hi), so a thread
+// makes two 16-byte loads (four 4-byte ones each when meta is not 16-byte
+// aligned, vec == false) and one 16-byte store.
 __global__ void __launch_bounds__(256) relayout_meta_i8_kernel(const uint32_t* __restrict__ meta, uint32_t rblocks16,
                                                               uint32_t cblocks128, uint32_t kblocks256,
-                                                              uint32_t* __restrict__ out, uint32_t total) {
+                                                              uint32_t* __restrict__ out, uint32_t total, bool vec) {
   pdl_gate();
   for (uint32_t i = blockIdx.x * blockDim.x + threadIdx.x; i < total; i += gridDim.x * blockDim.x) {
-    const uint32_t chunk = i >> 10, within = i & 1023u;  // 1024 words per chunk
-    const uint32_t r = within >> 3, w = within & 7u;     // row of the 128, word of the row's 8
+    const uint32_t chunk = i >> 8, within = i & 255u;  // 256 halves per chunk
+    const uint32_t r = within >> 1, c = within & 1u;   // row of the 128, half of the row's two
     const uint32_t rb128 = chunk / kblocks256, kb = chunk - rb128 * kblocks256;
     const uint32_t row = rb128 * 128 + r;
-    const uint32_t g0 = kb * 64 + 8 * w;                 // first group of the word (4 columns each)
-    uint32_t word = 0x44444444u;
-    const uint32_t rb = row >> 4, cb = g0 >> 5;
+    const uint32_t rb = row >> 4, cb = 2 * kb + c;     // tiled block: 16 rows x 128 columns (32 groups)
+    uint4 v = make_uint4(0x44444444u, 0x44444444u, 0x44444444u, 0x44444444u);
     if (rb < rblocks16 && cb < cblocks128) {
-      const uint32_t q = (g0 & 31u) >> 3;                // the tiled word's 32-column quarter
-      const uint32_t base = (rb * cblocks128 + cb) * 64 + 4 * (row & 7u) + q;
+      const uint32_t* src = meta + (rb * cblocks128 + cb) * 64 + 4 * (row & 7u);
+      uint4 lo, hi;  // quarters 0..3 of rows (row & 7) and +8: groups 8q .. 8q + 3; lane + 8: groups 8q + 4 .. 8q + 7
+      if (vec) {
+        lo = __ldg(reinterpret_cast<const uint4*>(src));
+        hi = __ldg(reinterpret_cast<const uint4*>(src + 32));
+      } else {
+        lo = make_uint4(__ldg(src), __ldg(src + 1), __ldg(src + 2), __ldg(src + 3));
+        hi = make_uint4(__ldg(src + 32), __ldg(src + 33), __ldg(src + 34), __ldg(src + 35));
+      }
       const uint32_t sh = 16 * ((row >> 3) & 1u);
-      const uint32_t lo = (__ldg(meta + base) >> sh) & 0xFFFFu;       // groups g0 .. g0 + 3 (lane h = 0)
-      const uint32_t hi = (__ldg(meta + base + 32) >> sh) & 0xFFFFu;  // groups g0 + 4 .. g0 + 7 (lane + 8)
-      word = lo | (hi << 16);
+      auto join = [&](uint32_t l, uint32_t h) { return ((l >> sh) & 0xFFFFu) | (((h >> sh) & 0xFFFFu) << 16); };
+      v = make_uint4(join(lo.x, hi.x), join(lo.y, hi.y), join(lo.z, hi.z), join(lo.w, hi.w));
     }
-    // word w of row r: half c = w / 4 at byte 128 c + 16 (r % 8) + 4 (w % 4) of the 8-row group r / 8
-    out[(int64_t)chunk * 1024 + (r >> 3) * 64 + (w >> 2) * 32 + (r & 7u) * 4 + (w & 3u)] = word;
+    // words 4c .. 4c + 3 of row r at byte 128 c + 16 (r % 8) of the 8-row group r / 8
+    *reinterpret_cast<uint4*>(out + (int64_t)chunk * 1024 + (r >> 3) * 64 + c * 32 + (r & 7u) * 4) = v;
   }
 }
 
 cudaError_t launch_relayout_meta_i8(const uint32_t* meta, int64_t R, int64_t K, uint32_t* out, int64_t rblocks128,
                                     cudaStream_t s) {
   const int64_t kblocks256 = (K + 255) / 256;
-  const int64_t total = rblocks128 * kblocks256 * 1024;
+  const int64_t total = rblocks128 * kblocks256 * 256;
   const int64_t want = (total + 255) / 256;
   const int64_t cap = (int64_t)sm_count_current() * 8;
   const int grid = (int)(want < cap ? (want > 0 ? want : 1) : cap);
   cudaError_t e = launch_pdl(relayout_meta_i8_kernel, dim3(grid), dim3(256), 0, s, meta, (uint32_t)meta_row_blocks(R),
-                             (uint32_t)meta_col_blocks(K), (uint32_t)kblocks256, out, (uint32_t)total);
+                             (uint32_t)meta_col_blocks(K), (uint32_t)kblocks256, out, (uint32_t)total,
+                             (reinterpret_cast<uintptr_t>(meta) & 15u) == 0);
   count_launch();
   return e != cudaSuccess ? e : cudaGetLastError();
 }

@@ -57,11 +57,13 @@ def test_decompress_i8_roundtrip(R, K):
 
 
 # T >= 192 with K % 32 == 0 runs on the sparse tensor cores (kind::i8, metadata re-laid out per row):
-# 256 x 192 tiles with two accumulators up to 24 stages of 256, 256 x 256 tiles beyond; other shapes on
+# 256 x 192 tiles with two accumulators up to 32 stages of 256, 256 x 256 tiles beyond; other shapes on
 # the decompressed dense operand.
 @pytest.mark.parametrize("R,K,T", [(300, 512, 264), (256, 1024, 256), (130, 384, 100), (64, 128, 16),
                                    (520, 256, 40), (600, 2048, 520), (260, 800, 320), (200, 1040, 256),
-                                   (260, 8192, 264)])  # 32 stages of 256: the 256 x 256 tile form
+                                   (260, 8192, 264),    # 32 stages: the last K of the 256 x 192 form
+                                   (520, 2048, 2000),   # 11 column tiles of 192, the last one 80 wide
+                                   (260, 8448, 264)])   # 33 stages: the 256 x 256 tile form
 def test_spmm_i8_exact(R, K, T):
     W = wl.integer_i8((R, K), -128, 127, seed=R + 7 * K)
     X = wl.integer_i8((K, T), -128, 127, seed=T + 3)
@@ -72,6 +74,28 @@ def test_spmm_i8_exact(R, K, T):
     ov, om = oracle.compress_i8(W)
     ref = oracle.spmm_i8(ov, om, K, X)
     assert np.array_equal(Y.cpu().numpy().astype(np.int64), ref)
+
+
+def test_spmm_i8_meta_only_4_byte_aligned():
+    """Metadata 4 bytes past a 16-byte boundary (the call asks for 4): the
+    re-layout reads it word by word; the product is unchanged."""
+    R, K, T = 300, 1024, 264
+    W = wl.integer_i8((R, K), -128, 127, seed=31)
+    X = wl.integer_i8((K, T), -128, 127, seed=32)
+    vals, meta = nm.prune_compress_i8(dev_i8(W))
+    Xd = dev_i8(X, ld=(T + 15) // 16 * 16)
+    Y = nm.spmm_i8(vals, meta, K, Xd)
+    buf = torch.zeros((meta.numel() + 4,), dtype=torch.int32, device=DEV)
+    off = next(o for o in range(4) if (buf.data_ptr() + 4 * o) % 16 == 4)
+    meta4 = buf[off:off + meta.numel()]
+    meta4.copy_(meta)
+    assert meta4.data_ptr() % 16 == 4
+    Y4 = nm.spmm_i8(vals, meta4, K, Xd)
+    torch.cuda.synchronize()
+    nm.nm_device_status()
+    assert torch.equal(Y, Y4)
+    ov, om = oracle.compress_i8(W)
+    assert np.array_equal(Y4.cpu().numpy().astype(np.int64), oracle.spmm_i8(ov, om, K, X))
 
 
 def test_spmm_i8_llama_layer_sampled():
