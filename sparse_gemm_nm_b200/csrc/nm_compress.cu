@@ -300,7 +300,8 @@ __global__ void __launch_bounds__(256) decompress_2of4_tiled_kernel(const uint16
                                                                     const uint32_t* __restrict__ meta, uint32_t R,
                                                                     uint32_t K, uint16_t* __restrict__ W,
                                                                     int64_t ldw, uint32_t cblocks, uint32_t total,
-                                                                    bool vec, const uint8_t* __restrict__ tile_map) {
+                                                                    bool vec, const uint8_t* __restrict__ tile_map,
+                                                                    uint32_t rtiles) {
   pdl_gate();
   for (uint32_t w = blockIdx.x * blockDim.x + threadIdx.x; w < total; w += gridDim.x * blockDim.x) {
     const uint32_t blk = w >> 6, wi = w & 63u;
@@ -309,8 +310,17 @@ __global__ void __launch_bounds__(256) decompress_2of4_tiled_kernel(const uint16
     const uint32_t r_lo = rb * 16 + (l & 7u);
     const uint32_t k0 = cb * 128 + q * 32 + (l >> 3) * 16;
     if (k0 >= K) continue;
-    // with a tile map (128 x 128 tiles, one column block each): 2:4 tiles only
-    if (tile_map && __ldg(tile_map + (int64_t)(r_lo >> 7) * cblocks + cb) == 0) continue;
+    // With a tile map (128 x 128 tiles, one column block each): the 2:4 tiles
+    // that the SM-pair hybrid kernel reads as dense tiles, i.e. those whose
+    // partner row tile (the other 128 rows of the pair's 256) exists and is
+    // dense in the same column block.  Where both are 2:4 the stage runs the
+    // sparse MMA on the compressed form; a lone last row tile pairs with itself.
+    if (tile_map) {
+      const uint32_t t = r_lo >> 7, partner = t ^ 1u;
+      if (__ldg(tile_map + (int64_t)t * cblocks + cb) == 0 || partner >= rtiles ||
+          __ldg(tile_map + (int64_t)partner * cblocks + cb) != 0)
+        continue;
+    }
     const uint32_t word = __ldg(meta + w);
     if (r_lo < R)
       decompress_half16(V + (int64_t)r_lo * (K >> 1), W + (int64_t)r_lo * ldw, word & 0xFFFFu, k0, K, vec);
@@ -502,7 +512,7 @@ cudaError_t launch_decompress(const uint16_t* values, const uint32_t* meta, int6
     const bool vec = K % 16 == 0 && ldw % 8 == 0 && aligned16(W_out) && aligned16(values);
     launch_pdl(decompress_2of4_tiled_kernel, grid_for(total, threads), threads, 0, s,
         values, meta, (uint32_t)R, (uint32_t)K, W_out, ldw, (uint32_t)meta_col_blocks(K), (uint32_t)total, vec,
-        nullptr);
+        nullptr, 0u);
   } else {
     const int64_t work = R * (K / m);
     const int grid = grid_for(work, threads);
@@ -524,7 +534,7 @@ cudaError_t launch_decompress_tiles(const uint16_t* values, const uint32_t* meta
   const bool vec = K % 16 == 0 && ldw % 8 == 0 && aligned16(W_out) && aligned16(values);
   launch_pdl(decompress_2of4_tiled_kernel, grid_for(total, threads), threads, 0, s,
       values, meta, (uint32_t)R, (uint32_t)K, W_out, ldw, (uint32_t)meta_col_blocks(K), (uint32_t)total, vec,
-      tile_map);
+      tile_map, (uint32_t)((R + 127) / 128));
   count_launch();
   return cudaGetLastError();
 }

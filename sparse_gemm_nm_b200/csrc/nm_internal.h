@@ -111,8 +111,10 @@ cudaError_t launch_compress(const uint16_t* W, int64_t R, int64_t K, int64_t ldw
                             uint32_t* meta, cudaStream_t s);
 cudaError_t launch_decompress(const uint16_t* values, const uint32_t* meta, int64_t R, int64_t K, int n, int m,
                               uint16_t* W_out, int64_t ldw, cudaStream_t s);
-// 2:4 decompress of the 128 x 128 tiles whose tile_map entry is non-zero
-// (tile map ceil(R/128) x ceil(K/128)); other tiles of W_out are not written.
+// 2:4 decompress of the 128 x 128 tiles that the SM-pair hybrid kernel reads as
+// dense tiles: tile_map entry non-zero (tile map ceil(R/128) x ceil(K/128)) and
+// the partner row tile (row tile index ^ 1) present and zero in the same column;
+// other tiles of W_out are not written.
 cudaError_t launch_decompress_tiles(const uint16_t* values, const uint32_t* meta, int64_t R, int64_t K,
                                     const uint8_t* tile_map, uint16_t* W_out, int64_t ldw, cudaStream_t s);
 // Xp[k] = X[idx[k]] (zero rows for idx outside [0, K)); with skip_if set, the
