@@ -544,6 +544,26 @@ def test_pair_permuted_integer_exact(R, K, T, out):
         assert np.array_equal(bits(Y)[rows], bf16_rne_of(ref))
 
 
+@pytest.mark.parametrize("R,K,T", [(1, 128, 192),      # one row, one stage, one 192-column tile
+                                   (257, 128, 192),    # a 1-row second row tile
+                                   (255, 1024, 200),   # 8 stages (the last of the 256 x 192 form), 8-column tail
+                                   (255, 1152, 200),   # 9 stages: the 256 x 256 form, one partial column tile
+                                   (513, 1152, 392),   # three row tiles, ragged rows and columns
+                                   (256, 1024, 184)])  # T < 192: the one-SM kernel
+@pytest.mark.parametrize("out", [torch.bfloat16, torch.float32])
+def test_pair_admission_boundaries_integer_exact(R, K, T, out):
+    """Shapes at the edges of the SM-pair kernel's rules (T >= 192, the eight-stage limit of the
+    two-accumulator form, ragged R): small integers, so the whole output equals the oracle bit for bit."""
+    W = wl.integer_bf16((R, K), -8, 8, seed=R + K)
+    X = wl.integer_bf16((K, T), -8, 8, seed=T + 1)
+    Y = run_spmm(W, X, 2, 4, out_dtype=out)
+    ref, _ = reference(W, X, 2, 4)
+    if out == torch.float32:
+        assert np.array_equal(Y.contiguous().cpu().numpy().astype(np.float64), ref)
+    else:
+        assert np.array_equal(bits(Y), bf16_rne_of(ref))
+
+
 def test_pair_double_buffered_permuted_tolerance():
     """ViT-depth tiles (6 stages, two accumulators) with an index map, sampled at full width."""
     R, K, T = 3072, 768, 6144
