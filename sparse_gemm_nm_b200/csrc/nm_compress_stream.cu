@@ -39,6 +39,12 @@ constexpr uint64_t kWaitNs = 2000000000ull;
 // and leave the last SMs to free up without work.
 constexpr size_t kSmem = 100 * 1024;
 static_assert(kSlots * kBlockBytes + 2 * kSlots * 8 + 64 + 1024 <= kSmem, "ring does not fit");
+// Block j goes to slot j % kSlots and to consumer warp j % kConsumers, and the
+// waits test barrier phases by parity.  With kSlots a multiple of kConsumers
+// every slot is always read by the same warp, which takes its uses in order, so
+// a warp never waits on use u of a slot before use u - 1 has completed (the
+// parity of use u - 2 would otherwise pass for use u).
+static_assert(kSlots % kConsumers == 0, "each ring slot must belong to one consumer warp");
 }  // namespace cstream
 
 template <bool GATHER>
