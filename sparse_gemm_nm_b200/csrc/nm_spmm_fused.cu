@@ -36,6 +36,7 @@ namespace nmk {
 namespace fused {
 constexpr int kSelectors = 8;  // warps per stage, one per 16-row block
 constexpr int kGroups = 2;     // selector groups, taking alternate stages
+static_assert(kGroups == 2, "full barriers are laid out per (slot, group) for two groups");
 constexpr int kSelWarps = kSelectors * kGroups;
 constexpr int kThreads = 32 * (2 + kSelWarps + 4);  // 0 copies, 1 MMA, 2..17 select, 18..21 epilogue
 constexpr int kAcc = 4;
@@ -70,8 +71,11 @@ __global__ void __launch_bounds__(fused::kThreads, 1) prune_spmm_skinny_kernel(c
   uint8_t* a_base = w_base + S * kW;     // S x 16 KB: compressed values, SW128 K-major
   uint8_t* b_base = a_base + S * kA;     // S x kB: X rows
   uint8_t* e_base = b_base + S * kB;     // S x 2 KB: metadata blocks
+  // full[2 s + g]: the copies of a stage in slot s taken by selector group g.  With S odd
+  // the uses of one slot alternate between the groups; a barrier per (slot, group) keeps
+  // every barrier's phases consumed in order by one group, as its parity waits need.
   uint64_t* full = reinterpret_cast<uint64_t*>(e_base + S * kE);
-  uint64_t* built = full + S;
+  uint64_t* built = full + 2 * S;
   uint64_t* empty = built + S;
   uint64_t* acc_full = empty + S;
   uint64_t* acc_empty = acc_full + kAcc;
@@ -85,7 +89,8 @@ __global__ void __launch_bounds__(fused::kThreads, 1) prune_spmm_skinny_kernel(c
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
-      mbar_init(&full[s], 1);
+      mbar_init(&full[2 * s], 1);
+      mbar_init(&full[2 * s + 1], 1);
       mbar_init(&built[s], kSelectors);
       mbar_init(&empty[s], 1);
     }
@@ -123,17 +128,18 @@ __global__ void __launch_bounds__(fused::kThreads, 1) prune_spmm_skinny_kernel(c
     // -------------------------------------------------------------- copies
     if (lane == 0) {
       int s = 0;
-      uint32_t ph = 0;
+      uint32_t ph = 0, j = 0;  // j: the CTA's stage counter (stage j goes to group j % kGroups)
       for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
         int tm;
         int64_t kt0, kt1;
         unit_range(u, tm, kt0, kt1);
-        for (int64_t kt = kt0; kt < kt1; ++kt) {
+        for (int64_t kt = kt0; kt < kt1; ++kt, ++j) {
           ok = mbar_wait(&empty[s], ph ^ 1u, abort_flag, p.status, kWaitNs);
           if (!ok) break;
-          mbar_arrive_expect_tx(&full[s], kW + kB);
-          tma_load_2d(w_base + s * kW, &p.tm_w, &full[s], (int32_t)(kt * 128), tm * 128);
-          tma_load_2d(b_base + s * kB, &p.tm_x, &full[s], 0, (int32_t)(kt * 128));
+          uint64_t* fb = &full[2 * s + (int)(j % kGroups)];
+          mbar_arrive_expect_tx(fb, kW + kB);
+          tma_load_2d(w_base + s * kW, &p.tm_w, fb, (int32_t)(kt * 128), tm * 128);
+          tma_load_2d(b_base + s * kB, &p.tm_x, fb, 0, (int32_t)(kt * 128));
           if (++s == S) { s = 0; ph ^= 1u; }
         }
       }
@@ -198,8 +204,10 @@ __global__ void __launch_bounds__(fused::kThreads, 1) prune_spmm_skinny_kernel(c
       unit_range(u, tm, kt0, kt1);
       for (int64_t kt = kt0; kt < kt1; ++kt, ++j) {
         if ((int)(j % kGroups) != group) continue;
-        const uint32_t s = j % S, ph = (j / S) & 1u;
-        ok = mbar_wait(&full[s], ph, abort_flag, p.status, kWaitNs);
+        // the group's uses of barrier (slot s, group) are its stages j = r mod lcm(S, kGroups)
+        constexpr uint32_t kCycle = S % kGroups == 0 ? S : S * kGroups;
+        const uint32_t s = j % S, ph = (j / kCycle) & 1u;
+        ok = mbar_wait(&full[2 * s + group], ph, abort_flag, p.status, kWaitNs);
         if (!ok) break;
         const uint8_t* wt = w_base + s * kW + blk16 * 16 * 256;
         uint4 in[8];
@@ -314,7 +322,7 @@ template <int BN>
 static cudaError_t launch_fused_bn(SpmmParams& p, cudaStream_t stream) {
   using namespace fused;
   constexpr int S = stages(BN);
-  const size_t bytes = (size_t)S * stage_bytes(BN) + (3 * S + 2 * kAcc + 1) * 8 + 16 + 1024;
+  const size_t bytes = (size_t)S * stage_bytes(BN) + (4 * S + 2 * kAcc + 1) * 8 + 16 + 1024;
   static bool configured[64] = {};
   int dev = 0;
   cudaGetDevice(&dev);
