@@ -59,8 +59,9 @@ def test_fused_matches_oracle(R, K, T, permuted):
 
 
 @pytest.mark.parametrize("out", [torch.bfloat16, torch.float32])
-def test_fused_integer_exact(out):
-    R, K, T = 384, 4096, 16  # several K ranges; every partial sum is an exact integer
+@pytest.mark.parametrize("T", [16, 32, 64])  # four stages (bn 16); three (bn 32, 64): a slot's uses alternate groups
+def test_fused_integer_exact(out, T):
+    R, K = 384, 4096  # several K ranges; every partial sum is an exact integer
     W = wl.integer_bf16((R, K), -8, 8, seed=201)
     X = wl.integer_bf16((K, T), -8, 8, seed=202)
     ref, _, ov, om = reference(W, X, 2, 4)
