@@ -12,6 +12,7 @@
 // are tiled in the sparse tensor core's order (one nibble per group, see
 // compress_2of4_tiled_kernel); other patterns are packed row-wise, b-bit
 // positions, survivor j of a row in word j/S at bit b*(j%S).
+#include <atomic>
 #include <cstdint>
 #include <cuda_runtime.h>
 
@@ -542,7 +543,7 @@ cudaError_t launch_decompress_tiles(const uint16_t* values, const uint32_t* meta
 cudaError_t launch_gather_rows(const uint16_t* X, int64_t ldx, const int32_t* idx, int64_t K, int64_t T,
                                uint16_t* Xp, int64_t ldp, cudaStream_t s, const uint32_t* skip_if) {
   const int threads = 256;
-  static bool configured[64] = {};
+  static std::atomic<bool> configured[64];  // zero-initialised: false
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev >= 0 && dev < 64 && !configured[dev]) {

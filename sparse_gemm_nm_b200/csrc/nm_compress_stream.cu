@@ -11,6 +11,7 @@
 // zero-filled, which selects positions (0, 1): exactly the padding nibble 0x4;
 // values are stored only inside R x K.  Optionally the same grid also gathers
 // the permuted rows of a GEMM input (see kGatherWarps).
+#include <atomic>
 #include <cstdint>
 #include <cuda.h>
 #include <cuda_runtime.h>
@@ -137,7 +138,7 @@ __global__ void __launch_bounds__(GATHER ? cstream::kThreadsGather : cstream::kT
 cudaError_t launch_compress_stream(const CUtensorMap& tm_w, int64_t R, int64_t K, uint16_t* values, uint32_t* meta,
                                    uint32_t* status, cudaStream_t s, const GatherJob* gather) {
   using namespace cstream;
-  static bool configured[2][64] = {};
+  static std::atomic<bool> configured[2][64];  // zero-initialised: false
   int dev = 0;
   cudaGetDevice(&dev);
   const int gi = gather ? 1 : 0;

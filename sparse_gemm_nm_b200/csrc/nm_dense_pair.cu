@@ -26,6 +26,7 @@
 // with K = 32 and K = 8 per MMA.  The plain store epilogue sends whole
 // 128-byte row chunks through a swizzled staging tile and TMA stores; with a
 // row map (dX under an index map) rows are stored one per lane.
+#include <atomic>
 #include <cstdint>
 #include <cuda.h>
 #include <cuda_runtime.h>
@@ -412,7 +413,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dpair::kThreads, 1)
 
 template <bool A_MN, bool B_MN, int EPI, bool I8 = false, bool TF32 = false>
 static cudaError_t launch_dp(const DenseParams& p, cudaStream_t stream) {
-  static bool configured[64] = {};
+  static std::atomic<bool> configured[64];  // zero-initialised: false
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev >= 0 && dev < 64 && !configured[dev]) {

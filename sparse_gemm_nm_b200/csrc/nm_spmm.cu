@@ -25,6 +25,7 @@
 //   warps 6-9   epilogue: TMEM -> registers -> bf16/fp32 -> global.
 // Stages of the shared-memory ring are handed over with mbarriers; every wait
 // is bounded in time and reports through a device status word.
+#include <atomic>
 #include <cstdint>
 #include <cuda.h>
 #include <cuda_runtime.h>
@@ -569,7 +570,7 @@ template <int BN>
 static cudaError_t launch_bn(const SpmmParams& p, int grid, cudaStream_t stream) {
   const SmemLayout L = smem_layout(p.stages, p.a_slot_bytes, 64u * BN * 2u);
   const size_t bytes = L.total + 1024;
-  static bool configured[64] = {};
+  static std::atomic<bool> configured[64];  // zero-initialised: false
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 64 && !configured[dev]) {

@@ -22,6 +22,7 @@
 // N = bn, K = 32).  Two groups of eight selector warps take alternate stages:
 // the selection is integer work on the ALU pipe, which one group cannot run
 // at the rate the tiles arrive.
+#include <atomic>
 #include <cstdint>
 #include <cuda.h>
 #include <cuda_runtime.h>
@@ -323,7 +324,7 @@ static cudaError_t launch_fused_bn(SpmmParams& p, cudaStream_t stream) {
   using namespace fused;
   constexpr int S = stages(BN);
   const size_t bytes = (size_t)S * stage_bytes(BN) + (4 * S + 2 * kAcc + 1) * 8 + 16 + 1024;
-  static bool configured[64] = {};
+  static std::atomic<bool> configured[64];  // zero-initialised: false
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev >= 0 && dev < 64 && !configured[dev]) {

@@ -55,6 +55,7 @@
 // 32-column strips in the 32-byte-unit swizzle the MMA reads for MN-major
 // 32-bit operands), 4 KB of metadata (relayout_meta_tf32_kernel); four K = 16
 // MMAs per stage, each with its own even TMEM metadata column.
+#include <atomic>
 #include <cstdint>
 #include <cuda.h>
 #include <cuda_runtime.h>
@@ -452,7 +453,7 @@ template <bool HYB, bool DB, bool I8 = false, bool TF32 = false>
 static cudaError_t launch_pair(SpmmParams& p, cudaStream_t stream) {
   constexpr pair::Layout L = pair::Cfg<HYB, DB, I8, TF32>::layout();
   const size_t bytes = L.total + 1024;
-  static bool configured[64] = {};
+  static std::atomic<bool> configured[64];  // zero-initialised: false
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 64 && !configured[dev]) {

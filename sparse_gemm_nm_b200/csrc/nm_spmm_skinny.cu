@@ -15,6 +15,7 @@
 // one unit overlaps the next.  With one K range the epilogue writes Y; with
 // several it writes fp32 partials, which skinny_reduce_kernel (launched as a
 // programmatic dependent of this kernel) sums in range order into Y.
+#include <atomic>
 #include <cstdint>
 #include <cuda.h>
 #include <cuda_runtime.h>
@@ -292,7 +293,7 @@ static cudaError_t launch_bn(SpmmParams& p, cudaStream_t stream) {
   using namespace skinny;
   constexpr int S = stages(BN, KD);
   const size_t bytes = (size_t)S * stage_bytes(BN, KD) + (2 * S + 2 * kAcc + 1) * 8 + 16 + 1024;  // + slots, align
-  static bool configured[64] = {};
+  static std::atomic<bool> configured[64];  // zero-initialised: false
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 64 && !configured[dev]) {
