@@ -591,15 +591,21 @@ int spmm_max_stages(int bn, uint32_t a_slot) {
   return st;
 }
 
+// Device address of the status word on the current device (looked up once per device; devices past the
+// cache are looked up on every call).
 uint32_t* status_word_ptr() {
-  static uint32_t* status_ptr[64] = {};
+  static std::atomic<uint32_t*> status_ptr[64];  // zero-initialised: not looked up yet
   int dev = 0;
-  cudaGetDevice(&dev);
-  if (dev < 0 || dev >= 64) dev = 0;
-  if (!status_ptr[dev]) {
-    if (cudaGetSymbolAddress(reinterpret_cast<void**>(&status_ptr[dev]), g_status) != cudaSuccess) return nullptr;
+  if (cudaGetDevice(&dev) != cudaSuccess) return nullptr;
+  const bool cached = dev >= 0 && dev < 64;
+  if (cached) {
+    uint32_t* p = status_ptr[dev].load(std::memory_order_relaxed);
+    if (p) return p;
   }
-  return status_ptr[dev];
+  void* addr = nullptr;
+  if (cudaGetSymbolAddress(&addr, g_status) != cudaSuccess) return nullptr;
+  if (cached) status_ptr[dev].store(static_cast<uint32_t*>(addr), std::memory_order_relaxed);
+  return static_cast<uint32_t*>(addr);
 }
 
 cudaError_t launch_spmm(SpmmParams& p, int bn, cudaStream_t stream) {
