@@ -250,6 +250,18 @@ def layer_mode(L, step_mode: str, algo: str, permuted: bool) -> str:
     return "split"
 
 
+def reencoded_bound_s(bufs, tc_peak: float, hbm_peak: float) -> float:
+    """Lower bound (seconds) on the GEMM launches of a 1:8 step run as re-encoded 2:4.
+
+    Each group of eight weights becomes two 2:4 groups, so the sparse tensor cores multiply four stored
+    values (one survivor, three zeros) where the pattern keeps one: 4x the useful products.  Stored
+    2:4 values are multiplied at the dense product rate (the sparse MMA's 2x is over the logical K it
+    covers), so the tensor term is the executed products over the dense peak.  The other term is the
+    algorithmic bytes at the HBM rate."""
+    executed = sum(4.0 * b["flops"] for b in bufs)
+    return max(executed / (tc_peak * 1e12), sum(b["gemm_bytes"] for b in bufs) / (hbm_peak * 1e9))
+
+
 def step_config(workload: str, layers, step_mode: str, algo: str, plain: bool, world: int) -> dict:
     """The `config` object of a bench line (the same for both arms)."""
     permuted = [L.permuted and not plain for L in layers]
@@ -565,13 +577,13 @@ def measure_config(name, args, dev, stream, nm, peaks, world, loaded_ms=0.0):
                                      "kernel": "nm_spmm: spmm_skinny_kernel + split-K reduction",
                                      "call_us": 1e3 * two}
     if name == "vit":
-        # executed MACs of the re-encoded 2:4 design: every 1:8 survivor rides in a 2:4 pair, 4x the useful
-        # products at the sparse rate (2x the dense rate)
-        ex = sum(4.0 * b["flops"] for b in r.bufs)
-        t_exec = max(ex / 2.0 / (tc_peak * 1e12), sum(b["gemm_bytes"] for b in r.bufs) / (hbm_peak * 1e9))
+        t_exec = reencoded_bound_s(r.bufs, tc_peak, hbm_peak)
         out["roofline_reencoded"] = {"t_bound_us": 1e6 * t_exec, "frac": t_exec / (gemm_step_ms * 1e-3),
-                                     "note": "max(executed 2:4 MACs at the sparse rate, algorithmic bytes at "
-                                             "the HBM rate) over the step's GEMM launches"}
+                                     "bound": "tensor" if t_exec * hbm_peak * 1e9 > sum(
+                                         b["gemm_bytes"] for b in r.bufs) * (1 + 1e-9) else "hbm",
+                                     "note": "max(the re-encoded 2:4 form's executed products (4x the useful "
+                                             "ones) at the dense product rate, algorithmic bytes at the HBM "
+                                             "rate) over the step's GEMM launches"}
     del r
     torch.cuda.synchronize()
     torch.cuda.empty_cache()

@@ -107,3 +107,16 @@ def test_peaks_file_or_fallback(tmp_path, monkeypatch):
                                                               "bf16_tflops_sustained": 3.0}))
     peaks, src = bench.load_peaks()
     assert src == "measured" and peaks["bf16_tflops_sustained"] == 3.0
+
+
+def test_reencoded_bound_counts_four_products_per_survivor():
+    # ViT 3072x768, T = 50432, at 1:8: 29.7 useful GFLOP; the re-encoded form multiplies 4x as many products,
+    # half of the dense GEMM's, at the dense product rate: 73 us per layer at 1630 TFLOP/s, above the HBM term
+    V = layers("vit")[0]
+    useful = 2.0 * 3072 * (768 // 8) * 50432
+    bufs = [{"flops": useful, "gemm_bytes": 388030464.0}]
+    t = bench.reencoded_bound_s(bufs, 1630.2, 6534.1)
+    assert t == pytest.approx(2.0 * 3072 * 768 * 50432 / 2 / 1630.2e12)
+    assert t == pytest.approx(4 * V.useful_flops / 1630.2e12) and 72e-6 < t < 74e-6
+    # bytes dominate when the products are few
+    assert bench.reencoded_bound_s([{"flops": 1.0, "gemm_bytes": 6534.1e9}], 1630.2, 6534.1) == pytest.approx(1.0)
