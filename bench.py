@@ -470,6 +470,36 @@ class Runner:
         torch.cuda.synchronize()
         return e0.elapsed_time(e1) / reps
 
+    def timed_graph(self, fn, calls, replays):
+        """Milliseconds per call of fn() from replays of a CUDA graph that holds `calls` of them (launches,
+        staging allocations and all), timed with CUDA events around the replays: no host work in the timed
+        region.  None when the calls do not capture."""
+        torch = self.torch
+        fn()
+        torch.cuda.synchronize()
+        side = torch.cuda.Stream(device=self.dev)
+        sp0, g = self.sp, torch.cuda.CUDAGraph()
+        try:
+            self.sp = side.cuda_stream
+            with torch.cuda.graph(g, stream=side):
+                for _ in range(calls):
+                    fn()
+        except Exception:  # noqa: BLE001 - a call that does not capture: the caller times it eagerly
+            return None
+        finally:
+            self.sp = sp0
+        with torch.cuda.stream(self.stream):
+            g.replay()
+            torch.cuda.synchronize()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(self.stream)
+            for _ in range(replays):
+                g.replay()
+            e1.record(self.stream)
+            torch.cuda.synchronize()
+        del g
+        return e0.elapsed_time(e1) / (replays * calls)
+
     def kernels(self, comp_ms, gemm_ms, tc_peak, hbm_peak):
         out = {}
         for i, b in enumerate(self.bufs):
@@ -733,19 +763,27 @@ def run_ours(args, rank: int, world: int, dist):
 
     if not args.quick and any(b["idx"] is not None for b in bufs) and all(b["tmap"] is None for b in bufs):
         # cost of the index-map read: per layer the GEMM call with the map (nm_spmm_permuted: gather pass +
-        # GEMM) and without it (nm_spmm), each in an event-bracketed loop on the compressed operand
+        # GEMM) and without it (nm_spmm) on the compressed operand, each timed from replays of a CUDA graph
+        # of 20 calls (an eager loop of a 30 us call can be bound by the host's call overhead instead)
         reps = max(10, min(200, args.steps))
         over = {}
+        how = set()
         for b in bufs:
             L = b["L"]
-            res = {name: r.timed(lambda: r.launch_gemm(b, permuted), reps, warm=3)
-                   for name, permuted in (("permuted", True), ("plain", False))}
+            res = {}
+            for name, permuted in (("permuted", True), ("plain", False)):
+                fn = (lambda b=b, permuted=permuted: r.launch_gemm(b, permuted))
+                t = r.timed_graph(fn, 20, max(1, reps // 20))
+                how.add("graph" if t is not None else "eager")
+                res[name] = t if t is not None else r.timed(fn, reps, warm=3)
             t_bound = max(b["flops"] / (tc_peak * 1e12), gemm_bytes(L, b["d"]) / (hbm_peak * 1e9))
             over[L.name] = {"plain_us": 1e3 * res["plain"], "permuted_us": 1e3 * res["permuted"],
                             "overhead": res["permuted"] / res["plain"] - 1.0,
                             "plain_tflops": b["flops"] / (res["plain"] * 1e-3) / 1e12,
                             "plain_frac": t_bound / (res["plain"] * 1e-3)}
         nm.nm_device_status(sp)
+        over["timing"] = ("CUDA events around replays of a CUDA graph of 20 calls per layer and form" if how == {"graph"}
+                          else "event-bracketed loops of calls (some calls did not capture into a CUDA graph)")
         line["permutation_overhead"] = over
 
     if not args.quick and all(b["tmap"] is None for b in bufs) and all(
