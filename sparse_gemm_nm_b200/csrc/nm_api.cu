@@ -223,10 +223,15 @@ static int pair_n_major(int64_t R, int64_t vcols, int64_t K, int64_t T) {
 
 // Store map of the SM-pair kernel's epilogue: bf16 Y in 64-column x 32-row boxes, 32-bit Y (fp32,
 // or int32 accumulator bits) in 32 x 32 boxes; both 128-byte rows with the 128-byte swizzle.
-static nm_status make_pair_store_map(CUtensorMap* tm, void* Y, int64_t R, int64_t T, int64_t ldy, bool out32) {
-  return out32 ? make_tmap(tm, Y, (uint64_t)T, (uint64_t)R, (uint64_t)ldy * 4, 32, 32, 128, "Y (32-bit)",
-                           CU_TENSOR_MAP_DATA_TYPE_FLOAT32)
-               : make_tmap(tm, Y, (uint64_t)T, (uint64_t)R, (uint64_t)ldy * 2, 64, 32, 128, "Y");
+// Store maps of the SM-pair epilogues: p.tm_y, and for bf16 Y also p.tm_y32
+// (the last 32 columns of the double-buffered form's 224-column tiles).
+static nm_status make_pair_store_maps(SpmmParams& p, void* Y, int64_t R, int64_t T, int64_t ldy, bool out32) {
+  if (out32)
+    return make_tmap(&p.tm_y, Y, (uint64_t)T, (uint64_t)R, (uint64_t)ldy * 4, 32, 32, 128, "Y (32-bit)",
+                     CU_TENSOR_MAP_DATA_TYPE_FLOAT32);
+  nm_status st = make_tmap(&p.tm_y, Y, (uint64_t)T, (uint64_t)R, (uint64_t)ldy * 2, 64, 32, 128, "Y");
+  if (st == NM_OK) st = make_tmap(&p.tm_y32, Y, (uint64_t)T, (uint64_t)R, (uint64_t)ldy * 2, 32, 32, 0, "Y (32 columns)");
+  return st;
 }
 
 static int pattern_id(int n, int m) {
@@ -416,7 +421,7 @@ static nm_status run_gemm(const GemmRequest& q, cudaStream_t stream) {
       st = make_tmap(&p.tm_w, q.W, (uint64_t)q.K, (uint64_t)q.R, (uint64_t)q.ldw * 2, 64, kPairBoxRows, 128, "W");
     if (st == NM_OK)
       st = make_tmap(&p.tm_wm, wm, (uint64_t)q.K, (uint64_t)q.R, (uint64_t)q.K * 2, 64, kPairBoxRows, 128, "W masked");
-    if (st == NM_OK) st = make_pair_store_map(&p.tm_y, q.Y, q.R, q.T, q.ldy, p.out_f32 != 0);
+    if (st == NM_OK) st = make_pair_store_maps(p, q.Y, q.R, q.T, q.ldy, p.out_f32 != 0);
     if (st == NM_OK) e = launch_spmm_pair_hybrid(p, stream);
     cudaFreeAsync(wm, stream);
     if (st != NM_OK) return st;
@@ -548,7 +553,7 @@ static nm_status run_gemm(const GemmRequest& q, cudaStream_t stream) {
       st = make_tmap(&p.tm_vals, vals, (uint64_t)p.vcols, (uint64_t)q.R, (uint64_t)p.vcols * 2, 64, kPairBoxRows,
                      128, "values");
     if (st == NM_OK && !dense_pair) st = make_meta_tmap(&p.tm_meta, meta, p.meta_rblocks, p.meta_cblocks);
-    if (st == NM_OK && !use_skinny) st = make_pair_store_map(&p.tm_y, q.Y, q.R, q.T, q.ldy, p.out_f32 != 0);
+    if (st == NM_OK && !use_skinny) st = make_pair_store_maps(p, q.Y, q.R, q.T, q.ldy, p.out_f32 != 0);
     if (!use_skinny && !dense_pair) p.n_major = pair_n_major(q.R, p.vcols, q.K, q.T);
     if (st == NM_OK)
       e = use_skinny   ? launch_spmm_skinny(p, stream)
@@ -684,7 +689,7 @@ nm_status build_pair_params(SpmmParams& p, const uint16_t* values, const uint32_
     st = make_tmap(&p.tm_vals, values, (uint64_t)p.vcols, (uint64_t)R, (uint64_t)p.vcols * 2, 64, kPairBoxRows, 128,
                    "values");
   if (st == NM_OK) st = make_meta_tmap(&p.tm_meta, meta, p.meta_rblocks, p.meta_cblocks);
-  if (st == NM_OK) st = make_pair_store_map(&p.tm_y, Y, R, T, ldy, out_f32);
+  if (st == NM_OK) st = make_pair_store_maps(p, Y, R, T, ldy, out_f32);
   p.n_major = pair_n_major(R, p.vcols, K, T);
   return st;
 }
@@ -1097,7 +1102,7 @@ static nm_status run_spmm_i8(const int8_t* values, const uint32_t* meta, int64_t
     if (e == cudaSuccess && st == NM_OK)
       st = make_tmap(&p.tm_meta, em, 256, (uint64_t)(rblocks128 * kblocks * 16), 256, 256, 16, 0,
                      "metadata (int8 order)", CU_TENSOR_MAP_DATA_TYPE_UINT8);
-    if (e == cudaSuccess && st == NM_OK) st = make_pair_store_map(&p.tm_y, Y, R, T, ldy, true);
+    if (e == cudaSuccess && st == NM_OK) st = make_pair_store_maps(p, Y, R, T, ldy, true);
     p.n_major = pair_n_major(R, K / 2, K, T);
     if (e == cudaSuccess && st == NM_OK) e = launch_spmm_pair_i8(p, stream);
     cudaFreeAsync(em, stream);
@@ -1242,7 +1247,7 @@ static nm_status run_spmm_tf32(const float* values, const uint32_t* meta, int64_
     if (e == cudaSuccess && st == NM_OK)
       st = make_tmap(&p.tm_meta, em, 256, (uint64_t)(rblocks128 * kblocks * 16), 256, 256, 16, 0,
                      "metadata (tf32 order)", CU_TENSOR_MAP_DATA_TYPE_UINT8);
-    if (e == cudaSuccess && st == NM_OK) st = make_pair_store_map(&p.tm_y, Y, R, T, ldy, p.out_f32 != 0);
+    if (e == cudaSuccess && st == NM_OK) st = make_pair_store_maps(p, Y, R, T, ldy, p.out_f32 != 0);
     p.n_major = pair_n_major(R, K / 2, K, T);
     if (e == cudaSuccess && st == NM_OK) e = launch_spmm_pair_tf32(p, stream);
     cudaFreeAsync(em, stream);

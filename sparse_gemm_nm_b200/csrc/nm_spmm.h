@@ -27,6 +27,7 @@ struct SpmmParams {
   CUtensorMap tm_x;     // X K x T, box {strip, 64} (one SM) or {64, kPairBoxRows} (SM pair)
   CUtensorMap tm_wm;    // W under the 2:4 mask (staged), box {64, 64}, 128B swizzle (SM-pair hybrid)
   CUtensorMap tm_y;     // Y R x T bf16, box {64, 32}, 128B swizzle (SM-pair epilogue stores)
+  CUtensorMap tm_y32;   // Y R x T bf16, box {32, 32}, no swizzle (last 32 columns of a 224-column SM-pair tile)
   CUtensorMap tm_meta;  // tiled 2:4 metadata {64 words, col blocks, row blocks}, box {64, 1, 8} (SM pair)
   const uint16_t* vals;
   const uint32_t* meta;

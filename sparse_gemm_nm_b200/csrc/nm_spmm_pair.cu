@@ -38,10 +38,12 @@
 // six-stage ViT tile a trace showed ~2.3 us of MMAs and ~1.6 us until the next
 // tile's first MMA.  Two accumulators let the next tile's MMAs run while the
 // epilogue drains, but two 256-column fp32 accumulators fill all 512 TMEM
-// columns and leave none for the sparse metadata.  So the DB form uses 256 x 192
-// tiles (each CTA supplies 96 columns of X: its first 64-column strip and half of
-// its second) and two 192-column accumulators (TMEM columns 0 and 256, metadata
-// from column 448).  It keeps four stages: a trace of the three-stage form on the
+// columns and leave none for the sparse metadata.  So the DB form uses 256 x 224
+// tiles (each CTA supplies 112 columns of X: its first 64-column strip and 48
+// columns of its second) and two 224-column accumulators (TMEM columns 0 and 256,
+// metadata from column 480).  A stage costs about the same at N = 192, 224 or 256
+// (each CTA loads both 64-column strips whole), so the widest N whose two
+// accumulators leave room for the metadata covers the most columns per stage.  It keeps four stages: a trace of the three-stage form on the
 // ViT shape showed the MMA thread waiting ~240 ns of each ~600 ns stage for data
 // (X rows 100 KB apart, a third of them from HBM).
 //
@@ -80,15 +82,15 @@ struct Layout {
 // HYB = false: 2:4 only, A slots of 16 KB (compressed values), four stages.
 // HYB = true (PATCH hybrid): A slots of 32 KB so that a stage can hold the
 // dense 128 x 128 tile instead, three stages.
-// DB = true (2:4, short tiles): 256 x 192 tiles, two accumulators, four stages.
+// DB = true (2:4, short tiles): 256 x 224 tiles, two accumulators, four stages.
 template <bool HYB, bool DB = false, bool I8 = false, bool TF32 = false>
 struct Cfg {
   static_assert(!((I8 || TF32) && (HYB || DB)) && !(I8 && TF32), "int8 / tf32 run the 256 x 256 sparse form only");
   static constexpr bool kWideE = I8 || TF32;  // 4 KB metadata chunks staged per row block and stage
   static constexpr int kStages = HYB ? 3 : 4;
-  static constexpr uint32_t kN = DB ? 192u : 256u;  // pair tile columns (per CTA: kN / 2 of X)
+  static constexpr uint32_t kN = DB ? 224u : 256u;  // pair tile columns (per CTA: kN / 2 of X)
   static constexpr int kAcc = DB ? 2 : 1;           // accumulators, 256 TMEM columns apart
-  static constexpr uint32_t kECol = DB ? 448u : 256u;
+  static constexpr uint32_t kECol = DB ? 480u : 256u;
   static constexpr uint32_t kE = kWideE ? 4096u : 2048u;  // metadata bytes per stage and CTA
   static constexpr uint32_t kECols = kWideE ? 8u : 4u;    // its TMEM columns
   static constexpr int kEpiBufs = 1;
@@ -105,6 +107,8 @@ struct Cfg {
                   kStages * (kA + kB + kE) + 4 * kEpiBufs * kEpi + kBars + 64};
   }
   static_assert(kStages * (kA + kB + kE) + 4 * kEpiBufs * kEpi + kBars + 64 + 1024 <= 232448, "shared memory");
+  static_assert(kN <= 256 && (kN / 2) % 16 == 0, "each CTA supplies a multiple of 16 columns of X");
+  static_assert(kECol >= 256u * (kAcc - 1) + kN && kECol + kECols * kStages <= kTmemCols, "TMEM columns");
 };
 }  // namespace pair
 
@@ -314,42 +318,54 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pair::kThreads, 1)
       const uint32_t t_addr = tmem_base + 256u * (uint32_t)acc + ((uint32_t)(quarter * 32) << 16);
       const uint32_t lead_acc_empty = lead_acc_empty0 + 8u * (uint32_t)acc;
       if (DB && !p.out_f32) {
-        // Three 64-column chunks through the warp's staging buffer, one TMA
-        // store each.  The accumulator is released after the last TMEM load; the
-        // next tile's MMAs run in the other accumulator meanwhile, so this
-        // epilogue has a whole tile period to finish.
+        // Column chunks of 64, 64, 64 and 32 through the warp's staging buffer,
+        // one TMA store each (the last through the 32-column map tm_y32).  The
+        // accumulator is released after the last TMEM load; the next tile's MMAs
+        // run in the other accumulator meanwhile, so this epilogue has a whole
+        // tile period to finish.
+        static_assert(!DB || C::kN == 224u, "the chunk split below covers 224 columns");
         const int32_t wrow0 = (int32_t)(tm * 256 + 128 * rank + quarter * 32);
         uint8_t* ebuf = smem + L.epi + quarter * (C::kEpiBufs * kEpi);
 #pragma unroll
-        for (int c = 0; c < 3; ++c) {
+        for (int c = 0; c < 4; ++c) {
           uint32_t v0[32], v1[32];
           tmem_ld_32x32b_x32(t_addr + c * 64, v0);
-          tmem_ld_32x32b_x32(t_addr + c * 64 + 32, v1);
+          if (c < 3) tmem_ld_32x32b_x32(t_addr + c * 64 + 32, v1);
           tc_wait_ld();
-          if (c == 2) {
+          if (c == 3) {
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive_cluster(lead_acc_empty);
           }
           if (lane == 0) bulk_wait_group_read<0>();  // the previous store has read the buffer
           __syncwarp();
+          if (c < 3) {
 #pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            *reinterpret_cast<uint4*>(ebuf + lane * 128 + ((j ^ (lane & 7)) << 4)) =
-                make_uint4(pack_bf16x2(__uint_as_float(v0[8 * j]), __uint_as_float(v0[8 * j + 1])),
-                           pack_bf16x2(__uint_as_float(v0[8 * j + 2]), __uint_as_float(v0[8 * j + 3])),
-                           pack_bf16x2(__uint_as_float(v0[8 * j + 4]), __uint_as_float(v0[8 * j + 5])),
-                           pack_bf16x2(__uint_as_float(v0[8 * j + 6]), __uint_as_float(v0[8 * j + 7])));
-            *reinterpret_cast<uint4*>(ebuf + lane * 128 + (((j + 4) ^ (lane & 7)) << 4)) =
-                make_uint4(pack_bf16x2(__uint_as_float(v1[8 * j]), __uint_as_float(v1[8 * j + 1])),
-                           pack_bf16x2(__uint_as_float(v1[8 * j + 2]), __uint_as_float(v1[8 * j + 3])),
-                           pack_bf16x2(__uint_as_float(v1[8 * j + 4]), __uint_as_float(v1[8 * j + 5])),
-                           pack_bf16x2(__uint_as_float(v1[8 * j + 6]), __uint_as_float(v1[8 * j + 7])));
+            for (int j = 0; j < 4; ++j) {
+              *reinterpret_cast<uint4*>(ebuf + lane * 128 + ((j ^ (lane & 7)) << 4)) =
+                  make_uint4(pack_bf16x2(__uint_as_float(v0[8 * j]), __uint_as_float(v0[8 * j + 1])),
+                             pack_bf16x2(__uint_as_float(v0[8 * j + 2]), __uint_as_float(v0[8 * j + 3])),
+                             pack_bf16x2(__uint_as_float(v0[8 * j + 4]), __uint_as_float(v0[8 * j + 5])),
+                             pack_bf16x2(__uint_as_float(v0[8 * j + 6]), __uint_as_float(v0[8 * j + 7])));
+              *reinterpret_cast<uint4*>(ebuf + lane * 128 + (((j + 4) ^ (lane & 7)) << 4)) =
+                  make_uint4(pack_bf16x2(__uint_as_float(v1[8 * j]), __uint_as_float(v1[8 * j + 1])),
+                             pack_bf16x2(__uint_as_float(v1[8 * j + 2]), __uint_as_float(v1[8 * j + 3])),
+                             pack_bf16x2(__uint_as_float(v1[8 * j + 4]), __uint_as_float(v1[8 * j + 5])),
+                             pack_bf16x2(__uint_as_float(v1[8 * j + 6]), __uint_as_float(v1[8 * j + 7])));
+            }
+          } else {  // 32 columns: 64-byte rows, unswizzled
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+              *reinterpret_cast<uint4*>(ebuf + lane * 64 + (j << 4)) =
+                  make_uint4(pack_bf16x2(__uint_as_float(v0[8 * j]), __uint_as_float(v0[8 * j + 1])),
+                             pack_bf16x2(__uint_as_float(v0[8 * j + 2]), __uint_as_float(v0[8 * j + 3])),
+                             pack_bf16x2(__uint_as_float(v0[8 * j + 4]), __uint_as_float(v0[8 * j + 5])),
+                             pack_bf16x2(__uint_as_float(v0[8 * j + 6]), __uint_as_float(v0[8 * j + 7])));
           }
           fence_proxy_async_smem();
           __syncwarp();
           if (lane == 0 && n0 + 64 * c < p.T && wrow0 < p.R) {
-            tma_store_2d(&p.tm_y, ebuf, (int32_t)(n0 + 64 * c), wrow0);
+            tma_store_2d(c < 3 ? &p.tm_y : &p.tm_y32, ebuf, (int32_t)(n0 + 64 * c), wrow0);
             bulk_commit_group();
           }
         }
@@ -471,16 +487,17 @@ static cudaError_t launch_pair(SpmmParams& p, cudaStream_t stream) {
 }
 
 // Tiles of at most kDbMaxStages 128-deep stages take the double-buffered
-// 256 x 192 form.  Measured on B200 (nm_spmm, event-timed loops): ViT
-// 3072 x 768 x 50432 at 1:8 (6 stages) 174 -> 166 us; at 24 stages (768 x 3072)
-// 125 -> 143 us, at 32 (4096 x 4096 x 2048) 33 -> 44 us.  A 192-column stage
-// costs about as much as a 256-column one, so the narrower tile pays only where
-// the hidden hand-over is a large part of a tile.
+// form (256 x 224 tiles).  Measured on B200 with 256 x 192 tiles (nm_spmm,
+// event-timed loops): ViT 3072 x 768 x 50432 at 1:8 (6 stages) 174 -> 166 us;
+// at 24 stages (768 x 3072) 125 -> 143 us, at 32 (4096 x 4096 x 2048) 33 -> 44
+// us.  A narrower stage costs about as much as a 256-column one, so the
+// double-buffered form pays only where the hidden hand-over is a large part of
+// a tile.
 constexpr int64_t kDbMaxStages = 8;
 
 cudaError_t launch_spmm_pair(SpmmParams& p, cudaStream_t stream) {
   if (p.k_tiles <= kDbMaxStages) {
-    p.tiles_n = (int)((p.T + 191) / 192);
+    p.tiles_n = (int)((p.T + 223) / 224);
     p.num_tiles = p.tiles_m * p.tiles_n;
     return launch_pair<false, true>(p, stream);
   }
