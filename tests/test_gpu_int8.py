@@ -56,14 +56,13 @@ def test_decompress_i8_roundtrip(R, K):
     assert np.array_equal(Wd.cpu().numpy(), oracle.decompress_i8(ov, om, K))
 
 
-# T >= 192 with K % 32 == 0 runs on the sparse tensor cores (kind::i8, metadata re-laid out per row):
-# 256 x 192 tiles with two accumulators up to 32 stages of 256, 256 x 256 tiles beyond; other shapes on
-# the decompressed dense operand.
+# T >= 192 with K % 32 == 0 runs on the sparse tensor cores (kind::i8, metadata re-laid out per row,
+# 256 x 256 tiles, 256-deep stages); other shapes on the decompressed dense operand.
 @pytest.mark.parametrize("R,K,T", [(300, 512, 264), (256, 1024, 256), (130, 384, 100), (64, 128, 16),
                                    (520, 256, 40), (600, 2048, 520), (260, 800, 320), (200, 1040, 256),
-                                   (260, 8192, 264),    # 32 stages: the last K of the 256 x 192 form
-                                   (520, 2048, 2000),   # 11 column tiles of 192, the last one 80 wide
-                                   (260, 8448, 264)])   # 33 stages: the 256 x 256 tile form
+                                   (260, 8192, 264),    # 32 stages, a second column tile 8 wide
+                                   (520, 2048, 2000),   # 8 column tiles, the last one 208 wide
+                                   (260, 8448, 264)])   # 33 stages, ragged rows
 def test_spmm_i8_exact(R, K, T):
     W = wl.integer_i8((R, K), -128, 127, seed=R + 7 * K)
     X = wl.integer_i8((K, T), -128, 127, seed=T + 3)

@@ -150,7 +150,7 @@ def test_permuted_matches_oracle(n, m):
     check(W, X, n, m, idx=idx, what="permuted")
 
 
-@pytest.mark.parametrize("K", [768, 2048])  # SM-pair kernel: 256 x 192 tiles (6 stages), 256 x 256 tiles (16)
+@pytest.mark.parametrize("K", [768, 2048])  # SM-pair kernel: 256 x 224 tiles (6 stages), 256 x 256 tiles (16)
 def test_permuted_identity_equals_plain_and_host_permuted(K):
     R, T = 256, 256
     W = wl.normal_bf16((R, K), 0.02, seed=61)
@@ -164,7 +164,7 @@ def test_permuted_identity_equals_plain_and_host_permuted(K):
     assert torch.equal(perm, host)  # same tiles, same MMA order: bitwise equal
 
 
-@pytest.mark.parametrize("K,T", [(512, 256),    # gather pass + SM-pair kernel, 256 x 192 tiles
+@pytest.mark.parametrize("K,T", [(512, 256),    # gather pass + SM-pair kernel, 256 x 224 tiles
                                  (1280, 264),   # the same with 256 x 256 tiles and a ragged column tile
                                  (512, 16),     # gather pass + split-K skinny kernel
                                  (512, 100)])   # one-SM kernel gathering its own rows
@@ -493,13 +493,13 @@ def test_dense_design_pair_integer_exact():
 
 # ----------------------------------------------------------------------------
 # SM-pair kernel tile forms: 256 x 256 tiles with one accumulator (more than 8
-# stages per tile) and 256 x 192 tiles with two accumulators (at most 8)
+# stages per tile) and 256 x 224 tiles with two accumulators (at most 8)
 # ----------------------------------------------------------------------------
 @pytest.mark.parametrize("R,K,T", [(2560, 8192, 2048),   # 64 stages: 256 x 256 tiles
                                    (4096, 11008, 2048),  # the LLaMA 4096 x 11008 layer
-                                   (1280, 512, 4096),    # 4 stages: 256 x 192 tiles, 22 column tiles
+                                   (1280, 512, 4096),    # 4 stages: 256 x 224 tiles, 19 column tiles, the last one 64 wide
                                    (2304, 768, 2560),    # 6 stages (the ViT depth), last column tile partial
-                                   (300, 1024, 200)])    # 8 stages, one partial 192-column tile, ragged rows
+                                   (300, 1024, 200)])    # 8 stages, one partial 224-column tile, ragged rows
 @pytest.mark.parametrize("out", [torch.bfloat16, torch.float32])
 def test_pair_tile_forms_integer_exact(R, K, T, out):
     """Small integers keep every fp32 sum exact: sampled rows equal the oracle bit for bit."""
@@ -520,9 +520,9 @@ def test_pair_tile_forms_integer_exact(R, K, T, out):
 
 @pytest.mark.parametrize("R,K,T", [(2560, 8192, 2048),   # 256 x 256 tiles, row tiles fastest
                                    (4096, 11008, 2048),  # 256 x 256 tiles, column tiles fastest
-                                   (1280, 512, 4096),    # 256 x 192 tiles
-                                   (2304, 768, 2568),    # 256 x 192 tiles, last column tile partial
-                                   (300, 1024, 200)])    # one partial 192-column tile, ragged rows
+                                   (1280, 512, 4096),    # 256 x 224 tiles
+                                   (2304, 768, 2568),    # 256 x 224 tiles, last column tile partial
+                                   (300, 1024, 200)])    # one partial 224-column tile, ragged rows
 @pytest.mark.parametrize("out", [torch.bfloat16, torch.float32])
 def test_pair_permuted_integer_exact(R, K, T, out):
     """The permuted two-SM path (gather pass, then the pair kernel) on small
@@ -544,9 +544,9 @@ def test_pair_permuted_integer_exact(R, K, T, out):
         assert np.array_equal(bits(Y)[rows], bf16_rne_of(ref))
 
 
-@pytest.mark.parametrize("R,K,T", [(1, 128, 192),      # one row, one stage, one 192-column tile
+@pytest.mark.parametrize("R,K,T", [(1, 128, 192),      # one row, one stage, one partial 224-column tile
                                    (257, 128, 192),    # a 1-row second row tile
-                                   (255, 1024, 200),   # 8 stages (the last of the 256 x 192 form), 8-column tail
+                                   (255, 1024, 200),   # 8 stages (the last of the 256 x 224 form), 8 columns in the last 32-column chunk
                                    (255, 1152, 200),   # 9 stages: the 256 x 256 form, one partial column tile
                                    (513, 1152, 392),   # three row tiles, ragged rows and columns
                                    (256, 1024, 184)])  # T < 192: the one-SM kernel
