@@ -147,6 +147,19 @@ def test_meta_sizes(R, K, n, m, words):
     assert oracle.value_cols(K, n, m) == K * n // m
 
 
+@pytest.mark.parametrize("m,bits,per_word", [(2, 1, 32), (4, 2, 16), (8, 3, 10), (16, 4, 8)])
+def test_position_width_and_packing(m, bits, per_word):
+    """b = ceil(log2 M) bits per survivor (the 2-bit positions of 2:4, generalised) and floor(32 / b) positions
+    per 32-bit word, no position straddling two words; a row's words cover its K*N/M survivors."""
+    assert oracle.index_bits(m) == bits == (m - 1).bit_length()
+    assert oracle.positions_per_word(m) == per_word == 32 // bits
+    for K, n in ((m, 1), (24 * m, 1), (24 * m, m // 2), (1000 * m, 1)):
+        survivors = K // m * n
+        assert oracle.meta_cols(K, n, m) == -(-survivors // per_word)
+        if not (n == 2 and m == 4):
+            assert oracle.meta_words(7, K, n, m) == 7 * oracle.meta_cols(K, n, m)
+
+
 def test_tiled_2of4_every_group_once():
     """Each group's nibble sits in its own slot; everything else is the padding nibble."""
     R, K = 21, 200                       # padded to 32 rows x 256 columns
