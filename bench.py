@@ -994,8 +994,9 @@ def run_i8(args, rank: int, world: int, dist):
                          "frac": achieved / i8_peak, "traffic": None,
                          "kernel": "nm_spmm_i8 calls: relayout_meta_i8_kernel + spmm_pair_kernel (sparse kind::i8)",
                          "peak_source": f"{peak_src} bf16 burst dense peak x 2 (the nominal int8 / bf16 dense ratio); "
-                                        "useful (survivor) operations, which the sparse MMA executes at twice the "
-                                        "dense rate",
+                                        "useful (survivor) operations: the sparse MMA multiplies the stored values "
+                                        "at the dense rate (its 2x is over the logical K), so they reach this peak "
+                                        "at most",
                          "timing": "CUDA events around back-to-back repetitions of the step's GEMM calls"},
             "gpu_launches": launches, "clocks": sampler.summary() if sampler else None, "cpu_baseline": None}
     if rank == 0:
@@ -1093,8 +1094,9 @@ def run_tf32(args, rank: int, world: int, dist):
                          "frac": achieved / tf32_peak, "traffic": None,
                          "kernel": "nm_spmm_tf32 calls: relayout_meta_tf32_kernel + spmm_pair_kernel (sparse kind::tf32)",
                          "peak_source": f"{peak_src} bf16 burst dense peak x 0.5 (the nominal tf32 / bf16 dense "
-                                        "ratio); useful (survivor) FLOPs, which the sparse MMA executes at twice "
-                                        "the dense rate",
+                                        "ratio); useful (survivor) FLOPs: the sparse MMA multiplies the stored "
+                                        "values at the dense rate (its 2x is over the logical K), so they reach "
+                                        "this peak at most",
                          "timing": "CUDA events around back-to-back repetitions of the step's GEMM calls"},
             "gpu_launches": launches, "clocks": sampler.summary() if sampler else None, "cpu_baseline": None}
     if rank == 0:
