@@ -137,7 +137,8 @@ NM_API nm_status nm_decompress(const uint16_t* values, const uint32_t* meta, int
  *   X            [in] K x T bf16, row stride ldx >= T, ldx % 8 == 0
  *   Y            [out] R x T, bf16 or fp32 (y_dtype), row stride ldy >= T
  * Kernel choice: shapes with K % 128 == 0, T >= 192 and T % 8 == 0 run on two
- * SMs per 256 x 256 tile.  2:4 reads the caller's operand directly.  1:2, 1:4,
+ * SMs per 256 x 256 tile (256 x 224 tiles with two accumulators when K <= 1024).
+ * 2:4 reads the caller's operand directly.  1:2, 1:4,
  * 1:8 and 2:8 (at most two survivors per aligned group of four) are first
  * re-encoded as 2:4 into a staging buffer (R*K bytes of values plus R*K/8
  * bytes of metadata) from the library's pool (see nm_spmm_permuted and
